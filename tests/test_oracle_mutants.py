@@ -1,0 +1,75 @@
+"""The oracle's pins must catch plausible mistakes in it.
+
+Each mutant is a copy of ``oracle/kda_oracle.c`` with one deliberate slip
+(a dropped term, a flipped sign, a wrong index, a transposed operand, the
+epsilon moved out of the root ...), compiled to a temporary library on the
+CPU.  With the mutant swapped in, at least one pin of
+``test_oracle_pins.py`` has to fail.  The real oracle source is never
+modified.
+"""
+import ctypes
+import inspect
+import os
+import subprocess
+
+import pytest
+
+import oracle as oracle_pkg
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle_pkg.__file__), "kda_oracle.c")
+
+MUTANTS = {
+    "no_decay": ("S[(int64_t)d * V + c] *= e;", "(void)e;"),
+    "residual_sign": ("r[c] = vt[c] - acc;", "r[c] = vt[c] + acc;"),
+    "no_beta": ("const double bk = bt * kt[d];", "const double bk = kt[d];"),
+    "output_uses_k": ("acc += (scale * qt[d])", "acc += (scale * kt[d])"),
+    "no_scale": ("acc += (scale * qt[d])", "acc += (qt[d])"),
+    "transposed_update": ("S[(int64_t)d * V + c] += bk * r[c];", "S[(int64_t)c * V + d] += bk * r[c];"),
+    "eps_outside_sqrt": ("sqrtf(ss + 1e-6f)", "(sqrtf(ss) + 1e-6f)"),
+    "gqa_modulo": ("const int hq = h / group;", "const int hq = h % H;"),
+    "gate_wrong_channel": ("const double e = exp(gt[d]);", "const double e = exp(gt[K - 1 - d]);"),
+    "norm_truncates": ("u += 0x7fffu + lsb;", "u += 0u * lsb;"),
+    "decay_after_update_output": ("ot[c] = acc;", "ot[c] = acc * exp(gt[0]);"),
+}
+
+
+def _pin_functions():
+    out = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if name.startswith("test_") and "oracle" in inspect.signature(fn).parameters:
+            if "chunk" in inspect.signature(fn).parameters:
+                out.append((name, lambda o, fn=fn: fn(o, 64)))
+            else:
+                out.append((name, fn))
+    return out
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_pins_catch_mutant(mutant, tmp_path):
+    old, new = MUTANTS[mutant]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {mutant} not found"
+    mutated = src.replace(old, new, 1)
+    c_path = tmp_path / "mut.c"
+    so_path = tmp_path / "libmut.so"
+    c_path.write_text(mutated)
+    subprocess.run(["gcc", *oracle_pkg.GCC_FLAGS, str(c_path), "-o", str(so_path), "-lm"], check=True)
+
+    real = oracle_pkg._load()
+    lib = ctypes.CDLL(str(so_path))
+    for fname in ("kda_oracle_l2norm_bf16", "kda_oracle_recurrence_f64", "kda_oracle_forward",
+                  "kda_oracle_max_threads", "kda_oracle_f64_to_bf16"):
+        f, r = getattr(lib, fname), getattr(real, fname)
+        f.argtypes, f.restype = r.argtypes, r.restype
+    caught = []
+    oracle_pkg._lib = lib
+    try:
+        for name, fn in _pin_functions():
+            try:
+                fn(oracle_pkg)
+            except AssertionError:
+                caught.append(name)
+    finally:
+        oracle_pkg._lib = real
+    assert caught, f"no pin caught mutant {mutant}"
