@@ -1,0 +1,354 @@
+#!/usr/bin/env python3
+"""Benchmark of the KDA chunk-prefill forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference] [--workload NAME]
+
+A step is one whole forward (normalisation, intra-chunk work and the state
+carry over all chunks) over the long-prefill workload: B=1, H=HV=64,
+T=65536, K=V=128, fp32 initial state (seeded synthetic inputs, resident in
+HBM before the timed region).  The inputs (6.5 GB) are far larger than the
+126 MB L2, so no flush is needed between steps.  Prints one JSON line on
+rank 0.
+
+Under torchrun (N > 1) every rank runs its own independent batch of the same
+shape (the (sequence, head) units shard without any exchange): weak scaling,
+no data-path collective; the time is the max over ranks.
+
+``--impl reference`` times the CPU oracle (the plain float64 recurrence) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA chunk-prefill tokens·heads/s @T=64K,HV=64,K=V=128; % of roofline"
+UNIT = "tokens·heads/s"
+BYTES_PER_TOKEN_HEAD = 256 + 256 + 256 + 512 + 4 + 256  # q, k, v, g, beta, o (H == HV)
+
+
+def algorithmic_bytes(case) -> int:
+    """Bytes the forward must move at least once: inputs read, o written, state read and written."""
+    group = case.HV // case.H
+    th = case.tokens * case.HV
+    per = 256 * 2 / group + 256 + 512 + 4 + 256
+    state = case.N * case.HV * 128 * 128 * 4 * (2 if case.state != "none" else 1)
+    return int(th * per + state)
+
+
+def chunk_flops(case) -> int:
+    """Dense chunk-form FLOPs (C=64 tiles): 180,224 per token-head."""
+    return case.tokens * case.HV * 180224
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "kda_gated_delta_prefill_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        rec = json.load(fh)
+    ent = rec.get(workload)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return int(ent["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5], parts[6], parts[7], parts[8]))
+                except ValueError:
+                    continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[2 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------------------- oracle
+
+def cpu_sample_inputs(case, heads: int, tokens: int):
+    """The first `tokens` tokens of value heads [0, heads) of the workload, on the CPU."""
+    import torch
+    from kda_gated_delta_prefill_b200 import inputs as gen
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = gen.make_inputs(case, device=dev)
+    group = case.HV // case.H
+    out = {
+        "q": x["q"][:, :tokens, : max(1, heads // group)].contiguous().cpu(),
+        "k": x["k"][:, :tokens, : max(1, heads // group)].contiguous().cpu(),
+        "v": x["v"][:, :tokens, :heads].contiguous().cpu(),
+        "g": x["g"][:, :tokens, :heads].contiguous().cpu(),
+        "beta": x["beta"][:, :tokens, :heads].contiguous().cpu(),
+        "initial_state": None if x["initial_state"] is None else x["initial_state"][:, :heads].contiguous().cpu(),
+        "cu_seqlens": None,
+    }
+    del x
+    if dev == "cuda":
+        torch.cuda.empty_cache()
+    return out
+
+
+def time_oracle(case, target_s: float = 15.0):
+    import oracle
+    cores = oracle.max_threads()
+    heads = min(case.HV, max(1, cores))
+    if case.HV // case.H > 1:
+        heads -= heads % (case.HV // case.H) or 0
+        heads = max(heads, case.HV // case.H)
+    # pilot: 256 tokens on the chosen heads, then size the sample to about target_s seconds
+    pilot_tok = min(case.T, 256)
+    xs = cpu_sample_inputs(case, heads, pilot_tok)
+    t0 = time.perf_counter()
+    oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["initial_state"])
+    dt = time.perf_counter() - t0
+    per_tok = dt / pilot_tok
+    tokens = int(min(case.T, max(pilot_tok, target_s / max(per_tok, 1e-9))))
+    xs = cpu_sample_inputs(case, heads, tokens)
+    t0 = time.perf_counter()
+    oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["initial_state"])
+    dt = time.perf_counter() - t0
+    return {"value": tokens * heads / dt, "unit": UNIT, "cores": min(cores, heads), "kind": "oracle",
+            "sample": f"first {tokens} tokens x value heads 0..{heads - 1} of {case.name}",
+            "seconds": dt}
+
+
+# ---------------------------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="long_T65536_H64_state")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    import torch
+    import torch.distributed as dist
+    from kda_gated_delta_prefill_b200 import inputs as gen
+
+    case = {c.name: c for c in gen.WORKLOADS}[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    config = {"workload": case.name, "B": case.B, "T": case.T, "H": case.H, "HV": case.HV, "K": case.K,
+              "V": case.V, "chunk": 64, "initial_state": case.state != "none",
+              "l2": "inputs (6.5 GB) larger than L2; no flush" if case.name.startswith("long")
+              else "inputs re-used across steps (may hit L2)",
+              "parallelism": f"independent replicas x{args.gpus} (weak)" if args.gpus > 1 else "single GPU"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cb = time_oracle(case)
+        line = {"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": 1,
+                "warmup": 0, "ms_per_step": cb["seconds"] * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config, "impl": "reference",
+                "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import kda_gated_delta_prefill_b200 as kda
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    kda.lib()
+
+    # ---- inputs resident in HBM (rank-specific seed: independent batches) ----
+    import dataclasses
+    rcase = dataclasses.replace(case, seed=case.seed + 1000 * rank)
+    x = gen.make_inputs(rcase, device=dev)
+    B, T, H, HV, K, V, N = case.B, case.T, case.H, case.HV, case.K, case.V, case.N
+    o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=dev)
+    s = torch.empty(N, HV, K, V, dtype=torch.float32, device=dev)
+    ws_n = kda.workspace_size(B, T, H, HV, K, V, N if x["cu_seqlens"] is not None else 0)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"], x["cu_seqlens"], o=o,
+                    final_state=s, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- timed region: K steps; per-launch CUDA events on the launching stream ----
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    total_ms = t0.elapsed_time(t1)
+    launch_ms = [a.elapsed_time(b) for a, b in evs]
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    th_per_step = case.tokens * HV
+    value = th_per_step * world / (total_ms / 1e3 / args.steps)
+
+    # ---- roofline of the dominant (only) compute kernel ----
+    hbm_gbs, bf16_tf, peak_kind = load_peaks()
+    alg = algorithmic_bytes(case)
+    avg_launch_s = statistics.mean(launch_ms) / 1e3
+    achieved = alg / avg_launch_s / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
+                "traffic": recorded_traffic(case.name), "peak_kind": peak_kind,
+                "algorithmic_bytes_per_launch": alg, "avg_launch_ms": avg_launch_s * 1e3,
+                "frac_nominal_8TBps": achieved / 8000.0,
+                "tensor_tflops": chunk_flops(case) / avg_launch_s / 1e12}
+
+    # ---- end to end through the host-buffer entry point ----
+    e2e = None
+    if not args.no_e2e:
+        del o, s
+        xh = {k: (v.cpu().pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+        del x
+        torch.cuda.empty_cache()
+        oh = torch.empty(B, T, HV, V, dtype=torch.bfloat16).pin_memory()
+        sh = torch.empty(N, HV, K, V, dtype=torch.float32).pin_memory()
+        has_cu = xh["cu_seqlens"] is not None
+        st_n = kda.host_staging_size(B, T, H, HV, K, V, N if has_cu else 0, xh["initial_state"] is not None, has_cu)
+        staging = torch.empty(st_n, dtype=torch.uint8, device=dev)
+
+        def hstep():
+            kda.forward_host(xh["q"], xh["k"], xh["v"], xh["g"], xh["beta"], xh["initial_state"], xh["cu_seqlens"],
+                             o=oh, final_state=sh, staging=staging, stream=stream)
+        for _ in range(2):
+            hstep()
+        torch.cuda.synchronize()
+        e_steps = max(3, min(args.steps, 5))
+        barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e_steps):
+            hstep()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        h2d = sum(t.numel() * t.element_size() for t in xh.values() if isinstance(t, torch.Tensor))
+        d2h = oh.numel() * 2 + sh.numel() * 4
+        e2e = {"value": th_per_step * world / (e_ms / 1e3 / e_steps), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": e_steps}
+        del xh, staging
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = time_oracle(case)
+        cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+
+    launches_per_step = 1 + (1 if case.lengths is not None else 0)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
+            "gpu_launches": launches_per_step * args.steps, "impl": "native",
+            "kernel_source": kernel_source_hash()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,136 @@
+/*
+ * kda_prefill.h -- C ABI of the KDA (Kimi Delta Attention) chunk-prefill
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ * The operation ("KDA Chunk Prefill on Ascend A3", sections "Function and
+ * tensor contract" and "Mathematical definition"):
+ *
+ *   forward(q, k, v, g, beta, initial_state) -> (o, final_state)
+ *
+ *   1. Q and K are L2-normalised along their last dimension in float32 in
+ *      the stated rounding order, epsilon 1e-6 inside the square root, and
+ *      rounded to bf16:  xn = bf16(f32(x) / sqrt(sum(f32(x)^2) + 1e-6)).
+ *   2. For every sequence and value head h (Q/K head h / (HV/H)), with a
+ *      float32 state S[K][V], the gated delta rule runs over the tokens:
+ *         S   <- exp(g_t)[:,None] * S
+ *         r_t  = v_t - k_t^T S
+ *         S   <- S + beta_t k_t r_t^T
+ *         o_t  = (K^-0.5 q_t)^T S
+ *      The library evaluates it in the page's chunk form (64-token chunks:
+ *      cumulative gate G, strictly lower L, causal Aqk, A = (I+L)^-1
+ *      diag(beta), W = A (exp(G) k), U = A v, and the inter-chunk carry
+ *      Vnew = U - W S, O = Qg S + Aqk Vnew, S' = exp(G_last) S + Kg^T Vnew).
+ *      A partial last chunk behaves as if zero-padded; its padded rows are
+ *      never written.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensors are dense, row-major (C order), contiguous.  Pointers are
+ *     caller-owned DEVICE memory unless the name says _host.  The library
+ *     never allocates device memory and never synchronises the stream.
+ *   - Inputs are never written.  final_state may alias initial_state
+ *     exactly (in-place update); any other overlap is rejected.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream).  Argument errors are detected on the host before any
+ *     launch; launch failures are reported as KDA_ERR_CUDA.  Values held in
+ *     device memory (cu_seqlens entries) are not checked on the host.
+ *   - Supported sizes: K == V == 128, HV % H == 0, all sizes positive
+ *     (T may be 0 only with cu_seqlens).  Other K/V give
+ *     KDA_ERR_UNSUPPORTED.
+ *   - Numerical domain: gates g <= 0 with sum over any 16 consecutive
+ *     tokens >= -80 (per-token g >= -5 suffices); beta in [0, 1].
+ */
+#ifndef KDA_PREFILL_H
+#define KDA_PREFILL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, HV % H != 0, bad overlap */
+    KDA_ERR_UNSUPPORTED = 2, /* K or V other than 128 */
+    KDA_ERR_MISALIGNED = 3,  /* a pointer is not aligned as documented */
+    KDA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than kda_prefill_workspace_size() */
+    KDA_ERR_CUDA = 5         /* a CUDA runtime call or a kernel launch failed */
+} kda_status_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *kda_status_string(kda_status_t status);
+
+/*
+ * Bytes of device workspace kda_prefill_forward needs for these sizes.
+ * num_seqs is the number of packed sequences when cu_seqlens is used, or 0
+ * for a plain [B, T] batch (then no workspace is needed and 0 is returned).
+ * The workspace holds the longest-first order of the packed sequences.
+ */
+size_t kda_prefill_workspace_size(int B, int T, int H, int HV, int K, int V, int num_seqs);
+
+/*
+ * The chunk-prefill forward.
+ *
+ *   q, k          bf16 [B, T, H, K]        16-byte aligned
+ *   v             bf16 [B, T, HV, V]       16-byte aligned
+ *   g             fp32 [B, T, HV, K]       16-byte aligned; natural-log gates
+ *   beta          fp32 [B, T, HV]          4-byte aligned
+ *   initial_state fp32 [N, HV, K, V] or NULL (zeros); 4-byte aligned
+ *   cu_seqlens    int32 [N + 1] or NULL.   When given: B == 1, N = num_seqs >= 1,
+ *                 cu_seqlens[0] == 0, non-decreasing, cu_seqlens[N] == T
+ *                 (device values, not checked).  Sequence n holds tokens
+ *                 [cu[n], cu[n+1]) and starts from initial_state[n].
+ *                 When NULL: N = B and num_seqs is ignored.
+ *   o             bf16 [B, T, HV, V] out;  16-byte aligned.  Rows of tokens
+ *                 that belong to no sequence are left untouched.
+ *   final_state   fp32 [N, HV, K, V] out (required); 4-byte aligned
+ *   workspace     device scratch of workspace_bytes, 256-byte aligned, may be
+ *                 NULL when kda_prefill_workspace_size() returns 0.
+ *   stream        cudaStream_t
+ */
+kda_status_t kda_prefill_forward(const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta,
+                                 const float *initial_state,
+                                 const int32_t *cu_seqlens, int num_seqs,
+                                 int B, int T, int H, int HV, int K, int V,
+                                 void *o, float *final_state,
+                                 void *workspace, size_t workspace_bytes,
+                                 void *stream);
+
+/*
+ * Bytes of device staging memory kda_prefill_forward_host needs: room for
+ * every input and output plus the workspace, each 256-byte aligned.
+ */
+size_t kda_prefill_host_staging_size(int B, int T, int H, int HV, int K, int V, int num_seqs,
+                                     int has_initial_state, int has_cu_seqlens);
+
+/*
+ * The same forward on HOST buffers (same shapes and dtypes as above; pinned
+ * memory makes the copies asynchronous).  Inputs are copied into the
+ * caller's device staging buffer, the forward runs there, and o and
+ * final_state are copied back -- all enqueued on `stream`; the caller
+ * synchronises before reading o_host / final_state_host.
+ */
+kda_status_t kda_prefill_forward_host(const void *q_host, const void *k_host, const void *v_host,
+                                      const float *g_host, const float *beta_host,
+                                      const float *initial_state_host,
+                                      const int32_t *cu_seqlens_host, int num_seqs,
+                                      int B, int T, int H, int HV, int K, int V,
+                                      void *o_host, float *final_state_host,
+                                      void *staging, size_t staging_bytes,
+                                      void *stream);
+
+/*
+ * Step 1 alone: L2-normalise `rows` rows of K bf16 values with the exact
+ * rounding order above ("KDA Chunk Prefill on Ascend A3", section
+ * "Mathematical definition", first formula).  x and out: bf16 [rows, K],
+ * 16-byte aligned, device; out may equal x.  K must be 128.
+ */
+kda_status_t kda_l2norm_bf16(const void *x, int64_t rows, int K, void *out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_PREFILL_H */

@@ -1,1 +1,147 @@
-"""KDA chunk-prefill forward for NVIDIA B200 (sm_100a)."""
+"""KDA chunk-prefill forward for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/kda_prefill.h``: argument
+marshalling only.  Every step of the forward runs in the CUDA kernels of
+``libkda_prefill.so``; there is no CPU path.  If the library is missing the
+calls raise, they never fall back.
+
+    o, final_state = forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None)
+
+Shapes ("KDA Chunk Prefill on Ascend A3", section "Function and tensor
+contract"): q, k [B,T,H,128] bf16; v [B,T,HV,128] bf16; g [B,T,HV,128]
+fp32; beta [B,T,HV] fp32; initial_state [N,HV,128,128] fp32 or None;
+cu_seqlens [N+1] int32 or None (then B must be 1).  Returns o
+[B,T,HV,128] bf16 and final_state [N,HV,128,128] fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libkda_prefill.so")
+
+STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_MISALIGNED",
+          4: "KDA_ERR_WORKSPACE", 5: "KDA_ERR_CUDA"}
+
+EXPORTED = ("kda_status_string", "kda_prefill_workspace_size", "kda_prefill_forward",
+            "kda_prefill_host_staging_size", "kda_prefill_forward_host", "kda_l2norm_bf16")
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib():
+    """Load libkda_prefill.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                               "(run python -m kda_gated_delta_prefill_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, Z, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_int64
+        L.kda_status_string.argtypes = [I]
+        L.kda_status_string.restype = ctypes.c_char_p
+        L.kda_prefill_workspace_size.argtypes = [I] * 7
+        L.kda_prefill_workspace_size.restype = Z
+        L.kda_prefill_forward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, Z, P]
+        L.kda_prefill_forward.restype = I
+        L.kda_prefill_host_staging_size.argtypes = [I] * 9
+        L.kda_prefill_host_staging_size.restype = Z
+        L.kda_prefill_forward_host.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, Z, P]
+        L.kda_prefill_forward_host.restype = I
+        L.kda_l2norm_bf16.argtypes = [P, I64, I, P, P]
+        L.kda_l2norm_bf16.restype = I
+        _lib = L
+        return L
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise KdaError(rc, where)
+
+
+def _dims(q, v, cu_seqlens):
+    B, T, H, K = q.shape
+    HV, V = v.shape[2], v.shape[3]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    return B, T, H, HV, K, V, N
+
+
+def workspace_size(B, T, H, HV, K=128, V=128, num_seqs=0) -> int:
+    return int(lib().kda_prefill_workspace_size(B, T, H, HV, K, V, num_seqs))
+
+
+def forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o=None, final_state=None,
+            workspace=None, stream=None):
+    """Run the forward on CUDA tensors; returns (o, final_state)."""
+    import torch
+    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if o is None:
+        o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=q.device)
+    if final_state is None:
+        final_state = torch.empty(N, HV, K, V, dtype=torch.float32, device=q.device)
+    num_seqs = N if cu_seqlens is not None else 0
+    ws_bytes = workspace_size(B, T, H, HV, K, V, num_seqs)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    rc = lib().kda_prefill_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                                   _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(o), _ptr(final_state),
+                                   _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                   _stream_ptr(stream))
+    _check(rc, "kda_prefill_forward")
+    return o, final_state
+
+
+def host_staging_size(B, T, H, HV, K=128, V=128, num_seqs=0, has_initial_state=False, has_cu_seqlens=False) -> int:
+    return int(lib().kda_prefill_host_staging_size(B, T, H, HV, K, V, num_seqs, int(has_initial_state),
+                                                    int(has_cu_seqlens)))
+
+
+def forward_host(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o, final_state, staging, stream=None):
+    """Forward on HOST (ideally pinned) tensors through a device staging buffer.
+
+    Enqueues the host->device copies, the forward and the device->host copies
+    of o and final_state on ``stream``; the caller synchronises.
+    """
+    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
+    num_seqs = N if cu_seqlens is not None else 0
+    rc = lib().kda_prefill_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                                        _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(o), _ptr(final_state),
+                                        _ptr(staging), staging.numel(), _stream_ptr(stream))
+    _check(rc, "kda_prefill_forward_host")
+    return o, final_state
+
+
+def l2norm_bf16(x, out=None, stream=None):
+    """Exact-rounding L2 normalisation of rows of 128 bf16 values (CUDA)."""
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    rows = x.numel() // x.shape[-1]
+    _check(lib().kda_l2norm_bf16(_ptr(x), rows, x.shape[-1], _ptr(out), _stream_ptr(stream)), "kda_l2norm_bf16")
+    return out

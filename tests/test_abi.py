@@ -1,0 +1,110 @@
+"""The C-ABI library builds, loads without a GPU, exports every symbol the
+header declares, and rejects bad arguments on the host (no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kda_gated_delta_prefill_b200 as kda
+from kda_gated_delta_prefill_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    kbuild.build()
+    return kda.lib()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_symbols()
+    assert names >= set(kda.EXPORTED) - set(), names
+    for n in names:
+        assert hasattr(L, n), f"{n} declared but not exported"
+
+
+def test_status_strings(L):
+    for code, name in kda.STATUS.items():
+        assert L.kda_status_string(code).decode() == name
+    assert L.kda_status_string(99).decode() == "KDA_ERR_UNKNOWN"
+
+
+def test_workspace_size(L):
+    assert L.kda_prefill_workspace_size(2, 4096, 96, 96, 128, 128, 0) == 0
+    assert L.kda_prefill_workspace_size(1, 11210, 8, 32, 128, 128, 7) == 256
+    assert L.kda_prefill_workspace_size(1, 10, 1, 1, 128, 128, 65) == 512
+
+
+def test_host_staging_size(L):
+    B, T, H, HV = 1, 1000, 4, 4
+    n = L.kda_prefill_host_staging_size(B, T, H, HV, 128, 128, 0, 1, 0)
+    expect = 2 * T * H * 128 * 2 + T * HV * 128 * 2 + T * HV * 128 * 4 + T * HV * 4 + 2 * HV * 128 * 128 * 4 \
+        + T * HV * 128 * 2
+    assert expect <= n <= expect + 16 * 256
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null address that is never dereferenced
+
+
+def call_forward(L, **over):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, g=FAKE * 4, beta=FAKE * 5, s0=None, cu=None, num_seqs=0,
+             B=1, T=64, H=1, HV=1, K=128, V=128, o=FAKE * 6, sN=FAKE * 7, ws=None, ws_bytes=0)
+    a.update(over)
+    return L.kda_prefill_forward(a["q"], a["k"], a["v"], a["g"], a["beta"], a["s0"], a["cu"], a["num_seqs"],
+                                 a["B"], a["T"], a["H"], a["HV"], a["K"], a["V"], a["o"], a["sN"], a["ws"],
+                                 a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(B=0), 1), (dict(T=0), 1), (dict(H=0), 1), (dict(HV=3, H=2), 1), (dict(K=64), 2), (dict(V=256), 2),
+    (dict(q=None), 1), (dict(sN=None), 1), (dict(o=None), 1),
+    (dict(q=FAKE + 2), 3), (dict(g=FAKE * 4 + 8), 3), (dict(beta=FAKE * 5 + 2), 3),
+    (dict(cu=FAKE * 8, num_seqs=0), 1), (dict(cu=FAKE * 8, num_seqs=2, B=2), 1),
+    (dict(cu=FAKE * 8, num_seqs=2), 4),                      # varlen needs a workspace
+    (dict(cu=FAKE * 8, num_seqs=2, ws=FAKE * 9, ws_bytes=16), 4),
+    (dict(cu=FAKE * 8, num_seqs=2, ws=FAKE * 9 + 16, ws_bytes=256), 3),
+    (dict(o=FAKE), 1),                                       # o overlaps q
+    (dict(sN=FAKE * 4), 1),                                  # final_state overlaps g
+])
+def test_forward_rejects_bad_arguments(L, over, code):
+    assert call_forward(L, **over) == code
+
+
+def test_partial_state_overlap_rejected(L):
+    s0 = FAKE * 16
+    assert call_forward(L, s0=s0, sN=s0 + 4096) == 1
+
+
+def test_l2norm_rejects_bad_arguments(L):
+    assert L.kda_l2norm_bf16(FAKE, 4, 64, FAKE * 2, None) == 2
+    assert L.kda_l2norm_bf16(FAKE, -1, 128, FAKE * 2, None) == 1
+    assert L.kda_l2norm_bf16(None, 4, 128, FAKE * 2, None) == 1
+    assert L.kda_l2norm_bf16(FAKE + 2, 4, 128, FAKE * 2, None) == 3
+    assert L.kda_l2norm_bf16(FAKE, 4, 128, FAKE + 256, None) == 1
+    assert L.kda_l2norm_bf16(FAKE, 0, 128, FAKE * 2, None) == 0
+
+
+def test_host_forward_rejects_small_staging(L):
+    P = ctypes.c_void_p
+    rc = L.kda_prefill_forward_host(P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), None, None, 0, 1, 64, 1, 1, 128,
+                                    128, P(FAKE), P(FAKE), P(FAKE * 4), 16, None)
+    assert rc == 4
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(kda, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(kda, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        kda.lib()

@@ -1,0 +1,204 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  Tolerances live in parity_util."""
+import numpy as np
+import pytest
+import torch
+
+from kda_gated_delta_prefill_b200 import inputs as gen
+from tests.parity_util import compare, gpu_forward, oracle_forward, select_heads, to_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import kda_gated_delta_prefill_b200 as kda
+    kda.lib()  # fail loudly if the library is missing
+
+
+# ------------------------------------------------------------------ normalisation
+
+@pytest.mark.parametrize("mode", ["normal", "gain", "tiny", "zero_rows"])
+def test_l2norm_within_one_ulp(mode):
+    import kda_gated_delta_prefill_b200 as kda
+    import oracle
+    case = gen.Case("norm", B=1, T=4096, H=4, HV=4, qk_mode=mode, seed=21)
+    x = gen.make_inputs(case)["q"]
+    ref = oracle.l2norm_bf16(x).astype(np.int32)
+    got = kda.l2norm_bf16(x.cuda()).cpu().view(torch.int16).numpy().astype(np.int32) & 0xFFFF
+
+    def ordered(b):  # bf16 bits -> integers ordered like the values (+0 and -0 both 0)
+        return np.where(b & 0x8000, -(b & 0x7FFF), b & 0x7FFF)
+
+    diff = np.abs(ordered(got) - ordered(ref))
+    assert diff.max() <= 1
+    assert (diff == 0).mean() > 0.99
+
+
+# ------------------------------------------------------------------ worked example
+
+def test_worked_example_exact():
+    x = gen.worked_example()
+    o, s = gpu_forward(x)
+    bits = o.cpu().view(torch.int16).numpy().astype(np.int32) & 0xFFFF
+    assert np.all(bits == 0x3DB5)
+    S = s.cpu().numpy()[0, 0]
+    assert np.all(S[0] == 1.0) and np.all(S[1:] == 0.0)
+
+
+def test_beta_zero_gives_zeros():
+    x = gen.make_inputs(gen.SMALLEST)
+    x["beta"] = torch.zeros_like(x["beta"])
+    o, s = gpu_forward(x)
+    assert torch.all(o == 0) and torch.all(s == 0)
+
+
+# ------------------------------------------------------------------ the workloads
+
+@pytest.mark.parametrize("case", [gen.SMALLEST, gen.TAIL_STATE, gen.VARLEN_GQA], ids=lambda c: c.name)
+def test_workload_full_parity(case):
+    x = gen.make_inputs(case)
+    o, s = gpu_forward(x)
+    ref = oracle_forward(x)
+    compare(o, s, ref)
+
+
+def test_wide_heads_sampled():
+    # B=2, H=HV=96, T=4096: all heads on the GPU, oracle on a sample of heads.
+    x = gen.make_inputs(gen.WIDE_HEADS)
+    o, s = gpu_forward(x)
+    heads = [0, 37, 95]
+    sub = select_heads(x, heads)
+    ref = oracle_forward(sub)
+    compare(o[:, :, heads].contiguous(), s[:, heads].contiguous(), ref)
+
+
+def test_long_prefill_sampled():
+    # B=1, H=HV=64, T=65536 with state, generated on the device as the benchmark does.
+    x = gen.make_inputs(gen.LONG_PREFILL, device="cuda")
+    import kda_gated_delta_prefill_b200 as kda
+    o, s = kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"])
+    torch.cuda.synchronize()
+    heads = [5, 63]
+    xc = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    sub = select_heads(xc, heads)
+    ref = oracle_forward(sub)
+    compare(o[:, :, heads].contiguous(), s[:, heads].contiguous(), ref)
+
+
+# ------------------------------------------------------------------ edges and modes
+
+@pytest.mark.parametrize("T", [1, 2, 15, 16, 17, 63, 64, 65, 127, 129, 200])
+def test_lengths(T):
+    case = gen.Case(f"len{T}", B=2, T=T, H=2, HV=2, state="n01", seed=100 + T)
+    x = gen.make_inputs(case)
+    o, s = gpu_forward(x)
+    compare(o, s, oracle_forward(x))
+
+
+@pytest.mark.parametrize("mode", [dict(qk_mode="gain"), dict(qk_mode="tiny"), dict(qk_mode="zero_rows"),
+                                  dict(gate="logsig128"), dict(gate="logsig8"), dict(gate="logsig1"),
+                                  dict(gate="zero"), dict(gate="uniform5"), dict(beta="one"), dict(beta="edge"),
+                                  dict(beta="zero", state="quarter"), dict(state="quarter"), dict(state="zeros")],
+                         ids=lambda m: "-".join(f"{k}={v}" for k, v in m.items()))
+def test_generator_modes(mode):
+    case = gen.Case("mode", B=1, T=300, H=2, HV=2, seed=7, **mode)
+    x = gen.make_inputs(case)
+    o, s = gpu_forward(x)
+    compare(o, s, oracle_forward(x))
+
+
+def test_gqa_group_8():
+    case = gen.Case("gqa8", B=1, T=257, H=2, HV=16, state="n01", seed=31)
+    x = gen.make_inputs(case)
+    o, s = gpu_forward(x)
+    compare(o, s, oracle_forward(x))
+
+
+def test_varlen_with_empty_sequences():
+    lengths = [0, 5, 0, 64, 1, 130, 0]
+    case = gen.Case("varlen0", B=1, T=sum(lengths), H=2, HV=4, lengths=lengths, state="n01", seed=41)
+    x = gen.make_inputs(case)
+    o, s = gpu_forward(x)
+    ref = oracle_forward(x)
+    compare(o, s, ref)
+    # empty sequences pass their state through unchanged
+    for n, L in enumerate(lengths):
+        if L == 0:
+            assert torch.equal(s[n].cpu(), x["initial_state"][n])
+
+
+def test_in_place_state_update():
+    case = gen.Case("inplace", B=1, T=150, H=2, HV=2, state="n01", seed=51)
+    x = gen.make_inputs(case)
+    ref = oracle_forward(x)
+    xc = to_cuda(x)
+    import kda_gated_delta_prefill_b200 as kda
+    st = xc["initial_state"].clone()
+    o, s = kda.forward(xc["q"], xc["k"], xc["v"], xc["g"], xc["beta"], st, final_state=st)
+    torch.cuda.synchronize()
+    assert s.data_ptr() == st.data_ptr()
+    compare(o, s, ref)
+
+
+def test_split_resume_matches_full():
+    case = gen.Case("split", B=1, T=333, H=2, HV=2, state="n01", seed=61)
+    x = gen.make_inputs(case)
+    full_o, full_s = gpu_forward(x)
+    t1 = 128 + 37
+    a = {k: (v[:, :t1].contiguous() if k in ("q", "k", "v", "g", "beta") else v) for k, v in x.items()}
+    oa, sa = gpu_forward(a)
+    b = {k: (v[:, t1:].contiguous() if k in ("q", "k", "v", "g", "beta") else v) for k, v in x.items()}
+    b["initial_state"] = sa.cpu()
+    ob, sb = gpu_forward(b)
+    ref = oracle_forward(x)
+    compare(torch.cat([oa, ob], dim=1), sb, ref)
+    assert torch.equal(oa, full_o[:, :t1])
+
+
+def test_outputs_fully_written():
+    # NaN canaries in o and final_state must all be overwritten.
+    case = gen.Case("canary", B=2, T=100, H=2, HV=4, seed=71)
+    x = to_cuda(gen.make_inputs(case))
+    import kda_gated_delta_prefill_b200 as kda
+    o = torch.full((2, 100, 4, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    s = torch.full((2, 4, 128, 128), float("nan"), device="cuda")
+    kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], None, o=o, final_state=s)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o.float()).all() and torch.isfinite(s).all()
+
+
+def test_inputs_not_mutated():
+    case = gen.Case("mut", B=1, T=130, H=2, HV=2, state="n01", seed=81)
+    x = to_cuda(gen.make_inputs(case))
+    before = {k: v.clone() for k, v in x.items() if isinstance(v, torch.Tensor)}
+    import kda_gated_delta_prefill_b200 as kda
+    kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"])
+    torch.cuda.synchronize()
+    for k, v in before.items():
+        assert torch.equal(v, x[k]), k
+
+
+def test_host_entry_point_matches_device_entry_point():
+    import kda_gated_delta_prefill_b200 as kda
+    x = gen.make_inputs(gen.TAIL_STATE)
+    o_dev, s_dev = gpu_forward(x)
+    B, T, H, HV = 1, 1000, 4, 4
+    staging = torch.empty(kda.host_staging_size(B, T, H, HV, has_initial_state=True), dtype=torch.uint8,
+                          device="cuda")
+    pin = {k: v.pin_memory() for k, v in x.items() if isinstance(v, torch.Tensor)}
+    o_h = torch.empty(B, T, HV, 128, dtype=torch.bfloat16).pin_memory()
+    s_h = torch.empty(B, HV, 128, 128).pin_memory()
+    kda.forward_host(pin["q"], pin["k"], pin["v"], pin["g"], pin["beta"], pin["initial_state"], None,
+                     o=o_h, final_state=s_h, staging=staging)
+    torch.cuda.synchronize()
+    assert torch.equal(o_h, o_dev.cpu()) and torch.equal(s_h, s_dev.cpu())
+
+
+def test_repeat_calls_are_deterministic():
+    x = gen.make_inputs(gen.TAIL_STATE)
+    o1, s1 = gpu_forward(x)
+    o2, s2 = gpu_forward(x)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
