@@ -37,7 +37,10 @@
  *     (T may be 0 only with cu_seqlens).  Other K/V give
  *     KDA_ERR_UNSUPPORTED.
  *   - Numerical domain: gates g <= 0 with sum over any 16 consecutive
- *     tokens >= -80 (per-token g >= -5 suffices); beta in [0, 1].
+ *     tokens >= -80 (per-token g >= -5 suffices); beta in [0, 1]; |v| and
+ *     the state entries below 6e4 (the state-carry contractions use fp16
+ *     operands with fp32 accumulation; the gate-rescaled L/Aqk operands use
+ *     bf16 for its range).
  */
 #ifndef KDA_PREFILL_H
 #define KDA_PREFILL_H
@@ -64,8 +67,11 @@ const char *kda_status_string(kda_status_t status);
 /*
  * Bytes of device workspace kda_prefill_forward needs for these sizes.
  * num_seqs is the number of packed sequences when cu_seqlens is used, or 0
- * for a plain [B, T] batch (then no workspace is needed and 0 is returned).
- * The workspace holds the longest-first order of the packed sequences.
+ * for a plain [B, T] batch.  The workspace holds, per (64-token chunk, value
+ * head), the chunk's state-independent results that the intra-chunk kernel
+ * hands to the carry kernel (72.5 KiB each), plus the chunk offsets and the
+ * longest-first order of packed sequences.  Returns 0 for sizes that
+ * kda_prefill_forward would reject.
  */
 size_t kda_prefill_workspace_size(int B, int T, int H, int HV, int K, int V, int num_seqs);
 
@@ -85,8 +91,9 @@ size_t kda_prefill_workspace_size(int B, int T, int H, int HV, int K, int V, int
  *   o             bf16 [B, T, HV, V] out;  16-byte aligned.  Rows of tokens
  *                 that belong to no sequence are left untouched.
  *   final_state   fp32 [N, HV, K, V] out (required); 4-byte aligned
- *   workspace     device scratch of workspace_bytes, 256-byte aligned, may be
- *                 NULL when kda_prefill_workspace_size() returns 0.
+ *   workspace     device scratch of at least kda_prefill_workspace_size()
+ *                 bytes, 256-byte aligned, overlapping no other argument.
+ *                 Its contents need no initialisation and are garbage after.
  *   stream        cudaStream_t
  */
 kda_status_t kda_prefill_forward(const void *q, const void *k, const void *v,
@@ -120,6 +127,15 @@ kda_status_t kda_prefill_forward_host(const void *q_host, const void *k_host, co
                                       void *o_host, float *final_state_host,
                                       void *staging, size_t staging_bytes,
                                       void *stream);
+
+/*
+ * Debug aid: the device error word of the current device.  Kernel waits on
+ * copies and pipeline stages are bounded (about one second); a wait that
+ * gives up sets a bit here (1: input tile copy, 2: stage fill, 4: stage
+ * release) and the kernel stops early instead of hanging.  Synchronises the
+ * device.  clear != 0 resets the word afterwards.
+ */
+kda_status_t kda_prefill_device_error(unsigned *word, int clear);
 
 /*
  * Step 1 alone: L2-normalise `rows` rows of K bf16 values with the exact

@@ -26,7 +26,8 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
           4: "KDA_ERR_WORKSPACE", 5: "KDA_ERR_CUDA"}
 
 EXPORTED = ("kda_status_string", "kda_prefill_workspace_size", "kda_prefill_forward",
-            "kda_prefill_host_staging_size", "kda_prefill_forward_host", "kda_l2norm_bf16")
+            "kda_prefill_host_staging_size", "kda_prefill_forward_host", "kda_prefill_device_error",
+            "kda_l2norm_bf16")
 
 
 class KdaError(RuntimeError):
@@ -60,6 +61,8 @@ def lib():
         L.kda_prefill_host_staging_size.restype = Z
         L.kda_prefill_forward_host.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, Z, P]
         L.kda_prefill_forward_host.restype = I
+        L.kda_prefill_device_error.argtypes = [P, I]
+        L.kda_prefill_device_error.restype = I
         L.kda_l2norm_bf16.argtypes = [P, I64, I, P, P]
         L.kda_l2norm_bf16.restype = I
         _lib = L
@@ -135,6 +138,13 @@ def forward_host(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o, fi
                                         _ptr(staging), staging.numel(), _stream_ptr(stream))
     _check(rc, "kda_prefill_forward_host")
     return o, final_state
+
+
+def device_error(clear: bool = True) -> int:
+    """Bits set by kernel waits that gave up on the current device (0 when none); synchronises."""
+    w = ctypes.c_uint(0)
+    _check(lib().kda_prefill_device_error(ctypes.byref(w), int(clear)), "kda_prefill_device_error")
+    return int(w.value)
 
 
 def l2norm_bf16(x, out=None, stream=None):

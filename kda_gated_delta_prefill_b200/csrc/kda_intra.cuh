@@ -1,0 +1,447 @@
+// kda_intra.cuh -- intra-chunk kernel: everything of the chunk construction
+// that does not depend on the carried state, for one (chunk, value head)
+// item per CTA, fully parallel over items.
+//
+// "KDA Chunk Prefill on Ascend A3", section "Mathematical definition": for a
+// chunk of 64 tokens with inclusive per-channel cumulative gate G,
+//   L_ij   = beta_i sum_d k_id k_jd exp(G_id - G_jd)   (j < i)
+//   Aqk_ij = K^-0.5 sum_d q_id k_jd exp(G_id - G_jd)   (j <= i)
+//   A = (I + L)^-1 diag(beta),  W = A (exp(G) k),  U = A v,
+//   Qg = K^-0.5 q exp(G),  Kg = k exp(G_last - G),  and exp(G_last).
+// The item's results -- -W, Qg, Kg, Aqk, U (fp16) and exp(G_last) (fp32) --
+// are written as one contiguous block that the carry kernel copies straight
+// into its shared memory.
+//
+// Steps inside the CTA (256 threads):
+//   1. TMA tile loads of q, k (Q/K head h / (HV/H)), v, g; beta by plain
+//      loads.  Rows past the end of the sequence are zeroed (the page's zero
+//      padding of a partial chunk).
+//   2. L2 normalisation of q and k in place (exact rounding order).
+//   3. Gate factors from e_u = exp(g_u), one exponential per gate element:
+//      within each 16-token block the inclusive running product base_i and
+//      the exclusive suffix product b_j, block products P_J, and
+//      per-channel factors built from them, so that for i >= j
+//      exp(G_i - G_j) = base_i * c_IJ * b_j with every factor <= 1 except the
+//      diagonal-block c_II = 1/P_I.
+//   4. L and Aqk: bf16 tensor-core MMAs over the ten lower 16x16 block pairs
+//      (bf16 keeps the range of the gate-rescaled operands).
+//   5. A: exact float32 forward substitution in the 16x16 diagonal blocks,
+//      tf32 MMAs for the off-diagonal blocks.
+//   6. W and U: fp16 tensor-core MMAs.
+//   7. One bulk store of the item block.
+#pragma once
+#include "kda_common.cuh"
+#include "kda_norm.cuh"
+#include "ptx.cuh"
+
+namespace kda {
+
+struct IntraSmem {
+    static constexpr int Q = 0;          // bf16 [64][128] (two SW128 halves): q -> normalised -> K^-0.5 q*base
+    static constexpr int K = 16384;      // bf16: k -> normalised -> k*base
+    static constexpr int V = 32768;      // bf16 v -> fp16 v
+    static constexpr int G = 49152;      // fp32 [64][128] g; then KEXP fp16 (first half) and KBB bf16 (second half)
+    static constexpr int KEXP = G;
+    static constexpr int KBB = G + 16384;
+    static constexpr int OUT = 81920;    // the item block (ItemLayout), 74240 bytes
+    static constexpr int L = 156672;     // fp32 [64][64]
+    static constexpr int X = 173056;     // fp32 [64][64]
+    static constexpr int A = 189440;     // fp16 [64][64]
+    static constexpr int BETA = 197632;  // fp32 [64]
+    static constexpr int CF = 197888;    // bf16x2 [10][64] block-pair factors
+    static constexpr int TS = 200448;    // fp32 3 x [16][24] solve scratch
+    static constexpr int BAR = 205056;   // mbarrier
+    static constexpr int TOTAL = 205120;
+};
+
+struct IntraParams {
+    const float *beta;
+    const int32_t *cu;         // [N+1] or null
+    const int32_t *chunk_off;  // [N+1] chunk offsets of the packed sequences, or null
+    uint8_t *items;            // [num_chunks][HV] item blocks
+    unsigned *err;
+    int B, T, H, HV, N;
+    int chunks_per_seq;        // ceil(T/64) when cu is null
+};
+
+constexpr int TSW = 24;  // row stride (floats) of the 16x16 solve scratch; conflict-free column reads
+
+// Off-diagonal block of X = (I+L)^-1: X_IJ = -D_I * sum_{M=J}^{I-1} L_IM X_MJ (one warp, tf32 MMAs).
+__device__ __forceinline__ void solve_block(const uint8_t *sL, uint8_t *sX, float *ts, int I, int J, int lane)
+{
+    const int g = lane >> 2, t = lane & 3;
+    auto Lat = [&](int r, int c) { return *reinterpret_cast<const float *>(sL + swz(r, c * 4, 256)); };
+    auto Xat = [&](int r, int c) { return *reinterpret_cast<const float *>(sX + swz(r, c * 4, 256)); };
+    float acc[2][4] = {};
+    for (int M = J; M < I; ++M) {
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t a[4];
+            a[0] = to_tf32(Lat(16 * I + g, 16 * M + 8 * ks + t));
+            a[1] = to_tf32(Lat(16 * I + g + 8, 16 * M + 8 * ks + t));
+            a[2] = to_tf32(Lat(16 * I + g, 16 * M + 8 * ks + t + 4));
+            a[3] = to_tf32(Lat(16 * I + g + 8, 16 * M + 8 * ks + t + 4));
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const uint32_t b0 = to_tf32(Xat(16 * M + 8 * ks + t, 16 * J + 8 * nt + g));
+                const uint32_t b1 = to_tf32(Xat(16 * M + 8 * ks + t + 4, 16 * J + 8 * nt + g));
+                mma_tf32(acc[nt], a, b0, b1);
+            }
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        ts[g * TSW + 8 * nt + 2 * t] = acc[nt][0];
+        ts[g * TSW + 8 * nt + 2 * t + 1] = acc[nt][1];
+        ts[(g + 8) * TSW + 8 * nt + 2 * t] = acc[nt][2];
+        ts[(g + 8) * TSW + 8 * nt + 2 * t + 1] = acc[nt][3];
+    }
+    __syncwarp();
+    float x[2][4] = {};
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        uint32_t a[4];
+        a[0] = to_tf32(Xat(16 * I + g, 16 * I + 8 * ks + t));
+        a[1] = to_tf32(Xat(16 * I + g + 8, 16 * I + 8 * ks + t));
+        a[2] = to_tf32(Xat(16 * I + g, 16 * I + 8 * ks + t + 4));
+        a[3] = to_tf32(Xat(16 * I + g + 8, 16 * I + 8 * ks + t + 4));
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t b0 = to_tf32(ts[(8 * ks + t) * TSW + 8 * nt + g]);
+            const uint32_t b1 = to_tf32(ts[(8 * ks + t + 4) * TSW + 8 * nt + g]);
+            mma_tf32(x[nt], a, b0, b1);
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int c = 16 * J + 8 * nt + 2 * t;
+        *reinterpret_cast<float2 *>(sX + swz(16 * I + g, c * 4, 256)) = make_float2(-x[nt][0], -x[nt][1]);
+        *reinterpret_cast<float2 *>(sX + swz(16 * I + g + 8, c * 4, 256)) = make_float2(-x[nt][2], -x[nt][3]);
+    }
+    __syncwarp();
+}
+
+__global__ void __launch_bounds__(256, 1)
+    kda_intra_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                     const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg,
+                     const IntraParams p)
+{
+    using S = IntraSmem;
+    extern __shared__ __align__(1024) uint8_t sm[];
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g8 = lane >> 2, t4 = lane & 3;
+
+    // ---- item -> (row of the chunk start, valid rows) ----
+    const int h = blockIdx.x % p.HV;
+    const int ci = blockIdx.x / p.HV;
+    int64_t row0;
+    int nvalid;
+    if (p.cu) {
+        const int nc = p.chunk_off[p.N];
+        if (ci >= nc) return;
+        int lo = 0, hi = p.N - 1;  // last n with chunk_off[n] <= ci
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.chunk_off[mid] <= ci) lo = mid; else hi = mid - 1;
+        }
+        const int c = ci - p.chunk_off[lo];
+        const int len = p.cu[lo + 1] - p.cu[lo];
+        row0 = p.cu[lo] + static_cast<int64_t>(c) * CH;
+        nvalid = min(CH, len - c * CH);
+    } else {
+        const int b = ci / p.chunks_per_seq, c = ci % p.chunks_per_seq;
+        row0 = static_cast<int64_t>(b) * p.T + static_cast<int64_t>(c) * CH;
+        nvalid = min(CH, p.T - c * CH);
+    }
+    const int hq = h / (p.HV / p.H);
+    uint8_t *out_g = p.items + (static_cast<int64_t>(ci) * p.HV + h) * ITEM_BYTES;
+    uint8_t *out = sm + S::OUT;
+
+    // ---- 1. loads ----
+    const uint32_t bar = sb + S::BAR;
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        mbar_expect_tx(bar, 3 * 16384 + 32768);
+        const int z = static_cast<int>(row0);
+        tma_load_3d(sb + S::Q, &tq, 0, hq, z, bar);
+        tma_load_3d(sb + S::Q + 8192, &tq, 64, hq, z, bar);
+        tma_load_3d(sb + S::K, &tk, 0, hq, z, bar);
+        tma_load_3d(sb + S::K + 8192, &tk, 64, hq, z, bar);
+        tma_load_3d(sb + S::V, &tv, 0, h, z, bar);
+        tma_load_3d(sb + S::V + 8192, &tv, 64, h, z, bar);
+        tma_load_3d(sb + S::G, &tg, 0, h, z, bar);
+    }
+    float *sbeta = reinterpret_cast<float *>(sm + S::BETA);
+    if (tid < CH) sbeta[tid] = (tid < nvalid) ? p.beta[(row0 + tid) * p.HV + h] : 0.f;
+    if (!mbar_wait(bar, 0)) {
+        atomicOr(p.err, ERR_TMA_WAIT);
+        return;
+    }
+    if (nvalid < CH) {  // zero the padding rows of a partial chunk
+        for (int idx = tid; idx < (CH - nvalid) * 64; idx += 256) {
+            const int r = nvalid + idx / 64, w = idx % 64;  // 64 words of 16 bytes per row over q,k,v,g
+            uint4 *dst;
+            if (w < 48) {
+                const int buf = w / 16, c16 = w % 16;  // q, k, v: two halves of 8 chunks
+                dst = reinterpret_cast<uint4 *>(sm + buf * 16384 + (c16 >> 3) * 8192 + r * 128 + ((c16 & 7) << 4));
+            } else {
+                dst = reinterpret_cast<uint4 *>(sm + S::G + r * 512 + (w - 48) * 16);
+                dst[16] = make_uint4(0, 0, 0, 0);  // g rows are 32 words; cover the second 16 too
+            }
+            *dst = make_uint4(0, 0, 0, 0);
+        }
+    }
+    __syncthreads();
+
+    // ---- 2. normalise q and k (thread = row half), v -> fp16 ----
+    {
+        const int r = tid >> 1, half = tid & 1;
+        uint8_t *tile = sm + (r < CH ? S::Q : S::K) + half * 8192 + (r & 63) * 128;
+        const int rs = r & 7;
+        uint4 raw[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) raw[c] = *reinterpret_cast<const uint4 *>(tile + ((c ^ rs) << 4));
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 x = unpack_bf16(w[j]);
+                acc = add2(acc, mul2(x, x));
+            }
+        }
+        float ss = __fadd_rn(acc.x, acc.y);
+        ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, 1));
+        const float den = __fsqrt_rn(__fadd_rn(ss, 1e-6f));
+        const float rr = __frcp_rn(den);
+        const float2 r2 = make_float2(rr, rr), nd2 = make_float2(-den, -den);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 x = unpack_bf16(w[j]);
+                const float2 q0 = mul2(x, r2);
+                const float2 e = fma2(q0, nd2, x);
+                const float2 y = fma2(e, r2, q0);
+                w[j] = pack_bf16(y.x, y.y);
+            }
+            *reinterpret_cast<uint4 *>(tile + ((c ^ rs) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        // v: 1024 chunks of 16 bytes, 4 per thread, bf16 -> fp16 in place
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            uint4 *pv = reinterpret_cast<uint4 *>(sm + S::V) + (tid + 256 * k);
+            uint4 u = *pv;
+            uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 x = unpack_bf16(w[j]);
+                w[j] = pack_f16(x.x, x.y);
+            }
+            *pv = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+    __syncthreads();
+
+    // ---- 3. gate factors and operands: thread = (block J, channel pair dp) ----
+    {
+        const int J = tid & 3, dp = tid >> 2, d0 = 2 * dp;
+        float2 e[16], bb[16];
+        const float2 l2e = make_float2(1.4426950408889634f, 1.4426950408889634f);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const float2 gv = *reinterpret_cast<const float2 *>(sm + S::G + (16 * J + u) * 512 + d0 * 4);
+            const float2 y = mul2(gv, l2e);
+            e[u] = make_float2(ex2(y.x), ex2(y.y));
+        }
+        bb[15] = make_float2(1.f, 1.f);
+#pragma unroll
+        for (int u = 14; u >= 0; --u) bb[u] = mul2(bb[u + 1], e[u + 1]);
+#pragma unroll
+        for (int u = 1; u < 16; ++u) e[u] = mul2(e[u - 1], e[u]);  // e -> inclusive running product (base)
+        // block products of this channel pair from the four lanes that hold blocks 0..3
+        float2 P[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            P[j].x = __shfl_sync(0xffffffffu, e[15].x, (lane & ~3) | j);
+            P[j].y = __shfl_sync(0xffffffffu, e[15].y, (lane & ~3) | j);
+        }
+        // E_J = prod_{J'<J} P_J' (gate from the chunk start to the block start), F_J = prod_{J'>J} P_J'
+        const float2 one2 = make_float2(1.f, 1.f);
+        const float2 P01 = mul2(P[0], P[1]), P23 = mul2(P[2], P[3]);
+        const float2 myE = (J == 0) ? one2 : (J == 1) ? P[0] : (J == 2) ? P01 : mul2(P01, P[2]);
+        const float2 myF = (J == 3) ? one2 : (J == 2) ? P[3] : (J == 1) ? P23 : mul2(P[1], P23);
+        const float scale = 0.08838834764831845f;  // 128^-0.5 in float32
+        const float2 sE = mul2(myE, make_float2(scale, scale));
+        if (J == 0) {
+            // per-channel factors of the ten block pairs, as bf16 pairs; c_II = 1/P_I
+            uint32_t *cf = reinterpret_cast<uint32_t *>(sm + S::CF);
+            auto rcp2 = [](float2 a) {
+                return make_float2(__frcp_rn(fmaxf(a.x, 1e-37f)), __frcp_rn(fmaxf(a.y, 1e-37f)));
+            };
+            const float2 one = make_float2(1.f, 1.f);
+            const float2 cv[10] = {rcp2(P[0]), one, rcp2(P[1]), P[1], one, rcp2(P[2]), mul2(P[1], P[2]), P[2], one,
+                                   rcp2(P[3])};
+#pragma unroll
+            for (int pi = 0; pi < 10; ++pi) cf[pi * 64 + dp] = pack_bf16(cv[pi].x, cv[pi].y);
+            const float2 gl = mul2(P01, P23);
+            *reinterpret_cast<float2 *>(out + ITEM_GL + d0 * 4) = gl;
+        }
+        __syncthreads();  // every g read is done: the G region becomes KEXP / KBB
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int i = 16 * J + u;
+            const uint32_t a16 = lh(i, d0);
+            const float2 xk = unpack_bf16(*reinterpret_cast<const uint32_t *>(sm + S::K + a16));
+            const float2 xq = unpack_bf16(*reinterpret_cast<const uint32_t *>(sm + S::Q + a16));
+            const float2 kb = mul2(xk, e[u]);
+            const float2 qb = mul2(mul2(xq, e[u]), make_float2(scale, scale));
+            const float2 kx = mul2(kb, myE);
+            const float2 qg = mul2(mul2(xq, e[u]), sE);
+            const float2 kbb = mul2(xk, bb[u]);
+            const float2 kg = mul2(kbb, myF);
+            *reinterpret_cast<uint32_t *>(sm + S::K + a16) = pack_bf16(kb.x, kb.y);
+            *reinterpret_cast<uint32_t *>(sm + S::Q + a16) = pack_bf16(qb.x, qb.y);
+            *reinterpret_cast<uint32_t *>(sm + S::KEXP + a16) = pack_f16(kx.x, kx.y);
+            *reinterpret_cast<uint32_t *>(sm + S::KBB + a16) = pack_bf16(kbb.x, kbb.y);
+            const uint32_t a256 = swz(i, d0 * 2, 256);
+            *reinterpret_cast<uint32_t *>(out + ITEM_QG + a256) = pack_f16(qg.x, qg.y);
+            *reinterpret_cast<uint32_t *>(out + ITEM_KG + a256) = pack_f16(kg.x, kg.y);
+        }
+    }
+    __syncthreads();
+
+    // ---- 4. L and Aqk over the ten lower block pairs (bf16 MMAs) ----
+    for (int pidx = warp; pidx < 10; pidx += 8) {
+        const int I = (pidx >= 6) ? 3 : (pidx >= 3) ? 2 : (pidx >= 1) ? 1 : 0;
+        const int J = pidx - I * (I + 1) / 2;
+        const uint32_t *cf = reinterpret_cast<const uint32_t *>(sm + S::CF) + pidx * 64;
+        float accL[2][4] = {}, accQ[2][4] = {};
+        const int mi = lane >> 3;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            uint32_t ak[4], aq[4], b[4];
+            const int ar = 16 * I + (mi & 1) * 8 + (lane & 7), ac = 16 * ks + (mi >> 1) * 8;
+            ldsm_x4(sb + S::K + lh(ar, ac), ak[0], ak[1], ak[2], ak[3]);
+            ldsm_x4(sb + S::Q + lh(ar, ac), aq[0], aq[1], aq[2], aq[3]);
+            const uint32_t c_lo = cf[8 * ks + t4], c_hi = cf[8 * ks + 4 + t4];
+            ak[0] = hmul2_bf16(ak[0], c_lo);
+            ak[1] = hmul2_bf16(ak[1], c_lo);
+            ak[2] = hmul2_bf16(ak[2], c_hi);
+            ak[3] = hmul2_bf16(ak[3], c_hi);
+            aq[0] = hmul2_bf16(aq[0], c_lo);
+            aq[1] = hmul2_bf16(aq[1], c_lo);
+            aq[2] = hmul2_bf16(aq[2], c_hi);
+            aq[3] = hmul2_bf16(aq[3], c_hi);
+            const int br = 16 * J + (mi >> 1) * 8 + (lane & 7), bc = 16 * ks + (mi & 1) * 8;
+            ldsm_x4(sb + S::KBB + lh(br, bc), b[0], b[1], b[2], b[3]);
+            mma_bf16(accL[0], ak, b[0], b[1]);
+            mma_bf16(accL[1], ak, b[2], b[3]);
+            mma_bf16(accQ[0], aq, b[0], b[1]);
+            mma_bf16(accQ[1], aq, b[2], b[3]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int i = 16 * I + g8 + 8 * hr;
+                const int j = 16 * J + 8 * nt + 2 * t4;
+                const float bi = sbeta[i];
+                const float l0 = (j < i) ? bi * accL[nt][2 * hr] : 0.f;
+                const float l1 = (j + 1 < i) ? bi * accL[nt][2 * hr + 1] : 0.f;
+                const float q0 = (j <= i) ? accQ[nt][2 * hr] : 0.f;
+                const float q1 = (j + 1 <= i) ? accQ[nt][2 * hr + 1] : 0.f;
+                *reinterpret_cast<float2 *>(sm + S::L + swz(i, j * 4, 256)) = make_float2(l0, l1);
+                *reinterpret_cast<uint32_t *>(out + ITEM_AQK + swz(i, j * 2, 128)) = pack_f16(q0, q1);
+            }
+    }
+    __syncthreads();
+
+    // ---- 5. A = (I+L)^-1 diag(beta) ----
+    uint8_t *sX = sm + S::X;
+    if (warp < 4 && lane < 16) {  // diagonal blocks: exact float32 forward substitution, lane = column
+        const int I = warp, cidx = lane;
+        float dcol[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float acc = (j == cidx) ? 1.f : 0.f;
+#pragma unroll
+            for (int m = 0; m < j; ++m)
+                acc = __fmaf_rn(-*reinterpret_cast<const float *>(sm + S::L + swz(16 * I + j, (16 * I + m) * 4, 256)),
+                                dcol[m], acc);
+            dcol[j] = acc;
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            *reinterpret_cast<float *>(sX + swz(16 * I + j, (16 * I + cidx) * 4, 256)) = dcol[j];
+    }
+    __syncthreads();
+    {
+        float *ts = reinterpret_cast<float *>(sm + S::TS) + (warp % 3) * 16 * TSW;
+        if (warp < 3) solve_block(sm + S::L, sX, ts, warp + 1, warp, lane);
+        __syncthreads();
+        if (warp < 2) solve_block(sm + S::L, sX, ts, warp + 2, warp, lane);
+        __syncthreads();
+        if (warp < 1) solve_block(sm + S::L, sX, ts, 3, 0, lane);
+        __syncthreads();
+    }
+    for (int idx = tid; idx < CH * CH / 2; idx += 256) {
+        const int i = idx >> 5, j = (idx & 31) * 2;
+        const float2 x = *reinterpret_cast<const float2 *>(sX + swz(i, j * 4, 256));
+        const float a0 = (j <= i) ? x.x * sbeta[j] : 0.f;
+        const float a1 = (j + 1 <= i) ? x.y * sbeta[j + 1] : 0.f;
+        *reinterpret_cast<uint32_t *>(sm + S::A + swz(i, j * 2, 128)) = pack_f16(a0, a1);
+    }
+    __syncthreads();
+
+    // ---- 6. -W = -A (exp(G) k) and U = A v (fp16 MMAs); warp = 16 columns ----
+    {
+        const int mi = lane >> 3;
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+            float w[2][4] = {}, u[2][4] = {};
+            for (int ks = 0; ks <= mt; ++ks) {
+                uint32_t a[4];
+                ldsm_x4(sb + S::A + swz(16 * mt + (mi & 1) * 8 + (lane & 7), (16 * ks + (mi >> 1) * 8) * 2, 128), a[0], a[1],
+                        a[2], a[3]);
+                const int tok = 16 * ks + (mi & 1) * 8 + (lane & 7), col = 16 * warp + (mi >> 1) * 8;
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(sb + S::KEXP + lh(tok, col), b0, b1, b2, b3);
+                mma_f16(w[0], a, b0, b1);
+                mma_f16(w[1], a, b2, b3);
+                ldsm_x4_t(sb + S::V + lh(tok, col), b0, b1, b2, b3);
+                mma_f16(u[0], a, b0, b1);
+                mma_f16(u[1], a, b2, b3);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int r = 16 * mt + g8 + 8 * hr;
+                    const int c = 16 * warp + 8 * nt + 2 * t4;
+                    *reinterpret_cast<uint32_t *>(out + ITEM_WN + swz(r, c * 2, 256)) =
+                        pack_f16(-w[nt][2 * hr], -w[nt][2 * hr + 1]);
+                    *reinterpret_cast<uint32_t *>(out + ITEM_U + (c >> 5) * 4096 + r * 64 + (c & 31) * 2) =
+                        pack_f16(u[nt][2 * hr], u[nt][2 * hr + 1]);
+                }
+        }
+    }
+
+    // ---- 7. bulk store of the item block ----
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+        bulk_store(out_g, sb + S::OUT, ITEM_BYTES);
+        bulk_commit();
+        bulk_wait_all();
+    }
+}
+
+}  // namespace kda

@@ -1,15 +1,26 @@
 // kda_prefill.cu -- C ABI of the KDA chunk-prefill forward (declared in
-// include/kda_prefill.h): host-side argument checks and kernel launches.
-// No numeric work happens on the host; every step of the forward runs in
-// the kernels of kda_fused.cuh / kda_norm.cuh.
+// include/kda_prefill.h): host-side argument checks, workspace layout,
+// tensor maps and kernel launches.  No numeric work happens on the host;
+// every step of the forward runs in the kernels of kda_intra.cuh,
+// kda_carry.cuh, kda_sched.cuh and kda_norm.cuh.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
-#include "kda_fused.cuh"
+#include "kda_carry.cuh"
+#include "kda_intra.cuh"
 #include "kda_norm.cuh"
 #include "kda_prefill.h"
+#include "kda_sched.cuh"
+
+// Bits set by kernels whose bounded waits gave up (see ptx.cuh).  Host code
+// reaches it only through the address cudaGetSymbolAddress returns.
+static __device__ unsigned g_kda_device_error;
 
 namespace {
 
@@ -18,6 +29,7 @@ using kda::DK;
 using kda::DV;
 
 constexpr size_t kAlign = 256;
+constexpr int kMaxDevices = 64;
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -30,28 +42,60 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb)
     return pa < pb + nb && pb < pa + na;
 }
 
-int num_sms(int dev)
+// Per-device facts looked up once: SM count and the error word's device address.
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 148;
+    unsigned *err = nullptr;
+};
+std::mutex g_info_mu;
+DeviceInfo g_info[kMaxDevices];
+
+cudaError_t device_info(DeviceInfo &out)
 {
-    static int cached[64] = {0};
-    if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
-    int n = 148;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
-    if (dev >= 0 && dev < 64) cached[dev] = n;
-    return n;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_info_mu);
+    DeviceInfo &d = g_info[dev];
+    if (!d.ready) {
+        e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_kda_device_error);
+        if (e != cudaSuccess) return e;
+        d.ready = true;
+    }
+    out = d;
+    return cudaSuccess;
 }
 
-template <int NW>
-cudaError_t launch_fused(const kda::FwdParams &p, int units, cudaStream_t stream)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 {
-    using S = kda::Smem<NW>;
-    cudaError_t err = cudaFuncSetAttribute(kda::kda_fused_fwd_kernel<NW>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, S::TOTAL);
-    if (err != cudaSuccess) return err;
-    kda::FwdParams q = p;
-    q.nslices = DV / S::VS;
-    const int grid = units * q.nslices;
-    kda::kda_fused_fwd_kernel<NW><<<grid, NW * 32, S::TOTAL, stream>>>(q);
-    return cudaGetLastError();
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// [rows][heads][128] tensor as a 3D tiled map; one TMA box = 64 rows of one head.
+bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes, int heads, int64_t rows,
+              int box_inner, CUtensorMapSwizzle sw)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(128) * elem_bytes, static_cast<cuuint64_t>(heads) * 128 * elem_bytes};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), 1, static_cast<cuuint32_t>(CH)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 struct Dims {
@@ -66,10 +110,52 @@ kda_status_t check_dims(int B, int T, int H, int HV, int K, int V, bool varlen, 
     if (HV % H != 0) return KDA_ERR_INVALID_ARG;
     if (K != DK || V != DV) return KDA_ERR_UNSUPPORTED;
     if (varlen && (B != 1 || num_seqs <= 0)) return KDA_ERR_INVALID_ARG;
-    const int64_t units = static_cast<int64_t>(varlen ? num_seqs : B) * HV;
-    if (units * 2 > INT32_MAX) return KDA_ERR_UNSUPPORTED;
-    d = Dims{B, T, H, HV, K, V, varlen ? num_seqs : B, varlen};
+    // token rows are TMA coordinates (int32); grids stay below 2^31 blocks
+    if (static_cast<int64_t>(B) * T > INT_MAX - CH) return KDA_ERR_UNSUPPORTED;
+    const int64_t N = varlen ? num_seqs : B;
+    const int64_t max_chunks = varlen ? (static_cast<int64_t>(T) + CH - 1) / CH + N
+                                      : static_cast<int64_t>(B) * ((T + CH - 1) / CH);
+    if (max_chunks * HV > INT_MAX || N * HV * 4 > INT_MAX) return KDA_ERR_UNSUPPORTED;
+    d = Dims{B, T, H, HV, K, V, static_cast<int>(N), varlen};
     return KDA_OK;
+}
+
+// Workspace: [chunk_off (N+1) | order (N)] for packed batches, then the item blocks.
+struct Workspace {
+    size_t chunk_off = 0, order = 0, items = 0, total = 0;
+    int64_t max_chunks = 0;
+};
+
+Workspace workspace_layout(int B, int T, int HV, int num_seqs)
+{
+    Workspace w;
+    const bool varlen = num_seqs > 0;
+    w.max_chunks = varlen ? (static_cast<int64_t>(T) + CH - 1) / CH + num_seqs
+                          : static_cast<int64_t>(B) * ((T + CH - 1) / CH);
+    size_t off = 0;
+    if (varlen) {
+        w.chunk_off = off;
+        off += round_up((static_cast<size_t>(num_seqs) + 1) * 4, kAlign);
+        w.order = off;
+        off += round_up(static_cast<size_t>(num_seqs) * 4, kAlign);
+    }
+    w.items = off;
+    off += static_cast<size_t>(w.max_chunks) * HV * kda::ITEM_BYTES;
+    w.total = round_up(off, kAlign);
+    return w;
+}
+
+template <int NW>
+cudaError_t launch_carry(const kda::CarryParams &p0, int units, cudaStream_t stream)
+{
+    using S = kda::CarrySmem<NW>;
+    cudaError_t err = cudaFuncSetAttribute(kda::kda_carry_kernel<NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           S::TOTAL);
+    if (err != cudaSuccess) return err;
+    kda::CarryParams p = p0;
+    p.nslices = DV / S::VS;
+    kda::kda_carry_kernel<NW><<<units * p.nslices, (NW + 1) * 32, S::TOTAL, stream>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -89,9 +175,19 @@ extern "C" const char *kda_status_string(kda_status_t s)
 
 extern "C" size_t kda_prefill_workspace_size(int B, int T, int H, int HV, int K, int V, int num_seqs)
 {
-    (void)B; (void)T; (void)H; (void)HV; (void)K; (void)V;
-    if (num_seqs <= 0) return 0;
-    return round_up(static_cast<size_t>(num_seqs) * sizeof(int32_t), kAlign);
+    Dims d;
+    if (check_dims(B, T, H, HV, K, V, num_seqs > 0, num_seqs, d) != KDA_OK) return 0;
+    return workspace_layout(B, T, HV, num_seqs > 0 ? num_seqs : 0).total;
+}
+
+extern "C" kda_status_t kda_prefill_device_error(unsigned *word, int clear)
+{
+    if (!word) return KDA_ERR_INVALID_ARG;
+    DeviceInfo info;
+    if (device_info(info) != cudaSuccess) return KDA_ERR_CUDA;
+    if (cudaMemcpy(word, info.err, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+    if (clear && cudaMemset(info.err, 0, sizeof(unsigned)) != cudaSuccess) return KDA_ERR_CUDA;
+    return KDA_OK;
 }
 
 extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const void *v, const float *g,
@@ -124,52 +220,74 @@ extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const 
     if (initial_state && initial_state != final_state && overlaps(initial_state, ns, final_state, ns))
         return KDA_ERR_INVALID_ARG;
 
-    const size_t need = kda_prefill_workspace_size(B, T, H, HV, K, V, varlen ? num_seqs : 0);
-    if (need > 0) {
-        if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
-        if (!aligned(workspace, kAlign)) return KDA_ERR_MISALIGNED;
-        if (overlaps(workspace, need, o, nvb) || overlaps(workspace, need, final_state, ns))
-            return KDA_ERR_INVALID_ARG;
-    }
+    const Workspace ws = workspace_layout(B, T, HV, varlen ? num_seqs : 0);
+    if (!workspace || workspace_bytes < ws.total) return KDA_ERR_WORKSPACE;
+    if (!aligned(workspace, kAlign)) return KDA_ERR_MISALIGNED;
+    for (int i = 0; i < 6; ++i)
+        if (overlaps(workspace, ws.total, ins[i], in_n[i])) return KDA_ERR_INVALID_ARG;
+    if (overlaps(workspace, ws.total, o, nvb) || overlaps(workspace, ws.total, final_state, ns) ||
+        overlaps(workspace, ws.total, initial_state, ns))
+        return KDA_ERR_INVALID_ARG;
 
+    DeviceInfo info;
+    if (device_info(info) != cudaSuccess) return KDA_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
-
-    kda::FwdParams p{};
-    p.q = static_cast<const __nv_bfloat16 *>(q);
-    p.k = static_cast<const __nv_bfloat16 *>(k);
-    p.v = static_cast<const __nv_bfloat16 *>(v);
-    p.g = g;
-    p.beta = beta;
-    p.s0 = initial_state;
-    p.cu = cu_seqlens;
-    p.order = nullptr;
-    p.o = static_cast<__nv_bfloat16 *>(o);
-    p.sN = final_state;
-    p.B = B;
-    p.T = T;
-    p.H = H;
-    p.HV = HV;
-    p.N = d.N;
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    int32_t *chunk_off = varlen ? reinterpret_cast<int32_t *>(wsb + ws.chunk_off) : nullptr;
+    int32_t *order = varlen ? reinterpret_cast<int32_t *>(wsb + ws.order) : nullptr;
+    uint8_t *items = wsb + ws.items;
 
     if (varlen) {
-        int32_t *order = static_cast<int32_t *>(workspace);
-        const int threads = 256;
-        const int blocks = (num_seqs + threads - 1) / threads;
-        kda::seq_order_kernel<<<blocks, threads, 0, s>>>(cu_seqlens, num_seqs, order);
+        kda::chunk_offsets_kernel<<<1, 1024, 0, s>>>(cu_seqlens, num_seqs, chunk_off);
+        kda::seq_order_kernel<<<(num_seqs + 255) / 256, 256, 0, s>>>(cu_seqlens, num_seqs, order);
         if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
-        p.order = order;
     }
 
-    // Two value-column slices (4 warps each) when the (sequence, head) units
-    // alone would leave SMs idle; otherwise one slice of 8 warps per unit.
+    if (tokens > 0) {
+        CUtensorMap tq, tk, tv, tg;
+        const int64_t rows = tokens;
+        if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HV, rows, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HV, rows, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return KDA_ERR_CUDA;
+        kda::IntraParams ip{};
+        ip.beta = beta;
+        ip.cu = cu_seqlens;
+        ip.chunk_off = chunk_off;
+        ip.items = items;
+        ip.err = info.err;
+        ip.B = B;
+        ip.T = T;
+        ip.H = H;
+        ip.HV = HV;
+        ip.N = d.N;
+        ip.chunks_per_seq = (T + CH - 1) / CH;
+        if (cudaFuncSetAttribute(kda::kda_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kda::IntraSmem::TOTAL) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        kda::kda_intra_kernel<<<static_cast<int>(ws.max_chunks * HV), 256, kda::IntraSmem::TOTAL, s>>>(tq, tk, tv, tg,
+                                                                                                        ip);
+        if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+    }
+
+    kda::CarryParams cp{};
+    cp.items = items;
+    cp.s0 = initial_state;
+    cp.cu = cu_seqlens;
+    cp.chunk_off = chunk_off;
+    cp.order = order;
+    cp.o = static_cast<__nv_bfloat16 *>(o);
+    cp.sN = final_state;
+    cp.err = info.err;
+    cp.T = T;
+    cp.HV = HV;
+    cp.N = d.N;
+    cp.chunks_per_seq = (T + CH - 1) / CH;
+    // Value-column slices: 4 slices of 32 columns when (sequence, head) units
+    // alone would leave most SMs idle, else 2 slices of 64.
     const int units = d.N * HV;
-    cudaError_t err;
-    if (units * 2 <= num_sms(dev))
-        err = launch_fused<4>(p, units, s);
-    else
-        err = launch_fused<8>(p, units, s);
+    const cudaError_t err = (units * 4 <= info.sms) ? launch_carry<2>(cp, units, s) : launch_carry<4>(cp, units, s);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -251,10 +369,10 @@ extern "C" kda_status_t kda_l2norm_bf16(const void *x, int64_t rows, int K, void
     if (!aligned(x, 16) || !aligned(out, 16)) return KDA_ERR_MISALIGNED;
     const size_t n = static_cast<size_t>(rows) * K * 2;
     if (x != out && overlaps(x, n, out, n)) return KDA_ERR_INVALID_ARG;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
+    DeviceInfo info;
+    if (device_info(info) != cudaSuccess) return KDA_ERR_CUDA;
     const int64_t blocks_needed = (rows + 7) / 8;
-    const int64_t cap = static_cast<int64_t>(num_sms(dev)) * 8;
+    const int64_t cap = static_cast<int64_t>(info.sms) * 8;
     const int blocks = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
     kda::l2norm_bf16_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const __nv_bfloat16 *>(x), rows, static_cast<__nv_bfloat16 *>(out));

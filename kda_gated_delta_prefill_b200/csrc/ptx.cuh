@@ -1,28 +1,85 @@
 // ptx.cuh -- thin inline-PTX wrappers used by the KDA kernels (sm_100a).
 #pragma once
-#include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
 
 namespace kda {
+
+// ---- device error word (bounded waits that gave up set a bit here) ----
+enum : unsigned { ERR_TMA_WAIT = 1u, ERR_PIPE_FULL_WAIT = 2u, ERR_PIPE_EMPTY_WAIT = 4u };
+// Spin budget of every wait, in SM clock cycles (about one second at 2 GHz).
+constexpr long long kWaitBudget = 2000000000LL;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// ---- asynchronous global -> shared copies (zero-filled when src_bytes == 0) ----
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+// ---- mbarrier ----
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
 {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes)
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Wait for the phase with the given parity; gives up after kWaitBudget cycles
+// and returns false (the caller records an error and stops).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > kWaitBudget) return false;
+    return true;
+}
+
+// ---- bulk / tensor copies (async proxy) ----
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
 }
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t src_bytes)
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes)
 {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src), "r"(src_bytes)
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst), "r"(src), "r"(bytes)
                  : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 
 // ---- ldmatrix ----
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
@@ -38,8 +95,7 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t 
                  : "r"(addr));
 }
 
-// ---- warp-level tensor-core MMAs ----
-// D = A(16x16 bf16, row) * B(16x8 bf16, col) + D, fp32 accumulate.
+// ---- warp-level tensor-core MMAs (fp32 accumulate) ----
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
     asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
@@ -47,7 +103,13 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
                  : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-// D = A(16x8 tf32, row) * B(8x8 tf32, col) + D, fp32 accumulate.
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+                 "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
     asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
@@ -62,14 +124,53 @@ __device__ __forceinline__ uint32_t to_tf32(float x)
     return r;
 }
 
-// ---- conversions ----
+// ---- packed conversions and arithmetic ----
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits), .y = hi
-    return *reinterpret_cast<uint32_t *>(&v);
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
 }
 __device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+__device__ __forceinline__ float2 unpack_bf16(uint32_t u) { return make_float2(bf16lo(u), bf16hi(u)); }
+__device__ __forceinline__ float2 unpack_f16(uint32_t u)
+{
+    __half2 h = *reinterpret_cast<__half2 *>(&u);
+    return __half22float2(h);
+}
+__device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;\n" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+// Packed float32 pairs (sm_100): one instruction for two lanes of work.
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
+{
+    unsigned long long A = *reinterpret_cast<unsigned long long *>(&a), B = *reinterpret_cast<unsigned long long *>(&b), D;
+    asm("mul.rn.f32x2 %0, %1, %2;\n" : "=l"(D) : "l"(A), "l"(B));
+    return *reinterpret_cast<float2 *>(&D);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b)
+{
+    unsigned long long A = *reinterpret_cast<unsigned long long *>(&a), B = *reinterpret_cast<unsigned long long *>(&b), D;
+    asm("add.rn.f32x2 %0, %1, %2;\n" : "=l"(D) : "l"(A), "l"(B));
+    return *reinterpret_cast<float2 *>(&D);
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    unsigned long long A = *reinterpret_cast<unsigned long long *>(&a), B = *reinterpret_cast<unsigned long long *>(&b),
+                       C = *reinterpret_cast<unsigned long long *>(&c), D;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(D) : "l"(A), "l"(B), "l"(C));
+    return *reinterpret_cast<float2 *>(&D);
+}
 
 // 2^x on the special-function unit.
 __device__ __forceinline__ float ex2(float x)
@@ -79,12 +180,19 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
-// Byte offset of (row, col_byte) in a row-major shared tile whose rows are
-// row_bytes long (>= 128): 16-byte chunks are XOR-swizzled by row % 8 so that
-// eight consecutive rows of one chunk column fall into distinct bank groups.
+// ---- shared-memory tile layouts ----
+// Rows of row_bytes (>= 128) with 16-byte chunks XOR-swizzled by row % 8 (the
+// chunk index's low three bits), so that eight consecutive rows of one chunk
+// column fall into distinct bank groups.
 __device__ __forceinline__ uint32_t swz(int row, int col_byte, int row_bytes)
 {
     return static_cast<uint32_t>(row * row_bytes + ((((col_byte >> 4) ^ (row & 7))) << 4) + (col_byte & 15));
+}
+// A [64][128] 16-bit tile stored as two column halves of [64][64] in the
+// 128-byte-swizzle layout that a TMA tile load with SWIZZLE_128B produces.
+__device__ __forceinline__ uint32_t lh(int row, int col)
+{
+    return static_cast<uint32_t>((col >> 6) * 8192 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2);
 }
 
 }  // namespace kda

@@ -42,16 +42,23 @@ def test_status_strings(L):
 
 
 def test_workspace_size(L):
-    assert L.kda_prefill_workspace_size(2, 4096, 96, 96, 128, 128, 0) == 0
-    assert L.kda_prefill_workspace_size(1, 11210, 8, 32, 128, 128, 7) == 256
-    assert L.kda_prefill_workspace_size(1, 10, 1, 1, 128, 128, 65) == 512
+    item = 74240
+    # plain batch: B * ceil(T/64) chunks x HV heads of item blocks
+    assert L.kda_prefill_workspace_size(2, 4096, 96, 96, 128, 128, 0) == 2 * 64 * 96 * item
+    assert L.kda_prefill_workspace_size(1, 1000, 4, 4, 128, 128, 0) == 16 * 4 * item
+    # packed batch: offsets and order, then (ceil(T/64) + N) chunks as an upper bound
+    n = L.kda_prefill_workspace_size(1, 11210, 8, 32, 128, 128, 7)
+    assert n == 256 + 256 + (176 + 7) * 32 * item
+    # rejected sizes
+    assert L.kda_prefill_workspace_size(1, 64, 1, 1, 64, 128, 0) == 0
+    assert L.kda_prefill_workspace_size(1, 64, 2, 3, 128, 128, 0) == 0
 
 
 def test_host_staging_size(L):
     B, T, H, HV = 1, 1000, 4, 4
     n = L.kda_prefill_host_staging_size(B, T, H, HV, 128, 128, 0, 1, 0)
     expect = 2 * T * H * 128 * 2 + T * HV * 128 * 2 + T * HV * 128 * 4 + T * HV * 4 + 2 * HV * 128 * 128 * 4 \
-        + T * HV * 128 * 2
+        + T * HV * 128 * 2 + L.kda_prefill_workspace_size(B, T, H, HV, 128, 128, 0)
     assert expect <= n <= expect + 16 * 256
 
 
@@ -74,7 +81,9 @@ def call_forward(L, **over):
     (dict(cu=FAKE * 8, num_seqs=0), 1), (dict(cu=FAKE * 8, num_seqs=2, B=2), 1),
     (dict(cu=FAKE * 8, num_seqs=2), 4),                      # varlen needs a workspace
     (dict(cu=FAKE * 8, num_seqs=2, ws=FAKE * 9, ws_bytes=16), 4),
-    (dict(cu=FAKE * 8, num_seqs=2, ws=FAKE * 9 + 16, ws_bytes=256), 3),
+    (dict(cu=FAKE * 8, num_seqs=2, ws=FAKE * 64 + 16, ws_bytes=1 << 30), 3),
+    (dict(ws=None), 4), (dict(ws=FAKE * 64, ws_bytes=1000), 4),
+    (dict(ws=FAKE * 2, ws_bytes=1 << 30), 1),                # workspace overlaps k
     (dict(o=FAKE), 1),                                       # o overlaps q
     (dict(sN=FAKE * 4), 1),                                  # final_state overlaps g
 ])
@@ -84,7 +93,7 @@ def test_forward_rejects_bad_arguments(L, over, code):
 
 def test_partial_state_overlap_rejected(L):
     s0 = FAKE * 16
-    assert call_forward(L, s0=s0, sN=s0 + 4096) == 1
+    assert call_forward(L, s0=s0, sN=s0 + 4096, ws=FAKE * 64, ws_bytes=1 << 26) == 1
 
 
 def test_l2norm_rejects_bad_arguments(L):

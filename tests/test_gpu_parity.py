@@ -155,7 +155,9 @@ def test_split_resume_matches_full():
     ob, sb = gpu_forward(b)
     ref = oracle_forward(x)
     compare(torch.cat([oa, ob], dim=1), sb, ref)
-    assert torch.equal(oa, full_o[:, :t1])
+    # The first part's rows come from a shorter last chunk, whose block-local gate products round
+    # differently, so the split and the full run agree to rounding, not bit for bit.
+    assert (oa.float() - full_o[:, :t1].float()).abs().max() < 1e-2
 
 
 def test_outputs_fully_written():
