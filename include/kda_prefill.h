@@ -129,6 +129,31 @@ kda_status_t kda_prefill_forward_host(const void *q_host, const void *k_host, co
                                       void *stream);
 
 /*
+ * kda_prefill_forward without a workspace argument, for callers that cannot
+ * allocate device memory: runtimes that freeze their device memory after
+ * warm-up (cudaMalloc synchronises the whole device and would stall every
+ * other stream) and plugin hosts that give plugins no allocator.  The page
+ * has no counterpart of this entry point; it is a packaging choice.
+ *
+ * Same arguments and behaviour as kda_prefill_forward minus workspace /
+ * workspace_bytes.  The workspace is a fixed 64 MiB device array that every
+ * GPU loading the library reserves until the process exits; sizes whose
+ * kda_prefill_workspace_size() exceeds 64 MiB (about 900 pairs of a 64-token
+ * chunk and a value head, e.g. T = 14,400 at HV = 4) are rejected with
+ * KDA_ERR_WORKSPACE before any launch.  The first call on a device looks up
+ * the array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  Every call shares the one array, so calls
+ * whose work overlaps on the GPU (other streams, other threads) race; issue
+ * them one after another.  Calls no cudaMalloc / cudaFree.
+ */
+kda_status_t kda_prefill_forward_noalloc(const void *q, const void *k, const void *v,
+                                         const float *g, const float *beta,
+                                         const float *initial_state,
+                                         const int32_t *cu_seqlens, int num_seqs,
+                                         int B, int T, int H, int HV, int K, int V,
+                                         void *o, float *final_state, void *stream);
+
+/*
  * Debug aid: the device error word of the current device.  Kernel waits on
  * copies and pipeline stages are bounded (about one second); a wait that
  * gives up sets a bit here (1: input tile copy, 2: stage fill, 4: stage

@@ -155,3 +155,29 @@ def l2norm_bf16(x, out=None, stream=None):
     rows = x.numel() // x.shape[-1]
     _check(lib().kda_l2norm_bf16(_ptr(x), rows, x.shape[-1], _ptr(out), _stream_ptr(stream)), "kda_l2norm_bf16")
     return out
+
+
+def forward_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o=None, final_state=None,
+                    stream=None):
+    """The forward through kda_prefill_forward_noalloc: no workspace argument.
+
+    For callers that may not allocate device memory during the call; the
+    library's fixed 64 MiB scratch array limits the problem size (larger
+    inputs raise KdaError with KDA_ERR_WORKSPACE).  Calls must not overlap.
+    """
+    import torch
+    L = lib()
+    f = L.kda_prefill_forward_noalloc
+    P, I = ctypes.c_void_p, ctypes.c_int
+    f.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P]
+    f.restype = I
+    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
+    if o is None:
+        o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=q.device)
+    if final_state is None:
+        final_state = torch.empty(N, HV, K, V, dtype=torch.float32, device=q.device)
+    num_seqs = N if cu_seqlens is not None else 0
+    rc = f(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), num_seqs,
+           B, T, H, HV, K, V, _ptr(o), _ptr(final_state), _stream_ptr(stream))
+    _check(rc, "kda_prefill_forward_noalloc")
+    return o, final_state

@@ -378,3 +378,55 @@ extern "C" kda_status_t kda_l2norm_bf16(const void *x, int64_t rows, int K, void
         static_cast<const __nv_bfloat16 *>(x), rows, static_cast<__nv_bfloat16 *>(out));
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of kda_prefill_forward.
+//
+// Some callers cannot hand the library a workspace: an inference runtime that
+// freezes its device memory after warm-up (a cudaMalloc would synchronise the
+// whole device and stall every other stream), or a plugin host that gives its
+// plugins no allocator at all.  For them the workspace lives in a fixed
+// file-scope device array that every GPU loading this library reserves until
+// the process exits.  Host code must not use the array's name as an address:
+// on the host it is only a stand-in symbol, so its device address is looked
+// up once per device with cudaGetSymbolAddress and cached.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
+static __device__ __align__(256) uint8_t g_kda_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+}  // namespace
+
+extern "C" kda_status_t kda_prefill_forward_noalloc(const void *q, const void *k, const void *v, const float *g,
+                                                    const float *beta, const float *initial_state,
+                                                    const int32_t *cu_seqlens, int num_seqs, int B, int T, int H,
+                                                    int HV, int K, int V, void *o, float *final_state, void *stream)
+{
+    Dims d;
+    const bool varlen = cu_seqlens != nullptr;
+    const kda_status_t st = check_dims(B, T, H, HV, K, V, varlen, num_seqs, d);
+    if (st != KDA_OK) return st;
+    const size_t need = workspace_layout(B, T, HV, varlen ? num_seqs : 0).total;
+    if (need > kNoAllocScratchBytes) return KDA_ERR_WORKSPACE;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_kda_noalloc_scratch) != cudaSuccess || !p) return KDA_ERR_CUDA;
+            g_noalloc_ptr[dev] = p;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    // Everything the kernels read from the scratch is written earlier in the
+    // same call (chunk offsets, sequence order, chunk blocks), so nothing
+    // needs clearing between calls.
+    return kda_prefill_forward(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, B, T, H, HV, K, V, o,
+                               final_state, scratch, kNoAllocScratchBytes, stream);
+}
