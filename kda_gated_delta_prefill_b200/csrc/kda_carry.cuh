@@ -1,34 +1,39 @@
-// kda_carry.cuh -- inter-chunk state carry ("KDA Chunk Prefill on Ascend A3",
-// section "Mathematical definition", last three formulas):
-//   Vnew  = U - W S_in
-//   O     = Qg S_in + Aqk Vnew
-//   S_out = exp(G_last)[:,None] * S_in + Kg^T Vnew
-// One CTA per (sequence, value head, slice of 16*NW value columns); the
-// columns of S evolve independently, so slicing is exact.  Every consumer
-// warp owns 16 value columns and keeps S^T for them in MMA accumulator
-// registers (float32) for the whole sequence.  A producer warp streams the
-// per-chunk blocks written by the intra-chunk kernel through a three-stage
-// shared-memory ring with bulk copies and mbarriers.
+// kda_carry.cuh -- inter-chunk state carry on the 5th-generation tensor cores
+// ("KDA Chunk Prefill on Ascend A3", section "Mathematical definition", last
+// three formulas), written transposed so that the value dimension (128) is
+// the MMA's M dimension:
+//   Vnew^T = U^T - S_in^T W^T
+//   O^T    = S_in^T Qg^T + Vnew^T Aqk^T
+//   S_out^T = S_in^T diag(exp(G_last)) + Vnew^T Kg
+// One CTA per (sequence, value head).  Warps 0-15 (epilogue) own TMEM lane
+// v = 32*(warp%4) + lane, i.e. value column v, and a quarter of the key and
+// token columns (warp/4); they keep the float32 master state S^T[v][:] in registers and
+// write its fp16 copy into TMEM, where it is the A operand of the next
+// chunk's MMAs.  Warp 16 streams the per-chunk blocks written by the
+// intra-chunk kernel into a two-stage shared-memory ring (one bulk copy per
+// chunk); the last warp allocates TMEM and issues the MMAs.  Every wait is
+// bounded.
 #pragma once
 #include "kda_common.cuh"
 #include "ptx.cuh"
+#include "tc.cuh"
 
 namespace kda {
 
-template <int NW>
 struct CarrySmem {
-    static constexpr int VS = 16 * NW;
-    static constexpr int U_BYTES = VS * CH * 2;                         // fp16 U columns of this slice
-    static constexpr int U_OFF = ITEM_U;                                // stage image follows the item layout
-    static constexpr int GL_OFF = ITEM_U + U_BYTES;
-    static constexpr int STAGE = ((GL_OFF + 512) + 1023) / 1024 * 1024;
-    static constexpr int NST = 3;
-    static constexpr int VN_STRIDE = 48;                                // bytes per Vnew row (16 fp16 + pad)
-    static constexpr int VN = NST * STAGE;
-    static constexpr int BAR = VN + NW * CH * VN_STRIDE;
-    static constexpr int TOTAL = BAR + 2 * NST * 8;
-    static constexpr uint32_t TX = ITEM_U + U_BYTES + 512;
+    static constexpr int STAGE = ((ITEM_BYTES + 1023) / 1024) * 1024;  // 75776
+    static constexpr int NST = 2;
+    static constexpr int BAR = NST * STAGE;   // mbarriers: full[2] empty[2] barP barS sready vready barO
+    static constexpr int TMEM_SLOT = BAR + 9 * 8;
+    static constexpr int ABORT = TMEM_SLOT + 4;
+    static constexpr int TOTAL = ABORT + 12;
 };
+
+constexpr int kCarryEpiWarps = 16;
+constexpr int kCarryThreads = (kCarryEpiWarps + 2) * 32;
+
+// TMEM column map (512 allocated): P^T (64), O^T x2 (64 each), S^T fp32 master (128), S^T fp16 (64), Vnew^T fp16 (32).
+constexpr uint32_t TM_P = 0, TM_O0 = 64, TM_S = 192, TA_S = 320, TA_V = 384, TM_COLS = 512;
 
 struct CarryParams {
     const uint8_t *items;
@@ -41,23 +46,17 @@ struct CarryParams {
     unsigned *err;
     int T, HV, N;
     int chunks_per_seq;
-    int nslices;
 };
 
-template <int NW>
-__global__ void __launch_bounds__((NW + 1) * 32, 1) kda_carry_kernel(const CarryParams p)
+__global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const CarryParams p)
 {
-    using S = CarrySmem<NW>;
+    using S = CarrySmem;
     extern __shared__ __align__(1024) uint8_t sm[];
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g8 = lane >> 2, t4 = lane & 3;
 
-    const int slice = blockIdx.x % p.nslices;
-    const int rest = blockIdx.x / p.nslices;
-    const int h = rest % p.HV;
-    const int r_idx = rest / p.HV;
-    const int n = p.order ? p.order[r_idx] : r_idx;
+    const int h = blockIdx.x % p.HV;
+    const int n = p.order ? p.order[blockIdx.x / p.HV] : blockIdx.x / p.HV;
     int64_t c_begin, tok0;
     int nck, len;
     if (p.cu) {
@@ -71,187 +70,236 @@ __global__ void __launch_bounds__((NW + 1) * 32, 1) kda_carry_kernel(const Carry
         tok0 = static_cast<int64_t>(n) * p.T;
         len = p.T;
     }
-    const int v0 = slice * S::VS;
 
-    const uint32_t full0 = sb + S::BAR, empty0 = sb + S::BAR + S::NST * 8;
+    const uint32_t full0 = sb + S::BAR, empty0 = full0 + 16, barP = full0 + 32, barS = full0 + 40,
+                   sready = full0 + 48, vready = full0 + 56, barO = full0 + 64;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + S::ABORT);
     if (tid == 0) {
         for (int s = 0; s < S::NST; ++s) {
             mbar_init(full0 + 8 * s, 1);
-            mbar_init(empty0 + 8 * s, NW);
+            mbar_init(empty0 + 8 * s, 1 + kCarryEpiWarps);
         }
+        mbar_init(barP, 1);
+        mbar_init(barS, 1);
+        mbar_init(barO, 1);
+        mbar_init(sready, kCarryEpiWarps);
+        mbar_init(vready, kCarryEpiWarps);
+        *abort_flag = 0;
         fence_mbar_init();
     }
+    if (warp == kCarryEpiWarps + 1) tc_alloc(sb + S::TMEM_SLOT, TM_COLS);
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + S::TMEM_SLOT);
 
-    if (warp == NW) {  // ---- producer ----
+    auto fail = [&](unsigned code) {
+        atomicOr(p.err, code);
+        *abort_flag = 1;
+    };
+
+    if (warp == kCarryEpiWarps) {
+        // ---------------- producer: one bulk copy per chunk block ----------------
         if (lane == 0) {
-            for (int c = 0; c < nck; ++c) {
+            for (int c = 0; c < nck && !*abort_flag; ++c) {
                 const int s = c % S::NST;
                 if (c >= S::NST && !mbar_wait(empty0 + 8 * s, ((c / S::NST) - 1) & 1)) {
-                    atomicOr(p.err, ERR_PIPE_EMPTY_WAIT);
-                    return;
+                    fail(ERR_PIPE_EMPTY_WAIT);
+                    break;
                 }
-                const uint8_t *item = p.items + ((c_begin + c) * p.HV + h) * ITEM_BYTES;
-                const uint32_t dst = sb + s * S::STAGE;
-                mbar_expect_tx(full0 + 8 * s, S::TX);
-                bulk_load(dst, item, ITEM_U, full0 + 8 * s);
-                bulk_load(dst + S::U_OFF, item + ITEM_U + slice * S::U_BYTES, S::U_BYTES, full0 + 8 * s);
-                bulk_load(dst + S::GL_OFF, item + ITEM_GL, 512, full0 + 8 * s);
+                mbar_expect_tx(full0 + 8 * s, ITEM_BYTES);
+                bulk_load(sb + s * S::STAGE, p.items + ((c_begin + c) * p.HV + h) * ITEM_BYTES, ITEM_BYTES,
+                          full0 + 8 * s);
             }
         }
-        return;
-    }
-
-    // ---- consumers: S^T for value columns vl = g8 + 8*(e>>1) of this warp, key kd = 8*nt + 2*t4 + (e&1) ----
-    float sT[16][4];
-    {
-        const int vcol = v0 + 16 * warp + g8;
-        const float *s0 = p.s0 ? p.s0 + (static_cast<int64_t>(n) * p.HV + h) * DK * DV : nullptr;
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int kd = 8 * nt + 2 * t4 + (e & 1);
-                sT[nt][e] = s0 ? s0[kd * DV + vcol + 8 * (e >> 1)] : 0.f;
-            }
-    }
-    uint8_t *vn = sm + S::VN + warp * CH * S::VN_STRIDE;
-    const uint32_t vn_s = smem_u32(vn);
-    const int mi = lane >> 3;
-
-    for (int c = 0; c < nck; ++c) {
-        const int s = c % S::NST;
-        if (!mbar_wait(full0 + 8 * s, (c / S::NST) & 1)) {
-            atomicOr(p.err, ERR_PIPE_FULL_WAIT);
-            return;
-        }
-        const uint8_t *st = sm + s * S::STAGE;
-        const uint32_t st_s = sb + s * S::STAGE;
-        const int nvalid = min(CH, len - c * CH);
-
-        // U -> accumulators (becomes Vnew)
-        float acc[4][2][4];
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-            for (int nv = 0; nv < 2; ++nv)
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                    const int tok = 16 * mt + g8 + 8 * hr;
-                    const int col = (warp & 1) * 16 + 8 * nv + 2 * t4;
-                    const float2 u = unpack_f16(
-                        *reinterpret_cast<const uint32_t *>(st + S::U_OFF + (warp >> 1) * 4096 + tok * 64 + col * 2));
-                    acc[mt][nv][2 * hr] = u.x;
-                    acc[mt][nv][2 * hr + 1] = u.y;
+    } else if (warp == kCarryEpiWarps + 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t i64 = idesc_f16(128, 64, false), i128mn = idesc_f16(128, 128, true);
+            // stage-0 descriptors; stage s adds s*STAGE/16 to the start-address field
+            const uint64_t dW = sw128_desc(sb + ITEM_WN, 16, 1024), dQ = sw128_desc(sb + ITEM_QG, 16, 1024);
+            const uint64_t dA = sw128_desc(sb + ITEM_AQK, 16, 1024), dK = sw128_desc(sb + ITEM_KG, 8192, 1024);
+            for (int c = 0; c < nck && !*abort_flag; ++c) {
+                const int s = c % S::NST;
+                const uint64_t so = static_cast<uint64_t>(s * (S::STAGE >> 4));
+                if (!mbar_wait(full0 + 8 * s, (c / S::NST) & 1) || !mbar_wait_spin(sready, c & 1)) {
+                    fail(ERR_PIPE_FULL_WAIT);
+                    break;
                 }
-        float oacc[4][2][4] = {};
-        // Vnew = U + (-W) S ;  O = Qg S
+                tc_fence_after();
+                const uint32_t tmo = tmem + TM_O0 + 64 * (c & 1);
+                // P^T = S^T W^T (K = 128 keys, 8 steps); W is stored negated, so P^T = -(S^T W^T)
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            uint32_t bs[2][2];
+                for (int ks = 0; ks < 8; ++ks)
+                    tc_mma_ts(tmem + TM_P, tmem + TA_S + 8 * ks, dW + so + (ks >> 2) * 512 + (ks & 3) * 2, i64, ks > 0);
+                tc_commit(barP);
+                // O^T = S^T Qg^T
 #pragma unroll
-            for (int nv = 0; nv < 2; ++nv) {
-                bs[nv][0] = pack_f16(sT[2 * ks][2 * nv], sT[2 * ks][2 * nv + 1]);
-                bs[nv][1] = pack_f16(sT[2 * ks + 1][2 * nv], sT[2 * ks + 1][2 * nv + 1]);
-            }
-#pragma unroll
-            for (int mt = 0; mt < 4; ++mt) {
-                const int r = 16 * mt + (mi & 1) * 8 + (lane & 7);
-                const int cc = 16 * ks + (mi >> 1) * 8;
-                uint32_t aw[4], aq[4];
-                ldsm_x4(st_s + ITEM_WN + swz(r, cc * 2, 256), aw[0], aw[1], aw[2], aw[3]);
-                ldsm_x4(st_s + ITEM_QG + swz(r, cc * 2, 256), aq[0], aq[1], aq[2], aq[3]);
-#pragma unroll
-                for (int nv = 0; nv < 2; ++nv) {
-                    mma_f16(acc[mt][nv], aw, bs[nv][0], bs[nv][1]);
-                    mma_f16(oacc[mt][nv], aq, bs[nv][0], bs[nv][1]);
+                for (int ks = 0; ks < 8; ++ks)
+                    tc_mma_ts(tmo, tmem + TA_S + 8 * ks, dQ + so + (ks >> 2) * 512 + (ks & 3) * 2, i64, ks > 0);
+                if (!mbar_wait_spin(vready, c & 1)) {
+                    fail(ERR_PIPE_FULL_WAIT);
+                    break;
                 }
+                tc_fence_after();
+                // S^T += Vnew^T Kg onto the decayed master state (on the chain to the next chunk, so first).
+                // Kg is MN-major: 64-key blocks 8192 bytes apart, token groups of 8 rows 1024 bytes apart.
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) tc_mma_ts(tmem + TM_S, tmem + TA_V + 8 * ks, dK + so + ks * 128, i128mn, 1);
+                tc_commit(barS);
+                // O^T += Vnew^T Aqk^T (K = 64 tokens)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    tc_mma_ts(tmo, tmem + TA_V + 8 * ks, dA + so + ks * 2, i64, 1);
+                tc_commit(barO);
+                tc_commit(empty0 + 8 * s);
             }
         }
-        // Vnew -> fp16 -> per-warp buffer [64 tok][16 v]
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-            for (int nv = 0; nv < 2; ++nv) {
-                const int r = 16 * mt + g8;
-                const int vc = 8 * nv + 2 * t4;
-                *reinterpret_cast<uint32_t *>(vn + r * S::VN_STRIDE + vc * 2) = pack_f16(acc[mt][nv][0], acc[mt][nv][1]);
-                *reinterpret_cast<uint32_t *>(vn + (r + 8) * S::VN_STRIDE + vc * 2) =
-                    pack_f16(acc[mt][nv][2], acc[mt][nv][3]);
-            }
-        __syncwarp();
-        // O += Aqk Vnew (causal: key blocks ks <= mt)
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
-            for (int ks = 0; ks <= mt; ++ks) {
-                uint32_t a[4];
-                ldsm_x4(st_s + ITEM_AQK + swz(16 * mt + (mi & 1) * 8 + (lane & 7), (16 * ks + (mi >> 1) * 8) * 2, 128),
-                        a[0], a[1], a[2], a[3]);
-                const int tok = 16 * ks + (mi & 1) * 8 + (lane & 7);
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(vn_s + tok * S::VN_STRIDE + (mi >> 1) * 16, b0, b1, b2, b3);
-                mma_f16(oacc[mt][0], a, b0, b1);
-                mma_f16(oacc[mt][1], a, b2, b3);
-            }
-        }
-        // o rows of valid tokens (bf16)
+    } else {
+        // ---------------- epilogue: value column v, key/token quarter kq ----------------
+        const int qd = warp & 3, kq = warp >> 2;
+        const int v = 32 * qd + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+        const uint32_t tS = tmem + lane_base + TM_S + 32 * kq;     // fp32 master S^T[v][32kq .. 32kq+31]
+        const uint32_t tA = tmem + lane_base + TA_S + 16 * kq;     // its fp16 copy (A operand)
+        const int64_t ostride = static_cast<int64_t>(p.HV) * DV;
         {
-            __nv_bfloat16 *ob = p.o + ((tok0 + static_cast<int64_t>(c) * CH) * p.HV + h) * DV + v0 + 16 * warp;
+            const float *s0 = p.s0 ? p.s0 + (static_cast<int64_t>(n) * p.HV + h) * DK * DV : nullptr;
+            uint32_t r[32], w[16];
 #pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
+            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s0 ? s0[(32 * kq + j) * DV + v] : 0.f);
 #pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                    const int tok = 16 * mt + g8 + 8 * hr;
-                    if (tok < nvalid) {
+            for (int j = 0; j < 16; ++j) w[j] = pack_f16(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+            tc_st32(tS, r);
+            tc_st16(tA, w);
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sready);
+        }
+        // o rows of chunk c: O^T[v][tok], tok in [16*kq, 16*kq+16); a warp writes 64 contiguous bytes per token
+        auto store_o = [&](int c) {
+            uint32_t orr[16];
+            tc_ld16(tmem + lane_base + TM_O0 + 64 * (c & 1) + 16 * kq, orr);
+            tc_wait_ld();
+            __nv_bfloat16 *ob = p.o + ((tok0 + static_cast<int64_t>(c) * CH + 16 * kq) * p.HV + h) * DV + v;
+            const int nrows = min(CH, len - c * CH) - 16 * kq;
+            if (nrows >= 16) {
 #pragma unroll
-                        for (int nv = 0; nv < 2; ++nv)
-                            *reinterpret_cast<uint32_t *>(ob + static_cast<int64_t>(tok) * p.HV * DV + 8 * nv + 2 * t4) =
-                                pack_bf16(oacc[mt][nv][2 * hr], oacc[mt][nv][2 * hr + 1]);
+                for (int t = 0; t < 16; ++t) ob[t * ostride] = __float2bfloat16_rn(__uint_as_float(orr[t]));
+            } else {
+#pragma unroll
+                for (int t = 0; t < 16; ++t)
+                    if (t < nrows) ob[t * ostride] = __float2bfloat16_rn(__uint_as_float(orr[t]));
+            }
+        };
+
+        for (int c = 0; c < nck && !*abort_flag; ++c) {
+            const int s = c % S::NST;
+            const uint8_t *st = sm + s * S::STAGE;
+            // --- while MMA1/O1 of chunk c run: S^T <- S^T diag(exp(G_last)) ---
+            if (!mbar_wait(full0 + 8 * s, (c / S::NST) & 1)) {
+                fail(ERR_PIPE_FULL_WAIT);
+                break;
+            }
+            {
+                const float2 *gl = reinterpret_cast<const float2 *>(st + ITEM_GL) + 16 * kq;
+                uint32_t r[32];
+                tc_ld32(tS, r);
+                tc_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float2 x = mul2(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])), gl[j]);
+                    r[2 * j] = __float_as_uint(x.x);
+                    r[2 * j + 1] = __float_as_uint(x.y);
+                }
+                tc_st32(tS, r);
+            }
+            // --- Vnew^T[v][tok] = U^T[v][tok] + P^T[v][tok], tok in [16*kq, 16*kq+16) ---
+            if (!mbar_wait_spin(barP, c & 1)) {
+                fail(ERR_PIPE_FULL_WAIT);
+                break;
+            }
+            tc_fence_after();
+            {
+                uint32_t pr[16];
+                tc_ld16(tmem + lane_base + TM_P + 16 * kq, pr);
+                uint4 ur[2];
+#pragma unroll
+                for (int q = 0; q < 2; ++q)
+                    ur[q] = *reinterpret_cast<const uint4 *>(st + ITEM_U + v * 128 + (((2 * kq + q) ^ (v & 7)) << 4));
+                tc_wait_ld();
+                uint32_t w[8];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const uint32_t uw[4] = {ur[q].x, ur[q].y, ur[q].z, ur[q].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int t = 8 * q + 2 * e;
+                        const float2 x = add2(unpack_f16(uw[e]), make_float2(__uint_as_float(pr[t]), __uint_as_float(pr[t + 1])));
+                        w[4 * q + e] = pack_f16(x.x, x.y);
                     }
                 }
-        }
-        // S^T <- S^T diag(exp(G_last)) + Vnew^T Kg
-        {
-            const float *gl = reinterpret_cast<const float *>(st + S::GL_OFF);
-#pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-                const float2 f = *reinterpret_cast<const float2 *>(gl + 8 * nt + 2 * t4);
-                sT[nt][0] *= f.x;
-                sT[nt][1] *= f.y;
-                sT[nt][2] *= f.x;
-                sT[nt][3] *= f.y;
-            }
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                uint32_t a[4];
-                ldsm_x4_t(vn_s + (16 * ks + (mi >> 1) * 8 + (lane & 7)) * S::VN_STRIDE + (mi & 1) * 16, a[0], a[1], a[2],
-                          a[3]);
-#pragma unroll
-                for (int np = 0; np < 16; np += 2) {
-                    const int tok = 16 * ks + (mi & 1) * 8 + (lane & 7);
-                    const int kd = 8 * np + (mi >> 1) * 8;
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4_t(st_s + ITEM_KG + swz(tok, kd * 2, 256), b0, b1, b2, b3);
-                    mma_f16(sT[np], a, b0, b1);
-                    mma_f16(sT[np + 1], a, b2, b3);
+                tc_st8(tmem + lane_base + TA_V + 8 * kq, w);
+                tc_wait_st();  // also covers the decayed master state
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(vready);
+                    mbar_arrive(empty0 + 8 * s);  // U and exp(G_last) of this stage are consumed
                 }
             }
+            if (c > 0) {  // the previous chunk's o rows, while MMA2 runs
+                if (!mbar_wait(barO, (c - 1) & 1)) {
+                    fail(ERR_PIPE_FULL_WAIT);
+                    break;
+                }
+                tc_fence_after();
+                store_o(c - 1);
+            }
+            // --- S^T (master, now S_out^T) -> fp16 A operand for the next chunk ---
+            if (!mbar_wait_spin(barS, c & 1)) {
+                fail(ERR_PIPE_FULL_WAIT);
+                break;
+            }
+            tc_fence_after();
+            {
+                uint32_t r[32], w[16];
+                tc_ld32(tS, r);
+                tc_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) w[j] = pack_f16(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                tc_st16(tA, w);
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sready);
+            }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + 8 * s);
+        if (nck > 0 && !*abort_flag) {
+            if (mbar_wait(barO, (nck - 1) & 1)) {
+                tc_fence_after();
+                store_o(nck - 1);
+            } else {
+                fail(ERR_PIPE_FULL_WAIT);
+            }
+        }
+        // final state (S^T[v][kd] -> final_state[kd][v])
+        {
+            uint32_t r[32];
+            tc_ld32(tS, r);
+            tc_wait_ld();
+            float *sN = p.sN + (static_cast<int64_t>(n) * p.HV + h) * DK * DV;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sN[(32 * kq + j) * DV + v] = __uint_as_float(r[j]);
+        }
     }
 
-    // ---- final state ----
-    {
-        float *sN = p.sN + (static_cast<int64_t>(n) * p.HV + h) * DK * DV;
-        const int vcol = v0 + 16 * warp + g8;
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int kd = 8 * nt + 2 * t4 + (e & 1);
-                sN[kd * DV + vcol + 8 * (e >> 1)] = sT[nt][e];
-            }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kCarryEpiWarps + 1) {
+        tc_fence_after();
+        tc_dealloc(tmem, TM_COLS);
     }
 }
 

@@ -8,9 +8,10 @@
 //   Aqk_ij = K^-0.5 sum_d q_id k_jd exp(G_id - G_jd)   (j <= i)
 //   A = (I + L)^-1 diag(beta),  W = A (exp(G) k),  U = A v,
 //   Qg = K^-0.5 q exp(G),  Kg = k exp(G_last - G),  and exp(G_last).
-// The item's results -- -W, Qg, Kg, Aqk, U (fp16) and exp(G_last) (fp32) --
-// are written as one contiguous block that the carry kernel copies straight
-// into its shared memory.
+// The item's results -- -W, Qg, Kg, Aqk, U^T (fp16) and exp(G_last) (fp32) --
+// are written as one contiguous block in the 128-byte-swizzled operand
+// layouts the carry kernel's tensor-core descriptors read, so the carry
+// kernel copies it into shared memory with one bulk copy.
 //
 // Steps inside the CTA (256 threads):
 //   1. TMA tile loads of q, k (Q/K head h / (HV/H)), v, g; beta by plain
@@ -21,14 +22,16 @@
 //      within each 16-token block the inclusive running product base_i and
 //      the exclusive suffix product b_j, block products P_J, and
 //      per-channel factors built from them, so that for i >= j
-//      exp(G_i - G_j) = base_i * c_IJ * b_j with every factor <= 1 except the
-//      diagonal-block c_II = 1/P_I.
+//      exp(G_i - G_j) = base_i * (c_IJ * b_j) with every factor <= 1 except the
+//      diagonal-block c_II = 1/P_I (then c_II * b_j = 1/base_j <= e^75).
 //   4. L and Aqk: bf16 tensor-core MMAs over the ten lower 16x16 block pairs
 //      (bf16 keeps the range of the gate-rescaled operands).
 //   5. A: exact float32 forward substitution in the 16x16 diagonal blocks,
 //      tf32 MMAs for the off-diagonal blocks.
-//   6. W and U: fp16 tensor-core MMAs.
-//   7. One bulk store of the item block.
+//   6. W and U^T: fp16 tensor-core MMAs.
+// Results go straight from registers to the item block in global memory
+// (coalesced rows), so the CTA needs about 105 KB of shared memory and two
+// CTAs share an SM.
 #pragma once
 #include "kda_common.cuh"
 #include "kda_norm.cuh"
@@ -37,21 +40,21 @@
 namespace kda {
 
 struct IntraSmem {
-    static constexpr int Q = 0;          // bf16 [64][128] (two SW128 halves): q -> normalised -> K^-0.5 q*base
-    static constexpr int K = 16384;      // bf16: k -> normalised -> k*base
+    static constexpr int Q = 0;          // bf16 [64][128] (two SW128 halves): q -> normalised -> K^-0.5 q*base; X (step 5)
+    static constexpr int K = 16384;      // bf16: k -> normalised -> k*base; A fp16 [64][64] (step 5)
     static constexpr int V = 32768;      // bf16 v -> fp16 v
     static constexpr int G = 49152;      // fp32 [64][128] g; then KEXP fp16 (first half) and KBB bf16 (second half)
     static constexpr int KEXP = G;
     static constexpr int KBB = G + 16384;
-    static constexpr int OUT = 81920;    // the item block (ItemLayout), 74240 bytes
-    static constexpr int L = 156672;     // fp32 [64][64]
-    static constexpr int X = 173056;     // fp32 [64][64]
-    static constexpr int A = 189440;     // fp16 [64][64]
-    static constexpr int BETA = 197632;  // fp32 [64]
-    static constexpr int CF = 197888;    // bf16x2 [10][64] block-pair factors
-    static constexpr int TS = 200448;    // fp32 3 x [16][24] solve scratch
-    static constexpr int BAR = 205056;   // mbarrier
-    static constexpr int TOTAL = 205120;
+    static constexpr int L = 81920;      // fp32 [64][64]
+    static constexpr int X = Q;          // fp32 [64][64], once q*base is no longer needed
+    static constexpr int A = K;          // fp16 [64][64], once k*base is no longer needed
+    static constexpr int BETA = 98304;   // fp32 [64]
+    static constexpr int CF = 98560;     // bf16x2 [10][64] block-pair factors
+    static constexpr int PS = 101120;    // float2 [4][64] block products
+    static constexpr int TS = 103168;    // fp32 3 x [16][24] solve scratch
+    static constexpr int BAR = 107776;   // mbarrier
+    static constexpr int TOTAL = 107840;
 };
 
 struct IntraParams {
@@ -121,7 +124,7 @@ __device__ __forceinline__ void solve_block(const uint8_t *sL, uint8_t *sX, floa
     __syncwarp();
 }
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(256, 2)
     kda_intra_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg,
                      const IntraParams p)
@@ -155,8 +158,7 @@ __global__ void __launch_bounds__(256, 1)
         nvalid = min(CH, p.T - c * CH);
     }
     const int hq = h / (p.HV / p.H);
-    uint8_t *out_g = p.items + (static_cast<int64_t>(ci) * p.HV + h) * ITEM_BYTES;
-    uint8_t *out = sm + S::OUT;
+    uint8_t *out = p.items + (static_cast<int64_t>(ci) * p.HV + h) * ITEM_BYTES;  // item block (global)
 
     // ---- 1. loads ----
     const uint32_t bar = sb + S::BAR;
@@ -250,9 +252,9 @@ __global__ void __launch_bounds__(256, 1)
     }
     __syncthreads();
 
-    // ---- 3. gate factors and operands: thread = (block J, channel pair dp) ----
+    // ---- 3. gate factors and operands: warp = (block J, channel half), lane = channel pair ----
     {
-        const int J = tid & 3, dp = tid >> 2, d0 = 2 * dp;
+        const int J = warp & 3, dp = 32 * (warp >> 2) + lane, d0 = 2 * dp;
         float2 e[16], bb[16];
         const float2 l2e = make_float2(1.4426950408889634f, 1.4426950408889634f);
 #pragma unroll
@@ -266,35 +268,31 @@ __global__ void __launch_bounds__(256, 1)
         for (int u = 14; u >= 0; --u) bb[u] = mul2(bb[u + 1], e[u + 1]);
 #pragma unroll
         for (int u = 1; u < 16; ++u) e[u] = mul2(e[u - 1], e[u]);  // e -> inclusive running product (base)
-        // block products of this channel pair from the four lanes that hold blocks 0..3
+        float2 *ps = reinterpret_cast<float2 *>(sm + S::PS);
+        ps[J * 64 + dp] = e[15];  // block product P_J of this channel pair
+        __syncthreads();          // every g read is done (the G region becomes KEXP / KBB); P visible
         float2 P[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            P[j].x = __shfl_sync(0xffffffffu, e[15].x, (lane & ~3) | j);
-            P[j].y = __shfl_sync(0xffffffffu, e[15].y, (lane & ~3) | j);
-        }
+        for (int j = 0; j < 4; ++j) P[j] = ps[j * 64 + dp];
         // E_J = prod_{J'<J} P_J' (gate from the chunk start to the block start), F_J = prod_{J'>J} P_J'
         const float2 one2 = make_float2(1.f, 1.f);
         const float2 P01 = mul2(P[0], P[1]), P23 = mul2(P[2], P[3]);
         const float2 myE = (J == 0) ? one2 : (J == 1) ? P[0] : (J == 2) ? P01 : mul2(P01, P[2]);
         const float2 myF = (J == 3) ? one2 : (J == 2) ? P[3] : (J == 1) ? P23 : mul2(P[1], P23);
         const float scale = 0.08838834764831845f;  // 128^-0.5 in float32
-        const float2 sE = mul2(myE, make_float2(scale, scale));
+        const float2 s2 = make_float2(scale, scale);
         if (J == 0) {
             // per-channel factors of the ten block pairs, as bf16 pairs; c_II = 1/P_I
             uint32_t *cf = reinterpret_cast<uint32_t *>(sm + S::CF);
             auto rcp2 = [](float2 a) {
                 return make_float2(__frcp_rn(fmaxf(a.x, 1e-37f)), __frcp_rn(fmaxf(a.y, 1e-37f)));
             };
-            const float2 one = make_float2(1.f, 1.f);
-            const float2 cv[10] = {rcp2(P[0]), one, rcp2(P[1]), P[1], one, rcp2(P[2]), mul2(P[1], P[2]), P[2], one,
+            const float2 cv[10] = {rcp2(P[0]), one2, rcp2(P[1]), P[1], one2, rcp2(P[2]), mul2(P[1], P[2]), P[2], one2,
                                    rcp2(P[3])};
 #pragma unroll
             for (int pi = 0; pi < 10; ++pi) cf[pi * 64 + dp] = pack_bf16(cv[pi].x, cv[pi].y);
-            const float2 gl = mul2(P01, P23);
-            *reinterpret_cast<float2 *>(out + ITEM_GL + d0 * 4) = gl;
+            *reinterpret_cast<float2 *>(out + ITEM_GL + d0 * 4) = mul2(P01, P23);
         }
-        __syncthreads();  // every g read is done: the G region becomes KEXP / KBB
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
             const int i = 16 * J + u;
@@ -302,18 +300,17 @@ __global__ void __launch_bounds__(256, 1)
             const float2 xk = unpack_bf16(*reinterpret_cast<const uint32_t *>(sm + S::K + a16));
             const float2 xq = unpack_bf16(*reinterpret_cast<const uint32_t *>(sm + S::Q + a16));
             const float2 kb = mul2(xk, e[u]);
-            const float2 qb = mul2(mul2(xq, e[u]), make_float2(scale, scale));
+            const float2 qb = mul2(xq, mul2(e[u], s2));
             const float2 kx = mul2(kb, myE);
-            const float2 qg = mul2(mul2(xq, e[u]), sE);
+            const float2 qg = mul2(qb, myE);
             const float2 kbb = mul2(xk, bb[u]);
             const float2 kg = mul2(kbb, myF);
             *reinterpret_cast<uint32_t *>(sm + S::K + a16) = pack_bf16(kb.x, kb.y);
             *reinterpret_cast<uint32_t *>(sm + S::Q + a16) = pack_bf16(qb.x, qb.y);
             *reinterpret_cast<uint32_t *>(sm + S::KEXP + a16) = pack_f16(kx.x, kx.y);
             *reinterpret_cast<uint32_t *>(sm + S::KBB + a16) = pack_bf16(kbb.x, kbb.y);
-            const uint32_t a256 = swz(i, d0 * 2, 256);
-            *reinterpret_cast<uint32_t *>(out + ITEM_QG + a256) = pack_f16(qg.x, qg.y);
-            *reinterpret_cast<uint32_t *>(out + ITEM_KG + a256) = pack_f16(kg.x, kg.y);
+            *reinterpret_cast<uint32_t *>(out + ITEM_QG + a16) = pack_f16(qg.x, qg.y);
+            *reinterpret_cast<uint32_t *>(out + ITEM_KG + a16) = pack_f16(kg.x, kg.y);
         }
     }
     __syncthreads();
@@ -331,17 +328,14 @@ __global__ void __launch_bounds__(256, 1)
             const int ar = 16 * I + (mi & 1) * 8 + (lane & 7), ac = 16 * ks + (mi >> 1) * 8;
             ldsm_x4(sb + S::K + lh(ar, ac), ak[0], ak[1], ak[2], ak[3]);
             ldsm_x4(sb + S::Q + lh(ar, ac), aq[0], aq[1], aq[2], aq[3]);
-            const uint32_t c_lo = cf[8 * ks + t4], c_hi = cf[8 * ks + 4 + t4];
-            ak[0] = hmul2_bf16(ak[0], c_lo);
-            ak[1] = hmul2_bf16(ak[1], c_lo);
-            ak[2] = hmul2_bf16(ak[2], c_hi);
-            ak[3] = hmul2_bf16(ak[3], c_hi);
-            aq[0] = hmul2_bf16(aq[0], c_lo);
-            aq[1] = hmul2_bf16(aq[1], c_lo);
-            aq[2] = hmul2_bf16(aq[2], c_hi);
-            aq[3] = hmul2_bf16(aq[3], c_hi);
             const int br = 16 * J + (mi >> 1) * 8 + (lane & 7), bc = 16 * ks + (mi & 1) * 8;
             ldsm_x4(sb + S::KBB + lh(br, bc), b[0], b[1], b[2], b[3]);
+            // the pair's per-channel factor scales the key side: b0/b2 hold channels 2t,2t+1, b1/b3 channels 2t+8,2t+9
+            const uint32_t c_lo = cf[8 * ks + t4], c_hi = cf[8 * ks + 4 + t4];
+            b[0] = hmul2_bf16(b[0], c_lo);
+            b[1] = hmul2_bf16(b[1], c_hi);
+            b[2] = hmul2_bf16(b[2], c_lo);
+            b[3] = hmul2_bf16(b[3], c_hi);
             mma_bf16(accL[0], ak, b[0], b[1]);
             mma_bf16(accL[1], ak, b[2], b[3]);
             mma_bf16(accQ[0], aq, b[0], b[1]);
@@ -362,12 +356,20 @@ __global__ void __launch_bounds__(256, 1)
                 *reinterpret_cast<uint32_t *>(out + ITEM_AQK + swz(i, j * 2, 128)) = pack_f16(q0, q1);
             }
     }
+    // The carry kernel multiplies the whole 64x64 Aqk tile: its six upper 16x16 blocks must be zeros.
+    for (int idx = tid; idx < 6 * 16 * 8; idx += 256) {
+        const int blk = idx >> 7, r = (idx >> 3) & 15, w = idx & 7;  // block, row in block, 4-byte word in block row
+        const int I = (blk < 3) ? 0 : (blk < 5) ? 1 : 2;
+        const int J = (blk < 3) ? blk + 1 : (blk < 5) ? blk - 1 : 3;
+        const int i = 16 * I + r, j = 16 * J + 2 * w;
+        *reinterpret_cast<uint32_t *>(out + ITEM_AQK + swz(i, j * 2, 128)) = 0u;
+    }
     __syncthreads();
 
     // ---- 5. A = (I+L)^-1 diag(beta) ----
-    uint8_t *sX = sm + S::X;
-    if (warp < 4 && lane < 16) {  // diagonal blocks: exact float32 forward substitution, lane = column
-        const int I = warp, cidx = lane;
+    uint8_t *sX = sm + S::X;  // overlays q*base, dead after step 4
+    if (warp < 2) {  // diagonal blocks: exact float32 forward substitution; half-warp = block, lane = column
+        const int I = 2 * warp + (lane >> 4), cidx = lane & 15;
         float dcol[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -401,12 +403,12 @@ __global__ void __launch_bounds__(256, 1)
     }
     __syncthreads();
 
-    // ---- 6. -W = -A (exp(G) k) and U = A v (fp16 MMAs); warp = 16 columns ----
+    // ---- 6. -W = -A (exp(G) k) (warp = 16 key columns) and U^T = v^T A^T (warp = 16 value rows); fp16 MMAs ----
     {
         const int mi = lane >> 3;
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
-            float w[2][4] = {}, u[2][4] = {};
+            float w[2][4] = {};
             for (int ks = 0; ks <= mt; ++ks) {
                 uint32_t a[4];
                 ldsm_x4(sb + S::A + swz(16 * mt + (mi & 1) * 8 + (lane & 7), (16 * ks + (mi >> 1) * 8) * 2, 128), a[0], a[1],
@@ -416,9 +418,6 @@ __global__ void __launch_bounds__(256, 1)
                 ldsm_x4_t(sb + S::KEXP + lh(tok, col), b0, b1, b2, b3);
                 mma_f16(w[0], a, b0, b1);
                 mma_f16(w[1], a, b2, b3);
-                ldsm_x4_t(sb + S::V + lh(tok, col), b0, b1, b2, b3);
-                mma_f16(u[0], a, b0, b1);
-                mma_f16(u[1], a, b2, b3);
             }
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
@@ -426,21 +425,37 @@ __global__ void __launch_bounds__(256, 1)
                 for (int hr = 0; hr < 2; ++hr) {
                     const int r = 16 * mt + g8 + 8 * hr;
                     const int c = 16 * warp + 8 * nt + 2 * t4;
-                    *reinterpret_cast<uint32_t *>(out + ITEM_WN + swz(r, c * 2, 256)) =
-                        pack_f16(-w[nt][2 * hr], -w[nt][2 * hr + 1]);
-                    *reinterpret_cast<uint32_t *>(out + ITEM_U + (c >> 5) * 4096 + r * 64 + (c & 31) * 2) =
+                    *reinterpret_cast<uint32_t *>(out + ITEM_WN + lh(r, c)) = pack_f16(-w[nt][2 * hr], -w[nt][2 * hr + 1]);
+                }
+        }
+        // U^T[v][i] = sum_j v[j][v] A[i][j]: A operand v^T from V (ldmatrix.trans), B operand A (rows i, K = j)
+        uint32_t av[4][4];
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const int tok = 16 * ks + (mi >> 1) * 8 + (lane & 7), col = 16 * warp + (mi & 1) * 8;
+            ldsm_x4_t(sb + S::V + lh(tok, col), av[ks][0], av[ks][1], av[ks][2], av[ks][3]);
+        }
+#pragma unroll
+        for (int nb = 0; nb < 4; ++nb) {
+            float u[2][4] = {};
+#pragma unroll
+            for (int ks = 0; ks <= nb; ++ks) {
+                const int i = 16 * nb + (mi >> 1) * 8 + (lane & 7), j = 16 * ks + (mi & 1) * 8;
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(sb + S::A + swz(i, j * 2, 128), b0, b1, b2, b3);
+                mma_f16(u[0], av[ks], b0, b1);
+                mma_f16(u[1], av[ks], b2, b3);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int vr = 16 * warp + g8 + 8 * hr;  // value row
+                    const int tk = 16 * nb + 8 * nt + 2 * t4;  // token column
+                    *reinterpret_cast<uint32_t *>(out + ITEM_U + vr * 128 + (((tk >> 3) ^ (vr & 7)) << 4) + (tk & 7) * 2) =
                         pack_f16(u[nt][2 * hr], u[nt][2 * hr + 1]);
                 }
         }
-    }
-
-    // ---- 7. bulk store of the item block ----
-    fence_proxy_async();
-    __syncthreads();
-    if (tid == 0) {
-        bulk_store(out_g, sb + S::OUT, ITEM_BYTES);
-        bulk_commit();
-        bulk_wait_all();
     }
 }
 

@@ -145,16 +145,12 @@ Workspace workspace_layout(int B, int T, int HV, int num_seqs)
     return w;
 }
 
-template <int NW>
-cudaError_t launch_carry(const kda::CarryParams &p0, int units, cudaStream_t stream)
+cudaError_t launch_carry(const kda::CarryParams &p, int units, cudaStream_t stream)
 {
-    using S = kda::CarrySmem<NW>;
-    cudaError_t err = cudaFuncSetAttribute(kda::kda_carry_kernel<NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           S::TOTAL);
+    cudaError_t err = cudaFuncSetAttribute(kda::kda_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kda::CarrySmem::TOTAL);
     if (err != cudaSuccess) return err;
-    kda::CarryParams p = p0;
-    p.nslices = DV / S::VS;
-    kda::kda_carry_kernel<NW><<<units * p.nslices, (NW + 1) * 32, S::TOTAL, stream>>>(p);
+    kda::kda_carry_kernel<<<units, kda::kCarryThreads, kda::CarrySmem::TOTAL, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -284,10 +280,7 @@ extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const 
     cp.HV = HV;
     cp.N = d.N;
     cp.chunks_per_seq = (T + CH - 1) / CH;
-    // Value-column slices: 4 slices of 32 columns when (sequence, head) units
-    // alone would leave most SMs idle, else 2 slices of 64.
-    const int units = d.N * HV;
-    const cudaError_t err = (units * 4 <= info.sms) ? launch_carry<2>(cp, units, s) : launch_carry<4>(cp, units, s);
+    const cudaError_t err = launch_carry(cp, d.N * HV, s);
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -172,6 +172,19 @@ def test_outputs_fully_written():
     assert torch.isfinite(o.float()).all() and torch.isfinite(s).all()
 
 
+def test_stale_workspace_contents_are_ignored():
+    # The workspace needs no initialisation: NaN bytes left in it must not reach the outputs.
+    import kda_gated_delta_prefill_b200 as kda
+    case = gen.Case("stale", B=1, T=200, H=2, HV=4, state="n01", seed=87)
+    x = gen.make_inputs(case)
+    xc = to_cuda(x)
+    n = kda.workspace_size(1, 200, 2, 4)
+    ws = torch.full((n,), 0xFF, dtype=torch.uint8, device="cuda")
+    o, s = kda.forward(xc["q"], xc["k"], xc["v"], xc["g"], xc["beta"], xc["initial_state"], workspace=ws)
+    torch.cuda.synchronize()
+    compare(o, s, oracle_forward(x))
+
+
 def test_inputs_not_mutated():
     case = gen.Case("mut", B=1, T=130, H=2, HV=2, state="n01", seed=81)
     x = to_cuda(gen.make_inputs(case))
