@@ -49,12 +49,14 @@ struct IntraSmem {
     static constexpr int L = 81920;      // fp32 [64][64]
     static constexpr int X = Q;          // fp32 [64][64], once q*base is no longer needed
     static constexpr int A = K;          // fp16 [64][64], once k*base is no longer needed
+    static constexpr int WST = Q;        // fp16 -W staging (step 6), once X is no longer needed
+    static constexpr int UST = L;        // fp16 U^T staging (step 6), once L is no longer needed
     static constexpr int BETA = 98304;   // fp32 [64]
     static constexpr int CF = 98560;     // bf16x2 [10][64] block-pair factors
     static constexpr int PS = 101120;    // float2 [4][64] block products
-    static constexpr int TS = 103168;    // fp32 3 x [16][24] solve scratch
-    static constexpr int BAR = 107776;   // mbarrier
-    static constexpr int TOTAL = 107840;
+    static constexpr int TS = 103168;    // fp32 8 x [16][8] solve scratch
+    static constexpr int BAR = 107776;   // mbarriers: q/k/g tiles, v tile
+    static constexpr int TOTAL = 107848;
 };
 
 struct IntraParams {
@@ -67,15 +69,16 @@ struct IntraParams {
     int chunks_per_seq;        // ceil(T/64) when cu is null
 };
 
-constexpr int TSW = 24;  // row stride (floats) of the 16x16 solve scratch; conflict-free column reads
-
-// Off-diagonal block of X = (I+L)^-1: X_IJ = -D_I * sum_{M=J}^{I-1} L_IM X_MJ (one warp, tf32 MMAs).
-__device__ __forceinline__ void solve_block(const uint8_t *sL, uint8_t *sX, float *ts, int I, int J, int lane)
+// Off-diagonal block of X = (I+L)^-1, columns 16J+8nt .. +7:
+//   X_IJ = -D_I * sum_{M=J}^{I-1} L_IM X_MJ   (D_I = X_II; one warp, tf32 MMAs).
+// ts: this warp's [16][8] float scratch for the intermediate sum.
+__device__ __forceinline__ void solve_block(const uint8_t *sL, uint8_t *sX, float *ts, int I, int J, int nt, int lane)
 {
     const int g = lane >> 2, t = lane & 3;
     auto Lat = [&](int r, int c) { return *reinterpret_cast<const float *>(sL + swz(r, c * 4, 256)); };
     auto Xat = [&](int r, int c) { return *reinterpret_cast<const float *>(sX + swz(r, c * 4, 256)); };
-    float acc[2][4] = {};
+    const int cn = 16 * J + 8 * nt + g;  // this lane's column of the B fragments
+    float acc[4] = {};
     for (int M = J; M < I; ++M) {
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
@@ -84,23 +87,15 @@ __device__ __forceinline__ void solve_block(const uint8_t *sL, uint8_t *sX, floa
             a[1] = to_tf32(Lat(16 * I + g + 8, 16 * M + 8 * ks + t));
             a[2] = to_tf32(Lat(16 * I + g, 16 * M + 8 * ks + t + 4));
             a[3] = to_tf32(Lat(16 * I + g + 8, 16 * M + 8 * ks + t + 4));
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const uint32_t b0 = to_tf32(Xat(16 * M + 8 * ks + t, 16 * J + 8 * nt + g));
-                const uint32_t b1 = to_tf32(Xat(16 * M + 8 * ks + t + 4, 16 * J + 8 * nt + g));
-                mma_tf32(acc[nt], a, b0, b1);
-            }
+            mma_tf32(acc, a, to_tf32(Xat(16 * M + 8 * ks + t, cn)), to_tf32(Xat(16 * M + 8 * ks + t + 4, cn)));
         }
     }
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        ts[g * TSW + 8 * nt + 2 * t] = acc[nt][0];
-        ts[g * TSW + 8 * nt + 2 * t + 1] = acc[nt][1];
-        ts[(g + 8) * TSW + 8 * nt + 2 * t] = acc[nt][2];
-        ts[(g + 8) * TSW + 8 * nt + 2 * t + 1] = acc[nt][3];
-    }
+    ts[g * 8 + 2 * t] = acc[0];
+    ts[g * 8 + 2 * t + 1] = acc[1];
+    ts[(g + 8) * 8 + 2 * t] = acc[2];
+    ts[(g + 8) * 8 + 2 * t + 1] = acc[3];
     __syncwarp();
-    float x[2][4] = {};
+    float x[4] = {};
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
         uint32_t a[4];
@@ -108,19 +103,11 @@ __device__ __forceinline__ void solve_block(const uint8_t *sL, uint8_t *sX, floa
         a[1] = to_tf32(Xat(16 * I + g + 8, 16 * I + 8 * ks + t));
         a[2] = to_tf32(Xat(16 * I + g, 16 * I + 8 * ks + t + 4));
         a[3] = to_tf32(Xat(16 * I + g + 8, 16 * I + 8 * ks + t + 4));
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const uint32_t b0 = to_tf32(ts[(8 * ks + t) * TSW + 8 * nt + g]);
-            const uint32_t b1 = to_tf32(ts[(8 * ks + t + 4) * TSW + 8 * nt + g]);
-            mma_tf32(x[nt], a, b0, b1);
-        }
+        mma_tf32(x, a, to_tf32(ts[(8 * ks + t) * 8 + g]), to_tf32(ts[(8 * ks + t + 4) * 8 + g]));
     }
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        const int c = 16 * J + 8 * nt + 2 * t;
-        *reinterpret_cast<float2 *>(sX + swz(16 * I + g, c * 4, 256)) = make_float2(-x[nt][0], -x[nt][1]);
-        *reinterpret_cast<float2 *>(sX + swz(16 * I + g + 8, c * 4, 256)) = make_float2(-x[nt][2], -x[nt][3]);
-    }
+    const int c = 16 * J + 8 * nt + 2 * t;
+    *reinterpret_cast<float2 *>(sX + swz(16 * I + g, c * 4, 256)) = make_float2(-x[0], -x[1]);
+    *reinterpret_cast<float2 *>(sX + swz(16 * I + g + 8, c * 4, 256)) = make_float2(-x[2], -x[3]);
     __syncwarp();
 }
 
@@ -164,18 +151,20 @@ __global__ void __launch_bounds__(256, 2)
     const uint32_t bar = sb + S::BAR;
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(bar + 8, 1);
         fence_mbar_init();
     }
     __syncthreads();
     if (tid == 0) {
-        mbar_expect_tx(bar, 3 * 16384 + 32768);
+        mbar_expect_tx(bar, 2 * 16384 + 32768);
+        mbar_expect_tx(bar + 8, 16384);
         const int z = static_cast<int>(row0);
         tma_load_3d(sb + S::Q, &tq, 0, hq, z, bar);
         tma_load_3d(sb + S::Q + 8192, &tq, 64, hq, z, bar);
         tma_load_3d(sb + S::K, &tk, 0, hq, z, bar);
         tma_load_3d(sb + S::K + 8192, &tk, 64, hq, z, bar);
-        tma_load_3d(sb + S::V, &tv, 0, h, z, bar);
-        tma_load_3d(sb + S::V + 8192, &tv, 64, h, z, bar);
+        tma_load_3d(sb + S::V, &tv, 0, h, z, bar + 8);
+        tma_load_3d(sb + S::V + 8192, &tv, 64, h, z, bar + 8);
         tma_load_3d(sb + S::G, &tg, 0, h, z, bar);
     }
     float *sbeta = reinterpret_cast<float *>(sm + S::BETA);
@@ -184,23 +173,23 @@ __global__ void __launch_bounds__(256, 2)
         atomicOr(p.err, ERR_TMA_WAIT);
         return;
     }
-    if (nvalid < CH) {  // zero the padding rows of a partial chunk
-        for (int idx = tid; idx < (CH - nvalid) * 64; idx += 256) {
-            const int r = nvalid + idx / 64, w = idx % 64;  // 64 words of 16 bytes per row over q,k,v,g
+    if (nvalid < CH) {  // zero the padding rows of a partial chunk (q, k, g; v once it has arrived)
+        for (int idx = tid; idx < (CH - nvalid) * 48; idx += 256) {
+            const int r = nvalid + idx / 48, w = idx % 48;  // 16-byte words: q 16, k 16, g 32 (two per step)
             uint4 *dst;
-            if (w < 48) {
-                const int buf = w / 16, c16 = w % 16;  // q, k, v: two halves of 8 chunks
+            if (w < 32) {
+                const int buf = w / 16, c16 = w % 16;  // q, k: two halves of 8 chunks
                 dst = reinterpret_cast<uint4 *>(sm + buf * 16384 + (c16 >> 3) * 8192 + r * 128 + ((c16 & 7) << 4));
             } else {
-                dst = reinterpret_cast<uint4 *>(sm + S::G + r * 512 + (w - 48) * 16);
-                dst[16] = make_uint4(0, 0, 0, 0);  // g rows are 32 words; cover the second 16 too
+                dst = reinterpret_cast<uint4 *>(sm + S::G + r * 512 + (w - 32) * 16);
+                dst[16] = make_uint4(0, 0, 0, 0);
             }
             *dst = make_uint4(0, 0, 0, 0);
         }
     }
     __syncthreads();
 
-    // ---- 2. normalise q and k (thread = row half), v -> fp16 ----
+    // ---- 2. normalise q and k (thread = row half) ----
     {
         const int r = tid >> 1, half = tid & 1;
         uint8_t *tile = sm + (r < CH ? S::Q : S::K) + half * 8192 + (r & 63) * 128;
@@ -235,19 +224,6 @@ __global__ void __launch_bounds__(256, 2)
                 w[j] = pack_bf16(y.x, y.y);
             }
             *reinterpret_cast<uint4 *>(tile + ((c ^ rs) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        // v: 1024 chunks of 16 bytes, 4 per thread, bf16 -> fp16 in place
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            uint4 *pv = reinterpret_cast<uint4 *>(sm + S::V) + (tid + 256 * k);
-            uint4 u = *pv;
-            uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 x = unpack_bf16(w[j]);
-                w[j] = pack_f16(x.x, x.y);
-            }
-            *pv = make_uint4(w[0], w[1], w[2], w[3]);
         }
     }
     __syncthreads();
@@ -315,46 +291,39 @@ __global__ void __launch_bounds__(256, 2)
     }
     __syncthreads();
 
-    // ---- 4. L and Aqk over the ten lower block pairs (bf16 MMAs) ----
-    for (int pidx = warp; pidx < 10; pidx += 8) {
+    // ---- 4. L and Aqk over the ten lower block pairs x two 8-column tiles (bf16 MMAs) ----
+    for (int task = warp; task < 20; task += 8) {
+        const int pidx = task >> 1, nt = task & 1;
         const int I = (pidx >= 6) ? 3 : (pidx >= 3) ? 2 : (pidx >= 1) ? 1 : 0;
         const int J = pidx - I * (I + 1) / 2;
         const uint32_t *cf = reinterpret_cast<const uint32_t *>(sm + S::CF) + pidx * 64;
-        float accL[2][4] = {}, accQ[2][4] = {};
+        float accL[4] = {}, accQ[4] = {};
         const int mi = lane >> 3;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-            uint32_t ak[4], aq[4], b[4];
+            uint32_t ak[4], aq[4], b0, b1;
             const int ar = 16 * I + (mi & 1) * 8 + (lane & 7), ac = 16 * ks + (mi >> 1) * 8;
             ldsm_x4(sb + S::K + lh(ar, ac), ak[0], ak[1], ak[2], ak[3]);
             ldsm_x4(sb + S::Q + lh(ar, ac), aq[0], aq[1], aq[2], aq[3]);
-            const int br = 16 * J + (mi >> 1) * 8 + (lane & 7), bc = 16 * ks + (mi & 1) * 8;
-            ldsm_x4(sb + S::KBB + lh(br, bc), b[0], b[1], b[2], b[3]);
-            // the pair's per-channel factor scales the key side: b0/b2 hold channels 2t,2t+1, b1/b3 channels 2t+8,2t+9
-            const uint32_t c_lo = cf[8 * ks + t4], c_hi = cf[8 * ks + 4 + t4];
-            b[0] = hmul2_bf16(b[0], c_lo);
-            b[1] = hmul2_bf16(b[1], c_hi);
-            b[2] = hmul2_bf16(b[2], c_lo);
-            b[3] = hmul2_bf16(b[3], c_hi);
-            mma_bf16(accL[0], ak, b[0], b[1]);
-            mma_bf16(accL[1], ak, b[2], b[3]);
-            mma_bf16(accQ[0], aq, b[0], b[1]);
-            mma_bf16(accQ[1], aq, b[2], b[3]);
+            ldsm_x2(sb + S::KBB + lh(16 * J + 8 * nt + (lane & 7), 16 * ks + (mi & 1) * 8), b0, b1);
+            // the pair's per-channel factor scales the key side: b0 holds channels 2t,2t+1, b1 channels 2t+8,2t+9
+            b0 = hmul2_bf16(b0, cf[8 * ks + t4]);
+            b1 = hmul2_bf16(b1, cf[8 * ks + 4 + t4]);
+            mma_bf16(accL, ak, b0, b1);
+            mma_bf16(accQ, aq, b0, b1);
         }
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int i = 16 * I + g8 + 8 * hr;
-                const int j = 16 * J + 8 * nt + 2 * t4;
-                const float bi = sbeta[i];
-                const float l0 = (j < i) ? bi * accL[nt][2 * hr] : 0.f;
-                const float l1 = (j + 1 < i) ? bi * accL[nt][2 * hr + 1] : 0.f;
-                const float q0 = (j <= i) ? accQ[nt][2 * hr] : 0.f;
-                const float q1 = (j + 1 <= i) ? accQ[nt][2 * hr + 1] : 0.f;
-                *reinterpret_cast<float2 *>(sm + S::L + swz(i, j * 4, 256)) = make_float2(l0, l1);
-                *reinterpret_cast<uint32_t *>(out + ITEM_AQK + swz(i, j * 2, 128)) = pack_f16(q0, q1);
-            }
+        for (int hr = 0; hr < 2; ++hr) {
+            const int i = 16 * I + g8 + 8 * hr;
+            const int j = 16 * J + 8 * nt + 2 * t4;
+            const float bi = sbeta[i];
+            const float l0 = (j < i) ? bi * accL[2 * hr] : 0.f;
+            const float l1 = (j + 1 < i) ? bi * accL[2 * hr + 1] : 0.f;
+            const float q0 = (j <= i) ? accQ[2 * hr] : 0.f;
+            const float q1 = (j + 1 <= i) ? accQ[2 * hr + 1] : 0.f;
+            *reinterpret_cast<float2 *>(sm + S::L + swz(i, j * 4, 256)) = make_float2(l0, l1);
+            *reinterpret_cast<uint32_t *>(out + ITEM_AQK + swz(i, j * 2, 128)) = pack_f16(q0, q1);
+        }
     }
     // The carry kernel multiplies the whole 64x64 Aqk tile: its six upper 16x16 blocks must be zeros.
     for (int idx = tid; idx < 6 * 16 * 8; idx += 256) {
@@ -385,13 +354,13 @@ __global__ void __launch_bounds__(256, 2)
             *reinterpret_cast<float *>(sX + swz(16 * I + j, (16 * I + cidx) * 4, 256)) = dcol[j];
     }
     __syncthreads();
-    {
-        float *ts = reinterpret_cast<float *>(sm + S::TS) + (warp % 3) * 16 * TSW;
-        if (warp < 3) solve_block(sm + S::L, sX, ts, warp + 1, warp, lane);
+    {  // block forward substitution by distance from the diagonal; one warp per (block, 8-column tile)
+        float *ts = reinterpret_cast<float *>(sm + S::TS) + warp * 128;
+        if (warp < 6) solve_block(sm + S::L, sX, ts, (warp >> 1) + 1, warp >> 1, warp & 1, lane);
         __syncthreads();
-        if (warp < 2) solve_block(sm + S::L, sX, ts, warp + 2, warp, lane);
+        if (warp < 4) solve_block(sm + S::L, sX, ts, (warp >> 1) + 2, warp >> 1, warp & 1, lane);
         __syncthreads();
-        if (warp < 1) solve_block(sm + S::L, sX, ts, 3, 0, lane);
+        if (warp < 2) solve_block(sm + S::L, sX, ts, 3, 0, warp & 1, lane);
         __syncthreads();
     }
     for (int idx = tid; idx < CH * CH / 2; idx += 256) {
@@ -400,6 +369,27 @@ __global__ void __launch_bounds__(256, 2)
         const float a0 = (j <= i) ? x.x * sbeta[j] : 0.f;
         const float a1 = (j + 1 <= i) ? x.y * sbeta[j + 1] : 0.f;
         *reinterpret_cast<uint32_t *>(sm + S::A + swz(i, j * 2, 128)) = pack_f16(a0, a1);
+    }
+    __syncthreads();
+
+    // ---- v tile (its copy overlapped steps 2-5): zero padding rows, bf16 -> fp16 in place ----
+    if (!mbar_wait(bar + 8, 0)) {
+        atomicOr(p.err, ERR_TMA_WAIT);
+        return;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int idx = tid + 256 * k;  // 16-byte chunk: half (idx >> 9), row ((idx >> 3) & 63)
+        uint4 *pv = reinterpret_cast<uint4 *>(sm + S::V) + idx;
+        uint4 u = *pv;
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        const bool pad = ((idx >> 3) & 63) >= nvalid;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 x = unpack_bf16(w[j]);
+            w[j] = pad ? 0u : pack_f16(x.x, x.y);
+        }
+        *pv = make_uint4(w[0], w[1], w[2], w[3]);
     }
     __syncthreads();
 
@@ -425,7 +415,7 @@ __global__ void __launch_bounds__(256, 2)
                 for (int hr = 0; hr < 2; ++hr) {
                     const int r = 16 * mt + g8 + 8 * hr;
                     const int c = 16 * warp + 8 * nt + 2 * t4;
-                    *reinterpret_cast<uint32_t *>(out + ITEM_WN + lh(r, c)) = pack_f16(-w[nt][2 * hr], -w[nt][2 * hr + 1]);
+                    *reinterpret_cast<uint32_t *>(sm + S::WST + lh(r, c)) = pack_f16(-w[nt][2 * hr], -w[nt][2 * hr + 1]);
                 }
         }
         // U^T[v][i] = sum_j v[j][v] A[i][j]: A operand v^T from V (ldmatrix.trans), B operand A (rows i, K = j)
@@ -452,10 +442,19 @@ __global__ void __launch_bounds__(256, 2)
                 for (int hr = 0; hr < 2; ++hr) {
                     const int vr = 16 * warp + g8 + 8 * hr;  // value row
                     const int tk = 16 * nb + 8 * nt + 2 * t4;  // token column
-                    *reinterpret_cast<uint32_t *>(out + ITEM_U + vr * 128 + (((tk >> 3) ^ (vr & 7)) << 4) + (tk & 7) * 2) =
+                    *reinterpret_cast<uint32_t *>(sm + S::UST + vr * 128 + (((tk >> 3) ^ (vr & 7)) << 4) + (tk & 7) * 2) =
                         pack_f16(u[nt][2 * hr], u[nt][2 * hr + 1]);
                 }
         }
+    }
+    // -W and U^T leave through two bulk copies (their smem images match the item layout)
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+        bulk_store(out + ITEM_WN, sb + S::WST, 16384);
+        bulk_store(out + ITEM_U, sb + S::UST, 16384);
+        bulk_commit();
+        bulk_wait_all();
     }
 }
 
