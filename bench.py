@@ -336,8 +336,9 @@ def main():
         cb = time_oracle(case)
         cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
 
-    # intra-chunk kernel + carry kernel (+ chunk-offset and order kernels for packed batches)
-    launches_per_step = 2 + (2 if case.lengths is not None else 0)
+    # intra-chunk and carry kernels per part of the sequence (+ chunk-offset and order kernels for packed batches)
+    launches_per_step = kda.kernel_launches(case.B, case.T, case.H, case.HV, case.K, case.V,
+                                            len(case.lengths) if case.lengths is not None else 0)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,

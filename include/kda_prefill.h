@@ -95,6 +95,17 @@ size_t kda_prefill_workspace_size(int B, int T, int H, int HV, int K, int V, int
  *                 bytes, 256-byte aligned, overlapping no other argument.
  *                 Its contents need no initialisation and are garbage after.
  *   stream        cudaStream_t
+ *
+ * Asynchronous on `stream`.  A plain batch (cu_seqlens NULL) with fewer
+ * (sequence, value head) pairs than the device has SMs and at least 32
+ * chunks per sequence is run as up to 8 consecutive parts of the sequence
+ * (whole chunks): the state carry of each part runs on a high-priority side
+ * stream that the library creates once per device, overlapping the
+ * intra-chunk work of the next part, and joins `stream` again through an
+ * event before the call returns, so the caller sees one ordered operation
+ * (under stream capture the side stream becomes a fork and join of the
+ * captured graph).  Calls from several host threads on one device share that
+ * side stream, so their carry parts run one after another.
  */
 kda_status_t kda_prefill_forward(const void *q, const void *k, const void *v,
                                  const float *g, const float *beta,
@@ -157,10 +168,18 @@ kda_status_t kda_prefill_forward_noalloc(const void *q, const void *k, const voi
  * Debug aid: the device error word of the current device.  Kernel waits on
  * copies and pipeline stages are bounded (about one second); a wait that
  * gives up sets a bit here (1: input tile copy, 2: stage fill, 4: stage
- * release) and the kernel stops early instead of hanging.  Synchronises the
+ * release) and the kernel stops early instead of hanging; bit 8 means a
+ * tensor-memory allocation did not start at column 0 (not expected to happen).  Synchronises the
  * device.  clear != 0 resets the word afterwards.
  */
 kda_status_t kda_prefill_device_error(unsigned *word, int clear);
+
+/*
+ * Number of kernel launches kda_prefill_forward makes for these sizes on the
+ * current device (the split into parts above depends on its SM count), or 0
+ * for sizes it would reject.
+ */
+int kda_prefill_kernel_launches(int B, int T, int H, int HV, int K, int V, int num_seqs);
 
 /*
  * Step 1 alone: L2-normalise `rows` rows of K bf16 values with the exact

@@ -27,7 +27,7 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 
 EXPORTED = ("kda_status_string", "kda_prefill_workspace_size", "kda_prefill_forward",
             "kda_prefill_host_staging_size", "kda_prefill_forward_host", "kda_prefill_device_error",
-            "kda_l2norm_bf16")
+            "kda_l2norm_bf16", "kda_prefill_kernel_launches")
 
 
 class KdaError(RuntimeError):
@@ -65,6 +65,8 @@ def lib():
         L.kda_prefill_device_error.restype = I
         L.kda_l2norm_bf16.argtypes = [P, I64, I, P, P]
         L.kda_l2norm_bf16.restype = I
+        L.kda_prefill_kernel_launches.argtypes = [I] * 7
+        L.kda_prefill_kernel_launches.restype = I
         _lib = L
         return L
 
@@ -94,6 +96,11 @@ def _dims(q, v, cu_seqlens):
 
 def workspace_size(B, T, H, HV, K=128, V=128, num_seqs=0) -> int:
     return int(lib().kda_prefill_workspace_size(B, T, H, HV, K, V, num_seqs))
+
+
+def kernel_launches(B, T, H, HV, K=128, V=128, num_seqs=0) -> int:
+    """Kernel launches one forward makes for these sizes on the current CUDA device (0 if rejected)."""
+    return int(lib().kda_prefill_kernel_launches(B, T, H, HV, K, V, num_seqs))
 
 
 def forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o=None, final_state=None,

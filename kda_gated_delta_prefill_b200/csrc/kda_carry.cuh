@@ -14,6 +14,8 @@
 // chunk); the last warp allocates TMEM and issues the MMAs.  Every wait is
 // bounded.
 #pragma once
+#include <type_traits>
+
 #include "kda_common.cuh"
 #include "ptx.cuh"
 #include "tc.cuh"
@@ -46,6 +48,8 @@ struct CarryParams {
     unsigned *err;
     int T, HV, N;
     int chunks_per_seq;
+    int chunk_begin;           // cu null: this launch carries chunks [chunk_begin, chunk_begin + chunk_count)
+    int chunk_count;           //   of every sequence, from s0 (cu given: whole sequences, chunk_begin = 0)
 };
 
 __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const CarryParams p)
@@ -65,10 +69,10 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
         tok0 = p.cu[n];
         len = p.cu[n + 1] - p.cu[n];
     } else {
-        c_begin = static_cast<int64_t>(n) * p.chunks_per_seq;
-        nck = p.chunks_per_seq;
-        tok0 = static_cast<int64_t>(n) * p.T;
-        len = p.T;
+        c_begin = static_cast<int64_t>(n) * p.chunks_per_seq + p.chunk_begin;
+        nck = p.chunk_count;
+        tok0 = static_cast<int64_t>(n) * p.T + static_cast<int64_t>(p.chunk_begin) * CH;
+        len = p.T - p.chunk_begin * CH;
     }
 
     const uint32_t full0 = sb + S::BAR, empty0 = full0 + 16, barP = full0 + 32, barS = full0 + 40,
@@ -91,12 +95,19 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + S::TMEM_SLOT);
+    // The CTA allocates all 512 columns, so the allocation can only start at lane 0, column 0: every TMEM
+    // address below is a compile-time constant (fewer instructions per MMA issue and per tcgen05.ld/st).
+    const uint32_t tmem_alloc = *reinterpret_cast<volatile uint32_t *>(sm + S::TMEM_SLOT);
+    constexpr uint32_t tmem = 0;
 
     auto fail = [&](unsigned code) {
         atomicOr(p.err, code);
         *abort_flag = 1;
     };
+    if (tmem_alloc != 0) {
+        if (tid == 0) fail(ERR_TMEM_BASE);
+        nck = 0;
+    }
 
     if (warp == kCarryEpiWarps) {
         // ---------------- producer: one bulk copy per chunk block ----------------
@@ -113,46 +124,61 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
             }
         }
     } else if (warp == kCarryEpiWarps + 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            const uint32_t i64 = idesc_f16(128, 64, false), i128mn = idesc_f16(128, 128, true);
-            // stage-0 descriptors; stage s adds s*STAGE/16 to the start-address field
-            const uint64_t dW = sw128_desc(sb + ITEM_WN, 16, 1024), dQ = sw128_desc(sb + ITEM_QG, 16, 1024);
-            const uint64_t dA = sw128_desc(sb + ITEM_AQK, 16, 1024), dK = sw128_desc(sb + ITEM_KG, 8192, 1024);
-            for (int c = 0; c < nck && !*abort_flag; ++c) {
-                const int s = c % S::NST;
-                const uint64_t so = static_cast<uint64_t>(s * (S::STAGE >> 4));
-                if (!mbar_wait(full0 + 8 * s, (c / S::NST) & 1) || !mbar_wait_spin(sready, c & 1)) {
-                    fail(ERR_PIPE_FULL_WAIT);
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t tmo = tmem + TM_O0 + 64 * (c & 1);
-                // P^T = S^T W^T (K = 128 keys, 8 steps); W is stored negated, so P^T = -(S^T W^T)
+        // ---------------- MMA issuer: the whole warp walks the chunks, one elected lane issues ----------------
+        // The body is instantiated once per ring stage, so every descriptor is a constant offset from the
+        // shared-memory base.
+        // Descriptor = high word (strides, swizzle) : low word (start address >> 4, leading offset).  Start
+        // addresses stay below 2^18 bytes, so offsets only ever touch the low word.
+        const uint32_t i64 = idesc_f16(128, 64, false), i128mn = idesc_f16(128, 128, true);
+        const uint64_t dk0 = sw128_desc(sb, 16, 1024), kk0 = sw128_desc(sb, 8192, 1024);
+        const uint32_t dhi = static_cast<uint32_t>(dk0 >> 32), khi = static_cast<uint32_t>(kk0 >> 32);
+        auto chunk = [&](int c, auto stage) -> bool {
+            constexpr int st = decltype(stage)::value;
+            constexpr uint32_t so = static_cast<uint32_t>(st * (S::STAGE >> 4));
+            // opaque per chunk, so the compiler forms each descriptor next to its MMA instead of keeping
+            // all of them live across the loop
+            uint32_t dlo = static_cast<uint32_t>(dk0), klo = static_cast<uint32_t>(kk0);
+            asm volatile("" : "+r"(dlo), "+r"(klo));
+            auto dbase = [&](uint32_t off) { return (static_cast<uint64_t>(dhi) << 32) | (dlo + off); };
+            auto kbase = [&](uint32_t off) { return (static_cast<uint64_t>(khi) << 32) | (klo + off); };
+            const bool ok = mbar_wait(full0 + 8 * st, (c / S::NST) & 1) && mbar_wait_spin(sready, c & 1);
+            if (!__all_sync(0xffffffffu, ok)) return false;
+            tc_fence_after();
+            const uint32_t tmo = tmem + TM_O0 + 64 * (c & 1);
+            // P^T = S^T W^T (K = 128 keys, 8 steps); W is stored negated, so P^T = -(S^T W^T)
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    tc_mma_ts(tmem + TM_P, tmem + TA_S + 8 * ks, dW + so + (ks >> 2) * 512 + (ks & 3) * 2, i64, ks > 0);
-                tc_commit(barP);
-                // O^T = S^T Qg^T
+            for (int ks = 0; ks < 8; ++ks)
+                tc_mma_ts_warp(tmem + TM_P, tmem + TA_S + 8 * ks,
+                               dbase(so + (ITEM_WN >> 4) + (ks >> 2) * 512 + (ks & 3) * 2), i64, ks > 0);
+            tc_commit_warp(barP);
+            // O^T = S^T Qg^T
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    tc_mma_ts(tmo, tmem + TA_S + 8 * ks, dQ + so + (ks >> 2) * 512 + (ks & 3) * 2, i64, ks > 0);
-                if (!mbar_wait_spin(vready, c & 1)) {
-                    fail(ERR_PIPE_FULL_WAIT);
-                    break;
-                }
-                tc_fence_after();
-                // S^T += Vnew^T Kg onto the decayed master state (on the chain to the next chunk, so first).
-                // Kg is MN-major: 64-key blocks 8192 bytes apart, token groups of 8 rows 1024 bytes apart.
+            for (int ks = 0; ks < 8; ++ks)
+                tc_mma_ts_warp(tmo, tmem + TA_S + 8 * ks, dbase(so + (ITEM_QG >> 4) + (ks >> 2) * 512 + (ks & 3) * 2),
+                               i64, ks > 0);
+            if (!__all_sync(0xffffffffu, mbar_wait_spin(vready, c & 1))) return false;
+            tc_fence_after();
+            // S^T += Vnew^T Kg onto the decayed master state (on the chain to the next chunk, so first).
+            // Kg is MN-major: 64-key blocks 8192 bytes apart, token groups of 8 rows 1024 bytes apart.
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) tc_mma_ts(tmem + TM_S, tmem + TA_V + 8 * ks, dK + so + ks * 128, i128mn, 1);
-                tc_commit(barS);
-                // O^T += Vnew^T Aqk^T (K = 64 tokens)
+            for (int ks = 0; ks < 4; ++ks)
+                tc_mma_ts_warp(tmem + TM_S, tmem + TA_V + 8 * ks, kbase(so + (ITEM_KG >> 4) + ks * 128), i128mn, 1);
+            tc_commit_warp(barS);
+            // O^T += Vnew^T Aqk^T (K = 64 tokens)
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    tc_mma_ts(tmo, tmem + TA_V + 8 * ks, dA + so + ks * 2, i64, 1);
-                tc_commit(barO);
-                tc_commit(empty0 + 8 * s);
+            for (int ks = 0; ks < 4; ++ks)
+                tc_mma_ts_warp(tmo, tmem + TA_V + 8 * ks, dbase(so + (ITEM_AQK >> 4) + ks * 2), i64, 1);
+            tc_commit_warp(barO);
+            tc_commit_warp(empty0 + 8 * st);
+            return true;
+        };
+        static_assert(S::NST == 2, "the issuer body is instantiated for two stages");
+        for (int c = 0; c < nck; ++c) {
+            if (__any_sync(0xffffffffu, *abort_flag)) break;
+            const bool ok = (c & 1) ? chunk(c, std::integral_constant<int, 1>{}) : chunk(c, std::integral_constant<int, 0>{});
+            if (!ok) {
+                if (lane == 0) fail(ERR_PIPE_FULL_WAIT);
+                break;
             }
         }
     } else {
@@ -163,19 +189,29 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
         const uint32_t tS = tmem + lane_base + TM_S + 32 * kq;     // fp32 master S^T[v][32kq .. 32kq+31]
         const uint32_t tA = tmem + lane_base + TA_S + 16 * kq;     // its fp16 copy (A operand)
         const int64_t ostride = static_cast<int64_t>(p.HV) * DV;
-        {
-            const float *s0 = p.s0 ? p.s0 + (static_cast<int64_t>(n) * p.HV + h) * DK * DV : nullptr;
-            uint32_t r[32], w[16];
+        // S^T[v][32kq ..] (this thread's 32 master-state values) -> fp16 A operand of the next chunk's MMAs.
+        auto publish = [&](const uint32_t (&r)[32]) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s0 ? s0[(32 * kq + j) * DV + v] : 0.f);
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t w[8];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) w[j] = pack_f16(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-            tc_st32(tS, r);
-            tc_st16(tA, w);
+                for (int j = 0; j < 8; ++j)
+                    w[j] = pack_f16(__uint_as_float(r[16 * hf + 2 * j]), __uint_as_float(r[16 * hf + 2 * j + 1]));
+                tc_st8(tA + 8 * hf, w);
+            }
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sready);
+        };
+        bool alive = tmem_alloc == 0;
+        if (alive) {
+            const float *s0 = p.s0 ? p.s0 + (static_cast<int64_t>(n) * p.HV + h) * DK * DV : nullptr;
+            uint32_t r[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s0 ? s0[(32 * kq + j) * DV + v] : 0.f);
+            tc_st32(tS, r);
+            publish(r);
         }
         // o rows of chunk c: O^T[v][tok], tok in [16*kq, 16*kq+16); a warp writes 64 contiguous bytes per token
         auto store_o = [&](int c) {
@@ -194,7 +230,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
             }
         };
 
-        for (int c = 0; c < nck && !*abort_flag; ++c) {
+        for (int c = 0; c < nck && alive && !*abort_flag; ++c) {
             const int s = c % S::NST;
             const uint8_t *st = sm + s * S::STAGE;
             // --- while MMA1/O1 of chunk c run: S^T <- S^T diag(exp(G_last)) ---
@@ -264,16 +300,10 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
             }
             tc_fence_after();
             {
-                uint32_t r[32], w[16];
+                uint32_t r[32];
                 tc_ld32(tS, r);
                 tc_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 16; ++j) w[j] = pack_f16(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-                tc_st16(tA, w);
-                tc_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(sready);
+                publish(r);
             }
         }
         if (nck > 0 && !*abort_flag) {
@@ -284,8 +314,8 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
                 fail(ERR_PIPE_FULL_WAIT);
             }
         }
-        // final state (S^T[v][kd] -> final_state[kd][v])
-        {
+        // final state (S^T[v][kd] -> final_state[kd][v]); skipped when the TMEM allocation was unusable
+        if (tmem_alloc == 0) {
             uint32_t r[32];
             tc_ld32(tS, r);
             tc_wait_ld();
@@ -299,7 +329,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
     __syncthreads();
     if (warp == kCarryEpiWarps + 1) {
         tc_fence_after();
-        tc_dealloc(tmem, TM_COLS);
+        tc_dealloc(tmem_alloc, TM_COLS);
     }
 }
 

@@ -67,6 +67,9 @@ struct IntraParams {
     unsigned *err;
     int B, T, H, HV, N;
     int chunks_per_seq;        // ceil(T/64) when cu is null
+    int chunk_begin;           // cu null: this launch covers chunks [chunk_begin, chunk_begin + chunk_count)
+    int chunk_count;           //   of every sequence (cu given: all chunks, chunk_begin = 0)
+    int prefetch_stride;       // CTAs resident at once (L2 prefetch distance), 0 = no prefetch
 };
 
 // Off-diagonal block of X = (I+L)^-1, columns 16J+8nt .. +7:
@@ -111,7 +114,9 @@ __device__ __forceinline__ void solve_block(const uint8_t *sL, uint8_t *sX, floa
     __syncwarp();
 }
 
-__global__ void __launch_bounds__(256, 2)
+constexpr int kIntraCtasPerSm = 2;  // the shared-memory footprint and register cap let two CTAs share an SM
+
+__global__ void __launch_bounds__(256, kIntraCtasPerSm)
     kda_intra_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg,
                      const IntraParams p)
@@ -122,28 +127,34 @@ __global__ void __launch_bounds__(256, 2)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g8 = lane >> 2, t4 = lane & 3;
 
-    // ---- item -> (row of the chunk start, valid rows) ----
+    // ---- launch-local chunk -> (item chunk index, row of the chunk start, valid rows); false past the end ----
+    const int nchunks = p.cu ? p.chunk_off[p.N] : p.B * p.chunk_count;
+    auto locate = [&](int local, int &ci, int64_t &row0, int &nvalid) {
+        if (local >= nchunks) return false;
+        if (p.cu) {
+            ci = local;
+            int lo = 0, hi = p.N - 1;  // last n with chunk_off[n] <= ci
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (p.chunk_off[mid] <= ci) lo = mid; else hi = mid - 1;
+            }
+            const int c = ci - p.chunk_off[lo];
+            const int len = p.cu[lo + 1] - p.cu[lo];
+            row0 = p.cu[lo] + static_cast<int64_t>(c) * CH;
+            nvalid = min(CH, len - c * CH);
+        } else {
+            const int b = local / p.chunk_count, c = p.chunk_begin + local % p.chunk_count;
+            ci = b * p.chunks_per_seq + c;
+            row0 = static_cast<int64_t>(b) * p.T + static_cast<int64_t>(c) * CH;
+            nvalid = min(CH, p.T - c * CH);
+        }
+        return true;
+    };
     const int h = blockIdx.x % p.HV;
-    const int ci = blockIdx.x / p.HV;
+    int ci;
     int64_t row0;
     int nvalid;
-    if (p.cu) {
-        const int nc = p.chunk_off[p.N];
-        if (ci >= nc) return;
-        int lo = 0, hi = p.N - 1;  // last n with chunk_off[n] <= ci
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (p.chunk_off[mid] <= ci) lo = mid; else hi = mid - 1;
-        }
-        const int c = ci - p.chunk_off[lo];
-        const int len = p.cu[lo + 1] - p.cu[lo];
-        row0 = p.cu[lo] + static_cast<int64_t>(c) * CH;
-        nvalid = min(CH, len - c * CH);
-    } else {
-        const int b = ci / p.chunks_per_seq, c = ci % p.chunks_per_seq;
-        row0 = static_cast<int64_t>(b) * p.T + static_cast<int64_t>(c) * CH;
-        nvalid = min(CH, p.T - c * CH);
-    }
+    if (!locate(blockIdx.x / p.HV, ci, row0, nvalid)) return;
     const int hq = h / (p.HV / p.H);
     uint8_t *out = p.items + (static_cast<int64_t>(ci) * p.HV + h) * ITEM_BYTES;  // item block (global)
 
@@ -166,6 +177,22 @@ __global__ void __launch_bounds__(256, 2)
         tma_load_3d(sb + S::V, &tv, 0, h, z, bar + 8);
         tma_load_3d(sb + S::V + 8192, &tv, 64, h, z, bar + 8);
         tma_load_3d(sb + S::G, &tg, 0, h, z, bar);
+        // The CTA that takes this slot after the current wave of resident CTAs will want item
+        // blockIdx.x + prefetch_stride: pull its inputs into L2 now, so that its loads overlap the compute
+        // of this wave instead of waiting on DRAM.
+        const int pi = blockIdx.x + p.prefetch_stride;
+        int pci, pvalid;
+        int64_t prow;
+        if (p.prefetch_stride > 0 && pi < static_cast<int>(gridDim.x) && locate(pi / p.HV, pci, prow, pvalid)) {
+            const int ph = pi % p.HV, pz = static_cast<int>(prow), phq = ph / (p.HV / p.H);
+            tma_prefetch_3d(&tq, 0, phq, pz);
+            tma_prefetch_3d(&tq, 64, phq, pz);
+            tma_prefetch_3d(&tk, 0, phq, pz);
+            tma_prefetch_3d(&tk, 64, phq, pz);
+            tma_prefetch_3d(&tv, 0, ph, pz);
+            tma_prefetch_3d(&tv, 64, ph, pz);
+            tma_prefetch_3d(&tg, 0, ph, pz);
+        }
     }
     float *sbeta = reinterpret_cast<float *>(sm + S::BETA);
     if (tid < CH) sbeta[tid] = (tid < nvalid) ? p.beta[(row0 + tid) * p.HV + h] : 0.f;

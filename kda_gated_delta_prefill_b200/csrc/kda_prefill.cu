@@ -45,6 +45,7 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb)
 // Per-device facts looked up once: SM count and the error word's device address.
 struct DeviceInfo {
     bool ready = false;
+    int dev = 0;
     int sms = 148;
     unsigned *err = nullptr;
 };
@@ -60,6 +61,7 @@ cudaError_t device_info(DeviceInfo &out)
     std::lock_guard<std::mutex> lock(g_info_mu);
     DeviceInfo &d = g_info[dev];
     if (!d.ready) {
+        d.dev = dev;
         e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
         e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_kda_device_error);
@@ -145,6 +147,52 @@ Workspace workspace_layout(int B, int T, int HV, int num_seqs)
     return w;
 }
 
+// Fixed-length batches with fewer (sequence, value head) units than SMs leave most of the GPU idle while the
+// state carry runs.  Such a forward is cut into parts along the sequence (whole chunks): the carry of part j
+// runs on a high-priority side stream, one CTA per unit, while the intra-chunk kernel of part j+1 fills the
+// remaining SMs.  The carry of part j starts from the state part j-1 left in final_state.
+constexpr int kMaxParts = 8;
+constexpr int kMinChunksPerPart = 16;
+
+int pipeline_parts(int B, int T, int HV, bool varlen, int sms)
+{
+    if (varlen || static_cast<int64_t>(B) * HV >= sms) return 1;
+    const int chunks = (T + CH - 1) / CH;
+    const int parts = chunks / kMinChunksPerPart;
+    return parts < 2 ? 1 : (parts < kMaxParts ? parts : kMaxParts);
+}
+
+// The side stream and the fork/join events of one device, created on first use.  The mutex keeps one
+// forward's launches and event records together when several host threads share the device.
+struct CarryLane {
+    bool ready = false;
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    std::mutex mu;
+};
+CarryLane g_lane[kMaxDevices];
+std::mutex g_lane_mu;
+
+cudaError_t carry_lane(int dev, CarryLane *&out)
+{
+    std::lock_guard<std::mutex> lock(g_lane_mu);
+    CarryLane &l = g_lane[dev];
+    if (!l.ready) {
+        int least = 0, greatest = 0;
+        cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+        if (e != cudaSuccess) return e;
+        e = cudaStreamCreateWithPriority(&l.stream, cudaStreamNonBlocking, greatest);
+        if (e != cudaSuccess) return e;
+        e = cudaEventCreateWithFlags(&l.fork, cudaEventDisableTiming);
+        if (e != cudaSuccess) return e;
+        e = cudaEventCreateWithFlags(&l.join, cudaEventDisableTiming);
+        if (e != cudaSuccess) return e;
+        l.ready = true;
+    }
+    out = &l;
+    return cudaSuccess;
+}
+
 cudaError_t launch_carry(const kda::CarryParams &p, int units, cudaStream_t stream)
 {
     cudaError_t err = cudaFuncSetAttribute(kda::kda_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -174,6 +222,17 @@ extern "C" size_t kda_prefill_workspace_size(int B, int T, int H, int HV, int K,
     Dims d;
     if (check_dims(B, T, H, HV, K, V, num_seqs > 0, num_seqs, d) != KDA_OK) return 0;
     return workspace_layout(B, T, HV, num_seqs > 0 ? num_seqs : 0).total;
+}
+
+extern "C" int kda_prefill_kernel_launches(int B, int T, int H, int HV, int K, int V, int num_seqs)
+{
+    Dims d;
+    const bool varlen = num_seqs > 0;
+    if (check_dims(B, T, H, HV, K, V, varlen, num_seqs, d) != KDA_OK) return 0;
+    DeviceInfo info;
+    if (device_info(info) != cudaSuccess) return 0;
+    if (varlen) return 2 + (T > 0 ? 1 : 0) + 1;  // chunk offsets, order, intra (if any token), carry
+    return 2 * pipeline_parts(B, T, HV, false, info.sms);
 }
 
 extern "C" kda_status_t kda_prefill_device_error(unsigned *word, int clear)
@@ -239,15 +298,15 @@ extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const 
         if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
     }
 
+    CUtensorMap tq, tk, tv, tg;
+    kda::IntraParams ip{};
     if (tokens > 0) {
-        CUtensorMap tq, tk, tv, tg;
         const int64_t rows = tokens;
         if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, rows, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HV, rows, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HV, rows, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
             return KDA_ERR_CUDA;
-        kda::IntraParams ip{};
         ip.beta = beta;
         ip.cu = cu_seqlens;
         ip.chunk_off = chunk_off;
@@ -259,13 +318,18 @@ extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const 
         ip.HV = HV;
         ip.N = d.N;
         ip.chunks_per_seq = (T + CH - 1) / CH;
+        ip.prefetch_stride = info.sms * kda::kIntraCtasPerSm;
         if (cudaFuncSetAttribute(kda::kda_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kda::IntraSmem::TOTAL) != cudaSuccess)
             return KDA_ERR_CUDA;
-        kda::kda_intra_kernel<<<static_cast<int>(ws.max_chunks * HV), 256, kda::IntraSmem::TOTAL, s>>>(tq, tk, tv, tg,
-                                                                                                        ip);
-        if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
     }
+    auto launch_intra = [&](int chunk_begin, int chunk_count, int64_t grid_chunks) {
+        ip.chunk_begin = chunk_begin;
+        ip.chunk_count = chunk_count;
+        kda::kda_intra_kernel<<<static_cast<int>(grid_chunks * HV), 256, kda::IntraSmem::TOTAL, s>>>(tq, tk, tv, tg,
+                                                                                                      ip);
+        return cudaGetLastError();
+    };
 
     kda::CarryParams cp{};
     cp.items = items;
@@ -280,8 +344,33 @@ extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const 
     cp.HV = HV;
     cp.N = d.N;
     cp.chunks_per_seq = (T + CH - 1) / CH;
-    const cudaError_t err = launch_carry(cp, d.N * HV, s);
-    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+
+    const int parts = pipeline_parts(B, T, HV, varlen, info.sms);
+    if (parts == 1) {
+        if (tokens > 0 && launch_intra(0, cp.chunks_per_seq, ws.max_chunks) != cudaSuccess) return KDA_ERR_CUDA;
+        cp.chunk_begin = 0;
+        cp.chunk_count = cp.chunks_per_seq;
+        return launch_carry(cp, d.N * HV, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
+
+    CarryLane *lane = nullptr;
+    if (carry_lane(info.dev, lane) != cudaSuccess) return KDA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(lane->mu);
+    const int nck = cp.chunks_per_seq;
+    for (int j = 0; j < parts; ++j) {
+        const int c0 = static_cast<int>(static_cast<int64_t>(nck) * j / parts);
+        const int c1 = static_cast<int>(static_cast<int64_t>(nck) * (j + 1) / parts);
+        if (launch_intra(c0, c1 - c0, static_cast<int64_t>(B) * (c1 - c0)) != cudaSuccess) return KDA_ERR_CUDA;
+        if (cudaEventRecord(lane->fork, s) != cudaSuccess || cudaStreamWaitEvent(lane->stream, lane->fork, 0) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        cp.s0 = j == 0 ? initial_state : final_state;
+        cp.chunk_begin = c0;
+        cp.chunk_count = c1 - c0;
+        if (launch_carry(cp, d.N * HV, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    if (cudaEventRecord(lane->join, lane->stream) != cudaSuccess || cudaStreamWaitEvent(s, lane->join, 0) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    return KDA_OK;
 }
 
 extern "C" size_t kda_prefill_host_staging_size(int B, int T, int H, int HV, int K, int V, int num_seqs,

@@ -9,7 +9,7 @@
 namespace kda {
 
 // ---- device error word (bounded waits that gave up set a bit here) ----
-enum : unsigned { ERR_TMA_WAIT = 1u, ERR_PIPE_FULL_WAIT = 2u, ERR_PIPE_EMPTY_WAIT = 4u };
+enum : unsigned { ERR_TMA_WAIT = 1u, ERR_PIPE_FULL_WAIT = 2u, ERR_PIPE_EMPTY_WAIT = 4u, ERR_TMEM_BASE = 8u };
 // Spin budget of every wait, in SM clock cycles (about one second at 2 GHz).
 constexpr long long kWaitBudget = 2000000000LL;
 
@@ -88,6 +88,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
         "[%5];\n" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
         : "memory");
+}
+// Start fetching a tensor tile into L2 only (no shared-memory destination, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int x, int y, int z)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];\n" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
 }
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
 {

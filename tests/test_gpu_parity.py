@@ -217,3 +217,56 @@ def test_repeat_calls_are_deterministic():
     o1, s1 = gpu_forward(x)
     o2, s2 = gpu_forward(x)
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+# ------------------------------------------------------------------ sequence cut into parts
+# A fixed-length batch with fewer (sequence, value head) units than SMs and at least 32 chunks per sequence is
+# run as consecutive parts of the sequence, the state carry of one part overlapping the intra-chunk work of the
+# next.  The cut points are whole chunks, so the arithmetic per chunk is that of the uncut run.
+
+@pytest.mark.parametrize("T,state", [(2088, "n01"), (5120, "none"), (8209, "n01")])
+def test_parts_full_parity(T, state):
+    case = gen.Case(f"parts{T}", B=1, T=T, H=2, HV=2, state=state, seed=300 + T)
+    x = gen.make_inputs(case)
+    o, s = gpu_forward(x)
+    compare(o, s, oracle_forward(x))
+
+
+def test_parts_match_the_uncut_run_bit_for_bit():
+    # The same sequence passed as a packed batch of one sequence takes the uncut path.
+    case = gen.Case("parts_vs_uncut", B=1, T=4160, H=2, HV=4, state="n01", seed=311)
+    x = gen.make_inputs(case)
+    o_cut, s_cut = gpu_forward(x)
+    xv = dict(x)
+    xv["cu_seqlens"] = torch.tensor([0, case.T], dtype=torch.int32)
+    o_one, s_one = gpu_forward(xv)
+    assert torch.equal(o_cut, o_one)
+    assert torch.equal(s_cut, s_one)
+
+
+def test_parts_in_place_state_update():
+    case = gen.Case("parts_inplace", B=1, T=3000, H=2, HV=2, state="n01", seed=321)
+    x = gen.make_inputs(case)
+    ref = oracle_forward(x)
+    xc = to_cuda(x)
+    import kda_gated_delta_prefill_b200 as kda
+    st = xc["initial_state"].clone()
+    o, s = kda.forward(xc["q"], xc["k"], xc["v"], xc["g"], xc["beta"], st, final_state=st)
+    torch.cuda.synchronize()
+    assert s.data_ptr() == st.data_ptr()
+    compare(o, s, ref)
+
+
+def test_parts_on_a_non_default_stream():
+    case = gen.Case("parts_stream", B=1, T=2600, H=2, HV=2, state="n01", seed=331)
+    x = gen.make_inputs(case)
+    ref = oracle_forward(x)
+    xc = to_cuda(x)
+    import kda_gated_delta_prefill_b200 as kda
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        o, s = kda.forward(xc["q"], xc["k"], xc["v"], xc["g"], xc["beta"], xc["initial_state"])
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    compare(o, s, ref)
