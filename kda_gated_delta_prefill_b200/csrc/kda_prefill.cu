@@ -356,10 +356,13 @@ extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const 
     CarryLane *lane = nullptr;
     if (carry_lane(info.dev, lane) != cudaSuccess) return KDA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(lane->mu);
+    // The last part's carry has nothing left to overlap with, so it is a quarter of the size of the others:
+    // part j starts at chunk nck * 4j / (4 parts - 3).
     const int nck = cp.chunks_per_seq;
+    const int64_t den = 4 * parts - 3;
     for (int j = 0; j < parts; ++j) {
-        const int c0 = static_cast<int>(static_cast<int64_t>(nck) * j / parts);
-        const int c1 = static_cast<int>(static_cast<int64_t>(nck) * (j + 1) / parts);
+        const int c0 = static_cast<int>(static_cast<int64_t>(nck) * 4 * j / den);
+        const int c1 = j + 1 == parts ? nck : static_cast<int>(static_cast<int64_t>(nck) * 4 * (j + 1) / den);
         if (launch_intra(c0, c1 - c0, static_cast<int64_t>(B) * (c1 - c0)) != cudaSuccess) return KDA_ERR_CUDA;
         if (cudaEventRecord(lane->fork, s) != cudaSuccess || cudaStreamWaitEvent(lane->stream, lane->fork, 0) != cudaSuccess)
             return KDA_ERR_CUDA;
