@@ -10,7 +10,7 @@
 // token columns (warp/4); they keep the float32 master state S^T[v][:] in registers and
 // write its fp16 copy into TMEM, where it is the A operand of the next
 // chunk's MMAs.  Warp 16 streams the per-chunk blocks written by the
-// intra-chunk kernel into a two-stage shared-memory ring (one bulk copy per
+// intra-chunk kernel into a three-stage shared-memory ring (one bulk copy per
 // chunk); the last warp allocates TMEM and issues the MMAs.  Every wait is
 // bounded.
 #pragma once
@@ -24,9 +24,11 @@ namespace kda {
 
 struct CarrySmem {
     static constexpr int STAGE = ((ITEM_BYTES + 1023) / 1024) * 1024;  // 75776
-    static constexpr int NST = 2;
-    static constexpr int BAR = NST * STAGE;   // mbarriers: full[2] empty[2] barP barS sready vready barO
-    static constexpr int TMEM_SLOT = BAR + 9 * 8;
+    // Three stages (222 KB): a chunk block is requested two chunk periods before it is needed, which covers
+    // the copy latency while the intra-chunk kernel loads HBM on the other SMs.
+    static constexpr int NST = 3;
+    static constexpr int BAR = NST * STAGE;   // mbarriers: full[NST] empty[NST] barP barS sready vready barO
+    static constexpr int TMEM_SLOT = BAR + (2 * NST + 5) * 8;
     static constexpr int ABORT = TMEM_SLOT + 4;
     static constexpr int TOTAL = ABORT + 12;
 };
@@ -75,8 +77,8 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
         len = p.T - p.chunk_begin * CH;
     }
 
-    const uint32_t full0 = sb + S::BAR, empty0 = full0 + 16, barP = full0 + 32, barS = full0 + 40,
-                   sready = full0 + 48, vready = full0 + 56, barO = full0 + 64;
+    const uint32_t full0 = sb + S::BAR, empty0 = full0 + 8 * S::NST, barP = full0 + 16 * S::NST, barS = barP + 8,
+                   sready = barP + 16, vready = barP + 24, barO = barP + 32;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + S::ABORT);
     if (tid == 0) {
         for (int s = 0; s < S::NST; ++s) {
@@ -172,10 +174,13 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
             tc_commit_warp(empty0 + 8 * st);
             return true;
         };
-        static_assert(S::NST == 2, "the issuer body is instantiated for two stages");
+        static_assert(S::NST == 3, "the issuer body is instantiated for three stages");
         for (int c = 0; c < nck; ++c) {
             if (__any_sync(0xffffffffu, *abort_flag)) break;
-            const bool ok = (c & 1) ? chunk(c, std::integral_constant<int, 1>{}) : chunk(c, std::integral_constant<int, 0>{});
+            const int st = c % S::NST;
+            const bool ok = st == 0   ? chunk(c, std::integral_constant<int, 0>{})
+                            : st == 1 ? chunk(c, std::integral_constant<int, 1>{})
+                                      : chunk(c, std::integral_constant<int, 2>{});
             if (!ok) {
                 if (lane == 0) fail(ERR_PIPE_FULL_WAIT);
                 break;

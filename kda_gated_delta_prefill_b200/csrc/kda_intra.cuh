@@ -73,9 +73,11 @@ struct IntraParams {
 };
 
 // Off-diagonal block of X = (I+L)^-1, columns 16J+8nt .. +7:
-//   X_IJ = -D_I * sum_{M=J}^{I-1} L_IM X_MJ   (D_I = X_II; one warp, tf32 MMAs).
+//   X_IJ = -D_I * sum_{M=J}^{I-1} L_IM X_MJ   (D_I = X_II; one warp, tf32 MMAs),
+// written as fp32 X (for later blocks) and as fp16 A = X diag(beta) (for W and U).
 // ts: this warp's [16][8] float scratch for the intermediate sum.
-__device__ __forceinline__ void solve_block(const uint8_t *sL, uint8_t *sX, float *ts, int I, int J, int nt, int lane)
+__device__ __forceinline__ void solve_block(const uint8_t *sL, uint8_t *sX, uint8_t *sA, const float *beta, float *ts, int I,
+                                            int J, int nt, int lane)
 {
     const int g = lane >> 2, t = lane & 3;
     auto Lat = [&](int r, int c) { return *reinterpret_cast<const float *>(sL + swz(r, c * 4, 256)); };
@@ -111,6 +113,10 @@ __device__ __forceinline__ void solve_block(const uint8_t *sL, uint8_t *sX, floa
     const int c = 16 * J + 8 * nt + 2 * t;
     *reinterpret_cast<float2 *>(sX + swz(16 * I + g, c * 4, 256)) = make_float2(-x[0], -x[1]);
     *reinterpret_cast<float2 *>(sX + swz(16 * I + g + 8, c * 4, 256)) = make_float2(-x[2], -x[3]);
+    // A = X diag(beta) in fp16 for step 6
+    const float b0 = beta[c], b1 = beta[c + 1];
+    *reinterpret_cast<uint32_t *>(sA + swz(16 * I + g, c * 2, 128)) = pack_f16(-x[0] * b0, -x[1] * b1);
+    *reinterpret_cast<uint32_t *>(sA + swz(16 * I + g + 8, c * 2, 128)) = pack_f16(-x[2] * b0, -x[3] * b1);
     __syncwarp();
 }
 
@@ -318,38 +324,46 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
     }
     __syncthreads();
 
-    // ---- 4. L and Aqk over the ten lower block pairs x two 8-column tiles (bf16 MMAs) ----
-    for (int task = warp; task < 20; task += 8) {
-        const int pidx = task >> 1, nt = task & 1;
-        const int I = (pidx >= 6) ? 3 : (pidx >= 3) ? 2 : (pidx >= 1) ? 1 : 0;
-        const int J = pidx - I * (I + 1) / 2;
-        const uint32_t *cf = reinterpret_cast<const uint32_t *>(sm + S::CF) + pidx * 64;
-        float accL[4] = {}, accQ[4] = {};
+    // ---- 4. L and Aqk over the ten lower block pairs (bf16 MMAs): warp = (row block I, 8-column tile nt);
+    //         its q and k fragments are loaded once per k-step and serve every column block J <= I ----
+    {
+        const int I = warp >> 1, nt = warp & 1;
+        const uint32_t *cf = reinterpret_cast<const uint32_t *>(sm + S::CF) + (I * (I + 1) / 2) * 64;
+        float accL[4][4] = {}, accQ[4][4] = {};
         const int mi = lane >> 3;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-            uint32_t ak[4], aq[4], b0, b1;
+            uint32_t ak[4], aq[4];
             const int ar = 16 * I + (mi & 1) * 8 + (lane & 7), ac = 16 * ks + (mi >> 1) * 8;
             ldsm_x4(sb + S::K + lh(ar, ac), ak[0], ak[1], ak[2], ak[3]);
             ldsm_x4(sb + S::Q + lh(ar, ac), aq[0], aq[1], aq[2], aq[3]);
-            ldsm_x2(sb + S::KBB + lh(16 * J + 8 * nt + (lane & 7), 16 * ks + (mi & 1) * 8), b0, b1);
-            // the pair's per-channel factor scales the key side: b0 holds channels 2t,2t+1, b1 channels 2t+8,2t+9
-            b0 = hmul2_bf16(b0, cf[8 * ks + t4]);
-            b1 = hmul2_bf16(b1, cf[8 * ks + 4 + t4]);
-            mma_bf16(accL, ak, b0, b1);
-            mma_bf16(accQ, aq, b0, b1);
+#pragma unroll
+            for (int J = 0; J < 4; ++J) {
+                if (J > I) continue;
+                uint32_t b0, b1;
+                ldsm_x2(sb + S::KBB + lh(16 * J + 8 * nt + (lane & 7), 16 * ks + (mi & 1) * 8), b0, b1);
+                // the pair's per-channel factor scales the key side: b0 holds channels 2t,2t+1, b1 channels 2t+8,2t+9
+                b0 = hmul2_bf16(b0, cf[J * 64 + 8 * ks + t4]);
+                b1 = hmul2_bf16(b1, cf[J * 64 + 8 * ks + 4 + t4]);
+                mma_bf16(accL[J], ak, b0, b1);
+                mma_bf16(accQ[J], aq, b0, b1);
+            }
         }
 #pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const int i = 16 * I + g8 + 8 * hr;
-            const int j = 16 * J + 8 * nt + 2 * t4;
-            const float bi = sbeta[i];
-            const float l0 = (j < i) ? bi * accL[2 * hr] : 0.f;
-            const float l1 = (j + 1 < i) ? bi * accL[2 * hr + 1] : 0.f;
-            const float q0 = (j <= i) ? accQ[2 * hr] : 0.f;
-            const float q1 = (j + 1 <= i) ? accQ[2 * hr + 1] : 0.f;
-            *reinterpret_cast<float2 *>(sm + S::L + swz(i, j * 4, 256)) = make_float2(l0, l1);
-            *reinterpret_cast<uint32_t *>(out + ITEM_AQK + swz(i, j * 2, 128)) = pack_f16(q0, q1);
+        for (int J = 0; J < 4; ++J) {
+            if (J > I) continue;
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int i = 16 * I + g8 + 8 * hr;
+                const int j = 16 * J + 8 * nt + 2 * t4;
+                const float bi = sbeta[i];
+                const float l0 = (j < i) ? bi * accL[J][2 * hr] : 0.f;
+                const float l1 = (j + 1 < i) ? bi * accL[J][2 * hr + 1] : 0.f;
+                const float q0 = (j <= i) ? accQ[J][2 * hr] : 0.f;
+                const float q1 = (j + 1 <= i) ? accQ[J][2 * hr + 1] : 0.f;
+                *reinterpret_cast<float2 *>(sm + S::L + swz(i, j * 4, 256)) = make_float2(l0, l1);
+                *reinterpret_cast<uint32_t *>(out + ITEM_AQK + swz(i, j * 2, 128)) = pack_f16(q0, q1);
+            }
         }
     }
     // The carry kernel multiplies the whole 64x64 Aqk tile: its six upper 16x16 blocks must be zeros.
@@ -366,38 +380,36 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
     uint8_t *sX = sm + S::X;  // overlays q*base, dead after step 4
     if (warp < 2) {  // diagonal blocks: exact float32 forward substitution; half-warp = block, lane = column
         const int I = 2 * warp + (lane >> 4), cidx = lane & 15;
+        // right-looking: once row m is final it updates every later row, so the 15 - m updates of a step are
+        // independent; each row still accumulates its terms in the order m = 0, 1, ...
         float dcol[16];
 #pragma unroll
+        for (int j = 0; j < 16; ++j) dcol[j] = (j == cidx) ? 1.f : 0.f;
+#pragma unroll
+        for (int m = 0; m < 15; ++m)
+#pragma unroll
+            for (int j = m + 1; j < 16; ++j)
+                dcol[j] = __fmaf_rn(-*reinterpret_cast<const float *>(sm + S::L + swz(16 * I + j, (16 * I + m) * 4, 256)),
+                                    dcol[m], dcol[j]);
+        const float bc = sbeta[16 * I + cidx];
+#pragma unroll
         for (int j = 0; j < 16; ++j) {
-            float acc = (j == cidx) ? 1.f : 0.f;
-#pragma unroll
-            for (int m = 0; m < j; ++m)
-                acc = __fmaf_rn(-*reinterpret_cast<const float *>(sm + S::L + swz(16 * I + j, (16 * I + m) * 4, 256)),
-                                dcol[m], acc);
-            dcol[j] = acc;
-        }
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
             *reinterpret_cast<float *>(sX + swz(16 * I + j, (16 * I + cidx) * 4, 256)) = dcol[j];
+            // A = X diag(beta) in fp16, zero above the diagonal (step 6 multiplies whole diagonal blocks)
+            *reinterpret_cast<__half *>(sm + S::A + swz(16 * I + j, (16 * I + cidx) * 2, 128)) =
+                __float2half_rn(j >= cidx ? dcol[j] * bc : 0.f);
+        }
     }
     __syncthreads();
     {  // block forward substitution by distance from the diagonal; one warp per (block, 8-column tile)
         float *ts = reinterpret_cast<float *>(sm + S::TS) + warp * 128;
-        if (warp < 6) solve_block(sm + S::L, sX, ts, (warp >> 1) + 1, warp >> 1, warp & 1, lane);
+        if (warp < 6) solve_block(sm + S::L, sX, sm + S::A, sbeta, ts, (warp >> 1) + 1, warp >> 1, warp & 1, lane);
         __syncthreads();
-        if (warp < 4) solve_block(sm + S::L, sX, ts, (warp >> 1) + 2, warp >> 1, warp & 1, lane);
+        if (warp < 4) solve_block(sm + S::L, sX, sm + S::A, sbeta, ts, (warp >> 1) + 2, warp >> 1, warp & 1, lane);
         __syncthreads();
-        if (warp < 2) solve_block(sm + S::L, sX, ts, 3, 0, warp & 1, lane);
+        if (warp < 2) solve_block(sm + S::L, sX, sm + S::A, sbeta, ts, 3, 0, warp & 1, lane);
         __syncthreads();
     }
-    for (int idx = tid; idx < CH * CH / 2; idx += 256) {
-        const int i = idx >> 5, j = (idx & 31) * 2;
-        const float2 x = *reinterpret_cast<const float2 *>(sX + swz(i, j * 4, 256));
-        const float a0 = (j <= i) ? x.x * sbeta[j] : 0.f;
-        const float a1 = (j + 1 <= i) ? x.y * sbeta[j + 1] : 0.f;
-        *reinterpret_cast<uint32_t *>(sm + S::A + swz(i, j * 2, 128)) = pack_f16(a0, a1);
-    }
-    __syncthreads();
 
     // ---- v tile (its copy overlapped steps 2-5): zero padding rows, bf16 -> fp16 in place ----
     if (!mbar_wait(bar + 8, 0)) {
@@ -481,7 +493,7 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
         bulk_store(out + ITEM_WN, sb + S::WST, 16384);
         bulk_store(out + ITEM_U, sb + S::UST, 16384);
         bulk_commit();
-        bulk_wait_all();
+        bulk_wait_read();  // the shared-memory images must outlive the reads, not the global writes
     }
 }
 
