@@ -324,46 +324,59 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
     }
     __syncthreads();
 
-    // ---- 4. L and Aqk over the ten lower block pairs (bf16 MMAs): warp = (row block I, 8-column tile nt);
-    //         its q and k fragments are loaded once per k-step and serve every column block J <= I ----
+    // ---- 4. L and Aqk over the ten lower block pairs x two 8-column tiles (bf16 MMAs).  A warp takes the
+    //         tiles of one row block I and a run of column blocks J, loading its q and k fragments once per
+    //         k-step for all of them; the 20 tiles split 2-2-2-2-3-3-3-3 over the warps:
+    //         warps 0-3: I = 3, J in {0,1} / {2,3};  warps 4-5: I = 2, J in {0,1,2};
+    //         warps 6-7: I = 1, J in {0,1}, then I = 0, J = 0.  nt = warp & 1. ----
     {
-        const int I = warp >> 1, nt = warp & 1;
-        const uint32_t *cf = reinterpret_cast<const uint32_t *>(sm + S::CF) + (I * (I + 1) / 2) * 64;
-        float accL[4][4] = {}, accQ[4][4] = {};
+        const int nt = warp & 1;
         const int mi = lane >> 3;
+        auto tiles = [&](int I, int J0, int nJ) {
+            const uint32_t *cf = reinterpret_cast<const uint32_t *>(sm + S::CF) + (I * (I + 1) / 2 + J0) * 64;
+            float accL[3][4] = {}, accQ[3][4] = {};
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            uint32_t ak[4], aq[4];
-            const int ar = 16 * I + (mi & 1) * 8 + (lane & 7), ac = 16 * ks + (mi >> 1) * 8;
-            ldsm_x4(sb + S::K + lh(ar, ac), ak[0], ak[1], ak[2], ak[3]);
-            ldsm_x4(sb + S::Q + lh(ar, ac), aq[0], aq[1], aq[2], aq[3]);
+            for (int ks = 0; ks < 8; ++ks) {
+                uint32_t ak[4], aq[4];
+                const int ar = 16 * I + (mi & 1) * 8 + (lane & 7), ac = 16 * ks + (mi >> 1) * 8;
+                ldsm_x4(sb + S::K + lh(ar, ac), ak[0], ak[1], ak[2], ak[3]);
+                ldsm_x4(sb + S::Q + lh(ar, ac), aq[0], aq[1], aq[2], aq[3]);
 #pragma unroll
-            for (int J = 0; J < 4; ++J) {
-                if (J > I) continue;
-                uint32_t b0, b1;
-                ldsm_x2(sb + S::KBB + lh(16 * J + 8 * nt + (lane & 7), 16 * ks + (mi & 1) * 8), b0, b1);
-                // the pair's per-channel factor scales the key side: b0 holds channels 2t,2t+1, b1 channels 2t+8,2t+9
-                b0 = hmul2_bf16(b0, cf[J * 64 + 8 * ks + t4]);
-                b1 = hmul2_bf16(b1, cf[J * 64 + 8 * ks + 4 + t4]);
-                mma_bf16(accL[J], ak, b0, b1);
-                mma_bf16(accQ[J], aq, b0, b1);
+                for (int jj = 0; jj < 3; ++jj) {
+                    if (jj >= nJ) continue;
+                    uint32_t b0, b1;
+                    ldsm_x2(sb + S::KBB + lh(16 * (J0 + jj) + 8 * nt + (lane & 7), 16 * ks + (mi & 1) * 8), b0, b1);
+                    // the pair's per-channel factor scales the key side: b0 holds channels 2t,2t+1, b1 2t+8,2t+9
+                    b0 = hmul2_bf16(b0, cf[jj * 64 + 8 * ks + t4]);
+                    b1 = hmul2_bf16(b1, cf[jj * 64 + 8 * ks + 4 + t4]);
+                    mma_bf16(accL[jj], ak, b0, b1);
+                    mma_bf16(accQ[jj], aq, b0, b1);
+                }
             }
-        }
 #pragma unroll
-        for (int J = 0; J < 4; ++J) {
-            if (J > I) continue;
+            for (int jj = 0; jj < 3; ++jj) {
+                if (jj >= nJ) continue;
 #pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int i = 16 * I + g8 + 8 * hr;
-                const int j = 16 * J + 8 * nt + 2 * t4;
-                const float bi = sbeta[i];
-                const float l0 = (j < i) ? bi * accL[J][2 * hr] : 0.f;
-                const float l1 = (j + 1 < i) ? bi * accL[J][2 * hr + 1] : 0.f;
-                const float q0 = (j <= i) ? accQ[J][2 * hr] : 0.f;
-                const float q1 = (j + 1 <= i) ? accQ[J][2 * hr + 1] : 0.f;
-                *reinterpret_cast<float2 *>(sm + S::L + swz(i, j * 4, 256)) = make_float2(l0, l1);
-                *reinterpret_cast<uint32_t *>(out + ITEM_AQK + swz(i, j * 2, 128)) = pack_f16(q0, q1);
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int i = 16 * I + g8 + 8 * hr;
+                    const int j = 16 * (J0 + jj) + 8 * nt + 2 * t4;
+                    const float bi = sbeta[i];
+                    const float l0 = (j < i) ? bi * accL[jj][2 * hr] : 0.f;
+                    const float l1 = (j + 1 < i) ? bi * accL[jj][2 * hr + 1] : 0.f;
+                    const float q0 = (j <= i) ? accQ[jj][2 * hr] : 0.f;
+                    const float q1 = (j + 1 <= i) ? accQ[jj][2 * hr + 1] : 0.f;
+                    *reinterpret_cast<float2 *>(sm + S::L + swz(i, j * 4, 256)) = make_float2(l0, l1);
+                    *reinterpret_cast<uint32_t *>(out + ITEM_AQK + swz(i, j * 2, 128)) = pack_f16(q0, q1);
+                }
             }
+        };
+        if (warp < 4) {
+            tiles(3, 2 * (warp >> 1), 2);
+        } else if (warp < 6) {
+            tiles(2, 0, 3);
+        } else {
+            tiles(1, 0, 2);
+            tiles(0, 0, 1);
         }
     }
     // The carry kernel multiplies the whole 64x64 Aqk tile: its six upper 16x16 blocks must be zeros.
@@ -378,26 +391,33 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
 
     // ---- 5. A = (I+L)^-1 diag(beta) ----
     uint8_t *sX = sm + S::X;  // overlays q*base, dead after step 4
-    if (warp < 2) {  // diagonal blocks: exact float32 forward substitution; half-warp = block, lane = column
-        const int I = 2 * warp + (lane >> 4), cidx = lane & 15;
-        // right-looking: once row m is final it updates every later row, so the 15 - m updates of a step are
-        // independent; each row still accumulates its terms in the order m = 0, 1, ...
-        float dcol[16];
+    {  // diagonal blocks: exact float32 forward substitution on all 256 threads.  Thread = (block I, column c,
+       // row group r4 owning rows r4, r4+4, r4+8, r4+12); the four threads of a column are adjacent lanes.
+       // Right-looking: row m, once final, is broadcast to the column's lanes and updates every later row,
+       // each row accumulating its terms in the order m = 0, 1, ...
+        const int I = tid >> 6, c = (tid >> 2) & 15, r4 = tid & 3;
+        const uint8_t *sLb = sm + S::L;
+        float x[4];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) dcol[j] = (j == cidx) ? 1.f : 0.f;
+        for (int q = 0; q < 4; ++q) x[q] = (4 * q + r4 == c) ? 1.f : 0.f;
 #pragma unroll
-        for (int m = 0; m < 15; ++m)
+        for (int m = 0; m < 15; ++m) {
+            const float xm = __shfl_sync(0xffffffffu, x[m >> 2], (lane & ~3) | (m & 3));
 #pragma unroll
-            for (int j = m + 1; j < 16; ++j)
-                dcol[j] = __fmaf_rn(-*reinterpret_cast<const float *>(sm + S::L + swz(16 * I + j, (16 * I + m) * 4, 256)),
-                                    dcol[m], dcol[j]);
-        const float bc = sbeta[16 * I + cidx];
+            for (int q = m >> 2; q < 4; ++q) {
+                const int j = 4 * q + r4;
+                const float l = *reinterpret_cast<const float *>(sLb + swz(16 * I + j, (16 * I + m) * 4, 256));
+                if (j > m) x[q] = __fmaf_rn(-l, xm, x[q]);
+            }
+        }
+        const float bc = sbeta[16 * I + c];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            *reinterpret_cast<float *>(sX + swz(16 * I + j, (16 * I + cidx) * 4, 256)) = dcol[j];
+        for (int q = 0; q < 4; ++q) {
+            const int j = 4 * q + r4;
+            *reinterpret_cast<float *>(sX + swz(16 * I + j, (16 * I + c) * 4, 256)) = x[q];
             // A = X diag(beta) in fp16, zero above the diagonal (step 6 multiplies whole diagonal blocks)
-            *reinterpret_cast<__half *>(sm + S::A + swz(16 * I + j, (16 * I + cidx) * 2, 128)) =
-                __float2half_rn(j >= cidx ? dcol[j] * bc : 0.f);
+            *reinterpret_cast<__half *>(sm + S::A + swz(16 * I + j, (16 * I + c) * 2, 128)) =
+                __float2half_rn(j >= c ? x[q] * bc : 0.f);
         }
     }
     __syncthreads();
