@@ -452,14 +452,23 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
     }
     __syncthreads();
 
-    // ---- 6. -W = -A (exp(G) k) (warp = 16 key columns) and U^T = v^T A^T (warp = 16 value rows); fp16 MMAs ----
+    // ---- 6. -W = -A (exp(G) k) (warp = 16 key columns) and U^T = v^T A^T (warp = 16 value rows); fp16 MMAs.
+    //         Each 16x16 tile of A is loaded once: as the A operand of W, and, with its fragment registers
+    //         reordered, as the two B fragments (8 rows of A each) of U^T. ----
     {
         const int mi = lane >> 3;
+        // U^T A operand: v^T rows 16*warp .. +15 for the four 16-token K steps (ldmatrix.trans of v)
+        uint32_t av[4][4];
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const int tok = 16 * ks + (mi >> 1) * 8 + (lane & 7), col = 16 * warp + (mi & 1) * 8;
+            ldsm_x4_t(sb + S::V + lh(tok, col), av[ks][0], av[ks][1], av[ks][2], av[ks][3]);
+        }
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
-            float w[2][4] = {};
+            float w[2][4] = {}, u[2][4] = {};
             for (int ks = 0; ks <= mt; ++ks) {
-                uint32_t a[4];
+                uint32_t a[4];  // A rows 16mt + (g, g+8), columns 16ks + (2t, 2t+8)
                 ldsm_x4(sb + S::A + swz(16 * mt + (mi & 1) * 8 + (lane & 7), (16 * ks + (mi >> 1) * 8) * 2, 128), a[0], a[1],
                         a[2], a[3]);
                 const int tok = 16 * ks + (mi & 1) * 8 + (lane & 7), col = 16 * warp + (mi >> 1) * 8;
@@ -467,6 +476,9 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
                 ldsm_x4_t(sb + S::KEXP + lh(tok, col), b0, b1, b2, b3);
                 mma_f16(w[0], a, b0, b1);
                 mma_f16(w[1], a, b2, b3);
+                // U^T[v][i] += v^T[v][j] A[i][j]: B fragment of rows i = 16mt + g is (a0, a2), of i + 8 is (a1, a3)
+                mma_f16(u[0], av[ks], a[0], a[2]);
+                mma_f16(u[1], av[ks], a[1], a[3]);
             }
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
@@ -475,32 +487,8 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
                     const int r = 16 * mt + g8 + 8 * hr;
                     const int c = 16 * warp + 8 * nt + 2 * t4;
                     *reinterpret_cast<uint32_t *>(sm + S::WST + lh(r, c)) = pack_f16(-w[nt][2 * hr], -w[nt][2 * hr + 1]);
-                }
-        }
-        // U^T[v][i] = sum_j v[j][v] A[i][j]: A operand v^T from V (ldmatrix.trans), B operand A (rows i, K = j)
-        uint32_t av[4][4];
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const int tok = 16 * ks + (mi >> 1) * 8 + (lane & 7), col = 16 * warp + (mi & 1) * 8;
-            ldsm_x4_t(sb + S::V + lh(tok, col), av[ks][0], av[ks][1], av[ks][2], av[ks][3]);
-        }
-#pragma unroll
-        for (int nb = 0; nb < 4; ++nb) {
-            float u[2][4] = {};
-#pragma unroll
-            for (int ks = 0; ks <= nb; ++ks) {
-                const int i = 16 * nb + (mi >> 1) * 8 + (lane & 7), j = 16 * ks + (mi & 1) * 8;
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(sb + S::A + swz(i, j * 2, 128), b0, b1, b2, b3);
-                mma_f16(u[0], av[ks], b0, b1);
-                mma_f16(u[1], av[ks], b2, b3);
-            }
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
                     const int vr = 16 * warp + g8 + 8 * hr;  // value row
-                    const int tk = 16 * nb + 8 * nt + 2 * t4;  // token column
+                    const int tk = 16 * mt + 8 * nt + 2 * t4;  // token column
                     *reinterpret_cast<uint32_t *>(sm + S::UST + vr * 128 + (((tk >> 3) ^ (vr & 7)) << 4) + (tk & 7) * 2) =
                         pack_f16(u[nt][2 * hr], u[nt][2 * hr + 1]);
                 }
