@@ -158,28 +158,40 @@ def cpu_sample_inputs(case, heads: int, tokens: int):
     return out
 
 
-def time_oracle(case, target_s: float = 15.0):
+def oracle_sample(case, target_s: float):
+    """A bounded CPU sample of the workload for the oracle: the first `tokens` tokens of the first `heads`
+    value heads (whole GQA groups), sized from a pilot run so that one oracle forward takes about target_s."""
     import oracle
     cores = oracle.max_threads()
     heads = min(case.HV, max(1, cores))
     if case.HV // case.H > 1:
         heads -= heads % (case.HV // case.H) or 0
         heads = max(heads, case.HV // case.H)
-    # pilot: 256 tokens on the chosen heads, then size the sample to about target_s seconds
     pilot_tok = min(case.T, 256)
     xs = cpu_sample_inputs(case, heads, pilot_tok)
     t0 = time.perf_counter()
     oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["initial_state"])
-    dt = time.perf_counter() - t0
-    per_tok = dt / pilot_tok
-    tokens = int(min(case.T, max(pilot_tok, target_s / max(per_tok, 1e-9))))
+    per_tok = (time.perf_counter() - t0) / pilot_tok
+    tokens = int(min(case.T, max(min(pilot_tok, 64), target_s / max(per_tok, 1e-9))))
     xs = cpu_sample_inputs(case, heads, tokens)
+    return xs, tokens, heads, min(cores, heads)
+
+
+def time_oracle(case, target_s: float = 15.0, steps: int = 1, warmup: int = 0):
+    """Time the oracle as it stands on the host cores: `warmup` untimed and `steps` timed forwards of one
+    bounded sample (about target_s seconds each)."""
+    import oracle
+    xs, tokens, heads, cores = oracle_sample(case, target_s)
+    run = lambda: oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["initial_state"])
+    for _ in range(warmup):
+        run()
     t0 = time.perf_counter()
-    oracle.forward(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["initial_state"])
+    for _ in range(steps):
+        run()
     dt = time.perf_counter() - t0
-    return {"value": tokens * heads / dt, "unit": UNIT, "cores": min(cores, heads), "kind": "oracle",
+    return {"value": tokens * heads * steps / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"first {tokens} tokens x value heads 0..{heads - 1} of {case.name}",
-            "seconds": dt}
+            "seconds": dt / steps}
 
 
 # ---------------------------------------------------------------------------------------------- main
@@ -193,6 +205,9 @@ def main():
     ap.add_argument("--workload", default="long_T65536_H64_state")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile-T", type=int, default=0,
+                    help="only run 3 forwards of B=1, H=HV=64, T=<value>, with state, and exit: the small case "
+                         "the ncu captures under profiles/ use")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -214,9 +229,11 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        cb = time_oracle(case)
-        line = {"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": 1,
-                "warmup": 0, "ms_per_step": cb["seconds"] * 1e3, "higher_is_better": True, "scaling": "weak",
+        # each step a bounded sample, sized so that warm-up plus timed steps stay within about 2.5 minutes
+        per_step = min(15.0, max(0.05, 150.0 / (args.steps + args.warmup)))
+        cb = time_oracle(case, per_step, steps=args.steps, warmup=args.warmup)
+        line = {"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": cb["seconds"] * 1e3, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config, "impl": "reference",
                 "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
                 "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -224,6 +241,15 @@ def main():
         return 0
 
     import kda_gated_delta_prefill_b200 as kda
+    if args.profile_T > 0:
+        pc = gen.Case(f"profile_T{args.profile_T}", B=1, T=args.profile_T, H=64, HV=64, state="n01", seed=5)
+        x = gen.make_inputs(pc, device="cuda")
+        for _ in range(3):
+            kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"])
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": pc.name, "forwards": 3, "kernel_launches_per_forward":
+                          kda.kernel_launches(pc.B, pc.T, pc.H, pc.HV)}), flush=True)
+        return 0
     if world > 1:
         torch.cuda.set_device(local)
         from datetime import timedelta
