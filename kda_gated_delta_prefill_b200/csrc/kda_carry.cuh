@@ -33,7 +33,8 @@ struct CarrySmem {
     static constexpr int TOTAL = ABORT + 12;
 };
 
-constexpr int kCarryEpiWarps = 16;
+constexpr int kCarryEpiWarps = 16;  // 4 or 8 or 16: warps per TMEM lane quarter x 4
+static_assert(kCarryEpiWarps == 4 || kCarryEpiWarps == 8 || kCarryEpiWarps == 16, "epilogue warps");
 constexpr int kCarryThreads = (kCarryEpiWarps + 2) * 32;
 
 // TMEM column map (512 allocated): P^T (64), O^T x2 (64 each), S^T fp32 master (128), S^T fp16 (64), Vnew^T fp16 (32).
@@ -188,50 +189,64 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
         }
     } else {
         // ---------------- epilogue: value column v, key/token quarter kq ----------------
-        const int qd = warp & 3, kq = warp >> 2;
+        // Sub-block kq (0..3) = key columns 32kq..32kq+31 of the state and token columns 16kq..16kq+15; a warp
+        // owns kSub consecutive sub-blocks of its lane quarter.
+        constexpr int kSub = 16 / kCarryEpiWarps;
+        const int qd = warp & 3, kq0 = (warp >> 2) * kSub;
         const int v = 32 * qd + lane;
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
-        const uint32_t tS = tmem + lane_base + TM_S + 32 * kq;     // fp32 master S^T[v][32kq .. 32kq+31]
-        const uint32_t tA = tmem + lane_base + TA_S + 16 * kq;     // its fp16 copy (A operand)
+        auto tS = [&](int kq) { return tmem + lane_base + TM_S + 32 * kq; };  // fp32 master S^T[v][32kq .. 32kq+31]
+        auto tA = [&](int kq) { return tmem + lane_base + TA_S + 16 * kq; };  // its fp16 copy (A operand)
         const int64_t ostride = static_cast<int64_t>(p.HV) * DV;
-        // S^T[v][32kq ..] (this thread's 32 master-state values) -> fp16 A operand of the next chunk's MMAs.
-        auto publish = [&](const uint32_t (&r)[32]) {
+        // S^T[v][32kq ..] (32 master-state values) -> fp16 A operand of the next chunk's MMAs.
+        auto pack_state = [&](const uint32_t (&r)[32], int kq) {
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 uint32_t w[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     w[j] = pack_f16(__uint_as_float(r[16 * hf + 2 * j]), __uint_as_float(r[16 * hf + 2 * j + 1]));
-                tc_st8(tA + 8 * hf, w);
+                tc_st8(tA(kq) + 8 * hf, w);
             }
+        };
+        auto arrive = [&](uint32_t bar) {
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(sready);
+            if (lane == 0) mbar_arrive(bar);
         };
         bool alive = tmem_alloc == 0;
         if (alive) {
             const float *s0 = p.s0 ? p.s0 + (static_cast<int64_t>(n) * p.HV + h) * DK * DV : nullptr;
-            uint32_t r[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s0 ? s0[(32 * kq + j) * DV + v] : 0.f);
-            tc_st32(tS, r);
-            publish(r);
+            for (int i = 0; i < kSub; ++i) {
+                const int kq = kq0 + i;
+                uint32_t r[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s0 ? s0[(32 * kq + j) * DV + v] : 0.f);
+                tc_st32(tS(kq), r);
+                pack_state(r, kq);
+            }
+            arrive(sready);
         }
         // o rows of chunk c: O^T[v][tok], tok in [16*kq, 16*kq+16); a warp writes 64 contiguous bytes per token
         auto store_o = [&](int c) {
-            uint32_t orr[16];
-            tc_ld16(tmem + lane_base + TM_O0 + 64 * (c & 1) + 16 * kq, orr);
-            tc_wait_ld();
-            __nv_bfloat16 *ob = p.o + ((tok0 + static_cast<int64_t>(c) * CH + 16 * kq) * p.HV + h) * DV + v;
-            const int nrows = min(CH, len - c * CH) - 16 * kq;
-            if (nrows >= 16) {
 #pragma unroll
-                for (int t = 0; t < 16; ++t) ob[t * ostride] = __float2bfloat16_rn(__uint_as_float(orr[t]));
-            } else {
+            for (int i = 0; i < kSub; ++i) {
+                const int kq = kq0 + i;
+                uint32_t orr[16];
+                tc_ld16(tmem + lane_base + TM_O0 + 64 * (c & 1) + 16 * kq, orr);
+                tc_wait_ld();
+                __nv_bfloat16 *ob = p.o + ((tok0 + static_cast<int64_t>(c) * CH + 16 * kq) * p.HV + h) * DV + v;
+                const int nrows = min(CH, len - c * CH) - 16 * kq;
+                if (nrows >= 16) {
 #pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    if (t < nrows) ob[t * ostride] = __float2bfloat16_rn(__uint_as_float(orr[t]));
+                    for (int t = 0; t < 16; ++t) ob[t * ostride] = __float2bfloat16_rn(__uint_as_float(orr[t]));
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 16; ++t)
+                        if (t < nrows) ob[t * ostride] = __float2bfloat16_rn(__uint_as_float(orr[t]));
+                }
             }
         };
 
@@ -243,10 +258,12 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
                 fail(ERR_PIPE_FULL_WAIT);
                 break;
             }
-            {
+#pragma unroll
+            for (int i = 0; i < kSub; ++i) {
+                const int kq = kq0 + i;
                 const float2 *gl = reinterpret_cast<const float2 *>(st + ITEM_GL) + 16 * kq;
                 uint32_t r[32];
-                tc_ld32(tS, r);
+                tc_ld32(tS(kq), r);
                 tc_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
@@ -254,7 +271,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
                     r[2 * j] = __float_as_uint(x.x);
                     r[2 * j + 1] = __float_as_uint(x.y);
                 }
-                tc_st32(tS, r);
+                tc_st32(tS(kq), r);
             }
             // --- Vnew^T[v][tok] = U^T[v][tok] + P^T[v][tok], tok in [16*kq, 16*kq+16) ---
             if (!mbar_wait_spin(barP, c & 1)) {
@@ -262,7 +279,9 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
                 break;
             }
             tc_fence_after();
-            {
+#pragma unroll
+            for (int i = 0; i < kSub; ++i) {
+                const int kq = kq0 + i;
                 uint32_t pr[16];
                 tc_ld16(tmem + lane_base + TM_P + 16 * kq, pr);
                 uint4 ur[2];
@@ -282,19 +301,18 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
                     }
                 }
                 tc_st8(tmem + lane_base + TA_V + 8 * kq, w);
-                tc_wait_st();  // also covers the decayed master state
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(vready);
-                    mbar_arrive(empty0 + 8 * s);  // U and exp(G_last) of this stage are consumed
-                }
             }
+            // O of the previous chunk must be observed complete BEFORE this warp arrives on vready: after the
+            // arrival, the issuer may finish chunk c's O as well, and a parity wait on barO would then see
+            // the barrier two phases on and never return.  (O2 of chunk c-1 ran ahead of MMA1 of chunk c,
+            // so this wait normally passes at once.)
+            if (c > 0 && !mbar_wait_spin(barO, (c - 1) & 1)) {
+                fail(ERR_PIPE_FULL_WAIT);
+                break;
+            }
+            arrive(vready);  // the wait also covers the decayed master state
+            if (lane == 0) mbar_arrive(empty0 + 8 * s);  // U and exp(G_last) of this stage are consumed
             if (c > 0) {  // the previous chunk's o rows, while MMA2 runs
-                if (!mbar_wait(barO, (c - 1) & 1)) {
-                    fail(ERR_PIPE_FULL_WAIT);
-                    break;
-                }
                 tc_fence_after();
                 store_o(c - 1);
             }
@@ -304,12 +322,15 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
                 break;
             }
             tc_fence_after();
-            {
+#pragma unroll
+            for (int i = 0; i < kSub; ++i) {
+                const int kq = kq0 + i;
                 uint32_t r[32];
-                tc_ld32(tS, r);
+                tc_ld32(tS(kq), r);
                 tc_wait_ld();
-                publish(r);
+                pack_state(r, kq);
             }
+            arrive(sready);
         }
         if (nck > 0 && !*abort_flag) {
             if (mbar_wait(barO, (nck - 1) & 1)) {
@@ -321,12 +342,16 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
         }
         // final state (S^T[v][kd] -> final_state[kd][v]); skipped when the TMEM allocation was unusable
         if (tmem_alloc == 0) {
-            uint32_t r[32];
-            tc_ld32(tS, r);
-            tc_wait_ld();
             float *sN = p.sN + (static_cast<int64_t>(n) * p.HV + h) * DK * DV;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) sN[(32 * kq + j) * DV + v] = __uint_as_float(r[j]);
+            for (int i = 0; i < kSub; ++i) {
+                const int kq = kq0 + i;
+                uint32_t r[32];
+                tc_ld32(tS(kq), r);
+                tc_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sN[(32 * kq + j) * DV + v] = __uint_as_float(r[j]);
+            }
         }
     }
 

@@ -270,3 +270,25 @@ def test_parts_on_a_non_default_stream():
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
     compare(o, s, ref)
+
+
+def test_parts_repeatable_under_load():
+    # The carry of each part runs beside the next part's intra-chunk kernel.  Repeated calls must agree bit for
+    # bit with the uncut run and leave the device error word clear: a pipeline wait that gave up (for
+    # instance on a barrier that had already moved two phases on) sets a bit there and corrupts the result.
+    import kda_gated_delta_prefill_b200 as kda
+    case = gen.Case("parts_load", B=1, T=16384, H=32, HV=32, state="n01", seed=341)
+    x = gen.make_inputs(case, device="cuda")
+    assert kda.kernel_launches(1, case.T, case.H, case.HV) == 16
+    cu = torch.tensor([0, case.T], dtype=torch.int32, device="cuda")
+    o_ref, s_ref = kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"], cu)
+    torch.cuda.synchronize()
+    kda.device_error(clear=True)
+    o = torch.empty_like(o_ref)
+    s = torch.empty_like(s_ref)
+    for _ in range(12):
+        kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"], o=o, final_state=s)
+    torch.cuda.synchronize()
+    assert kda.device_error(clear=True) == 0
+    assert torch.equal(o, o_ref)
+    assert torch.equal(s, s_ref)
