@@ -27,7 +27,8 @@
 //   4. L and Aqk: bf16 tensor-core MMAs over the ten lower 16x16 block pairs
 //      (bf16 keeps the range of the gate-rescaled operands).
 //   5. A: exact float32 forward substitution in the 16x16 diagonal blocks,
-//      tf32 MMAs for the off-diagonal blocks.
+//      tf32 MMAs for the blocks next to them and then for the lower-left
+//      32x32 block as -X_B (L_C X_A).
 //   6. W and U^T: fp16 tensor-core MMAs.
 // Results go straight from registers to the item block in global memory
 // (coalesced rows), so the CTA needs about 105 KB of shared memory and two
@@ -53,7 +54,7 @@ struct IntraSmem {
     static constexpr int UST = L;        // fp16 U^T staging (step 6), once L is no longer needed
     static constexpr int BETA = 98304;   // fp32 [64]
     static constexpr int CF = 98560;     // bf16x2 [10][64] block-pair factors
-    static constexpr int PS = 101120;    // float2 [4][64] block products
+    static constexpr int PS = 101120;    // float2 [4][64] block products; later float [32][40] (over PS and TS)
     static constexpr int TS = 103168;    // fp32 8 x [16][8] solve scratch
     static constexpr int BAR = 107776;   // mbarriers: q/k/g tiles, v tile
     static constexpr int TOTAL = 107848;
@@ -421,15 +422,50 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
         }
     }
     __syncthreads();
-    {  // block forward substitution by distance from the diagonal; one warp per (block, 8-column tile)
+    {  // blocks next to the diagonal (X_10, X_21, X_32); one warp per (block, 8-column tile)
         float *ts = reinterpret_cast<float *>(sm + S::TS) + warp * 128;
         if (warp < 6) solve_block(sm + S::L, sX, sm + S::A, sbeta, ts, (warp >> 1) + 1, warp >> 1, warp & 1, lane);
         __syncthreads();
-        if (warp < 4) solve_block(sm + S::L, sX, sm + S::A, sbeta, ts, (warp >> 1) + 2, warp >> 1, warp & 1, lane);
-        __syncthreads();
-        if (warp < 2) solve_block(sm + S::L, sX, sm + S::A, sbeta, ts, 3, 0, warp & 1, lane);
-        __syncthreads();
     }
+    {  // the rest as 32x32 blocks: with X_A = X[0..31][0..31] and X_B = X[32..63][32..63] now complete,
+       // X[32..63][0..31] = -X_B (L[32..63][0..31] X_A).  Warp = 16x8 output tile, tf32 MMAs; the 16x16
+       // blocks above the diagonal of X_A and X_B are zero and skipped.
+        const int mt = warp >> 2, nt = warp & 3;
+        float *sT = reinterpret_cast<float *>(sm + S::PS);  // [32][40] floats over PS and TS
+        auto Lat = [&](int r, int cc) { return *reinterpret_cast<const float *>(sm + S::L + swz(r, cc * 4, 256)); };
+        auto Xat = [&](int r, int cc) { return *reinterpret_cast<const float *>(sX + swz(r, cc * 4, 256)); };
+        float d[4] = {};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            if (nt >= 2 && ks < 2) continue;  // X_A[0..15][16..31] = 0
+            uint32_t a[4];
+            a[0] = to_tf32(Lat(32 + 16 * mt + g8, 8 * ks + t4));
+            a[1] = to_tf32(Lat(32 + 16 * mt + g8 + 8, 8 * ks + t4));
+            a[2] = to_tf32(Lat(32 + 16 * mt + g8, 8 * ks + t4 + 4));
+            a[3] = to_tf32(Lat(32 + 16 * mt + g8 + 8, 8 * ks + t4 + 4));
+            mma_tf32(d, a, to_tf32(Xat(8 * ks + t4, 8 * nt + g8)), to_tf32(Xat(8 * ks + t4 + 4, 8 * nt + g8)));
+        }
+        *reinterpret_cast<float2 *>(sT + (16 * mt + g8) * 40 + 8 * nt + 2 * t4) = make_float2(d[0], d[1]);
+        *reinterpret_cast<float2 *>(sT + (16 * mt + g8 + 8) * 40 + 8 * nt + 2 * t4) = make_float2(d[2], d[3]);
+        __syncthreads();
+        float e[4] = {};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            if (mt == 0 && ks >= 2) continue;  // X_B[0..15][16..31] = 0
+            uint32_t a[4];
+            a[0] = to_tf32(Xat(32 + 16 * mt + g8, 32 + 8 * ks + t4));
+            a[1] = to_tf32(Xat(32 + 16 * mt + g8 + 8, 32 + 8 * ks + t4));
+            a[2] = to_tf32(Xat(32 + 16 * mt + g8, 32 + 8 * ks + t4 + 4));
+            a[3] = to_tf32(Xat(32 + 16 * mt + g8 + 8, 32 + 8 * ks + t4 + 4));
+            mma_tf32(e, a, to_tf32(sT[(8 * ks + t4) * 40 + 8 * nt + g8]), to_tf32(sT[(8 * ks + t4 + 4) * 40 + 8 * nt + g8]));
+        }
+        // only A = X diag(beta) is needed from here on
+        const int cc = 8 * nt + 2 * t4;
+        const float b0 = sbeta[cc], b1 = sbeta[cc + 1];
+        *reinterpret_cast<uint32_t *>(sm + S::A + swz(32 + 16 * mt + g8, cc * 2, 128)) = pack_f16(-e[0] * b0, -e[1] * b1);
+        *reinterpret_cast<uint32_t *>(sm + S::A + swz(32 + 16 * mt + g8 + 8, cc * 2, 128)) = pack_f16(-e[2] * b0, -e[3] * b1);
+    }
+    __syncthreads();
 
     // ---- v tile (its copy overlapped steps 2-5): zero padding rows, bf16 -> fp16 in place ----
     if (!mbar_wait(bar + 8, 0)) {
