@@ -53,6 +53,18 @@ struct CarryParams {
     int chunks_per_seq;
     int chunk_begin;           // cu null: this launch carries chunks [chunk_begin, chunk_begin + chunk_count)
     int chunk_count;           //   of every sequence, from s0 (cu given: whole sequences, chunk_begin = 0)
+    // Segmented carry of plain batches (seg_phase != 0): the chunks of every sequence are split into seg_count
+    // segments [nck*p/seg_count, nck*(p+1)/seg_count), unit = (sequence, value head) = blockIdx % units.
+    //  seg_phase 1, j = blockIdx / units: j = 0 carries segment 0 from s0 and stores its end state, which is the
+    //    start of segment 1, in seg_S[unit][1]; j = 2p-1 carries segment p from zero into seg_B[unit][p]; j = 2p
+    //    carries segment p from the identity with U taken as zero (the segment's linear map) into seg_M[unit][p].
+    //    No o is written.
+    //    CTA j = 0 also copies the initial state (s0, or zeros) into seg_S[unit][0].
+    //  seg_phase 2, p = blockIdx / units: segment p from seg_S[unit][p], writing o; the last segment writes sN
+    //    (which may be the buffer s0 points to).
+    int seg_phase;
+    int seg_count;
+    float *seg_S, *seg_M, *seg_B;  // [units][seg_count][K][V]
 };
 
 __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const CarryParams p)
@@ -62,11 +74,48 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    const int h = blockIdx.x % p.HV;
-    const int n = p.order ? p.order[blockIdx.x / p.HV] : blockIdx.x / p.HV;
+    int h = blockIdx.x % p.HV;
+    int n = p.order ? p.order[blockIdx.x / p.HV] : blockIdx.x / p.HV;
     int64_t c_begin, tok0;
     int nck, len;
-    if (p.cu) {
+    // where the state starts and ends, and what the chunk loop produces
+    enum { FROM_S0, FROM_ZERO, FROM_IDENTITY };
+    int from = FROM_S0;
+    const float *s_in = p.s0 ? p.s0 + (static_cast<int64_t>(n) * p.HV + h) * DK * DV : nullptr;
+    float *s_out = p.sN + (static_cast<int64_t>(n) * p.HV + h) * DK * DV;
+    float *s_copy = nullptr;  // where the initial state is also stored (segmented first pass only)
+    bool with_o = true, homogeneous = false;
+    if (p.seg_phase != 0) {
+        const int units = p.N * p.HV, unit = blockIdx.x % units, j = blockIdx.x / units;
+        n = unit / p.HV;
+        h = unit % p.HV;
+        const int seg = p.seg_phase == 1 ? (j + 1) / 2 : j;
+        const int cb = static_cast<int>(static_cast<int64_t>(p.chunks_per_seq) * seg / p.seg_count);
+        const int ce = static_cast<int>(static_cast<int64_t>(p.chunks_per_seq) * (seg + 1) / p.seg_count);
+        c_begin = static_cast<int64_t>(n) * p.chunks_per_seq + cb;
+        nck = ce - cb;
+        tok0 = static_cast<int64_t>(n) * p.T + static_cast<int64_t>(cb) * CH;
+        len = p.T - cb * CH;
+        const int64_t slot = (static_cast<int64_t>(unit) * p.seg_count + seg) * DK * DV;
+        s_in = p.s0 ? p.s0 + (static_cast<int64_t>(n) * p.HV + h) * DK * DV : nullptr;
+        if (p.seg_phase == 1) {
+            with_o = false;
+            if (j == 0) {  // also keeps a copy of the initial state for the second pass (final_state may alias it)
+                s_copy = p.seg_S + slot;
+                s_out = p.seg_S + (static_cast<int64_t>(unit) * p.seg_count + 1) * DK * DV;
+            } else if (j & 1) {
+                from = FROM_ZERO;
+                s_out = p.seg_B + slot;
+            } else {
+                from = FROM_IDENTITY;
+                homogeneous = true;
+                s_out = p.seg_M + slot;
+            }
+        } else {
+            s_in = p.seg_S + slot;
+            s_out = seg + 1 == p.seg_count ? p.sN + (static_cast<int64_t>(n) * p.HV + h) * DK * DV : nullptr;
+        }
+    } else if (p.cu) {
         c_begin = p.chunk_off[n];
         nck = p.chunk_off[n + 1] - p.chunk_off[n];
         tok0 = p.cu[n];
@@ -155,10 +204,12 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
                                dbase(so + (ITEM_WN >> 4) + (ks >> 2) * 512 + (ks & 3) * 2), i64, ks > 0);
             tc_commit_warp(barP);
             // O^T = S^T Qg^T
+            if (with_o) {
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                tc_mma_ts_warp(tmo, tmem + TA_S + 8 * ks, dbase(so + (ITEM_QG >> 4) + (ks >> 2) * 512 + (ks & 3) * 2),
-                               i64, ks > 0);
+                for (int ks = 0; ks < 8; ++ks)
+                    tc_mma_ts_warp(tmo, tmem + TA_S + 8 * ks,
+                                   dbase(so + (ITEM_QG >> 4) + (ks >> 2) * 512 + (ks & 3) * 2), i64, ks > 0);
+            }
             if (!__all_sync(0xffffffffu, mbar_wait_spin(vready, c & 1))) return false;
             tc_fence_after();
             // S^T += Vnew^T Kg onto the decayed master state (on the chain to the next chunk, so first).
@@ -168,10 +219,12 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
                 tc_mma_ts_warp(tmem + TM_S, tmem + TA_V + 8 * ks, kbase(so + (ITEM_KG >> 4) + ks * 128), i128mn, 1);
             tc_commit_warp(barS);
             // O^T += Vnew^T Aqk^T (K = 64 tokens)
+            if (with_o) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                tc_mma_ts_warp(tmo, tmem + TA_V + 8 * ks, dbase(so + (ITEM_AQK >> 4) + ks * 2), i64, 1);
-            tc_commit_warp(barO);
+                for (int ks = 0; ks < 4; ++ks)
+                    tc_mma_ts_warp(tmo, tmem + TA_V + 8 * ks, dbase(so + (ITEM_AQK >> 4) + ks * 2), i64, 1);
+                tc_commit_warp(barO);
+            }
             tc_commit_warp(empty0 + 8 * st);
             return true;
         };
@@ -217,13 +270,19 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
         };
         bool alive = tmem_alloc == 0;
         if (alive) {
-            const float *s0 = p.s0 ? p.s0 + (static_cast<int64_t>(n) * p.HV + h) * DK * DV : nullptr;
+            const float *s0 = from == FROM_S0 ? s_in : nullptr;
 #pragma unroll
             for (int i = 0; i < kSub; ++i) {
                 const int kq = kq0 + i;
                 uint32_t r[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(s0 ? s0[(32 * kq + j) * DV + v] : 0.f);
+                for (int j = 0; j < 32; ++j)
+                    r[j] = __float_as_uint(s0 ? s0[(32 * kq + j) * DV + v]
+                                              : (from == FROM_IDENTITY && 32 * kq + j == v ? 1.f : 0.f));
+                if (s_copy) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) s_copy[(32 * kq + j) * DV + v] = __uint_as_float(r[j]);
+                }
                 tc_st32(tS(kq), r);
                 pack_state(r, kq);
             }
@@ -296,7 +355,8 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int t = 8 * q + 2 * e;
-                        const float2 x = add2(unpack_f16(uw[e]), make_float2(__uint_as_float(pr[t]), __uint_as_float(pr[t + 1])));
+                        const float2 pv = make_float2(__uint_as_float(pr[t]), __uint_as_float(pr[t + 1]));
+                        const float2 x = homogeneous ? pv : add2(unpack_f16(uw[e]), pv);
                         w[4 * q + e] = pack_f16(x.x, x.y);
                     }
                 }
@@ -306,13 +366,13 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
             // arrival, the issuer may finish chunk c's O as well, and a parity wait on barO would then see
             // the barrier two phases on and never return.  (O2 of chunk c-1 ran ahead of MMA1 of chunk c,
             // so this wait normally passes at once.)
-            if (c > 0 && !mbar_wait_spin(barO, (c - 1) & 1)) {
+            if (with_o && c > 0 && !mbar_wait_spin(barO, (c - 1) & 1)) {
                 fail(ERR_PIPE_FULL_WAIT);
                 break;
             }
             arrive(vready);  // the wait also covers the decayed master state
             if (lane == 0) mbar_arrive(empty0 + 8 * s);  // U and exp(G_last) of this stage are consumed
-            if (c > 0) {  // the previous chunk's o rows, while MMA2 runs
+            if (with_o && c > 0) {  // the previous chunk's o rows, while MMA2 runs
                 tc_fence_after();
                 store_o(c - 1);
             }
@@ -332,7 +392,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
             }
             arrive(sready);
         }
-        if (nck > 0 && !*abort_flag) {
+        if (with_o && nck > 0 && !*abort_flag) {
             if (mbar_wait(barO, (nck - 1) & 1)) {
                 tc_fence_after();
                 store_o(nck - 1);
@@ -341,8 +401,8 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
             }
         }
         // final state (S^T[v][kd] -> final_state[kd][v]); skipped when the TMEM allocation was unusable
-        if (tmem_alloc == 0) {
-            float *sN = p.sN + (static_cast<int64_t>(n) * p.HV + h) * DK * DV;
+        if (tmem_alloc == 0 && s_out) {
+            float *sN = s_out;
 #pragma unroll
             for (int i = 0; i < kSub; ++i) {
                 const int kq = kq0 + i;

@@ -16,6 +16,7 @@
 #include "kda_intra.cuh"
 #include "kda_norm.cuh"
 #include "kda_prefill.h"
+#include "kda_scan.cuh"
 #include "kda_sched.cuh"
 
 // Bits set by kernels whose bounded waits gave up (see ptx.cuh).  Host code
@@ -123,9 +124,25 @@ kda_status_t check_dims(int B, int T, int H, int HV, int K, int V, bool varlen, 
 }
 
 // Workspace: [chunk_off (N+1) | order (N)] for packed batches, then the item blocks.
+// Plain batches with few (sequence, value head) units and long sequences: one carry CTA per unit would run far
+// longer than everything else, so the carry runs on segments of every sequence at once (segment maps, a scan
+// of the start states, then the segments with outputs).  The count keeps the first pass, two CTAs per segment
+// and unit, within about 128 CTAs, and every segment at 16 chunks or more; it does not depend on the device,
+// so the workspace size does not either.  Returns 1 (no segments) below 3.
+int carry_segments(int B, int T, int HV, bool varlen)
+{
+    if (varlen) return 1;
+    const int64_t units = static_cast<int64_t>(B) * HV;
+    const int64_t by_ctas = 128 / (2 * units + 1);
+    const int64_t by_len = ((static_cast<int64_t>(T) + CH - 1) / CH) / 16;
+    const int64_t segs = by_ctas < by_len ? by_ctas : by_len;
+    return segs >= 3 ? static_cast<int>(segs) : 1;
+}
+
 struct Workspace {
-    size_t chunk_off = 0, order = 0, items = 0, total = 0;
+    size_t chunk_off = 0, order = 0, items = 0, seg = 0, total = 0;
     int64_t max_chunks = 0;
+    int segments = 1;
 };
 
 Workspace workspace_layout(int B, int T, int HV, int num_seqs)
@@ -143,6 +160,12 @@ Workspace workspace_layout(int B, int T, int HV, int num_seqs)
     }
     w.items = off;
     off += static_cast<size_t>(w.max_chunks) * HV * kda::ITEM_BYTES;
+    w.segments = carry_segments(B, T, HV, varlen);
+    if (w.segments > 1) {  // start states, maps and zero-start images: 3 x units x segments fp32 [K][V]
+        off = round_up(off, kAlign);
+        w.seg = off;
+        off += 3 * static_cast<size_t>(B) * HV * w.segments * DK * DV * sizeof(float);
+    }
     w.total = round_up(off, kAlign);
     return w;
 }
@@ -232,6 +255,7 @@ extern "C" int kda_prefill_kernel_launches(int B, int T, int H, int HV, int K, i
     DeviceInfo info;
     if (device_info(info) != cudaSuccess) return 0;
     if (varlen) return 2 + (T > 0 ? 1 : 0) + 1;  // chunk offsets, order, intra (if any token), carry
+    if (carry_segments(B, T, HV, false) > 1) return 4;  // intra, segment maps, scan, segments with outputs
     return 2 * pipeline_parts(B, T, HV, false, info.sms);
 }
 
@@ -345,6 +369,23 @@ extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const 
     cp.N = d.N;
     cp.chunks_per_seq = (T + CH - 1) / CH;
 
+    if (ws.segments > 1) {
+        if (launch_intra(0, cp.chunks_per_seq, ws.max_chunks) != cudaSuccess) return KDA_ERR_CUDA;
+        const int units = d.N * HV;
+        float *seg = reinterpret_cast<float *>(wsb + ws.seg);
+        const size_t per = static_cast<size_t>(units) * ws.segments * DK * DV;
+        cp.seg_count = ws.segments;
+        cp.seg_S = seg;
+        cp.seg_M = seg + per;
+        cp.seg_B = seg + 2 * per;
+        cp.seg_phase = 1;
+        if (launch_carry(cp, units * (2 * ws.segments - 1), s) != cudaSuccess) return KDA_ERR_CUDA;
+        kda::kda_seg_scan_kernel<<<units * kda::kScanCtasPerUnit, 256, 0, s>>>(cp.seg_S, cp.seg_M, cp.seg_B,
+                                                                             ws.segments);
+        if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+        cp.seg_phase = 2;
+        return launch_carry(cp, units * ws.segments, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
     const int parts = pipeline_parts(B, T, HV, varlen, info.sms);
     if (parts == 1) {
         if (tokens > 0 && launch_intra(0, cp.chunks_per_seq, ws.max_chunks) != cudaSuccess) return KDA_ERR_CUDA;

@@ -226,7 +226,8 @@ def test_repeat_calls_are_deterministic():
 
 @pytest.mark.parametrize("T,state", [(2088, "n01"), (5120, "none"), (8209, "n01")])
 def test_parts_full_parity(T, state):
-    case = gen.Case(f"parts{T}", B=1, T=T, H=2, HV=2, state=state, seed=300 + T)
+    # 24 value heads (GQA groups of 3): enough units that the carry is overlapped rather than segmented
+    case = gen.Case(f"parts{T}", B=1, T=T, H=8, HV=24, state=state, seed=300 + T)
     x = gen.make_inputs(case)
     o, s = gpu_forward(x)
     compare(o, s, oracle_forward(x))
@@ -234,7 +235,7 @@ def test_parts_full_parity(T, state):
 
 def test_parts_match_the_uncut_run_bit_for_bit():
     # The same sequence passed as a packed batch of one sequence takes the uncut path.
-    case = gen.Case("parts_vs_uncut", B=1, T=4160, H=2, HV=4, state="n01", seed=311)
+    case = gen.Case("parts_vs_uncut", B=1, T=4160, H=8, HV=32, state="n01", seed=311)
     x = gen.make_inputs(case)
     o_cut, s_cut = gpu_forward(x)
     xv = dict(x)
@@ -292,3 +293,48 @@ def test_parts_repeatable_under_load():
     assert kda.device_error(clear=True) == 0
     assert torch.equal(o, o_ref)
     assert torch.equal(s, s_ref)
+
+
+
+# ------------------------------------------------------------------ segmented carry
+# A plain batch with few (sequence, value head) units and long sequences carries segments of every sequence
+# at once: per segment its linear map and its image of zero, a scan of the segment start states, then all
+# segments with outputs.  The results follow the same recurrence with different rounding, so they are compared
+# with the oracle at the usual tolerances.
+
+@pytest.mark.parametrize("B,T,H,HV,state", [(1, 5120, 2, 2, "none"), (1, 8209, 2, 2, "n01"), (2, 4096, 1, 1, "n01"),
+                                            (1, 6000, 1, 2, "n01")])
+def test_segmented_full_parity(B, T, H, HV, state):
+    import kda_gated_delta_prefill_b200 as kda
+    case = gen.Case(f"seg{T}", B=B, T=T, H=H, HV=HV, state=state, seed=400 + T + HV)
+    assert kda.kernel_launches(B, T, H, HV) == 4
+    x = gen.make_inputs(case)
+    o, s = gpu_forward(x)
+    compare(o, s, oracle_forward(x))
+
+
+def test_segmented_in_place_state_update():
+    case = gen.Case("seg_inplace", B=1, T=5120, H=2, HV=2, state="n01", seed=431)
+    x = gen.make_inputs(case)
+    ref = oracle_forward(x)
+    xc = to_cuda(x)
+    import kda_gated_delta_prefill_b200 as kda
+    st = xc["initial_state"].clone()
+    o, s = kda.forward(xc["q"], xc["k"], xc["v"], xc["g"], xc["beta"], st, final_state=st)
+    torch.cuda.synchronize()
+    assert s.data_ptr() == st.data_ptr()
+    assert kda.device_error(clear=True) == 0
+    compare(o, s, ref)
+
+
+def test_segmented_long_few_heads_sampled():
+    # B=1, H=HV=4, T=65536 (14 segments per unit); the oracle checks one head.
+    import kda_gated_delta_prefill_b200 as kda
+    case = gen.Case("seg_long", B=1, T=65536, H=4, HV=4, state="n01", seed=441)
+    x = gen.make_inputs(case, device="cuda")
+    o, s = kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"])
+    torch.cuda.synchronize()
+    assert kda.device_error(clear=True) == 0
+    xc = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    sub = select_heads(xc, [3])
+    compare(o[:, :, [3]].contiguous(), s[:, [3]].contiguous(), oracle_forward(sub))
