@@ -107,12 +107,14 @@ size_t kda_prefill_workspace_size(int B, int T, int H, int HV, int K, int V, int
  * captured graph).  Calls from several host threads on one device share that
  * side stream, so their carry parts run one after another.
  *
- * A plain batch with few units and long sequences (the workspace rule:
- * S = min(128 / (2 B HV + 1), ceil(T/64) / 16) segments, used when S >= 3)
- * instead carries S segments of every sequence at once: the segments' linear
+ * A plain batch with few units (B * HV <= 48) and long sequences may
+ * instead carry S segments of every sequence at once: the segments' linear
  * maps and images of zero, a scan of their start states, then all segments
- * with outputs (4 launches in all, on `stream`).  Its results follow the same
- * recurrence with a different rounding order.
+ * with outputs (4 launches in all, on `stream`).  The workspace reserves
+ * room for S up to min(1024 / (2 B HV + 1), ceil(T/64) / 16); the forward
+ * picks S on the device when its cost model says the segments are faster
+ * than the overlapped carry.  The results follow the same recurrence with a
+ * different rounding order.
  */
 kda_status_t kda_prefill_forward(const void *q, const void *k, const void *v,
                                  const float *g, const float *beta,

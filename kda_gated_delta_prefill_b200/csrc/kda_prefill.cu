@@ -125,18 +125,44 @@ kda_status_t check_dims(int B, int T, int H, int HV, int K, int V, bool varlen, 
 
 // Workspace: [chunk_off (N+1) | order (N)] for packed batches, then the item blocks.
 // Plain batches with few (sequence, value head) units and long sequences: one carry CTA per unit would run far
-// longer than everything else, so the carry runs on segments of every sequence at once (segment maps, a scan
-// of the start states, then the segments with outputs).  The count keeps the first pass, two CTAs per segment
-// and unit, within about 128 CTAs, and every segment at 16 chunks or more; it does not depend on the device,
-// so the workspace size does not either.  Returns 1 (no segments) below 3.
-int carry_segments(int B, int T, int HV, bool varlen)
+// longer than everything else, so the carry can run on segments of every sequence at once (segment maps, a
+// scan of the start states, then the segments with outputs).  The workspace reserves room for up to
+// max_carry_segments segments (a bound that does not depend on the device: segments of 16 chunks or more, at
+// most 1024 first-pass CTAs, units <= 48); the forward picks the count on the device.
+int max_carry_segments(int B, int T, int HV, bool varlen)
 {
-    if (varlen) return 1;
     const int64_t units = static_cast<int64_t>(B) * HV;
-    const int64_t by_ctas = 128 / (2 * units + 1);
+    if (varlen || units > 48) return 1;
+    const int64_t by_ctas = 1024 / (2 * units + 1);
     const int64_t by_len = ((static_cast<int64_t>(T) + CH - 1) / CH) / 16;
     const int64_t segs = by_ctas < by_len ? by_ctas : by_len;
     return segs >= 3 ? static_cast<int>(segs) : 1;
+}
+
+// Segment count for this device, from a cost model in carry chunk periods fitted to measurements on B200
+// (intra-chunk work of one (chunk, head) item is about 1/32 of a period):
+//   segmented = intra + (waves of the first pass + waves of the second) x (chunks per segment + 3) + 4 per
+//               scan step (the +3: pipeline fill and the state's load and store in each pass),
+//   otherwise = max(5/4 carry + intra / 4, 27/20 intra) (the carry overlapping the intra-chunk work).
+// Picks the cheapest count, and segments only when that is under 90 % of the alternative.  1 = no segments.
+int carry_segments(int B, int T, int HV, bool varlen, int sms)
+{
+    const int smax = max_carry_segments(B, T, HV, varlen);
+    if (smax < 3) return 1;
+    const int64_t units = static_cast<int64_t>(B) * HV, nck = (static_cast<int64_t>(T) + CH - 1) / CH;
+    const int64_t intra = units * nck / 32;
+    const int64_t a = 5 * nck / 4 + intra / 4, b = 27 * intra / 20;
+    int best = 1;
+    int64_t best_cost = (a > b ? a : b) * 9 / 10;
+    for (int sg = 3; sg <= smax; ++sg) {
+        const int64_t w1 = (units * (2 * sg - 1) + sms - 1) / sms, w2 = (units * sg + sms - 1) / sms;
+        const int64_t cost = intra + (w1 + w2) * ((nck + sg - 1) / sg + 3) + 4 * sg;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = sg;
+        }
+    }
+    return best;
 }
 
 struct Workspace {
@@ -160,7 +186,7 @@ Workspace workspace_layout(int B, int T, int HV, int num_seqs)
     }
     w.items = off;
     off += static_cast<size_t>(w.max_chunks) * HV * kda::ITEM_BYTES;
-    w.segments = carry_segments(B, T, HV, varlen);
+    w.segments = max_carry_segments(B, T, HV, varlen);
     if (w.segments > 1) {  // start states, maps and zero-start images: 3 x units x segments fp32 [K][V]
         off = round_up(off, kAlign);
         w.seg = off;
@@ -255,7 +281,7 @@ extern "C" int kda_prefill_kernel_launches(int B, int T, int H, int HV, int K, i
     DeviceInfo info;
     if (device_info(info) != cudaSuccess) return 0;
     if (varlen) return 2 + (T > 0 ? 1 : 0) + 1;  // chunk offsets, order, intra (if any token), carry
-    if (carry_segments(B, T, HV, false) > 1) return 4;  // intra, segment maps, scan, segments with outputs
+    if (carry_segments(B, T, HV, false, info.sms) > 1) return 4;  // intra, segment maps, scan, segments with outputs
     return 2 * pipeline_parts(B, T, HV, false, info.sms);
 }
 
@@ -369,22 +395,23 @@ extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const 
     cp.N = d.N;
     cp.chunks_per_seq = (T + CH - 1) / CH;
 
-    if (ws.segments > 1) {
+    const int segments = ws.segments > 1 ? carry_segments(B, T, HV, varlen, info.sms) : 1;
+    if (segments > 1) {
         if (launch_intra(0, cp.chunks_per_seq, ws.max_chunks) != cudaSuccess) return KDA_ERR_CUDA;
         const int units = d.N * HV;
         float *seg = reinterpret_cast<float *>(wsb + ws.seg);
-        const size_t per = static_cast<size_t>(units) * ws.segments * DK * DV;
-        cp.seg_count = ws.segments;
+        const size_t per = static_cast<size_t>(units) * ws.segments * DK * DV;  // reserved for the maximum count
+        cp.seg_count = segments;
         cp.seg_S = seg;
         cp.seg_M = seg + per;
         cp.seg_B = seg + 2 * per;
         cp.seg_phase = 1;
-        if (launch_carry(cp, units * (2 * ws.segments - 1), s) != cudaSuccess) return KDA_ERR_CUDA;
+        if (launch_carry(cp, units * (2 * segments - 1), s) != cudaSuccess) return KDA_ERR_CUDA;
         kda::kda_seg_scan_kernel<<<units * kda::kScanCtasPerUnit, 256, 0, s>>>(cp.seg_S, cp.seg_M, cp.seg_B,
-                                                                             ws.segments);
+                                                                             segments);
         if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
         cp.seg_phase = 2;
-        return launch_carry(cp, units * ws.segments, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+        return launch_carry(cp, units * segments, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     }
     const int parts = pipeline_parts(B, T, HV, varlen, info.sms);
     if (parts == 1) {
