@@ -70,7 +70,9 @@ const char *kda_status_string(kda_status_t status);
  * for a plain [B, T] batch.  The workspace holds, per (64-token chunk, value
  * head), the chunk's state-independent results that the intra-chunk kernel
  * hands to the carry kernel (72.5 KiB each), plus the chunk offsets and the
- * longest-first order of packed sequences.  Returns 0 for sizes that
+ * longest-first order of packed sequences, and, for plain batches of few long
+ * sequences, room for the segmented carry's states (3 x B x HV x S x 64 KiB,
+ * S as described at kda_prefill_forward).  Returns 0 for sizes that
  * kda_prefill_forward would reject.
  */
 size_t kda_prefill_workspace_size(int B, int T, int H, int HV, int K, int V, int num_seqs);
