@@ -193,6 +193,37 @@ kda_status_t kda_prefill_device_error(unsigned *word, int clear);
 int kda_prefill_kernel_launches(int B, int T, int H, int HV, int K, int V, int num_seqs);
 
 /*
+ * One recurrent decode step (one token per row) on a caller-owned bf16 state
+ * pool, as on the "flashinfer.kda_decode.packed_kda_decode" page, with the
+ * recurrence of "KDA Chunk Prefill on Ascend A3" (section "Mathematical
+ * definition") for T = 1.  The page's gate and beta activations (its
+ * lower-bound gate formula is not given there) are the caller's: g and beta
+ * arrive activated, as in kda_prefill_forward.
+ *
+ *   q, k          bf16, row b at q + b * q_row_stride: [H, K]; rows 8-byte
+ *                 aligned, strides multiples of 4 elements (a packed QKV row
+ *                 [q | k | v] is passed as three pointers with one stride)
+ *   v             bf16, row b at v + b * v_row_stride: [HV, V]
+ *   g             fp32 [B, HV, K]  natural-log gates, <= 0
+ *   beta          fp32 [B, HV]
+ *   state         bf16 pool of num_slots slots; slot s at state +
+ *                 s * slot_stride elements holds [HV, K, V] (compact inside;
+ *                 slot_stride >= HV*K*V, a multiple of 8); 16-byte aligned.
+ *                 Updated in place: slot <- bf16 (nearest even) of the new
+ *                 state computed in fp32.
+ *   state_indices int32 [B] device: the slot of each row, or -1 for a padding
+ *                 row, whose output is zeros and which touches no state.
+ *                 Active indices must be unique and < num_slots (device
+ *                 values, not checked).
+ *   o             bf16 [B, HV, V] out, overlapping no other argument.
+ * B = 0 is a no-op.  K = V = 128.  Asynchronous on `stream`.
+ */
+kda_status_t kda_decode_step(const void *q, int64_t q_row_stride, const void *k, int64_t k_row_stride,
+                             const void *v, int64_t v_row_stride, const float *g, const float *beta,
+                             void *state, int64_t slot_stride, int num_slots, const int32_t *state_indices,
+                             int B, int H, int HV, int K, int V, void *o, void *stream);
+
+/*
  * Step 1 alone: L2-normalise `rows` rows of K bf16 values with the exact
  * rounding order above ("KDA Chunk Prefill on Ascend A3", section
  * "Mathematical definition", first formula).  x and out: bf16 [rows, K],

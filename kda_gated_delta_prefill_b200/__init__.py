@@ -27,7 +27,7 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 
 EXPORTED = ("kda_status_string", "kda_prefill_workspace_size", "kda_prefill_forward",
             "kda_prefill_host_staging_size", "kda_prefill_forward_host", "kda_prefill_device_error",
-            "kda_l2norm_bf16", "kda_prefill_kernel_launches")
+            "kda_l2norm_bf16", "kda_prefill_kernel_launches", "kda_decode_step")
 
 
 class KdaError(RuntimeError):
@@ -67,6 +67,8 @@ def lib():
         L.kda_l2norm_bf16.restype = I
         L.kda_prefill_kernel_launches.argtypes = [I] * 7
         L.kda_prefill_kernel_launches.restype = I
+        L.kda_decode_step.argtypes = [P, I64, P, I64, P, I64, P, P, P, I64, I, P, I, I, I, I, I, P, P]
+        L.kda_decode_step.restype = I
         _lib = L
         return L
 
@@ -152,6 +154,32 @@ def device_error(clear: bool = True) -> int:
     w = ctypes.c_uint(0)
     _check(lib().kda_prefill_device_error(ctypes.byref(w), int(clear)), "kda_prefill_device_error")
     return int(w.value)
+
+
+def decode_step(q, k, v, g, beta, state, state_indices, *, o=None, stream=None):
+    """One recurrent decode step on a bf16 state pool (CUDA); returns o [B, HV, V].
+
+    q, k: bf16 [B, H, K] and v: bf16 [B, HV, V], each row compact but rows may be strided (e.g. views of a
+    packed [B, (2H + HV) * 128] QKV tensor); g: fp32 [B, HV, K]; beta: fp32 [B, HV]; state: bf16 pool
+    [num_slots, HV, K, V] (compact inside a slot), updated in place; state_indices: int32 [B], -1 = padding row.
+    """
+    import torch
+    B, H, K = q.shape
+    HV, V = v.shape[1], v.shape[2]
+    for name, t, inner in (("q", q, H * K), ("k", k, H * K), ("v", v, HV * V)):
+        if not t.is_cuda or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError(f"{name} must be a CUDA tensor with compact rows")
+    for name, t in (("g", g), ("beta", beta), ("state_indices", state_indices)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if not state.is_cuda or state[0].stride() != (K * V, V, 1):
+        raise ValueError("state must be a CUDA pool [num_slots, HV, K, V] compact inside each slot")
+    if o is None:
+        o = torch.empty(B, HV, V, dtype=torch.bfloat16, device=q.device)
+    _check(lib().kda_decode_step(_ptr(q), q.stride(0), _ptr(k), k.stride(0), _ptr(v), v.stride(0), _ptr(g),
+                                 _ptr(beta), _ptr(state), state.stride(0), state.shape[0], _ptr(state_indices),
+                                 B, H, HV, K, V, _ptr(o), _stream_ptr(stream)), "kda_decode_step")
+    return o
 
 
 def l2norm_bf16(x, out=None, stream=None):

@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "kda_carry.cuh"
+#include "kda_decode.cuh"
 #include "kda_intra.cuh"
 #include "kda_norm.cuh"
 #include "kda_prefill.h"
@@ -511,6 +512,55 @@ extern "C" kda_status_t kda_prefill_forward_host(const void *q_h, const void *k_
     if (nvb && cudaMemcpyAsync(o_h, dO, nvb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return KDA_ERR_CUDA;
     if (cudaMemcpyAsync(sN_h, dsN, ns, cudaMemcpyDeviceToHost, s) != cudaSuccess) return KDA_ERR_CUDA;
     return KDA_OK;
+}
+
+extern "C" kda_status_t kda_decode_step(const void *q, int64_t q_row_stride, const void *k, int64_t k_row_stride,
+                                        const void *v, int64_t v_row_stride, const float *g, const float *beta,
+                                        void *state, int64_t slot_stride, int num_slots, const int32_t *state_indices,
+                                        int B, int H, int HV, int K, int V, void *o, void *stream)
+{
+    if (B < 0 || H <= 0 || HV <= 0 || num_slots <= 0 || HV % H != 0) return KDA_ERR_INVALID_ARG;
+    if (K != DK || V != DV) return KDA_ERR_UNSUPPORTED;
+    if (B == 0) return KDA_OK;
+    if (static_cast<int64_t>(B) * HV > INT_MAX) return KDA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !g || !beta || !state || !state_indices || !o) return KDA_ERR_INVALID_ARG;
+    if (q_row_stride < static_cast<int64_t>(H) * K || k_row_stride < static_cast<int64_t>(H) * K ||
+        v_row_stride < static_cast<int64_t>(HV) * V || slot_stride < static_cast<int64_t>(HV) * K * V)
+        return KDA_ERR_INVALID_ARG;
+    if (!aligned(q, 8) || !aligned(k, 8) || !aligned(v, 2) || !aligned(g, 4) || !aligned(beta, 4) ||
+        !aligned(state, 16) || !aligned(state_indices, 4) || !aligned(o, 4) || q_row_stride % 4 || k_row_stride % 4 ||
+        slot_stride % 8)
+        return KDA_ERR_MISALIGNED;
+    const size_t nq = static_cast<size_t>(B - 1) * q_row_stride * 2 + static_cast<size_t>(H) * K * 2;
+    const size_t nk = static_cast<size_t>(B - 1) * k_row_stride * 2 + static_cast<size_t>(H) * K * 2;
+    const size_t nv = static_cast<size_t>(B - 1) * v_row_stride * 2 + static_cast<size_t>(HV) * V * 2;
+    const size_t ng = static_cast<size_t>(B) * HV * K * 4, nb = static_cast<size_t>(B) * HV * 4;
+    const size_t ns = static_cast<size_t>(num_slots - 1) * slot_stride * 2 + static_cast<size_t>(HV) * K * V * 2;
+    const size_t no = static_cast<size_t>(B) * HV * V * 2, ni = static_cast<size_t>(B) * 4;
+    // o overlaps nothing; the pool overlaps no input
+    const void *ins[] = {q, k, v, g, beta, state_indices};
+    const size_t in_n[] = {nq, nk, nv, ng, nb, ni};
+    for (int i = 0; i < 6; ++i)
+        if (overlaps(o, no, ins[i], in_n[i]) || overlaps(state, ns, ins[i], in_n[i])) return KDA_ERR_INVALID_ARG;
+    if (overlaps(o, no, state, ns)) return KDA_ERR_INVALID_ARG;
+
+    kda::DecodeParams dp{};
+    dp.q = static_cast<const __nv_bfloat16 *>(q);
+    dp.k = static_cast<const __nv_bfloat16 *>(k);
+    dp.v = static_cast<const __nv_bfloat16 *>(v);
+    dp.q_stride = q_row_stride;
+    dp.k_stride = k_row_stride;
+    dp.v_stride = v_row_stride;
+    dp.g = g;
+    dp.beta = beta;
+    dp.state = static_cast<__nv_bfloat16 *>(state);
+    dp.slot_stride = slot_stride;
+    dp.state_indices = state_indices;
+    dp.o = static_cast<__nv_bfloat16 *>(o);
+    dp.H = H;
+    dp.HV = HV;
+    kda::kda_decode_kernel<<<B * HV, kda::kDecodeThreads, 0, static_cast<cudaStream_t>(stream)>>>(dp);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 extern "C" kda_status_t kda_l2norm_bf16(const void *x, int64_t rows, int K, void *out, void *stream)

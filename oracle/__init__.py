@@ -169,3 +169,35 @@ def forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, return_normal
     if return_normalized:
         out["qn"], out["kn"] = qn, kn
     return out
+
+
+def decode_step(q, k, v, g, beta, state, state_indices):
+    """One recurrent decode step per row on a state pool ("flashinfer.kda_decode.packed_kda_decode" page; the
+    recurrence of "KDA Chunk Prefill on Ascend A3", section "Mathematical definition", for one token).
+
+    q, k [B,H,K] and v [B,HV,V] (bf16 values), g [B,HV,K], beta [B,HV] (float32 values), state [N,HV,K,V]
+    (the pool's values, e.g. bf16 held in float32), state_indices [B] (slot per row, -1 = padding row).
+    Returns (o [B,HV,V] float64, zero on padding rows; new_state [N,HV,K,V] float64, where the slots of the
+    active rows hold the updated state before any rounding and the other slots are unchanged).
+    """
+    qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
+    gf, bf = _f32(g), _f32(beta)
+    pool = np.array(state.float().cpu().numpy() if hasattr(state, "cpu") else state, dtype=np.float64)
+    idx = np.asarray(state_indices.cpu() if hasattr(state_indices, "cpu") else state_indices).astype(np.int64)
+    B, H, K = qb.shape
+    HV, V = vb.shape[1], vb.shape[2]
+    o = np.zeros((B, HV, V), np.float64)
+    rows = np.nonzero(idx >= 0)[0]
+    if len(rows) == 0:
+        return o, pool
+    # the active rows as a batch of one-token sequences, each starting from its slot
+    s0 = np.ascontiguousarray(pool[idx[rows]], dtype=np.float32)
+    if not np.array_equal(s0.astype(np.float64), pool[idx[rows]]):
+        raise ValueError("pool values must be float32-representable")
+    res = forward(np.ascontiguousarray(qb[rows][:, None]), np.ascontiguousarray(kb[rows][:, None]),
+                  np.ascontiguousarray(vb[rows][:, None]), np.ascontiguousarray(gf[rows][:, None]),
+                  np.ascontiguousarray(bf[rows][:, None]), s0)
+    o[rows] = res["o64"][:, 0]
+    pool[idx[rows]] = res["state"]
+    return o, pool
+

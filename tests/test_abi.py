@@ -117,3 +117,30 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(kda, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         kda.lib()
+
+
+def call_decode(L, B=4, H=2, HV=4, K=128, V=128, q=1, k=2, v=3, g=4, beta=5, state=6, idx=7, o=8,
+                qs=None, ks=None, vs=None, slot_stride=None, slots=8):
+    P = ctypes.c_void_p
+    step = 1 << 32  # arguments live far apart unless a case moves one
+    ptr = lambda i: None if i is None else P(FAKE + int(i * step))
+    qs = H * K if qs is None else qs
+    ks = H * K if ks is None else ks
+    vs = HV * V if vs is None else vs
+    slot_stride = HV * K * V if slot_stride is None else slot_stride
+    return L.kda_decode_step(ptr(q), qs, ptr(k), ks, ptr(v), vs, ptr(g), ptr(beta), ptr(state), slot_stride, slots,
+                             ptr(idx), B, H, HV, K, V, ptr(o), None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(K=64), 2), (dict(V=64), 2), (dict(HV=3), 1), (dict(H=0), 1), (dict(B=-1), 1), (dict(slots=0), 1),
+    (dict(q=None), 1), (dict(idx=None), 1), (dict(o=None), 1), (dict(qs=128), 1), (dict(vs=100), 1),
+    (dict(slot_stride=1000), 1), (dict(state=6 + 2 ** -32 * 8), 3), (dict(qs=258), 3), (dict(q=1 + 2 ** -32 * 2), 3),
+    (dict(o=6), 1), (dict(o=1), 1), (dict(state=3), 1),
+])
+def test_decode_rejects_bad_arguments(L, over, code):
+    assert call_decode(L, **over) == code
+
+
+def test_decode_empty_batch_is_a_no_op(L):
+    assert call_decode(L, B=0) == 0
