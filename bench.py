@@ -194,6 +194,146 @@ def time_oracle(case, target_s: float = 15.0, steps: int = 1, warmup: int = 0):
             "seconds": dt / steps}
 
 
+# ---------------------------------------------------------------------------------------------- decode step
+
+DECODE_METRIC = "KDA decode step rows·heads/s @B=1024,H=HV=12,K=V=128; % of roofline"
+DECODE_UNIT = "rows·heads/s"
+
+
+def decode_bytes(case) -> int:
+    """Algorithmic bytes of one decode step: every active (row, value head) reads and writes its 128x128 bf16
+    state and reads v, g, beta, writes o; q and k once per query/key head; the slot indices."""
+    per_head = 2 * 128 * 128 * 2 + 128 * 2 + 128 * 4 + 4 + 128 * 2
+    return case.B * case.HV * per_head + case.B * case.H * 2 * 128 * 2 + case.B * 4
+
+
+def time_oracle_decode(case, target_s: float = 10.0, steps: int = 1, warmup: int = 0):
+    """The oracle's decode step, as it stands, on the first rows of the workload (about target_s per step)."""
+    import oracle
+    from kda_gated_delta_prefill_b200 import inputs as gen
+    x = gen.make_decode_inputs(case)
+    pool = x["state"].float()
+    run = lambda rows: oracle.decode_step(x["q"][:rows], x["k"][:rows], x["v"][:rows], x["g"][:rows],
+                                          x["beta"][:rows], pool, x["state_indices"][:rows])
+    t0 = time.perf_counter()
+    run(8)
+    per_row = (time.perf_counter() - t0) / 8
+    rows = int(min(case.B, max(8, target_s / max(per_row, 1e-9))))
+    for _ in range(warmup):
+        run(rows)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        run(rows)
+    dt = (time.perf_counter() - t0) / steps
+    return {"value": rows * case.HV / dt, "unit": DECODE_UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"first {rows} rows of {case.name}", "seconds": dt}
+
+
+def bench_decode(args, case, world, rank, dev):
+    import torch
+    import torch.distributed as dist
+    import dataclasses
+    import kda_gated_delta_prefill_b200 as kda
+    from kda_gated_delta_prefill_b200 import inputs as gen
+    config = {"workload": case.name, "B": case.B, "H": case.H, "HV": case.HV, "K": 128, "V": 128,
+              "state_slots": case.slots, "state_dtype": "bf16",
+              "l2": "state pool (%.0f MB) larger than L2; no flush" % (case.slots * case.HV * 32768 / 1e6),
+              "parallelism": f"independent replicas x{args.gpus} (weak)" if args.gpus > 1 else "single GPU"}
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        per_step = min(10.0, max(0.05, 150.0 / (args.steps + args.warmup)))
+        cb = time_oracle_decode(case, per_step, steps=args.steps, warmup=args.warmup)
+        line = {"metric": DECODE_METRIC, "value": cb["value"], "unit": DECODE_UNIT, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["seconds"] * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config, "impl": "reference",
+                "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": cb["value"], "unit": DECODE_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+    x = gen.make_decode_inputs(dataclasses.replace(case, seed=case.seed + 1000 * rank), device=dev)
+    o = torch.empty(case.B, case.HV, 128, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], x["state"], x["state_indices"], o=o,
+                        stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    total_ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    active = int((x["state_indices"] >= 0).sum().item())
+    value = active * case.HV * world / (total_ms / 1e3 / args.steps)
+    hbm_gbs, _, peak_kind = load_peaks()
+    avg_s = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
+    achieved = decode_bytes(case) / avg_s / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
+                "traffic": None, "peak_kind": peak_kind, "algorithmic_bytes_per_launch": decode_bytes(case),
+                "avg_launch_ms": avg_s * 1e3}
+    e2e = None
+    if not args.no_e2e:  # per step: the step's inputs from pinned host memory in, o out; the pool stays resident
+        names = ("q", "k", "v", "g", "beta", "state_indices")
+        xh = {k: x[k].cpu().pin_memory() for k in names}
+        xd = {k: torch.empty_like(x[k]) for k in names}
+        oh = torch.empty(case.B, case.HV, 128, dtype=torch.bfloat16).pin_memory()
+
+        def hstep():
+            for k in names:
+                xd[k].copy_(xh[k], non_blocking=True)
+            kda.decode_step(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], x["state"], xd["state_indices"], o=o,
+                            stream=stream)
+            oh.copy_(o, non_blocking=True)
+        for _ in range(2):
+            hstep()
+        torch.cuda.synchronize()
+        n_e = max(3, min(args.steps, 20))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e):
+            hstep()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        e2e = {"value": active * case.HV * world / (e_ms / 1e3 / n_e), "unit": DECODE_UNIT,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in xh.values()),
+               "d2h_bytes_per_step": oh.numel() * 2, "steps": n_e}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = time_oracle_decode(case)
+        cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    line = {"metric": DECODE_METRIC, "value": value, "unit": DECODE_UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
+            "gpu_launches": args.steps, "impl": "native", "kernel_source": kernel_source_hash()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 # ---------------------------------------------------------------------------------------------- main
 
 def main():
@@ -202,7 +342,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="long_T65536_H64_state")
+    ap.add_argument("--workload", default="long_T65536_H64_state",
+                    help="a prefill workload name, or decode_B1024_H12 for the decode step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile-T", type=int, default=0,
@@ -216,11 +357,14 @@ def main():
     import torch.distributed as dist
     from kda_gated_delta_prefill_b200 import inputs as gen
 
-    case = {c.name: c for c in gen.WORKLOADS}[args.workload]
+    decode = args.workload.startswith("decode")
+    case = gen.DECODE_SERVING if decode else {c.name: c for c in gen.WORKLOADS}[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    config = {"workload": case.name, "B": case.B, "T": case.T, "H": case.H, "HV": case.HV, "K": case.K,
+    if decode and args.impl == "reference":
+        return bench_decode(args, case, world, rank, None)
+    config = None if decode else {"workload": case.name, "B": case.B, "T": case.T, "H": case.H, "HV": case.HV, "K": case.K,
               "V": case.V, "chunk": 64, "initial_state": case.state != "none",
               "l2": "inputs (6.5 GB) larger than L2; no flush" if case.name.startswith("long")
               else "inputs re-used across steps (may hit L2)",
@@ -257,6 +401,8 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     kda.lib()
+    if decode:
+        return bench_decode(args, case, world, rank, dev)
 
     # ---- inputs resident in HBM (rank-specific seed: independent batches) ----
     import dataclasses

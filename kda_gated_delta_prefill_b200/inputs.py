@@ -151,3 +151,42 @@ def worked_example(T: int = 128, K: int = 128, V: int = 128) -> dict:
     return {"q": q.to(torch.bfloat16), "k": q.clone().to(torch.bfloat16),
             "v": torch.ones(1, T, 1, V).to(torch.bfloat16), "g": torch.zeros(1, T, 1, K),
             "beta": torch.ones(1, T, 1), "initial_state": None, "cu_seqlens": None}
+
+
+# ---------------------------------------------------------------------------------------------- decode step
+@dataclass
+class DecodeCase:
+    """One decode step of B rows on a pool of ``slots`` bf16 states; ``pad`` of the rows are -1 padding."""
+    name: str
+    B: int
+    H: int
+    HV: int
+    slots: int
+    pad: float = 0.0
+    seed: int = 0
+
+
+# The decode page's serving shape (H = 12, K = V = 128) at a large batch.
+DECODE_SERVING = DecodeCase("decode_B1024_H12", B=1024, H=12, HV=12, slots=2048, seed=11)
+
+
+def make_decode_inputs(case: DecodeCase, device: str | torch.device = "cpu") -> dict:
+    """Draw q, k, v, g, beta, the state pool and the slot indices (in that order) for one decode step."""
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(case.seed)
+    B, H, HV = case.B, case.H, case.HV
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, device=dev, dtype=torch.float32)
+
+    q = randn(B, H, 128).to(torch.bfloat16)
+    k = randn(B, H, 128).to(torch.bfloat16)
+    v = randn(B, HV, 128).to(torch.bfloat16)
+    g = -F.softplus(randn(B, HV, 128)) / 8.0
+    beta = torch.sigmoid(randn(B, HV))
+    state = (0.1 * randn(case.slots, HV, 128, 128)).to(torch.bfloat16)
+    slots = torch.randperm(case.slots, generator=gen, device=dev)[:B].to(torch.int32)
+    drop = torch.rand(B, generator=gen, device=dev) < case.pad
+    idx = torch.where(drop, torch.full_like(slots, -1), slots)
+    return {"q": q, "k": k, "v": v, "g": g, "beta": beta, "state": state, "state_indices": idx}
