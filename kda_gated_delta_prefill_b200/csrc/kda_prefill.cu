@@ -557,9 +557,20 @@ extern "C" kda_status_t kda_decode_step(const void *q, int64_t q_row_stride, con
     dp.slot_stride = slot_stride;
     dp.state_indices = state_indices;
     dp.o = static_cast<__nv_bfloat16 *>(o);
+    dp.B = B;
     dp.H = H;
     dp.HV = HV;
-    kda::kda_decode_kernel<<<B * HV, kda::kDecodeThreads, 0, static_cast<cudaStream_t>(stream)>>>(dp);
+    DeviceInfo info;
+    if (device_info(info) != cudaSuccess) return KDA_ERR_CUDA;
+    dp.err = info.err;
+    using namespace kda;
+    auto kern = kda_decode_kernel<kDecodeThreads, kDecodeStages>;
+    constexpr int smem = DecodeSmem<kDecodeThreads, kDecodeStages>::TOTAL;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    const int64_t units = static_cast<int64_t>(B) * HV, cap = static_cast<int64_t>(info.sms) * kDecodeCtasPerSm;
+    const int grid = static_cast<int>(units < cap ? units : cap);
+    kern<<<grid, kDecodeThreads, smem, static_cast<cudaStream_t>(stream)>>>(dp);
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

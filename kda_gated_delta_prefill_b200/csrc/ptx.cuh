@@ -113,6 +113,12 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 // Wait only until every committed bulk store has finished reading its shared-memory source (the CTA may then
 // exit or reuse the buffer); the global writes complete on their own before the grid is done.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+// Same, but the N most recently committed groups may still be reading.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read_allow()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;\n" ::"n"(N) : "memory");
+}
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy.
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 
