@@ -216,7 +216,10 @@ int kda_prefill_kernel_launches(int B, int T, int H, int HV, int K, int V, int n
  *                 Active indices must be unique and < num_slots (device
  *                 values, not checked).
  *   o             bf16 [B, HV, V] out, overlapping no other argument.
- * B = 0 is a no-op.  K = V = 128.  Asynchronous on `stream`.
+ * B = 0 is a no-op.  K = V = 128.  Asynchronous on `stream`.  Each (row,
+ * value head) state block moves by bulk copy through shared memory; a copy
+ * that has not landed after about a second sets bit 1 of the device error
+ * word (kda_prefill_device_error) and the kernel stops.
  */
 kda_status_t kda_decode_step(const void *q, int64_t q_row_stride, const void *k, int64_t k_row_stride,
                              const void *v, int64_t v_row_stride, const float *g, const float *beta,

@@ -66,8 +66,9 @@ def _check(o, new_pool, ref_o, ref_pool, pool, idx, g):
             assert torch.equal(new_pool[s], pool[s]), s
 
 
+# (400, 4, 8): 3200 (row, head) units, several per persistent CTA, with padding rows among them
 @pytest.mark.parametrize("B,H,HV,N,pad", [(1, 1, 1, 1, 0.0), (37, 2, 4, 64, 0.25), (64, 12, 12, 96, 0.1),
-                                          (5, 1, 8, 5, 0.0)])
+                                          (5, 1, 8, 5, 0.0), (400, 4, 8, 512, 0.3)])
 def test_decode_parity(B, H, HV, N, pad):
     q, k, v, g, beta, pool, idx = _case(B, H, HV, N, seed=500 + B + HV, pad=pad)
     o, new_pool = _gpu(q, k, v, g, beta, pool, idx)
@@ -118,3 +119,30 @@ def test_decode_steps_follow_the_oracle():
         pool_ref = torch.from_numpy(ref_pool).bfloat16().float()
     diff = (pool_gpu.cpu().float() - pool_ref).abs().max().item()
     assert diff <= 4 * BF16_ULP * pool_ref.abs().max().item(), diff
+
+
+def test_decode_full_workload_sampled():
+    """The 1024-row, 12-head serving step on its 2048-slot pool, in the launch shape the benchmark times:
+    rows are independent, so a sample of rows is checked against the oracle on just their slots."""
+    import kda_gated_delta_prefill_b200 as kda
+    from kda_gated_delta_prefill_b200.inputs import DECODE_SERVING, make_decode_inputs
+    case = DECODE_SERVING
+    d = make_decode_inputs(case, device="cuda")
+    before = d["state"].clone()
+    o = kda.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], d["state"], d["state_indices"])
+    torch.cuda.synchronize()
+    assert kda.device_error(clear=True) == 0
+    rows = torch.arange(0, case.B, 33)  # 32 rows spread over the batch (and so over the CTAs' unit lists)
+    idx = d["state_indices"][rows].cpu()
+    slots = idx.clamp(min=0).long()
+    mini = before[slots.cuda()].cpu()
+    mini_idx = torch.where(idx >= 0, torch.arange(len(rows), dtype=torch.int32), idx)
+    sub = [d[n][rows.cuda()].cpu() for n in ("q", "k", "v", "g", "beta")]
+    ref_o, ref_pool = oracle.decode_step(*sub, mini.float(), mini_idx)
+    got_pool = d["state"][slots.cuda()].cpu()
+    _check(o[rows.cuda()].cpu(), got_pool, ref_o, ref_pool, mini, mini_idx, sub[3])
+    # slots no row selects keep their bytes
+    unused = torch.ones(case.slots, dtype=torch.bool)
+    unused[d["state_indices"][d["state_indices"] >= 0].long().cpu()] = False
+    free = torch.nonzero(unused).flatten()[:64].cuda()
+    assert torch.equal(d["state"][free], before[free])
