@@ -60,6 +60,8 @@ def _load():
         lib.kda_oracle_recurrence_f64.restype = I
         lib.kda_oracle_forward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P]
         lib.kda_oracle_forward.restype = I
+        lib.kda_oracle_backward_f64.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P]
+        lib.kda_oracle_backward_f64.restype = I
         lib.kda_oracle_max_threads.argtypes = []
         lib.kda_oracle_max_threads.restype = I
         lib.kda_oracle_f64_to_bf16.argtypes = [ctypes.c_double]
@@ -169,6 +171,82 @@ def forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, return_normal
     if return_normalized:
         out["qn"], out["kn"] = qn, kn
     return out
+
+
+def backward_f64(qn, kn, v, g, beta, initial_state, do, dht, cu_seqlens=None):
+    """Reverse mode of ``recurrence_f64`` (same shapes and conventions) for the loss
+    sum(o * do) + sum(final_state * dht) of the backward left optional on "KDA Chunk Prefill on Ascend A3"
+    (section "Timing and required submission").  ``dht`` may be None (zero).
+
+    Returns float64 arrays (dqn, dkn [B,T,HV,K] -- the gradient reaching the normalised q/k row that value
+    head h read, not yet summed over a Q/K head's group --, dv [B,T,HV,V], dg [B,T,HV,K], dbeta [B,T,HV],
+    ds0 [N,HV,K,V]).
+    """
+    qn = np.ascontiguousarray(qn, dtype=np.float64)
+    kn = np.ascontiguousarray(kn, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    beta = np.ascontiguousarray(beta, dtype=np.float64)
+    do = np.ascontiguousarray(do, dtype=np.float64)
+    B, T, H, K = qn.shape
+    HV, V = v.shape[2], v.shape[3]
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    N = B if cu is None else len(cu) - 1
+    s0 = None if initial_state is None else np.ascontiguousarray(initial_state, dtype=np.float64)
+    dh = None if dht is None else np.ascontiguousarray(dht, dtype=np.float64)
+    dqn = np.zeros((B, T, HV, K), np.float64)
+    dkn = np.zeros((B, T, HV, K), np.float64)
+    dv = np.zeros((B, T, HV, V), np.float64)
+    dg = np.zeros((B, T, HV, K), np.float64)
+    dbeta = np.zeros((B, T, HV), np.float64)
+    ds0 = np.zeros((N, HV, K, V), np.float64)
+    rc = _load().kda_oracle_backward_f64(_ptr(qn), _ptr(kn), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0), _ptr(cu),
+                                         N, B, T, H, HV, K, V, _ptr(do), _ptr(dh), _ptr(dqn), _ptr(dkn),
+                                         _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(ds0))
+    if rc != 0:
+        raise ValueError("oracle backward rejected the shapes")
+    return dqn, dkn, dv, dg, dbeta, ds0
+
+
+def l2norm_backward_f64(x, dy, eps=1e-6):
+    """Gradient through y = x / sqrt(sum(x^2) + eps) along the last axis, in float64:
+    dx = dy / n - x (x . dy) / n^3 with n = sqrt(sum(x^2) + eps)."""
+    x = np.asarray(x, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    n = np.sqrt((x * x).sum(-1, keepdims=True) + eps)
+    return dy / n - x * (x * dy).sum(-1, keepdims=True) / n ** 3
+
+
+def backward(q, k, v, g, beta, initial_state, do, dht, cu_seqlens=None):
+    """Oracle backward from the raw inputs the library's forward takes.
+
+    The forward's normalised q/k are the bf16-rounded values it uses; the rounding is passed through (its
+    derivative taken as one), so dq = J_norm(q)^T sum_h dqn_h over the value heads h of q's group, with the
+    normalisation's Jacobian at the raw float values.  Returns float64 (dq, dk [B,T,H,K], dv [B,T,HV,V],
+    dg [B,T,HV,K], dbeta [B,T,HV], dh0 [N,HV,K,V] or None when ``initial_state`` is None).
+    """
+    qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
+    qn = bits_to_f32(l2norm_bf16(qb)).astype(np.float64)
+    kn = bits_to_f32(l2norm_bf16(kb)).astype(np.float64)
+    vf = bits_to_f32(vb).astype(np.float64)
+    gf = _f32(g).astype(np.float64)
+    bf = _f32(beta).astype(np.float64)
+    s0 = None if initial_state is None else _f32(initial_state).astype(np.float64)
+    dof = _f32(do).astype(np.float64) if not isinstance(do, np.ndarray) or do.dtype != np.uint16 else \
+        bits_to_f32(do).astype(np.float64)
+    dh = None if dht is None else _f32(dht).astype(np.float64)
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens).astype(np.int32)
+    dqn, dkn, dv, dg, dbeta, ds0 = backward_f64(qn, kn, vf, gf, bf, s0, dof, dh, cu)
+    B, T, H, K = qb.shape
+    HV = vb.shape[2]
+    grp = HV // H
+    dqn = dqn.reshape(B, T, H, grp, K).sum(3)
+    dkn = dkn.reshape(B, T, H, grp, K).sum(3)
+    dq = l2norm_backward_f64(bits_to_f32(qb), dqn)
+    dk = l2norm_backward_f64(bits_to_f32(kb), dkn)
+    return dq, dk, dv, dg, dbeta, (None if initial_state is None else ds0)
 
 
 def decode_step(q, k, v, g, beta, state, state_indices):

@@ -282,3 +282,176 @@ done:
 
 /* Exposed for tests of the rounding helper itself. */
 uint16_t kda_oracle_f64_to_bf16(double x) { return f64_to_bf16_rne(x); }
+
+/*
+ * Reverse mode of the float64 recurrence above, for the backward the page
+ * "KDA Chunk Prefill on Ascend A3" leaves optional (section "Timing and
+ * required submission"): the loss is sum(o * do) + sum(final_state * dht),
+ * and the gradients are those of q, k, v, g, beta and the initial state.
+ * This function differentiates the recurrence on the normalised inputs it is
+ * given; the L2 normalisation's own derivative is applied by the caller.
+ *
+ * Inputs as kda_oracle_recurrence_f64, plus do_ [B,T,HV,V] and dht
+ * [N,HV,K,V] (NULL = zero).  Outputs (all float64):
+ *   dq, dk [B,T,HV,K]  gradient with respect to the normalised q/k row that
+ *                      value head h read (the caller sums a Q/K head's group)
+ *   dv [B,T,HV,V], dg [B,T,HV,K], dbeta [B,T,HV], ds0 [N,HV,K,V]
+ * Rows outside every sequence (varlen) are left untouched.
+ *
+ * For a token t with S' = diag(exp g_t) S_{t-1}, r = v_t - S'^T k_t,
+ * S_t = S' + beta_t k_t r^T and o_t = K^-0.5 S_t^T q_t, the adjoints, with dS
+ * the gradient arriving at S_t, are taken in this order:
+ *   dS  += K^-0.5 q_t do_t^T          dq_t  = K^-0.5 S_t do_t
+ *   dr   = beta_t dS^T k_t             dbeta = k_t^T dS r
+ *   dk_t = beta_t dS r - S' dr         dv_t  = dr
+ *   dS'  = dS - k_t dr^T               dg_t  = rowsum(S' * dS')
+ *   dS_{t-1} = diag(exp g_t) dS'
+ * The states S_t are recomputed forward from checkpoints every 32 tokens.
+ */
+int kda_oracle_backward_f64(const double *q, const double *k, const double *v, const double *g,
+                            const double *beta, const double *s0, const int32_t *cu, int N, int B, int T,
+                            int H, int HV, int K, int V, const double *do_, const double *dht, double *dq,
+                            double *dk, double *dv, double *dg, double *dbeta, double *ds0)
+{
+    if (N <= 0 || B <= 0 || T < 0 || H <= 0 || HV <= 0 || K <= 0 || V <= 0) return -1;
+    if (HV % H != 0) return -1;
+    if (cu && B != 1) return -1;
+    if (!cu && N != B) return -1;
+    const int group = HV / H;
+    const double scale = 1.0 / sqrt((double)K);
+    const int64_t units = (int64_t)N * HV;
+    const int CK = 32;
+    const size_t KV = (size_t)K * V;
+    int bad = 0;
+
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t u = 0; u < units; ++u) {
+        const int n = (int)(u / HV);
+        const int h = (int)(u % HV);
+        const int hq = h / group;
+        int64_t b, t0, t1;
+        seq_range(cu, n, T, &b, &t0, &t1);
+        if (t0 < 0 || t1 < t0 || t1 > T) { bad |= 1; continue; }
+        const int64_t len = t1 - t0, nblk = (len + CK - 1) / CK;
+        /* ckpt[m] = state before token t0 + m*CK; blk[j] = state after token j of the current block */
+        double *ckpt = (double *)malloc(sizeof(double) * KV * (size_t)(nblk > 0 ? nblk : 1));
+        double *blk = (double *)malloc(sizeof(double) * KV * (size_t)(CK + 1));
+        double *dS = (double *)malloc(sizeof(double) * KV);
+        double *Sd = (double *)malloc(sizeof(double) * KV);
+        double *r = (double *)malloc(sizeof(double) * V);
+        double *dr = (double *)malloc(sizeof(double) * V);
+        if (!ckpt || !blk || !dS || !Sd || !r || !dr) {
+            free(ckpt); free(blk); free(dS); free(Sd); free(r); free(dr);
+            bad |= 1;
+            continue;
+        }
+        double *S = blk; /* running state during the checkpoint pass */
+        if (s0) memcpy(S, s0 + u * (int64_t)KV, sizeof(double) * KV);
+        else memset(S, 0, sizeof(double) * KV);
+
+        /* one token forward: S_in -> S_out (may alias); fills Sd = S' and r */
+#define KDA_STEP(t, S_in, S_out)                                                                   \
+    do {                                                                                           \
+        const int64_t row_ = b * T + (t);                                                          \
+        const double *kt_ = k + (row_ * H + hq) * K;                                               \
+        const double *vt_ = v + (row_ * HV + h) * V;                                               \
+        const double *gt_ = g + (row_ * HV + h) * K;                                               \
+        const double bt_ = beta[row_ * HV + h];                                                    \
+        for (int d = 0; d < K; ++d) {                                                              \
+            const double e_ = exp(gt_[d]);                                                         \
+            for (int c = 0; c < V; ++c) Sd[(int64_t)d * V + c] = (S_in)[(int64_t)d * V + c] * e_; \
+        }                                                                                          \
+        for (int c = 0; c < V; ++c) {                                                              \
+            double acc_ = 0.0;                                                                     \
+            for (int d = 0; d < K; ++d) acc_ += kt_[d] * Sd[(int64_t)d * V + c];                   \
+            r[c] = vt_[c] - acc_;                                                                  \
+        }                                                                                          \
+        for (int d = 0; d < K; ++d) {                                                              \
+            const double bk_ = bt_ * kt_[d];                                                       \
+            for (int c = 0; c < V; ++c) (S_out)[(int64_t)d * V + c] = Sd[(int64_t)d * V + c] + bk_ * r[c]; \
+        }                                                                                          \
+    } while (0)
+
+        for (int64_t m = 0; m < nblk; ++m) {
+            memcpy(ckpt + (size_t)m * KV, S, sizeof(double) * KV);
+            const int64_t te = t0 + (m + 1) * CK < t1 ? t0 + (m + 1) * CK : t1;
+            for (int64_t t = t0 + m * CK; t < te; ++t) KDA_STEP(t, S, S);
+        }
+        /* S now holds the final state: the gradient arriving there is dht */
+        if (dht) memcpy(dS, dht + u * (int64_t)KV, sizeof(double) * KV);
+        else memset(dS, 0, sizeof(double) * KV);
+
+        for (int64_t m = nblk - 1; m >= 0; --m) {
+            const int64_t tb = t0 + m * CK;
+            const int64_t te = tb + CK < t1 ? tb + CK : t1;
+            const int cnt = (int)(te - tb);
+            memcpy(blk, ckpt + (size_t)m * KV, sizeof(double) * KV);
+            for (int j = 0; j < cnt; ++j) KDA_STEP(tb + j, blk + (size_t)j * KV, blk + (size_t)(j + 1) * KV);
+            for (int j = cnt - 1; j >= 0; --j) {
+                const int64_t t = tb + j;
+                const int64_t row = b * T + t;
+                const double *qt = q + (row * H + hq) * K;
+                const double *kt = k + (row * H + hq) * K;
+                const double *gt = g + (row * HV + h) * K;
+                const double bt = beta[row * HV + h];
+                const double *dot = do_ + (row * HV + h) * V;
+                const double *Sp = blk + (size_t)j * KV, *St = blk + (size_t)(j + 1) * KV;
+                double *dqt = dq + (row * HV + h) * K, *dkt = dk + (row * HV + h) * K;
+                double *dvt = dv + (row * HV + h) * V, *dgt = dg + (row * HV + h) * K;
+                /* S' and r of this token again (from S_{t-1}) */
+                for (int d = 0; d < K; ++d) {
+                    const double e = exp(gt[d]);
+                    for (int c = 0; c < V; ++c) Sd[(int64_t)d * V + c] = Sp[(int64_t)d * V + c] * e;
+                }
+                const double *vt = v + (row * HV + h) * V;
+                for (int c = 0; c < V; ++c) {
+                    double acc = 0.0;
+                    for (int d = 0; d < K; ++d) acc += kt[d] * Sd[(int64_t)d * V + c];
+                    r[c] = vt[c] - acc;
+                }
+                /* output: dq_t = K^-0.5 S_t do_t, dS += K^-0.5 q_t do_t^T */
+                for (int d = 0; d < K; ++d) {
+                    double acc = 0.0;
+                    for (int c = 0; c < V; ++c) acc += St[(int64_t)d * V + c] * dot[c];
+                    dqt[d] = scale * acc;
+                    const double sq = scale * qt[d];
+                    for (int c = 0; c < V; ++c) dS[(int64_t)d * V + c] += sq * dot[c];
+                }
+                /* dr = beta dS^T k, dbeta = k^T dS r */
+                double db = 0.0;
+                for (int c = 0; c < V; ++c) {
+                    double acc = 0.0;
+                    for (int d = 0; d < K; ++d) acc += kt[d] * dS[(int64_t)d * V + c];
+                    dr[c] = bt * acc;
+                    db += acc * r[c];
+                }
+                dbeta[row * HV + h] = db;
+                /* dk = beta dS r - S' dr; dv = dr */
+                for (int d = 0; d < K; ++d) {
+                    double a1 = 0.0, a2 = 0.0;
+                    for (int c = 0; c < V; ++c) {
+                        a1 += dS[(int64_t)d * V + c] * r[c];
+                        a2 += Sd[(int64_t)d * V + c] * dr[c];
+                    }
+                    dkt[d] = bt * a1 - a2;
+                }
+                for (int c = 0; c < V; ++c) dvt[c] = dr[c];
+                /* dS' = dS - k dr^T; dg = rowsum(S' * dS'); dS_{t-1} = diag(exp g) dS' */
+                for (int d = 0; d < K; ++d) {
+                    const double e = exp(gt[d]);
+                    double acc = 0.0;
+                    for (int c = 0; c < V; ++c) {
+                        const double x = dS[(int64_t)d * V + c] - kt[d] * dr[c];
+                        acc += Sd[(int64_t)d * V + c] * x;
+                        dS[(int64_t)d * V + c] = e * x;
+                    }
+                    dgt[d] = acc;
+                }
+            }
+        }
+#undef KDA_STEP
+        if (ds0) memcpy(ds0 + u * (int64_t)KV, dS, sizeof(double) * KV);
+        free(ckpt); free(blk); free(dS); free(Sd); free(r); free(dr);
+    }
+    return bad ? -1 : 0;
+}

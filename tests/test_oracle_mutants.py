@@ -15,6 +15,7 @@ import subprocess
 import pytest
 
 import oracle as oracle_pkg
+from tests import test_oracle_backward as bwd_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle_pkg.__file__), "kda_oracle.c")
@@ -33,6 +34,20 @@ MUTANTS = {
     "decay_after_update_output": ("ot[c] = acc;", "ot[c] = acc * exp(gt[0]);"),
 }
 
+# slips in the reverse mode (each site occurs only in the backward)
+BWD_MUTANTS = {
+    "bwd_dq_no_scale": ("dqt[d] = scale * acc;", "dqt[d] = acc;"),
+    "bwd_dq_from_previous_state": ("acc += St[(int64_t)d * V + c] * dot[c];", "acc += Sp[(int64_t)d * V + c] * dot[c];"),
+    "bwd_dr_no_beta": ("dr[c] = bt * acc;", "dr[c] = acc;"),
+    "bwd_dbeta_uses_v": ("db += acc * r[c];", "db += acc * vt[c];"),
+    "bwd_dk_sign": ("dkt[d] = bt * a1 - a2;", "dkt[d] = bt * a1 + a2;"),
+    "bwd_dropped_rank1_term": ("const double x = dS[(int64_t)d * V + c] - kt[d] * dr[c];",
+                               "const double x = dS[(int64_t)d * V + c];"),
+    "bwd_dg_from_undecayed_state": ("acc += Sd[(int64_t)d * V + c] * x;", "acc += Sp[(int64_t)d * V + c] * x;"),
+    "bwd_adjoint_not_decayed": ("dS[(int64_t)d * V + c] = e * x;", "dS[(int64_t)d * V + c] = x;"),
+    "bwd_wrong_checkpoint": ("memcpy(blk, ckpt + (size_t)m * KV,", "memcpy(blk, ckpt + (size_t)(m > 0 ? m - 1 : 0) * KV,"),
+}
+
 
 def _pin_functions():
     out = []
@@ -45,9 +60,7 @@ def _pin_functions():
     return out
 
 
-@pytest.mark.parametrize("mutant", sorted(MUTANTS))
-def test_pins_catch_mutant(mutant, tmp_path):
-    old, new = MUTANTS[mutant]
+def _run_mutant(old, new, tmp_path, pin_functions):
     src = open(SRC).read()
     assert src.count(old) >= 1, f"mutation site for {mutant} not found"
     mutated = src.replace(old, new, 1)
@@ -59,17 +72,34 @@ def test_pins_catch_mutant(mutant, tmp_path):
     real = oracle_pkg._load()
     lib = ctypes.CDLL(str(so_path))
     for fname in ("kda_oracle_l2norm_bf16", "kda_oracle_recurrence_f64", "kda_oracle_forward",
-                  "kda_oracle_max_threads", "kda_oracle_f64_to_bf16"):
+                  "kda_oracle_max_threads", "kda_oracle_f64_to_bf16", "kda_oracle_backward_f64"):
         f, r = getattr(lib, fname), getattr(real, fname)
         f.argtypes, f.restype = r.argtypes, r.restype
     caught = []
     oracle_pkg._lib = lib
     try:
-        for name, fn in _pin_functions():
+        for name, fn in pin_functions:
             try:
                 fn(oracle_pkg)
             except AssertionError:
                 caught.append(name)
     finally:
         oracle_pkg._lib = real
-    assert caught, f"no pin caught mutant {mutant}"
+    return caught
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_pins_catch_mutant(mutant, tmp_path):
+    old, new = MUTANTS[mutant]
+    assert _run_mutant(old, new, tmp_path, _pin_functions()), f"no pin caught mutant {mutant}"
+
+
+def _bwd_pin_functions():
+    return [(name, fn) for name, fn in inspect.getmembers(bwd_pins, inspect.isfunction)
+            if name.startswith("test_") and "oracle" in inspect.signature(fn).parameters]
+
+
+@pytest.mark.parametrize("mutant", sorted(BWD_MUTANTS))
+def test_backward_pins_catch_mutant(mutant, tmp_path):
+    old, new = BWD_MUTANTS[mutant]
+    assert _run_mutant(old, new, tmp_path, _bwd_pin_functions()), f"no pin caught mutant {mutant}"
