@@ -193,6 +193,49 @@ kda_status_t kda_prefill_device_error(unsigned *word, int clear);
 int kda_prefill_kernel_launches(int B, int T, int H, int HV, int K, int V, int num_seqs);
 
 /*
+ * Backward of kda_prefill_forward, which "KDA Chunk Prefill on Ascend A3"
+ * leaves optional (section "Timing and required submission"): for the loss
+ * sum(o * dout) + sum(final_state * dht) it returns the gradients of q, k,
+ * v, g, beta and the initial state in their own dtypes.  The bf16 rounding
+ * of the normalised q/k rows is passed straight through (its derivative is
+ * taken as one): dq = J(q)^T sum_h dqn_h, J the Jacobian of
+ * q / sqrt(sum q^2 + 1e-6) and the sum over the value heads h that read q.
+ *
+ *   q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, B, T, H, HV, K, V
+ *                as for kda_prefill_forward (initial_state may be NULL)
+ *   dout         bf16 [B,T,HV,V]   gradient of the loss at o
+ *   dht          fp32 [N,HV,K,V]   gradient at final_state, or NULL (zero)
+ *   dq, dk       bf16 [B,T,H,K]    out
+ *   dv           bf16 [B,T,HV,V]   out
+ *   dg           fp32 [B,T,HV,K]   out
+ *   dbeta        fp32 [B,T,HV]     out
+ *   dh0          fp32 [N,HV,K,V]   out, or NULL when not wanted
+ *   workspace    kda_prefill_backward_workspace_size(...) bytes, 256-byte
+ *                aligned, device; holds the recomputed forward's per-chunk
+ *                blocks, every chunk's start state and the gradient at every
+ *                chunk's end state (fp32), and per-value-head gradients at the
+ *                normalised rows.
+ * Outputs overlap no input, no other output and the workspace.  Pointers are
+ * 16-byte aligned (beta, dbeta, cu_seqlens: 4).  Rows outside every packed
+ * sequence are left untouched.  Asynchronous on `stream`; kernel waits that
+ * give up set the device error word (kda_prefill_device_error).
+ *
+ * The forward is recomputed (intra-chunk blocks, then the state carry storing
+ * each chunk's start state); a reverse carry walks each sequence backwards
+ * for the gradient at every chunk's end state; a per-chunk kernel forms the
+ * chunk's gradients; a last kernel sums each Q/K group and applies the
+ * normalisation's Jacobian.  Accuracy assumes g <= 0 with every 8 consecutive
+ * gates of a channel summing to >= -40 (per-token g >= -5 suffices).
+ */
+size_t kda_prefill_backward_workspace_size(int B, int T, int H, int HV, int K, int V, int num_seqs);
+int kda_prefill_backward_kernel_launches(int B, int T, int H, int HV, int K, int V, int num_seqs);
+kda_status_t kda_prefill_backward(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                                  const float *initial_state, const int32_t *cu_seqlens, int num_seqs, int B,
+                                  int T, int H, int HV, int K, int V, const void *dout, const float *dht, void *dq,
+                                  void *dk, void *dv, float *dg, float *dbeta, float *dh0, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+
+/*
  * One recurrent decode step (one token per row) on a caller-owned bf16 state
  * pool, as on the "flashinfer.kda_decode.packed_kda_decode" page, with the
  * recurrence of "KDA Chunk Prefill on Ascend A3" (section "Mathematical

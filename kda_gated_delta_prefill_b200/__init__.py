@@ -27,7 +27,8 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 
 EXPORTED = ("kda_status_string", "kda_prefill_workspace_size", "kda_prefill_forward",
             "kda_prefill_host_staging_size", "kda_prefill_forward_host", "kda_prefill_device_error",
-            "kda_l2norm_bf16", "kda_prefill_kernel_launches", "kda_decode_step")
+            "kda_l2norm_bf16", "kda_prefill_kernel_launches", "kda_decode_step",
+            "kda_prefill_backward_workspace_size", "kda_prefill_backward_kernel_launches", "kda_prefill_backward")
 
 
 class KdaError(RuntimeError):
@@ -69,6 +70,12 @@ def lib():
         L.kda_prefill_kernel_launches.restype = I
         L.kda_decode_step.argtypes = [P, I64, P, I64, P, I64, P, P, P, I64, I, P, I, I, I, I, I, P, P]
         L.kda_decode_step.restype = I
+        L.kda_prefill_backward_workspace_size.argtypes = [I] * 7
+        L.kda_prefill_backward_workspace_size.restype = Z
+        L.kda_prefill_backward_kernel_launches.argtypes = [I] * 7
+        L.kda_prefill_backward_kernel_launches.restype = I
+        L.kda_prefill_backward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, Z, P]
+        L.kda_prefill_backward.restype = I
         _lib = L
         return L
 
@@ -127,6 +134,48 @@ def forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o=None, fi
                                    _stream_ptr(stream))
     _check(rc, "kda_prefill_forward")
     return o, final_state
+
+
+def backward_workspace_size(B, T, H, HV, K=128, V=128, num_seqs=0) -> int:
+    return int(lib().kda_prefill_backward_workspace_size(B, T, H, HV, K, V, num_seqs))
+
+
+def backward_kernel_launches(B, T, H, HV, K=128, V=128, num_seqs=0) -> int:
+    """Kernel launches one backward makes for these sizes (0 if rejected)."""
+    return int(lib().kda_prefill_backward_kernel_launches(B, T, H, HV, K, V, num_seqs))
+
+
+def backward(q, k, v, g, beta, dout, initial_state=None, dht=None, cu_seqlens=None, *, want_dh0=None,
+             workspace=None, stream=None):
+    """Gradients of sum(o * dout) + sum(final_state * dht) for the forward on the same inputs (CUDA).
+
+    Returns (dq, dk [B,T,H,K] bf16, dv [B,T,HV,V] bf16, dg [B,T,HV,K] fp32, dbeta [B,T,HV] fp32,
+    dh0 [N,HV,K,V] fp32, or None when there is no initial state and want_dh0 is not set).
+    """
+    import torch
+    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("dout", dout)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    dev = q.device
+    dq = torch.empty(B, T, H, K, dtype=torch.bfloat16, device=dev)
+    dk = torch.empty(B, T, H, K, dtype=torch.bfloat16, device=dev)
+    dv = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=dev)
+    dg = torch.empty(B, T, HV, K, dtype=torch.float32, device=dev)
+    dbeta = torch.empty(B, T, HV, dtype=torch.float32, device=dev)
+    if want_dh0 is None:
+        want_dh0 = initial_state is not None
+    dh0 = torch.empty(N, HV, K, V, dtype=torch.float32, device=dev) if want_dh0 else None
+    num_seqs = N if cu_seqlens is not None else 0
+    ws_bytes = backward_workspace_size(B, T, H, HV, K, V, num_seqs)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    rc = lib().kda_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                                    _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(dout), _ptr(dht),
+                                    _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dh0),
+                                    _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _check(rc, "kda_prefill_backward")
+    return dq, dk, dv, dg, dbeta, dh0
 
 
 def host_staging_size(B, T, H, HV, K=128, V=128, num_seqs=0, has_initial_state=False, has_cu_seqlens=False) -> int:

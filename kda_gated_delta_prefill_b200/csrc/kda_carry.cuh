@@ -65,8 +65,14 @@ struct CarryParams {
     int seg_phase;
     int seg_count;
     float *seg_S, *seg_M, *seg_B;  // [units][seg_count][K][V]
+    // Unsegmented launches only: when set, the state at the start of every chunk is also stored, fp32
+    // [K][V] at states + (global chunk * HV + h) * K * V (the item's index), for the backward.
+    float *states;
+    int no_o;                      // unsegmented launches: skip o (the O products and stores)
 };
 
+// kDump: the backward's instantiation, which also stores every chunk's start state (p.states)
+template <bool kDump>
 __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const CarryParams p)
 {
     using S = CarrySmem;
@@ -116,11 +122,13 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
             s_out = seg + 1 == p.seg_count ? p.sN + (static_cast<int64_t>(n) * p.HV + h) * DK * DV : nullptr;
         }
     } else if (p.cu) {
+        with_o = !p.no_o;
         c_begin = p.chunk_off[n];
         nck = p.chunk_off[n + 1] - p.chunk_off[n];
         tok0 = p.cu[n];
         len = p.cu[n + 1] - p.cu[n];
     } else {
+        with_o = !p.no_o;
         c_begin = static_cast<int64_t>(n) * p.chunks_per_seq + p.chunk_begin;
         nck = p.chunk_count;
         tok0 = static_cast<int64_t>(n) * p.T + static_cast<int64_t>(p.chunk_begin) * CH;
@@ -268,6 +276,13 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
             __syncwarp();
             if (lane == 0) mbar_arrive(bar);
         };
+        // the state at the start of chunk c (S^T[v][32kq + j] in r) -> states, rows kd = 32kq + j, column v
+        float *dump = kDump && p.seg_phase == 0 ? p.states : nullptr;
+        auto dump_state = [&](const uint32_t (&r)[32], int kq, int c) {
+            float *dst = dump + ((c_begin + c) * p.HV + h) * DK * DV + v;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) dst[(32 * kq + j) * DV] = __uint_as_float(r[j]);
+        };
         bool alive = tmem_alloc == 0;
         if (alive) {
             const float *s0 = from == FROM_S0 ? s_in : nullptr;
@@ -285,6 +300,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
                 }
                 tc_st32(tS(kq), r);
                 pack_state(r, kq);
+                if (kDump && dump && nck > 0) dump_state(r, kq, 0);
             }
             arrive(sready);
         }
@@ -389,6 +405,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
                 tc_ld32(tS(kq), r);
                 tc_wait_ld();
                 pack_state(r, kq);
+                if (kDump && dump && c + 1 < nck) dump_state(r, kq, c + 1);
             }
             arrive(sready);
         }

@@ -27,9 +27,9 @@ __device__ __forceinline__ float div_rn_with_rcp(float x, float d, float r)
     return __fmaf_rn(e, r, q0);
 }
 
-// One warp normalises one row of 128 bf16 values; lane l holds elements
-// 4l..4l+3 as two packed bf16 pairs (lo, hi).  Returns the packed result.
-__device__ __forceinline__ uint2 l2norm_row128_warp(uint2 raw)
+// The row's denominator sqrt(sum x^2 + 1e-6) when a warp holds a row of 128
+// bf16 values, lane l holding elements 4l..4l+3 as two packed bf16 pairs.
+__device__ __forceinline__ float l2norm_den128_warp(uint2 raw)
 {
     const float x0 = bf16lo(raw.x), x1 = bf16hi(raw.x), x2 = bf16lo(raw.y), x3 = bf16hi(raw.y);
     float ss = __fmul_rn(x0, x0);
@@ -38,7 +38,15 @@ __device__ __forceinline__ uint2 l2norm_row128_warp(uint2 raw)
     ss = __fadd_rn(ss, __fmul_rn(x3, x3));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
-    const float den = __fsqrt_rn(__fadd_rn(ss, 1e-6f));
+    return __fsqrt_rn(__fadd_rn(ss, 1e-6f));
+}
+
+// One warp normalises one row of 128 bf16 values; lane l holds elements
+// 4l..4l+3 as two packed bf16 pairs (lo, hi).  Returns the packed result.
+__device__ __forceinline__ uint2 l2norm_row128_warp(uint2 raw)
+{
+    const float x0 = bf16lo(raw.x), x1 = bf16hi(raw.x), x2 = bf16lo(raw.y), x3 = bf16hi(raw.y);
+    const float den = l2norm_den128_warp(raw);
     const float r = __frcp_rn(den);
     uint2 out;
     out.x = pack_bf16(div_rn_with_rcp(x0, den, r), div_rn_with_rcp(x1, den, r));

@@ -1,0 +1,118 @@
+"""GPU parity of the backward (kda_prefill_backward through the C ABI) against the oracle's float64 reverse mode.
+
+Bar, per gradient tensor (dq, dk, dv, dg, dbeta, dh0):
+  ||gpu - ref||_F / ||ref||_F <= 1e-2   and   max |gpu - ref| <= 2e-2 * max |ref|.
+Where it comes from: the recomputed forward's chunk start states carry the forward's own error (its bar is a
+relative Frobenius error of 5e-3 on the state); the reverse carry multiplies by the forward's fp16 blocks (2^-11
+relative per operand); dq, dk and dv are returned in bf16 (2^-9 relative).  Single gradient elements can cancel
+to near zero, so the element-wise bound is taken relative to the tensor's scale.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+REL_FRO = 1e-2
+MAX_REL = 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import kda_gated_delta_prefill_b200 as kda
+    kda.lib()
+
+
+def _case(B, T, H, HV, seed, state=True, dht=True, cu=None, gate=8.0, beta_zero=False):
+    gen = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, T, H, 128, generator=gen).bfloat16()
+    k = torch.randn(B, T, H, 128, generator=gen).bfloat16()
+    v = torch.randn(B, T, HV, 128, generator=gen).bfloat16()
+    g = -torch.nn.functional.softplus(torch.randn(B, T, HV, 128, generator=gen)) / gate
+    beta = torch.sigmoid(torch.randn(B, T, HV, generator=gen))
+    if beta_zero:
+        beta.zero_()
+    N = B if cu is None else len(cu) - 1
+    s0 = 0.1 * torch.randn(N, HV, 128, 128, generator=gen) if state else None
+    dout = torch.randn(B, T, HV, 128, generator=gen).bfloat16()
+    dh = 0.1 * torch.randn(N, HV, 128, 128, generator=gen) if dht else None
+    cu_t = None if cu is None else torch.tensor(cu, dtype=torch.int32)
+    return q, k, v, g, beta, s0, dout, dh, cu_t
+
+
+def _run(q, k, v, g, beta, s0, dout, dh, cu):
+    import kda_gated_delta_prefill_b200 as kda
+    c = lambda t: None if t is None else t.cuda()
+    out = kda.backward(c(q), c(k), c(v), c(g), c(beta), c(dout), c(s0), c(dh), c(cu), want_dh0=True)
+    torch.cuda.synchronize()
+    assert kda.device_error(clear=True) == 0
+    ref = oracle.backward(q, k, v, g, beta, s0, dout.float().numpy(), None if dh is None else dh.numpy(), cu)
+    return [t.float().cpu().numpy().astype(np.float64) for t in out[:5]] + [out[5].cpu().numpy()], ref
+
+
+def _compare(got, ref, rows=None):
+    names = ["dq", "dk", "dv", "dg", "dbeta", "dh0"]
+    report = {}
+    for name, a, b in zip(names, got, ref):
+        if b is None:
+            b = np.zeros_like(a)
+        if rows is not None and name != "dh0":
+            a, b = a[rows], b[rows]
+        assert np.isfinite(a).all(), f"{name}: NaN/Inf"
+        scale = np.abs(b).max()
+        if scale == 0:
+            assert np.abs(a).max() <= 1e-6, name
+            continue
+        fro = np.linalg.norm(a - b) / np.linalg.norm(b)
+        mx = np.abs(a - b).max() / scale
+        report[name] = (fro, mx)
+        assert fro <= REL_FRO and mx <= MAX_REL, f"{name}: rel Frobenius {fro:.3g}, max {mx:.3g}"
+    return report
+
+
+@pytest.mark.parametrize("B,T,H,HV", [(1, 128, 1, 1), (2, 150, 1, 2), (1, 64, 2, 2), (1, 1, 1, 1),
+                                      (1, 333, 2, 4)])
+def test_backward_parity(B, T, H, HV):
+    got, ref = _run(*_case(B, T, H, HV, seed=900 + T + HV))
+    _compare(got, ref)
+
+
+def test_backward_no_state_no_dht():
+    q, k, v, g, beta, s0, dout, dh, cu = _case(1, 200, 1, 2, seed=931, state=False, dht=False)
+    got, ref = _run(q, k, v, g, beta, s0, dout, dh, cu)
+    ref = list(ref)
+    # the initial state's gradient exists even without a state passed (zeros are a state)
+    ref[5] = oracle.backward_f64(
+        oracle.bits_to_f32(oracle.l2norm_bf16(q)).astype(np.float64),
+        oracle.bits_to_f32(oracle.l2norm_bf16(k)).astype(np.float64),
+        v.float().numpy().astype(np.float64), g.numpy().astype(np.float64), beta.numpy().astype(np.float64),
+        None, dout.float().numpy().astype(np.float64), None)[5]
+    _compare(got, ref)
+
+
+def test_backward_beta_zero():
+    got, ref = _run(*_case(1, 130, 1, 1, seed=941, beta_zero=True))
+    _compare(got, ref)
+
+
+def test_backward_varlen():
+    cu = [0, 1, 64, 65, 65, 300]  # one token, exactly a chunk, one token, empty, a ragged multi-chunk sequence
+    q, k, v, g, beta, s0, dout, dh, cu_t = _case(1, 300, 2, 4, seed=951, cu=cu)
+    got, ref = _run(q, k, v, g, beta, s0, dout, dh, cu_t)
+    _compare(got, ref)
+
+
+def test_backward_strong_gates():
+    """Gates down to about -5 per token (softplus without the /8): the factored gate terms stay in range."""
+    got, ref = _run(*_case(1, 192, 1, 1, seed=961, gate=1.0))
+    _compare(got, ref)
+
+
+def test_backward_config2_shape():
+    """The 4-head, 1000-token shape with a ragged tail (15 full chunks and one of 40 tokens)."""
+    got, ref = _run(*_case(1, 1000, 4, 4, seed=2))
+    _compare(got, ref)
