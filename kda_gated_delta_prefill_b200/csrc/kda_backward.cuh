@@ -81,35 +81,32 @@ __device__ __forceinline__ void bwd_locate(const BwdParams &p, int chunk, int &n
 __device__ __forceinline__ float bwd_exp(float x) { return ex2(x * 1.4426950408889634f); }
 
 // ---------------------------------------------------------------------------------------------------------
-// Reverse carry: one CTA per (sequence, value head, half of the value columns).  dS (128 x 64 fp32) lives in
-// shared memory; chunk c's block (the -W, Qg, Kg, Aqk tiles and exp(G_L)) arrives by bulk copy one chunk ahead.
-// Before chunk c is folded in, dS is the gradient at chunk c's end state and is stored for the chunk kernel.
-constexpr int kBcThreads = 512, kBcCols = 64;
+// Reverse carry: one CTA (16 warps) per (sequence, value head, half of the value columns), on fp16 tensor-core
+// MMAs (mma.sync m16n8k16, fp32 accumulate).  The fp32 gradient dS (128 keys x 64 columns) stays in the warps'
+// accumulator registers; an fp16 copy in shared memory feeds the next chunk's Kg dS.  Chunk c's block (the -W,
+// Qg, Kg, Aqk tiles in their SW128 layout, and exp(G_L)) arrives by bulk copy one chunk ahead.  Before chunk c
+// is folded in, dS is the gradient at chunk c's end state and is stored for the chunk kernel.
+constexpr int kBcThreads = 512, kBcCols = 64, kBcPad = 72;  // fp16 row stride (halves) of dS, dO, dVnew copies
 struct BcSmem {
-    static constexpr int PART = ITEM_U;                 // bytes [0, ITEM_U) of a block: -W, Qg, Kg, Aqk
-    static constexpr int STAGE = PART + 512;            // + exp(G_L)
-    static constexpr int DS = 2 * STAGE;                // float [128][64]
-    static constexpr int DO = DS + DK * kBcCols * 4;    // float [64][64]
-    static constexpr int DVN = DO + CH * kBcCols * 4;   // float [64][64]
-    static constexpr int BAR = DVN + CH * kBcCols * 4;  // mbarriers [2]
+    static constexpr int PART = ITEM_U;                   // bytes [0, ITEM_U) of a block: -W, Qg, Kg, Aqk
+    static constexpr int STAGE = PART + 512;              // + exp(G_L)
+    static constexpr int DSH = 2 * STAGE;                 // fp16 [128][72]  dS
+    static constexpr int DOH = DSH + DK * kBcPad * 2;     // fp16 [64][72]   dO
+    static constexpr int DVH = DOH + CH * kBcPad * 2;     // fp16 [64][72]   dVnew
+    static constexpr int BAR = DVH + CH * kBcPad * 2;     // mbarriers [2]
     static constexpr int FLAG = BAR + 16;
     static constexpr int TOTAL = FLAG + 16;
 };
 static_assert(ITEM_GL == ITEM_U + 16384, "block layout");
 
-// fp16 element (r, col) of a [64][128] SW128 tile pair, and of a [64][64] SW128 tile
-__device__ __forceinline__ float tile128_at(const uint8_t *t, int r, int col)
+// byte offset of the 16-byte group (row r, columns c..c+7) of a [64][128] SW128 tile pair / a [64][64] tile
+__device__ __forceinline__ uint32_t sw_off128(int r, int c)
 {
-    const int cb = (col & 63) * 2;
-    const __half hv =
-        *reinterpret_cast<const __half *>(t + (col >> 6) * 8192 + r * 128 + ((((cb >> 4) ^ (r & 7))) << 4) + (cb & 15));
-    return __half2float(hv);
+    return static_cast<uint32_t>((c >> 6) * 8192 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4));
 }
-__device__ __forceinline__ float tile64_at(const uint8_t *t, int r, int col)
+__device__ __forceinline__ uint32_t sw_off64(int r, int c)
 {
-    const int cb = col * 2;
-    const __half hv = *reinterpret_cast<const __half *>(t + r * 128 + ((((cb >> 4) ^ (r & 7))) << 4) + (cb & 15));
-    return __half2float(hv);
+    return static_cast<uint32_t>(r * 128 + (((c >> 3) ^ (r & 7)) << 4));
 }
 
 __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdParams p)
@@ -117,7 +114,7 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
     using S = BcSmem;
     extern __shared__ __align__(1024) uint8_t sm[];
     const uint32_t sb = smem_u32(sm);
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
     const int unit = blockIdx.x >> 1, vc0 = (blockIdx.x & 1) * kBcCols;
     const int n = unit / p.HV, h = unit % p.HV;
     int64_t c_begin, row0;
@@ -133,9 +130,9 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
         row0 = static_cast<int64_t>(n) * p.T;
         len = p.T;
     }
-    float(*dS)[kBcCols] = reinterpret_cast<float(*)[kBcCols]>(sm + S::DS);
-    float(*dO)[kBcCols] = reinterpret_cast<float(*)[kBcCols]>(sm + S::DO);
-    float(*dVn)[kBcCols] = reinterpret_cast<float(*)[kBcCols]>(sm + S::DVN);
+    __half *dSh = reinterpret_cast<__half *>(sm + S::DSH);
+    __half *dOh = reinterpret_cast<__half *>(sm + S::DOH);
+    __half *dVh = reinterpret_cast<__half *>(sm + S::DVH);
     volatile int *flag = reinterpret_cast<volatile int *>(sm + S::FLAG);
     const int64_t unit_off = (static_cast<int64_t>(n) * p.HV + h) * DK * DV;
 
@@ -155,46 +152,54 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
         fence_mbar_init();
         if (nck > 0) request(nck - 1, 0);
     }
-    // dS <- dht (or zero)
-    {
-        const int d = tid >> 2, c0 = 16 * (tid & 3);
+    // the warp's dS tile: keys 16 ms .. +15, value columns 32 nh .. +31 of this CTA's 64 (four n8 tiles)
+    const int ms = warp & 7, nh = warp >> 3;
+    float acc[4][4];
+    auto key_of = [&](int half) { return 16 * ms + g + 8 * half; };
+    auto col_of = [&](int j, int e) { return 32 * nh + 8 * j + 2 * t4 + e; };
 #pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (p.dht) x = *reinterpret_cast<const float4 *>(p.dht + unit_off + d * DV + vc0 + c0 + e);
-            *reinterpret_cast<float4 *>(&dS[d][c0 + e]) = x;
-        }
-    }
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            acc[j][q] = p.dht ? p.dht[unit_off + key_of(q >> 1) * DV + vc0 + col_of(j, q & 1)] : 0.f;
+    auto store_dsh = [&]() {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+                *reinterpret_cast<__half2 *>(dSh + key_of(hf) * kBcPad + col_of(j, 0)) =
+                    __floats2half2_rn(acc[j][2 * hf], acc[j][2 * hf + 1]);
+    };
+    store_dsh();
     __syncthreads();
 
     bool ok = true;
     for (int it = 0; it < nck; ++it) {
         const int c = nck - 1 - it, st = it & 1;
-        const uint8_t *blk = sm + st * S::STAGE;
+        const uint32_t blk = sb + st * S::STAGE;
         if (tid == 0 && c > 0) request(c - 1, st ^ 1);  // that stage was released by the previous iteration
         const int nrows = min(CH, len - c * CH);
         {
             // dS is the gradient at chunk c's end state: store it
-            const int d = tid >> 2, c0 = 16 * (tid & 3);
-            float *dst = p.dstates + ((c_begin + c) * p.HV + h) * DK * DV + d * DV + vc0 + c0;
+            float *dst = p.dstates + ((c_begin + c) * p.HV + h) * DK * DV + vc0;
 #pragma unroll
-            for (int e = 0; e < 16; e += 4)
-                *reinterpret_cast<float4 *>(dst + e) = *reinterpret_cast<const float4 *>(&dS[d][c0 + e]);
-            // dO rows of the chunk (zero past the sequence's end)
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+                    *reinterpret_cast<float2 *>(dst + key_of(hf) * DV + col_of(j, 0)) =
+                        make_float2(acc[j][2 * hf], acc[j][2 * hf + 1]);
+            // dO rows of the chunk as fp16 (zero past the sequence's end)
             const int i = tid >> 3, cc = 8 * (tid & 7);
-            float x[8] = {};
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
             if (i < nrows) {
                 const uint4 raw = *reinterpret_cast<const uint4 *>(
                     p.dout + ((row0 + static_cast<int64_t>(c) * CH + i) * p.HV + h) * DV + vc0 + cc);
-                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    x[2 * e] = bf16lo(w[e]);
-                    x[2 * e + 1] = bf16hi(w[e]);
-                }
+                w.x = pack_f16(bf16lo(raw.x), bf16hi(raw.x));
+                w.y = pack_f16(bf16lo(raw.y), bf16hi(raw.y));
+                w.z = pack_f16(bf16lo(raw.z), bf16hi(raw.z));
+                w.w = pack_f16(bf16lo(raw.w), bf16hi(raw.w));
             }
-            *reinterpret_cast<float4 *>(&dO[i][cc]) = make_float4(x[0], x[1], x[2], x[3]);
-            *reinterpret_cast<float4 *>(&dO[i][cc + 4]) = make_float4(x[4], x[5], x[6], x[7]);
+            *reinterpret_cast<uint4 *>(dOh + i * kBcPad + cc) = w;
         }
         if (tid == 0) {
             const bool landed = mbar_wait(sb + S::BAR + 8 * st, waited[st] & 1);
@@ -206,63 +211,75 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
             ok = false;
             break;
         }
+        const uint32_t dsh = smem_u32(dSh), doh = smem_u32(dOh), dvh = smem_u32(dVh);
         {
-            // dVnew[i][cc..cc+7] = sum_d Kg[i][d] dS[d][.] + sum_{j >= i} Aqk[j][i] dO[j][.]
-            const int i = tid >> 3, cc = 8 * (tid & 7);
-            float acc[8] = {};
-            for (int d = 0; d < DK; ++d) {
-                const float kg = tile128_at(blk + ITEM_KG, i, d);
-                const float4 a = *reinterpret_cast<const float4 *>(&dS[d][cc]);
-                const float4 b = *reinterpret_cast<const float4 *>(&dS[d][cc + 4]);
-                acc[0] = __fmaf_rn(kg, a.x, acc[0]);
-                acc[1] = __fmaf_rn(kg, a.y, acc[1]);
-                acc[2] = __fmaf_rn(kg, a.z, acc[2]);
-                acc[3] = __fmaf_rn(kg, a.w, acc[3]);
-                acc[4] = __fmaf_rn(kg, b.x, acc[4]);
-                acc[5] = __fmaf_rn(kg, b.y, acc[5]);
-                acc[6] = __fmaf_rn(kg, b.z, acc[6]);
-                acc[7] = __fmaf_rn(kg, b.w, acc[7]);
+            // dVnew = Kg dS + Aqk^T dO; warp: tokens 16 mt .., columns 16 nq .. +15 (two n8 tiles)
+            const int mt = warp & 3, nq = warp >> 2;
+            float v[2][4] = {};
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                uint32_t a[4], b[4];
+                ldsm_x4(blk + ITEM_KG + sw_off128(16 * mt + (lane & 15), 16 * ks + (lane >> 4) * 8), a[0], a[1], a[2],
+                        a[3]);
+                ldsm_x4_t(dsh + 2 * ((16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8) * kBcPad + 16 * nq + (lane >> 4) * 8),
+                          b[0], b[1], b[2], b[3]);
+                mma_f16(v[0], a, b[0], b[1]);
+                mma_f16(v[1], a, b[2], b[3]);
             }
-            for (int j = i; j < CH; ++j) {
-                const float aq = tile64_at(blk + ITEM_AQK, j, i);
-                const float4 a = *reinterpret_cast<const float4 *>(&dO[j][cc]);
-                const float4 b = *reinterpret_cast<const float4 *>(&dO[j][cc + 4]);
-                acc[0] = __fmaf_rn(aq, a.x, acc[0]);
-                acc[1] = __fmaf_rn(aq, a.y, acc[1]);
-                acc[2] = __fmaf_rn(aq, a.z, acc[2]);
-                acc[3] = __fmaf_rn(aq, a.w, acc[3]);
-                acc[4] = __fmaf_rn(aq, b.x, acc[4]);
-                acc[5] = __fmaf_rn(aq, b.y, acc[5]);
-                acc[6] = __fmaf_rn(aq, b.z, acc[6]);
-                acc[7] = __fmaf_rn(aq, b.w, acc[7]);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                uint32_t a[4], b[4];
+                ldsm_x4_t(blk + ITEM_AQK + sw_off64(16 * ks + (lane & 7) + ((lane >> 4) & 1) * 8,
+                                                   16 * mt + ((lane >> 3) & 1) * 8),
+                          a[0], a[1], a[2], a[3]);
+                ldsm_x4_t(doh + 2 * ((16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8) * kBcPad + 16 * nq + (lane >> 4) * 8),
+                          b[0], b[1], b[2], b[3]);
+                mma_f16(v[0], a, b[0], b[1]);
+                mma_f16(v[1], a, b[2], b[3]);
             }
-            *reinterpret_cast<float4 *>(&dVn[i][cc]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            *reinterpret_cast<float4 *>(&dVn[i][cc + 4]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+                    *reinterpret_cast<__half2 *>(dVh + (16 * mt + g + 8 * hf) * kBcPad + 16 * nq + 8 * j + 2 * t4) =
+                        __floats2half2_rn(v[j][2 * hf], v[j][2 * hf + 1]);
         }
         __syncthreads();
         {
-            // dS[d][.] <- exp(G_L)_d dS[d][.] + sum_i Qg[i][d] dO[i][.] + sum_i (-W)[i][d] dVnew[i][.]
-            const int d = tid >> 2, c0 = 16 * (tid & 3);
-            const float e = reinterpret_cast<const float *>(blk + S::PART)[d];
-            float acc[16];
+            // dS <- exp(G_L) dS + Qg^T dO + (-W)^T dVnew
+            const float *egl = reinterpret_cast<const float *>(sm + st * S::STAGE + S::PART);
+            const float e0 = egl[key_of(0)], e1 = egl[key_of(1)];
 #pragma unroll
-            for (int x = 0; x < 16; ++x) acc[x] = __fmul_rn(e, dS[d][c0 + x]);
-            for (int i = 0; i < CH; ++i) {
-                const float qg = tile128_at(blk + ITEM_QG, i, d), wn = tile128_at(blk + ITEM_WN, i, d);
-#pragma unroll
-                for (int x = 0; x < 16; x += 4) {
-                    const float4 a = *reinterpret_cast<const float4 *>(&dO[i][c0 + x]);
-                    const float4 b = *reinterpret_cast<const float4 *>(&dVn[i][c0 + x]);
-                    acc[x] = __fmaf_rn(wn, b.x, __fmaf_rn(qg, a.x, acc[x]));
-                    acc[x + 1] = __fmaf_rn(wn, b.y, __fmaf_rn(qg, a.y, acc[x + 1]));
-                    acc[x + 2] = __fmaf_rn(wn, b.z, __fmaf_rn(qg, a.z, acc[x + 2]));
-                    acc[x + 3] = __fmaf_rn(wn, b.w, __fmaf_rn(qg, a.w, acc[x + 3]));
-                }
+            for (int j = 0; j < 4; ++j) {
+                acc[j][0] *= e0;
+                acc[j][1] *= e0;
+                acc[j][2] *= e1;
+                acc[j][3] *= e1;
             }
 #pragma unroll
-            for (int x = 0; x < 16; ++x) dS[d][c0 + x] = acc[x];
+            for (int ks = 0; ks < 4; ++ks) {
+                const int tr = 16 * ks + (lane & 7) + ((lane >> 4) & 1) * 8, kc = 16 * ms + ((lane >> 3) & 1) * 8;
+                const int br = 16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8;
+                uint32_t a[4], b[4], c2[4];
+                ldsm_x4_t(blk + ITEM_QG + sw_off128(tr, kc), a[0], a[1], a[2], a[3]);
+                ldsm_x4_t(doh + 2 * (br * kBcPad + 32 * nh + (lane >> 4) * 8), b[0], b[1], b[2], b[3]);
+                ldsm_x4_t(doh + 2 * (br * kBcPad + 32 * nh + 16 + (lane >> 4) * 8), c2[0], c2[1], c2[2], c2[3]);
+                mma_f16(acc[0], a, b[0], b[1]);
+                mma_f16(acc[1], a, b[2], b[3]);
+                mma_f16(acc[2], a, c2[0], c2[1]);
+                mma_f16(acc[3], a, c2[2], c2[3]);
+                ldsm_x4_t(blk + ITEM_WN + sw_off128(tr, kc), a[0], a[1], a[2], a[3]);
+                ldsm_x4_t(dvh + 2 * (br * kBcPad + 32 * nh + (lane >> 4) * 8), b[0], b[1], b[2], b[3]);
+                ldsm_x4_t(dvh + 2 * (br * kBcPad + 32 * nh + 16 + (lane >> 4) * 8), c2[0], c2[1], c2[2], c2[3]);
+                mma_f16(acc[0], a, b[0], b[1]);
+                mma_f16(acc[1], a, b[2], b[3]);
+                mma_f16(acc[2], a, c2[0], c2[1]);
+                mma_f16(acc[3], a, c2[2], c2[3]);
+            }
         }
-        __syncthreads();  // dS complete; this stage, dO and dVnew are free
+        __syncthreads();  // every read of dS's fp16 copy, dO, dVnew and the stage is done
+        store_dsh();
+        // (the next iteration's barrier orders these writes before their reads)
     }
     if (!ok) {
         if (tid == 0) {
@@ -276,11 +293,12 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
         return;
     }
     if (p.dh0) {
-        const int d = tid >> 2, c0 = 16 * (tid & 3);
 #pragma unroll
-        for (int e = 0; e < 16; e += 4)
-            *reinterpret_cast<float4 *>(p.dh0 + unit_off + d * DV + vc0 + c0 + e) =
-                *reinterpret_cast<const float4 *>(&dS[d][c0 + e]);
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+                *reinterpret_cast<float2 *>(p.dh0 + unit_off + key_of(hf) * DV + vc0 + col_of(j, 0)) =
+                    make_float2(acc[j][2 * hf], acc[j][2 * hf + 1]);
     }
 }
 
@@ -308,15 +326,17 @@ struct BwSmem {
     static constexpr int DGL = EGL + 512;                 // [128] gradient at G_L
     static constexpr int DBETA = DGL + 512;               // [64]
     static constexpr int WK = DBETA + 256;                // work region
-    // V pass buffers (inside WK)
-    static constexpr int SVT = WK;                        // [8][kSt]  S[:, cols]^T
-    static constexpr int DST = SVT + kBwCols * kSt * 4;   // [8][kSt]  dS'[:, cols]^T
-    static constexpr int DOV = DST + kBwCols * kSt * 4;   // [64][kVl] dO
-    static constexpr int DD = DOV + CH * kVl * 4;         // [64][kVl] D = v - Kb S
+    // V pass buffers (inside WK); S, dS' and dO columns are double-buffered (cp.async, one pass ahead)
+    static constexpr int SV = WK;                         // [2][128][8]  S[:, cols]
+    static constexpr int DSV = SV + 2 * DK * kBwCols * 4; // [2][128][8]  dS'[:, cols]
+    static constexpr int DOB = DSV + 2 * DK * kBwCols * 4;  // bf16 [2][64][8] dO
+    static constexpr int DD = DOB + 2 * CH * kBwCols * 2; // [64][kVl] D = v - Kb S
     static constexpr int VN = DD + CH * kVl * 4;          // [64][kVl] Vnew
     static constexpr int DVN = VN + CH * kVl * 4;         // [64][kVl] dVnew
     static constexpr int DV = DVN + CH * kVl * 4;         // [64][kVl] dv
     static constexpr int WK_END = DV + CH * kVl * 4;
+    // phase-3 use of WK: the off-diagonal products of the blocked solve, up to 3 x [16][16]
+    static constexpr int XS = WK;
     // phase-6 use of WK: dA, then Y = T^T dA diag(beta)
     static constexpr int DA = WK;                         // [64][kRowC]
     static constexpr int TOTAL = (WK_END > DA + CH * kRowC * 4 ? WK_END : DA + CH * kRowC * 4);
@@ -356,6 +376,17 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     const int64_t item = static_cast<int64_t>(chunk) * p.HV + h;
 
     // ---- 1. gates: G = cumulative g, block references, beta ----
+    // this warp's eight q and k rows, requested first so that their latency overlaps the gate work
+    uint2 rqv[CH / 8], rkv[CH / 8];
+#pragma unroll
+    for (int m = 0; m < CH / 8; ++m) {
+        const int r = warp + 8 * m;
+        rqv[m] = rkv[m] = make_uint2(0u, 0u);
+        if (r < nvalid) {
+            rqv[m] = *reinterpret_cast<const uint2 *>(p.q + ((row0 + r) * p.H + hq) * DK + 4 * lane);
+            rkv[m] = *reinterpret_cast<const uint2 *>(p.k + ((row0 + r) * p.H + hq) * DK + 4 * lane);
+        }
+    }
     {
         const int i = tid >> 2, c0 = 32 * (tid & 3);
         const float *gr = p.g + ((row0 + i) * p.HV + h) * DK + c0;
@@ -392,15 +423,13 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     }
     __syncthreads();
     // ---- normalised q/k rows and the gate-scaled operands ----
-    for (int r = warp; r < CH; r += kBwThreads / 32) {
-        uint2 rq = make_uint2(0u, 0u), rk = make_uint2(0u, 0u);
-        if (r < nvalid) {
-            rq = *reinterpret_cast<const uint2 *>(p.q + ((row0 + r) * p.H + hq) * DK + 4 * lane);
-            rk = *reinterpret_cast<const uint2 *>(p.k + ((row0 + r) * p.H + hq) * DK + 4 * lane);
-        }
-        const uint2 nq = l2norm_row128_warp(rq), nk = l2norm_row128_warp(rk);
+#pragma unroll
+    for (int m = 0; m < CH / 8; ++m) {
+        const int r = warp + 8 * m;
+        const uint2 rq = rqv[m], rk = rkv[m];
         // the forward's row denominators, kept to rebuild qn/kn bit for bit at the end
         const float dq = l2norm_den128_warp(rq), dk = l2norm_den128_warp(rk);
+        const uint2 nq = l2norm_apply128(rq, dq), nk = l2norm_apply128(rk, dk);
         if (lane == 0) {
             denq[r] = dq;
             denk[r] = dk;
@@ -468,159 +497,205 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     }
     __syncthreads();
 
-    // ---- 3. T = (I + diag(beta) P)^-1, right-looking: row k is final before step k ----
-    for (int k = 0; k < CH - 1; ++k) {
-        const int rows = CH - 1 - k, cols = k + 1;
-        for (int x = tid; x < rows * cols; x += kBwThreads) {
-            const int i = k + 1 + x / cols, j = x % cols;
-            TT[i][j] = __fmaf_rn(-__fmul_rn(beta[i], PP[i][k]), TT[k][j], TT[i][j]);
+    // ---- 3. T = (I + diag(beta) P)^-1 in 16 x 16 blocks: the four diagonal blocks right-looking side by side,
+    //         then T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ by distance I - J ----
+    {
+        const int I = tid >> 6, pidx = tid & 63;
+        for (int k = 0; k < 15; ++k) {
+            const int cols = k + 1;
+            if (pidx < (15 - k) * cols) {
+                const int i = 16 * I + k + 1 + pidx / cols, j = 16 * I + pidx % cols, kk = 16 * I + k;
+                TT[i][j] = __fmaf_rn(-__fmul_rn(beta[i], PP[i][kk]), TT[kk][j], TT[i][j]);
+            }
+            __syncthreads();
         }
-        __syncthreads();
+        float(*X)[16][17] = reinterpret_cast<float(*)[16][17]>(sm + S::XS);
+        for (int dist = 1; dist < 4; ++dist) {
+            const int pairs = 4 - dist;  // blocks (I, J) = (J + dist, J), J = 0 .. pairs - 1
+            for (int x = tid; x < pairs * 256; x += kBwThreads) {
+                const int J = x >> 8, i = (x >> 4) & 15, j = x & 15, Ib = J + dist;
+                float acc = 0.f;
+                for (int kk = 16 * J; kk < 16 * Ib; ++kk) acc = __fmaf_rn(PP[16 * Ib + i][kk], TT[kk][16 * J + j], acc);
+                X[J][i][j] = __fmul_rn(beta[16 * Ib + i], acc);
+            }
+            __syncthreads();
+            for (int x = tid; x < pairs * 256; x += kBwThreads) {
+                const int J = x >> 8, i = (x >> 4) & 15, j = x & 15, Ib = J + dist;
+                float acc = 0.f;
+                for (int kk = 0; kk <= i; ++kk) acc = __fmaf_rn(TT[16 * Ib + i][16 * Ib + kk], X[J][kk][j], acc);
+                TT[16 * Ib + i][16 * J + j] = -acc;
+            }
+            __syncthreads();
+        }
     }
 
-    // ---- 4-5. passes over 8 value columns at a time ----
-    float(*SVT)[kSt] = reinterpret_cast<float(*)[kSt]>(sm + S::SVT);
-    float(*DST)[kSt] = reinterpret_cast<float(*)[kSt]>(sm + S::DST);
-    float(*DOV)[kVl] = reinterpret_cast<float(*)[kVl]>(sm + S::DOV);
+    // ---- 4-5. passes over 8 value columns at a time, on TF32 tensor-core MMAs (m16n8k8, fp32 accumulate) ----
+    // S, dS' [128][8] and dO [64][8] (bf16) of the current pass, the next pass's in the other buffer
+    auto SVb = [&](int b) { return reinterpret_cast<float(*)[kBwCols]>(sm + S::SV + b * DK * kBwCols * 4); };
+    auto DSVb = [&](int b) { return reinterpret_cast<float(*)[kBwCols]>(sm + S::DSV + b * DK * kBwCols * 4); };
+    auto DOBb = [&](int b) { return reinterpret_cast<__nv_bfloat16(*)[kBwCols]>(sm + S::DOB + b * CH * kBwCols * 2); };
     float(*DDv)[kVl] = reinterpret_cast<float(*)[kVl]>(sm + S::DD);
     float(*VN)[kVl] = reinterpret_cast<float(*)[kVl]>(sm + S::VN);
     float(*DVN)[kVl] = reinterpret_cast<float(*)[kVl]>(sm + S::DVN);
     float(*DVv)[kVl] = reinterpret_cast<float(*)[kVl]>(sm + S::DV);
     const float *Sg = p.states + item * DK * DV;
     const float *dSg = p.dstates + item * DK * DV;
-    // register accumulators over the value columns: thread rows 4rg..+3, key columns 8cg..+7 (dQg, dKb, dKg)
-    // and rows 4rg..+3, token columns cg + 16jb (dAqk, dA)
-    const int rg = tid >> 4, cg = tid & 15;
-    float aQ[4][8] = {}, aB[4][8] = {}, aG[4][8] = {}, aAq[4][4] = {}, aA[4][4] = {};
+    const int rg = tid >> 4, cg = tid & 15;  // ownership of the 64 x 64 steps of phase 6
+    // MMA fragment ownership (g = lane / 4, t4 = lane % 4): warp (mt, nh) holds rows 16 mt + g and + 8, and key
+    // columns 64 nh + 8 j + 2 t4 (+1), j = 0..7 (dQg, dKb, dKg), or token columns 32 nh + 8 j + 2 t4 (+1),
+    // j = 0..3 (dAqk, dA)
+    const int g = lane >> 2, t4 = lane & 3, mt = warp & 3, nh = warp >> 2;
+    const int r0 = 16 * mt + g, r1 = r0 + 8;
+    float aQ[8][4] = {}, aB[8][4] = {}, aG[8][4] = {}, aAq[4][4] = {}, aA[4][4] = {};
+    // pass vb's columns into buffer b: S and dS' rows are 32 bytes (two 16-byte copies each), dO rows 16 bytes
+    auto fetch = [&](int vb, int b) {
+        const int row = tid >> 1, half = 4 * (tid & 1);
+        cp_async16(smem_u32(&SVb(b)[row][half]), Sg + row * DV + vb + half);
+        cp_async16(smem_u32(&DSVb(b)[row][half]), dSg + row * DV + vb + half);
+        if (tid < nvalid) cp_async16(smem_u32(&DOBb(b)[tid][0]), p.dout + ((row0 + tid) * p.HV + h) * DV + vb);
+        cp_async_commit();
+    };
+    if (tid < CH && tid >= nvalid) {  // rows past the end stay zero in both buffers
+        *reinterpret_cast<uint4 *>(&DOBb(0)[tid][0]) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4 *>(&DOBb(1)[tid][0]) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fetch(0, 0);
+    float gl_acc = 0.f;  // thread d < 128: sum over all columns of S[d][.] dS'[d][.]
     for (int vb = 0; vb < DV; vb += kBwCols) {
-        {
-            // S and dS' columns vb..vb+7, transposed; thread: key row d = tid >> 1, 4 columns
-            const int d = tid >> 1, c4 = 4 * (tid & 1);
-            const float4 x = *reinterpret_cast<const float4 *>(Sg + d * DV + vb + c4);
-            const float4 y = *reinterpret_cast<const float4 *>(dSg + d * DV + vb + c4);
-            SVT[c4][d] = x.x;
-            SVT[c4 + 1][d] = x.y;
-            SVT[c4 + 2][d] = x.z;
-            SVT[c4 + 3][d] = x.w;
-            DST[c4][d] = y.x;
-            DST[c4 + 1][d] = y.y;
-            DST[c4 + 2][d] = y.z;
-            DST[c4 + 3][d] = y.w;
-            // dE_L term of dG_L: sum over these columns of exp(G_L) S dS'
-            const float part = __fmaf_rn(x.w, y.w, __fmaf_rn(x.z, y.z, __fmaf_rn(x.y, y.y, __fmul_rn(x.x, y.x))));
-            atomicAdd(&dgl[d], __fmul_rn(egl[d], part));
-            // dO rows (zero past the end)
-            if (tid < 2 * CH) {
-                const int i = tid >> 1, cc = 4 * (tid & 1);
-                float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (i < nvalid) {
-                    const uint2 raw = *reinterpret_cast<const uint2 *>(p.dout + ((row0 + i) * p.HV + h) * DV + vb + cc);
-                    o = make_float4(bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y));
-                }
-                *reinterpret_cast<float4 *>(&DOV[i][cc]) = o;
+        const int buf = (vb / kBwCols) & 1;
+        if (vb + kBwCols < DV) {
+            fetch(vb + kBwCols, buf ^ 1);  // that buffer was released by the previous pass's last barrier
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        float(*SVT)[kBwCols] = SVb(buf);
+        float(*DST)[kBwCols] = DSVb(buf);
+        const __nv_bfloat16(*DOV)[kBwCols] = DOBb(buf);
+        if (tid < DK) {
+            const float4 x0 = *reinterpret_cast<const float4 *>(&SVT[tid][0]), x1 = *reinterpret_cast<const float4 *>(&SVT[tid][4]);
+            const float4 y0 = *reinterpret_cast<const float4 *>(&DST[tid][0]), y1 = *reinterpret_cast<const float4 *>(&DST[tid][4]);
+            gl_acc = __fmaf_rn(x0.x, y0.x, gl_acc);
+            gl_acc = __fmaf_rn(x0.y, y0.y, gl_acc);
+            gl_acc = __fmaf_rn(x0.z, y0.z, gl_acc);
+            gl_acc = __fmaf_rn(x0.w, y0.w, gl_acc);
+            gl_acc = __fmaf_rn(x1.x, y1.x, gl_acc);
+            gl_acc = __fmaf_rn(x1.y, y1.y, gl_acc);
+            gl_acc = __fmaf_rn(x1.z, y1.z, gl_acc);
+            gl_acc = __fmaf_rn(x1.w, y1.w, gl_acc);
+        }
+        if (warp < 4) {
+            // (a) D = v - Kb S for rows 16 mt .. (Kb = KA exp(m_I), block I = mt)
+            float c[4] = {};
+            for (int ks = 0; ks < DK; ks += 8) {
+                const float e0 = EM[mt][ks + t4], e1 = EM[mt][ks + t4 + 4];
+                const uint32_t a[4] = {to_tf32(__fmul_rn(KA[r0][ks + t4], e0)), to_tf32(__fmul_rn(KA[r1][ks + t4], e0)),
+                                       to_tf32(__fmul_rn(KA[r0][ks + t4 + 4], e1)),
+                                       to_tf32(__fmul_rn(KA[r1][ks + t4 + 4], e1))};
+                mma_tf32(c, a, to_tf32(SVT[ks + t4][g]), to_tf32(SVT[ks + t4 + 4][g]));
+            }
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int i = hf ? r1 : r0;
+                float2 vv = make_float2(0.f, 0.f);
+                if (i < nvalid)
+                    vv = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162 *>(p.v + ((row0 + i) * p.HV + h) * DV + vb + 2 * t4));
+                *reinterpret_cast<float2 *>(&DDv[i][2 * t4]) =
+                    make_float2(__fsub_rn(vv.x, c[2 * hf]), __fsub_rn(vv.y, c[2 * hf + 1]));
+            }
+        } else {
+            // (c) dVnew = Kg dS' + Aqk^T dO for rows 16 mt .. (Kg = KB exp(G_L - m_I))
+            float c[4] = {};
+            for (int ks = 0; ks < DK; ks += 8) {
+                const float e0 = EGLM[mt][ks + t4], e1 = EGLM[mt][ks + t4 + 4];
+                const uint32_t a[4] = {to_tf32(__fmul_rn(KB[r0][ks + t4], e0)), to_tf32(__fmul_rn(KB[r1][ks + t4], e0)),
+                                       to_tf32(__fmul_rn(KB[r0][ks + t4 + 4], e1)),
+                                       to_tf32(__fmul_rn(KB[r1][ks + t4 + 4], e1))};
+                mma_tf32(c, a, to_tf32(DST[ks + t4][g]), to_tf32(DST[ks + t4 + 4][g]));
+            }
+            for (int js = 16 * mt; js < CH; js += 8) {  // Aqk^T[i][j] = Aqk[j][i], nonzero for j >= i
+                const uint32_t a[4] = {to_tf32(AQ[js + t4][r0]), to_tf32(AQ[js + t4][r1]), to_tf32(AQ[js + t4 + 4][r0]),
+                                       to_tf32(AQ[js + t4 + 4][r1])};
+                mma_tf32(c, a, to_tf32(__bfloat162float(DOV[js + t4][g])), to_tf32(__bfloat162float(DOV[js + t4 + 4][g])));
+            }
+            *reinterpret_cast<float2 *>(&DVN[r0][2 * t4]) = make_float2(c[0], c[1]);
+            *reinterpret_cast<float2 *>(&DVN[r1][2 * t4]) = make_float2(c[2], c[3]);
+        }
+        __syncthreads();
+        if (warp < 4) {
+            // (b) Vnew = T diag(beta) D (T lower triangular: j < 16 (mt + 1))
+            float c[4] = {};
+            for (int js = 0; js < 16 * (mt + 1); js += 8) {
+                const float b0 = beta[js + t4], b1 = beta[js + t4 + 4];
+                const uint32_t a[4] = {to_tf32(__fmul_rn(TT[r0][js + t4], b0)), to_tf32(__fmul_rn(TT[r1][js + t4], b0)),
+                                       to_tf32(__fmul_rn(TT[r0][js + t4 + 4], b1)),
+                                       to_tf32(__fmul_rn(TT[r1][js + t4 + 4], b1))};
+                mma_tf32(c, a, to_tf32(DDv[js + t4][g]), to_tf32(DDv[js + t4 + 4][g]));
+            }
+            *reinterpret_cast<float2 *>(&VN[r0][2 * t4]) = make_float2(c[0], c[1]);
+            *reinterpret_cast<float2 *>(&VN[r1][2 * t4]) = make_float2(c[2], c[3]);
+        } else {
+            // (d) dv = diag(beta) T^T dVnew (j >= i)
+            float c[4] = {};
+            for (int js = 16 * mt; js < CH; js += 8) {
+                const uint32_t a[4] = {to_tf32(TT[js + t4][r0]), to_tf32(TT[js + t4][r1]), to_tf32(TT[js + t4 + 4][r0]),
+                                       to_tf32(TT[js + t4 + 4][r1])};
+                mma_tf32(c, a, to_tf32(DVN[js + t4][g]), to_tf32(DVN[js + t4 + 4][g]));
+            }
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int i = hf ? r1 : r0;
+                const float x0 = __fmul_rn(beta[i], c[2 * hf]), x1 = __fmul_rn(beta[i], c[2 * hf + 1]);
+                *reinterpret_cast<float2 *>(&DVv[i][2 * t4]) = make_float2(x0, x1);
+                if (i < nvalid)
+                    *reinterpret_cast<__nv_bfloat162 *>(p.dv + ((row0 + i) * p.HV + h) * DV + vb + 2 * t4) =
+                        __floats2bfloat162_rn(x0, x1);
             }
         }
         __syncthreads();
         {
-            // (a) D[i][c] = v[i][c] - sum_d Kb_id S[d][c], Kb = KA exp(m_I); thread: row i = tid >> 2, 2 columns
-            const int i = tid >> 2, c2 = 2 * (tid & 3), I = i >> 4;
-            float a0 = 0.f, a1 = 0.f;
-            for (int d = 0; d < DK; ++d) {
-                const float kb = __fmul_rn(KA[i][d], EM[I][d]);
-                a0 = __fmaf_rn(kb, SVT[c2][d], a0);
-                a1 = __fmaf_rn(kb, SVT[c2 + 1][d], a1);
-            }
-            float v0 = 0.f, v1 = 0.f;
-            if (i < nvalid) {
-                const __nv_bfloat162 vv =
-                    *reinterpret_cast<const __nv_bfloat162 *>(p.v + ((row0 + i) * p.HV + h) * DV + vb + c2);
-                v0 = __low2float(vv);
-                v1 = __high2float(vv);
-            }
-            DDv[i][c2] = __fsub_rn(v0, a0);
-            DDv[i][c2 + 1] = __fsub_rn(v1, a1);
-        }
-        __syncthreads();
-        {
-            // (b) Vnew = T diag(beta) D;  (c) dVnew = Kg dS' + Aqk^T dO, Kg = KB exp(G_L - m_I)
-            const int i = tid >> 2, c2 = 2 * (tid & 3), I = i >> 4;
-            float x0 = 0.f, x1 = 0.f;
-            for (int j = 0; j <= i; ++j) {
-                const float t = __fmul_rn(TT[i][j], beta[j]);
-                x0 = __fmaf_rn(t, DDv[j][c2], x0);
-                x1 = __fmaf_rn(t, DDv[j][c2 + 1], x1);
-            }
-            VN[i][c2] = x0;
-            VN[i][c2 + 1] = x1;
-            float y0 = 0.f, y1 = 0.f;
-            for (int d = 0; d < DK; ++d) {
-                const float kg = __fmul_rn(KB[i][d], EGLM[I][d]);
-                y0 = __fmaf_rn(kg, DST[c2][d], y0);
-                y1 = __fmaf_rn(kg, DST[c2 + 1][d], y1);
-            }
-            for (int j = i; j < CH; ++j) {
-                y0 = __fmaf_rn(AQ[j][i], DOV[j][c2], y0);
-                y1 = __fmaf_rn(AQ[j][i], DOV[j][c2 + 1], y1);
-            }
-            DVN[i][c2] = y0;
-            DVN[i][c2 + 1] = y1;
-        }
-        __syncthreads();
-        {
-            // (d) dv = diag(beta) T^T dVnew
-            const int i = tid >> 2, c2 = 2 * (tid & 3);
-            float x0 = 0.f, x1 = 0.f;
-            for (int j = i; j < CH; ++j) {
-                x0 = __fmaf_rn(TT[j][i], DVN[j][c2], x0);
-                x1 = __fmaf_rn(TT[j][i], DVN[j][c2 + 1], x1);
-            }
-            x0 = __fmul_rn(beta[i], x0);
-            x1 = __fmul_rn(beta[i], x1);
-            DVv[i][c2] = x0;
-            DVv[i][c2 + 1] = x1;
-            if (i < nvalid)
-                *reinterpret_cast<__nv_bfloat162 *>(p.dv + ((row0 + i) * p.HV + h) * DV + vb + c2) =
-                    __floats2bfloat162_rn(x0, x1);
-        }
-        __syncthreads();
-        // (e) accumulate dQg += dO S^T, dKb -= dv S^T, dKg += Vnew dS'^T, dAqk += dO Vnew^T, dA += dVnew D^T
+            // (e) dQg += dO S^T, dKb -= dv S^T, dKg += Vnew dS'^T (K = these 8 columns); dAqk += dO Vnew^T,
+            //     dA += dVnew D^T
+            const uint32_t aO[4] = {to_tf32(__bfloat162float(DOV[r0][t4])), to_tf32(__bfloat162float(DOV[r1][t4])),
+                                    to_tf32(__bfloat162float(DOV[r0][t4 + 4])), to_tf32(__bfloat162float(DOV[r1][t4 + 4]))};
+            const uint32_t aV[4] = {to_tf32(-DVv[r0][t4]), to_tf32(-DVv[r1][t4]), to_tf32(-DVv[r0][t4 + 4]),
+                                    to_tf32(-DVv[r1][t4 + 4])};
+            const uint32_t aN[4] = {to_tf32(VN[r0][t4]), to_tf32(VN[r1][t4]), to_tf32(VN[r0][t4 + 4]),
+                                    to_tf32(VN[r1][t4 + 4])};
+            const uint32_t aD[4] = {to_tf32(DVN[r0][t4]), to_tf32(DVN[r1][t4]), to_tf32(DVN[r0][t4 + 4]),
+                                    to_tf32(DVN[r1][t4 + 4])};
 #pragma unroll
-        for (int c = 0; c < kBwCols; ++c) {
-            float sv[8], dsv[8];
-            *reinterpret_cast<float4 *>(&sv[0]) = *reinterpret_cast<const float4 *>(&SVT[c][8 * cg]);
-            *reinterpret_cast<float4 *>(&sv[4]) = *reinterpret_cast<const float4 *>(&SVT[c][8 * cg + 4]);
-            *reinterpret_cast<float4 *>(&dsv[0]) = *reinterpret_cast<const float4 *>(&DST[c][8 * cg]);
-            *reinterpret_cast<float4 *>(&dsv[4]) = *reinterpret_cast<const float4 *>(&DST[c][8 * cg + 4]);
+            for (int j = 0; j < 8; ++j) {
+                const int d = 64 * nh + 8 * j + g;
+                const uint32_t s0 = to_tf32(SVT[d][t4]), s1 = to_tf32(SVT[d][t4 + 4]);
+                const uint32_t q0 = to_tf32(DST[d][t4]), q1 = to_tf32(DST[d][t4 + 4]);
+                mma_tf32(aQ[j], aO, s0, s1);
+                mma_tf32(aB[j], aV, s0, s1);
+                mma_tf32(aG[j], aN, q0, q1);
+            }
 #pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
-                const int i = 4 * rg + ii;
-                const float o = DOV[i][c], dv_ = DVv[i][c], vn = VN[i][c], dvn = DVN[i][c];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    aQ[ii][e] = __fmaf_rn(o, sv[e], aQ[ii][e]);
-                    aB[ii][e] = __fmaf_rn(-dv_, sv[e], aB[ii][e]);
-                    aG[ii][e] = __fmaf_rn(vn, dsv[e], aG[ii][e]);
-                }
-#pragma unroll
-                for (int jb = 0; jb < 4; ++jb) {
-                    const int j = cg + 16 * jb;
-                    aAq[ii][jb] = __fmaf_rn(o, VN[j][c], aAq[ii][jb]);
-                    aA[ii][jb] = __fmaf_rn(dvn, DDv[j][c], aA[ii][jb]);
-                }
+            for (int j = 0; j < 4; ++j) {
+                const int tk = 32 * nh + 8 * j + g;
+                mma_tf32(aAq[j], aO, to_tf32(VN[tk][t4]), to_tf32(VN[tk][t4 + 4]));
+                mma_tf32(aA[j], aD, to_tf32(DDv[tk][t4]), to_tf32(DDv[tk][t4 + 4]));
             }
         }
         __syncthreads();
     }
 
+    if (tid < DK) dgl[tid] = __fmaf_rn(egl[tid], gl_acc, dgl[tid]);  // the exp(G_L) S dS' term of dG_L
+
     // ---- 6. dbeta, dL, M = diag(beta) dL, N = dAqk ----
     float(*DA)[kRowC] = reinterpret_cast<float(*)[kRowC]>(sm + S::DA);
 #pragma unroll
-    for (int ii = 0; ii < 4; ++ii)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
-        for (int jb = 0; jb < 4; ++jb) {
-            const int i = 4 * rg + ii, j = cg + 16 * jb;
-            DA[i][j] = aA[ii][jb];
-            AQ[i][j] = j <= i ? aAq[ii][jb] : 0.f;  // Aqk is no longer needed: N takes its place
+        for (int q = 0; q < 4; ++q) {
+            const int i = (q >> 1) ? r1 : r0, tk = 32 * nh + 8 * j + 2 * t4 + (q & 1);
+            DA[i][tk] = aA[j][q];
+            AQ[i][tk] = tk <= i ? aAq[j][q] : 0.f;  // Aqk is no longer needed: N takes its place
         }
     __syncthreads();
     if (tid < CH) {  // dbeta_j += sum_{i >= j} dA_ij T_ij
@@ -687,167 +762,151 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     float(*MM)[kRowC] = PP;
     float(*NN)[kRowC] = AQ;
 
-    // ---- 7. element terms and pairwise terms; thread: rows 4rg..+3 (block I), key columns 8cg..+7 ----
-    const int I = rg >> 2;
-    float rq[4][8], rk[4][8], rG[4][8];
+    // ---- 7. element terms and pairwise terms, in the fragment ownership of phase 5 ----
+    float rq[8][4], rk[8][4], rG[8][4];
     {
-        // rebuild qn/kn of the owned rows from the raw rows (the same normalisation, bit for bit)
-        float qn[4][8], kn[4][8];
+        // qn/kn of the owned elements, rebuilt from the raw rows (the same normalisation, bit for bit)
+        float glp[8][2] = {};
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-            const int i = 4 * rg + ii;
-            uint4 rqw = make_uint4(0u, 0u, 0u, 0u), rkw = rqw;
-            if (i < nvalid) {
-                rqw = *reinterpret_cast<const uint4 *>(p.q + ((row0 + i) * p.H + hq) * DK + 8 * cg);
-                rkw = *reinterpret_cast<const uint4 *>(p.k + ((row0 + i) * p.H + hq) * DK + 8 * cg);
-            }
-            const uint32_t wq[4] = {rqw.x, rqw.y, rqw.z, rqw.w}, wk[4] = {rkw.x, rkw.y, rkw.z, rkw.w};
+        for (int hf = 0; hf < 2; ++hf) {
+            const int i = hf ? r1 : r0;
+            const float dq = denq[i], dk = denk[i], rqi = __frcp_rn(dq), rki = __frcp_rn(dk);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                qn[ii][2 * e] = bf16lo(wq[e]);
-                qn[ii][2 * e + 1] = bf16hi(wq[e]);
-                kn[ii][2 * e] = bf16lo(wk[e]);
-                kn[ii][2 * e + 1] = bf16hi(wk[e]);
-            }
-        }
-        // the quotient and rounding of the normalisation, with the row denominators stored above
+            for (int j = 0; j < 8; ++j) {
+                const int d = 64 * nh + 8 * j + 2 * t4;
+                uint32_t wq = 0u, wk = 0u;
+                if (i < nvalid) {
+                    wq = *reinterpret_cast<const uint32_t *>(p.q + ((row0 + i) * p.H + hq) * DK + d);
+                    wk = *reinterpret_cast<const uint32_t *>(p.k + ((row0 + i) * p.H + hq) * DK + d);
+                }
+                const uint32_t pq = pack_bf16(div_rn_with_rcp(bf16lo(wq), dq, rqi), div_rn_with_rcp(bf16hi(wq), dq, rqi));
+                const uint32_t pk = pack_bf16(div_rn_with_rcp(bf16lo(wk), dk, rki), div_rn_with_rcp(bf16hi(wk), dk, rki));
+                const float qn[2] = {bf16lo(pq), bf16hi(pq)}, kn[2] = {bf16lo(pk), bf16hi(pk)};
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-            const float dq = denq[4 * rg + ii], dk = denk[4 * rg + ii];
-            const float rqi = __frcp_rn(dq), rki = __frcp_rn(dk);
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-                const uint32_t pq = pack_bf16(div_rn_with_rcp(qn[ii][e], dq, rqi), div_rn_with_rcp(qn[ii][e + 1], dq, rqi));
-                const uint32_t pk = pack_bf16(div_rn_with_rcp(kn[ii][e], dk, rki), div_rn_with_rcp(kn[ii][e + 1], dk, rki));
-                qn[ii][e] = bf16lo(pq);
-                qn[ii][e + 1] = bf16hi(pq);
-                kn[ii][e] = bf16lo(pk);
-                kn[ii][e + 1] = bf16hi(pk);
-            }
-        }
-        // X3 = s exp(G) dQg, X1 = exp(G) dKb, X2 = exp(G_L - G) dKg
-        float glp[8] = {};
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-            const int i = 4 * rg + ii;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int d = 8 * cg + e;
-                const float x = __fsub_rn(G[i][d], G[16 * I + 7][d]);
-                const float eg = __fmul_rn(bwd_exp(x), EM[I][d]), eglg = __fmul_rn(bwd_exp(-x), EGLM[I][d]);
-                const float x3 = __fmul_rn(__fmul_rn(s, eg), aQ[ii][e]);
-                const float x1 = __fmul_rn(eg, aB[ii][e]);
-                const float x2 = __fmul_rn(eglg, aG[ii][e]);
-                rq[ii][e] = x3;
-                rk[ii][e] = __fadd_rn(x1, x2);
-                rG[ii][e] = __fmaf_rn(qn[ii][e], x3, __fmul_rn(kn[ii][e], __fsub_rn(x1, x2)));
-                glp[e] = __fmaf_rn(kn[ii][e], x2, glp[e]);
+                for (int e = 0; e < 2; ++e) {
+                    const int q = 2 * hf + e, dd = d + e;
+                    // X3 = s exp(G) dQg, X1 = exp(G) dKb, X2 = exp(G_L - G) dKg
+                    const float x = __fsub_rn(G[i][dd], G[16 * mt + 7][dd]);
+                    const float eg = __fmul_rn(bwd_exp(x), EM[mt][dd]), eglg = __fmul_rn(bwd_exp(-x), EGLM[mt][dd]);
+                    const float x3 = __fmul_rn(__fmul_rn(s, eg), aQ[j][q]);
+                    const float x1 = __fmul_rn(eg, aB[j][q]);
+                    const float x2 = __fmul_rn(eglg, aG[j][q]);
+                    rq[j][q] = x3;
+                    rk[j][q] = __fadd_rn(x1, x2);
+                    rG[j][q] = __fmaf_rn(qn[e], x3, __fmul_rn(kn[e], __fsub_rn(x1, x2)));
+                    glp[j][e] = __fmaf_rn(kn[e], x2, glp[j][e]);
+                }
             }
         }
+        // dG_L += sum over rows of kn X2: the eight lanes g of a column, then the warps of the other row blocks
 #pragma unroll
-        for (int e = 0; e < 8; ++e) atomicAdd(&dgl[8 * cg + e], glp[e]);
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float x = glp[j][e];
+                x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, 4));
+                x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, 8));
+                x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, 16));
+                if (g == 0) atomicAdd(&dgl[64 * nh + 8 * j + 2 * t4 + e], x);
+            }
     }
     {
-        // R1'_id = sum_{J <= I} sum_{j in J} M_ij KB_jd c_IJd,  R3'_id = the same with N
-        float r1[4][8] = {}, r3[4][8] = {};
-        for (int J = 0; J <= I; ++J) {
-            for (int j = 16 * J; j < 16 * J + 16; ++j) {
-                float kb[8];
-                *reinterpret_cast<float4 *>(&kb[0]) = *reinterpret_cast<const float4 *>(&KB[j][8 * cg]);
-                *reinterpret_cast<float4 *>(&kb[4]) = *reinterpret_cast<const float4 *>(&KB[j][8 * cg + 4]);
-                if (J < I) {
+        // R1'_id = sum_{J <= I} sum_{j in J} M_ij KB_jd c_IJd and R3' the same with N (I = mt)
+        float ra[8][4] = {}, rb[8][4] = {};
+        for (int J = 0; J <= mt; ++J) {
+            const float *cf = J < mt ? CF[cf_index(mt, J)] : nullptr;
+            for (int ks = 16 * J; ks < 16 * J + 16; ks += 8) {
+                const uint32_t am[4] = {to_tf32(MM[r0][ks + t4]), to_tf32(MM[r1][ks + t4]), to_tf32(MM[r0][ks + t4 + 4]),
+                                        to_tf32(MM[r1][ks + t4 + 4])};
+                const uint32_t an[4] = {to_tf32(NN[r0][ks + t4]), to_tf32(NN[r1][ks + t4]), to_tf32(NN[r0][ks + t4 + 4]),
+                                        to_tf32(NN[r1][ks + t4 + 4])};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) kb[e] = __fmul_rn(kb[e], CF[cf_index(I, J)][8 * cg + e]);
-                }
-#pragma unroll
-                for (int ii = 0; ii < 4; ++ii) {
-                    const float m = MM[4 * rg + ii][j], nn = NN[4 * rg + ii][j];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        r1[ii][e] = __fmaf_rn(m, kb[e], r1[ii][e]);
-                        r3[ii][e] = __fmaf_rn(nn, kb[e], r3[ii][e]);
+                for (int j = 0; j < 8; ++j) {
+                    const int d = 64 * nh + 8 * j + g;
+                    float b0 = KB[ks + t4][d], b1 = KB[ks + t4 + 4][d];
+                    if (cf) {
+                        b0 = __fmul_rn(b0, cf[d]);
+                        b1 = __fmul_rn(b1, cf[d]);
                     }
+                    const uint32_t u0 = to_tf32(b0), u1 = to_tf32(b1);
+                    mma_tf32(ra[j], am, u0, u1);
+                    mma_tf32(rb[j], an, u0, u1);
                 }
             }
         }
-        // R1 = a R1', R3 = s a R3' with a = exp(G - m_I); dkn += R1, dqn += R3, dG += kn R1 + qn R3
+        // R1 = a R1', R3 = s a R3' (a = exp(G - m_I)): dkn += R1, dqn += R3, dG += kn R1 + qn R3
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-            const int i = 4 * rg + ii;
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int d = 8 * cg + e;
-                const float a = bwd_exp(__fsub_rn(G[i][d], G[16 * I + 7][d]));
-                const float R1 = __fmul_rn(a, r1[ii][e]), R3 = __fmul_rn(__fmul_rn(s, a), r3[ii][e]);
-                rk[ii][e] = __fadd_rn(rk[ii][e], R1);
-                rq[ii][e] = __fadd_rn(rq[ii][e], R3);
-                rG[ii][e] = __fmaf_rn(KA[i][d], r1[ii][e], rG[ii][e]);
-                rG[ii][e] = __fmaf_rn(__fmul_rn(s, QA[i][d]), r3[ii][e], rG[ii][e]);
+            for (int q = 0; q < 4; ++q) {
+                const int i = (q >> 1) ? r1 : r0, d = 64 * nh + 8 * j + 2 * t4 + (q & 1);
+                const float a = bwd_exp(__fsub_rn(G[i][d], G[16 * mt + 7][d]));
+                rk[j][q] = __fmaf_rn(a, ra[j][q], rk[j][q]);
+                rq[j][q] = __fmaf_rn(__fmul_rn(s, a), rb[j][q], rq[j][q]);
+                rG[j][q] = __fmaf_rn(KA[i][d], ra[j][q], rG[j][q]);
+                rG[j][q] = __fmaf_rn(__fmul_rn(s, QA[i][d]), rb[j][q], rG[j][q]);
             }
-        }
     }
     {
-        // R24'_jd = sum_{I' >= J} sum_{i in I'} (M_ij KA_id + s N_ij QA_id) c_I'Jd  (rows j = 4rg..+3, J = I)
-        float r2[4][8] = {};
-        for (int I2 = I; I2 < 4; ++I2) {
-            for (int i = 16 * I2; i < 16 * I2 + 16; ++i) {
-                float ka[8], qa[8];
-                *reinterpret_cast<float4 *>(&ka[0]) = *reinterpret_cast<const float4 *>(&KA[i][8 * cg]);
-                *reinterpret_cast<float4 *>(&ka[4]) = *reinterpret_cast<const float4 *>(&KA[i][8 * cg + 4]);
-                *reinterpret_cast<float4 *>(&qa[0]) = *reinterpret_cast<const float4 *>(&QA[i][8 * cg]);
-                *reinterpret_cast<float4 *>(&qa[4]) = *reinterpret_cast<const float4 *>(&QA[i][8 * cg + 4]);
+        // R24'_jd = sum_{I' >= J} sum_{i in I'} (M_ij KA_id + s N_ij QA_id) c_I'Jd for rows j of block J = mt
+        float ra[8][4] = {};
+        for (int I2 = mt; I2 < 4; ++I2) {
+            const float *cf = I2 > mt ? CF[cf_index(I2, mt)] : nullptr;
+            for (int ks = 16 * I2; ks < 16 * I2 + 16; ks += 8) {
+                const uint32_t am[4] = {to_tf32(MM[ks + t4][r0]), to_tf32(MM[ks + t4][r1]), to_tf32(MM[ks + t4 + 4][r0]),
+                                        to_tf32(MM[ks + t4 + 4][r1])};
+                const uint32_t an[4] = {to_tf32(NN[ks + t4][r0]), to_tf32(NN[ks + t4][r1]), to_tf32(NN[ks + t4 + 4][r0]),
+                                        to_tf32(NN[ks + t4 + 4][r1])};
 #pragma unroll
-                for (int e = 0; e < 8; ++e) qa[e] = __fmul_rn(s, qa[e]);
-                if (I2 > I) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float cf = CF[cf_index(I2, I)][8 * cg + e];
-                        ka[e] = __fmul_rn(ka[e], cf);
-                        qa[e] = __fmul_rn(qa[e], cf);
+                for (int j = 0; j < 8; ++j) {
+                    const int d = 64 * nh + 8 * j + g;
+                    float k0 = KA[ks + t4][d], k1 = KA[ks + t4 + 4][d];
+                    float q0 = __fmul_rn(s, QA[ks + t4][d]), q1 = __fmul_rn(s, QA[ks + t4 + 4][d]);
+                    if (cf) {
+                        const float c = cf[d];
+                        k0 = __fmul_rn(k0, c);
+                        k1 = __fmul_rn(k1, c);
+                        q0 = __fmul_rn(q0, c);
+                        q1 = __fmul_rn(q1, c);
                     }
+                    mma_tf32(ra[j], am, to_tf32(k0), to_tf32(k1));
+                    mma_tf32(ra[j], an, to_tf32(q0), to_tf32(q1));
                 }
-                const float4 m4 = *reinterpret_cast<const float4 *>(&MM[i][4 * rg]);
-                const float4 n4 = *reinterpret_cast<const float4 *>(&NN[i][4 * rg]);
-                const float m[4] = {m4.x, m4.y, m4.z, m4.w}, nn[4] = {n4.x, n4.y, n4.z, n4.w};
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) r2[jj][e] = __fmaf_rn(m[jj], ka[e], __fmaf_rn(nn[jj], qa[e], r2[jj][e]));
             }
         }
-        // R24 = b R24' with b = exp(m_I - G); dkn += R24, dG -= kn R24 = KB R24'
+        // R24 = b R24' (b = exp(m_J - G)): dkn += R24, dG -= kn R24 = KB R24'
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const int j = 4 * rg + jj;
+        for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int d = 8 * cg + e;
-                const float b = bwd_exp(__fsub_rn(G[16 * I + 7][d], G[j][d]));
-                rk[jj][e] = __fmaf_rn(b, r2[jj][e], rk[jj][e]);
-                rG[jj][e] = __fmaf_rn(-KB[j][d], r2[jj][e], rG[jj][e]);
+            for (int q = 0; q < 4; ++q) {
+                const int i = (q >> 1) ? r1 : r0, d = 64 * nh + 8 * j + 2 * t4 + (q & 1);
+                const float b = bwd_exp(__fsub_rn(G[16 * mt + 7][d], G[i][d]));
+                rk[j][q] = __fmaf_rn(b, ra[j][q], rk[j][q]);
+                rG[j][q] = __fmaf_rn(-KB[i][d], ra[j][q], rG[j][q]);
             }
-        }
     }
     // dqn, dkn out (valid rows)
 #pragma unroll
-    for (int ii = 0; ii < 4; ++ii) {
-        const int i = 4 * rg + ii;
+    for (int hf = 0; hf < 2; ++hf) {
+        const int i = hf ? r1 : r0;
         if (i < nvalid) {
-            float *dq = p.dqn + ((row0 + i) * p.HV + h) * DK + 8 * cg;
-            float *dk = p.dkn + ((row0 + i) * p.HV + h) * DK + 8 * cg;
-            *reinterpret_cast<float4 *>(dq) = make_float4(rq[ii][0], rq[ii][1], rq[ii][2], rq[ii][3]);
-            *reinterpret_cast<float4 *>(dq + 4) = make_float4(rq[ii][4], rq[ii][5], rq[ii][6], rq[ii][7]);
-            *reinterpret_cast<float4 *>(dk) = make_float4(rk[ii][0], rk[ii][1], rk[ii][2], rk[ii][3]);
-            *reinterpret_cast<float4 *>(dk + 4) = make_float4(rk[ii][4], rk[ii][5], rk[ii][6], rk[ii][7]);
+            float *dq = p.dqn + ((row0 + i) * p.HV + h) * DK + 64 * nh + 2 * t4;
+            float *dk = p.dkn + ((row0 + i) * p.HV + h) * DK + 64 * nh + 2 * t4;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                *reinterpret_cast<float2 *>(dq + 8 * j) = make_float2(rq[j][2 * hf], rq[j][2 * hf + 1]);
+                *reinterpret_cast<float2 *>(dk + 8 * j) = make_float2(rk[j][2 * hf], rk[j][2 * hf + 1]);
+            }
         }
     }
     __syncthreads();  // KA/QA/KB/G reads done; dgl complete
     // dG rows into the KA region (unpadded [64][128]), then the reverse cumulative sum per key column
     float(*dG)[DK] = reinterpret_cast<float(*)[DK]>(sm + S::KA);
 #pragma unroll
-    for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) dG[4 * rg + ii][8 * cg + e] = rG[ii][e];
+    for (int j = 0; j < 8; ++j) {
+        *reinterpret_cast<float2 *>(&dG[r0][64 * nh + 8 * j + 2 * t4]) = make_float2(rG[j][0], rG[j][1]);
+        *reinterpret_cast<float2 *>(&dG[r1][64 * nh + 8 * j + 2 * t4]) = make_float2(rG[j][2], rG[j][3]);
+    }
     __syncthreads();
     if (tid < DK) {
         float acc = dgl[tid];  // G_L = G of the last row

@@ -41,18 +41,20 @@ __device__ __forceinline__ float l2norm_den128_warp(uint2 raw)
     return __fsqrt_rn(__fadd_rn(ss, 1e-6f));
 }
 
-// One warp normalises one row of 128 bf16 values; lane l holds elements
-// 4l..4l+3 as two packed bf16 pairs (lo, hi).  Returns the packed result.
-__device__ __forceinline__ uint2 l2norm_row128_warp(uint2 raw)
+// The normalised values of lane l's four elements given the row's denominator.
+__device__ __forceinline__ uint2 l2norm_apply128(uint2 raw, float den)
 {
     const float x0 = bf16lo(raw.x), x1 = bf16hi(raw.x), x2 = bf16lo(raw.y), x3 = bf16hi(raw.y);
-    const float den = l2norm_den128_warp(raw);
     const float r = __frcp_rn(den);
     uint2 out;
     out.x = pack_bf16(div_rn_with_rcp(x0, den, r), div_rn_with_rcp(x1, den, r));
     out.y = pack_bf16(div_rn_with_rcp(x2, den, r), div_rn_with_rcp(x3, den, r));
     return out;
 }
+
+// One warp normalises one row of 128 bf16 values; lane l holds elements
+// 4l..4l+3 as two packed bf16 pairs (lo, hi).  Returns the packed result.
+__device__ __forceinline__ uint2 l2norm_row128_warp(uint2 raw) { return l2norm_apply128(raw, l2norm_den128_warp(raw)); }
 
 // Standalone pass: rows of 128 bf16, one warp per row, grid-stride.
 __global__ void __launch_bounds__(256) l2norm_bf16_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,

@@ -153,6 +153,18 @@ def worked_example(T: int = 128, K: int = 128, V: int = 128) -> dict:
             "beta": torch.ones(1, T, 1), "initial_state": None, "cu_seqlens": None}
 
 
+# ---------------------------------------------------------------------------------------------- backward
+def make_backward_grads(case: Case, device: str | torch.device = "cpu") -> dict:
+    """Seeded loss gradients for a backward of ``case``: dout ~ N(0,1) bf16 [B,T,HV,V] and dht ~ N(0, 0.1^2)
+    fp32 [N,HV,K,V] (drawn in that order from their own generator, seed + 7919)."""
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(case.seed + 7919)
+    dout = torch.randn(case.B, case.T, case.HV, case.V, generator=gen, device=dev).to(torch.bfloat16)
+    dht = 0.1 * torch.randn(case.N, case.HV, case.K, case.V, generator=gen, device=dev)
+    return {"dout": dout, "dht": dht}
+
+
 # ---------------------------------------------------------------------------------------------- decode step
 @dataclass
 class DecodeCase:
