@@ -334,6 +334,171 @@ def bench_decode(args, case, world, rank, dev):
     return 0
 
 
+# ---------------------------------------------------------------------------------------------- backward
+
+BWD_METRIC = "KDA chunk-prefill backward tokens·heads/s @T=64K,HV=64,K=V=128; % of HBM roofline"
+
+
+def backward_bytes(case) -> int:
+    """Bytes the backward must move at least once: q, k, v, g, beta, dout read; dq, dk, dv, dg, dbeta written;
+    the initial state and dht read, dh0 written."""
+    group = case.HV // case.H
+    th = case.tokens * case.HV
+    per = (256 * 2 / group) * 2 + 256 * 2 + 512 * 2 + 4 * 2 + 256
+    state = case.N * case.HV * 128 * 128 * 4 * (3 if case.state != "none" else 2)
+    return int(th * per + state)
+
+
+def time_oracle_backward(case, target_s: float = 15.0, steps: int = 1, warmup: int = 0):
+    """The oracle's backward, as it stands, on a bounded sample: the first tokens of the first value heads."""
+    import oracle
+    from kda_gated_delta_prefill_b200 import inputs as gen
+    cores = oracle.max_threads()
+    heads = min(case.HV, max(1, cores))
+    gr = gen.make_backward_grads(case)
+
+    def sample(tokens):
+        xs = cpu_sample_inputs(case, heads, tokens)
+        do = gr["dout"][:, :tokens, :heads].float().numpy()
+        dh = gr["dht"][:, :heads].numpy()
+        return lambda: oracle.backward(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["initial_state"], do, dh)
+
+    pilot = min(case.T, 128)
+    run = sample(pilot)
+    t0 = time.perf_counter()
+    run()
+    per_tok = (time.perf_counter() - t0) / pilot
+    tokens = int(min(case.T, max(64, target_s / max(per_tok, 1e-9))))
+    run = sample(tokens)
+    for _ in range(warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        run()
+    dt = (time.perf_counter() - t0) / steps
+    return {"value": tokens * heads / dt, "unit": UNIT, "cores": min(cores, heads), "kind": "oracle",
+            "sample": f"first {tokens} tokens x value heads 0..{heads - 1} of {case.name}", "seconds": dt}
+
+
+def bench_backward(args, case, world, rank, dev):
+    import dataclasses
+    import torch
+    import torch.distributed as dist
+    import kda_gated_delta_prefill_b200 as kda
+    from kda_gated_delta_prefill_b200 import inputs as gen
+    name = "backward_" + case.name
+    config = {"workload": name, "B": case.B, "T": case.T, "H": case.H, "HV": case.HV, "K": case.K, "V": case.V,
+              "chunk": 64, "initial_state": case.state != "none", "dht": True,
+              "l2": "inputs and workspace larger than L2; no flush",
+              "parallelism": f"independent replicas x{args.gpus} (weak)" if args.gpus > 1 else "single GPU"}
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        per_step = min(15.0, max(0.05, 150.0 / (args.steps + args.warmup)))
+        cb = time_oracle_backward(case, per_step, steps=args.steps, warmup=args.warmup)
+        line = {"metric": BWD_METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": cb["seconds"] * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "impl": "reference", "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+    rcase = dataclasses.replace(case, seed=case.seed + 1000 * rank)
+    x = gen.make_inputs(rcase, device=dev)
+    gr = gen.make_backward_grads(rcase, device=dev)
+    B, T, H, HV, K, V, N = case.B, case.T, case.H, case.HV, case.K, case.V, case.N
+    num_seqs = N if x["cu_seqlens"] is not None else 0
+    ws = torch.empty(kda.backward_workspace_size(B, T, H, HV, K, V, num_seqs), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return kda.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], gr["dout"], x["initial_state"], gr["dht"],
+                            x["cu_seqlens"], workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    total_ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    th = case.tokens * HV
+    value = th * world / (total_ms / 1e3 / args.steps)
+    hbm_gbs, _, peak_kind = load_peaks()
+    avg_s = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
+    alg = backward_bytes(case)
+    roofline = {"bound": "hbm", "achieved": alg / avg_s / 1e9, "peak": hbm_gbs, "unit": "GB/s",
+                "frac": alg / avg_s / 1e9 / hbm_gbs, "traffic": None, "peak_kind": peak_kind,
+                "algorithmic_bytes_per_launch": alg, "avg_launch_ms": avg_s * 1e3,
+                "scope": "the whole backward call (forward recomputation included)"}
+    e2e = None
+    if not args.no_e2e:  # inputs from pinned host memory in, every gradient out, each step
+        names = ("q", "k", "v", "g", "beta", "initial_state")
+        xh = {k: x[k].cpu().pin_memory() for k in names}
+        gh = {k: gr[k].cpu().pin_memory() for k in ("dout", "dht")}
+        xd = {k: torch.empty_like(x[k]) for k in names}
+        gd = {k: torch.empty_like(gr[k]) for k in ("dout", "dht")}
+        outs_h = None
+
+        def hstep():
+            nonlocal outs_h
+            for k in names:
+                xd[k].copy_(xh[k], non_blocking=True)
+            for k in gd:
+                gd[k].copy_(gh[k], non_blocking=True)
+            outs = kda.backward(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], gd["dout"], xd["initial_state"],
+                                gd["dht"], None, workspace=ws, stream=stream)
+            if outs_h is None:
+                outs_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+            for a, b in zip(outs_h, outs):
+                a.copy_(b, non_blocking=True)
+        for _ in range(2):
+            hstep()
+        torch.cuda.synchronize()
+        n_e = max(3, min(args.steps, 5))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e):
+            hstep()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        e2e = {"value": th * world / (e_ms / 1e3 / n_e), "unit": UNIT,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in list(xh.values()) + list(gh.values())),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs_h), "steps": n_e}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = time_oracle_backward(case)
+        cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    launches = kda.backward_kernel_launches(B, T, H, HV, K, V, num_seqs)
+    line = {"metric": BWD_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
+            "gpu_launches": launches * args.steps, "impl": "native", "kernel_source": kernel_source_hash()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 # ---------------------------------------------------------------------------------------------- main
 
 def main():
@@ -343,7 +508,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="long_T65536_H64_state",
-                    help="a prefill workload name, or decode_B1024_H12 for the decode step")
+                    help="a prefill workload name, backward_<prefill workload name> for the backward, or "
+                         "decode_B1024_H12 for the decode step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile-T", type=int, default=0,
@@ -358,12 +524,16 @@ def main():
     from kda_gated_delta_prefill_b200 import inputs as gen
 
     decode = args.workload.startswith("decode")
-    case = gen.DECODE_SERVING if decode else {c.name: c for c in gen.WORKLOADS}[args.workload]
+    backward = args.workload.startswith("backward_")
+    wname = args.workload[len("backward_"):] if backward else args.workload
+    case = gen.DECODE_SERVING if decode else {c.name: c for c in gen.WORKLOADS}[wname]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if decode and args.impl == "reference":
         return bench_decode(args, case, world, rank, None)
+    if backward and args.impl == "reference":
+        return bench_backward(args, case, world, rank, None)
     config = None if decode else {"workload": case.name, "B": case.B, "T": case.T, "H": case.H, "HV": case.HV, "K": case.K,
               "V": case.V, "chunk": 64, "initial_state": case.state != "none",
               "l2": "inputs (6.5 GB) larger than L2; no flush" if case.name.startswith("long")
@@ -403,6 +573,8 @@ def main():
     kda.lib()
     if decode:
         return bench_decode(args, case, world, rank, dev)
+    if backward:
+        return bench_backward(args, case, world, rank, dev)
 
     # ---- inputs resident in HBM (rank-specific seed: independent batches) ----
     import dataclasses
