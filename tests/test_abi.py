@@ -144,3 +144,36 @@ def test_decode_rejects_bad_arguments(L, over, code):
 
 def test_decode_empty_batch_is_a_no_op(L):
     assert call_decode(L, B=0) == 0
+
+
+def call_backward(L, B=1, T=64, H=1, HV=1, K=128, V=128, q=1, k=2, v=3, g=4, beta=5, s0=None, do=6, dht=None,
+                  dq=7, dk=8, dv=9, dg=10, db=11, dh0=None, ws=12, ws_bytes=None, cu=None, num_seqs=0):
+    P = ctypes.c_void_p
+    step = 1 << 32  # arguments live far apart unless a case moves one
+    ptr = lambda i: None if i is None else P(FAKE + int(i * step))
+    if ws_bytes is None:
+        ws_bytes = L.kda_prefill_backward_workspace_size(B, T, H, HV, K, V, num_seqs)
+    return L.kda_prefill_backward(ptr(q), ptr(k), ptr(v), ptr(g), ptr(beta), ptr(s0), ptr(cu), num_seqs, B, T, H, HV,
+                                  K, V, ptr(do), ptr(dht), ptr(dq), ptr(dk), ptr(dv), ptr(dg), ptr(db), ptr(dh0),
+                                  ptr(ws), ws_bytes, None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(K=64), 2), (dict(V=256), 2), (dict(HV=3, H=2), 1), (dict(B=0), 1), (dict(T=-1), 1),
+    (dict(q=None), 1), (dict(do=None), 1), (dict(dg=None), 1), (dict(db=None), 1),
+    (dict(q=1 + 2 ** -32 * 8), 3), (dict(dv=9 + 2 ** -32 * 4), 3), (dict(ws=12 + 2 ** -32 * 16), 3),
+    (dict(dq=1), 1), (dict(dg=4), 1), (dict(dk=7), 1), (dict(dh0=13, s0=13), 1), (dict(ws=6), 1), (dict(ws=7), 1),
+    (dict(ws_bytes=16), 4), (dict(ws=None), 4), (dict(cu=14, B=2, num_seqs=2), 1),
+])
+def test_backward_rejects_bad_arguments(L, over, code):
+    assert call_backward(L, **over) == code
+
+
+def test_backward_workspace_and_launch_counts(L):
+    # per chunk and value head: the forward's block, a start state and an end-state gradient (fp32 K x V each)
+    one = L.kda_prefill_backward_workspace_size(1, 64, 1, 1, 128, 128, 0)
+    two = L.kda_prefill_backward_workspace_size(1, 128, 1, 1, 128, 128, 0)
+    assert two - one >= 74240 + 2 * 65536
+    assert L.kda_prefill_backward_workspace_size(1, 64, 1, 1, 64, 128, 0) == 0
+    assert L.kda_prefill_backward_kernel_launches(1, 64, 1, 1, 128, 128, 0) == 5
+    assert L.kda_prefill_backward_kernel_launches(1, 64, 1, 1, 128, 128, 3) == 6
