@@ -193,6 +193,24 @@ kda_status_t kda_prefill_device_error(unsigned *word, int clear);
 int kda_prefill_kernel_launches(int B, int T, int H, int HV, int K, int V, int num_seqs);
 
 /*
+ * The forward with the state stored in bf16 (a precision variant the pages
+ * allow: "KDA Chunk Prefill on Ascend A3", section "Function and tensor
+ * contract", leaves the state's storage open beyond fp32 results): arguments
+ * as kda_prefill_forward except
+ *   initial_state  bf16 [N,HV,K,V] or NULL, 16-byte aligned
+ *   final_state    bf16 [N,HV,K,V] out (nearest-even rounding of the fp32
+ *                  state the forward computes); may equal initial_state
+ *   workspace      kda_prefill_state_bf16_workspace_size(...) bytes
+ * The state is widened to fp32 before the carry and rounded after it; the
+ * arithmetic in between is the fp32-state forward's.
+ */
+size_t kda_prefill_state_bf16_workspace_size(int B, int T, int H, int HV, int K, int V, int num_seqs);
+kda_status_t kda_prefill_forward_state_bf16(const void *q, const void *k, const void *v, const float *g,
+                                            const float *beta, const void *initial_state, const int32_t *cu_seqlens,
+                                            int num_seqs, int B, int T, int H, int HV, int K, int V, void *o,
+                                            void *final_state, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Backward of kda_prefill_forward, which "KDA Chunk Prefill on Ascend A3"
  * leaves optional (section "Timing and required submission"): for the loss
  * sum(o * dout) + sum(final_state * dht) it returns the gradients of q, k,

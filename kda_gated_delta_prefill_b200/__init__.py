@@ -28,7 +28,8 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 EXPORTED = ("kda_status_string", "kda_prefill_workspace_size", "kda_prefill_forward",
             "kda_prefill_host_staging_size", "kda_prefill_forward_host", "kda_prefill_device_error",
             "kda_l2norm_bf16", "kda_prefill_kernel_launches", "kda_decode_step",
-            "kda_prefill_backward_workspace_size", "kda_prefill_backward_kernel_launches", "kda_prefill_backward")
+            "kda_prefill_backward_workspace_size", "kda_prefill_backward_kernel_launches", "kda_prefill_backward",
+            "kda_prefill_state_bf16_workspace_size", "kda_prefill_forward_state_bf16")
 
 
 class KdaError(RuntimeError):
@@ -76,6 +77,10 @@ def lib():
         L.kda_prefill_backward_kernel_launches.restype = I
         L.kda_prefill_backward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, Z, P]
         L.kda_prefill_backward.restype = I
+        L.kda_prefill_state_bf16_workspace_size.argtypes = [I] * 7
+        L.kda_prefill_state_bf16_workspace_size.restype = Z
+        L.kda_prefill_forward_state_bf16.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, Z, P]
+        L.kda_prefill_forward_state_bf16.restype = I
         _lib = L
         return L
 
@@ -133,6 +138,29 @@ def forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o=None, fi
                                    _ptr(workspace), workspace.numel() if workspace is not None else 0,
                                    _stream_ptr(stream))
     _check(rc, "kda_prefill_forward")
+    return o, final_state
+
+
+def forward_state_bf16(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o=None, final_state=None,
+                       workspace=None, stream=None):
+    """The forward with a bf16 state: initial_state bf16 [N,HV,K,V] or None; returns (o, final_state bf16)."""
+    import torch
+    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
+    if initial_state is not None and initial_state.dtype != torch.bfloat16:
+        raise ValueError("initial_state must be bf16")
+    if o is None:
+        o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=q.device)
+    if final_state is None:
+        final_state = torch.empty(N, HV, K, V, dtype=torch.bfloat16, device=q.device)
+    num_seqs = N if cu_seqlens is not None else 0
+    ws_bytes = int(lib().kda_prefill_state_bf16_workspace_size(B, T, H, HV, K, V, num_seqs))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    rc = lib().kda_prefill_forward_state_bf16(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                                              _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(o),
+                                              _ptr(final_state), _ptr(workspace), workspace.numel(),
+                                              _stream_ptr(stream))
+    _check(rc, "kda_prefill_forward_state_bf16")
     return o, final_state
 
 

@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cstdint>
 #include <cstring>
@@ -849,4 +850,79 @@ extern "C" kda_status_t kda_prefill_forward_noalloc(const void *q, const void *k
     // needs clearing between calls.
     return kda_prefill_forward(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, B, T, H, HV, K, V, o,
                                final_state, scratch, kNoAllocScratchBytes, stream);
+}
+
+// ---------------------------------------------------------------------------------------------------------
+// bf16 state storage: the forward with a bf16 initial and final state.  The state is widened into fp32 scratch
+// before the carry and rounded (nearest even) after it, so every mode of the forward applies unchanged.
+namespace kda {
+__global__ void __launch_bounds__(256) state_bf16_to_f32_kernel(const __nv_bfloat16 *__restrict__ in,
+                                                                float *__restrict__ out, int64_t n8)
+{
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint4 r = reinterpret_cast<const uint4 *>(in)[i];
+        float4 *o = reinterpret_cast<float4 *>(out) + 2 * i;
+        o[0] = make_float4(bf16lo(r.x), bf16hi(r.x), bf16lo(r.y), bf16hi(r.y));
+        o[1] = make_float4(bf16lo(r.z), bf16hi(r.z), bf16lo(r.w), bf16hi(r.w));
+    }
+}
+__global__ void __launch_bounds__(256) state_f32_to_bf16_kernel(const float *__restrict__ in,
+                                                                __nv_bfloat16 *__restrict__ out, int64_t n8)
+{
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float4 a = reinterpret_cast<const float4 *>(in)[2 * i], b = reinterpret_cast<const float4 *>(in)[2 * i + 1];
+        reinterpret_cast<uint4 *>(out)[i] =
+            make_uint4(pack_bf16(a.x, a.y), pack_bf16(a.z, a.w), pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
+    }
+}
+}  // namespace kda
+
+extern "C" size_t kda_prefill_state_bf16_workspace_size(int B, int T, int H, int HV, int K, int V, int num_seqs)
+{
+    Dims d;
+    if (check_dims(B, T, H, HV, K, V, num_seqs > 0, num_seqs, d) != KDA_OK) return 0;
+    const size_t state = static_cast<size_t>(d.N) * HV * K * V * sizeof(float);
+    return workspace_layout(B, T, HV, num_seqs > 0 ? num_seqs : 0).total + 2 * round_up(state, kAlign);
+}
+
+extern "C" kda_status_t kda_prefill_forward_state_bf16(const void *q, const void *k, const void *v, const float *g,
+                                                       const float *beta, const void *initial_state,
+                                                       const int32_t *cu_seqlens, int num_seqs, int B, int T, int H,
+                                                       int HV, int K, int V, void *o, void *final_state,
+                                                       void *workspace, size_t workspace_bytes, void *stream)
+{
+    Dims d;
+    const bool varlen = cu_seqlens != nullptr;
+    kda_status_t st = check_dims(B, T, H, HV, K, V, varlen, num_seqs, d);
+    if (st != KDA_OK) return st;
+    if (!final_state) return KDA_ERR_INVALID_ARG;
+    if (!aligned(initial_state, 16) || !aligned(final_state, 16)) return KDA_ERR_MISALIGNED;
+    const size_t nstate = static_cast<size_t>(d.N) * HV * K * V;
+    const size_t fwd = workspace_layout(B, T, HV, varlen ? num_seqs : 0).total;
+    const size_t need = fwd + 2 * round_up(nstate * sizeof(float), kAlign);
+    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    if (!aligned(workspace, kAlign)) return KDA_ERR_MISALIGNED;
+    if (overlaps(workspace, need, initial_state, initial_state ? nstate * 2 : 0) ||
+        overlaps(workspace, need, final_state, nstate * 2) ||
+        (initial_state && initial_state != final_state && overlaps(initial_state, nstate * 2, final_state, nstate * 2)))
+        return KDA_ERR_INVALID_ARG;
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    float *s0 = reinterpret_cast<float *>(wsb + fwd);
+    float *sN = reinterpret_cast<float *>(wsb + fwd + round_up(nstate * sizeof(float), kAlign));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    DeviceInfo info;
+    if (device_info(info) != cudaSuccess) return KDA_ERR_CUDA;
+    const int64_t n8 = static_cast<int64_t>(nstate / 8);
+    const int grid = static_cast<int>(std::min<int64_t>((n8 + 255) / 256, static_cast<int64_t>(info.sms) * 8));
+    if (initial_state) {
+        kda::state_bf16_to_f32_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(initial_state), s0, n8);
+        if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    st = kda_prefill_forward(q, k, v, g, beta, initial_state ? s0 : nullptr, cu_seqlens, num_seqs, B, T, H, HV, K, V, o,
+                             sN, workspace, fwd, stream);
+    if (st != KDA_OK) return st;
+    kda::state_f32_to_bf16_kernel<<<grid, 256, 0, s>>>(sN, static_cast<__nv_bfloat16 *>(final_state), n8);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

@@ -338,3 +338,45 @@ def test_segmented_long_few_heads_sampled():
     xc = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     sub = select_heads(xc, [3])
     compare(o[:, :, [3]].contiguous(), s[:, [3]].contiguous(), oracle_forward(sub))
+
+
+@pytest.mark.parametrize("B,T,H,HV,varlen", [(1, 200, 2, 4, False), (2, 1000, 4, 4, False), (1, 300, 1, 2, True)])
+def test_bf16_state_forward(B, T, H, HV, varlen):
+    """bf16 state storage: the oracle runs from the bf16 initial state's values; the kernel's final state is the
+    nearest-even bf16 of its fp32 state, so the state bar widens by one bf16 unit (2^-8 relative) of each element."""
+    import kda_gated_delta_prefill_b200 as kda
+    import oracle
+    gen_ = torch.Generator().manual_seed(1700 + T)
+    cu = torch.tensor([0, 37, 37, 300], dtype=torch.int32) if varlen else None
+    N = 3 if varlen else B
+    q = torch.randn(B, T, H, 128, generator=gen_).bfloat16()
+    k = torch.randn(B, T, H, 128, generator=gen_).bfloat16()
+    v = torch.randn(B, T, HV, 128, generator=gen_).bfloat16()
+    g = -torch.nn.functional.softplus(torch.randn(B, T, HV, 128, generator=gen_)) / 8
+    beta = torch.sigmoid(torch.randn(B, T, HV, generator=gen_))
+    s0 = (0.1 * torch.randn(N, HV, 128, 128, generator=gen_)).bfloat16()
+    c = lambda t: None if t is None else t.cuda()
+    o, sN = kda.forward_state_bf16(c(q), c(k), c(v), c(g), c(beta), c(s0), c(cu))
+    torch.cuda.synchronize()
+    assert sN.dtype == torch.bfloat16
+    ref = oracle.forward(q, k, v, g, beta, s0.float(), cu)
+    og = o.float().cpu().numpy()
+    if varlen:
+        rows = np.zeros((B, T), bool)
+        rows[0, :300] = True
+        og, orf = og[rows], ref["o64"][rows]
+    else:
+        orf = ref["o64"]
+    assert np.abs(og - orf).max() <= 2e-2 * max(1.0, np.abs(orf).max())
+    sg = sN.float().cpu().numpy().astype(np.float64)
+    sr = ref["state"]
+    for n in range(N):
+        for h in range(HV):
+            den = np.linalg.norm(sr[n, h])
+            assert np.linalg.norm(sg[n, h] - sr[n, h]) <= (5e-3 + 2 ** -8) * den
+    assert (np.abs(sg - sr) <= 0.02 + 0.02 * np.abs(sr) + 2 ** -8 * np.abs(sr)).all()
+    # in place: final_state may be the initial state's buffer
+    s_io = c(s0.clone())
+    kda.forward_state_bf16(c(q), c(k), c(v), c(g), c(beta), s_io, c(cu), final_state=s_io)
+    torch.cuda.synchronize()
+    assert torch.equal(s_io.cpu(), sN.cpu())
