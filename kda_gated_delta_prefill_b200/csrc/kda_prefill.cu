@@ -672,7 +672,15 @@ extern "C" kda_status_t kda_prefill_backward(const void *q, const void *k, const
     cp.chunk_count = cp.chunks_per_seq;
     cp.states = states;
     cp.no_o = 1;
-    if (launch_carry(cp, d.N * HV, s) != cudaSuccess) return KDA_ERR_CUDA;
+    // The forward carry (start states) and the reverse carry (end-state gradients) both read only the blocks,
+    // so they run side by side: the forward one on the high-priority side stream, joined before the chunk kernel.
+    CarryLane *lane = nullptr;
+    if (carry_lane(info.dev, lane) != cudaSuccess) return KDA_ERR_CUDA;
+    std::lock_guard<std::mutex> lane_lock(lane->mu);
+    if (cudaEventRecord(lane->fork, s) != cudaSuccess || cudaStreamWaitEvent(lane->stream, lane->fork, 0) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (launch_carry(cp, d.N * HV, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
+    if (cudaEventRecord(lane->join, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
 
     // 2. reverse carry: the gradient at every chunk's end state, and at the initial state
     kda::BwdParams bp{};
@@ -708,6 +716,7 @@ extern "C" kda_status_t kda_prefill_backward(const void *q, const void *k, const
         return KDA_ERR_CUDA;
     kda::kda_bwd_carry_kernel<<<d.N * HV * (DV / kda::kBcCols), kda::kBcThreads, kda::BcSmem::TOTAL, s>>>(bp);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+    if (cudaStreamWaitEvent(s, lane->join, 0) != cudaSuccess) return KDA_ERR_CUDA;
     if (tokens == 0) return KDA_OK;
 
     // 3. every chunk's gradients, 4. the Q/K groups through the normalisation
