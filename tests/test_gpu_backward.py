@@ -116,3 +116,24 @@ def test_backward_config2_shape():
     """The 4-head, 1000-token shape with a ragged tail (15 full chunks and one of 40 tokens)."""
     got, ref = _run(*_case(1, 1000, 4, 4, seed=2))
     _compare(got, ref)
+
+
+def test_backward_full_workload_sampled():
+    """The backward of the benchmark's workload (B=1, H=HV=64, T=65536, fp32 state; dout and dht from the
+    benchmark's generator), computed for all heads on the GPU in the launch shape the benchmark times; heads are
+    independent (H == HV), so the oracle checks two heads over the whole sequence."""
+    import kda_gated_delta_prefill_b200 as kda
+    from kda_gated_delta_prefill_b200 import inputs as gen
+    case = gen.LONG_PREFILL
+    x = gen.make_inputs(case, device="cuda")
+    gr = gen.make_backward_grads(case, device="cuda")
+    out = kda.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], gr["dout"], x["initial_state"], gr["dht"])
+    torch.cuda.synchronize()
+    assert kda.device_error(clear=True) == 0
+    heads = [3, 62]
+    sel = lambda t, dim: t.index_select(dim, torch.tensor(heads, device=t.device)).contiguous().cpu()
+    ref = oracle.backward(sel(x["q"], 2), sel(x["k"], 2), sel(x["v"], 2), sel(x["g"], 2), sel(x["beta"], 2),
+                          sel(x["initial_state"], 1), sel(gr["dout"], 2).float().numpy(), sel(gr["dht"], 1).numpy())
+    got = [sel(out[i], 2).float().numpy().astype(np.float64) for i in range(5)] + [sel(out[5], 1).numpy()]
+    report = _compare(got, ref)
+    assert report["dq"][0] < REL_FRO
