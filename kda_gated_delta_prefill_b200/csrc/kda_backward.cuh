@@ -41,8 +41,8 @@ struct BwdParams {
     const __nv_bfloat16 *q, *k, *v, *dout;  // q, k: [rows][H][K]; v, dout: [rows][HV][V]
     const float *g, *beta;                  // [rows][HV][K], [rows][HV]
     const uint8_t *items;                   // the forward's per-(chunk, head) blocks
-    const float *states;                    // [chunks][HV][K][V]: state at each chunk's start
-    float *dstates;                         // [chunks][HV][K][V]: gradient at each chunk's end state
+    const __nv_bfloat16 *states;            // [chunks][HV][K][V] bf16: state at each chunk's start
+    __nv_bfloat16 *dstates;                 // [chunks][HV][K][V] bf16: gradient at each chunk's end state
     const float *dht;                       // [N][HV][K][V] or null (zero)
     float *dh0;                             // [N][HV][K][V] or null (not wanted)
     float *dqn, *dkn;                       // [rows][HV][K]: gradient at the normalised rows, per value head
@@ -181,13 +181,13 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
         const int nrows = min(CH, len - c * CH);
         {
             // dS is the gradient at chunk c's end state: store it
-            float *dst = p.dstates + ((c_begin + c) * p.HV + h) * DK * DV + vc0;
+            __nv_bfloat16 *dst = p.dstates + ((c_begin + c) * p.HV + h) * DK * DV + vc0;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf)
-                    *reinterpret_cast<float2 *>(dst + key_of(hf) * DV + col_of(j, 0)) =
-                        make_float2(acc[j][2 * hf], acc[j][2 * hf + 1]);
+                    *reinterpret_cast<__nv_bfloat162 *>(dst + key_of(hf) * DV + col_of(j, 0)) =
+                        __floats2bfloat162_rn(acc[j][2 * hf], acc[j][2 * hf + 1]);
             // dO rows of the chunk as fp16 (zero past the sequence's end)
             const int i = tid >> 3, cc = 8 * (tid & 7);
             uint4 w = make_uint4(0u, 0u, 0u, 0u);
@@ -304,11 +304,12 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
 
 // ---------------------------------------------------------------------------------------------------------
 // Chunk gradients: one CTA of 256 threads per (chunk, value head), fp32 throughout.
-constexpr int kBwThreads = 256, kBwCols = 8;  // value columns per pass over the state
-constexpr int kRow = 132;                     // padded row stride (floats) of the [64][128] operand tiles
-constexpr int kRowC = 68;                     // padded row stride of the [64][64] tiles
-constexpr int kVl = 12;                       // padded row stride of the [64][8] value-column tiles
-constexpr int kSt = 132;                      // padded row stride of the transposed [8][128] state tiles
+constexpr int kBwThreads = 256, kBwCols = 16;  // value columns per pass over the state
+constexpr int kRow = 132;                      // padded row stride (floats) of the [64][128] operand tiles
+constexpr int kRowC = 68;                      // padded row stride of the [64][64] tiles
+// element (r, c) of a [64][16] fp32 value-column tile: rows of 16 floats, columns XOR-swizzled by 4 (r / 2 % 4)
+// so that the eight rows of an MMA fragment fall into distinct banks
+__device__ __forceinline__ int vsw(int r, int c) { return r * kBwCols + (c ^ (((r >> 1) & 3) << 2)); }
 struct BwSmem {
     static constexpr int KA = 0;                          // kn_id exp(G_id - m_Id)
     static constexpr int QA = KA + CH * kRow * 4;         // qn_id exp(G_id - m_Id)
@@ -327,15 +328,15 @@ struct BwSmem {
     static constexpr int DBETA = DGL + 512;               // [64]
     static constexpr int WK = DBETA + 256;                // work region
     // V pass buffers (inside WK); S, dS' and dO columns are double-buffered (cp.async, one pass ahead)
-    static constexpr int SV = WK;                         // [2][128][8]  S[:, cols]
-    static constexpr int DSV = SV + 2 * DK * kBwCols * 4; // [2][128][8]  dS'[:, cols]
-    static constexpr int DOB = DSV + 2 * DK * kBwCols * 4;  // bf16 [2][64][8] dO
-    static constexpr int DD = DOB + 2 * CH * kBwCols * 2; // [64][kVl] D = v - Kb S
-    static constexpr int VN = DD + CH * kVl * 4;          // [64][kVl] Vnew
-    static constexpr int DVN = VN + CH * kVl * 4;         // [64][kVl] dVnew
-    static constexpr int DV = DVN + CH * kVl * 4;         // [64][kVl] dv
-    static constexpr int WK_END = DV + CH * kVl * 4;
-    // phase-3 use of WK: the off-diagonal products of the blocked solve, up to 3 x [16][16]
+    static constexpr int SV = WK;                         // bf16 [2][128][16]  S[:, cols]
+    static constexpr int DSV = SV + 2 * DK * kBwCols * 2; // bf16 [2][128][16]  dS'[:, cols]
+    static constexpr int DOB = DSV + 2 * DK * kBwCols * 2;  // bf16 [2][64][16] dO
+    static constexpr int DD = DOB + 2 * CH * kBwCols * 2; // [64][16] (vsw) D = v - Kb S
+    static constexpr int VN = DD + CH * kBwCols * 4;      // [64][16] Vnew
+    static constexpr int DVN = VN + CH * kBwCols * 4;     // [64][16] dVnew
+    static constexpr int DV = DVN + CH * kBwCols * 4;     // [64][16] dv
+    static constexpr int WK_END = DV + CH * kBwCols * 4;
+    // phase-3 use of WK: the off-diagonal products of the blocked solve, up to 3 x [16][17]
     static constexpr int XS = WK;
     // phase-6 use of WK: dA, then Y = T^T dA diag(beta)
     static constexpr int DA = WK;                         // [64][kRowC]
@@ -529,35 +530,40 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         }
     }
 
-    // ---- 4-5. passes over 8 value columns at a time, on TF32 tensor-core MMAs (m16n8k8, fp32 accumulate) ----
-    // S, dS' [128][8] and dO [64][8] (bf16) of the current pass, the next pass's in the other buffer
-    auto SVb = [&](int b) { return reinterpret_cast<float(*)[kBwCols]>(sm + S::SV + b * DK * kBwCols * 4); };
-    auto DSVb = [&](int b) { return reinterpret_cast<float(*)[kBwCols]>(sm + S::DSV + b * DK * kBwCols * 4); };
+    // ---- 4-5. passes over 16 value columns at a time, on TF32 tensor-core MMAs (m16n8k8, fp32 accumulate) ----
+    // S, dS' (bf16 [128][16]) and dO (bf16 [64][16]) of the current pass, the next pass's in the other buffer
+    auto SVb = [&](int b) { return reinterpret_cast<__nv_bfloat16(*)[kBwCols]>(sm + S::SV + b * DK * kBwCols * 2); };
+    auto DSVb = [&](int b) { return reinterpret_cast<__nv_bfloat16(*)[kBwCols]>(sm + S::DSV + b * DK * kBwCols * 2); };
     auto DOBb = [&](int b) { return reinterpret_cast<__nv_bfloat16(*)[kBwCols]>(sm + S::DOB + b * CH * kBwCols * 2); };
-    float(*DDv)[kVl] = reinterpret_cast<float(*)[kVl]>(sm + S::DD);
-    float(*VN)[kVl] = reinterpret_cast<float(*)[kVl]>(sm + S::VN);
-    float(*DVN)[kVl] = reinterpret_cast<float(*)[kVl]>(sm + S::DVN);
-    float(*DVv)[kVl] = reinterpret_cast<float(*)[kVl]>(sm + S::DV);
-    const float *Sg = p.states + item * DK * DV;
-    const float *dSg = p.dstates + item * DK * DV;
+    float *DDv = reinterpret_cast<float *>(sm + S::DD);
+    float *VN = reinterpret_cast<float *>(sm + S::VN);
+    float *DVN = reinterpret_cast<float *>(sm + S::DVN);
+    float *DVv = reinterpret_cast<float *>(sm + S::DV);
+    const __nv_bfloat16 *Sg = p.states + item * DK * DV;
+    const __nv_bfloat16 *dSg = p.dstates + item * DK * DV;
     const int rg = tid >> 4, cg = tid & 15;  // ownership of the 64 x 64 steps of phase 6
     // MMA fragment ownership (g = lane / 4, t4 = lane % 4): warp (mt, nh) holds rows 16 mt + g and + 8, and key
     // columns 64 nh + 8 j + 2 t4 (+1), j = 0..7 (dQg, dKb, dKg), or token columns 32 nh + 8 j + 2 t4 (+1),
     // j = 0..3 (dAqk, dA)
     const int g = lane >> 2, t4 = lane & 3, mt = warp & 3, nh = warp >> 2;
     const int r0 = 16 * mt + g, r1 = r0 + 8;
+    auto bf = [](__nv_bfloat16 x) { return to_tf32(__bfloat162float(x)); };
     float aQ[8][4] = {}, aB[8][4] = {}, aG[8][4] = {}, aAq[4][4] = {}, aA[4][4] = {};
-    // pass vb's columns into buffer b: S and dS' rows are 32 bytes (two 16-byte copies each), dO rows 16 bytes
+    // pass vb's columns into buffer b: S, dS' and dO rows are 32 bytes (two 16-byte copies each)
     auto fetch = [&](int vb, int b) {
-        const int row = tid >> 1, half = 4 * (tid & 1);
+        const int row = tid >> 1, half = 8 * (tid & 1);
         cp_async16(smem_u32(&SVb(b)[row][half]), Sg + row * DV + vb + half);
         cp_async16(smem_u32(&DSVb(b)[row][half]), dSg + row * DV + vb + half);
-        if (tid < nvalid) cp_async16(smem_u32(&DOBb(b)[tid][0]), p.dout + ((row0 + tid) * p.HV + h) * DV + vb);
+        if (row < nvalid && tid < 2 * CH)
+            cp_async16(smem_u32(&DOBb(b)[row][half]), p.dout + ((row0 + row) * p.HV + h) * DV + vb + half);
         cp_async_commit();
     };
     if (tid < CH && tid >= nvalid) {  // rows past the end stay zero in both buffers
-        *reinterpret_cast<uint4 *>(&DOBb(0)[tid][0]) = make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4 *>(&DOBb(1)[tid][0]) = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            *reinterpret_cast<uint4 *>(&DOBb(b)[tid][0]) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(&DOBb(b)[tid][8]) = make_uint4(0u, 0u, 0u, 0u);
+        }
     }
     fetch(0, 0);
     float gl_acc = 0.f;  // thread d < 128: sum over all columns of S[d][.] dS'[d][.]
@@ -570,107 +576,121 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
             cp_async_wait<0>();
         }
         __syncthreads();
-        float(*SVT)[kBwCols] = SVb(buf);
-        float(*DST)[kBwCols] = DSVb(buf);
+        const __nv_bfloat16(*SVT)[kBwCols] = SVb(buf);
+        const __nv_bfloat16(*DST)[kBwCols] = DSVb(buf);
         const __nv_bfloat16(*DOV)[kBwCols] = DOBb(buf);
         if (tid < DK) {
-            const float4 x0 = *reinterpret_cast<const float4 *>(&SVT[tid][0]), x1 = *reinterpret_cast<const float4 *>(&SVT[tid][4]);
-            const float4 y0 = *reinterpret_cast<const float4 *>(&DST[tid][0]), y1 = *reinterpret_cast<const float4 *>(&DST[tid][4]);
-            gl_acc = __fmaf_rn(x0.x, y0.x, gl_acc);
-            gl_acc = __fmaf_rn(x0.y, y0.y, gl_acc);
-            gl_acc = __fmaf_rn(x0.z, y0.z, gl_acc);
-            gl_acc = __fmaf_rn(x0.w, y0.w, gl_acc);
-            gl_acc = __fmaf_rn(x1.x, y1.x, gl_acc);
-            gl_acc = __fmaf_rn(x1.y, y1.y, gl_acc);
-            gl_acc = __fmaf_rn(x1.z, y1.z, gl_acc);
-            gl_acc = __fmaf_rn(x1.w, y1.w, gl_acc);
+#pragma unroll
+            for (int c = 0; c < kBwCols; c += 2) {
+                const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&SVT[tid][c]));
+                const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&DST[tid][c]));
+                gl_acc = __fmaf_rn(x.y, y.y, __fmaf_rn(x.x, y.x, gl_acc));
+            }
         }
         if (warp < 4) {
-            // (a) D = v - Kb S for rows 16 mt .. (Kb = KA exp(m_I), block I = mt)
-            float c[4] = {};
+            // (a) D = v - Kb S for rows 16 mt .. (Kb = KA exp(m_I), block I = mt), two n8 tiles of columns
+            float c[2][4] = {};
             for (int ks = 0; ks < DK; ks += 8) {
                 const float e0 = EM[mt][ks + t4], e1 = EM[mt][ks + t4 + 4];
                 const uint32_t a[4] = {to_tf32(__fmul_rn(KA[r0][ks + t4], e0)), to_tf32(__fmul_rn(KA[r1][ks + t4], e0)),
                                        to_tf32(__fmul_rn(KA[r0][ks + t4 + 4], e1)),
                                        to_tf32(__fmul_rn(KA[r1][ks + t4 + 4], e1))};
-                mma_tf32(c, a, to_tf32(SVT[ks + t4][g]), to_tf32(SVT[ks + t4 + 4][g]));
+                mma_tf32(c[0], a, bf(SVT[ks + t4][g]), bf(SVT[ks + t4 + 4][g]));
+                mma_tf32(c[1], a, bf(SVT[ks + t4][8 + g]), bf(SVT[ks + t4 + 4][8 + g]));
             }
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int i = hf ? r1 : r0;
-                float2 vv = make_float2(0.f, 0.f);
-                if (i < nvalid)
-                    vv = __bfloat1622float2(
-                        *reinterpret_cast<const __nv_bfloat162 *>(p.v + ((row0 + i) * p.HV + h) * DV + vb + 2 * t4));
-                *reinterpret_cast<float2 *>(&DDv[i][2 * t4]) =
-                    make_float2(__fsub_rn(vv.x, c[2 * hf]), __fsub_rn(vv.y, c[2 * hf + 1]));
-            }
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int i = hf ? r1 : r0, cc = 8 * nt + 2 * t4;
+                    float2 vv = make_float2(0.f, 0.f);
+                    if (i < nvalid)
+                        vv = __bfloat1622float2(
+                            *reinterpret_cast<const __nv_bfloat162 *>(p.v + ((row0 + i) * p.HV + h) * DV + vb + cc));
+                    *reinterpret_cast<float2 *>(&DDv[vsw(i, cc)]) =
+                        make_float2(__fsub_rn(vv.x, c[nt][2 * hf]), __fsub_rn(vv.y, c[nt][2 * hf + 1]));
+                }
         } else {
             // (c) dVnew = Kg dS' + Aqk^T dO for rows 16 mt .. (Kg = KB exp(G_L - m_I))
-            float c[4] = {};
+            float c[2][4] = {};
             for (int ks = 0; ks < DK; ks += 8) {
                 const float e0 = EGLM[mt][ks + t4], e1 = EGLM[mt][ks + t4 + 4];
                 const uint32_t a[4] = {to_tf32(__fmul_rn(KB[r0][ks + t4], e0)), to_tf32(__fmul_rn(KB[r1][ks + t4], e0)),
                                        to_tf32(__fmul_rn(KB[r0][ks + t4 + 4], e1)),
                                        to_tf32(__fmul_rn(KB[r1][ks + t4 + 4], e1))};
-                mma_tf32(c, a, to_tf32(DST[ks + t4][g]), to_tf32(DST[ks + t4 + 4][g]));
+                mma_tf32(c[0], a, bf(DST[ks + t4][g]), bf(DST[ks + t4 + 4][g]));
+                mma_tf32(c[1], a, bf(DST[ks + t4][8 + g]), bf(DST[ks + t4 + 4][8 + g]));
             }
             for (int js = 16 * mt; js < CH; js += 8) {  // Aqk^T[i][j] = Aqk[j][i], nonzero for j >= i
                 const uint32_t a[4] = {to_tf32(AQ[js + t4][r0]), to_tf32(AQ[js + t4][r1]), to_tf32(AQ[js + t4 + 4][r0]),
                                        to_tf32(AQ[js + t4 + 4][r1])};
-                mma_tf32(c, a, to_tf32(__bfloat162float(DOV[js + t4][g])), to_tf32(__bfloat162float(DOV[js + t4 + 4][g])));
+                mma_tf32(c[0], a, bf(DOV[js + t4][g]), bf(DOV[js + t4 + 4][g]));
+                mma_tf32(c[1], a, bf(DOV[js + t4][8 + g]), bf(DOV[js + t4 + 4][8 + g]));
             }
-            *reinterpret_cast<float2 *>(&DVN[r0][2 * t4]) = make_float2(c[0], c[1]);
-            *reinterpret_cast<float2 *>(&DVN[r1][2 * t4]) = make_float2(c[2], c[3]);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                *reinterpret_cast<float2 *>(&DVN[vsw(r0, 8 * nt + 2 * t4)]) = make_float2(c[nt][0], c[nt][1]);
+                *reinterpret_cast<float2 *>(&DVN[vsw(r1, 8 * nt + 2 * t4)]) = make_float2(c[nt][2], c[nt][3]);
+            }
         }
         __syncthreads();
         if (warp < 4) {
             // (b) Vnew = T diag(beta) D (T lower triangular: j < 16 (mt + 1))
-            float c[4] = {};
+            float c[2][4] = {};
             for (int js = 0; js < 16 * (mt + 1); js += 8) {
                 const float b0 = beta[js + t4], b1 = beta[js + t4 + 4];
                 const uint32_t a[4] = {to_tf32(__fmul_rn(TT[r0][js + t4], b0)), to_tf32(__fmul_rn(TT[r1][js + t4], b0)),
                                        to_tf32(__fmul_rn(TT[r0][js + t4 + 4], b1)),
                                        to_tf32(__fmul_rn(TT[r1][js + t4 + 4], b1))};
-                mma_tf32(c, a, to_tf32(DDv[js + t4][g]), to_tf32(DDv[js + t4 + 4][g]));
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+                    mma_tf32(c[nt], a, to_tf32(DDv[vsw(js + t4, 8 * nt + g)]), to_tf32(DDv[vsw(js + t4 + 4, 8 * nt + g)]));
             }
-            *reinterpret_cast<float2 *>(&VN[r0][2 * t4]) = make_float2(c[0], c[1]);
-            *reinterpret_cast<float2 *>(&VN[r1][2 * t4]) = make_float2(c[2], c[3]);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                *reinterpret_cast<float2 *>(&VN[vsw(r0, 8 * nt + 2 * t4)]) = make_float2(c[nt][0], c[nt][1]);
+                *reinterpret_cast<float2 *>(&VN[vsw(r1, 8 * nt + 2 * t4)]) = make_float2(c[nt][2], c[nt][3]);
+            }
         } else {
             // (d) dv = diag(beta) T^T dVnew (j >= i)
-            float c[4] = {};
+            float c[2][4] = {};
             for (int js = 16 * mt; js < CH; js += 8) {
                 const uint32_t a[4] = {to_tf32(TT[js + t4][r0]), to_tf32(TT[js + t4][r1]), to_tf32(TT[js + t4 + 4][r0]),
                                        to_tf32(TT[js + t4 + 4][r1])};
-                mma_tf32(c, a, to_tf32(DVN[js + t4][g]), to_tf32(DVN[js + t4 + 4][g]));
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+                    mma_tf32(c[nt], a, to_tf32(DVN[vsw(js + t4, 8 * nt + g)]), to_tf32(DVN[vsw(js + t4 + 4, 8 * nt + g)]));
             }
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const int i = hf ? r1 : r0;
-                const float x0 = __fmul_rn(beta[i], c[2 * hf]), x1 = __fmul_rn(beta[i], c[2 * hf + 1]);
-                *reinterpret_cast<float2 *>(&DVv[i][2 * t4]) = make_float2(x0, x1);
-                if (i < nvalid)
-                    *reinterpret_cast<__nv_bfloat162 *>(p.dv + ((row0 + i) * p.HV + h) * DV + vb + 2 * t4) =
-                        __floats2bfloat162_rn(x0, x1);
-            }
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int i = hf ? r1 : r0, cc = 8 * nt + 2 * t4;
+                    const float x0 = __fmul_rn(beta[i], c[nt][2 * hf]), x1 = __fmul_rn(beta[i], c[nt][2 * hf + 1]);
+                    *reinterpret_cast<float2 *>(&DVv[vsw(i, cc)]) = make_float2(x0, x1);
+                    if (i < nvalid)
+                        *reinterpret_cast<__nv_bfloat162 *>(p.dv + ((row0 + i) * p.HV + h) * DV + vb + cc) =
+                            __floats2bfloat162_rn(x0, x1);
+                }
         }
         __syncthreads();
-        {
-            // (e) dQg += dO S^T, dKb -= dv S^T, dKg += Vnew dS'^T (K = these 8 columns); dAqk += dO Vnew^T,
-            //     dA += dVnew D^T
-            const uint32_t aO[4] = {to_tf32(__bfloat162float(DOV[r0][t4])), to_tf32(__bfloat162float(DOV[r1][t4])),
-                                    to_tf32(__bfloat162float(DOV[r0][t4 + 4])), to_tf32(__bfloat162float(DOV[r1][t4 + 4]))};
-            const uint32_t aV[4] = {to_tf32(-DVv[r0][t4]), to_tf32(-DVv[r1][t4]), to_tf32(-DVv[r0][t4 + 4]),
-                                    to_tf32(-DVv[r1][t4 + 4])};
-            const uint32_t aN[4] = {to_tf32(VN[r0][t4]), to_tf32(VN[r1][t4]), to_tf32(VN[r0][t4 + 4]),
-                                    to_tf32(VN[r1][t4 + 4])};
-            const uint32_t aD[4] = {to_tf32(DVN[r0][t4]), to_tf32(DVN[r1][t4]), to_tf32(DVN[r0][t4 + 4]),
-                                    to_tf32(DVN[r1][t4 + 4])};
+        // (e) dQg += dO S^T, dKb -= dv S^T, dKg += Vnew dS'^T (K = these 16 columns, two k8 steps);
+        //     dAqk += dO Vnew^T, dA += dVnew D^T
+#pragma unroll
+        for (int kc = 0; kc < kBwCols; kc += 8) {
+            const int c0 = kc + t4, c1 = kc + t4 + 4;
+            const uint32_t aO[4] = {bf(DOV[r0][c0]), bf(DOV[r1][c0]), bf(DOV[r0][c1]), bf(DOV[r1][c1])};
+            const uint32_t aV[4] = {to_tf32(-DVv[vsw(r0, c0)]), to_tf32(-DVv[vsw(r1, c0)]), to_tf32(-DVv[vsw(r0, c1)]),
+                                    to_tf32(-DVv[vsw(r1, c1)])};
+            const uint32_t aN[4] = {to_tf32(VN[vsw(r0, c0)]), to_tf32(VN[vsw(r1, c0)]), to_tf32(VN[vsw(r0, c1)]),
+                                    to_tf32(VN[vsw(r1, c1)])};
+            const uint32_t aD[4] = {to_tf32(DVN[vsw(r0, c0)]), to_tf32(DVN[vsw(r1, c0)]), to_tf32(DVN[vsw(r0, c1)]),
+                                    to_tf32(DVN[vsw(r1, c1)])};
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int d = 64 * nh + 8 * j + g;
-                const uint32_t s0 = to_tf32(SVT[d][t4]), s1 = to_tf32(SVT[d][t4 + 4]);
-                const uint32_t q0 = to_tf32(DST[d][t4]), q1 = to_tf32(DST[d][t4 + 4]);
+                const uint32_t s0 = bf(SVT[d][c0]), s1 = bf(SVT[d][c1]);
+                const uint32_t q0 = bf(DST[d][c0]), q1 = bf(DST[d][c1]);
                 mma_tf32(aQ[j], aO, s0, s1);
                 mma_tf32(aB[j], aV, s0, s1);
                 mma_tf32(aG[j], aN, q0, q1);
@@ -678,8 +698,8 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int tk = 32 * nh + 8 * j + g;
-                mma_tf32(aAq[j], aO, to_tf32(VN[tk][t4]), to_tf32(VN[tk][t4 + 4]));
-                mma_tf32(aA[j], aD, to_tf32(DDv[tk][t4]), to_tf32(DDv[tk][t4 + 4]));
+                mma_tf32(aAq[j], aO, to_tf32(VN[vsw(tk, c0)]), to_tf32(VN[vsw(tk, c1)]));
+                mma_tf32(aA[j], aD, to_tf32(DDv[vsw(tk, c0)]), to_tf32(DDv[vsw(tk, c1)]));
             }
         }
         __syncthreads();

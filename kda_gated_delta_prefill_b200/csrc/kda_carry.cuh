@@ -65,9 +65,9 @@ struct CarryParams {
     int seg_phase;
     int seg_count;
     float *seg_S, *seg_M, *seg_B;  // [units][seg_count][K][V]
-    // Unsegmented launches only: when set, the state at the start of every chunk is also stored, fp32
-    // [K][V] at states + (global chunk * HV + h) * K * V (the item's index), for the backward.
-    float *states;
+    // Unsegmented launches only: when set, the state at the start of every chunk is also stored, bf16
+    // [K][V] (nearest even) at states + (global chunk * HV + h) * K * V (the item's index), for the backward.
+    __nv_bfloat16 *states;
     int no_o;                      // unsegmented launches: skip o (the O products and stores)
 };
 
@@ -277,11 +277,11 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
             if (lane == 0) mbar_arrive(bar);
         };
         // the state at the start of chunk c (S^T[v][32kq + j] in r) -> states, rows kd = 32kq + j, column v
-        float *dump = kDump && p.seg_phase == 0 ? p.states : nullptr;
+        __nv_bfloat16 *dump = kDump && p.seg_phase == 0 ? p.states : nullptr;
         auto dump_state = [&](const uint32_t (&r)[32], int kq, int c) {
-            float *dst = dump + ((c_begin + c) * p.HV + h) * DK * DV + v;
+            __nv_bfloat16 *dst = dump + ((c_begin + c) * p.HV + h) * DK * DV + v;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) dst[(32 * kq + j) * DV] = __uint_as_float(r[j]);
+            for (int j = 0; j < 32; ++j) dst[(32 * kq + j) * DV] = __float2bfloat16_rn(__uint_as_float(r[j]));
         };
         bool alive = tmem_alloc == 0;
         if (alive) {

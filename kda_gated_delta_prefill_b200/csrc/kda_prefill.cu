@@ -534,6 +534,7 @@ BwdWorkspace bwd_workspace_layout(int B, int T, int HV, int num_seqs)
     w.max_chunks = varlen ? (static_cast<int64_t>(T) + CH - 1) / CH + num_seqs
                           : static_cast<int64_t>(B) * ((T + CH - 1) / CH);
     const size_t rows = static_cast<size_t>(B) * T, state = static_cast<size_t>(DK) * DV * sizeof(float);
+    const size_t state16 = static_cast<size_t>(DK) * DV * 2;  // the per-chunk states and gradients are bf16
     size_t off = 0;
     if (varlen) {
         w.chunk_off = off;
@@ -542,9 +543,9 @@ BwdWorkspace bwd_workspace_layout(int B, int T, int HV, int num_seqs)
     w.items = off;
     off = round_up(off + static_cast<size_t>(w.max_chunks) * HV * kda::ITEM_BYTES, kAlign);
     w.states = off;
-    off = round_up(off + static_cast<size_t>(w.max_chunks) * HV * state, kAlign);
+    off = round_up(off + static_cast<size_t>(w.max_chunks) * HV * state16, kAlign);
     w.dstates = off;
-    off = round_up(off + static_cast<size_t>(w.max_chunks) * HV * state, kAlign);
+    off = round_up(off + static_cast<size_t>(w.max_chunks) * HV * state16, kAlign);
     w.final_state = off;
     off = round_up(off + static_cast<size_t>(N) * HV * state, kAlign);
     w.dqn = off;
@@ -621,8 +622,8 @@ extern "C" kda_status_t kda_prefill_backward(const void *q, const void *k, const
     uint8_t *wsb = static_cast<uint8_t *>(workspace);
     int32_t *chunk_off = varlen ? reinterpret_cast<int32_t *>(wsb + ws.chunk_off) : nullptr;
     uint8_t *items = wsb + ws.items;
-    float *states = reinterpret_cast<float *>(wsb + ws.states);
-    float *dstates = reinterpret_cast<float *>(wsb + ws.dstates);
+    __nv_bfloat16 *states = reinterpret_cast<__nv_bfloat16 *>(wsb + ws.states);
+    __nv_bfloat16 *dstates = reinterpret_cast<__nv_bfloat16 *>(wsb + ws.dstates);
     if (varlen) {
         kda::chunk_offsets_kernel<<<1, 1024, 0, s>>>(cu_seqlens, num_seqs, chunk_off);
         if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
