@@ -51,9 +51,16 @@ def chunk_flops(case) -> int:
     return case.tokens * case.HV * 180224
 
 
+# device and host sources of the other paths (backward, decode step): edits there leave the forward unchanged
+OTHER_PATH_SOURCES = {"kda_backward.cuh", "kda_backward_api.cuh", "kda_decode.cuh"}
+
+
 def kernel_source_hash() -> str:
+    """Hash of the sources the forward's kernels and launches are built from."""
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "kda_gated_delta_prefill_b200", "csrc", "*"))):
+        if os.path.basename(f) in OTHER_PATH_SOURCES:
+            continue
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())
             h.update(fh.read())

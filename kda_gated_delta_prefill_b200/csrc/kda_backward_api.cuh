@@ -1,0 +1,219 @@
+// kda_backward_api.cuh -- host side of the backward (included at the end of kda_prefill.cu, whose argument
+// checks, workspace helpers, tensor-map encoding and carry launch it uses).
+#pragma once
+
+namespace {
+
+// Backward workspace: [chunk_off (N+1)] for packed batches, then the forward's per-chunk blocks, the chunk
+// start states, the gradients at the chunk end states, the final state of the recomputed forward, and the
+// per-value-head gradients at the normalised q/k rows.
+struct BwdWorkspace {
+    size_t chunk_off = 0, items = 0, states = 0, dstates = 0, final_state = 0, dqn = 0, dkn = 0, total = 0;
+    int64_t max_chunks = 0;
+};
+
+BwdWorkspace bwd_workspace_layout(int B, int T, int HV, int num_seqs)
+{
+    BwdWorkspace w;
+    const bool varlen = num_seqs > 0;
+    const int64_t N = varlen ? num_seqs : B;
+    w.max_chunks = varlen ? (static_cast<int64_t>(T) + CH - 1) / CH + num_seqs
+                          : static_cast<int64_t>(B) * ((T + CH - 1) / CH);
+    const size_t rows = static_cast<size_t>(B) * T, state = static_cast<size_t>(DK) * DV * sizeof(float);
+    const size_t state16 = static_cast<size_t>(DK) * DV * 2;  // the per-chunk states and gradients are bf16
+    size_t off = 0;
+    if (varlen) {
+        w.chunk_off = off;
+        off += round_up((static_cast<size_t>(num_seqs) + 1) * 4, kAlign);
+    }
+    w.items = off;
+    off = round_up(off + static_cast<size_t>(w.max_chunks) * HV * kda::ITEM_BYTES, kAlign);
+    w.states = off;
+    off = round_up(off + static_cast<size_t>(w.max_chunks) * HV * state16, kAlign);
+    w.dstates = off;
+    off = round_up(off + static_cast<size_t>(w.max_chunks) * HV * state16, kAlign);
+    w.final_state = off;
+    off = round_up(off + static_cast<size_t>(N) * HV * state, kAlign);
+    w.dqn = off;
+    off = round_up(off + rows * HV * DK * sizeof(float), kAlign);
+    w.dkn = off;
+    off = round_up(off + rows * HV * DK * sizeof(float), kAlign);
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+
+extern "C" size_t kda_prefill_backward_workspace_size(int B, int T, int H, int HV, int K, int V, int num_seqs)
+{
+    Dims d;
+    if (check_dims(B, T, H, HV, K, V, num_seqs > 0, num_seqs, d) != KDA_OK) return 0;
+    return bwd_workspace_layout(B, T, HV, num_seqs > 0 ? num_seqs : 0).total;
+}
+
+extern "C" int kda_prefill_backward_kernel_launches(int B, int T, int H, int HV, int K, int V, int num_seqs)
+{
+    Dims d;
+    const bool varlen = num_seqs > 0;
+    if (check_dims(B, T, H, HV, K, V, varlen, num_seqs, d) != KDA_OK) return 0;
+    const int with_tokens = static_cast<int64_t>(B) * T > 0 ? 1 : 0;
+    // chunk offsets (packed), intra-chunk, carry with the start states, reverse carry, chunk gradients, norms
+    return (varlen ? 1 : 0) + with_tokens + 1 + 1 + 2 * with_tokens;
+}
+
+extern "C" kda_status_t kda_prefill_backward(const void *q, const void *k, const void *v, const float *g,
+                                             const float *beta, const float *initial_state,
+                                             const int32_t *cu_seqlens, int num_seqs, int B, int T, int H, int HV,
+                                             int K, int V, const void *dout, const float *dht, void *dq, void *dk,
+                                             void *dv, float *dg, float *dbeta, float *dh0, void *workspace,
+                                             size_t workspace_bytes, void *stream)
+{
+    Dims d;
+    const bool varlen = cu_seqlens != nullptr;
+    kda_status_t st = check_dims(B, T, H, HV, K, V, varlen, num_seqs, d);
+    if (st != KDA_OK) return st;
+    const int64_t tokens = static_cast<int64_t>(B) * T;
+    if (tokens > 0 && (!q || !k || !v || !g || !beta || !dout || !dq || !dk || !dv || !dg || !dbeta))
+        return KDA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) || !aligned(dout, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(dg, 16) || !aligned(dbeta, 4) ||
+        !aligned(beta, 4) || !aligned(initial_state, 16) || !aligned(dht, 16) || !aligned(dh0, 16) ||
+        !aligned(cu_seqlens, 4))
+        return KDA_ERR_MISALIGNED;
+    const size_t nq = static_cast<size_t>(tokens) * H * K * 2, nvb = static_cast<size_t>(tokens) * HV * V * 2;
+    const size_t ng = static_cast<size_t>(tokens) * HV * K * 4, nb = static_cast<size_t>(tokens) * HV * 4;
+    const size_t ns = static_cast<size_t>(d.N) * HV * K * V * 4;
+    const void *ins[] = {q, k, v, g, beta, initial_state, cu_seqlens, dout, dht};
+    const size_t in_n[] = {nq, nq, nvb, ng, nb, initial_state ? ns : 0,
+                           varlen ? static_cast<size_t>(num_seqs + 1) * 4 : 0, nvb, dht ? ns : 0};
+    const void *outs[] = {dq, dk, dv, dg, dbeta, dh0};
+    const size_t out_n[] = {nq, nq, nvb, ng, nb, dh0 ? ns : 0};
+    for (int o = 0; o < 6; ++o) {
+        for (int i = 0; i < 9; ++i)
+            if (overlaps(outs[o], out_n[o], ins[i], in_n[i])) return KDA_ERR_INVALID_ARG;
+        for (int o2 = o + 1; o2 < 6; ++o2)
+            if (overlaps(outs[o], out_n[o], outs[o2], out_n[o2])) return KDA_ERR_INVALID_ARG;
+    }
+    const BwdWorkspace ws = bwd_workspace_layout(B, T, HV, varlen ? num_seqs : 0);
+    if (!workspace || workspace_bytes < ws.total) return KDA_ERR_WORKSPACE;
+    if (!aligned(workspace, kAlign)) return KDA_ERR_MISALIGNED;
+    for (int i = 0; i < 9; ++i)
+        if (overlaps(workspace, ws.total, ins[i], in_n[i])) return KDA_ERR_INVALID_ARG;
+    for (int o = 0; o < 6; ++o)
+        if (overlaps(workspace, ws.total, outs[o], out_n[o])) return KDA_ERR_INVALID_ARG;
+
+    DeviceInfo info;
+    if (device_info(info) != cudaSuccess) return KDA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    int32_t *chunk_off = varlen ? reinterpret_cast<int32_t *>(wsb + ws.chunk_off) : nullptr;
+    uint8_t *items = wsb + ws.items;
+    __nv_bfloat16 *states = reinterpret_cast<__nv_bfloat16 *>(wsb + ws.states);
+    __nv_bfloat16 *dstates = reinterpret_cast<__nv_bfloat16 *>(wsb + ws.dstates);
+    if (varlen) {
+        kda::chunk_offsets_kernel<<<1, 1024, 0, s>>>(cu_seqlens, num_seqs, chunk_off);
+        if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    // 1. the forward's per-chunk blocks, then its carry storing every chunk's start state (no o)
+    if (tokens > 0) {
+        CUtensorMap tq, tk, tv, tg;
+        if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HV, tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HV, tokens, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return KDA_ERR_CUDA;
+        kda::IntraParams ip{};
+        ip.beta = beta;
+        ip.cu = cu_seqlens;
+        ip.chunk_off = chunk_off;
+        ip.items = items;
+        ip.err = info.err;
+        ip.B = B;
+        ip.T = T;
+        ip.H = H;
+        ip.HV = HV;
+        ip.N = d.N;
+        ip.chunks_per_seq = (T + CH - 1) / CH;
+        ip.prefetch_stride = info.sms * kda::kIntraCtasPerSm;
+        ip.chunk_begin = 0;
+        ip.chunk_count = ip.chunks_per_seq;
+        if (cudaFuncSetAttribute(kda::kda_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kda::IntraSmem::TOTAL) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        kda::kda_intra_kernel<<<static_cast<int>(ws.max_chunks * HV), 256, kda::IntraSmem::TOTAL, s>>>(tq, tk, tv,
+                                                                                                      tg, ip);
+        if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    kda::CarryParams cp{};
+    cp.items = items;
+    cp.s0 = initial_state;
+    cp.cu = cu_seqlens;
+    cp.chunk_off = chunk_off;
+    cp.sN = reinterpret_cast<float *>(wsb + ws.final_state);
+    cp.err = info.err;
+    cp.T = T;
+    cp.HV = HV;
+    cp.N = d.N;
+    cp.chunks_per_seq = (T + CH - 1) / CH;
+    cp.chunk_begin = 0;
+    cp.chunk_count = cp.chunks_per_seq;
+    cp.states = states;
+    cp.no_o = 1;
+    // The forward carry (start states) and the reverse carry (end-state gradients) both read only the blocks,
+    // so they run side by side: the forward one on the high-priority side stream, joined before the chunk kernel.
+    CarryLane *lane = nullptr;
+    if (carry_lane(info.dev, lane) != cudaSuccess) return KDA_ERR_CUDA;
+    std::lock_guard<std::mutex> lane_lock(lane->mu);
+    if (cudaEventRecord(lane->fork, s) != cudaSuccess || cudaStreamWaitEvent(lane->stream, lane->fork, 0) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (launch_carry(cp, d.N * HV, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
+    if (cudaEventRecord(lane->join, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
+
+    // 2. reverse carry: the gradient at every chunk's end state, and at the initial state
+    kda::BwdParams bp{};
+    bp.q = static_cast<const __nv_bfloat16 *>(q);
+    bp.k = static_cast<const __nv_bfloat16 *>(k);
+    bp.v = static_cast<const __nv_bfloat16 *>(v);
+    bp.dout = static_cast<const __nv_bfloat16 *>(dout);
+    bp.g = g;
+    bp.beta = beta;
+    bp.items = items;
+    bp.states = states;
+    bp.dstates = dstates;
+    bp.dht = dht;
+    bp.dh0 = dh0;
+    bp.dqn = reinterpret_cast<float *>(wsb + ws.dqn);
+    bp.dkn = reinterpret_cast<float *>(wsb + ws.dkn);
+    bp.dq = static_cast<__nv_bfloat16 *>(dq);
+    bp.dk = static_cast<__nv_bfloat16 *>(dk);
+    bp.dv = static_cast<__nv_bfloat16 *>(dv);
+    bp.dg = dg;
+    bp.dbeta = dbeta;
+    bp.cu = cu_seqlens;
+    bp.chunk_off = chunk_off;
+    bp.err = info.err;
+    bp.T = T;
+    bp.H = H;
+    bp.HV = HV;
+    bp.N = d.N;
+    bp.chunks_per_seq = (T + CH - 1) / CH;
+    bp.total_chunks = static_cast<int>(ws.max_chunks);
+    if (cudaFuncSetAttribute(kda::kda_bwd_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kda::BcSmem::TOTAL) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    kda::kda_bwd_carry_kernel<<<d.N * HV * (DV / kda::kBcCols), kda::kBcThreads, kda::BcSmem::TOTAL, s>>>(bp);
+    if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+    if (cudaStreamWaitEvent(s, lane->join, 0) != cudaSuccess) return KDA_ERR_CUDA;
+    if (tokens == 0) return KDA_OK;
+
+    // 3. every chunk's gradients, 4. the Q/K groups through the normalisation
+    if (cudaFuncSetAttribute(kda::kda_bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kda::BwSmem::TOTAL) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    kda::kda_bwd_chunk_kernel<<<static_cast<int>(ws.max_chunks * HV), kda::kBwThreads, kda::BwSmem::TOTAL, s>>>(bp);
+    if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+    const int64_t warps = tokens * H * 2;
+    kda::kda_bwd_norm_kernel<<<static_cast<int>((warps + 7) / 8), 256, 0, s>>>(bp, tokens);
+    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
