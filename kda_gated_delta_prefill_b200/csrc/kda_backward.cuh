@@ -336,8 +336,7 @@ struct BwSmem {
     static constexpr int DVN = VN + CH * kBwCols * 4;     // [64][16] dVnew
     static constexpr int DV = DVN + CH * kBwCols * 4;     // [64][16] dv
     static constexpr int WK_END = DV + CH * kBwCols * 4;
-    // phase-3 use of WK: the off-diagonal products of the blocked solve, up to 3 x [16][17]
-    static constexpr int XS = WK;
+    // phase-3 use of WK: the solve's products, 3 x [16][16] then [32][33]
     // phase-6 use of WK: dA, then Y = T^T dA diag(beta)
     static constexpr int DA = WK;                         // [64][kRowC]
     static constexpr int TOTAL = (WK_END > DA + CH * kRowC * 4 ? WK_END : DA + CH * kRowC * 4);
@@ -498,36 +497,82 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     }
     __syncthreads();
 
-    // ---- 3. T = (I + diag(beta) P)^-1 in 16 x 16 blocks: the four diagonal blocks right-looking side by side,
-    //         then T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ by distance I - J ----
+    // ---- 3. T = (I + L)^-1, L = diag(beta) P, in three steps:
+    //         the four 16 x 16 diagonal blocks by right-looking substitution in registers (thread = block I,
+    //         column c, rows r4 + 4q; row m reaches the column's lanes by shuffle), then the blocks next to the
+    //         diagonal T_{I,I-1} = -T_II L_{I,I-1} T_{I-1,I-1}, then the lower-left 32 x 32 block as
+    //         -T_B (L_C T_A) with T_A, T_B the two 32 x 32 diagonal blocks ----
     {
-        const int I = tid >> 6, pidx = tid & 63;
-        for (int k = 0; k < 15; ++k) {
-            const int cols = k + 1;
-            if (pidx < (15 - k) * cols) {
-                const int i = 16 * I + k + 1 + pidx / cols, j = 16 * I + pidx % cols, kk = 16 * I + k;
-                TT[i][j] = __fmaf_rn(-__fmul_rn(beta[i], PP[i][kk]), TT[kk][j], TT[i][j]);
+        const int I = tid >> 6, c = (tid >> 2) & 15, r4 = tid & 3;
+        float x[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) x[q] = (4 * q + r4 == c) ? 1.f : 0.f;
+#pragma unroll
+        for (int m = 0; m < 15; ++m) {
+            const float xm = __shfl_sync(0xffffffffu, x[m >> 2], (lane & ~3) | (m & 3));
+#pragma unroll
+            for (int q = m >> 2; q < 4; ++q) {
+                const int j = 4 * q + r4;
+                if (j > m) x[q] = __fmaf_rn(-__fmul_rn(beta[16 * I + j], PP[16 * I + j][16 * I + m]), xm, x[q]);
             }
-            __syncthreads();
         }
-        float(*X)[16][17] = reinterpret_cast<float(*)[16][17]>(sm + S::XS);
-        for (int dist = 1; dist < 4; ++dist) {
-            const int pairs = 4 - dist;  // blocks (I, J) = (J + dist, J), J = 0 .. pairs - 1
-            for (int x = tid; x < pairs * 256; x += kBwThreads) {
-                const int J = x >> 8, i = (x >> 4) & 15, j = x & 15, Ib = J + dist;
-                float acc = 0.f;
-                for (int kk = 16 * J; kk < 16 * Ib; ++kk) acc = __fmaf_rn(PP[16 * Ib + i][kk], TT[kk][16 * J + j], acc);
-                X[J][i][j] = __fmul_rn(beta[16 * Ib + i], acc);
-            }
-            __syncthreads();
-            for (int x = tid; x < pairs * 256; x += kBwThreads) {
-                const int J = x >> 8, i = (x >> 4) & 15, j = x & 15, Ib = J + dist;
-                float acc = 0.f;
-                for (int kk = 0; kk <= i; ++kk) acc = __fmaf_rn(TT[16 * Ib + i][16 * Ib + kk], X[J][kk][j], acc);
-                TT[16 * Ib + i][16 * J + j] = -acc;
-            }
-            __syncthreads();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) TT[16 * I + 4 * q + r4][16 * I + c] = x[q];
+    }
+    __syncthreads();
+    {
+        // (the blocks above the diagonal of T are zero, so every sum below runs over a fixed range)
+        float(*X)[16][16] = reinterpret_cast<float(*)[16][16]>(sm + S::WK);  // L_{I,I-1} T_{I-1,I-1}, I = 1..3
+        {
+            const int i = (tid >> 4) & 15, j = tid & 15;  // this thread: element (i, j) of each of the three blocks
+            float acc[3] = {};
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+#pragma unroll
+                for (int b = 0; b < 3; ++b)
+                    acc[b] = __fmaf_rn(PP[16 * (b + 1) + i][16 * b + k], TT[16 * b + k][16 * b + j], acc[b]);
+#pragma unroll
+            for (int b = 0; b < 3; ++b) X[b][i][j] = __fmul_rn(beta[16 * (b + 1) + i], acc[b]);
         }
+        __syncthreads();
+        {
+            const int i = (tid >> 4) & 15, j = tid & 15;
+            float acc[3] = {};
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+#pragma unroll
+                for (int b = 0; b < 3; ++b) acc[b] = __fmaf_rn(TT[16 * (b + 1) + i][16 * (b + 1) + k], X[b][k][j], acc[b]);
+#pragma unroll
+            for (int b = 0; b < 3; ++b) TT[16 * (b + 1) + i][16 * b + j] = -acc[b];
+        }
+        __syncthreads();
+        float(*Y)[33] = reinterpret_cast<float(*)[33]>(sm + S::WK + 3 * 256 * 4);  // L_C T_A, [32][33]
+        {
+            const int j = tid & 31, i0 = tid >> 5;  // this thread: rows i0 + 8 it, column j
+            float acc[4] = {};
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const float tk = TT[k][j];
+#pragma unroll
+                for (int it = 0; it < 4; ++it) acc[it] = __fmaf_rn(PP[32 + i0 + 8 * it][k], tk, acc[it]);
+            }
+#pragma unroll
+            for (int it = 0; it < 4; ++it) Y[i0 + 8 * it][j] = __fmul_rn(beta[32 + i0 + 8 * it], acc[it]);
+        }
+        __syncthreads();
+        {
+            const int j = tid & 31, i0 = tid >> 5;
+            float acc[4] = {};
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const float yk = Y[k][j];
+#pragma unroll
+                for (int it = 0; it < 4; ++it) acc[it] = __fmaf_rn(TT[32 + i0 + 8 * it][32 + k], yk, acc[it]);
+            }
+#pragma unroll
+            for (int it = 0; it < 4; ++it) TT[32 + i0 + 8 * it][j] = -acc[it];
+        }
+        __syncthreads();
     }
 
     // ---- 4-5. passes over 16 value columns at a time, on TF32 tensor-core MMAs (m16n8k8, fp32 accumulate) ----
