@@ -141,6 +141,31 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# ---------------------------------------------------------------------------------------------- ranks
+# One process per GPU; every rank runs its own batch of the same shape (the units shard with no exchange).
+
+def rank_case(case, rank: int):
+    """The workload of one rank: the same shape, its own inputs (seed offset by 1000 per rank)."""
+    import dataclasses
+    return dataclasses.replace(case, seed=case.seed + 1000 * rank)
+
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The slowest rank's time (every rank calls this, in the same order)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def weak_throughput(units_per_step: float, world: int, total_ms: float, steps: int) -> float:
+    """Whole-job units per second: every rank processed units_per_step per step in total_ms / steps."""
+    return units_per_step * world / (total_ms / 1e3 / steps)
+
+
 # ---------------------------------------------------------------------------------------------- oracle
 
 def cpu_sample_inputs(case, heads: int, tokens: int):
@@ -259,7 +284,7 @@ def bench_decode(args, case, world, rank, dev):
                 "e2e": {"value": cb["value"], "unit": DECODE_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return 0
-    x = gen.make_decode_inputs(dataclasses.replace(case, seed=case.seed + 1000 * rank), device=dev)
+    x = gen.make_decode_inputs(rank_case(case, rank), device=dev)
     o = torch.empty(case.B, case.HV, 128, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -285,13 +310,9 @@ def bench_decode(args, case, world, rank, dev):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-    total_ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     active = int((x["state_indices"] >= 0).sum().item())
-    value = active * case.HV * world / (total_ms / 1e3 / args.steps)
+    value = weak_throughput(active * case.HV, world, total_ms, args.steps)
     hbm_gbs, _, peak_kind = load_peaks()
     avg_s = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
     achieved = decode_bytes(case) / avg_s / 1e9
@@ -321,8 +342,8 @@ def bench_decode(args, case, world, rank, dev):
             hstep()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
-        e2e = {"value": active * case.HV * world / (e_ms / 1e3 / n_e), "unit": DECODE_UNIT,
+        e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
+        e2e = {"value": weak_throughput(active * case.HV, world, e_ms, n_e), "unit": DECODE_UNIT,
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in xh.values()),
                "d2h_bytes_per_step": oh.numel() * 2, "steps": n_e}
     cpu = None
@@ -410,7 +431,7 @@ def bench_backward(args, case, world, rank, dev):
                 "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return 0
-    rcase = dataclasses.replace(case, seed=case.seed + 1000 * rank)
+    rcase = rank_case(case, rank)
     x = gen.make_inputs(rcase, device=dev)
     gr = gen.make_backward_grads(rcase, device=dev)
     B, T, H, HV, K, V, N = case.B, case.T, case.H, case.HV, case.K, case.V, case.N
@@ -440,13 +461,9 @@ def bench_backward(args, case, world, rank, dev):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-    total_ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     th = case.tokens * HV
-    value = th * world / (total_ms / 1e3 / args.steps)
+    value = weak_throughput(th, world, total_ms, args.steps)
     hbm_gbs, _, peak_kind = load_peaks()
     avg_s = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
     alg = backward_bytes(case)
@@ -485,8 +502,8 @@ def bench_backward(args, case, world, rank, dev):
             hstep()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
-        e2e = {"value": th * world / (e_ms / 1e3 / n_e), "unit": UNIT,
+        e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
+        e2e = {"value": weak_throughput(th, world, e_ms, n_e), "unit": UNIT,
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in list(xh.values()) + list(gh.values())),
                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs_h), "steps": n_e}
     cpu = None
@@ -585,7 +602,7 @@ def main():
 
     # ---- inputs resident in HBM (rank-specific seed: independent batches) ----
     import dataclasses
-    rcase = dataclasses.replace(case, seed=case.seed + 1000 * rank)
+    rcase = rank_case(case, rank)
     x = gen.make_inputs(rcase, device=dev)
     B, T, H, HV, K, V, N = case.B, case.T, case.H, case.HV, case.K, case.V, case.N
     o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=dev)
@@ -621,15 +638,11 @@ def main():
         t1.record(stream)
         torch.cuda.synchronize()
         barrier()
-    total_ms = t0.elapsed_time(t1)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     launch_ms = [a.elapsed_time(b) for a, b in evs]
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
     ms_per_step = total_ms / args.steps
     th_per_step = case.tokens * HV
-    value = th_per_step * world / (total_ms / 1e3 / args.steps)
+    value = weak_throughput(th_per_step, world, total_ms, args.steps)
 
     # ---- roofline of the dominant (only) compute kernel ----
     hbm_gbs, bf16_tf, peak_kind = load_peaks()
@@ -671,14 +684,10 @@ def main():
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e_ms = a.elapsed_time(b)
-        if world > 1:
-            tt = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
         h2d = sum(t.numel() * t.element_size() for t in xh.values() if isinstance(t, torch.Tensor))
         d2h = oh.numel() * 2 + sh.numel() * 4
-        e2e = {"value": th_per_step * world / (e_ms / 1e3 / e_steps), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": weak_throughput(th_per_step, world, e_ms, e_steps), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": e_steps}
         del xh, staging
 
