@@ -592,7 +592,8 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     // j = 0..3 (dAqk, dA)
     const int g = lane >> 2, t4 = lane & 3, mt = warp & 3, nh = warp >> 2;
     const int r0 = 16 * mt + g, r1 = r0 + 8;
-    auto bf = [](__nv_bfloat16 x) { return to_tf32(__bfloat162float(x)); };
+    // bf16 values are exact in TF32 (8 of its 10 mantissa bits): the widened bits are the operand as they are
+    auto bf = [](__nv_bfloat16 x) { return static_cast<uint32_t>(__bfloat16_as_ushort(x)) << 16; };
     float aQ[8][4] = {}, aB[8][4] = {}, aG[8][4] = {}, aAq[4][4] = {}, aA[4][4] = {};
     // pass vb's columns into buffer b: S, dS' and dO rows are 32 bytes (two 16-byte copies each)
     auto fetch = [&](int vb, int b) {
