@@ -254,6 +254,29 @@ kda_status_t kda_prefill_backward(const void *q, const void *k, const void *v, c
                                   size_t workspace_bytes, void *stream);
 
 /*
+ * The forward that keeps what the backward needs, and the backward from it
+ * (the usual save-for-backward split of a training step):
+ *   kda_prefill_forward_save   the forward (arguments as kda_prefill_forward)
+ *                              that also leaves its per-chunk blocks and
+ *                              every chunk's start state (bf16) in `saved`;
+ *   kda_prefill_backward_saved the backward (arguments as kda_prefill_backward)
+ *                              with `saved` as its workspace; it skips the
+ *                              forward's recomputation.
+ * `saved` is kda_prefill_backward_workspace_size(...) bytes, 256-byte aligned,
+ * device, overlapping no argument; it must reach the backward unchanged and the
+ * backward must get the same q, k, v, g, beta, initial_state and cu_seqlens.
+ */
+kda_status_t kda_prefill_forward_save(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                                      const float *initial_state, const int32_t *cu_seqlens, int num_seqs, int B,
+                                      int T, int H, int HV, int K, int V, void *o, float *final_state, void *saved,
+                                      size_t saved_bytes, void *stream);
+kda_status_t kda_prefill_backward_saved(const void *q, const void *k, const void *v, const float *g,
+                                        const float *beta, const float *initial_state, const int32_t *cu_seqlens,
+                                        int num_seqs, int B, int T, int H, int HV, int K, int V, const void *dout,
+                                        const float *dht, void *dq, void *dk, void *dv, float *dg, float *dbeta,
+                                        float *dh0, void *saved, size_t saved_bytes, void *stream);
+
+/*
  * One recurrent decode step (one token per row) on a caller-owned bf16 state
  * pool, as on the "flashinfer.kda_decode.packed_kda_decode" page, with the
  * recurrence of "KDA Chunk Prefill on Ascend A3" (section "Mathematical

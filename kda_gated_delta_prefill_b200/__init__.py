@@ -29,7 +29,8 @@ EXPORTED = ("kda_status_string", "kda_prefill_workspace_size", "kda_prefill_forw
             "kda_prefill_host_staging_size", "kda_prefill_forward_host", "kda_prefill_device_error",
             "kda_l2norm_bf16", "kda_prefill_kernel_launches", "kda_decode_step",
             "kda_prefill_backward_workspace_size", "kda_prefill_backward_kernel_launches", "kda_prefill_backward",
-            "kda_prefill_state_bf16_workspace_size", "kda_prefill_forward_state_bf16")
+            "kda_prefill_state_bf16_workspace_size", "kda_prefill_forward_state_bf16",
+            "kda_prefill_forward_save", "kda_prefill_backward_saved")
 
 
 class KdaError(RuntimeError):
@@ -81,6 +82,10 @@ def lib():
         L.kda_prefill_state_bf16_workspace_size.restype = Z
         L.kda_prefill_forward_state_bf16.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, Z, P]
         L.kda_prefill_forward_state_bf16.restype = I
+        L.kda_prefill_forward_save.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, Z, P]
+        L.kda_prefill_forward_save.restype = I
+        L.kda_prefill_backward_saved.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, Z, P]
+        L.kda_prefill_backward_saved.restype = I
         _lib = L
         return L
 
@@ -173,12 +178,34 @@ def backward_kernel_launches(B, T, H, HV, K=128, V=128, num_seqs=0) -> int:
     return int(lib().kda_prefill_backward_kernel_launches(B, T, H, HV, K, V, num_seqs))
 
 
+def forward_save(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o=None, final_state=None, saved=None,
+                 stream=None):
+    """The forward that also keeps what the backward needs; returns (o, final_state, saved).  Pass ``saved`` to
+    ``backward(..., saved=saved)`` with the same inputs."""
+    import torch
+    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
+    if o is None:
+        o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=q.device)
+    if final_state is None:
+        final_state = torch.empty(N, HV, K, V, dtype=torch.float32, device=q.device)
+    num_seqs = N if cu_seqlens is not None else 0
+    if saved is None:
+        saved = torch.empty(max(backward_workspace_size(B, T, H, HV, K, V, num_seqs), 1), dtype=torch.uint8,
+                            device=q.device)
+    rc = lib().kda_prefill_forward_save(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                                        _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(o), _ptr(final_state),
+                                        _ptr(saved), saved.numel(), _stream_ptr(stream))
+    _check(rc, "kda_prefill_forward_save")
+    return o, final_state, saved
+
+
 def backward(q, k, v, g, beta, dout, initial_state=None, dht=None, cu_seqlens=None, *, want_dh0=None,
-             workspace=None, stream=None):
+             workspace=None, saved=None, stream=None):
     """Gradients of sum(o * dout) + sum(final_state * dht) for the forward on the same inputs (CUDA).
 
     Returns (dq, dk [B,T,H,K] bf16, dv [B,T,HV,V] bf16, dg [B,T,HV,K] fp32, dbeta [B,T,HV] fp32,
-    dh0 [N,HV,K,V] fp32, or None when there is no initial state and want_dh0 is not set).
+    dh0 [N,HV,K,V] fp32, or None when there is no initial state and want_dh0 is not set).  With ``saved`` (from
+    ``forward_save`` on the same inputs) the forward is not recomputed.
     """
     import torch
     B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
@@ -195,14 +222,16 @@ def backward(q, k, v, g, beta, dout, initial_state=None, dht=None, cu_seqlens=No
         want_dh0 = initial_state is not None
     dh0 = torch.empty(N, HV, K, V, dtype=torch.float32, device=dev) if want_dh0 else None
     num_seqs = N if cu_seqlens is not None else 0
-    ws_bytes = backward_workspace_size(B, T, H, HV, K, V, num_seqs)
-    if workspace is None:
+    fn, name = lib().kda_prefill_backward, "kda_prefill_backward"
+    if saved is not None:
+        workspace, fn, name = saved, lib().kda_prefill_backward_saved, "kda_prefill_backward_saved"
+    elif workspace is None:
+        ws_bytes = backward_workspace_size(B, T, H, HV, K, V, num_seqs)
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    rc = lib().kda_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
-                                    _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(dout), _ptr(dht),
-                                    _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dh0),
-                                    _ptr(workspace), workspace.numel(), _stream_ptr(stream))
-    _check(rc, "kda_prefill_backward")
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), num_seqs, B, T,
+            H, HV, K, V, _ptr(dout), _ptr(dht), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dh0),
+            _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _check(rc, name)
     return dq, dk, dv, dg, dbeta, dh0
 
 

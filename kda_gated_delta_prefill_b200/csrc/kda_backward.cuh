@@ -864,7 +864,9 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 }
             }
         }
-        // dG_L += sum over rows of kn X2: the eight lanes g of a column, then the warps of the other row blocks
+        // dG_L += sum over rows of kn X2: the eight lanes g of a column, then (in a fixed order, after the next
+        // barrier) the four row blocks' partial sums, kept in the work region (free since phase 6)
+        float(*glpart)[DK] = reinterpret_cast<float(*)[DK]>(sm + S::WK);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
 #pragma unroll
@@ -873,7 +875,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, 4));
                 x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, 8));
                 x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, 16));
-                if (g == 0) atomicAdd(&dgl[64 * nh + 8 * j + 2 * t4 + e], x);
+                if (g == 0) glpart[mt][64 * nh + 8 * j + 2 * t4 + e] = x;
             }
     }
     {
@@ -975,7 +977,10 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     }
     __syncthreads();
     if (tid < DK) {
+        const float(*glpart)[DK] = reinterpret_cast<const float(*)[DK]>(sm + S::WK);
         float acc = dgl[tid];  // G_L = G of the last row
+#pragma unroll
+        for (int m = 0; m < 4; ++m) acc = __fadd_rn(acc, glpart[m][tid]);
         for (int i = CH - 1; i >= 0; --i) {
             acc = __fadd_rn(acc, dG[i][tid]);
             if (i < nvalid) p.dg[((row0 + i) * p.HV + h) * DK + tid] = acc;

@@ -4,11 +4,13 @@
 
 namespace {
 
-// Backward workspace: [chunk_off (N+1)] for packed batches, then the forward's per-chunk blocks, the chunk
-// start states, the gradients at the chunk end states, the final state of the recomputed forward, and the
-// per-value-head gradients at the normalised q/k rows.
+// Backward workspace (also the buffer a forward saves for the backward): the forward's own workspace (chunk
+// offsets and order for packed batches, the per-chunk blocks, segment scratch), then the chunk start states and
+// the gradients at the chunk end states (bf16), the final state of a recomputed forward, and the per-value-head
+// gradients at the normalised q/k rows.
 struct BwdWorkspace {
-    size_t chunk_off = 0, items = 0, states = 0, dstates = 0, final_state = 0, dqn = 0, dkn = 0, total = 0;
+    size_t chunk_off = 0, items = 0, fwd_total = 0, states = 0, dstates = 0, final_state = 0, dqn = 0, dkn = 0,
+           total = 0;
     int64_t max_chunks = 0;
 };
 
@@ -17,17 +19,14 @@ BwdWorkspace bwd_workspace_layout(int B, int T, int HV, int num_seqs)
     BwdWorkspace w;
     const bool varlen = num_seqs > 0;
     const int64_t N = varlen ? num_seqs : B;
-    w.max_chunks = varlen ? (static_cast<int64_t>(T) + CH - 1) / CH + num_seqs
-                          : static_cast<int64_t>(B) * ((T + CH - 1) / CH);
+    const Workspace f = workspace_layout(B, T, HV, num_seqs);
+    w.max_chunks = f.max_chunks;
+    w.chunk_off = f.chunk_off;
+    w.items = f.items;
+    w.fwd_total = f.total;
     const size_t rows = static_cast<size_t>(B) * T, state = static_cast<size_t>(DK) * DV * sizeof(float);
     const size_t state16 = static_cast<size_t>(DK) * DV * 2;  // the per-chunk states and gradients are bf16
-    size_t off = 0;
-    if (varlen) {
-        w.chunk_off = off;
-        off += round_up((static_cast<size_t>(num_seqs) + 1) * 4, kAlign);
-    }
-    w.items = off;
-    off = round_up(off + static_cast<size_t>(w.max_chunks) * HV * kda::ITEM_BYTES, kAlign);
+    size_t off = round_up(f.total, kAlign);
     w.states = off;
     off = round_up(off + static_cast<size_t>(w.max_chunks) * HV * state16, kAlign);
     w.dstates = off;
@@ -41,6 +40,12 @@ BwdWorkspace bwd_workspace_layout(int B, int T, int HV, int num_seqs)
     w.total = off;
     return w;
 }
+
+kda_status_t backward_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                           const float *initial_state, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H,
+                           int HV, int K, int V, const void *dout, const float *dht, void *dq, void *dk, void *dv,
+                           float *dg, float *dbeta, float *dh0, void *workspace, size_t workspace_bytes, void *stream,
+                           bool recompute);
 
 }  // namespace
 
@@ -67,6 +72,55 @@ extern "C" kda_status_t kda_prefill_backward(const void *q, const void *k, const
                                              int K, int V, const void *dout, const float *dht, void *dq, void *dk,
                                              void *dv, float *dg, float *dbeta, float *dh0, void *workspace,
                                              size_t workspace_bytes, void *stream)
+{
+    return backward_impl(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, B, T, H, HV, K, V, dout, dht, dq, dk,
+                         dv, dg, dbeta, dh0, workspace, workspace_bytes, stream, true);
+}
+
+extern "C" kda_status_t kda_prefill_backward_saved(const void *q, const void *k, const void *v, const float *g,
+                                                   const float *beta, const float *initial_state,
+                                                   const int32_t *cu_seqlens, int num_seqs, int B, int T, int H,
+                                                   int HV, int K, int V, const void *dout, const float *dht, void *dq,
+                                                   void *dk, void *dv, float *dg, float *dbeta, float *dh0,
+                                                   void *saved, size_t saved_bytes, void *stream)
+{
+    return backward_impl(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, B, T, H, HV, K, V, dout, dht, dq, dk,
+                         dv, dg, dbeta, dh0, saved, saved_bytes, stream, false);
+}
+
+extern "C" kda_status_t kda_prefill_forward_save(const void *q, const void *k, const void *v, const float *g,
+                                                 const float *beta, const float *initial_state,
+                                                 const int32_t *cu_seqlens, int num_seqs, int B, int T, int H, int HV,
+                                                 int K, int V, void *o, float *final_state, void *saved,
+                                                 size_t saved_bytes, void *stream)
+{
+    Dims d;
+    const bool varlen = cu_seqlens != nullptr;
+    kda_status_t st = check_dims(B, T, H, HV, K, V, varlen, num_seqs, d);
+    if (st != KDA_OK) return st;
+    const BwdWorkspace ws = bwd_workspace_layout(B, T, HV, varlen ? num_seqs : 0);
+    if (!saved || saved_bytes < ws.total) return KDA_ERR_WORKSPACE;
+    if (!aligned(saved, kAlign)) return KDA_ERR_MISALIGNED;
+    const int64_t tokens = static_cast<int64_t>(B) * T;
+    const size_t nq = static_cast<size_t>(tokens) * H * K * 2, nvb = static_cast<size_t>(tokens) * HV * V * 2;
+    const size_t ng = static_cast<size_t>(tokens) * HV * K * 4, nb = static_cast<size_t>(tokens) * HV * 4;
+    const size_t ns = static_cast<size_t>(d.N) * HV * K * V * 4;
+    const void *ext[] = {q, k, v, g, beta, initial_state, cu_seqlens, o, final_state};
+    const size_t ext_n[] = {nq, nq, nvb, ng, nb, initial_state ? ns : 0,
+                            varlen ? static_cast<size_t>(num_seqs + 1) * 4 : 0, nvb, ns};
+    for (int i = 0; i < 9; ++i)
+        if (overlaps(saved, ws.total, ext[i], ext_n[i])) return KDA_ERR_INVALID_ARG;
+    uint8_t *sb = static_cast<uint8_t *>(saved);
+    return forward_impl(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, B, T, H, HV, K, V, o, final_state, sb,
+                        ws.fwd_total, stream, reinterpret_cast<__nv_bfloat16 *>(sb + ws.states));
+}
+
+namespace {
+kda_status_t backward_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                           const float *initial_state, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H,
+                           int HV, int K, int V, const void *dout, const float *dht, void *dq, void *dk, void *dv,
+                           float *dg, float *dbeta, float *dh0, void *workspace, size_t workspace_bytes, void *stream,
+                           bool recompute)
 {
     Dims d;
     const bool varlen = cu_seqlens != nullptr;
@@ -110,12 +164,13 @@ extern "C" kda_status_t kda_prefill_backward(const void *q, const void *k, const
     uint8_t *items = wsb + ws.items;
     __nv_bfloat16 *states = reinterpret_cast<__nv_bfloat16 *>(wsb + ws.states);
     __nv_bfloat16 *dstates = reinterpret_cast<__nv_bfloat16 *>(wsb + ws.dstates);
-    if (varlen) {
+    if (varlen && recompute) {
         kda::chunk_offsets_kernel<<<1, 1024, 0, s>>>(cu_seqlens, num_seqs, chunk_off);
         if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
     }
-    // 1. the forward's per-chunk blocks, then its carry storing every chunk's start state (no o)
-    if (tokens > 0) {
+    // 1. the forward's per-chunk blocks, then its carry storing every chunk's start state (no o); a saved
+    //    forward left both (and the chunk offsets) in the workspace
+    if (tokens > 0 && recompute) {
         CUtensorMap tq, tk, tv, tg;
         if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -162,12 +217,16 @@ extern "C" kda_status_t kda_prefill_backward(const void *q, const void *k, const
     // The forward carry (start states) and the reverse carry (end-state gradients) both read only the blocks,
     // so they run side by side: the forward one on the high-priority side stream, joined before the chunk kernel.
     CarryLane *lane = nullptr;
-    if (carry_lane(info.dev, lane) != cudaSuccess) return KDA_ERR_CUDA;
-    std::lock_guard<std::mutex> lane_lock(lane->mu);
-    if (cudaEventRecord(lane->fork, s) != cudaSuccess || cudaStreamWaitEvent(lane->stream, lane->fork, 0) != cudaSuccess)
-        return KDA_ERR_CUDA;
-    if (launch_carry(cp, d.N * HV, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
-    if (cudaEventRecord(lane->join, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
+    std::unique_lock<std::mutex> lane_lock;
+    if (recompute) {
+        if (carry_lane(info.dev, lane) != cudaSuccess) return KDA_ERR_CUDA;
+        lane_lock = std::unique_lock<std::mutex>(lane->mu);
+        if (cudaEventRecord(lane->fork, s) != cudaSuccess ||
+            cudaStreamWaitEvent(lane->stream, lane->fork, 0) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        if (launch_carry(cp, d.N * HV, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
+        if (cudaEventRecord(lane->join, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
+    }
 
     // 2. reverse carry: the gradient at every chunk's end state, and at the initial state
     kda::BwdParams bp{};
@@ -203,7 +262,7 @@ extern "C" kda_status_t kda_prefill_backward(const void *q, const void *k, const
         return KDA_ERR_CUDA;
     kda::kda_bwd_carry_kernel<<<d.N * HV * (DV / kda::kBcCols), kda::kBcThreads, kda::BcSmem::TOTAL, s>>>(bp);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
-    if (cudaStreamWaitEvent(s, lane->join, 0) != cudaSuccess) return KDA_ERR_CUDA;
+    if (recompute && cudaStreamWaitEvent(s, lane->join, 0) != cudaSuccess) return KDA_ERR_CUDA;
     if (tokens == 0) return KDA_OK;
 
     // 3. every chunk's gradients, 4. the Q/K groups through the normalisation
@@ -216,4 +275,4 @@ extern "C" kda_status_t kda_prefill_backward(const void *q, const void *k, const
     kda::kda_bwd_norm_kernel<<<static_cast<int>((warps + 7) / 8), 256, 0, s>>>(bp, tokens);
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
-
+}  // namespace

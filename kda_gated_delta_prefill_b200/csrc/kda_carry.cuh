@@ -65,7 +65,7 @@ struct CarryParams {
     int seg_phase;
     int seg_count;
     float *seg_S, *seg_M, *seg_B;  // [units][seg_count][K][V]
-    // Unsegmented launches only: when set, the state at the start of every chunk is also stored, bf16
+    // When set (not in the segment-map pass), the state at the start of every chunk is also stored, bf16
     // [K][V] (nearest even) at states + (global chunk * HV + h) * K * V (the item's index), for the backward.
     __nv_bfloat16 *states;
     int no_o;                      // unsegmented launches: skip o (the O products and stores)
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
             if (lane == 0) mbar_arrive(bar);
         };
         // the state at the start of chunk c (S^T[v][32kq + j] in r) -> states, rows kd = 32kq + j, column v
-        __nv_bfloat16 *dump = kDump && p.seg_phase == 0 ? p.states : nullptr;
+        __nv_bfloat16 *dump = kDump && p.seg_phase != 1 ? p.states : nullptr;
         auto dump_state = [&](const uint32_t (&r)[32], int kq, int c) {
             __nv_bfloat16 *dst = dump + ((c_begin + c) * p.HV + h) * DK * DV + v;
 #pragma unroll

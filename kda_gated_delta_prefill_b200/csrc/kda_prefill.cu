@@ -298,11 +298,30 @@ extern "C" kda_status_t kda_prefill_device_error(unsigned *word, int clear)
     return KDA_OK;
 }
 
+namespace {
+// The forward; `states` (optional): also store every chunk's start state, bf16 [chunks][HV][K][V] (the
+// backward's saved form).
+kda_status_t forward_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                          const float *initial_state, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H,
+                          int HV, int K, int V, void *o, float *final_state, void *workspace, size_t workspace_bytes,
+                          void *stream, __nv_bfloat16 *states);
+}  // namespace
+
 extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const void *v, const float *g,
                                             const float *beta, const float *initial_state,
                                             const int32_t *cu_seqlens, int num_seqs, int B, int T, int H, int HV,
                                             int K, int V, void *o, float *final_state, void *workspace,
                                             size_t workspace_bytes, void *stream)
+{
+    return forward_impl(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, B, T, H, HV, K, V, o, final_state,
+                        workspace, workspace_bytes, stream, nullptr);
+}
+
+namespace {
+kda_status_t forward_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                          const float *initial_state, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H,
+                          int HV, int K, int V, void *o, float *final_state, void *workspace, size_t workspace_bytes,
+                          void *stream, __nv_bfloat16 *states)
 {
     Dims d;
     const bool varlen = cu_seqlens != nullptr;
@@ -397,6 +416,7 @@ extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const 
     cp.HV = HV;
     cp.N = d.N;
     cp.chunks_per_seq = (T + CH - 1) / CH;
+    cp.states = states;
 
     const int segments = ws.segments > 1 ? carry_segments(B, T, HV, varlen, info.sms) : 1;
     if (segments > 1) {
@@ -446,6 +466,7 @@ extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const 
         return KDA_ERR_CUDA;
     return KDA_OK;
 }
+}  // namespace
 
 extern "C" size_t kda_prefill_host_staging_size(int B, int T, int H, int HV, int K, int V, int num_seqs,
                                                 int has_initial_state, int has_cu_seqlens)

@@ -137,3 +137,35 @@ def test_backward_full_workload_sampled():
     got = [sel(out[i], 2).float().numpy().astype(np.float64) for i in range(5)] + [sel(out[5], 1).numpy()]
     report = _compare(got, ref)
     assert report["dq"][0] < REL_FRO
+
+
+@pytest.mark.parametrize("B,T,H,HV,cu,exact", [
+    (2, 150, 1, 2, None, True),      # one carry launch
+    (1, 2048, 4, 4, None, True),     # the forward cut into parts (side-stream carries)
+    (1, 8192, 1, 1, None, False),    # one unit, long: the segmented carry (affine maps and a scan)
+    (1, 300, 2, 4, [0, 1, 64, 65, 65, 300], True),  # packed sequences
+])
+def test_saved_forward_then_backward(B, T, H, HV, cu, exact):
+    """forward_save + backward(saved=...) against the oracle, against the recomputing backward (bit for bit
+    where the saved forward's carry is the same computation) and with o/final_state equal to the forward's."""
+    import kda_gated_delta_prefill_b200 as kda
+    q, k, v, g, beta, s0, dout, dh, cu_t = _case(B, T, H, HV, seed=970 + T, cu=cu)
+    c = lambda t: None if t is None else t.cuda()
+    xs = [c(t) for t in (q, k, v, g, beta)]
+    o1, sN1, saved = kda.forward_save(*xs, c(s0), c(cu_t))
+    o2, sN2 = kda.forward(*xs, c(s0), c(cu_t))
+    torch.cuda.synchronize()
+    if cu is None:
+        assert torch.equal(o1, o2)
+    else:
+        assert torch.equal(o1[:, :cu[-1]], o2[:, :cu[-1]])
+    assert torch.equal(sN1, sN2)
+    got_s = kda.backward(*xs, c(dout), c(s0), c(dh), c(cu_t), want_dh0=True, saved=saved)
+    got_r = kda.backward(*xs, c(dout), c(s0), c(dh), c(cu_t), want_dh0=True)
+    torch.cuda.synchronize()
+    assert kda.device_error(clear=True) == 0
+    if exact:
+        for a, b in zip(got_s, got_r):
+            assert torch.equal(a, b)
+    ref = oracle.backward(q, k, v, g, beta, s0, dout.float().numpy(), dh.numpy(), cu_t)
+    _compare([t.float().cpu().numpy().astype(np.float64) for t in got_s[:5]] + [got_s[5].cpu().numpy()], ref)
