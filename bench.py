@@ -438,10 +438,16 @@ def bench_backward(args, case, world, rank, dev):
     num_seqs = N if x["cu_seqlens"] is not None else 0
     ws = torch.empty(kda.backward_workspace_size(B, T, H, HV, K, V, num_seqs), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    saved = None
+    if args.saved:  # the forward that keeps the blocks and chunk states, once, outside the timed region
+        _, _, saved = kda.forward_save(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"],
+                                       x["cu_seqlens"], saved=ws, stream=stream)
+        config["saved_forward"] = True
 
     def step():
         return kda.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], gr["dout"], x["initial_state"], gr["dht"],
-                            x["cu_seqlens"], workspace=ws, stream=stream)
+                            x["cu_seqlens"], workspace=None if saved is not None else ws, saved=saved,
+                            stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -487,7 +493,8 @@ def bench_backward(args, case, world, rank, dev):
             for k in gd:
                 gd[k].copy_(gh[k], non_blocking=True)
             outs = kda.backward(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], gd["dout"], xd["initial_state"],
-                                gd["dht"], None, workspace=ws, stream=stream)
+                                gd["dht"], None, workspace=None if saved is not None else ws, saved=saved,
+                                stream=stream)
             if outs_h is None:
                 outs_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
             for a, b in zip(outs_h, outs):
@@ -510,7 +517,8 @@ def bench_backward(args, case, world, rank, dev):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = time_oracle_backward(case)
         cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
-    launches = kda.backward_kernel_launches(B, T, H, HV, K, V, num_seqs)
+    # the saved form skips the recomputation (intra-chunk and forward carry launches, and the chunk offsets)
+    launches = kda.backward_kernel_launches(B, T, H, HV, K, V, num_seqs) - (2 + (1 if num_seqs else 0) if saved is not None else 0)
     line = {"metric": BWD_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config,
@@ -534,6 +542,9 @@ def main():
     ap.add_argument("--workload", default="long_T65536_H64_state",
                     help="a prefill workload name, backward_<prefill workload name> for the backward, or "
                          "decode_B1024_H12 for the decode step")
+    ap.add_argument("--saved", action="store_true",
+                    help="prefill workloads: time the forward that saves for the backward; backward workloads: time "
+                         "the backward from a saved forward (forward_save once, untimed)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile-T", type=int, default=0,
@@ -607,13 +618,22 @@ def main():
     B, T, H, HV, K, V, N = case.B, case.T, case.H, case.HV, case.K, case.V, case.N
     o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=dev)
     s = torch.empty(N, HV, K, V, dtype=torch.float32, device=dev)
-    ws_n = kda.workspace_size(B, T, H, HV, K, V, N if x["cu_seqlens"] is not None else 0)
-    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
+    num_seqs = N if x["cu_seqlens"] is not None else 0
     stream = torch.cuda.current_stream(dev)
+    if args.saved:  # the forward that also keeps what the backward needs
+        ws = torch.empty(max(kda.backward_workspace_size(B, T, H, HV, K, V, num_seqs), 1), dtype=torch.uint8,
+                         device=dev)
+        config["saves_for_backward"] = True
 
-    def step():
-        kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"], x["cu_seqlens"], o=o,
-                    final_state=s, workspace=ws, stream=stream)
+        def step():
+            kda.forward_save(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"], x["cu_seqlens"], o=o,
+                             final_state=s, saved=ws, stream=stream)
+    else:
+        ws = torch.empty(max(kda.workspace_size(B, T, H, HV, K, V, num_seqs), 1), dtype=torch.uint8, device=dev)
+
+        def step():
+            kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"], x["cu_seqlens"], o=o,
+                        final_state=s, workspace=ws, stream=stream)
 
     for _ in range(args.warmup):
         step()
