@@ -23,7 +23,8 @@
 // cumulative sum is dg.  Three kernels:
 //   kda_bwd_carry_kernel  dS' of every chunk, walking each sequence backwards
 //                         (reads the forward's per-chunk blocks),
-//   kda_bwd_chunk_kernel  every chunk's gradients at once (fp32 CUDA cores),
+//   kda_bwd_chunk_kernel  every chunk's gradients at once (fp32 arithmetic,
+//                         TF32 tensor-core MMAs for the products),
 //   kda_bwd_norm_kernel   sums a Q/K head's group and applies the L2
 //                         normalisation's Jacobian.
 // Gate factors exp(G_i - G_j) are formed per 16-token block I with the
@@ -50,7 +51,7 @@ struct BwdParams {
     float *dg, *dbeta;                      // [rows][HV][K], [rows][HV]
     const int32_t *cu, *chunk_off;          // packed sequences (cu [N+1], chunk_off [N+1]) or null
     unsigned *err;
-    int T, H, HV, N, chunks_per_seq, total_chunks;
+    int T, H, HV, N, chunks_per_seq;
 };
 
 // (sequence, first token row, valid rows) of global chunk index `chunk`
@@ -303,7 +304,7 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
 }
 
 // ---------------------------------------------------------------------------------------------------------
-// Chunk gradients: one CTA of 256 threads per (chunk, value head), fp32 throughout.
+// Chunk gradients: one CTA of 256 threads per (chunk, value head); fp32 values, TF32 MMAs (fp32 accumulate).
 constexpr int kBwThreads = 256, kBwCols = 16;  // value columns per pass over the state
 constexpr int kRow = 132;                      // padded row stride (floats) of the [64][128] operand tiles
 constexpr int kRowC = 68;                      // padded row stride of the [64][64] tiles

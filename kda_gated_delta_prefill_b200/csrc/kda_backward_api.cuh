@@ -256,7 +256,6 @@ kda_status_t backward_impl(const void *q, const void *k, const void *v, const fl
     bp.HV = HV;
     bp.N = d.N;
     bp.chunks_per_seq = (T + CH - 1) / CH;
-    bp.total_chunks = static_cast<int>(ws.max_chunks);
     if (cudaFuncSetAttribute(kda::kda_bwd_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kda::BcSmem::TOTAL) != cudaSuccess)
         return KDA_ERR_CUDA;
