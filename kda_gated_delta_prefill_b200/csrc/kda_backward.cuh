@@ -174,12 +174,29 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
     store_dsh();
     __syncthreads();
 
+    // this thread's share of a chunk's dO rows (row tid / 8, eight columns), loaded one chunk ahead
+    auto load_dout = [&](int c) {
+        const int i = tid >> 3, cc = 8 * (tid & 7);
+        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+        if (c >= 0 && i < min(CH, len - c * CH))
+            raw = *reinterpret_cast<const uint4 *>(p.dout + ((row0 + static_cast<int64_t>(c) * CH + i) * p.HV + h) * DV +
+                                                   vc0 + cc);
+        return raw;
+    };
+    auto put_dout = [&](uint4 raw) {  // as fp16 (zero past the sequence's end)
+        const int i = tid >> 3, cc = 8 * (tid & 7);
+        const uint4 w = make_uint4(pack_f16(bf16lo(raw.x), bf16hi(raw.x)), pack_f16(bf16lo(raw.y), bf16hi(raw.y)),
+                                   pack_f16(bf16lo(raw.z), bf16hi(raw.z)), pack_f16(bf16lo(raw.w), bf16hi(raw.w)));
+        *reinterpret_cast<uint4 *>(dOh + i * kBcPad + cc) = w;
+    };
+    if (nck > 0) put_dout(load_dout(nck - 1));  // visible after the first barrier below
+
     bool ok = true;
     for (int it = 0; it < nck; ++it) {
         const int c = nck - 1 - it, st = it & 1;
         const uint32_t blk = sb + st * S::STAGE;
         if (tid == 0 && c > 0) request(c - 1, st ^ 1);  // that stage was released by the previous iteration
-        const int nrows = min(CH, len - c * CH);
+        const uint4 next_dout = load_dout(c - 1);       // lands while this chunk computes
         {
             // dS is the gradient at chunk c's end state: store it
             __nv_bfloat16 *dst = p.dstates + ((c_begin + c) * p.HV + h) * DK * DV + vc0;
@@ -189,18 +206,6 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
                 for (int hf = 0; hf < 2; ++hf)
                     *reinterpret_cast<__nv_bfloat162 *>(dst + key_of(hf) * DV + col_of(j, 0)) =
                         __floats2bfloat162_rn(acc[j][2 * hf], acc[j][2 * hf + 1]);
-            // dO rows of the chunk as fp16 (zero past the sequence's end)
-            const int i = tid >> 3, cc = 8 * (tid & 7);
-            uint4 w = make_uint4(0u, 0u, 0u, 0u);
-            if (i < nrows) {
-                const uint4 raw = *reinterpret_cast<const uint4 *>(
-                    p.dout + ((row0 + static_cast<int64_t>(c) * CH + i) * p.HV + h) * DV + vc0 + cc);
-                w.x = pack_f16(bf16lo(raw.x), bf16hi(raw.x));
-                w.y = pack_f16(bf16lo(raw.y), bf16hi(raw.y));
-                w.z = pack_f16(bf16lo(raw.z), bf16hi(raw.z));
-                w.w = pack_f16(bf16lo(raw.w), bf16hi(raw.w));
-            }
-            *reinterpret_cast<uint4 *>(dOh + i * kBcPad + cc) = w;
         }
         if (tid == 0) {
             const bool landed = mbar_wait(sb + S::BAR + 8 * st, waited[st] & 1);
@@ -280,6 +285,7 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
         }
         __syncthreads();  // every read of dS's fp16 copy, dO, dVnew and the stage is done
         store_dsh();
+        put_dout(next_dout);
         // (the next iteration's barrier orders these writes before their reads)
     }
     if (!ok) {
