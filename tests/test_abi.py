@@ -177,3 +177,42 @@ def test_backward_workspace_and_launch_counts(L):
     assert L.kda_prefill_backward_workspace_size(1, 64, 1, 1, 64, 128, 0) == 0
     assert L.kda_prefill_backward_kernel_launches(1, 64, 1, 1, 128, 128, 0) == 5
     assert L.kda_prefill_backward_kernel_launches(1, 64, 1, 1, 128, 128, 3) == 6
+
+
+def test_saved_forward_and_backward_reject_small_or_overlapping_buffers(L):
+    P = ctypes.c_void_p
+    step = 1 << 32
+    ptr = lambda i: P(FAKE + int(i * step))
+    need = L.kda_prefill_backward_workspace_size(1, 64, 1, 1, 128, 128, 0)
+    assert need > L.kda_prefill_workspace_size(1, 64, 1, 1, 128, 128, 0)  # the forward's workspace, then more
+    fwd = lambda saved, nbytes, o=8: L.kda_prefill_forward_save(ptr(1), ptr(2), ptr(3), ptr(4), ptr(5), None, None, 0,
+                                                                1, 64, 1, 1, 128, 128, ptr(o), ptr(9), saved, nbytes,
+                                                                None)
+    assert fwd(ptr(12), need - 256) == 4           # too small
+    assert fwd(None, need) == 4                    # missing
+    assert fwd(P(FAKE + 12 * step + 8), need) == 3  # misaligned
+    assert fwd(ptr(8), need) == 1                  # overlaps o
+    assert L.kda_prefill_forward_save(ptr(1), ptr(2), ptr(3), ptr(4), ptr(5), None, None, 0, 1, 64, 1, 1, 64, 128,
+                                      ptr(8), ptr(9), ptr(12), need, None) == 2
+    bwd = lambda saved, nbytes: L.kda_prefill_backward_saved(ptr(1), ptr(2), ptr(3), ptr(4), ptr(5), None, None, 0, 1,
+                                                             64, 1, 1, 128, 128, ptr(6), None, ptr(7), ptr(8), ptr(9),
+                                                             ptr(10), ptr(11), None, saved, nbytes, None)
+    assert bwd(ptr(12), need - 256) == 4
+    assert bwd(ptr(6), need) == 1  # overlaps dout
+
+
+def test_bf16_state_forward_rejects_bad_arguments(L):
+    P = ctypes.c_void_p
+    step = 1 << 32
+    ptr = lambda i: P(FAKE + int(i * step))
+    need = L.kda_prefill_state_bf16_workspace_size(1, 64, 1, 1, 128, 128, 0)
+    # two fp32 states more than the forward's workspace
+    assert need >= L.kda_prefill_workspace_size(1, 64, 1, 1, 128, 128, 0) + 2 * 128 * 128 * 4
+    f = lambda s0, sN, ws, nbytes, K=128: L.kda_prefill_forward_state_bf16(
+        ptr(1), ptr(2), ptr(3), ptr(4), ptr(5), s0, None, 0, 1, 64, 1, 1, K, 128, ptr(8), sN, ws, nbytes, None)
+    assert f(ptr(6), ptr(9), ptr(12), need, K=64) == 2
+    assert f(ptr(6), None, ptr(12), need) == 1                      # final_state required
+    assert f(ptr(6), P(FAKE + 9 * step + 8), ptr(12), need) == 3    # final_state misaligned
+    assert f(ptr(6), ptr(9), ptr(12), need - 256) == 4
+    assert f(ptr(6), ptr(9), ptr(9), need) == 1                     # workspace overlaps final_state
+    assert f(ptr(6), P(FAKE + 6 * step + 16384), ptr(12), need) == 1  # states partly overlap
