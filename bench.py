@@ -35,6 +35,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "KDA chunk-prefill tokens·heads/s @T=64K,HV=64,K=V=128; % of roofline"
 UNIT = "tokens·heads/s"
+FLUSH_BELOW_BYTES = 512 << 20  # workloads under this many bytes get an L2 flush between timed steps
+FLUSH_BYTES = 256 << 20
 BYTES_PER_TOKEN_HEAD = 256 + 256 + 256 + 512 + 4 + 256  # q, k, v, g, beta, o (H == HV)
 
 
@@ -575,10 +577,12 @@ def main():
         return bench_decode(args, case, world, rank, None)
     if backward and args.impl == "reference":
         return bench_backward(args, case, world, rank, None)
+    # workloads whose bytes fit a few times in the 126 MB L2 get an L2 flush between timed steps
+    flush = not decode and algorithmic_bytes(case) < FLUSH_BELOW_BYTES
     config = None if decode else {"workload": case.name, "B": case.B, "T": case.T, "H": case.H, "HV": case.HV, "K": case.K,
               "V": case.V, "chunk": 64, "initial_state": case.state != "none",
-              "l2": "inputs (6.5 GB) larger than L2; no flush" if case.name.startswith("long")
-              else "inputs re-used across steps (may hit L2)",
+              "l2": ("L2 flushed between steps (a %d MB write outside the per-step events)" % (FLUSH_BYTES >> 20))
+              if flush else "inputs (%.1f GB) larger than L2; no flush" % (algorithmic_bytes(case) / 1e9),
               "parallelism": f"independent replicas x{args.gpus} (weak)" if args.gpus > 1 else "single GPU"}
 
     if args.impl == "reference":
@@ -651,6 +655,7 @@ def main():
 
     # ---- timed region: K steps; per-launch CUDA events on the launching stream ----
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    scratch = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev) if flush else None
     with ClockSampler(torch.cuda.current_device()) as clk:
         barrier()
         torch.cuda.synchronize()
@@ -658,14 +663,17 @@ def main():
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for i in range(args.steps):
+            if flush:
+                scratch.zero_()  # evict the previous step's data from L2
             evs[i][0].record(stream)
             step()
             evs[i][1].record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
         barrier()
-    total_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     launch_ms = [a.elapsed_time(b) for a, b in evs]
+    # with flushes the steps are timed by their own events (the flushes excluded), else by the whole bracket
+    total_ms = max_over_ranks(sum(launch_ms) if flush else t0.elapsed_time(t1), world, dev)
     ms_per_step = total_ms / args.steps
     th_per_step = case.tokens * HV
     value = weak_throughput(th_per_step, world, total_ms, args.steps)
