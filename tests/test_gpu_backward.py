@@ -169,3 +169,61 @@ def test_saved_forward_then_backward(B, T, H, HV, cu, exact):
             assert torch.equal(a, b)
     ref = oracle.backward(q, k, v, g, beta, s0, dout.float().numpy(), dh.numpy(), cu_t)
     _compare([t.float().cpu().numpy().astype(np.float64) for t in got_s[:5]] + [got_s[5].cpu().numpy()], ref)
+
+
+def _gen_run(x, gr, want_dh0):
+    import kda_gated_delta_prefill_b200 as kda
+    c = lambda t: None if t is None else t.cuda()
+    out = kda.backward(c(x["q"]), c(x["k"]), c(x["v"]), c(x["g"]), c(x["beta"]), c(gr["dout"]),
+                       c(x["initial_state"]), c(gr["dht"]), c(x["cu_seqlens"]), want_dh0=want_dh0)
+    torch.cuda.synchronize()
+    assert kda.device_error(clear=True) == 0
+    return out
+
+
+@pytest.mark.parametrize("mode", [dict(qk_mode="gain"), dict(qk_mode="tiny"), dict(qk_mode="zero_rows"),
+                                  dict(gate="logsig128"), dict(gate="logsig1"), dict(gate="zero"),
+                                  dict(gate="uniform5"), dict(beta="one"), dict(beta="edge"),
+                                  dict(beta="zero", state="quarter"), dict(state="quarter"), dict(state="zeros")],
+                         ids=lambda m: "-".join(f"{k}={v}" for k, v in m.items()))
+def test_backward_generator_modes(mode):
+    """The forward's input modes (Q/K gain, tiny and all-zero rows; gates from -log(1+e^x)/128 down to
+    U[-5, 0] per token; beta of one, zero and the repeating edge pattern; state scales) through the backward."""
+    from kda_gated_delta_prefill_b200 import inputs as gen
+    case = gen.Case("mode", B=1, T=300, H=2, HV=2, seed=17, **mode)
+    x = gen.make_inputs(case)
+    gr = gen.make_backward_grads(case)
+    has_state = x["initial_state"] is not None
+    out = _gen_run(x, gr, want_dh0=has_state)
+    ref = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"],
+                          gr["dout"].float().numpy(), gr["dht"].numpy())
+    got = [t.float().cpu().numpy().astype(np.float64) for t in out[:5]]
+    if has_state:
+        got.append(out[5].cpu().numpy())
+    _compare(got, list(ref[:len(got)]))
+
+
+def test_backward_gqa_group_8():
+    got, ref = _run(*_case(1, 257, 2, 16, seed=977))
+    _compare(got, ref)
+
+
+def test_backward_varlen_gqa_workload_sampled():
+    """The packed-sequence GQA workload (lengths 1, 63, 64, 65, 777, 2048, 8192; H=8, HV=32; gates U[-5, 0];
+    beta = sigmoid(N(0, 4)); per-sequence states) on the GPU for all heads; the oracle checks Q/K head 5 and
+    its four value heads over every sequence."""
+    from kda_gated_delta_prefill_b200 import inputs as gen
+    case = gen.VARLEN_GQA
+    x = gen.make_inputs(case)
+    gr = gen.make_backward_grads(case)
+    out = _gen_run(x, gr, want_dh0=True)
+    hq, grp = 5, case.HV // case.H
+    hv = torch.arange(hq * grp, (hq + 1) * grp)
+    sel = lambda t, dim, idx: t.index_select(dim, idx).contiguous()
+    hqi = torch.tensor([hq])
+    ref = oracle.backward(sel(x["q"], 2, hqi), sel(x["k"], 2, hqi), sel(x["v"], 2, hv), sel(x["g"], 2, hv),
+                          sel(x["beta"], 2, hv), sel(x["initial_state"], 1, hv),
+                          sel(gr["dout"], 2, hv).float().numpy(), sel(gr["dht"], 1, hv).numpy(), x["cu_seqlens"])
+    got = [sel(out[0].cpu(), 2, hqi), sel(out[1].cpu(), 2, hqi)] + \
+          [sel(out[i].cpu(), 2, hv) for i in (2, 3, 4)] + [sel(out[5].cpu(), 1, hv)]
+    _compare([t.float().numpy().astype(np.float64) for t in got], ref)
