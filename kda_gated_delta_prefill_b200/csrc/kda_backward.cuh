@@ -314,9 +314,13 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
 constexpr int kBwThreads = 256, kBwCols = 16;  // value columns per pass over the state
 constexpr int kRow = 132;                      // padded row stride (floats) of the [64][128] operand tiles
 constexpr int kRowC = 68;                      // padded row stride of the [64][64] tiles
-// element (r, c) of a [64][16] fp32 value-column tile: rows of 16 floats, columns XOR-swizzled by 4 (r / 2 % 4)
-// so that the eight rows of an MMA fragment fall into distinct banks
-__device__ __forceinline__ int vsw(int r, int c) { return r * kBwCols + (c ^ (((r >> 1) & 3) << 2)); }
+// element (r, c) of a [64][16] fp32 value-column tile: rows of 16 floats, the two 8-column halves swapped in
+// rows with bit 1 set.  Scalar reads of 4 rows x 8 columns and 8-byte accesses of 4 rows x 4 column pairs
+// (a half warp) then fall into 32 distinct banks.
+__device__ __forceinline__ int vsw(int r, int c) { return r * kBwCols + (c ^ (((r >> 1) & 1) << 3)); }
+// column of element (r, c) in a [rows][16] bf16 pass buffer (S, dS', dO): the two 16-byte halves of a row swapped
+// in rows with bit 2 set, so that 4-byte reads of one column pair from 8 consecutive rows hit 8 distinct bank quads
+__device__ __forceinline__ int bsw(int r, int c) { return c ^ (((r >> 2) & 1) << 3); }
 struct BwSmem {
     static constexpr int KA = 0;                          // kn_id exp(G_id - m_Id)
     static constexpr int QA = KA + CH * kRow * 4;         // qn_id exp(G_id - m_Id)
@@ -605,10 +609,10 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     // pass vb's columns into buffer b: S, dS' and dO rows are 32 bytes (two 16-byte copies each)
     auto fetch = [&](int vb, int b) {
         const int row = tid >> 1, half = 8 * (tid & 1);
-        cp_async16(smem_u32(&SVb(b)[row][half]), Sg + row * DV + vb + half);
-        cp_async16(smem_u32(&DSVb(b)[row][half]), dSg + row * DV + vb + half);
+        cp_async16(smem_u32(&SVb(b)[row][bsw(row, half)]), Sg + row * DV + vb + half);
+        cp_async16(smem_u32(&DSVb(b)[row][bsw(row, half)]), dSg + row * DV + vb + half);
         if (row < nvalid && tid < 2 * CH)
-            cp_async16(smem_u32(&DOBb(b)[row][half]), p.dout + ((row0 + row) * p.HV + h) * DV + vb + half);
+            cp_async16(smem_u32(&DOBb(b)[row][bsw(row, half)]), p.dout + ((row0 + row) * p.HV + h) * DV + vb + half);
         cp_async_commit();
     };
     if (tid < CH && tid >= nvalid) {  // rows past the end stay zero in both buffers
@@ -632,7 +636,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         const __nv_bfloat16(*SVT)[kBwCols] = SVb(buf);
         const __nv_bfloat16(*DST)[kBwCols] = DSVb(buf);
         const __nv_bfloat16(*DOV)[kBwCols] = DOBb(buf);
-        if (tid < DK) {
+        if (tid < DK) {  // S and dS' rows share one column order, so physical positions pair up
 #pragma unroll
             for (int c = 0; c < kBwCols; c += 2) {
                 const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&SVT[tid][c]));
@@ -648,8 +652,9 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 const uint32_t a[4] = {to_tf32(__fmul_rn(KA[r0][ks + t4], e0)), to_tf32(__fmul_rn(KA[r1][ks + t4], e0)),
                                        to_tf32(__fmul_rn(KA[r0][ks + t4 + 4], e1)),
                                        to_tf32(__fmul_rn(KA[r1][ks + t4 + 4], e1))};
-                mma_tf32(c[0], a, bf(SVT[ks + t4][g]), bf(SVT[ks + t4 + 4][g]));
-                mma_tf32(c[1], a, bf(SVT[ks + t4][8 + g]), bf(SVT[ks + t4 + 4][8 + g]));
+                const int k0 = ks + t4, k1 = ks + t4 + 4;
+                mma_tf32(c[0], a, bf(SVT[k0][bsw(k0, g)]), bf(SVT[k1][bsw(k1, g)]));
+                mma_tf32(c[1], a, bf(SVT[k0][bsw(k0, 8 + g)]), bf(SVT[k1][bsw(k1, 8 + g)]));
             }
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
@@ -671,14 +676,16 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 const uint32_t a[4] = {to_tf32(__fmul_rn(KB[r0][ks + t4], e0)), to_tf32(__fmul_rn(KB[r1][ks + t4], e0)),
                                        to_tf32(__fmul_rn(KB[r0][ks + t4 + 4], e1)),
                                        to_tf32(__fmul_rn(KB[r1][ks + t4 + 4], e1))};
-                mma_tf32(c[0], a, bf(DST[ks + t4][g]), bf(DST[ks + t4 + 4][g]));
-                mma_tf32(c[1], a, bf(DST[ks + t4][8 + g]), bf(DST[ks + t4 + 4][8 + g]));
+                const int k0 = ks + t4, k1 = ks + t4 + 4;
+                mma_tf32(c[0], a, bf(DST[k0][bsw(k0, g)]), bf(DST[k1][bsw(k1, g)]));
+                mma_tf32(c[1], a, bf(DST[k0][bsw(k0, 8 + g)]), bf(DST[k1][bsw(k1, 8 + g)]));
             }
             for (int js = 16 * mt; js < CH; js += 8) {  // Aqk^T[i][j] = Aqk[j][i], nonzero for j >= i
                 const uint32_t a[4] = {to_tf32(AQ[js + t4][r0]), to_tf32(AQ[js + t4][r1]), to_tf32(AQ[js + t4 + 4][r0]),
                                        to_tf32(AQ[js + t4 + 4][r1])};
-                mma_tf32(c[0], a, bf(DOV[js + t4][g]), bf(DOV[js + t4 + 4][g]));
-                mma_tf32(c[1], a, bf(DOV[js + t4][8 + g]), bf(DOV[js + t4 + 4][8 + g]));
+                const int k0 = js + t4, k1 = js + t4 + 4;
+                mma_tf32(c[0], a, bf(DOV[k0][bsw(k0, g)]), bf(DOV[k1][bsw(k1, g)]));
+                mma_tf32(c[1], a, bf(DOV[k0][bsw(k0, 8 + g)]), bf(DOV[k1][bsw(k1, 8 + g)]));
             }
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
@@ -728,31 +735,42 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         }
         __syncthreads();
         // (e) dQg += dO S^T, dKb -= dv S^T, dKg += Vnew dS'^T (K = these 16 columns, two k8 steps);
-        //     dAqk += dO Vnew^T, dA += dVnew D^T
+        //     dAqk += dO Vnew^T, dA += dVnew D^T.  A k8 step's slots t4 and t4 + 4 carry this thread's column pair
+        //     cp, cp + 1 (any order of K is a valid order as long as A and B share it), so every operand pair
+        //     comes from one 4- or 8-byte shared-memory read.
+        auto pair = [](const __nv_bfloat16(*B)[kBwCols], int r, int c) {
+            return *reinterpret_cast<const uint32_t *>(&B[r][bsw(r, c)]);
+        };
+        constexpr uint32_t kHi = 0xffff0000u;
 #pragma unroll
         for (int kc = 0; kc < kBwCols; kc += 8) {
-            const int c0 = kc + t4, c1 = kc + t4 + 4;
-            const uint32_t aO[4] = {bf(DOV[r0][c0]), bf(DOV[r1][c0]), bf(DOV[r0][c1]), bf(DOV[r1][c1])};
-            const uint32_t aV[4] = {to_tf32(-DVv[vsw(r0, c0)]), to_tf32(-DVv[vsw(r1, c0)]), to_tf32(-DVv[vsw(r0, c1)]),
-                                    to_tf32(-DVv[vsw(r1, c1)])};
-            const uint32_t aN[4] = {to_tf32(VN[vsw(r0, c0)]), to_tf32(VN[vsw(r1, c0)]), to_tf32(VN[vsw(r0, c1)]),
-                                    to_tf32(VN[vsw(r1, c1)])};
-            const uint32_t aD[4] = {to_tf32(DVN[vsw(r0, c0)]), to_tf32(DVN[vsw(r1, c0)]), to_tf32(DVN[vsw(r0, c1)]),
-                                    to_tf32(DVN[vsw(r1, c1)])};
+            const int cp = kc + 2 * t4;
+            const uint32_t o0 = pair(DOV, r0, cp), o1 = pair(DOV, r1, cp);
+            const uint32_t aO[4] = {o0 << 16, o1 << 16, o0 & kHi, o1 & kHi};
+            const float2 v0 = *reinterpret_cast<const float2 *>(&DVv[vsw(r0, cp)]);
+            const float2 v1 = *reinterpret_cast<const float2 *>(&DVv[vsw(r1, cp)]);
+            const float2 n0 = *reinterpret_cast<const float2 *>(&VN[vsw(r0, cp)]);
+            const float2 n1 = *reinterpret_cast<const float2 *>(&VN[vsw(r1, cp)]);
+            const float2 e0 = *reinterpret_cast<const float2 *>(&DVN[vsw(r0, cp)]);
+            const float2 e1 = *reinterpret_cast<const float2 *>(&DVN[vsw(r1, cp)]);
+            const uint32_t aV[4] = {to_tf32(-v0.x), to_tf32(-v1.x), to_tf32(-v0.y), to_tf32(-v1.y)};
+            const uint32_t aN[4] = {to_tf32(n0.x), to_tf32(n1.x), to_tf32(n0.y), to_tf32(n1.y)};
+            const uint32_t aD[4] = {to_tf32(e0.x), to_tf32(e1.x), to_tf32(e0.y), to_tf32(e1.y)};
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int d = 64 * nh + 8 * j + g;
-                const uint32_t s0 = bf(SVT[d][c0]), s1 = bf(SVT[d][c1]);
-                const uint32_t q0 = bf(DST[d][c0]), q1 = bf(DST[d][c1]);
-                mma_tf32(aQ[j], aO, s0, s1);
-                mma_tf32(aB[j], aV, s0, s1);
-                mma_tf32(aG[j], aN, q0, q1);
+                const uint32_t sp = pair(SVT, d, cp), qp = pair(DST, d, cp);
+                mma_tf32(aQ[j], aO, sp << 16, sp & kHi);
+                mma_tf32(aB[j], aV, sp << 16, sp & kHi);
+                mma_tf32(aG[j], aN, qp << 16, qp & kHi);
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int tk = 32 * nh + 8 * j + g;
-                mma_tf32(aAq[j], aO, to_tf32(VN[vsw(tk, c0)]), to_tf32(VN[vsw(tk, c1)]));
-                mma_tf32(aA[j], aD, to_tf32(DDv[vsw(tk, c0)]), to_tf32(DDv[vsw(tk, c1)]));
+                const float2 vn = *reinterpret_cast<const float2 *>(&VN[vsw(tk, cp)]);
+                const float2 dd = *reinterpret_cast<const float2 *>(&DDv[vsw(tk, cp)]);
+                mma_tf32(aAq[j], aO, to_tf32(vn.x), to_tf32(vn.y));
+                mma_tf32(aA[j], aD, to_tf32(dd.x), to_tf32(dd.y));
             }
         }
         __syncthreads();
