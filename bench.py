@@ -377,11 +377,11 @@ BWD_METRIC = "KDA chunk-prefill backward tokens·heads/s @T=64K,HV=64,K=V=128; %
 
 def backward_bytes(case) -> int:
     """Bytes the backward must move at least once: q, k, v, g, beta, dout read; dq, dk, dv, dg, dbeta written;
-    the initial state and dht read, dh0 written."""
+    dht read; with an initial state, that state read and dh0 written."""
     group = case.HV // case.H
     th = case.tokens * case.HV
     per = (256 * 2 / group) * 2 + 256 * 2 + 512 * 2 + 4 * 2 + 256
-    state = case.N * case.HV * 128 * 128 * 4 * (3 if case.state != "none" else 2)
+    state = case.N * case.HV * 128 * 128 * 4 * (3 if case.state != "none" else 1)
     return int(th * per + state)
 
 
