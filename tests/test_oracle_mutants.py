@@ -16,6 +16,7 @@ import pytest
 
 import oracle as oracle_pkg
 from tests import test_oracle_backward as bwd_pins
+from tests import test_oracle_decode as dec_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle_pkg.__file__), "kda_oracle.c")
@@ -62,7 +63,7 @@ def _pin_functions():
 
 def _run_mutant(old, new, tmp_path, pin_functions):
     src = open(SRC).read()
-    assert src.count(old) >= 1, f"mutation site for {mutant} not found"
+    assert src.count(old) >= 1, f"mutation site {old!r} not found"
     mutated = src.replace(old, new, 1)
     c_path = tmp_path / "mut.c"
     so_path = tmp_path / "libmut.so"
@@ -103,3 +104,42 @@ def _bwd_pin_functions():
 def test_backward_pins_catch_mutant(mutant, tmp_path):
     old, new = BWD_MUTANTS[mutant]
     assert _run_mutant(old, new, tmp_path, _bwd_pin_functions()), f"no pin caught mutant {mutant}"
+
+
+# slips in the decode step's row and slot bookkeeping (``oracle.decode_step``, Python); the arithmetic under it is
+# the recurrence above, whose mutants are caught by the forward pins
+DECODE_MUTANTS = {
+    "dec_output_at_slot": ('o[rows] = res["o64"][:, 0]', 'o[idx[rows] % B] = res["o64"][:, 0]'),
+    "dec_state_not_written_back": ('pool[idx[rows]] = res["state"]', "pass"),
+    "dec_state_written_to_row": ('pool[idx[rows]] = res["state"]', 'pool[rows % pool.shape[0]] = res["state"]'),
+    "dec_start_from_row_slot": ("s0 = np.ascontiguousarray(pool[idx[rows]], dtype=np.float32)",
+                                "s0 = np.ascontiguousarray(pool[rows % pool.shape[0]], dtype=np.float32)"),
+    "dec_padding_rows_kept": ("rows = np.nonzero(idx >= 0)[0]", "rows = np.arange(B)"),
+}
+
+
+def _decode_pins_failing(monkeypatch, old, new):
+    src = inspect.getsource(oracle_pkg.decode_step)
+    assert src.count(old) == 1, f"mutation site {old!r} not found"
+    namespace = dict(vars(oracle_pkg))
+    exec(compile(src.replace(old, new), "<decode mutant>", "exec"), namespace)
+    monkeypatch.setattr(oracle_pkg, "decode_step", namespace["decode_step"])
+    caught = []
+    for name, fn in inspect.getmembers(dec_pins, inspect.isfunction):
+        if name.startswith("test_"):
+            try:
+                fn()
+            except (AssertionError, IndexError, ValueError):
+                caught.append(name)
+    return caught
+
+
+def test_decode_mutant_harness_passes_the_unchanged_function(monkeypatch):
+    old = "rows = np.nonzero(idx >= 0)[0]"
+    assert _decode_pins_failing(monkeypatch, old, old) == []
+
+
+@pytest.mark.parametrize("mutant", sorted(DECODE_MUTANTS))
+def test_decode_pins_catch_mutant(mutant, monkeypatch):
+    old, new = DECODE_MUTANTS[mutant]
+    assert _decode_pins_failing(monkeypatch, old, new), f"no pin caught mutant {mutant}"
