@@ -183,11 +183,17 @@ def test_raw_input_backward_matches_differences_loosely(oracle):
         o, sN = oracle.recurrence_f64(nrm(qq), nrm(kk), *args)
         return float((o * do).sum() + (sN * dht).sum())
 
-    fd_q = np.zeros(K)
+    fd_q, fd_k = np.zeros(K), np.zeros(K)
     for c in range(K):
         p, m = qf.copy(), qf.copy()
         p[0, 2, 0, c] += 1e-6
         m[0, 2, 0, c] -= 1e-6
         fd_q[c] = (loss(p, kf) - loss(m, kf)) / 2e-6
+        p, m = kf.copy(), kf.copy()
+        p[0, 1, 0, c] += 1e-6
+        m[0, 1, 0, c] -= 1e-6
+        fd_k[c] = (loss(qf, p) - loss(qf, m)) / 2e-6
     rel = np.linalg.norm(dq[0, 2, 0] - fd_q) / np.linalg.norm(fd_q)
+    assert rel < 2e-2, rel
+    rel = np.linalg.norm(dk[0, 1, 0] - fd_k) / np.linalg.norm(fd_k)
     assert rel < 2e-2, rel

@@ -118,20 +118,26 @@ DECODE_MUTANTS = {
 }
 
 
-def _decode_pins_failing(monkeypatch, old, new):
-    src = inspect.getsource(oracle_pkg.decode_step)
+def _python_pins_failing(monkeypatch, func, old, new, pins):
+    """Swap a copy of oracle function ``func`` with one slip into the oracle module and run ``pins``
+    (name, callable) against it; returns the names of the pins that failed."""
+    src = inspect.getsource(getattr(oracle_pkg, func))
     assert src.count(old) == 1, f"mutation site {old!r} not found"
     namespace = dict(vars(oracle_pkg))
-    exec(compile(src.replace(old, new), "<decode mutant>", "exec"), namespace)
-    monkeypatch.setattr(oracle_pkg, "decode_step", namespace["decode_step"])
+    exec(compile(src.replace(old, new), "<oracle mutant>", "exec"), namespace)
+    monkeypatch.setattr(oracle_pkg, func, namespace[func])
     caught = []
-    for name, fn in inspect.getmembers(dec_pins, inspect.isfunction):
-        if name.startswith("test_"):
-            try:
-                fn()
-            except (AssertionError, IndexError, ValueError):
-                caught.append(name)
+    for name, fn in pins:
+        try:
+            fn()
+        except (AssertionError, IndexError, ValueError):
+            caught.append(name)
     return caught
+
+
+def _decode_pins_failing(monkeypatch, old, new):
+    pins = [(n, f) for n, f in inspect.getmembers(dec_pins, inspect.isfunction) if n.startswith("test_")]
+    return _python_pins_failing(monkeypatch, "decode_step", old, new, pins)
 
 
 def test_decode_mutant_harness_passes_the_unchanged_function(monkeypatch):
@@ -143,3 +149,33 @@ def test_decode_mutant_harness_passes_the_unchanged_function(monkeypatch):
 def test_decode_pins_catch_mutant(mutant, monkeypatch):
     old, new = DECODE_MUTANTS[mutant]
     assert _decode_pins_failing(monkeypatch, old, new), f"no pin caught mutant {mutant}"
+
+
+# slips in the backward's raw-input wrapper (group sums over the value heads of a Q/K head, the normalisation's
+# Jacobian); each is caught by the differences of the smooth forward or of the normalisation
+WRAPPER_MUTANTS = {
+    "wrap_no_group_sum": ("backward", "dqn = dqn.reshape(B, T, H, grp, K).sum(3)",
+                          "dqn = dqn.reshape(B, T, H, grp, K)[:, :, :, 0]"),
+    "wrap_dk_through_q": ("backward", "dk = l2norm_backward_f64(bits_to_f32(kb), dkn)",
+                          "dk = l2norm_backward_f64(bits_to_f32(qb), dkn)"),
+    "jac_no_projection": ("l2norm_backward_f64", "return dy / n - x * (x * dy).sum(-1, keepdims=True) / n ** 3",
+                          "return dy / n"),
+    "jac_wrong_power": ("l2norm_backward_f64", "/ n ** 3", "/ n ** 2"),
+}
+
+
+def _wrapper_pins():
+    return [(name, lambda fn=fn: fn(oracle_pkg)) for name, fn in inspect.getmembers(bwd_pins, inspect.isfunction)
+            if name in ("test_raw_input_backward_matches_differences_loosely", "test_l2norm_jacobian")]
+
+
+def test_wrapper_mutant_harness_passes_the_unchanged_functions(monkeypatch):
+    for func, old, _ in WRAPPER_MUTANTS.values():
+        assert _python_pins_failing(monkeypatch, func, old, old, _wrapper_pins()) == []
+        monkeypatch.undo()  # the next site is read from the real function's source
+
+
+@pytest.mark.parametrize("mutant", sorted(WRAPPER_MUTANTS))
+def test_wrapper_pins_catch_mutant(mutant, monkeypatch):
+    func, old, new = WRAPPER_MUTANTS[mutant]
+    assert _python_pins_failing(monkeypatch, func, old, new, _wrapper_pins()), f"no pin caught mutant {mutant}"
