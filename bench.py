@@ -525,8 +525,9 @@ def bench_backward(args, case, world, rank, dev):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = time_oracle_backward(case)
         cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
-    # the saved form skips the recomputation (intra-chunk and forward carry launches, and the chunk offsets)
-    launches = kda.backward_kernel_launches(B, T, H, HV, K, V, num_seqs) - (2 + (1 if num_seqs else 0) if saved is not None else 0)
+    launches = kda.backward_kernel_launches(B, T, H, HV, K, V, num_seqs)
+    if saved is not None:  # the recomputation is skipped: reverse carry, chunk gradients, norms
+        launches = 1 + (2 if case.tokens > 0 else 0)
     line = {"metric": BWD_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": config,

@@ -231,21 +231,25 @@ kda_status_t kda_prefill_forward_state_bf16(const void *q, const void *k, const 
  *   workspace    kda_prefill_backward_workspace_size(...) bytes, 256-byte
  *                aligned, device; holds the recomputed forward's per-chunk
  *                blocks, every chunk's start state and the gradient at every
- *                chunk's end state (fp32), and per-value-head gradients at the
- *                normalised rows.
+ *                chunk's end state (bf16), and per-value-head gradients at the
+ *                normalised rows (fp32).
  * Outputs overlap no input, no other output and the workspace.  Pointers are
  * 16-byte aligned (beta, dbeta, cu_seqlens: 4).  Rows outside every packed
  * sequence are left untouched.  Asynchronous on `stream`; kernel waits that
  * give up set the device error word (kda_prefill_device_error).
  *
  * The forward is recomputed (intra-chunk blocks, then the state carry storing
- * each chunk's start state); a reverse carry walks each sequence backwards
+ * each chunk's start state; a long sequence is cut into parts as the forward
+ * cuts it, each part's carry beside the next part's blocks); a reverse carry
+ * walks each sequence backwards
  * for the gradient at every chunk's end state; a per-chunk kernel forms the
  * chunk's gradients; a last kernel sums each Q/K group and applies the
  * normalisation's Jacobian.  Accuracy assumes g <= 0 with every 8 consecutive
  * gates of a channel summing to >= -40 (per-token g >= -5 suffices).
  */
 size_t kda_prefill_backward_workspace_size(int B, int T, int H, int HV, int K, int V, int num_seqs);
+/* Kernel launches of one kda_prefill_backward call (the recomputing form); 0 for invalid sizes, or when the
+ * sizes are long enough to be cut into parts and the current device cannot be queried. */
 int kda_prefill_backward_kernel_launches(int B, int T, int H, int HV, int K, int V, int num_seqs);
 kda_status_t kda_prefill_backward(const void *q, const void *k, const void *v, const float *g, const float *beta,
                                   const float *initial_state, const int32_t *cu_seqlens, int num_seqs, int B,

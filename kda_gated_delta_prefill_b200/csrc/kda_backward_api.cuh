@@ -62,8 +62,16 @@ extern "C" int kda_prefill_backward_kernel_launches(int B, int T, int H, int HV,
     const bool varlen = num_seqs > 0;
     if (check_dims(B, T, H, HV, K, V, varlen, num_seqs, d) != KDA_OK) return 0;
     const int with_tokens = static_cast<int64_t>(B) * T > 0 ? 1 : 0;
-    // chunk offsets (packed), intra-chunk, carry with the start states, reverse carry, chunk gradients, norms
-    return (varlen ? 1 : 0) + with_tokens + 1 + 1 + 2 * with_tokens;
+    // the forward's cut into parts (it depends on the SM count only for sequences long enough to be cut)
+    int parts = 1;
+    if (!varlen && with_tokens && (T + CH - 1) / CH / kMinChunksPerPart >= 2) {
+        DeviceInfo info;
+        if (device_info(info) != cudaSuccess) return 0;
+        parts = pipeline_parts(B, T, HV, false, info.sms);
+    }
+    // chunk offsets (packed), intra-chunk and carry with the start states per part, reverse carry, chunk
+    // gradients, norms
+    return (varlen ? 1 : 0) + (with_tokens + 1) * parts + 1 + 2 * with_tokens;
 }
 
 extern "C" kda_status_t kda_prefill_backward(const void *q, const void *k, const void *v, const float *g,
@@ -170,14 +178,14 @@ kda_status_t backward_impl(const void *q, const void *k, const void *v, const fl
     }
     // 1. the forward's per-chunk blocks, then its carry storing every chunk's start state (no o); a saved
     //    forward left both (and the chunk offsets) in the workspace
+    CUtensorMap tq, tk, tv, tg;
+    kda::IntraParams ip{};
     if (tokens > 0 && recompute) {
-        CUtensorMap tq, tk, tv, tg;
         if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HV, tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HV, tokens, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
             return KDA_ERR_CUDA;
-        kda::IntraParams ip{};
         ip.beta = beta;
         ip.cu = cu_seqlens;
         ip.chunk_off = chunk_off;
@@ -190,15 +198,17 @@ kda_status_t backward_impl(const void *q, const void *k, const void *v, const fl
         ip.N = d.N;
         ip.chunks_per_seq = (T + CH - 1) / CH;
         ip.prefetch_stride = info.sms * kda::kIntraCtasPerSm;
-        ip.chunk_begin = 0;
-        ip.chunk_count = ip.chunks_per_seq;
         if (cudaFuncSetAttribute(kda::kda_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kda::IntraSmem::TOTAL) != cudaSuccess)
             return KDA_ERR_CUDA;
-        kda::kda_intra_kernel<<<static_cast<int>(ws.max_chunks * HV), 256, kda::IntraSmem::TOTAL, s>>>(tq, tk, tv,
-                                                                                                      tg, ip);
-        if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
     }
+    auto launch_intra = [&](int chunk_begin, int chunk_count, int64_t grid_chunks) {
+        ip.chunk_begin = chunk_begin;
+        ip.chunk_count = chunk_count;
+        kda::kda_intra_kernel<<<static_cast<int>(grid_chunks * HV), 256, kda::IntraSmem::TOTAL, s>>>(tq, tk, tv, tg,
+                                                                                                      ip);
+        return cudaGetLastError();
+    };
     kda::CarryParams cp{};
     cp.items = items;
     cp.s0 = initial_state;
@@ -214,17 +224,34 @@ kda_status_t backward_impl(const void *q, const void *k, const void *v, const fl
     cp.chunk_count = cp.chunks_per_seq;
     cp.states = states;
     cp.no_o = 1;
-    // The forward carry (start states) and the reverse carry (end-state gradients) both read only the blocks,
-    // so they run side by side: the forward one on the high-priority side stream, joined before the chunk kernel.
+    // The forward carry runs on the high-priority side stream, joined before the chunk kernel.  A sequence long
+    // enough for the forward's cut into parts is cut the same way here: the carry of part j beside the
+    // intra-chunk work of part j + 1 (each part's carry starting from the previous part's fp32 end state, so
+    // the stored start states are the ones one launch gives).  The reverse carry reads only the blocks, so it
+    // follows the last intra-chunk part on the main stream, beside the last forward-carry parts.
     CarryLane *lane = nullptr;
     std::unique_lock<std::mutex> lane_lock;
     if (recompute) {
         if (carry_lane(info.dev, lane) != cudaSuccess) return KDA_ERR_CUDA;
         lane_lock = std::unique_lock<std::mutex>(lane->mu);
-        if (cudaEventRecord(lane->fork, s) != cudaSuccess ||
-            cudaStreamWaitEvent(lane->stream, lane->fork, 0) != cudaSuccess)
-            return KDA_ERR_CUDA;
-        if (launch_carry(cp, d.N * HV, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
+        const int parts = tokens > 0 ? pipeline_parts(B, T, HV, varlen, info.sms) : 1;
+        const int nck = cp.chunks_per_seq;
+        const int64_t den = 4 * parts - 3;  // the last part a quarter of the others, as in the forward
+        for (int j = 0; j < parts; ++j) {
+            const int c0 = parts == 1 ? 0 : static_cast<int>(static_cast<int64_t>(nck) * 4 * j / den);
+            const int c1 = j + 1 == parts ? nck : static_cast<int>(static_cast<int64_t>(nck) * 4 * (j + 1) / den);
+            if (tokens > 0) {
+                const int64_t grid = parts == 1 ? ws.max_chunks : static_cast<int64_t>(B) * (c1 - c0);
+                if (launch_intra(c0, c1 - c0, grid) != cudaSuccess) return KDA_ERR_CUDA;
+            }
+            if (cudaEventRecord(lane->fork, s) != cudaSuccess ||
+                cudaStreamWaitEvent(lane->stream, lane->fork, 0) != cudaSuccess)
+                return KDA_ERR_CUDA;
+            cp.s0 = j == 0 ? initial_state : cp.sN;
+            cp.chunk_begin = c0;
+            cp.chunk_count = c1 - c0;
+            if (launch_carry(cp, d.N * HV, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
+        }
         if (cudaEventRecord(lane->join, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
     }
 
