@@ -94,11 +94,64 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream_ptr(stream):
+def _stream_ptr(stream, device=None):
     import torch
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _on(device):
+    """The calls launch on the CUDA runtime's current device: make it the tensors' device for the call."""
+    import torch
+    return torch.cuda.device(device)
+
+
+def _need_all(checks, device=None, *, host=False):
+    """The library reads and writes raw pointers, so a tensor of another dtype or size would let its kernels run
+    past the buffer.  ``checks``: (name, tensor or None, dtype, element count or None, contiguous); first every
+    dtype and size, then placement (``device``, or host memory) and layout."""
+    checks = [c for c in checks if c[1] is not None]
+    for name, t, dtype, numel, _ in checks:
+        if t.dtype != dtype:
+            raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+        if numel is not None and t.numel() != numel:
+            raise ValueError(f"{name} must hold {numel} elements, got {t.numel()}")
+    for name, t, _, _, contiguous in checks:
+        if host:
+            if t.is_cuda:
+                raise ValueError(f"{name} must be a host tensor")
+        else:
+            if not t.is_cuda:
+                raise ValueError(f"{name} must be a CUDA tensor")
+            if device is not None and t.device != device:
+                raise ValueError(f"{name} is on {t.device}, the other tensors on {device}")
+        if contiguous and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def _need(name, t, dtype, numel, device=None, *, host=False, contiguous=True):
+    _need_all([(name, t, dtype, numel, contiguous)], device, host=host)
+
+
+def _need_inputs(q, k, v, g, beta, initial_state, cu_seqlens, state_dtype=None, host=False, more=None):
+    """Checks of the forward's inputs, and of ``more(B, T, H, HV, K, V, N)``: further checks in ``_need_all``'s
+    form.  Returns (B, T, H, HV, K, V, N, device)."""
+    import torch
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q must be [B,T,H,K] and v [B,T,HV,V]")
+    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
+    dev = None if host else q.device
+    bt = B * T
+    checks = [("q", q, torch.bfloat16, bt * H * K, True), ("k", k, torch.bfloat16, bt * H * K, True),
+              ("v", v, torch.bfloat16, bt * HV * V, True), ("g", g, torch.float32, bt * HV * K, True),
+              ("beta", beta, torch.float32, bt * HV, True),
+              ("initial_state", initial_state, state_dtype or torch.float32, N * HV * K * V, True),
+              ("cu_seqlens", cu_seqlens, torch.int32, None, True)]
+    if more is not None:
+        checks += more(B, T, H, HV, K, V, N)
+    _need_all(checks, dev, host=host)
+    return B, T, H, HV, K, V, N, dev
 
 
 def _check(rc: int, where: str):
@@ -126,22 +179,24 @@ def forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o=None, fi
             workspace=None, stream=None):
     """Run the forward on CUDA tensors; returns (o, final_state)."""
     import torch
-    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
-    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta)):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    B, T, H, HV, K, V, N, dev = _need_inputs(q, k, v, g, beta, initial_state, cu_seqlens)
     if o is None:
-        o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=q.device)
+        o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=dev)
     if final_state is None:
-        final_state = torch.empty(N, HV, K, V, dtype=torch.float32, device=q.device)
+        final_state = torch.empty(N, HV, K, V, dtype=torch.float32, device=dev)
+    _need("o", o, torch.bfloat16, B * T * HV * V, dev)
+    _need("final_state", final_state, torch.float32, N * HV * K * V, dev)
     num_seqs = N if cu_seqlens is not None else 0
     ws_bytes = workspace_size(B, T, H, HV, K, V, num_seqs)
     if ws_bytes and workspace is None:
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    rc = lib().kda_prefill_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
-                                   _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(o), _ptr(final_state),
-                                   _ptr(workspace), workspace.numel() if workspace is not None else 0,
-                                   _stream_ptr(stream))
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    if workspace is not None:
+        _need("workspace", workspace, torch.uint8, None, dev)
+    with _on(dev):
+        rc = lib().kda_prefill_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                                       _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(o), _ptr(final_state),
+                                       _ptr(workspace), workspace.numel() if workspace is not None else 0,
+                                       _stream_ptr(stream, dev))
     _check(rc, "kda_prefill_forward")
     return o, final_state
 
@@ -150,21 +205,24 @@ def forward_state_bf16(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,
                        workspace=None, stream=None):
     """The forward with a bf16 state: initial_state bf16 [N,HV,K,V] or None; returns (o, final_state bf16)."""
     import torch
-    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
-    if initial_state is not None and initial_state.dtype != torch.bfloat16:
-        raise ValueError("initial_state must be bf16")
+    B, T, H, HV, K, V, N, dev = _need_inputs(q, k, v, g, beta, initial_state, cu_seqlens,
+                                             state_dtype=torch.bfloat16)
     if o is None:
-        o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=q.device)
+        o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=dev)
     if final_state is None:
-        final_state = torch.empty(N, HV, K, V, dtype=torch.bfloat16, device=q.device)
+        final_state = torch.empty(N, HV, K, V, dtype=torch.bfloat16, device=dev)
+    _need("o", o, torch.bfloat16, B * T * HV * V, dev)
+    _need("final_state", final_state, torch.bfloat16, N * HV * K * V, dev)
     num_seqs = N if cu_seqlens is not None else 0
     ws_bytes = int(lib().kda_prefill_state_bf16_workspace_size(B, T, H, HV, K, V, num_seqs))
     if workspace is None:
-        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
-    rc = lib().kda_prefill_forward_state_bf16(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
-                                              _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(o),
-                                              _ptr(final_state), _ptr(workspace), workspace.numel(),
-                                              _stream_ptr(stream))
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    _need("workspace", workspace, torch.uint8, None, dev)
+    with _on(dev):
+        rc = lib().kda_prefill_forward_state_bf16(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                                  _ptr(initial_state), _ptr(cu_seqlens), num_seqs, B, T, H, HV, K,
+                                                  V, _ptr(o), _ptr(final_state), _ptr(workspace), workspace.numel(),
+                                                  _stream_ptr(stream, dev))
     _check(rc, "kda_prefill_forward_state_bf16")
     return o, final_state
 
@@ -183,18 +241,22 @@ def forward_save(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o=Non
     """The forward that also keeps what the backward needs; returns (o, final_state, saved).  Pass ``saved`` to
     ``backward(..., saved=saved)`` with the same inputs."""
     import torch
-    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
+    B, T, H, HV, K, V, N, dev = _need_inputs(q, k, v, g, beta, initial_state, cu_seqlens)
     if o is None:
-        o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=q.device)
+        o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=dev)
     if final_state is None:
-        final_state = torch.empty(N, HV, K, V, dtype=torch.float32, device=q.device)
+        final_state = torch.empty(N, HV, K, V, dtype=torch.float32, device=dev)
+    _need("o", o, torch.bfloat16, B * T * HV * V, dev)
+    _need("final_state", final_state, torch.float32, N * HV * K * V, dev)
     num_seqs = N if cu_seqlens is not None else 0
     if saved is None:
         saved = torch.empty(max(backward_workspace_size(B, T, H, HV, K, V, num_seqs), 1), dtype=torch.uint8,
-                            device=q.device)
-    rc = lib().kda_prefill_forward_save(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
-                                        _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(o), _ptr(final_state),
-                                        _ptr(saved), saved.numel(), _stream_ptr(stream))
+                            device=dev)
+    _need("saved", saved, torch.uint8, None, dev)
+    with _on(dev):
+        rc = lib().kda_prefill_forward_save(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                                            _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(o),
+                                            _ptr(final_state), _ptr(saved), saved.numel(), _stream_ptr(stream, dev))
     _check(rc, "kda_prefill_forward_save")
     return o, final_state, saved
 
@@ -208,11 +270,10 @@ def backward(q, k, v, g, beta, dout, initial_state=None, dht=None, cu_seqlens=No
     ``forward_save`` on the same inputs) the forward is not recomputed.
     """
     import torch
-    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
-    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("dout", dout)):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous CUDA tensor")
-    dev = q.device
+    B, T, H, HV, K, V, N, dev = _need_inputs(
+        q, k, v, g, beta, initial_state, cu_seqlens,
+        more=lambda B, T, H, HV, K, V, N: [("dout", dout, torch.bfloat16, B * T * HV * V, True),
+                                           ("dht", dht, torch.float32, N * HV * K * V, True)])
     dq = torch.empty(B, T, H, K, dtype=torch.bfloat16, device=dev)
     dk = torch.empty(B, T, H, K, dtype=torch.bfloat16, device=dev)
     dv = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=dev)
@@ -228,9 +289,11 @@ def backward(q, k, v, g, beta, dout, initial_state=None, dht=None, cu_seqlens=No
     elif workspace is None:
         ws_bytes = backward_workspace_size(B, T, H, HV, K, V, num_seqs)
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), num_seqs, B, T,
-            H, HV, K, V, _ptr(dout), _ptr(dht), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dh0),
-            _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _need("saved" if saved is not None else "workspace", workspace, torch.uint8, None, dev)
+    with _on(dev):
+        rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), num_seqs,
+                B, T, H, HV, K, V, _ptr(dout), _ptr(dht), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta),
+                _ptr(dh0), _ptr(workspace), workspace.numel(), _stream_ptr(stream, dev))
     _check(rc, name)
     return dq, dk, dv, dg, dbeta, dh0
 
@@ -246,11 +309,19 @@ def forward_host(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o, fi
     Enqueues the host->device copies, the forward and the device->host copies
     of o and final_state on ``stream``; the caller synchronises.
     """
-    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
+    import torch
+    B, T, H, HV, K, V, N, _ = _need_inputs(
+        q, k, v, g, beta, initial_state, cu_seqlens, host=True,
+        more=lambda B, T, H, HV, K, V, N: [("o", o, torch.bfloat16, B * T * HV * V, True),
+                                           ("final_state", final_state, torch.float32, N * HV * K * V, True)])
+    _need("staging", staging, torch.uint8, None)
+    dev = staging.device
     num_seqs = N if cu_seqlens is not None else 0
-    rc = lib().kda_prefill_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
-                                        _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(o), _ptr(final_state),
-                                        _ptr(staging), staging.numel(), _stream_ptr(stream))
+    with _on(dev):
+        rc = lib().kda_prefill_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
+                                            _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(o),
+                                            _ptr(final_state), _ptr(staging), staging.numel(),
+                                            _stream_ptr(stream, dev))
     _check(rc, "kda_prefill_forward_host")
     return o, final_state
 
@@ -270,31 +341,44 @@ def decode_step(q, k, v, g, beta, state, state_indices, *, o=None, stream=None):
     [num_slots, HV, K, V] (compact inside a slot), updated in place; state_indices: int32 [B], -1 = padding row.
     """
     import torch
+    if q.dim() != 3 or k.shape != q.shape or v.dim() != 3 or v.shape[0] != q.shape[0]:
+        raise ValueError("q and k must be [B,H,K] and v [B,HV,V]")
+    if state.dim() != 4 or state.shape[1] != v.shape[1]:
+        raise ValueError("state must be a pool [num_slots, HV, K, V]")
     B, H, K = q.shape
     HV, V = v.shape[1], v.shape[2]
-    for name, t, inner in (("q", q, H * K), ("k", k, H * K), ("v", v, HV * V)):
-        if not t.is_cuda or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
-            raise ValueError(f"{name} must be a CUDA tensor with compact rows")
-    for name, t in (("g", g), ("beta", beta), ("state_indices", state_indices)):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous CUDA tensor")
-    if not state.is_cuda or state[0].stride() != (K * V, V, 1):
-        raise ValueError("state must be a CUDA pool [num_slots, HV, K, V] compact inside each slot")
+    dev = q.device
+    _need_all([("q", q, torch.bfloat16, None, False), ("k", k, torch.bfloat16, None, False),
+               ("v", v, torch.bfloat16, None, False), ("g", g, torch.float32, B * HV * K, True),
+               ("beta", beta, torch.float32, B * HV, True), ("state", state, torch.bfloat16, None, False),
+               ("state_indices", state_indices, torch.int32, B, True)], dev)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError(f"{name} must have compact rows")
+    if tuple(state.shape[1:]) != (HV, K, V) or state[0].stride() != (K * V, V, 1):
+        raise ValueError("state must be a pool [num_slots, HV, K, V] compact inside each slot")
     if o is None:
-        o = torch.empty(B, HV, V, dtype=torch.bfloat16, device=q.device)
-    _check(lib().kda_decode_step(_ptr(q), q.stride(0), _ptr(k), k.stride(0), _ptr(v), v.stride(0), _ptr(g),
-                                 _ptr(beta), _ptr(state), state.stride(0), state.shape[0], _ptr(state_indices),
-                                 B, H, HV, K, V, _ptr(o), _stream_ptr(stream)), "kda_decode_step")
+        o = torch.empty(B, HV, V, dtype=torch.bfloat16, device=dev)
+    _need("o", o, torch.bfloat16, B * HV * V, dev)
+    with _on(dev):
+        rc = lib().kda_decode_step(_ptr(q), q.stride(0), _ptr(k), k.stride(0), _ptr(v), v.stride(0), _ptr(g),
+                                   _ptr(beta), _ptr(state), state.stride(0), state.shape[0], _ptr(state_indices),
+                                   B, H, HV, K, V, _ptr(o), _stream_ptr(stream, dev))
+    _check(rc, "kda_decode_step")
     return o
 
 
 def l2norm_bf16(x, out=None, stream=None):
     """Exact-rounding L2 normalisation of rows of 128 bf16 values (CUDA)."""
     import torch
+    _need("x", x, torch.bfloat16, None, x.device)
     if out is None:
         out = torch.empty_like(x)
+    _need("out", out, torch.bfloat16, x.numel(), x.device)
     rows = x.numel() // x.shape[-1]
-    _check(lib().kda_l2norm_bf16(_ptr(x), rows, x.shape[-1], _ptr(out), _stream_ptr(stream)), "kda_l2norm_bf16")
+    with _on(x.device):
+        rc = lib().kda_l2norm_bf16(_ptr(x), rows, x.shape[-1], _ptr(out), _stream_ptr(stream, x.device))
+    _check(rc, "kda_l2norm_bf16")
     return out
 
 
@@ -312,13 +396,16 @@ def forward_noalloc(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o=
     P, I = ctypes.c_void_p, ctypes.c_int
     f.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P]
     f.restype = I
-    B, T, H, HV, K, V, N = _dims(q, v, cu_seqlens)
+    B, T, H, HV, K, V, N, dev = _need_inputs(q, k, v, g, beta, initial_state, cu_seqlens)
     if o is None:
-        o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=q.device)
+        o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=dev)
     if final_state is None:
-        final_state = torch.empty(N, HV, K, V, dtype=torch.float32, device=q.device)
+        final_state = torch.empty(N, HV, K, V, dtype=torch.float32, device=dev)
+    _need("o", o, torch.bfloat16, B * T * HV * V, dev)
+    _need("final_state", final_state, torch.float32, N * HV * K * V, dev)
     num_seqs = N if cu_seqlens is not None else 0
-    rc = f(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), num_seqs,
-           B, T, H, HV, K, V, _ptr(o), _ptr(final_state), _stream_ptr(stream))
+    with _on(dev):
+        rc = f(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), num_seqs,
+               B, T, H, HV, K, V, _ptr(o), _ptr(final_state), _stream_ptr(stream, dev))
     _check(rc, "kda_prefill_forward_noalloc")
     return o, final_state

@@ -216,3 +216,76 @@ def test_bf16_state_forward_rejects_bad_arguments(L):
     assert f(ptr(6), ptr(9), ptr(12), need - 256) == 4
     assert f(ptr(6), ptr(9), ptr(9), need) == 1                     # workspace overlaps final_state
     assert f(ptr(6), P(FAKE + 6 * step + 16384), ptr(12), need) == 1  # states partly overlap
+
+
+def _small_inputs(dtype_overrides=None):
+    import torch
+    x = {"q": torch.zeros(1, 64, 2, 128, dtype=torch.bfloat16), "k": torch.zeros(1, 64, 2, 128, dtype=torch.bfloat16),
+         "v": torch.zeros(1, 64, 4, 128, dtype=torch.bfloat16), "g": torch.zeros(1, 64, 4, 128),
+         "beta": torch.zeros(1, 64, 4)}
+    for name, t in (dtype_overrides or {}).items():
+        x[name] = t
+    return x
+
+
+@pytest.mark.parametrize("name,bad,msg", [
+    ("g", lambda t: t.g.bfloat16(), "g must be torch.float32"),
+    ("beta", lambda t: t.beta.double(), "beta must be torch.float32"),
+    ("q", lambda t: t.q.float(), "q must be torch.bfloat16"),
+    ("k", lambda t: t.k[:, :32], "k must hold"),
+    ("v", lambda t: t.v[:, :32], "v must hold"),
+])
+def test_binding_rejects_wrong_dtype_or_size_before_any_launch(name, bad, msg):
+    """The binding checks dtypes and element counts: the library only sees raw pointers, and a wrong-size
+    buffer would let the kernels read or write past it."""
+    import types
+    import kda_gated_delta_prefill_b200 as kda
+    x = _small_inputs()
+    x[name] = bad(types.SimpleNamespace(**x))
+    with pytest.raises(ValueError, match=msg):
+        kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"])
+    with pytest.raises(ValueError, match=msg):
+        kda.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], torch_zeros_dout())
+
+
+def torch_zeros_dout():
+    import torch
+    return torch.zeros(1, 64, 4, 128, dtype=torch.bfloat16)
+
+
+def test_binding_rejects_host_tensors_and_wrong_optional_buffers():
+    import torch
+    import kda_gated_delta_prefill_b200 as kda
+    x = _small_inputs()
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"])
+    with pytest.raises(ValueError, match="initial_state must hold"):
+        kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], torch.zeros(1, 4, 128, 64))
+    with pytest.raises(ValueError, match="initial_state must be torch.bfloat16"):
+        kda.forward_state_bf16(x["q"], x["k"], x["v"], x["g"], x["beta"], torch.zeros(1, 4, 128, 128))
+    with pytest.raises(ValueError, match="cu_seqlens must be torch.int32"):
+        kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], None, torch.tensor([0, 64]))
+    with pytest.raises(ValueError, match="dout must be torch.bfloat16"):
+        kda.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], torch.zeros(1, 64, 4, 128))
+    with pytest.raises(ValueError, match="dht must hold"):
+        kda.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], torch_zeros_dout(), None, torch.zeros(1, 4, 128))
+    # the host-buffer entry point wants host inputs and outputs of the right types, and a device staging buffer
+    o_h = torch.empty(1, 64, 4, 128, dtype=torch.bfloat16)
+    s_h = torch.empty(1, 4, 128, 128)
+    with pytest.raises(ValueError, match="final_state must be torch.float32"):
+        kda.forward_host(x["q"], x["k"], x["v"], x["g"], x["beta"], o=o_h, final_state=s_h.bfloat16(),
+                         staging=torch.empty(16, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="staging must be a CUDA tensor"):
+        kda.forward_host(x["q"], x["k"], x["v"], x["g"], x["beta"], o=o_h, final_state=s_h,
+                         staging=torch.empty(16, dtype=torch.uint8))
+    # the decode step: a bf16 pool, int32 slot indices
+    q1 = torch.zeros(3, 2, 128, dtype=torch.bfloat16)
+    v1 = torch.zeros(3, 4, 128, dtype=torch.bfloat16)
+    g1, b1 = torch.zeros(3, 4, 128), torch.zeros(3, 4)
+    with pytest.raises(ValueError, match="state must be torch.bfloat16"):
+        kda.decode_step(q1, q1, v1, g1, b1, torch.zeros(5, 4, 128, 128), torch.zeros(3, dtype=torch.int32))
+    with pytest.raises(ValueError, match="state_indices must be torch.int32"):
+        kda.decode_step(q1, q1, v1, g1, b1, torch.zeros(5, 4, 128, 128, dtype=torch.bfloat16),
+                        torch.zeros(3, dtype=torch.int64))
+    with pytest.raises(ValueError, match="x must be torch.bfloat16"):
+        kda.l2norm_bf16(torch.zeros(4, 128))
