@@ -54,6 +54,69 @@ def chunk_flops(case) -> int:
     return case.tokens * case.HV * 180224
 
 
+def chunk_flops_triangular(C: int = 64, K: int = 128, V: int = 128) -> float:
+    """FLOPs per token-head of the chunk form counting only the triangles the method needs (C=64, K=V=128):
+    L (j < i) and Aqk (j <= i) over K; the unit-triangular inverse (sum over j < i of (i - j) multiply-adds) and
+    its beta scaling; W and U with lower-triangular A; the carry's three dense products (W S, Qg S, Kg^T Vnew)
+    and the triangular Aqk Vnew."""
+    lower_strict, lower = C * (C - 1) // 2, C * (C + 1) // 2
+    inverse = sum(i - j for i in range(C) for j in range(i)) * 2 + lower
+    per_chunk = (lower_strict * K * 2 + lower * K * 2 + inverse + lower * K * 2 + lower * V * 2
+                 + 3 * C * K * V * 2 + lower * V * 2)
+    return per_chunk / C
+
+
+def kernel_split(step, steps: int = 3):
+    """Device time of each of this library's kernels per step, from a CUPTI trace (torch.profiler) of `steps`
+    extra steps run after the timed region: {kernel name: ms per step}.  Kernels that overlap on two streams are
+    each counted in full, so the sum can exceed the step time.  An "unavailable" note if the trace fails."""
+    try:
+        import torch
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            for _ in range(steps):
+                step()
+            torch.cuda.synchronize()
+        out = {}
+        for ev in prof.key_averages():
+            key = ev.key
+            if "kda::" not in key:
+                continue
+            name = key[key.index("kda::"):]
+            for stop in ("(", "<"):
+                if stop in name:
+                    name = name[:name.index(stop)] + ("<...>" if stop == "<" else "")
+            us = getattr(ev, "device_time_total", None)
+            if us is None:
+                us = getattr(ev, "cuda_time_total", 0.0)
+            out[name] = out.get(name, 0.0) + us / 1e3 / steps
+        return {k: round(v, 4) for k, v in sorted(out.items(), key=lambda kv: -kv[1])} or {"unavailable": "no kernels"}
+    except Exception as e:  # the bench line stays valid without the split
+        return {"unavailable": str(e)[:120]}
+
+
+def sustained(step, stream, seconds: float, device_index: int):
+    """Back-to-back steps for about `seconds` (the power cap engages on long runs), timed by CUDA events on the
+    launching stream, with the clocks sampled meanwhile."""
+    import torch
+    if seconds <= 0:
+        return None
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    n = max(20, int(seconds * 1e3 / max(a.elapsed_time(b), 1e-3)))
+    with ClockSampler(device_index) as clk:
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(n):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+    return {"steps": n, "ms_per_step": a.elapsed_time(b) / n, "clocks": clk.summary()}
+
+
 # device and host sources of the other paths (backward, decode step): edits there leave the forward unchanged
 OTHER_PATH_SOURCES = {"kda_backward.cuh", "kda_backward_api.cuh", "kda_decode.cuh"}
 
@@ -556,6 +619,9 @@ def main():
                          "the backward from a saved forward (forward_save once, untimed)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sustain-s", type=float, default=3.0,
+                    help="prefill workloads: seconds of back-to-back steps after the timed region for the sustained "
+                         "(power-capped) figure; 0 skips it")
     ap.add_argument("--profile-T", type=int, default=0,
                     help="only run 3 forwards of B=1, H=HV=64, T=<value>, with state, and exit: the small case "
                          "the ncu captures under profiles/ use")
@@ -684,11 +750,18 @@ def main():
     alg = algorithmic_bytes(case)
     avg_launch_s = statistics.mean(launch_ms) / 1e3
     achieved = alg / avg_launch_s / 1e9
+    tri = chunk_flops_triangular()
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
                 "traffic": recorded_traffic(case.name), "peak_kind": peak_kind,
                 "algorithmic_bytes_per_launch": alg, "avg_launch_ms": avg_launch_s * 1e3,
                 "frac_nominal_8TBps": achieved / 8000.0,
-                "tensor_tflops": chunk_flops(case) / avg_launch_s / 1e12}
+                "flops_per_token_head": {"dense": 180224, "triangular": round(tri, 1)},
+                "tensor_tflops": chunk_flops(case) / avg_launch_s / 1e12,
+                "tensor_tflops_triangular": case.tokens * HV * tri / avg_launch_s / 1e12}
+    step_ms = {"mean": statistics.mean(launch_ms), "median": statistics.median(launch_ms), "min": min(launch_ms),
+               "max": max(launch_ms)}
+    split = kernel_split(step)
+    sus = sustained(step, stream, args.sustain_s, torch.cuda.current_device())
 
     # ---- end to end through the host-buffer entry point ----
     e2e = None
@@ -739,7 +812,8 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk.summary(),
             "gpu_launches": launches_per_step * args.steps, "impl": "native",
-            "kernel_source": kernel_source_hash()}
+            "kernel_source": kernel_source_hash(), "step_ms": step_ms, "kernel_ms_per_step": split,
+            "sustained": sus}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -164,7 +164,10 @@ kda_status_t kda_prefill_forward_host(const void *q_host, const void *k_host, co
  * chunk and a value head, e.g. T = 14,400 at HV = 4) are rejected with
  * KDA_ERR_WORKSPACE before any launch.  The first call on a device looks up
  * the array's device address (cudaGetSymbolAddress); make that first call
- * before any stream capture.  Every call shares the one array, so calls
+ * before any stream capture.  The address is kept for the life of the
+ * process: after cudaDeviceReset (or anything else that destroys the
+ * device's primary context) it is stale, so do not call this entry point on
+ * that device again in the same process.  Every call shares the one array, so calls
  * whose work overlaps on the GPU (other streams, other threads) race; issue
  * them one after another.  Calls no cudaMalloc / cudaFree.
  */

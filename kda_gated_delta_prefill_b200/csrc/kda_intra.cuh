@@ -231,34 +231,9 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
         uint4 raw[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) raw[c] = *reinterpret_cast<const uint4 *>(tile + ((c ^ rs) << 4));
-        float2 acc = make_float2(0.f, 0.f);
+        l2norm_half_row(raw);  // the routine the standalone kda_l2norm_bf16 kernel runs
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 x = unpack_bf16(w[j]);
-                acc = add2(acc, mul2(x, x));
-            }
-        }
-        float ss = __fadd_rn(acc.x, acc.y);
-        ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, 1));
-        const float den = __fsqrt_rn(__fadd_rn(ss, 1e-6f));
-        const float rr = __frcp_rn(den);
-        const float2 r2 = make_float2(rr, rr), nd2 = make_float2(-den, -den);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 x = unpack_bf16(w[j]);
-                const float2 q0 = mul2(x, r2);
-                const float2 e = fma2(q0, nd2, x);
-                const float2 y = fma2(e, r2, q0);
-                w[j] = pack_bf16(y.x, y.y);
-            }
-            *reinterpret_cast<uint4 *>(tile + ((c ^ rs) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
+        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(tile + ((c ^ rs) << 4)) = raw[c];
     }
     __syncthreads();
 

@@ -46,7 +46,9 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb)
     return pa < pb + nb && pb < pa + na;
 }
 
-// Per-device facts looked up once: SM count and the error word's device address.
+// Per-device facts: the SM count (looked up once; it belongs to the device, not to a context) and the error
+// word's device address, looked up on every call so that a recreated context (after cudaDeviceReset) never
+// receives a stale address.
 struct DeviceInfo {
     bool ready = false;
     int dev = 0;
@@ -62,18 +64,18 @@ cudaError_t device_info(DeviceInfo &out)
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_info_mu);
-    DeviceInfo &d = g_info[dev];
-    if (!d.ready) {
-        d.dev = dev;
-        e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return e;
-        e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.err), g_kda_device_error);
-        if (e != cudaSuccess) return e;
-        d.ready = true;
+    {
+        std::lock_guard<std::mutex> lock(g_info_mu);
+        DeviceInfo &d = g_info[dev];
+        if (!d.ready) {
+            d.dev = dev;
+            e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return e;
+            d.ready = true;
+        }
+        out = d;
     }
-    out = d;
-    return cudaSuccess;
+    return cudaGetSymbolAddress(reinterpret_cast<void **>(&out.err), g_kda_device_error);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
@@ -608,7 +610,7 @@ extern "C" kda_status_t kda_l2norm_bf16(const void *x, int64_t rows, int K, void
     if (x != out && overlaps(x, n, out, n)) return KDA_ERR_INVALID_ARG;
     DeviceInfo info;
     if (device_info(info) != cudaSuccess) return KDA_ERR_CUDA;
-    const int64_t blocks_needed = (rows + 7) / 8;
+    const int64_t blocks_needed = (rows + 127) / 128;  // 8 warps of 16 rows
     const int64_t cap = static_cast<int64_t>(info.sms) * 8;
     const int blocks = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
     kda::l2norm_bf16_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
@@ -626,7 +628,9 @@ extern "C" kda_status_t kda_l2norm_bf16(const void *x, int64_t rows, int K, void
 // file-scope device array that every GPU loading this library reserves until
 // the process exits.  Host code must not use the array's name as an address:
 // on the host it is only a stand-in symbol, so its device address is looked
-// up once per device with cudaGetSymbolAddress and cached.
+// up once per device with cudaGetSymbolAddress and cached for the life of the
+// process (so a context destroyed by cudaDeviceReset leaves a stale address:
+// the header tells callers not to use this entry point after a reset).
 // ---------------------------------------------------------------------------
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
 static __device__ __align__(256) uint8_t g_kda_noalloc_scratch[kNoAllocScratchBytes];

@@ -2,10 +2,15 @@
 
 It exists for callers that may not allocate device memory during a call, so
 its workspace is the library's fixed device array.  This file is collected
-last so that a failure here cannot hide the result of any other test.  Two
-calls in a row, on different inputs, must each match kda_prefill_forward on
-the same inputs within the parity tolerances: the second call must not see
-anything the first one left in the shared array.
+last so that a failure here cannot hide the result of any other test.
+
+Both entry points run the same kernels over the same workspace layout, so
+each no-allocation call must equal kda_prefill_forward on the same inputs bit
+for bit.  The array keeps whatever the previous call left in it: the calls
+below first fill it with a larger packed batch (more sequences, longer ones),
+then run a smaller packed batch and a plain batch, so a kernel that read
+stale chunk offsets, sequence order or chunk blocks from an earlier call
+would break the equality.  One case is also compared with the oracle.
 """
 import ctypes
 
@@ -14,7 +19,7 @@ import pytest
 import torch
 
 from kda_gated_delta_prefill_b200 import inputs as gen
-from tests.parity_util import O_TOL, STATE_REL_FRO, to_cuda
+from tests.parity_util import O_TOL, STATE_REL_FRO, compare, oracle_forward, to_cuda
 
 pytestmark = pytest.mark.gpu
 
@@ -47,22 +52,39 @@ def _close(o, s, o_ref, s_ref):
             assert num <= STATE_REL_FRO * den + 1e-6
 
 
-def test_noalloc_matches_forward_on_two_calls_in_a_row():
+def _run_noalloc(L, x, case):
+    o = torch.full((case.B, case.T, case.HV, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    s = torch.full((case.N, case.HV, 128, 128), float("nan"), device="cuda")
+    assert _call_noalloc(L, x, o, s) == 0
+    torch.cuda.synchronize()
+    return o, s
+
+
+def test_noalloc_matches_forward_on_calls_in_a_row():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     import kda_gated_delta_prefill_b200 as kda
     L = kda.lib()
-    cases = [gen.Case("noalloc_varlen", B=1, T=400, H=2, HV=8, lengths=[130, 1, 64, 205], state="n01", seed=91),
-             gen.TAIL_STATE]
-    for case in cases:
-        x = to_cuda(gen.make_inputs(case))
+    poison = gen.Case("noalloc_poison", B=1, T=1201, H=2, HV=8, lengths=[300, 2, 129, 64, 500, 1, 205], state="n01",
+                      seed=90)
+    small = gen.Case("noalloc_varlen", B=1, T=400, H=2, HV=8, lengths=[130, 1, 64, 205], state="n01", seed=91)
+    cases = [poison, small, gen.TAIL_STATE]
+    for i, case in enumerate(cases):
+        x_cpu = gen.make_inputs(case)
+        x = to_cuda(x_cpu)
         o_ref, s_ref = kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"], x["cu_seqlens"])
-        B, T, H, HV = case.B, case.T, case.H, case.HV
-        o = torch.full((B, T, HV, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
-        s = torch.full((case.N, HV, 128, 128), float("nan"), device="cuda")
-        assert _call_noalloc(L, x, o, s) == 0
         torch.cuda.synchronize()
+        o, s = _run_noalloc(L, x, case)
         _close(o, s, o_ref, s_ref)
+        assert torch.equal(o, o_ref), case.name
+        assert torch.equal(s, s_ref), case.name
+        if case is small:  # the packed batch after the larger one, also against the oracle
+            compare(o, s, oracle_forward(x_cpu))
+    # the same small packed batch once more right after the plain batch
+    x = to_cuda(gen.make_inputs(small))
+    o_ref, s_ref = kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"], x["cu_seqlens"])
+    o, s = _run_noalloc(L, x, small)
+    assert torch.equal(o, o_ref) and torch.equal(s, s_ref)
 
 
 def test_noalloc_rejects_sizes_over_its_limit():
