@@ -236,6 +236,13 @@ __device__ __forceinline__ float ex2(float x)
     asm("ex2.approx.f32 %0, %1;\n" : "=f"(y) : "f"(x));
     return y;
 }
+// The same with subnormal inputs and results flushed to zero (a single special-function instruction).
+__device__ __forceinline__ float ex2_ftz(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // ---- shared-memory tile layouts ----
 // Rows of row_bytes (>= 128) with 16-byte chunks XOR-swizzled by row % 8 (the
