@@ -9,7 +9,7 @@ namespace {
 // the gradients at the chunk end states (bf16), the final state of a recomputed forward, and the per-value-head
 // gradients at the normalised q/k rows.
 struct BwdWorkspace {
-    size_t chunk_off = 0, ctr = 0, items = 0, fwd_total = 0, states = 0, dstates = 0, final_state = 0, dqn = 0, dkn = 0,
+    size_t chunk_off = 0, items = 0, fwd_total = 0, states = 0, dstates = 0, final_state = 0, dqn = 0, dkn = 0,
            total = 0;
     int64_t max_chunks = 0;
 };
@@ -22,7 +22,6 @@ BwdWorkspace bwd_workspace_layout(int B, int T, int HV, int num_seqs)
     const Workspace f = workspace_layout(B, T, HV, num_seqs);
     w.max_chunks = f.max_chunks;
     w.chunk_off = f.chunk_off;
-    w.ctr = f.ctr;
     w.items = f.items;
     w.fwd_total = f.total;
     const size_t rows = static_cast<size_t>(B) * T, state = static_cast<size_t>(DK) * DV * sizeof(float);
@@ -187,7 +186,6 @@ kda_status_t backward_impl(const void *q, const void *k, const void *v, const fl
             !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HV, tokens, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HV, tokens, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
             return KDA_ERR_CUDA;
-        ip.g = g;
         ip.beta = beta;
         ip.cu = cu_seqlens;
         ip.chunk_off = chunk_off;
@@ -199,14 +197,17 @@ kda_status_t backward_impl(const void *q, const void *k, const void *v, const fl
         ip.HV = HV;
         ip.N = d.N;
         ip.chunks_per_seq = (T + CH - 1) / CH;
-        if (cudaMemsetAsync(wsb + ws.ctr, 0, kCounterBytes, s) != cudaSuccess) return KDA_ERR_CUDA;
+        ip.prefetch_stride = info.sms * kda::kIntraCtasPerSm;
+        if (cudaFuncSetAttribute(kda::kda_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kda::IntraSmem::TOTAL) != cudaSuccess)
+            return KDA_ERR_CUDA;
     }
-    int *counters = reinterpret_cast<int *>(wsb + ws.ctr);
-    // launch j of the recomputed forward (j > 0: beside the carry of part j - 1)
-    auto launch_intra = [&](int chunk_begin, int chunk_count, int64_t grid_chunks, int j) {
+    auto launch_intra = [&](int chunk_begin, int chunk_count, int64_t grid_chunks) {
         ip.chunk_begin = chunk_begin;
         ip.chunk_count = chunk_count;
-        return launch_intra_kernel(tq, tk, tv, tg, ip, grid_chunks * HV, info.sms, counters + j, j > 0, s);
+        kda::kda_intra_kernel<<<static_cast<int>(grid_chunks * HV), 256, kda::IntraSmem::TOTAL, s>>>(tq, tk, tv, tg,
+                                                                                                      ip);
+        return cudaGetLastError();
     };
     kda::CarryParams cp{};
     cp.items = items;
@@ -241,7 +242,7 @@ kda_status_t backward_impl(const void *q, const void *k, const void *v, const fl
             const int c1 = j + 1 == parts ? nck : static_cast<int>(static_cast<int64_t>(nck) * 4 * (j + 1) / den);
             if (tokens > 0) {
                 const int64_t grid = parts == 1 ? ws.max_chunks : static_cast<int64_t>(B) * (c1 - c0);
-                if (launch_intra(c0, c1 - c0, grid, j) != cudaSuccess) return KDA_ERR_CUDA;
+                if (launch_intra(c0, c1 - c0, grid) != cudaSuccess) return KDA_ERR_CUDA;
             }
             if (cudaEventRecord(lane->fork, s) != cudaSuccess ||
                 cudaStreamWaitEvent(lane->stream, lane->fork, 0) != cudaSuccess)

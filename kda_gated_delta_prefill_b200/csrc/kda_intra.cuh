@@ -1,7 +1,6 @@
 // kda_intra.cuh -- intra-chunk kernel: everything of the chunk construction
 // that does not depend on the carried state, for one (chunk, value head)
-// item per CTA, fully parallel over items, with its contractions on the
-// 5th-generation tensor cores (tcgen05, accumulators in tensor memory).
+// item per CTA, fully parallel over items.
 //
 // "KDA Chunk Prefill on Ascend A3", section "Mathematical definition": for a
 // chunk of 64 tokens with inclusive per-channel cumulative gate G,
@@ -14,83 +13,54 @@
 // layouts the carry kernel's tensor-core descriptors read, so the carry
 // kernel copies it into shared memory with one bulk copy.
 //
-// Gate references.  exp(G_i - G_j) is split into a row factor and a column
-// factor that the tensor core multiplies over d.  The chunk is cut into two
-// 32-token halves; inside half h the reference is the midpoint
-// m_h = (G at the half's start + G at its end) / 2, so both factors stay
-// within exp(+-|half's gate sum| / 2); across the halves (rows of the second,
-// columns of the first) the reference is G_31 and both factors are <= 1.
-// With per-channel half sums >= -170 every factor the method needs stays a
-// normal bf16 number (per-token g >= -5 suffices).  All exponents are formed
-// in base 2: G2 = log2(e) G, factors 2^(G2 - m).
-//
-// A CTA (256 threads, two per SM) is persistent: it takes items from a
-// counter and, for each, runs
-//   1. Rows past the end of the sequence are zeroed (the page's zero padding
-//      of a partial chunk); q, k (Q/K head h / (HV/H)) and v arrived by TMA
-//      tile loads issued during the previous item, g and beta by plain loads
-//      into registers.
-//   2. L2 normalisation of q and k in place (l2norm_half_row, the routine of
-//      the standalone kda_l2norm_bf16 kernel).
-//   3. Gate sums and the operands: A1 = [k exp(G - m); K^-0.5 q exp(G - m)]
-//      (128 rows), B1 = k exp(m - G) (64 rows), A2 = the second half's k and q
-//      rows against G_31, B2 = the first half's k rows against G_31 (bf16),
-//      exp(G) k (fp16, W's operand), Qg and Kg (fp16, to the item block).
-//   4. MMA1 on tcgen05: D1 = A1 B1^T (128 x 64), D2 = A2 B2^T (128 x 32).  Once
-//      it completes, the next item's q/k tiles are requested into A1's place
-//      and its g values into registers.  Epilogue: L (beta-scaled, strictly
-//      lower) transposed into shared memory, Aqk (causal) to the item block.
-//   5. A: exact float32 forward substitution for the two diagonal 32 x 32
-//      blocks (one warp each, lane = column) while the other warps store Aqk,
-//      then the lower-left block -X_1 (L_10 X_0) on tf32 mma.sync, scaled by
-//      beta into fp16 A.
-//   6. MMA2 on tcgen05: W = A (exp(G) k) (M = 128 with 64 rows used) and
-//      U^T = v^T A^T; once it completes the next item's v tile is requested,
-//      and -W and U^T go from the accumulators straight to the item block.
-// One warp polls each tensor-core completion while the others wait at a
-// hardware barrier.  Every wait is bounded; a wait that gives up sets the
-// device error word and the CTA finishes its steps on whatever shared memory
-// holds.
+// Steps inside the CTA (256 threads):
+//   1. TMA tile loads of q, k (Q/K head h / (HV/H)), v, g; beta by plain
+//      loads.  Rows past the end of the sequence are zeroed (the page's zero
+//      padding of a partial chunk).
+//   2. L2 normalisation of q and k in place (exact rounding order).
+//   3. Gate factors from e_u = exp(g_u), one exponential per gate element:
+//      within each 16-token block the inclusive running product base_i and
+//      the exclusive suffix product b_j, block products P_J, and
+//      per-channel factors built from them, so that for i >= j
+//      exp(G_i - G_j) = base_i * (c_IJ * b_j) with every factor <= 1 except the
+//      diagonal-block c_II = 1/P_I (then c_II * b_j = 1/base_j <= e^75).
+//   4. L and Aqk: bf16 tensor-core MMAs over the ten lower 16x16 block pairs
+//      (bf16 keeps the range of the gate-rescaled operands).
+//   5. A: exact float32 forward substitution in the 16x16 diagonal blocks,
+//      tf32 MMAs for the blocks next to them and then for the lower-left
+//      32x32 block as -X_B (L_C X_A).
+//   6. W and U^T: fp16 tensor-core MMAs.
+// Results go straight from registers to the item block in global memory
+// (coalesced rows), so the CTA needs about 105 KB of shared memory and two
+// CTAs share an SM.
 #pragma once
 #include "kda_common.cuh"
 #include "kda_norm.cuh"
 #include "ptx.cuh"
-#include "tc.cuh"
 
 namespace kda {
 
 struct IntraSmem {
-    static constexpr int A1 = 0;          // bf16 [2 K-halves, 16384 apart][128 rows][128 B]: rows 0-63 k, 64-127 q
-    static constexpr int V = 32768;       // [2 value halves][64 tok][128 B]: v bf16, then fp16 in place
-    static constexpr int B1 = 49152;      // bf16 [2 K-halves, 8192 apart][64 tok][128 B]
-    static constexpr int A2 = 65536;      // bf16 [2 K-halves, 8192 apart][64 rows][128 B]: k (rows 0-31), q (32-63)
-    static constexpr int B2 = 81920;      // bf16 [2 K-halves, 4096 apart][32 tok][128 B]
-    static constexpr int KEXP = 90112;    // fp16 [2 K-halves, 8192 apart][64 tok][128 B]: exp(G) k
-    // once MMA1 has completed (B1's second K-half, A2 and B2 are free; A1 takes the next item's q and k)
-    static constexpr int ASOL = B1;       // fp16 [64 i][64 j] SW128: A = (I + L)^-1 diag(beta)
-    static constexpr int LD0 = 57344;     // fp32 [32 j][32]: column j of L_00, row i at (i % 4) * 8 + i / 4
-    static constexpr int LD1 = 61440;     // fp32 [32 j][32]: column j of L_11, the same order
-    static constexpr int L10T = 65536;    // fp32 [32 k][40]: L_10 transposed
-    static constexpr int X0 = 70656;      // fp32 [32][40]: (I + L_00)^-1
-    static constexpr int X1 = 75776;      // fp32 [32][36]: (I + L_11)^-1
-    static constexpr int Y = 80384;       // fp32 [32][40]: L_10 X_0
-    // once MMA2 has completed: the images of -W and U^T, stored by two bulk copies (read before the next
-    // item writes B1 and A2 again)
-    static constexpr int WST = B1;
-    static constexpr int UST = A2;
-    static constexpr int BETA = 106496;   // fp32 [64]
-    static constexpr int OT = 106752;     // fp32 [8 octets][128 channels]: gate sums of 8-token octets (base 2)
-    static constexpr int BAR = 110848;    // mbarriers: q/k tiles, v tile, MMA1, MMA2
-    static constexpr int TSLOT = BAR + 32;   // tensor-memory base address
-    static constexpr int NEXT = TSLOT + 4;   // the next item this CTA takes
-    static constexpr int TOTAL = NEXT + 12;
+    static constexpr int Q = 0;          // bf16 [64][128] (two SW128 halves): q -> normalised -> K^-0.5 q*base; X (step 5)
+    static constexpr int K = 16384;      // bf16: k -> normalised -> k*base; A fp16 [64][64] (step 5)
+    static constexpr int V = 32768;      // bf16 v -> fp16 v
+    static constexpr int G = 49152;      // fp32 [64][128] g; then KEXP fp16 (first half) and KBB bf16 (second half)
+    static constexpr int KEXP = G;
+    static constexpr int KBB = G + 16384;
+    static constexpr int L = 81920;      // fp32 [64][64]
+    static constexpr int X = Q;          // fp32 [64][64], once q*base is no longer needed
+    static constexpr int A = K;          // fp16 [64][64], once k*base is no longer needed
+    static constexpr int WST = Q;        // fp16 -W staging (step 6), once X is no longer needed
+    static constexpr int UST = L;        // fp16 U^T staging (step 6), once L is no longer needed
+    static constexpr int BETA = 98304;   // fp32 [64]
+    static constexpr int CF = 98560;     // bf16x2 [10][64] block-pair factors
+    static constexpr int PS = 101120;    // float2 [4][64] block products; later float [32][40] (over PS and TS)
+    static constexpr int TS = 103168;    // fp32 8 x [16][8] solve scratch
+    static constexpr int BAR = 107776;   // mbarriers: q/k/g tiles, v tile
+    static constexpr int TOTAL = 107848;
 };
-static_assert(IntraSmem::Y + 32 * 40 * 4 <= IntraSmem::KEXP, "solve scratch overlaps exp(G) k");
-static_assert(IntraSmem::LD0 == IntraSmem::B1 + 8192, "the solve scratch starts after A");
-static_assert(IntraSmem::UST + 16384 <= IntraSmem::KEXP, "the U^T image overlaps exp(G) k");
 
 struct IntraParams {
-    const float *g;            // [rows][HV][128]
     const float *beta;
     const int32_t *cu;         // [N+1] or null
     const int32_t *chunk_off;  // [N+1] chunk offsets of the packed sequences, or null
@@ -100,26 +70,58 @@ struct IntraParams {
     int chunks_per_seq;        // ceil(T/64) when cu is null
     int chunk_begin;           // cu null: this launch covers chunks [chunk_begin, chunk_begin + chunk_count)
     int chunk_count;           //   of every sequence (cu given: all chunks, chunk_begin = 0)
-    int *counter;              // persistent launch: items taken so far beyond the first gridDim.x (zero before
-                               //   the launch); null: one item per CTA
-    int n_items;               // (chunk, value head) items of this launch
-    int prefetch_stride;       // one item per CTA: CTAs resident at once (the item whose inputs to pull into L2)
+    int prefetch_stride;       // CTAs resident at once (L2 prefetch distance), 0 = no prefetch
 };
 
-constexpr int kIntraCtasPerSm = 2;           // the shared-memory footprint lets two CTAs share an SM
-constexpr uint32_t kIntraTmemCols = 256;     // D1 + D2 (96 columns), later W (128) + U^T (64)
-
-__device__ __forceinline__ void intra_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
-
-__device__ __forceinline__ float4 f4add(float4 a, float4 b)
+// Off-diagonal block of X = (I+L)^-1, columns 16J+8nt .. +7:
+//   X_IJ = -D_I * sum_{M=J}^{I-1} L_IM X_MJ   (D_I = X_II; one warp, tf32 MMAs),
+// written as fp32 X (for later blocks) and as fp16 A = X diag(beta) (for W and U).
+// ts: this warp's [16][8] float scratch for the intermediate sum.
+__device__ __forceinline__ void solve_block(const uint8_t *sL, uint8_t *sX, uint8_t *sA, const float *beta, float *ts, int I,
+                                            int J, int nt, int lane)
 {
-    const float2 lo = add2(make_float2(a.x, a.y), make_float2(b.x, b.y));
-    const float2 hi = add2(make_float2(a.z, a.w), make_float2(b.z, b.w));
-    return make_float4(lo.x, lo.y, hi.x, hi.y);
+    const int g = lane >> 2, t = lane & 3;
+    auto Lat = [&](int r, int c) { return *reinterpret_cast<const float *>(sL + swz(r, c * 4, 256)); };
+    auto Xat = [&](int r, int c) { return *reinterpret_cast<const float *>(sX + swz(r, c * 4, 256)); };
+    const int cn = 16 * J + 8 * nt + g;  // this lane's column of the B fragments
+    float acc[4] = {};
+    for (int M = J; M < I; ++M) {
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t a[4];
+            a[0] = to_tf32(Lat(16 * I + g, 16 * M + 8 * ks + t));
+            a[1] = to_tf32(Lat(16 * I + g + 8, 16 * M + 8 * ks + t));
+            a[2] = to_tf32(Lat(16 * I + g, 16 * M + 8 * ks + t + 4));
+            a[3] = to_tf32(Lat(16 * I + g + 8, 16 * M + 8 * ks + t + 4));
+            mma_tf32(acc, a, to_tf32(Xat(16 * M + 8 * ks + t, cn)), to_tf32(Xat(16 * M + 8 * ks + t + 4, cn)));
+        }
+    }
+    ts[g * 8 + 2 * t] = acc[0];
+    ts[g * 8 + 2 * t + 1] = acc[1];
+    ts[(g + 8) * 8 + 2 * t] = acc[2];
+    ts[(g + 8) * 8 + 2 * t + 1] = acc[3];
+    __syncwarp();
+    float x[4] = {};
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        uint32_t a[4];
+        a[0] = to_tf32(Xat(16 * I + g, 16 * I + 8 * ks + t));
+        a[1] = to_tf32(Xat(16 * I + g + 8, 16 * I + 8 * ks + t));
+        a[2] = to_tf32(Xat(16 * I + g, 16 * I + 8 * ks + t + 4));
+        a[3] = to_tf32(Xat(16 * I + g + 8, 16 * I + 8 * ks + t + 4));
+        mma_tf32(x, a, to_tf32(ts[(8 * ks + t) * 8 + g]), to_tf32(ts[(8 * ks + t + 4) * 8 + g]));
+    }
+    const int c = 16 * J + 8 * nt + 2 * t;
+    *reinterpret_cast<float2 *>(sX + swz(16 * I + g, c * 4, 256)) = make_float2(-x[0], -x[1]);
+    *reinterpret_cast<float2 *>(sX + swz(16 * I + g + 8, c * 4, 256)) = make_float2(-x[2], -x[3]);
+    // A = X diag(beta) in fp16 for step 6
+    const float b0 = beta[c], b1 = beta[c + 1];
+    *reinterpret_cast<uint32_t *>(sA + swz(16 * I + g, c * 2, 128)) = pack_f16(-x[0] * b0, -x[1] * b1);
+    *reinterpret_cast<uint32_t *>(sA + swz(16 * I + g + 8, c * 2, 128)) = pack_f16(-x[2] * b0, -x[3] * b1);
+    __syncwarp();
 }
 
-// 16-byte chunk c of row r in a 128-byte-swizzled tile of 128-byte rows
-__device__ __forceinline__ uint32_t sw_chunk(int r, int c) { return static_cast<uint32_t>(r * 128 + ((c ^ (r & 7)) << 4)); }
+constexpr int kIntraCtasPerSm = 2;  // the shared-memory footprint and register cap let two CTAs share an SM
 
 __global__ void __launch_bounds__(256, kIntraCtasPerSm)
     kda_intra_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -132,510 +134,385 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g8 = lane >> 2, t4 = lane & 3;
 
-    // ---- item -> (item chunk index, value head, row of the chunk start, valid rows); false past the end ----
+    // ---- launch-local chunk -> (item chunk index, row of the chunk start, valid rows); false past the end ----
     const int nchunks = p.cu ? p.chunk_off[p.N] : p.B * p.chunk_count;
-    struct Item {
-        int ci, h, hq, nvalid;
-        int64_t row0;
-    };
-    auto locate = [&](int item, Item &it) {
-        if (item >= p.n_items) return false;
-        const int local = item / p.HV;
+    auto locate = [&](int local, int &ci, int64_t &row0, int &nvalid) {
         if (local >= nchunks) return false;
-        it.h = item % p.HV;
-        it.hq = it.h / (p.HV / p.H);
         if (p.cu) {
-            it.ci = local;
+            ci = local;
             int lo = 0, hi = p.N - 1;  // last n with chunk_off[n] <= ci
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
-                if (p.chunk_off[mid] <= local) lo = mid; else hi = mid - 1;
+                if (p.chunk_off[mid] <= ci) lo = mid; else hi = mid - 1;
             }
-            const int c = local - p.chunk_off[lo];
+            const int c = ci - p.chunk_off[lo];
             const int len = p.cu[lo + 1] - p.cu[lo];
-            it.row0 = p.cu[lo] + static_cast<int64_t>(c) * CH;
-            it.nvalid = min(CH, len - c * CH);
+            row0 = p.cu[lo] + static_cast<int64_t>(c) * CH;
+            nvalid = min(CH, len - c * CH);
         } else {
             const int b = local / p.chunk_count, c = p.chunk_begin + local % p.chunk_count;
-            it.ci = b * p.chunks_per_seq + c;
-            it.row0 = static_cast<int64_t>(b) * p.T + static_cast<int64_t>(c) * CH;
-            it.nvalid = min(CH, p.T - c * CH);
+            ci = b * p.chunks_per_seq + c;
+            row0 = static_cast<int64_t>(b) * p.T + static_cast<int64_t>(c) * CH;
+            nvalid = min(CH, p.T - c * CH);
         }
         return true;
     };
-    // this thread's gate values: tokens 8*warp .. 8*warp+7, channels 4*lane .. 4*lane+3 (zero past the valid
-    // rows), and the item's beta (threads 0-63)
-    auto load_g = [&](const Item &it, float4 (&gv)[8], float &bt) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = 8 * warp + u;
-            gv[u] = i < it.nvalid
-                        ? __ldg(reinterpret_cast<const float4 *>(p.g + ((it.row0 + i) * p.HV + it.h) * DK) + lane)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        bt = (tid < it.nvalid) ? __ldg(p.beta + (it.row0 + tid) * p.HV + it.h) : 0.f;
-    };
-    const uint32_t bar_qk = sb + S::BAR, bar_v = bar_qk + 8, bar_m1 = bar_qk + 16, bar_m2 = bar_qk + 24;
-    auto load_qk = [&](const Item &it) {  // thread 0
-        mbar_expect_tx(bar_qk, 32768);
-        const int z = static_cast<int>(it.row0);
-        tma_load_3d(sb + S::A1, &tk, 0, it.hq, z, bar_qk);           // k, channels 0-63: rows 0-63 of K-half 0
-        tma_load_3d(sb + S::A1 + 16384, &tk, 64, it.hq, z, bar_qk);  // k, channels 64-127: rows 0-63 of K-half 1
-        tma_load_3d(sb + S::A1 + 8192, &tq, 0, it.hq, z, bar_qk);    // q: rows 64-127
-        tma_load_3d(sb + S::A1 + 24576, &tq, 64, it.hq, z, bar_qk);
-    };
-    auto load_v = [&](const Item &it) {  // thread 0
-        mbar_expect_tx(bar_v, 16384);
-        const int z = static_cast<int>(it.row0);
-        tma_load_3d(sb + S::V, &tv, 0, it.h, z, bar_v);
-        tma_load_3d(sb + S::V + 8192, &tv, 64, it.h, z, bar_v);
-    };
-    auto prefetch = [&](const Item &it) {  // thread 0: the item's inputs into L2
-        const int z = static_cast<int>(it.row0);
-        tma_prefetch_3d(&tq, 0, it.hq, z);
-        tma_prefetch_3d(&tq, 64, it.hq, z);
-        tma_prefetch_3d(&tk, 0, it.hq, z);
-        tma_prefetch_3d(&tk, 64, it.hq, z);
-        tma_prefetch_3d(&tv, 0, it.h, z);
-        tma_prefetch_3d(&tv, 64, it.h, z);
-        tma_prefetch_3d(&tg, 0, it.h, z);
-    };
+    const int h = blockIdx.x % p.HV;
+    int ci;
+    int64_t row0;
+    int nvalid;
+    if (!locate(blockIdx.x / p.HV, ci, row0, nvalid)) return;
+    const int hq = h / (p.HV / p.H);
+    uint8_t *out = p.items + (static_cast<int64_t>(ci) * p.HV + h) * ITEM_BYTES;  // item block (global)
 
-    Item cur;
-    if (!locate(blockIdx.x, cur)) return;
+    // ---- 1. loads ----
+    const uint32_t bar = sb + S::BAR;
     if (tid == 0) {
-        mbar_init(bar_qk, 1);
-        mbar_init(bar_v, 1);
-        mbar_init(bar_m1, 1);
-        mbar_init(bar_m2, 1);
+        mbar_init(bar, 1);
+        mbar_init(bar + 8, 1);
         fence_mbar_init();
-        load_qk(cur);
-        load_v(cur);
     }
-    if (warp == 0) tc_alloc(sb + S::TSLOT, kIntraTmemCols);
-    float4 gv[8];
-    float bt;
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + S::TSLOT);
-    float *sbeta = reinterpret_cast<float *>(sm + S::BETA);
-    volatile int *snext = reinterpret_cast<volatile int *>(sm + S::NEXT);
-
-    for (int iter = 0;; ++iter) {
-        const uint32_t par = iter & 1;
-        uint8_t *out = p.items + (static_cast<int64_t>(cur.ci) * p.HV + cur.h) * ITEM_BYTES;  // item block (global)
-        // this item's gate values and beta into registers (used after the normalisation); the next item: in a
-        // persistent launch claimed now and published (its inputs pulled into L2) after the normalisation, so
-        // that the atomic's latency is off the path; otherwise none
-        load_g(cur, gv, bt);
-        int claim = p.n_items;
-        if (tid == 0 && p.counter) claim = static_cast<int>(gridDim.x) + atomicAdd(p.counter, 1);
-        if (!mbar_wait(bar_qk, par)) atomicOr(p.err, ERR_TMA_WAIT);
-        if (cur.nvalid < CH) {  // zero the rows past the sequence's end (another sequence's or batch row's tokens)
-            for (int idx = tid; idx < (CH - cur.nvalid) * 32; idx += 256) {
-                const int r = cur.nvalid + idx / 32, w = idx % 32;  // 16-byte words of the row: k and q, two K-halves
-                const int isq = w >> 4, kh = (w >> 3) & 1, c = w & 7;
-                *reinterpret_cast<uint4 *>(sm + S::A1 + kh * 16384 + (64 * isq + r) * 128 + c * 16) =
-                    make_uint4(0, 0, 0, 0);
-            }
+    if (tid == 0) {
+        mbar_expect_tx(bar, 2 * 16384 + 32768);
+        mbar_expect_tx(bar + 8, 16384);
+        const int z = static_cast<int>(row0);
+        tma_load_3d(sb + S::Q, &tq, 0, hq, z, bar);
+        tma_load_3d(sb + S::Q + 8192, &tq, 64, hq, z, bar);
+        tma_load_3d(sb + S::K, &tk, 0, hq, z, bar);
+        tma_load_3d(sb + S::K + 8192, &tk, 64, hq, z, bar);
+        tma_load_3d(sb + S::V, &tv, 0, h, z, bar + 8);
+        tma_load_3d(sb + S::V + 8192, &tv, 64, h, z, bar + 8);
+        tma_load_3d(sb + S::G, &tg, 0, h, z, bar);
+        // The CTA that takes this slot after the current wave of resident CTAs will want item
+        // blockIdx.x + prefetch_stride: pull its inputs into L2 now, so that its loads overlap the compute
+        // of this wave instead of waiting on DRAM.
+        const int pi = blockIdx.x + p.prefetch_stride;
+        int pci, pvalid;
+        int64_t prow;
+        if (p.prefetch_stride > 0 && pi < static_cast<int>(gridDim.x) && locate(pi / p.HV, pci, prow, pvalid)) {
+            const int ph = pi % p.HV, pz = static_cast<int>(prow), phq = ph / (p.HV / p.H);
+            tma_prefetch_3d(&tq, 0, phq, pz);
+            tma_prefetch_3d(&tq, 64, phq, pz);
+            tma_prefetch_3d(&tk, 0, phq, pz);
+            tma_prefetch_3d(&tk, 64, phq, pz);
+            tma_prefetch_3d(&tv, 0, ph, pz);
+            tma_prefetch_3d(&tv, 64, ph, pz);
+            tma_prefetch_3d(&tg, 0, ph, pz);
         }
-        intra_sync();
-
-        // ---- 2. normalise k (rows 0-63) and q (rows 64-127): thread = row half, the partner lane holds the rest ----
-        {
-            const int r = tid >> 1, kh = tid & 1;
-            uint8_t *row = sm + S::A1 + kh * 16384 + r * 128;
-            uint4 raw[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) raw[c] = *reinterpret_cast<const uint4 *>(row + ((c ^ (r & 7)) << 4));
-            l2norm_half_row(raw);  // the routine the standalone kda_l2norm_bf16 kernel runs
-#pragma unroll
-            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(row + ((c ^ (r & 7)) << 4)) = raw[c];
-        }
-
-        // ---- 3. gate sums (base 2) and the operands: warp = token octet, lane = channel quad ----
-        {
-            const float2 l2e = make_float2(1.4426950408889634f, 1.4426950408889634f);
-            float4 *ot = reinterpret_cast<float4 *>(sm + S::OT);
-            {
-                float2 lo = make_float2(0.f, 0.f), hi = lo;
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    lo = add2(lo, mul2(make_float2(gv[u].x, gv[u].y), l2e));
-                    hi = add2(hi, mul2(make_float2(gv[u].z, gv[u].w), l2e));
-                }
-                ot[warp * 32 + lane] = make_float4(lo.x, lo.y, hi.x, hi.y);
-            }
-            if (tid == 0) {
-                *snext = claim;
-                Item ni;
-                // the item a later CTA (or this one next) takes: its inputs into L2
-                if (locate(p.counter ? claim : static_cast<int>(blockIdx.x) + p.prefetch_stride, ni)) prefetch(ni);
-                bulk_wait_read();  // the previous item's -W and U^T images (over B1 and A2) have been read
-            }
-            if (tid < CH) sbeta[tid] = bt;
-            intra_sync();  // also: every row is normalised
-            float4 before = make_float4(0.f, 0.f, 0.f, 0.f), g31 = before, g63 = before;
-#pragma unroll
-            for (int o = 0; o < 8; ++o) {
-                const float4 t = ot[o * 32 + lane];
-                if (o < warp) before = f4add(before, t);
-                if (o < 4) g31 = f4add(g31, t);
-                g63 = f4add(g63, t);
-            }
-            const int half = warp >> 2;
-            // reference of this half: m0 = G31 / 2, m1 = (G31 + G63) / 2
-            const float4 m = half == 0 ? make_float4(0.5f * g31.x, 0.5f * g31.y, 0.5f * g31.z, 0.5f * g31.w)
-                                       : make_float4(0.5f * (g31.x + g63.x), 0.5f * (g31.y + g63.y),
-                                                     0.5f * (g31.z + g63.z), 0.5f * (g31.w + g63.w));
-            // per-channel factors: 2^m (exp(G) = f 2^m), 2^(G63 - m) (exp(G_last - G) = fi 2^(G63 - m)), and the
-            // change to the reference G31: 2^(G31 / 2) for the first half's key rows (G31 - m0), 2^((G63 - G31) / 2)
-            // for the second half's rows (m1 - G31)
-            const float4 eM = make_float4(ex2(m.x), ex2(m.y), ex2(m.z), ex2(m.w));
-            const float4 eL = make_float4(ex2(g63.x - m.x), ex2(g63.y - m.y), ex2(g63.z - m.z), ex2(g63.w - m.w));
-            const float4 cx = half == 0 ? make_float4(ex2(0.5f * g31.x), ex2(0.5f * g31.y), ex2(0.5f * g31.z),
-                                                      ex2(0.5f * g31.w))
-                                        : make_float4(ex2(0.5f * (g63.x - g31.x)), ex2(0.5f * (g63.y - g31.y)),
-                                                      ex2(0.5f * (g63.z - g31.z)), ex2(0.5f * (g63.w - g31.w)));
-            if (warp == 0)
-                *reinterpret_cast<float4 *>(out + ITEM_GL + 16 * lane) =
-                    make_float4(ex2(g63.x), ex2(g63.y), ex2(g63.z), ex2(g63.w));
-            // K^-0.5 = 128^-0.5 in float32 is applied to Qg here and to Aqk in its epilogue
-            const float sc = 0.08838834764831845f;
-            const float2 eM01 = make_float2(eM.x, eM.y), eM23 = make_float2(eM.z, eM.w);
-            const float2 eQ01 = make_float2(eM.x * sc, eM.y * sc), eQ23 = make_float2(eM.z * sc, eM.w * sc);
-            const float2 eL01 = make_float2(eL.x, eL.y), eL23 = make_float2(eL.z, eL.w);
-            const float2 cx01 = make_float2(cx.x, cx.y), cx23 = make_float2(cx.z, cx.w);
-            const float2 mlo = make_float2(m.x, m.y), mhi = make_float2(m.z, m.w);
-            const int kh = lane >> 4, cq = (lane & 15) >> 1, sub = (lane & 1) * 8;  // K-half, 16-byte chunk, offset
-            float2 Glo = make_float2(before.x, before.y), Ghi = make_float2(before.z, before.w);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int i = 8 * warp + u;  // token; i % 8 == u
-                Glo = add2(Glo, mul2(make_float2(gv[u].x, gv[u].y), l2e));  // inclusive cumulative gate (base 2)
-                Ghi = add2(Ghi, mul2(make_float2(gv[u].z, gv[u].w), l2e));
-                const float2 x01 = make_float2(Glo.x - mlo.x, Glo.y - mlo.y), x23 = make_float2(Ghi.x - mhi.x, Ghi.y - mhi.y);
-                const float2 f01 = make_float2(ex2_ftz(x01.x), ex2_ftz(x01.y)), f23 = make_float2(ex2_ftz(x23.x), ex2_ftz(x23.y));
-                const float2 fi01 = make_float2(ex2_ftz(-x01.x), ex2_ftz(-x01.y));
-                const float2 fi23 = make_float2(ex2_ftz(-x23.x), ex2_ftz(-x23.y));
-                const uint32_t o1 = kh * 16384 + ((cq ^ u) << 4) + sub;  // in A1 (row offset added below)
-                const uint32_t o2 = kh * 8192 + ((cq ^ u) << 4) + sub;   // in the [2][rows][128 B] tiles
-                const uint2 kr = *reinterpret_cast<const uint2 *>(sm + S::A1 + i * 128 + o1);
-                const uint2 qr = *reinterpret_cast<const uint2 *>(sm + S::A1 + (64 + i) * 128 + o1);
-                const float2 k01 = unpack_bf16(kr.x), k23 = unpack_bf16(kr.y);
-                const float2 q01 = unpack_bf16(qr.x), q23 = unpack_bf16(qr.y);
-                const float2 ak01 = mul2(k01, f01), ak23 = mul2(k23, f23);
-                const float2 aq01 = mul2(q01, f01), aq23 = mul2(q23, f23);
-                const float2 bk01 = mul2(k01, fi01), bk23 = mul2(k23, fi23);
-                *reinterpret_cast<uint2 *>(sm + S::A1 + i * 128 + o1) =
-                    make_uint2(pack_bf16(ak01.x, ak01.y), pack_bf16(ak23.x, ak23.y));
-                *reinterpret_cast<uint2 *>(sm + S::A1 + (64 + i) * 128 + o1) =
-                    make_uint2(pack_bf16(aq01.x, aq01.y), pack_bf16(aq23.x, aq23.y));
-                *reinterpret_cast<uint2 *>(sm + S::B1 + i * 128 + o2) =
-                    make_uint2(pack_bf16(bk01.x, bk01.y), pack_bf16(bk23.x, bk23.y));
-                const float2 ke01 = mul2(ak01, eM01), ke23 = mul2(ak23, eM23);
-                *reinterpret_cast<uint2 *>(sm + S::KEXP + i * 128 + o2) =
-                    make_uint2(pack_f16(ke01.x, ke01.y), pack_f16(ke23.x, ke23.y));
-                const float2 qg01 = mul2(aq01, eQ01), qg23 = mul2(aq23, eQ23);
-                *reinterpret_cast<uint2 *>(out + ITEM_QG + i * 128 + o2) =
-                    make_uint2(pack_f16(qg01.x, qg01.y), pack_f16(qg23.x, qg23.y));
-                const float2 kg01 = mul2(bk01, eL01), kg23 = mul2(bk23, eL23);
-                *reinterpret_cast<uint2 *>(out + ITEM_KG + i * 128 + o2) =
-                    make_uint2(pack_f16(kg01.x, kg01.y), pack_f16(kg23.x, kg23.y));
-                if (half == 0) {  // B2 row i: k exp(G31 - G)
-                    const float2 b01 = mul2(bk01, cx01), b23 = mul2(bk23, cx23);
-                    *reinterpret_cast<uint2 *>(sm + S::B2 + kh * 4096 + i * 128 + ((cq ^ u) << 4) + sub) =
-                        make_uint2(pack_bf16(b01.x, b01.y), pack_bf16(b23.x, b23.y));
-                } else {          // A2 rows i - 32 (k) and i (q): exp(G - G31)
-                    const float2 a01 = mul2(ak01, cx01), a23 = mul2(ak23, cx23);
-                    const float2 c01 = mul2(aq01, cx01), c23 = mul2(aq23, cx23);
-                    *reinterpret_cast<uint2 *>(sm + S::A2 + (i - 32) * 128 + o2) =
-                        make_uint2(pack_bf16(a01.x, a01.y), pack_bf16(a23.x, a23.y));
-                    *reinterpret_cast<uint2 *>(sm + S::A2 + i * 128 + o2) =
-                        make_uint2(pack_bf16(c01.x, c01.y), pack_bf16(c23.x, c23.y));
-                }
-            }
-        }
-        fence_proxy_async();  // the operands are read by the tensor core (async proxy)
-        tc_fence_before();
-        intra_sync();
-
-        // ---- 4. MMA1: D1 = A1 B1^T (TMEM columns 0-63), D2 = A2 B2^T (columns 64-95) ----
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t i1 = idesc_kind_f16(128, 64, true, false, false);
-            const uint32_t i2 = idesc_kind_f16(128, 32, true, false, false);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t kb = (ks & 3) * 32;
-                tc_mma_ss(tmem, sw128_desc(sb + S::A1 + (ks >> 2) * 16384 + kb, 16, 1024),
-                          sw128_desc(sb + S::B1 + (ks >> 2) * 8192 + kb, 16, 1024), i1, ks > 0);
-            }
-            // A2 spans 128 rows of which 64 are used: its rows 64-127 read the next 8 KB (the other K-half, or B2)
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t kb = (ks & 3) * 32;
-                tc_mma_ss(tmem + 64, sw128_desc(sb + S::A2 + (ks >> 2) * 8192 + kb, 16, 1024),
-                          sw128_desc(sb + S::B2 + (ks >> 2) * 4096 + kb, 16, 1024), i2, ks > 0);
-            }
-            tc_commit(bar_m1);
-        }
-        // v (its copy overlapped the steps above): zero the padding rows, bf16 -> fp16 in place
-        if (!mbar_wait(bar_v, par)) atomicOr(p.err, ERR_TMA_WAIT);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int idx = tid + 256 * k;  // 16-byte chunk: half (idx >> 9), row ((idx >> 3) & 63)
-            uint4 *pv = reinterpret_cast<uint4 *>(sm + S::V) + idx;
-            const uint4 uu = *pv;
-            uint32_t w[4] = {uu.x, uu.y, uu.z, uu.w};
-            const bool pad = ((idx >> 3) & 63) >= cur.nvalid;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 xv = unpack_bf16(w[j]);
-                w[j] = pad ? 0u : pack_f16(xv.x, xv.y);
-            }
-            *pv = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        if (warp == 0 && !mbar_wait_spin(bar_m1, par) && lane == 0) atomicOr(p.err, ERR_PIPE_FULL_WAIT);
-        intra_sync();
-        tc_fence_after();
-        // A1 is free: the next item's q and k tiles
-        Item nxt;
-        const bool more = locate(*snext, nxt);
-        if (more && tid == 0) load_qk(nxt);
-
-        // ---- 4b. MMA1 epilogue: warp = TMEM lane quarter (warp & 3) x role ----
-        {
-            float *LD0 = reinterpret_cast<float *>(sm + S::LD0);
-            float *LD1 = reinterpret_cast<float *>(sm + S::LD1);
-            float *L10T = reinterpret_cast<float *>(sm + S::L10T);
-            const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
-            const int perm = (lane & 3) * 8 + (lane >> 2);  // where row `lane` of a diagonal block sits in LD
-            uint32_t r[32];
-            // Aqk row i (times K^-0.5), 16-byte chunks c0 .. c0+3 from 32 accumulator columns; j <= jmax kept
-            auto aqk_row = [&](int i, int c0, int jmax) {
-                const float sc = 0.08838834764831845f;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = 8 * c + 2 * e;
-                        w[e] = pack_f16(j <= jmax ? sc * __uint_as_float(r[j]) : 0.f,
-                                        j + 1 <= jmax ? sc * __uint_as_float(r[j + 1]) : 0.f);
-                    }
-                    *reinterpret_cast<uint4 *>(out + ITEM_AQK + sw_chunk(i, c0 + c)) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            };
-            switch (warp) {
-            case 0: {  // L_00, rows i = lane (D1 lanes 0-31, columns 0-31)
-                tc_ld32(tl, r);
-                tc_wait_ld();
-                const float bi = sbeta[lane];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) LD0[j * 32 + perm] = j < lane ? bi * __uint_as_float(r[j]) : 0.f;
-                break;
-            }
-            case 1: {  // L_11, rows 32 + lane (D1 lanes 32-63, columns 32-63)
-                tc_ld32(tl + 32, r);
-                tc_wait_ld();
-                const float bi = sbeta[32 + lane];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) LD1[j * 32 + perm] = j < lane ? bi * __uint_as_float(r[j]) : 0.f;
-                break;
-            }
-            case 4: {  // L_10, rows 32 + lane (D2 lanes 0-31): every column j < 32 is below the diagonal
-                tc_ld32(tl + 64, r);
-                tc_wait_ld();
-                const float bi = sbeta[32 + lane];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) L10T[j * 40 + lane] = bi * __uint_as_float(r[j]);
-                break;
-            }
-            case 5:  // Aqk_10: rows 32 + lane (D2 lanes 32-63), columns 0-31
-                tc_ld32(tl + 64, r);
-                tc_wait_ld();
-                aqk_row(32 + lane, 0, 31);
-                break;
-            case 2:  // Aqk_00: rows lane (D1 lanes 64-95), columns 0-31, causal
-                tc_ld32(tl, r);
-                tc_wait_ld();
-                aqk_row(lane, 0, lane);
-                break;
-            case 3:  // Aqk_11: rows 32 + lane (D1 lanes 96-127), columns 32-63, causal
-                tc_ld32(tl + 32, r);
-                tc_wait_ld();
-                aqk_row(32 + lane, 4, lane);
-                break;
-            case 6:  // Aqk rows 0-31, columns 32-63: above the diagonal
-#pragma unroll
-                for (int c = 4; c < 8; ++c)
-                    *reinterpret_cast<uint4 *>(out + ITEM_AQK + sw_chunk(lane, c)) = make_uint4(0, 0, 0, 0);
-                break;
-            default:  // A rows 0-31, columns 32-63: above the diagonal
-#pragma unroll
-                for (int c = 4; c < 8; ++c)
-                    *reinterpret_cast<uint4 *>(sm + S::ASOL + sw_chunk(lane, c)) = make_uint4(0, 0, 0, 0);
-                break;
-            }
-        }
-        tc_fence_before();
-        intra_sync();
-
-        // ---- 5. A = (I + L)^-1 diag(beta) ----
-        {  // diagonal blocks: exact float32 substitution on all 256 threads.  Thread = (block, column c, row group
-           // r4 holding rows r4, r4 + 4, ..., r4 + 28); the four threads of a column are adjacent lanes.
-           // Right-looking: row j, once final, is broadcast to its column's lanes and updates every later row,
-           // each row taking its terms in the order j = 0, 1, ...; L's zeros above the diagonal make the
-           // updates of earlier rows no-ops.
-            const int blk = warp >> 2, c = (warp & 3) * 8 + (lane >> 2), r4 = lane & 3;
-            const float *LD = reinterpret_cast<const float *>(sm + (blk ? S::LD1 : S::LD0));
-            float x[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) x[q] = 4 * q + r4 == c ? 1.f : 0.f;
-#pragma unroll
-            for (int j = 0; j < 31; ++j) {
-                const float xj = __shfl_sync(0xffffffffu, x[j >> 2], (lane & ~3) | (j & 3));
-                const float4 *col = reinterpret_cast<const float4 *>(LD + j * 32 + r4 * 8);  // L[4q + r4][j], q = 0..7
-                float l[8];
-                if (j < 16) {
-                    const float4 lo = col[0];
-                    l[0] = lo.x; l[1] = lo.y; l[2] = lo.z; l[3] = lo.w;
-                }
-                const float4 hi = col[1];
-                l[4] = hi.x; l[5] = hi.y; l[6] = hi.z; l[7] = hi.w;
-#pragma unroll
-                for (int q = j >> 2; q < 8; ++q)
-                    if (j < 16 || q >= 4) x[q] = __fmaf_rn(-l[q], xj, x[q]);
-            }
-            float *Xs = reinterpret_cast<float *>(sm + (blk ? S::X1 : S::X0));
-            const int xs = blk ? 36 : 40, o = 32 * blk;
-            const float bc = sbeta[o + c];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int i = 4 * q + r4;
-                Xs[i * xs + c] = x[q];
-                *reinterpret_cast<__half *>(sm + S::ASOL + sw_chunk(o + i, (o + c) >> 3) + ((o + c) & 7) * 2) =
-                    __float2half_rn(x[q] * bc);
-            }
-        }
-        intra_sync();
-        {  // Y = L_10 X_0 (tf32, warp = 16 x 8 tile)
-            const int mt = warp >> 2, nt = warp & 3;
-            const float *L10T = reinterpret_cast<const float *>(sm + S::L10T);
-            const float *X0 = reinterpret_cast<const float *>(sm + S::X0);
-            float d[4] = {};
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const int kb = 8 * ks, m0 = 16 * mt + g8;  // L_10[m][k] = L10T[k][m]
-                uint32_t a[4];
-                a[0] = to_tf32(L10T[(kb + t4) * 40 + m0]);
-                a[1] = to_tf32(L10T[(kb + t4) * 40 + m0 + 8]);
-                a[2] = to_tf32(L10T[(kb + t4 + 4) * 40 + m0]);
-                a[3] = to_tf32(L10T[(kb + t4 + 4) * 40 + m0 + 8]);
-                mma_tf32(d, a, to_tf32(X0[(kb + t4) * 40 + 8 * nt + g8]), to_tf32(X0[(kb + t4 + 4) * 40 + 8 * nt + g8]));
-            }
-            float *Yf = reinterpret_cast<float *>(sm + S::Y);
-            *reinterpret_cast<float2 *>(Yf + (16 * mt + g8) * 40 + 8 * nt + 2 * t4) = make_float2(d[0], d[1]);
-            *reinterpret_cast<float2 *>(Yf + (16 * mt + g8 + 8) * 40 + 8 * nt + 2 * t4) = make_float2(d[2], d[3]);
-        }
-        intra_sync();
-        {  // A_10 = -(X_1 Y) diag(beta_0..31) (tf32; X_1 rows 0-15 are zero beyond column 15)
-            const int mt = warp >> 2, nt = warp & 3;
-            const float *X1 = reinterpret_cast<const float *>(sm + S::X1);
-            const float *Yf = reinterpret_cast<const float *>(sm + S::Y);
-            float d[4] = {};
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                if (mt == 0 && ks >= 2) continue;
-                const int kb = 8 * ks, m0 = 16 * mt + g8;
-                uint32_t a[4];
-                a[0] = to_tf32(X1[m0 * 36 + kb + t4]);
-                a[1] = to_tf32(X1[(m0 + 8) * 36 + kb + t4]);
-                a[2] = to_tf32(X1[m0 * 36 + kb + t4 + 4]);
-                a[3] = to_tf32(X1[(m0 + 8) * 36 + kb + t4 + 4]);
-                mma_tf32(d, a, to_tf32(Yf[(kb + t4) * 40 + 8 * nt + g8]), to_tf32(Yf[(kb + t4 + 4) * 40 + 8 * nt + g8]));
-            }
-            const int cc = 8 * nt + 2 * t4, r0 = 32 + 16 * mt + g8;
-            const float b0 = sbeta[cc], b1 = sbeta[cc + 1];
-            *reinterpret_cast<uint32_t *>(sm + S::ASOL + sw_chunk(r0, cc >> 3) + (cc & 7) * 2) =
-                pack_f16(-d[0] * b0, -d[1] * b1);
-            *reinterpret_cast<uint32_t *>(sm + S::ASOL + sw_chunk(r0 + 8, cc >> 3) + (cc & 7) * 2) =
-                pack_f16(-d[2] * b0, -d[3] * b1);
-        }
-        fence_proxy_async();  // A and the fp16 v are read by the tensor core
-        intra_sync();
-
-        // ---- 6. MMA2: W = A (exp(G) k) into columns 0-127 (rows 0-63 used), U^T = v^T A^T into 128-191 ----
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t iw = idesc_kind_f16(128, 128, false, false, true);  // A K-major, exp(G) k MN-major
-            const uint32_t iu = idesc_kind_f16(128, 64, false, true, false);   // v^T MN-major, A^T K-major
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // A's rows 64-127 read the next 8 KB of shared memory (unused rows)
-                tc_mma_ss(tmem, sw128_desc(sb + S::ASOL + ks * 32, 16, 1024),
-                          sw128_desc(sb + S::KEXP + ks * 2048, 8192, 1024), iw, ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                tc_mma_ss(tmem + 128, sw128_desc(sb + S::V + ks * 2048, 8192, 1024),
-                          sw128_desc(sb + S::ASOL + ks * 32, 16, 1024), iu, ks > 0);
-            tc_commit(bar_m2);
-        }
-        if (warp == 0 && !mbar_wait_spin(bar_m2, par) && lane == 0) atomicOr(p.err, ERR_PIPE_FULL_WAIT);
-        intra_sync();
-        tc_fence_after();
-        if (more && tid == 0) load_v(nxt);  // v's place is free
-        {  // epilogue: -W (lanes 0-63 = tokens) and U^T (lanes = value rows) into their item images
-            const int qd = warp & 3, ch = warp >> 2;
-            const uint32_t tl = tmem + (static_cast<uint32_t>(32 * qd) << 16);
-            uint32_t r[32];
-            if (qd < 2) {  // -W row i, keys 64 ch .. 64 ch + 63 (K-half ch of the item's [64 tok][128 key] tile)
-                const int i = 32 * qd + lane;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    tc_ld32(tl + 64 * ch + 32 * hh, r);
-                    tc_wait_ld();
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            w[e] = pack_f16(-__uint_as_float(r[8 * c4 + 2 * e]), -__uint_as_float(r[8 * c4 + 2 * e + 1]));
-                        *reinterpret_cast<uint4 *>(sm + S::WST + ch * 8192 + sw_chunk(i, 4 * hh + c4)) =
-                            make_uint4(w[0], w[1], w[2], w[3]);
-                    }
-                }
-            }
-            {  // U^T row vv, tokens 32 ch .. 32 ch + 31
-                const int vv = 32 * qd + lane;
-                tc_ld32(tl + 128 + 32 * ch, r);
-                tc_wait_ld();
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        w[e] = pack_f16(__uint_as_float(r[8 * c4 + 2 * e]), __uint_as_float(r[8 * c4 + 2 * e + 1]));
-                    *reinterpret_cast<uint4 *>(sm + S::UST + sw_chunk(vv, 4 * ch + c4)) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
-        }
-        fence_proxy_async();  // the images are read by the bulk copies
-        tc_fence_before();
-        intra_sync();  // every TMEM read is done before the next MMA1 writes
-        if (tid == 0) {
-            bulk_store(out + ITEM_WN, sb + S::WST, 16384);
-            bulk_store(out + ITEM_U, sb + S::UST, 16384);
-            bulk_commit();
-        }
-        if (!more) break;
-        cur = nxt;
     }
-    if (tid == 0) bulk_wait_read();  // shared memory must outlive the last images' reads
-    if (warp == 0) {
-        tc_fence_after();
-        tc_dealloc(tmem, kIntraTmemCols);
+    float *sbeta = reinterpret_cast<float *>(sm + S::BETA);
+    if (tid < CH) sbeta[tid] = (tid < nvalid) ? p.beta[(row0 + tid) * p.HV + h] : 0.f;
+    if (!mbar_wait(bar, 0)) {
+        atomicOr(p.err, ERR_TMA_WAIT);
+        return;
+    }
+    if (nvalid < CH) {  // zero the padding rows of a partial chunk (q, k, g; v once it has arrived)
+        for (int idx = tid; idx < (CH - nvalid) * 48; idx += 256) {
+            const int r = nvalid + idx / 48, w = idx % 48;  // 16-byte words: q 16, k 16, g 32 (two per step)
+            uint4 *dst;
+            if (w < 32) {
+                const int buf = w / 16, c16 = w % 16;  // q, k: two halves of 8 chunks
+                dst = reinterpret_cast<uint4 *>(sm + buf * 16384 + (c16 >> 3) * 8192 + r * 128 + ((c16 & 7) << 4));
+            } else {
+                dst = reinterpret_cast<uint4 *>(sm + S::G + r * 512 + (w - 32) * 16);
+                dst[16] = make_uint4(0, 0, 0, 0);
+            }
+            *dst = make_uint4(0, 0, 0, 0);
+        }
+    }
+    __syncthreads();
+
+    // ---- 2. normalise q and k (thread = row half) ----
+    {
+        const int r = tid >> 1, half = tid & 1;
+        uint8_t *tile = sm + (r < CH ? S::Q : S::K) + half * 8192 + (r & 63) * 128;
+        const int rs = r & 7;
+        uint4 raw[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) raw[c] = *reinterpret_cast<const uint4 *>(tile + ((c ^ rs) << 4));
+        l2norm_half_row(raw);  // the routine the standalone kda_l2norm_bf16 kernel runs
+#pragma unroll
+        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(tile + ((c ^ rs) << 4)) = raw[c];
+    }
+    __syncthreads();
+
+    // ---- 3. gate factors and operands: warp = (block J, channel half), lane = channel pair ----
+    {
+        const int J = warp & 3, dp = 32 * (warp >> 2) + lane, d0 = 2 * dp;
+        float2 e[16], bb[16];
+        const float2 l2e = make_float2(1.4426950408889634f, 1.4426950408889634f);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const float2 gv = *reinterpret_cast<const float2 *>(sm + S::G + (16 * J + u) * 512 + d0 * 4);
+            const float2 y = mul2(gv, l2e);
+            e[u] = make_float2(ex2_ftz(y.x), ex2_ftz(y.y));
+        }
+        bb[15] = make_float2(1.f, 1.f);
+#pragma unroll
+        for (int u = 14; u >= 0; --u) bb[u] = mul2(bb[u + 1], e[u + 1]);
+#pragma unroll
+        for (int u = 1; u < 16; ++u) e[u] = mul2(e[u - 1], e[u]);  // e -> inclusive running product (base)
+        float2 *ps = reinterpret_cast<float2 *>(sm + S::PS);
+        ps[J * 64 + dp] = e[15];  // block product P_J of this channel pair
+        __syncthreads();          // every g read is done (the G region becomes KEXP / KBB); P visible
+        float2 P[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) P[j] = ps[j * 64 + dp];
+        // E_J = prod_{J'<J} P_J' (gate from the chunk start to the block start), F_J = prod_{J'>J} P_J'
+        const float2 one2 = make_float2(1.f, 1.f);
+        const float2 P01 = mul2(P[0], P[1]), P23 = mul2(P[2], P[3]);
+        const float2 myE = (J == 0) ? one2 : (J == 1) ? P[0] : (J == 2) ? P01 : mul2(P01, P[2]);
+        const float2 myF = (J == 3) ? one2 : (J == 2) ? P[3] : (J == 1) ? P23 : mul2(P[1], P23);
+        const float scale = 0.08838834764831845f;  // 128^-0.5 in float32
+        const float2 s2 = make_float2(scale, scale);
+        if (J == 0) {
+            // per-channel factors of the ten block pairs, as bf16 pairs; c_II = 1/P_I
+            uint32_t *cf = reinterpret_cast<uint32_t *>(sm + S::CF);
+            auto rcp2 = [](float2 a) {
+                return make_float2(__frcp_rn(fmaxf(a.x, 1e-37f)), __frcp_rn(fmaxf(a.y, 1e-37f)));
+            };
+            const float2 cv[10] = {rcp2(P[0]), one2, rcp2(P[1]), P[1], one2, rcp2(P[2]), mul2(P[1], P[2]), P[2], one2,
+                                   rcp2(P[3])};
+#pragma unroll
+            for (int pi = 0; pi < 10; ++pi) cf[pi * 64 + dp] = pack_bf16(cv[pi].x, cv[pi].y);
+            *reinterpret_cast<float2 *>(out + ITEM_GL + d0 * 4) = mul2(P01, P23);
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int i = 16 * J + u;
+            const uint32_t a16 = lh(i, d0);
+            const float2 xk = unpack_bf16(*reinterpret_cast<const uint32_t *>(sm + S::K + a16));
+            const float2 xq = unpack_bf16(*reinterpret_cast<const uint32_t *>(sm + S::Q + a16));
+            const float2 kb = mul2(xk, e[u]);
+            const float2 qb = mul2(xq, mul2(e[u], s2));
+            const float2 kx = mul2(kb, myE);
+            const float2 qg = mul2(qb, myE);
+            const float2 kbb = mul2(xk, bb[u]);
+            const float2 kg = mul2(kbb, myF);
+            *reinterpret_cast<uint32_t *>(sm + S::K + a16) = pack_bf16(kb.x, kb.y);
+            *reinterpret_cast<uint32_t *>(sm + S::Q + a16) = pack_bf16(qb.x, qb.y);
+            *reinterpret_cast<uint32_t *>(sm + S::KEXP + a16) = pack_f16(kx.x, kx.y);
+            *reinterpret_cast<uint32_t *>(sm + S::KBB + a16) = pack_bf16(kbb.x, kbb.y);
+            *reinterpret_cast<uint32_t *>(out + ITEM_QG + a16) = pack_f16(qg.x, qg.y);
+            *reinterpret_cast<uint32_t *>(out + ITEM_KG + a16) = pack_f16(kg.x, kg.y);
+        }
+    }
+    __syncthreads();
+
+    // ---- 4. L and Aqk over the ten lower block pairs x two 8-column tiles (bf16 MMAs).  A warp takes the
+    //         tiles of one row block I and a run of column blocks J, loading its q and k fragments once per
+    //         k-step for all of them; the 20 tiles split 2-2-2-2-3-3-3-3 over the warps:
+    //         warps 0-3: I = 3, J in {0,1} / {2,3};  warps 4-5: I = 2, J in {0,1,2};
+    //         warps 6-7: I = 1, J in {0,1}, then I = 0, J = 0.  nt = warp & 1. ----
+    {
+        const int nt = warp & 1;
+        const int mi = lane >> 3;
+        auto tiles = [&](int I, int J0, int nJ) {
+            const uint32_t *cf = reinterpret_cast<const uint32_t *>(sm + S::CF) + (I * (I + 1) / 2 + J0) * 64;
+            float accL[3][4] = {}, accQ[3][4] = {};
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                uint32_t ak[4], aq[4];
+                const int ar = 16 * I + (mi & 1) * 8 + (lane & 7), ac = 16 * ks + (mi >> 1) * 8;
+                ldsm_x4(sb + S::K + lh(ar, ac), ak[0], ak[1], ak[2], ak[3]);
+                ldsm_x4(sb + S::Q + lh(ar, ac), aq[0], aq[1], aq[2], aq[3]);
+#pragma unroll
+                for (int jj = 0; jj < 3; ++jj) {
+                    if (jj >= nJ) continue;
+                    uint32_t b0, b1;
+                    ldsm_x2(sb + S::KBB + lh(16 * (J0 + jj) + 8 * nt + (lane & 7), 16 * ks + (mi & 1) * 8), b0, b1);
+                    // the pair's per-channel factor scales the key side: b0 holds channels 2t,2t+1, b1 2t+8,2t+9
+                    b0 = hmul2_bf16(b0, cf[jj * 64 + 8 * ks + t4]);
+                    b1 = hmul2_bf16(b1, cf[jj * 64 + 8 * ks + 4 + t4]);
+                    mma_bf16(accL[jj], ak, b0, b1);
+                    mma_bf16(accQ[jj], aq, b0, b1);
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < 3; ++jj) {
+                if (jj >= nJ) continue;
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int i = 16 * I + g8 + 8 * hr;
+                    const int j = 16 * (J0 + jj) + 8 * nt + 2 * t4;
+                    const float bi = sbeta[i];
+                    const float l0 = (j < i) ? bi * accL[jj][2 * hr] : 0.f;
+                    const float l1 = (j + 1 < i) ? bi * accL[jj][2 * hr + 1] : 0.f;
+                    const float q0 = (j <= i) ? accQ[jj][2 * hr] : 0.f;
+                    const float q1 = (j + 1 <= i) ? accQ[jj][2 * hr + 1] : 0.f;
+                    *reinterpret_cast<float2 *>(sm + S::L + swz(i, j * 4, 256)) = make_float2(l0, l1);
+                    *reinterpret_cast<uint32_t *>(out + ITEM_AQK + swz(i, j * 2, 128)) = pack_f16(q0, q1);
+                }
+            }
+        };
+        if (warp < 4) {
+            tiles(3, 2 * (warp >> 1), 2);
+        } else if (warp < 6) {
+            tiles(2, 0, 3);
+        } else {
+            tiles(1, 0, 2);
+            tiles(0, 0, 1);
+        }
+    }
+    // The carry kernel multiplies the whole 64x64 Aqk tile: its six upper 16x16 blocks must be zeros.
+    for (int idx = tid; idx < 6 * 16 * 8; idx += 256) {
+        const int blk = idx >> 7, r = (idx >> 3) & 15, w = idx & 7;  // block, row in block, 4-byte word in block row
+        const int I = (blk < 3) ? 0 : (blk < 5) ? 1 : 2;
+        const int J = (blk < 3) ? blk + 1 : (blk < 5) ? blk - 1 : 3;
+        const int i = 16 * I + r, j = 16 * J + 2 * w;
+        *reinterpret_cast<uint32_t *>(out + ITEM_AQK + swz(i, j * 2, 128)) = 0u;
+    }
+    __syncthreads();
+
+    // ---- 5. A = (I+L)^-1 diag(beta) ----
+    uint8_t *sX = sm + S::X;  // overlays q*base, dead after step 4
+    {  // diagonal blocks: exact float32 forward substitution on all 256 threads.  Thread = (block I, column c,
+       // row group r4 owning rows r4, r4+4, r4+8, r4+12); the four threads of a column are adjacent lanes.
+       // Right-looking: row m, once final, is broadcast to the column's lanes and updates every later row,
+       // each row accumulating its terms in the order m = 0, 1, ...
+        const int I = tid >> 6, c = (tid >> 2) & 15, r4 = tid & 3;
+        const uint8_t *sLb = sm + S::L;
+        float x[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) x[q] = (4 * q + r4 == c) ? 1.f : 0.f;
+#pragma unroll
+        for (int m = 0; m < 15; ++m) {
+            const float xm = __shfl_sync(0xffffffffu, x[m >> 2], (lane & ~3) | (m & 3));
+#pragma unroll
+            for (int q = m >> 2; q < 4; ++q) {
+                const int j = 4 * q + r4;
+                const float l = *reinterpret_cast<const float *>(sLb + swz(16 * I + j, (16 * I + m) * 4, 256));
+                if (j > m) x[q] = __fmaf_rn(-l, xm, x[q]);
+            }
+        }
+        const float bc = sbeta[16 * I + c];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int j = 4 * q + r4;
+            *reinterpret_cast<float *>(sX + swz(16 * I + j, (16 * I + c) * 4, 256)) = x[q];
+            // A = X diag(beta) in fp16, zero above the diagonal (step 6 multiplies whole diagonal blocks)
+            *reinterpret_cast<__half *>(sm + S::A + swz(16 * I + j, (16 * I + c) * 2, 128)) =
+                __float2half_rn(j >= c ? x[q] * bc : 0.f);
+        }
+    }
+    __syncthreads();
+    {  // blocks next to the diagonal (X_10, X_21, X_32); one warp per (block, 8-column tile)
+        float *ts = reinterpret_cast<float *>(sm + S::TS) + warp * 128;
+        if (warp < 6) solve_block(sm + S::L, sX, sm + S::A, sbeta, ts, (warp >> 1) + 1, warp >> 1, warp & 1, lane);
+        __syncthreads();
+    }
+    {  // the rest as 32x32 blocks: with X_A = X[0..31][0..31] and X_B = X[32..63][32..63] now complete,
+       // X[32..63][0..31] = -X_B (L[32..63][0..31] X_A).  Warp = 16x8 output tile, tf32 MMAs; the 16x16
+       // blocks above the diagonal of X_A and X_B are zero and skipped.
+        const int mt = warp >> 2, nt = warp & 3;
+        float *sT = reinterpret_cast<float *>(sm + S::PS);  // [32][40] floats over PS and TS
+        auto Lat = [&](int r, int cc) { return *reinterpret_cast<const float *>(sm + S::L + swz(r, cc * 4, 256)); };
+        auto Xat = [&](int r, int cc) { return *reinterpret_cast<const float *>(sX + swz(r, cc * 4, 256)); };
+        float d[4] = {};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            if (nt >= 2 && ks < 2) continue;  // X_A[0..15][16..31] = 0
+            uint32_t a[4];
+            a[0] = to_tf32(Lat(32 + 16 * mt + g8, 8 * ks + t4));
+            a[1] = to_tf32(Lat(32 + 16 * mt + g8 + 8, 8 * ks + t4));
+            a[2] = to_tf32(Lat(32 + 16 * mt + g8, 8 * ks + t4 + 4));
+            a[3] = to_tf32(Lat(32 + 16 * mt + g8 + 8, 8 * ks + t4 + 4));
+            mma_tf32(d, a, to_tf32(Xat(8 * ks + t4, 8 * nt + g8)), to_tf32(Xat(8 * ks + t4 + 4, 8 * nt + g8)));
+        }
+        *reinterpret_cast<float2 *>(sT + (16 * mt + g8) * 40 + 8 * nt + 2 * t4) = make_float2(d[0], d[1]);
+        *reinterpret_cast<float2 *>(sT + (16 * mt + g8 + 8) * 40 + 8 * nt + 2 * t4) = make_float2(d[2], d[3]);
+        __syncthreads();
+        float e[4] = {};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            if (mt == 0 && ks >= 2) continue;  // X_B[0..15][16..31] = 0
+            uint32_t a[4];
+            a[0] = to_tf32(Xat(32 + 16 * mt + g8, 32 + 8 * ks + t4));
+            a[1] = to_tf32(Xat(32 + 16 * mt + g8 + 8, 32 + 8 * ks + t4));
+            a[2] = to_tf32(Xat(32 + 16 * mt + g8, 32 + 8 * ks + t4 + 4));
+            a[3] = to_tf32(Xat(32 + 16 * mt + g8 + 8, 32 + 8 * ks + t4 + 4));
+            mma_tf32(e, a, to_tf32(sT[(8 * ks + t4) * 40 + 8 * nt + g8]), to_tf32(sT[(8 * ks + t4 + 4) * 40 + 8 * nt + g8]));
+        }
+        // only A = X diag(beta) is needed from here on
+        const int cc = 8 * nt + 2 * t4;
+        const float b0 = sbeta[cc], b1 = sbeta[cc + 1];
+        *reinterpret_cast<uint32_t *>(sm + S::A + swz(32 + 16 * mt + g8, cc * 2, 128)) = pack_f16(-e[0] * b0, -e[1] * b1);
+        *reinterpret_cast<uint32_t *>(sm + S::A + swz(32 + 16 * mt + g8 + 8, cc * 2, 128)) = pack_f16(-e[2] * b0, -e[3] * b1);
+    }
+    __syncthreads();
+
+    // ---- v tile (its copy overlapped steps 2-5): zero padding rows, bf16 -> fp16 in place ----
+    if (!mbar_wait(bar + 8, 0)) {
+        atomicOr(p.err, ERR_TMA_WAIT);
+        return;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int idx = tid + 256 * k;  // 16-byte chunk: half (idx >> 9), row ((idx >> 3) & 63)
+        uint4 *pv = reinterpret_cast<uint4 *>(sm + S::V) + idx;
+        uint4 u = *pv;
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        const bool pad = ((idx >> 3) & 63) >= nvalid;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 x = unpack_bf16(w[j]);
+            w[j] = pad ? 0u : pack_f16(x.x, x.y);
+        }
+        *pv = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __syncthreads();
+
+    // ---- 6. -W = -A (exp(G) k) (warp = 16 key columns) and U^T = v^T A^T (warp = 16 value rows); fp16 MMAs.
+    //         Each 16x16 tile of A is loaded once: as the A operand of W, and, with its fragment registers
+    //         reordered, as the two B fragments (8 rows of A each) of U^T. ----
+    {
+        const int mi = lane >> 3;
+        // U^T A operand: v^T rows 16*warp .. +15 for the four 16-token K steps (ldmatrix.trans of v)
+        uint32_t av[4][4];
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const int tok = 16 * ks + (mi >> 1) * 8 + (lane & 7), col = 16 * warp + (mi & 1) * 8;
+            ldsm_x4_t(sb + S::V + lh(tok, col), av[ks][0], av[ks][1], av[ks][2], av[ks][3]);
+        }
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+            float w[2][4] = {}, u[2][4] = {};
+            for (int ks = 0; ks <= mt; ++ks) {
+                uint32_t a[4];  // A rows 16mt + (g, g+8), columns 16ks + (2t, 2t+8)
+                ldsm_x4(sb + S::A + swz(16 * mt + (mi & 1) * 8 + (lane & 7), (16 * ks + (mi >> 1) * 8) * 2, 128), a[0], a[1],
+                        a[2], a[3]);
+                const int tok = 16 * ks + (mi & 1) * 8 + (lane & 7), col = 16 * warp + (mi >> 1) * 8;
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(sb + S::KEXP + lh(tok, col), b0, b1, b2, b3);
+                mma_f16(w[0], a, b0, b1);
+                mma_f16(w[1], a, b2, b3);
+                // U^T[v][i] += v^T[v][j] A[i][j]: B fragment of rows i = 16mt + g is (a0, a2), of i + 8 is (a1, a3)
+                mma_f16(u[0], av[ks], a[0], a[2]);
+                mma_f16(u[1], av[ks], a[1], a[3]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int r = 16 * mt + g8 + 8 * hr;
+                    const int c = 16 * warp + 8 * nt + 2 * t4;
+                    *reinterpret_cast<uint32_t *>(sm + S::WST + lh(r, c)) = pack_f16(-w[nt][2 * hr], -w[nt][2 * hr + 1]);
+                    const int vr = 16 * warp + g8 + 8 * hr;  // value row
+                    const int tk = 16 * mt + 8 * nt + 2 * t4;  // token column
+                    *reinterpret_cast<uint32_t *>(sm + S::UST + vr * 128 + (((tk >> 3) ^ (vr & 7)) << 4) + (tk & 7) * 2) =
+                        pack_f16(u[nt][2 * hr], u[nt][2 * hr + 1]);
+                }
+        }
+    }
+    // -W and U^T leave through two bulk copies (their smem images match the item layout)
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+        bulk_store(out + ITEM_WN, sb + S::WST, 16384);
+        bulk_store(out + ITEM_U, sb + S::UST, 16384);
+        bulk_commit();
+        bulk_wait_read();  // the shared-memory images must outlive the reads, not the global writes
     }
 }
 

@@ -170,12 +170,8 @@ int carry_segments(int B, int T, int HV, bool varlen, int sms)
     return best;
 }
 
-// The intra-chunk kernel's item counters: one int per launch of a forward (kMaxParts at most), zeroed once per
-// forward.
-constexpr size_t kCounterBytes = 64;
-
 struct Workspace {
-    size_t chunk_off = 0, order = 0, ctr = 0, items = 0, seg = 0, total = 0;
+    size_t chunk_off = 0, order = 0, items = 0, seg = 0, total = 0;
     int64_t max_chunks = 0;
     int segments = 1;
 };
@@ -193,8 +189,6 @@ Workspace workspace_layout(int B, int T, int HV, int num_seqs)
         w.order = off;
         off += round_up(static_cast<size_t>(num_seqs) * 4, kAlign);
     }
-    w.ctr = off;
-    off += kAlign;
     w.items = off;
     off += static_cast<size_t>(w.max_chunks) * HV * kda::ITEM_BYTES;
     w.segments = max_carry_segments(B, T, HV, varlen);
@@ -259,26 +253,6 @@ cudaError_t launch_carry(const kda::CarryParams &p, int units, cudaStream_t stre
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kda::CarrySmem::TOTAL);
     if (err != cudaSuccess) return err;
     kern<<<units, kda::kCarryThreads, kda::CarrySmem::TOTAL, stream>>>(p);
-    return cudaGetLastError();
-}
-
-// The intra-chunk kernel over `items` (chunk, value head) items.  Alone on the GPU it is persistent: two CTAs
-// per SM take their items from `counter` (zero before).  Beside a carry (the previous part's) it runs one item
-// per CTA, so that the block scheduler places the carry CTAs as soon as intra-chunk CTAs exit.
-cudaError_t launch_intra_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                const CUtensorMap &tg, kda::IntraParams ip, int64_t items, int sms, int *counter,
-                                bool beside_carry, cudaStream_t s)
-{
-    if (items <= 0) return cudaSuccess;
-    cudaError_t err = cudaFuncSetAttribute(kda::kda_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           kda::IntraSmem::TOTAL);
-    if (err != cudaSuccess) return err;
-    const int64_t slots = static_cast<int64_t>(sms) * kda::kIntraCtasPerSm;
-    ip.counter = beside_carry ? nullptr : counter;
-    ip.n_items = static_cast<int>(items);
-    ip.prefetch_stride = static_cast<int>(slots);
-    const int64_t grid = beside_carry || items < slots ? items : slots;
-    kda::kda_intra_kernel<<<static_cast<int>(grid), 256, kda::IntraSmem::TOTAL, s>>>(tq, tk, tv, tg, ip);
     return cudaGetLastError();
 }
 
@@ -391,8 +365,6 @@ kda_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     int32_t *chunk_off = varlen ? reinterpret_cast<int32_t *>(wsb + ws.chunk_off) : nullptr;
     int32_t *order = varlen ? reinterpret_cast<int32_t *>(wsb + ws.order) : nullptr;
     uint8_t *items = wsb + ws.items;
-    int *counters = reinterpret_cast<int *>(wsb + ws.ctr);
-    if (tokens > 0 && cudaMemsetAsync(counters, 0, kCounterBytes, s) != cudaSuccess) return KDA_ERR_CUDA;
 
     if (varlen) {
         kda::chunk_offsets_kernel<<<1, 1024, 0, s>>>(cu_seqlens, num_seqs, chunk_off);
@@ -409,7 +381,6 @@ kda_status_t forward_impl(const void *q, const void *k, const void *v, const flo
             !make_map(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, HV, rows, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map(&tg, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, HV, rows, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
             return KDA_ERR_CUDA;
-        ip.g = g;
         ip.beta = beta;
         ip.cu = cu_seqlens;
         ip.chunk_off = chunk_off;
@@ -421,12 +392,17 @@ kda_status_t forward_impl(const void *q, const void *k, const void *v, const flo
         ip.HV = HV;
         ip.N = d.N;
         ip.chunks_per_seq = (T + CH - 1) / CH;
+        ip.prefetch_stride = info.sms * kda::kIntraCtasPerSm;
+        if (cudaFuncSetAttribute(kda::kda_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kda::IntraSmem::TOTAL) != cudaSuccess)
+            return KDA_ERR_CUDA;
     }
-    // launch j of this forward (j > 0: beside the carry of part j - 1)
-    auto launch_intra = [&](int chunk_begin, int chunk_count, int64_t grid_chunks, int j) {
+    auto launch_intra = [&](int chunk_begin, int chunk_count, int64_t grid_chunks) {
         ip.chunk_begin = chunk_begin;
         ip.chunk_count = chunk_count;
-        return launch_intra_kernel(tq, tk, tv, tg, ip, grid_chunks * HV, info.sms, counters + j, j > 0, s);
+        kda::kda_intra_kernel<<<static_cast<int>(grid_chunks * HV), 256, kda::IntraSmem::TOTAL, s>>>(tq, tk, tv, tg,
+                                                                                                      ip);
+        return cudaGetLastError();
     };
 
     kda::CarryParams cp{};
@@ -446,7 +422,7 @@ kda_status_t forward_impl(const void *q, const void *k, const void *v, const flo
 
     const int segments = ws.segments > 1 ? carry_segments(B, T, HV, varlen, info.sms) : 1;
     if (segments > 1) {
-        if (launch_intra(0, cp.chunks_per_seq, ws.max_chunks, 0) != cudaSuccess) return KDA_ERR_CUDA;
+        if (launch_intra(0, cp.chunks_per_seq, ws.max_chunks) != cudaSuccess) return KDA_ERR_CUDA;
         const int units = d.N * HV;
         float *seg = reinterpret_cast<float *>(wsb + ws.seg);
         const size_t per = static_cast<size_t>(units) * ws.segments * DK * DV;  // reserved for the maximum count
@@ -464,7 +440,7 @@ kda_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     }
     const int parts = pipeline_parts(B, T, HV, varlen, info.sms);
     if (parts == 1) {
-        if (tokens > 0 && launch_intra(0, cp.chunks_per_seq, ws.max_chunks, 0) != cudaSuccess) return KDA_ERR_CUDA;
+        if (tokens > 0 && launch_intra(0, cp.chunks_per_seq, ws.max_chunks) != cudaSuccess) return KDA_ERR_CUDA;
         cp.chunk_begin = 0;
         cp.chunk_count = cp.chunks_per_seq;
         return launch_carry(cp, d.N * HV, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
@@ -480,7 +456,7 @@ kda_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     for (int j = 0; j < parts; ++j) {
         const int c0 = static_cast<int>(static_cast<int64_t>(nck) * 4 * j / den);
         const int c1 = j + 1 == parts ? nck : static_cast<int>(static_cast<int64_t>(nck) * 4 * (j + 1) / den);
-        if (launch_intra(c0, c1 - c0, static_cast<int64_t>(B) * (c1 - c0), j) != cudaSuccess) return KDA_ERR_CUDA;
+        if (launch_intra(c0, c1 - c0, static_cast<int64_t>(B) * (c1 - c0)) != cudaSuccess) return KDA_ERR_CUDA;
         if (cudaEventRecord(lane->fork, s) != cudaSuccess || cudaStreamWaitEvent(lane->stream, lane->fork, 0) != cudaSuccess)
             return KDA_ERR_CUDA;
         cp.s0 = j == 0 ? initial_state : final_state;

@@ -23,24 +23,6 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn_major)
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Instruction descriptor, kind::f16 with a choice of element type (fp16 or bf16 for both operands, which must
-// agree) and of each operand's major-ness (MN-major = the M (or N) index is the contiguous one).
-__host__ __device__ constexpr uint32_t idesc_kind_f16(int M, int N, bool bf16, bool a_mn_major, bool b_mn_major)
-{
-    return (1u << 4) | (bf16 ? (1u << 7) | (1u << 10) : 0u) | (a_mn_major ? (1u << 15) : 0u) |
-           (b_mn_major ? (1u << 16) : 0u) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
-}
-
-// D[tmem] (+)= A[smem desc] * B[smem desc], issued by the calling thread alone; accumulate != 0 keeps D.
-__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate)
-{
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-
 // D[tmem] (+)= A[tmem] * B[smem desc]; accumulate != 0 keeps D.
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate)

@@ -43,13 +43,12 @@ def test_status_strings(L):
 
 def test_workspace_size(L):
     item = 74240
-    ctr = 256  # the intra-chunk kernel's item counters
-    # plain batch: the counters, then B * ceil(T/64) chunks x HV heads of item blocks
-    assert L.kda_prefill_workspace_size(2, 4096, 96, 96, 128, 128, 0) == ctr + 2 * 64 * 96 * item
-    assert L.kda_prefill_workspace_size(1, 1000, 4, 4, 128, 128, 0) == ctr + 16 * 4 * item
-    # packed batch: offsets and order, the counters, then (ceil(T/64) + N) chunks as an upper bound
+    # plain batch: B * ceil(T/64) chunks x HV heads of item blocks
+    assert L.kda_prefill_workspace_size(2, 4096, 96, 96, 128, 128, 0) == 2 * 64 * 96 * item
+    assert L.kda_prefill_workspace_size(1, 1000, 4, 4, 128, 128, 0) == 16 * 4 * item
+    # packed batch: offsets and order, then (ceil(T/64) + N) chunks as an upper bound
     n = L.kda_prefill_workspace_size(1, 11210, 8, 32, 128, 128, 7)
-    assert n == 256 + 256 + ctr + (176 + 7) * 32 * item
+    assert n == 256 + 256 + (176 + 7) * 32 * item
     # rejected sizes
     assert L.kda_prefill_workspace_size(1, 64, 1, 1, 64, 128, 0) == 0
     assert L.kda_prefill_workspace_size(1, 64, 2, 3, 128, 128, 0) == 0
