@@ -138,8 +138,15 @@ size_t kda_prefill_host_staging_size(int B, int T, int H, int HV, int K, int V, 
  * The same forward on HOST buffers (same shapes and dtypes as above; pinned
  * memory makes the copies asynchronous).  Inputs are copied into the
  * caller's device staging buffer, the forward runs there, and o and
- * final_state are copied back -- all enqueued on `stream`; the caller
- * synchronises before reading o_host / final_state_host.
+ * final_state are copied back -- all ordered after `stream`'s earlier work
+ * and before its later work; the caller synchronises before reading
+ * o_host / final_state_host.  Where the forward cuts a plain batch into
+ * parts (see kda_prefill_kernel_launches), each part's input rows are
+ * uploaded on a copy stream of the library while the earlier parts compute,
+ * and each part's o rows are downloaded as soon as its carry has run, so
+ * the two copy directions overlap; the results equal kda_prefill_forward's
+ * bit for bit.  Calls on one device are serialised by the library while
+ * they enqueue (the copy streams are shared).
  */
 kda_status_t kda_prefill_forward_host(const void *q_host, const void *k_host, const void *v_host,
                                       const float *g_host, const float *beta_host,

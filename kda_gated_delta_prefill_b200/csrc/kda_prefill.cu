@@ -222,6 +222,10 @@ struct CarryLane {
     bool ready = false;
     cudaStream_t stream = nullptr;
     cudaEvent_t fork = nullptr, join = nullptr;
+    // the host-buffer forward: an upload stream (inputs, part by part), a download stream (o, part by part)
+    bool io_ready = false;
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t start = nullptr, down_done = nullptr, up_done[8] = {}, part_done[8] = {};
     std::mutex mu;
 };
 CarryLane g_lane[kMaxDevices];
@@ -245,6 +249,50 @@ cudaError_t carry_lane(int dev, CarryLane *&out)
     }
     out = &l;
     return cudaSuccess;
+}
+
+static_assert(kMaxParts <= 8, "a lane holds one upload and one download event per part");
+
+// The host-buffer forward's copy streams and events of a lane, created on first use.
+cudaError_t host_io_lane(CarryLane &l)
+{
+    std::lock_guard<std::mutex> lock(g_lane_mu);
+    if (l.io_ready) return cudaSuccess;
+    cudaError_t e = cudaStreamCreateWithFlags(&l.up, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&l.down, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&l.start, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&l.down_done, cudaEventDisableTiming);
+    for (int j = 0; j < 8 && e == cudaSuccess; ++j) {
+        e = cudaEventCreateWithFlags(&l.up_done[j], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&l.part_done[j], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) l.io_ready = true;
+    return e;
+}
+
+// Host buffers of the host-buffer forward when it runs part by part: each part's input rows are uploaded on
+// their own stream while the previous parts compute, and each part's o rows are downloaded as soon as its
+// carry has run, so the two copy directions overlap each other and the kernels.
+struct HostIO {
+    const void *src[5];     // q, k, v, g, beta on the host ([B, T, heads, width] rows)
+    void *dst[5];           // their device copies (the same layout)
+    size_t row_bytes[5];    // bytes of one token row of each
+    const float *s0_host;   // initial state on the host, or null
+    float *s0_dev;          // its device copy
+    void *o_host;           // o on the host
+    size_t o_row_bytes;
+    float *sN_host;         // final state on the host
+    size_t state_bytes;
+};
+
+// Rows [t0, t1) of every batch row of a [B, T, ...] tensor: one strided copy.
+cudaError_t copy_rows(void *dst, const void *src, size_t row_bytes, int B, int T, int t0, int t1, cudaMemcpyKind kind,
+                      cudaStream_t st)
+{
+    if (t1 <= t0 || B <= 0) return cudaSuccess;
+    const size_t pitch = static_cast<size_t>(T) * row_bytes, off = static_cast<size_t>(t0) * row_bytes;
+    return cudaMemcpy2DAsync(static_cast<char *>(dst) + off, pitch, static_cast<const char *>(src) + off, pitch,
+                             static_cast<size_t>(t1 - t0) * row_bytes, B, kind, st);
 }
 
 cudaError_t launch_carry(const kda::CarryParams &p, int units, cudaStream_t stream)
@@ -306,7 +354,7 @@ namespace {
 kda_status_t forward_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
                           const float *initial_state, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H,
                           int HV, int K, int V, void *o, float *final_state, void *workspace, size_t workspace_bytes,
-                          void *stream, __nv_bfloat16 *states);
+                          void *stream, __nv_bfloat16 *states, const HostIO *hio = nullptr);
 }  // namespace
 
 extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const void *v, const float *g,
@@ -323,7 +371,7 @@ namespace {
 kda_status_t forward_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
                           const float *initial_state, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H,
                           int HV, int K, int V, void *o, float *final_state, void *workspace, size_t workspace_bytes,
-                          void *stream, __nv_bfloat16 *states)
+                          void *stream, __nv_bfloat16 *states, const HostIO *hio)
 {
     Dims d;
     const bool varlen = cu_seqlens != nullptr;
@@ -439,6 +487,7 @@ kda_status_t forward_impl(const void *q, const void *k, const void *v, const flo
         return launch_carry(cp, units * segments, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     }
     const int parts = pipeline_parts(B, T, HV, varlen, info.sms);
+    if (hio && parts == 1) return KDA_ERR_INVALID_ARG;  // the host-buffer forward copies part by part only here
     if (parts == 1) {
         if (tokens > 0 && launch_intra(0, cp.chunks_per_seq, ws.max_chunks) != cudaSuccess) return KDA_ERR_CUDA;
         cp.chunk_begin = 0;
@@ -453,9 +502,27 @@ kda_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     // part j starts at chunk nck * 4j / (4 parts - 3).
     const int nck = cp.chunks_per_seq;
     const int64_t den = 4 * parts - 3;
+    auto chunk_at = [&](int j) { return j >= parts ? nck : static_cast<int>(static_cast<int64_t>(nck) * 4 * j / den); };
+    auto tok = [&](int c) { return c * CH < T ? c * CH : T; };
+    if (hio) {  // uploads: the initial state, then every part's rows, in order, after the stream's earlier work
+        if (host_io_lane(*lane) != cudaSuccess || cudaEventRecord(lane->start, s) != cudaSuccess ||
+            cudaStreamWaitEvent(lane->up, lane->start, 0) != cudaSuccess ||
+            cudaStreamWaitEvent(lane->down, lane->start, 0) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        if (hio->s0_host && cudaMemcpyAsync(hio->s0_dev, hio->s0_host, hio->state_bytes, cudaMemcpyHostToDevice,
+                                            lane->up) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        for (int j = 0; j < parts; ++j) {
+            for (int t = 0; t < 5; ++t)
+                if (copy_rows(hio->dst[t], hio->src[t], hio->row_bytes[t], B, T, tok(chunk_at(j)), tok(chunk_at(j + 1)),
+                              cudaMemcpyHostToDevice, lane->up) != cudaSuccess)
+                    return KDA_ERR_CUDA;
+            if (cudaEventRecord(lane->up_done[j], lane->up) != cudaSuccess) return KDA_ERR_CUDA;
+        }
+    }
     for (int j = 0; j < parts; ++j) {
-        const int c0 = static_cast<int>(static_cast<int64_t>(nck) * 4 * j / den);
-        const int c1 = j + 1 == parts ? nck : static_cast<int>(static_cast<int64_t>(nck) * 4 * (j + 1) / den);
+        const int c0 = chunk_at(j), c1 = chunk_at(j + 1);
+        if (hio && cudaStreamWaitEvent(s, lane->up_done[j], 0) != cudaSuccess) return KDA_ERR_CUDA;
         if (launch_intra(c0, c1 - c0, static_cast<int64_t>(B) * (c1 - c0)) != cudaSuccess) return KDA_ERR_CUDA;
         if (cudaEventRecord(lane->fork, s) != cudaSuccess || cudaStreamWaitEvent(lane->stream, lane->fork, 0) != cudaSuccess)
             return KDA_ERR_CUDA;
@@ -463,9 +530,23 @@ kda_status_t forward_impl(const void *q, const void *k, const void *v, const flo
         cp.chunk_begin = c0;
         cp.chunk_count = c1 - c0;
         if (launch_carry(cp, d.N * HV, lane->stream) != cudaSuccess) return KDA_ERR_CUDA;
+        if (hio) {  // this part's o rows are final: download them beside the next parts
+            if (cudaEventRecord(lane->part_done[j], lane->stream) != cudaSuccess ||
+                cudaStreamWaitEvent(lane->down, lane->part_done[j], 0) != cudaSuccess ||
+                copy_rows(hio->o_host, o, hio->o_row_bytes, B, T, tok(c0), tok(c1), cudaMemcpyDeviceToHost,
+                          lane->down) != cudaSuccess)
+                return KDA_ERR_CUDA;
+        }
     }
     if (cudaEventRecord(lane->join, lane->stream) != cudaSuccess || cudaStreamWaitEvent(s, lane->join, 0) != cudaSuccess)
         return KDA_ERR_CUDA;
+    if (hio) {  // the final state after the last carry, then the caller's stream waits for every download
+        if (cudaMemcpyAsync(hio->sN_host, final_state, hio->state_bytes, cudaMemcpyDeviceToHost, lane->down) !=
+                cudaSuccess ||
+            cudaEventRecord(lane->down_done, lane->down) != cudaSuccess ||
+            cudaStreamWaitEvent(s, lane->down_done, 0) != cudaSuccess)
+            return KDA_ERR_CUDA;
+    }
     return KDA_OK;
 }
 }  // namespace
@@ -521,6 +602,32 @@ extern "C" kda_status_t kda_prefill_forward_host(const void *q_h, const void *k_
     char *dws = ws ? take(ws) : nullptr;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // A plain batch that the forward cuts into parts: uploads and downloads part by part beside the kernels.
+    DeviceInfo info;
+    if (device_info(info) != cudaSuccess) return KDA_ERR_CUDA;
+    if (!varlen && tokens > 0 && carry_segments(B, T, HV, false, info.sms) == 1 &&
+        pipeline_parts(B, T, HV, false, info.sms) > 1) {
+        HostIO io{};
+        const void *srcs[5] = {q_h, k_h, v_h, g_h, beta_h};
+        void *dsts[5] = {dq, dk, dv, dg, db};
+        const size_t rows[5] = {static_cast<size_t>(H) * K * 2, static_cast<size_t>(H) * K * 2,
+                                static_cast<size_t>(HV) * V * 2, static_cast<size_t>(HV) * K * 4,
+                                static_cast<size_t>(HV) * 4};
+        for (int t = 0; t < 5; ++t) {
+            io.src[t] = srcs[t];
+            io.dst[t] = dsts[t];
+            io.row_bytes[t] = rows[t];
+        }
+        io.s0_host = s0_h;
+        io.s0_dev = reinterpret_cast<float *>(ds0);
+        io.o_host = o_h;
+        io.o_row_bytes = static_cast<size_t>(HV) * V * 2;
+        io.sN_host = sN_h;
+        io.state_bytes = ns;
+        return forward_impl(dq, dk, dv, reinterpret_cast<float *>(dg), reinterpret_cast<float *>(db),
+                            reinterpret_cast<float *>(ds0), nullptr, 0, B, T, H, HV, K, V, dO,
+                            reinterpret_cast<float *>(dsN), dws, ws, stream, nullptr, &io);
+    }
     struct Cp {
         void *dst;
         const void *src;

@@ -231,6 +231,27 @@ def test_host_entry_point_matches_device_entry_point():
     assert torch.equal(o_h, o_dev.cpu()) and torch.equal(s_h, s_dev.cpu())
 
 
+@pytest.mark.parametrize("B,T,H,HV,state", [(1, 2088, 8, 24, "n01"), (2, 2600, 2, 4, "n01"), (2, 2600, 2, 4, "none")])
+def test_host_entry_point_part_by_part(B, T, H, HV, state):
+    # Plain batches that the forward cuts into parts: the host-buffer entry point uploads and downloads each
+    # part's rows beside the kernels (strided copies when B > 1); the results equal the device entry point's.
+    import kda_gated_delta_prefill_b200 as kda
+    case = gen.Case(f"host_parts{B}_{T}", B=B, T=T, H=H, HV=HV, state=state, seed=350 + B + T)
+    assert kda.kernel_launches(B, T, H, HV) > 2  # cut into parts
+    x = gen.make_inputs(case)
+    o_dev, s_dev = gpu_forward(x)
+    staging = torch.empty(kda.host_staging_size(B, T, H, HV, has_initial_state=x["initial_state"] is not None),
+                          dtype=torch.uint8, device="cuda")
+    pin = {k: (v.pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    o_h = torch.full((B, T, HV, 128), float("nan"), dtype=torch.bfloat16).pin_memory()
+    s_h = torch.full((case.N, HV, 128, 128), float("nan")).pin_memory()
+    for _ in range(2):  # twice: the second call reuses the copy streams and the staging buffer
+        kda.forward_host(pin["q"], pin["k"], pin["v"], pin["g"], pin["beta"], pin["initial_state"], None,
+                         o=o_h, final_state=s_h, staging=staging)
+        torch.cuda.synchronize()
+        assert torch.equal(o_h, o_dev.cpu()) and torch.equal(s_h, s_dev.cpu())
+
+
 def test_repeat_calls_are_deterministic():
     x = gen.make_inputs(gen.TAIL_STATE)
     o1, s1 = gpu_forward(x)
