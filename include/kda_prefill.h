@@ -102,12 +102,13 @@ size_t kda_prefill_workspace_size(int B, int T, int H, int HV, int K, int V, int
  * (sequence, value head) pairs than the device has SMs and at least 32
  * chunks per sequence is run as up to 8 consecutive parts of the sequence
  * (whole chunks): the state carry of each part runs on a high-priority side
- * stream that the library creates once per device, overlapping the
- * intra-chunk work of the next part, and joins `stream` again through an
- * event before the call returns, so the caller sees one ordered operation
- * (under stream capture the side stream becomes a fork and join of the
- * captured graph).  Calls from several host threads on one device share that
- * side stream, so their carry parts run one after another.
+ * stream of the library, overlapping the intra-chunk work of the next part,
+ * and joins `stream` again through an event before the call returns, so the
+ * caller sees one ordered operation (under stream capture the side stream
+ * becomes a fork and join of the captured graph).  The library keeps four
+ * such side streams per device and a call takes a free one, so calls that
+ * host threads make at the same time get different side streams (a fifth
+ * concurrent call waits on the host for the first to finish enqueueing).
  *
  * A plain batch with few units (B * HV <= 48) and long sequences may
  * instead carry S segments of every sequence at once: the segments' linear

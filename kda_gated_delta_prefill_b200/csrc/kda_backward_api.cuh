@@ -232,8 +232,7 @@ kda_status_t backward_impl(const void *q, const void *k, const void *v, const fl
     CarryLane *lane = nullptr;
     std::unique_lock<std::mutex> lane_lock;
     if (recompute) {
-        if (carry_lane(info.dev, lane) != cudaSuccess) return KDA_ERR_CUDA;
-        lane_lock = std::unique_lock<std::mutex>(lane->mu);
+        if (carry_lane(info.dev, lane, lane_lock) != cudaSuccess) return KDA_ERR_CUDA;
         const int parts = tokens > 0 ? pipeline_parts(B, T, HV, varlen, info.sms) : 1;
         const int nck = cp.chunks_per_seq;
         const int64_t den = 4 * parts - 3;  // the last part a quarter of the others, as in the forward

@@ -216,8 +216,10 @@ int pipeline_parts(int B, int T, int HV, bool varlen, int sms)
     return parts < 2 ? 1 : (parts < kMaxParts ? parts : kMaxParts);
 }
 
-// The side stream and the fork/join events of one device, created on first use.  The mutex keeps one
-// forward's launches and event records together when several host threads share the device.
+// A lane: a side stream for the carry and its fork/join events, created on first use.  A forward that cuts its
+// sequence into parts holds one lane (its mutex) while it enqueues, so that one forward's launches and event
+// records stay together.  Each device has several lanes and a call takes a free one, so forwards that host
+// threads issue at the same time on different streams get different side streams and their carries overlap.
 struct CarryLane {
     bool ready = false;
     cudaStream_t stream = nullptr;
@@ -228,13 +230,27 @@ struct CarryLane {
     cudaEvent_t start = nullptr, down_done = nullptr, up_done[8] = {}, part_done[8] = {};
     std::mutex mu;
 };
-CarryLane g_lane[kMaxDevices];
+constexpr int kLanesPerDevice = 4;
+CarryLane g_lane[kMaxDevices][kLanesPerDevice];
 std::mutex g_lane_mu;
 
-cudaError_t carry_lane(int dev, CarryLane *&out)
+// Takes a lane of device `dev` (a free one if any, else waits for the first) and returns it locked.
+cudaError_t carry_lane(int dev, CarryLane *&out, std::unique_lock<std::mutex> &held)
 {
+    CarryLane *pick = nullptr;
+    for (int i = 0; i < kLanesPerDevice && !pick; ++i) {
+        std::unique_lock<std::mutex> trial(g_lane[dev][i].mu, std::try_to_lock);
+        if (trial.owns_lock()) {
+            pick = &g_lane[dev][i];
+            held = std::move(trial);
+        }
+    }
+    if (!pick) {
+        pick = &g_lane[dev][0];
+        held = std::unique_lock<std::mutex>(pick->mu);
+    }
     std::lock_guard<std::mutex> lock(g_lane_mu);
-    CarryLane &l = g_lane[dev];
+    CarryLane &l = *pick;
     if (!l.ready) {
         int least = 0, greatest = 0;
         cudaError_t e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
@@ -496,8 +512,8 @@ kda_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     }
 
     CarryLane *lane = nullptr;
-    if (carry_lane(info.dev, lane) != cudaSuccess) return KDA_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(lane->mu);
+    std::unique_lock<std::mutex> lane_lock;
+    if (carry_lane(info.dev, lane, lane_lock) != cudaSuccess) return KDA_ERR_CUDA;
     // The last part's carry has nothing left to overlap with, so it is a quarter of the size of the others:
     // part j starts at chunk nck * 4j / (4 parts - 3).
     const int nck = cp.chunks_per_seq;

@@ -313,6 +313,41 @@ def test_parts_on_a_non_default_stream():
     compare(o, s, ref)
 
 
+def test_parts_from_concurrent_host_threads():
+    # Forwards cut into parts, issued at the same time from several host threads on their own streams: each
+    # takes its own side stream (or waits for one) and must equal the single-threaded result bit for bit.
+    import threading
+    import kda_gated_delta_prefill_b200 as kda
+    case = gen.Case("parts_threads", B=1, T=2600, H=4, HV=8, state="n01", seed=361)
+    x = to_cuda(gen.make_inputs(case))
+    assert kda.kernel_launches(1, case.T, case.H, case.HV) > 2
+    o_ref, s_ref = kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"])
+    torch.cuda.synchronize()
+    results, errors = [None] * 6, []
+
+    def run(i):
+        try:
+            st = torch.cuda.Stream()
+            st.wait_stream(torch.cuda.default_stream())
+            with torch.cuda.stream(st):
+                outs = [kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"]) for _ in range(3)]
+            st.synchronize()
+            results[i] = outs
+        except Exception as e:  # reported below
+            errors.append(repr(e))
+
+    threads = [threading.Thread(target=run, args=(i,)) for i in range(6)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    for outs in results:
+        for o, s in outs:
+            assert torch.equal(o, o_ref) and torch.equal(s, s_ref)
+    assert kda.device_error(clear=True) == 0
+
+
 def test_parts_repeatable_under_load():
     # The carry of each part runs beside the next part's intra-chunk kernel.  Repeated calls must agree bit for
     # bit with the uncut run and leave the device error word clear: a pipeline wait that gave up (for
