@@ -457,3 +457,51 @@ def test_bf16_state_forward(B, T, H, HV, varlen):
     kda.forward_state_bf16(c(q), c(k), c(v), c(g), c(beta), s_io, c(cu), final_state=s_io)
     torch.cuda.synchronize()
     assert torch.equal(s_io.cpu(), sN.cpu())
+
+
+# ------------------------------------------------------------------ CUDA graphs
+# The library allocates nothing and never synchronises, so a forward can be captured in a CUDA graph and
+# replayed; the side stream of a sequence cut into parts becomes a fork and a join inside the graph.
+
+@pytest.mark.parametrize("B,T,H,HV,lengths", [(1, 2600, 4, 8, None),      # cut into parts (side stream)
+                                              (1, 5120, 2, 2, None),      # segmented carry
+                                              (1, 1300, 2, 4, [700, 0, 64, 536]),  # packed sequences
+                                              (2, 300, 2, 4, None)],      # plain, uncut
+                         ids=["parts", "segmented", "packed", "plain"])
+def test_forward_captured_in_a_cuda_graph(B, T, H, HV, lengths):
+    import kda_gated_delta_prefill_b200 as kda
+    cases = [gen.Case(f"graph{i}", B=B, T=T, H=H, HV=HV, lengths=lengths, state="n01", seed=500 + 7 * i + T)
+             for i in range(2)]
+    xs = [to_cuda(gen.make_inputs(c)) for c in cases]
+    N = cases[0].N
+    num_seqs = N if lengths is not None else 0
+    buf = {k: v.clone() for k, v in xs[0].items() if isinstance(v, torch.Tensor)}
+    ws = torch.empty(kda.workspace_size(B, T, H, HV, 128, 128, num_seqs), dtype=torch.uint8, device="cuda")
+    o = torch.empty(B, T, HV, 128, dtype=torch.bfloat16, device="cuda")
+    s = torch.empty(N, HV, 128, 128, device="cuda")
+
+    def call():
+        kda.forward(buf["q"], buf["k"], buf["v"], buf["g"], buf["beta"], buf["initial_state"], buf.get("cu_seqlens"),
+                    o=o, final_state=s, workspace=ws)
+
+    call()  # eager warm-up before the capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    for x in xs:  # replay on new inputs copied into the captured buffers
+        for k, t in buf.items():
+            t.copy_(x[k])
+        o.fill_(float("nan"))
+        s.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        o_ref, s_ref = kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"], x["cu_seqlens"])
+        torch.cuda.synchronize()
+        if lengths is None:
+            assert torch.equal(o, o_ref)
+        else:  # rows outside every packed sequence are not written; here the sequences cover all rows
+            assert torch.equal(o[:, :sum(lengths)], o_ref[:, :sum(lengths)])
+        assert torch.equal(s, s_ref)
+    del graph
+    assert kda.device_error(clear=True) == 0
