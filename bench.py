@@ -696,6 +696,10 @@ def main():
     o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=dev)
     s = torch.empty(N, HV, K, V, dtype=torch.float32, device=dev)
     num_seqs = N if x["cu_seqlens"] is not None else 0
+    # packed batches: the host copy of the boundaries lets the library overlap the carry (chunk windows)
+    cu_host = gen.cu_seqlens_of(case.lengths) if case.lengths is not None else None
+    if cu_host is not None:
+        config["cu_seqlens_host"] = True
     stream = torch.cuda.current_stream(dev)
     if args.saved:  # the forward that also keeps what the backward needs
         ws = torch.empty(max(kda.backward_workspace_size(B, T, H, HV, K, V, num_seqs), 1), dtype=torch.uint8,
@@ -710,7 +714,7 @@ def main():
 
         def step():
             kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"], x["cu_seqlens"], o=o,
-                        final_state=s, workspace=ws, stream=stream)
+                        final_state=s, workspace=ws, stream=stream, cu_seqlens_host=cu_host)
 
     for _ in range(args.warmup):
         step()
@@ -804,9 +808,13 @@ def main():
         cb = time_oracle(case)
         cpu = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
 
-    # intra-chunk and carry kernels per part of the sequence (+ chunk-offset and order kernels for packed batches)
-    launches_per_step = kda.kernel_launches(case.B, case.T, case.H, case.HV, case.K, case.V,
-                                            len(case.lengths) if case.lengths is not None else 0)
+    # intra-chunk and carry kernels per part of the sequence (+ chunk-offset, order and window-offset kernels for
+    # packed batches)
+    if cu_host is not None and not args.saved:
+        launches_per_step = kda.varlen_kernel_launches(case.T, case.H, case.HV, cu_host, case.K, case.V)
+    else:
+        launches_per_step = kda.kernel_launches(case.B, case.T, case.H, case.HV, case.K, case.V,
+                                                len(case.lengths) if case.lengths is not None else 0)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,

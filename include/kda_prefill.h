@@ -69,8 +69,9 @@ const char *kda_status_string(kda_status_t status);
  * num_seqs is the number of packed sequences when cu_seqlens is used, or 0
  * for a plain [B, T] batch.  The workspace holds, per (64-token chunk, value
  * head), the chunk's state-independent results that the intra-chunk kernel
- * hands to the carry kernel (72.5 KiB each), plus the chunk offsets and the
- * longest-first order of packed sequences, and, for plain batches of few long
+ * hands to the carry kernel (72.5 KiB each), plus the chunk offsets, the
+ * longest-first order and the chunk-window offsets (4 x (N + 1) int32) of
+ * packed sequences, and, for plain batches of few long
  * sequences, room for the segmented carry's states (3 x B x HV x S x 64 KiB,
  * S as described at kda_prefill_forward).  Returns 0 for sizes that
  * kda_prefill_forward would reject.
@@ -129,6 +130,46 @@ kda_status_t kda_prefill_forward(const void *q, const void *k, const void *v,
                                  void *stream);
 
 /*
+ * kda_prefill_forward on a packed batch whose sequence boundaries the caller
+ * also holds on the host (the page's packed-sequence contract, "Function and
+ * tensor contract": sequence n is tokens [cu[n], cu[n+1]) with its own
+ * state).  Same arguments as kda_prefill_forward with B = 1, plus:
+ *   cu_seqlens_host  int32 [num_seqs + 1] in host memory holding the same
+ *                    values as cu_seqlens; read during the call only.  It
+ *                    must start at 0, end at T and not decrease, else
+ *                    KDA_ERR_INVALID_ARG.
+ * Knowing the lengths, the library can overlap the state carry with the
+ * intra-chunk work.  This happens when the longest sequence has at least 32
+ * chunks, and the (sequence, value head) pairs of the sequences longer than
+ * the first window are fewer than the device's SMs.  The batch is then cut
+ * into up to 4 windows of chunk index within each sequence (the longest
+ * sequence's chunks in equal windows but the last, which is a quarter of
+ * the others).  The state carry of window j (every sequence with chunks in
+ * it, longest first) runs beside the intra-chunk work of window j+1: that
+ * intra-chunk kernel is a programmatic dependent launch of the carry, which
+ * lets it start once every carry CTA is resident.  Everything stays on
+ * `stream`.  Otherwise the call runs exactly as kda_prefill_forward.  Either
+ * way the results are bit-identical to kda_prefill_forward's.  Workspace:
+ * kda_prefill_workspace_size(1, T, H, HV, K, V, num_seqs).
+ */
+kda_status_t kda_prefill_forward_varlen(const void *q, const void *k, const void *v,
+                                        const float *g, const float *beta,
+                                        const float *initial_state,
+                                        const int32_t *cu_seqlens,
+                                        const int32_t *cu_seqlens_host, int num_seqs,
+                                        int T, int H, int HV, int K, int V,
+                                        void *o, float *final_state,
+                                        void *workspace, size_t workspace_bytes,
+                                        void *stream);
+
+/*
+ * Kernel launches kda_prefill_forward_varlen makes for these lengths on the
+ * current device (0 if it would reject them).
+ */
+int kda_prefill_varlen_kernel_launches(int T, int H, int HV, int K, int V, int num_seqs,
+                                       const int32_t *cu_seqlens_host);
+
+/*
  * Bytes of device staging memory kda_prefill_forward_host needs: room for
  * every input and output plus the workspace, each 256-byte aligned.
  */
@@ -146,7 +187,9 @@ size_t kda_prefill_host_staging_size(int B, int T, int H, int HV, int K, int V, 
  * uploaded on a copy stream of the library while the earlier parts compute,
  * and each part's o rows are downloaded as soon as its carry has run, so
  * the two copy directions overlap; the results equal kda_prefill_forward's
- * bit for bit.  Calls on one device are serialised by the library while
+ * bit for bit.  A packed batch runs through kda_prefill_forward_varlen with
+ * cu_seqlens_host as its host copy of the boundaries, so its carry can
+ * overlap the intra-chunk work (its copies are not split).  Calls on one device are serialised by the library while
  * they enqueue (the copy streams are shared).
  */
 kda_status_t kda_prefill_forward_host(const void *q_host, const void *k_host, const void *v_host,

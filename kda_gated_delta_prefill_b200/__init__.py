@@ -30,7 +30,8 @@ EXPORTED = ("kda_status_string", "kda_prefill_workspace_size", "kda_prefill_forw
             "kda_l2norm_bf16", "kda_prefill_kernel_launches", "kda_decode_step",
             "kda_prefill_backward_workspace_size", "kda_prefill_backward_kernel_launches", "kda_prefill_backward",
             "kda_prefill_state_bf16_workspace_size", "kda_prefill_forward_state_bf16",
-            "kda_prefill_forward_save", "kda_prefill_backward_saved")
+            "kda_prefill_forward_save", "kda_prefill_backward_saved", "kda_prefill_forward_varlen",
+            "kda_prefill_varlen_kernel_launches")
 
 
 class KdaError(RuntimeError):
@@ -86,6 +87,10 @@ def lib():
         L.kda_prefill_forward_save.restype = I
         L.kda_prefill_backward_saved.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, Z, P]
         L.kda_prefill_backward_saved.restype = I
+        L.kda_prefill_forward_varlen.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, Z, P]
+        L.kda_prefill_forward_varlen.restype = I
+        L.kda_prefill_varlen_kernel_launches.argtypes = [I, I, I, I, I, I, P]
+        L.kda_prefill_varlen_kernel_launches.restype = I
         _lib = L
         return L
 
@@ -175,11 +180,34 @@ def kernel_launches(B, T, H, HV, K=128, V=128, num_seqs=0) -> int:
     return int(lib().kda_prefill_kernel_launches(B, T, H, HV, K, V, num_seqs))
 
 
+def _host_cu(cu_seqlens_host):
+    """A host copy of cu_seqlens (sequence, numpy array or CPU tensor) as contiguous int32 numpy."""
+    import numpy as np
+    if hasattr(cu_seqlens_host, "detach"):
+        if cu_seqlens_host.device.type != "cpu":
+            raise ValueError("cu_seqlens_host must be in host memory")
+        cu_seqlens_host = cu_seqlens_host.detach().numpy()
+    return np.ascontiguousarray(np.asarray(cu_seqlens_host, dtype=np.int32))
+
+
+def varlen_kernel_launches(T, H, HV, cu_seqlens_host, K=128, V=128) -> int:
+    """Kernel launches forward(..., cu_seqlens_host=...) makes for these lengths (0 if rejected)."""
+    cu = _host_cu(cu_seqlens_host)
+    return int(lib().kda_prefill_varlen_kernel_launches(T, H, HV, K, V, cu.size - 1,
+                                                        cu.ctypes.data_as(ctypes.c_void_p)))
+
+
 def forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o=None, final_state=None,
-            workspace=None, stream=None):
-    """Run the forward on CUDA tensors; returns (o, final_state)."""
+            workspace=None, stream=None, cu_seqlens_host=None):
+    """Run the forward on CUDA tensors; returns (o, final_state).
+
+    cu_seqlens_host: optional host copy of cu_seqlens (same values).  With it the library knows the sequence
+    lengths and can overlap a packed batch's state carry with its intra-chunk work (kda_prefill_forward_varlen).
+    """
     import torch
     B, T, H, HV, K, V, N, dev = _need_inputs(q, k, v, g, beta, initial_state, cu_seqlens)
+    if cu_seqlens_host is not None and cu_seqlens is None:
+        raise ValueError("cu_seqlens_host needs cu_seqlens")
     if o is None:
         o = torch.empty(B, T, HV, V, dtype=torch.bfloat16, device=dev)
     if final_state is None:
@@ -192,11 +220,22 @@ def forward(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *, o=None, fi
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     if workspace is not None:
         _need("workspace", workspace, torch.uint8, None, dev)
+    ws_n = workspace.numel() if workspace is not None else 0
     with _on(dev):
+        if cu_seqlens_host is not None:
+            cu_h = _host_cu(cu_seqlens_host)
+            if cu_h.size != N + 1:
+                raise ValueError(f"cu_seqlens_host has {cu_h.size} entries, expected {N + 1}")
+            rc = lib().kda_prefill_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                                  _ptr(initial_state), _ptr(cu_seqlens),
+                                                  cu_h.ctypes.data_as(ctypes.c_void_p), num_seqs, T, H, HV, K, V,
+                                                  _ptr(o), _ptr(final_state), _ptr(workspace), ws_n,
+                                                  _stream_ptr(stream, dev))
+            _check(rc, "kda_prefill_forward_varlen")
+            return o, final_state
         rc = lib().kda_prefill_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state),
                                        _ptr(cu_seqlens), num_seqs, B, T, H, HV, K, V, _ptr(o), _ptr(final_state),
-                                       _ptr(workspace), workspace.numel() if workspace is not None else 0,
-                                       _stream_ptr(stream, dev))
+                                       _ptr(workspace), ws_n, _stream_ptr(stream, dev))
     _check(rc, "kda_prefill_forward")
     return o, final_state
 

@@ -51,8 +51,8 @@ struct CarryParams {
     unsigned *err;
     int T, HV, N;
     int chunks_per_seq;
-    int chunk_begin;           // cu null: this launch carries chunks [chunk_begin, chunk_begin + chunk_count)
-    int chunk_count;           //   of every sequence, from s0 (cu given: whole sequences, chunk_begin = 0)
+    int chunk_begin;           // this launch carries chunks [chunk_begin, chunk_begin + chunk_count) of every
+    int chunk_count;           //   sequence, from s0 (cu given: clipped to the sequence's own chunks)
     // Segmented carry of plain batches (seg_phase != 0): the chunks of every sequence are split into seg_count
     // segments [nck*p/seg_count, nck*(p+1)/seg_count), unit = (sequence, value head) = blockIdx % units.
     //  seg_phase 1, j = blockIdx / units: j = 0 carries segment 0 from s0 and stores its end state, which is the
@@ -79,6 +79,9 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
     extern __shared__ __align__(1024) uint8_t sm[];
     const uint32_t sb = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // A launch that the host made a programmatic dependent of this one (the next chunk window's intra-chunk
+    // work, which reads nothing this kernel writes) may start once every CTA of this grid is resident.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     int h = blockIdx.x % p.HV;
     int n = p.order ? p.order[blockIdx.x / p.HV] : blockIdx.x / p.HV;
@@ -123,10 +126,13 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
         }
     } else if (p.cu) {
         with_o = !p.no_o;
-        c_begin = p.chunk_off[n];
-        nck = p.chunk_off[n + 1] - p.chunk_off[n];
-        tok0 = p.cu[n];
-        len = p.cu[n + 1] - p.cu[n];
+        const int all = p.chunk_off[n + 1] - p.chunk_off[n], a = min(p.chunk_begin, all);
+        c_begin = p.chunk_off[n] + a;
+        nck = min(all - a, p.chunk_count);
+        tok0 = p.cu[n] + static_cast<int64_t>(a) * CH;
+        len = p.cu[n + 1] - p.cu[n] - a * CH;
+        // A window past this sequence's end, with the state carried in place: nothing to do.
+        if (nck == 0 && s_in == s_out) return;
     } else {
         with_o = !p.no_o;
         c_begin = static_cast<int64_t>(n) * p.chunks_per_seq + p.chunk_begin;

@@ -71,6 +71,10 @@ struct IntraParams {
     int chunk_begin;           // cu null: this launch covers chunks [chunk_begin, chunk_begin + chunk_count)
     int chunk_count;           //   of every sequence (cu given: all chunks, chunk_begin = 0)
     int prefetch_stride;       // CTAs resident at once (L2 prefetch distance), 0 = no prefetch
+    // cu given, optional: this launch covers one chunk window, chunks [win_begin, ...) of every sequence, with
+    // win_off[n] = the window's chunks in the sequences before n and win_off[N] = its total
+    const int32_t *win_off;
+    int win_begin;
 };
 
 // Off-diagonal block of X = (I+L)^-1, columns 16J+8nt .. +7:
@@ -135,17 +139,18 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
     const int g8 = lane >> 2, t4 = lane & 3;
 
     // ---- launch-local chunk -> (item chunk index, row of the chunk start, valid rows); false past the end ----
-    const int nchunks = p.cu ? p.chunk_off[p.N] : p.B * p.chunk_count;
+    const int32_t *offs = p.cu ? (p.win_off ? p.win_off : p.chunk_off) : nullptr;
+    const int nchunks = p.cu ? offs[p.N] : p.B * p.chunk_count;
     auto locate = [&](int local, int &ci, int64_t &row0, int &nvalid) {
         if (local >= nchunks) return false;
         if (p.cu) {
-            ci = local;
-            int lo = 0, hi = p.N - 1;  // last n with chunk_off[n] <= ci
+            int lo = 0, hi = p.N - 1;  // last n with offs[n] <= local: the sequence that holds it
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
-                if (p.chunk_off[mid] <= ci) lo = mid; else hi = mid - 1;
+                if (offs[mid] <= local) lo = mid; else hi = mid - 1;
             }
-            const int c = ci - p.chunk_off[lo];
+            const int c = (p.win_off ? p.win_begin : 0) + local - offs[lo];
+            ci = p.chunk_off[lo] + c;
             const int len = p.cu[lo + 1] - p.cu[lo];
             row0 = p.cu[lo] + static_cast<int64_t>(c) * CH;
             nvalid = min(CH, len - c * CH);

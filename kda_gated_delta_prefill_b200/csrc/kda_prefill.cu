@@ -128,7 +128,8 @@ kda_status_t check_dims(int B, int T, int H, int HV, int K, int V, bool varlen, 
     return KDA_OK;
 }
 
-// Workspace: [chunk_off (N+1) | order (N)] for packed batches, then the item blocks.
+// Workspace: [chunk_off (N+1) | order (N) | window offsets (4 x (N+1))] for packed batches, then the
+// item blocks.
 // Plain batches with few (sequence, value head) units and long sequences: one carry CTA per unit would run far
 // longer than everything else, so the carry can run on segments of every sequence at once (segment maps, a
 // scan of the start states, then the segments with outputs).  The workspace reserves room for up to
@@ -171,7 +172,7 @@ int carry_segments(int B, int T, int HV, bool varlen, int sms)
 }
 
 struct Workspace {
-    size_t chunk_off = 0, order = 0, items = 0, seg = 0, total = 0;
+    size_t chunk_off = 0, order = 0, win_off = 0, items = 0, seg = 0, total = 0;
     int64_t max_chunks = 0;
     int segments = 1;
 };
@@ -188,6 +189,8 @@ Workspace workspace_layout(int B, int T, int HV, int num_seqs)
         off += round_up((static_cast<size_t>(num_seqs) + 1) * 4, kAlign);
         w.order = off;
         off += round_up(static_cast<size_t>(num_seqs) * 4, kAlign);
+        w.win_off = off;
+        off += round_up(static_cast<size_t>(kda::kMaxWindows) * (num_seqs + 1) * 4, kAlign);
     }
     w.items = off;
     off += static_cast<size_t>(w.max_chunks) * HV * kda::ITEM_BYTES;
@@ -214,6 +217,55 @@ int pipeline_parts(int B, int T, int HV, bool varlen, int sms)
     const int chunks = (T + CH - 1) / CH;
     const int parts = chunks / kMinChunksPerPart;
     return parts < 2 ? 1 : (parts < kMaxParts ? parts : kMaxParts);
+}
+
+// Packed batches whose lengths the host knows: when the longest sequence is long and the units carried past its
+// first window fit beside the intra-chunk work, the batch is cut into windows of chunk index within each
+// sequence, the longest sequence's chunks split like a plain sequence into parts (the last a quarter of the
+// others).  The carry of window j (every sequence with chunks in it, longest first) runs while the intra-chunk
+// kernel works on window j+1.  Window 0 holds every sequence's first chunks; later windows only the longer
+// sequences.  At most kMaxWindows (4) windows: each intra-chunk launch ends in a partly filled wave of CTAs,
+// which short windows cannot amortise (on the packed GQA workload 4 windows beat 2, 3, 6 and 8).
+struct WindowPlan {
+    kda::ChunkWindows win{};
+    int64_t items[kda::kMaxWindows] = {};  // chunks in each window
+    int seqs[kda::kMaxWindows] = {};       // sequences with chunks in each window (window 0: all)
+};
+
+int plan_windows(const int32_t *cu_host, int N, int HV, int sms, WindowPlan &pl)
+{
+    if (!cu_host || N <= 0) return 1;
+    int longest = 0;
+    for (int n = 0; n < N; ++n) {
+        const int64_t len = static_cast<int64_t>(cu_host[n + 1]) - cu_host[n];
+        const int nck = len > 0 ? static_cast<int>((len + CH - 1) / CH) : 0;
+        longest = nck > longest ? nck : longest;
+    }
+    int parts = longest / kMinChunksPerPart;
+    parts = parts < 2 ? 1 : (parts < kda::kMaxWindows ? parts : kda::kMaxWindows);
+    if (parts == 1) return 1;
+    const int64_t den = 4 * parts - 3;  // the last window a quarter of the others, as for plain batches
+    for (int j = 0; j <= parts; ++j) {
+        const int a = j == parts ? longest : static_cast<int>(static_cast<int64_t>(longest) * 4 * j / den);
+        if (j < parts) pl.win.a[j] = a;
+        if (j > 0) pl.win.w[j - 1] = a - pl.win.a[j - 1];
+    }
+    pl.win.count = parts;
+    for (int j = 0; j < parts; ++j) {
+        pl.items[j] = 0;
+        pl.seqs[j] = j == 0 ? N : 0;
+        for (int n = 0; n < N; ++n) {
+            const int64_t len = static_cast<int64_t>(cu_host[n + 1]) - cu_host[n];
+            const int nck = len > 0 ? static_cast<int>((len + CH - 1) / CH) : 0;
+            const int in = nck - pl.win.a[j];
+            if (in > 0) {
+                pl.items[j] += in < pl.win.w[j] ? in : pl.win.w[j];
+                if (j > 0) ++pl.seqs[j];
+            }
+        }
+    }
+    // the later windows' carries must leave room for the intra-chunk work beside them
+    return static_cast<int64_t>(pl.seqs[1]) * HV < sms ? parts : 1;
 }
 
 // A lane: a side stream for the carry and its fork/join events, created on first use.  A forward that cuts its
@@ -370,7 +422,8 @@ namespace {
 kda_status_t forward_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
                           const float *initial_state, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H,
                           int HV, int K, int V, void *o, float *final_state, void *workspace, size_t workspace_bytes,
-                          void *stream, __nv_bfloat16 *states, const HostIO *hio = nullptr);
+                          void *stream, __nv_bfloat16 *states, const HostIO *hio = nullptr,
+                          const int32_t *cu_host = nullptr);
 }  // namespace
 
 extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const void *v, const float *g,
@@ -384,10 +437,47 @@ extern "C" kda_status_t kda_prefill_forward(const void *q, const void *k, const 
 }
 
 namespace {
+// A host copy of cu_seqlens: 0 first, T last, non-decreasing.
+bool host_cu_ok(const int32_t *cu, int N, int T)
+{
+    if (!cu || N <= 0 || cu[0] != 0 || cu[N] != T) return false;
+    for (int n = 0; n < N; ++n)
+        if (cu[n + 1] < cu[n]) return false;
+    return true;
+}
+}  // namespace
+
+extern "C" kda_status_t kda_prefill_forward_varlen(const void *q, const void *k, const void *v, const float *g,
+                                                   const float *beta, const float *initial_state,
+                                                   const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                                                   int num_seqs, int T, int H, int HV, int K, int V, void *o,
+                                                   float *final_state, void *workspace, size_t workspace_bytes,
+                                                   void *stream)
+{
+    if (!cu_seqlens || !host_cu_ok(cu_seqlens_host, num_seqs, T)) return KDA_ERR_INVALID_ARG;
+    return forward_impl(q, k, v, g, beta, initial_state, cu_seqlens, num_seqs, 1, T, H, HV, K, V, o, final_state,
+                        workspace, workspace_bytes, stream, nullptr, nullptr, cu_seqlens_host);
+}
+
+extern "C" int kda_prefill_varlen_kernel_launches(int T, int H, int HV, int K, int V, int num_seqs,
+                                                  const int32_t *cu_seqlens_host)
+{
+    Dims d;
+    if (check_dims(1, T, H, HV, K, V, true, num_seqs, d) != KDA_OK || !host_cu_ok(cu_seqlens_host, num_seqs, T))
+        return 0;
+    DeviceInfo info;
+    if (device_info(info) != cudaSuccess) return 0;
+    WindowPlan wp;
+    const int windows = T > 0 ? plan_windows(cu_seqlens_host, num_seqs, HV, info.sms, wp) : 1;
+    if (windows > 1) return 3 + 2 * windows;  // chunk offsets, order, window offsets; intra and carry per window
+    return 2 + (T > 0 ? 1 : 0) + 1;
+}
+
+namespace {
 kda_status_t forward_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
                           const float *initial_state, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H,
                           int HV, int K, int V, void *o, float *final_state, void *workspace, size_t workspace_bytes,
-                          void *stream, __nv_bfloat16 *states, const HostIO *hio)
+                          void *stream, __nv_bfloat16 *states, const HostIO *hio, const int32_t *cu_host)
 {
     Dims d;
     const bool varlen = cu_seqlens != nullptr;
@@ -501,6 +591,41 @@ kda_status_t forward_impl(const void *q, const void *k, const void *v, const flo
         if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
         cp.seg_phase = 2;
         return launch_carry(cp, units * segments, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
+    WindowPlan wp;
+    const int windows = varlen && tokens > 0 && !hio ? plan_windows(cu_host, d.N, HV, info.sms, wp) : 1;
+    if (windows > 1) {
+        int32_t *woff = reinterpret_cast<int32_t *>(wsb + ws.win_off);
+        kda::window_offsets_kernel<<<windows, 1024, 0, s>>>(chunk_off, d.N, wp.win, woff);
+        if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+        // All on `stream`.  Each window's carry is launched right after its intra-chunk kernel and signals on
+        // entry (griddepcontrol.launch_dependents) once its CTAs are resident; the next window's intra-chunk kernel
+        // is a programmatic dependent launch of that carry, so it fills the SMs the carry left free instead of
+        // racing it for them.  It reads nothing the carry writes.  Every later launch in the stream is ordered as
+        // usual: window j+1's carry starts after both window j+1's intra-chunk kernel and window j's carry.
+        for (int j = 0; j < windows; ++j) {
+            ip.win_off = woff + static_cast<int64_t>(j) * (d.N + 1);
+            ip.win_begin = wp.win.a[j];
+            ip.chunk_begin = 0;
+            ip.chunk_count = 0;
+            cudaLaunchConfig_t cfg{};
+            cudaLaunchAttribute attr[1]{};
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.gridDim = dim3(static_cast<unsigned>(wp.items[j] * HV));
+            cfg.blockDim = dim3(256);
+            cfg.dynamicSmemBytes = kda::IntraSmem::TOTAL;
+            cfg.stream = s;
+            cfg.attrs = attr;
+            cfg.numAttrs = j > 0 ? 1 : 0;
+            if (cudaLaunchKernelEx(&cfg, kda::kda_intra_kernel, tq, tk, tv, tg, ip) != cudaSuccess)
+                return KDA_ERR_CUDA;
+            cp.s0 = j == 0 ? initial_state : final_state;
+            cp.chunk_begin = wp.win.a[j];
+            cp.chunk_count = wp.win.w[j];
+            if (launch_carry(cp, wp.seqs[j] * HV, s) != cudaSuccess) return KDA_ERR_CUDA;
+        }
+        return KDA_OK;
     }
     const int parts = pipeline_parts(B, T, HV, varlen, info.sms);
     if (hio && parts == 1) return KDA_ERR_INVALID_ARG;  // the host-buffer forward copies part by part only here
@@ -653,9 +778,13 @@ extern "C" kda_status_t kda_prefill_forward_host(const void *q_h, const void *k_
     for (const Cp &c : ins)
         if (c.dst && c.n && cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, s) != cudaSuccess)
             return KDA_ERR_CUDA;
-    st = kda_prefill_forward(dq, dk, dv, reinterpret_cast<float *>(dg), reinterpret_cast<float *>(db),
-                             reinterpret_cast<float *>(ds0), reinterpret_cast<int32_t *>(dcu), num_seqs, B, T, H, HV,
-                             K, V, dO, reinterpret_cast<float *>(dsN), dws, ws, stream);
+    st = varlen ? kda_prefill_forward_varlen(dq, dk, dv, reinterpret_cast<float *>(dg), reinterpret_cast<float *>(db),
+                                             reinterpret_cast<float *>(ds0), reinterpret_cast<int32_t *>(dcu), cu_h,
+                                             num_seqs, T, H, HV, K, V, dO, reinterpret_cast<float *>(dsN), dws, ws,
+                                             stream)
+                : kda_prefill_forward(dq, dk, dv, reinterpret_cast<float *>(dg), reinterpret_cast<float *>(db),
+                                      reinterpret_cast<float *>(ds0), nullptr, 0, B, T, H, HV, K, V, dO,
+                                      reinterpret_cast<float *>(dsN), dws, ws, stream);
     if (st != KDA_OK) return st;
     if (nvb && cudaMemcpyAsync(o_h, dO, nvb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return KDA_ERR_CUDA;
     if (cudaMemcpyAsync(sN_h, dsN, ns, cudaMemcpyDeviceToHost, s) != cudaSuccess) return KDA_ERR_CUDA;

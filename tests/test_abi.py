@@ -46,9 +46,12 @@ def test_workspace_size(L):
     # plain batch: B * ceil(T/64) chunks x HV heads of item blocks
     assert L.kda_prefill_workspace_size(2, 4096, 96, 96, 128, 128, 0) == 2 * 64 * 96 * item
     assert L.kda_prefill_workspace_size(1, 1000, 4, 4, 128, 128, 0) == 16 * 4 * item
-    # packed batch: offsets and order, then (ceil(T/64) + N) chunks as an upper bound
+    # packed batch: offsets, order and 4 x (N + 1) chunk-window offsets, then (ceil(T/64) + N) chunks as an
+    # upper bound
     n = L.kda_prefill_workspace_size(1, 11210, 8, 32, 128, 128, 7)
-    assert n == 256 + 256 + (176 + 7) * 32 * item
+    assert n == 256 + 256 + 256 + (176 + 7) * 32 * item
+    n = L.kda_prefill_workspace_size(1, 11210, 8, 32, 128, 128, 100)
+    assert n == 512 + 512 + 1792 + (176 + 100) * 32 * item
     # rejected sizes
     assert L.kda_prefill_workspace_size(1, 64, 1, 1, 64, 128, 0) == 0
     assert L.kda_prefill_workspace_size(1, 64, 2, 3, 128, 128, 0) == 0
@@ -89,6 +92,22 @@ def call_forward(L, **over):
 ])
 def test_forward_rejects_bad_arguments(L, over, code):
     assert call_forward(L, **over) == code
+
+
+@pytest.mark.parametrize("cu_host,num_seqs,code", [
+    (None, 2, 1),              # no host copy
+    ([1, 30, 64], 2, 1),       # does not start at 0
+    ([0, 30, 63], 2, 1),       # does not end at T
+    ([0, 40, 30, 64], 3, 1),   # decreasing
+    ([0, 64], 0, 1),           # no sequences
+])
+def test_varlen_forward_checks_the_host_boundaries(L, cu_host, num_seqs, code):
+    arr = None if cu_host is None else (ctypes.c_int32 * len(cu_host))(*cu_host)
+    rc = L.kda_prefill_forward_varlen(FAKE, FAKE * 2, FAKE * 3, FAKE * 4, FAKE * 5, None, FAKE * 8, arr, num_seqs,
+                                      64, 1, 1, 128, 128, FAKE * 6, FAKE * 7, FAKE * 64, 1 << 30, None)
+    assert rc == code
+    # the same boundaries size the launch plan; malformed ones give 0
+    assert L.kda_prefill_varlen_kernel_launches(64, 1, 1, 128, 128, num_seqs, arr) == 0
 
 
 def test_partial_state_overlap_rejected(L):

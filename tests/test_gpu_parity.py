@@ -285,6 +285,137 @@ def test_parts_match_the_uncut_run_bit_for_bit():
     assert torch.equal(s_cut, s_one)
 
 
+# ------------------------------------------------------------------ packed batches cut into chunk windows
+# Given a host copy of cu_seqlens (kda_prefill_forward_varlen), the library knows the lengths and may cut a packed
+# batch into windows of chunk index within each sequence, carrying window j beside the intra-chunk work of window
+# j+1.  Each window's carry starts from the float32 state the previous one left in final_state, so the results
+# equal the uncut packed run bit for bit.
+
+WINDOW_MIXES = {
+    "gqa_mix": ([1, 63, 64, 65, 777, 2048, 8192], 8, 32),  # the packed GQA workload's lengths
+    "empty_and_short": ([0, 2100, 0, 1, 129, 3000, 0], 2, 4),
+    "one_long": ([5000], 2, 4),
+    "two_equal": ([2048, 2048], 4, 8),
+    "ragged_tail": ([2049, 63, 2111], 2, 2),
+}
+
+
+def _window_count(T, H, HV, cu_h):
+    import kda_gated_delta_prefill_b200 as kda
+    n = kda.varlen_kernel_launches(T, H, HV, cu_h)
+    return (n - 3) // 2 if n > 4 else 1
+
+
+@pytest.mark.parametrize("mix", list(WINDOW_MIXES))
+def test_windows_match_the_uncut_packed_run_bit_for_bit(mix):
+    lengths, H, HV = WINDOW_MIXES[mix]
+    case = gen.Case(f"win_{mix}", B=1, T=sum(lengths), H=H, HV=HV, lengths=lengths, state="n01",
+                    seed=600 + len(mix))
+    x = gen.make_inputs(case)
+    cu_h = x["cu_seqlens"]
+    assert _window_count(case.T, H, HV, cu_h) >= 2  # the windowed path is taken
+    o_w, s_w = gpu_forward(x, cu_seqlens_host=cu_h)
+    o_u, s_u = gpu_forward(x)
+    assert torch.equal(o_w, o_u)
+    assert torch.equal(s_w, s_u)
+    import kda_gated_delta_prefill_b200 as kda
+    assert kda.device_error(clear=True) == 0
+
+
+def test_windows_full_parity():
+    lengths = [2049, 63, 0, 2111]
+    case = gen.Case("win_oracle", B=1, T=sum(lengths), H=2, HV=2, lengths=lengths, state="n01", seed=641)
+    x = gen.make_inputs(case)
+    assert _window_count(case.T, 2, 2, x["cu_seqlens"]) >= 2
+    o, s = gpu_forward(x, cu_seqlens_host=x["cu_seqlens"])
+    compare(o, s, oracle_forward(x))
+
+
+def test_windows_short_batch_runs_uncut():
+    lengths = [300, 1900, 64]  # the longest has 30 chunks: too short to cut
+    case = gen.Case("win_short", B=1, T=sum(lengths), H=2, HV=4, lengths=lengths, state="n01", seed=651)
+    x = gen.make_inputs(case)
+    import kda_gated_delta_prefill_b200 as kda
+    assert kda.varlen_kernel_launches(case.T, 2, 4, x["cu_seqlens"]) == 4
+    o_w, s_w = gpu_forward(x, cu_seqlens_host=x["cu_seqlens"])
+    o_u, s_u = gpu_forward(x)
+    assert torch.equal(o_w, o_u) and torch.equal(s_w, s_u)
+
+
+def test_windows_in_place_state_update():
+    lengths = [3000, 0, 700]
+    case = gen.Case("win_inplace", B=1, T=sum(lengths), H=2, HV=2, lengths=lengths, state="n01", seed=661)
+    x = gen.make_inputs(case)
+    xc = to_cuda(x)
+    import kda_gated_delta_prefill_b200 as kda
+    st = xc["initial_state"].clone()
+    o, s = kda.forward(xc["q"], xc["k"], xc["v"], xc["g"], xc["beta"], st, xc["cu_seqlens"], final_state=st,
+                       cu_seqlens_host=x["cu_seqlens"])
+    o_u, s_u = gpu_forward(x)
+    torch.cuda.synchronize()
+    assert s.data_ptr() == st.data_ptr()
+    assert torch.equal(o, o_u) and torch.equal(s, s_u)
+
+
+def test_windows_host_entry_point():
+    # kda_prefill_forward_host passes its host cu_seqlens on, so a packed batch takes the windowed path there
+    lengths = [2500, 17, 900]
+    case = gen.Case("win_host", B=1, T=sum(lengths), H=2, HV=4, lengths=lengths, state="n01", seed=671)
+    x = gen.make_inputs(case)
+    import kda_gated_delta_prefill_b200 as kda
+    assert _window_count(case.T, 2, 4, x["cu_seqlens"]) >= 2
+    N, T, HV = case.N, case.T, case.HV
+    pin = {k: v.pin_memory() for k, v in x.items() if isinstance(v, torch.Tensor)}
+    o_h = torch.empty(1, T, HV, 128, dtype=torch.bfloat16).pin_memory()
+    s_h = torch.empty(N, HV, 128, 128).pin_memory()
+    staging = torch.empty(kda.host_staging_size(1, T, 2, HV, num_seqs=N, has_initial_state=True,
+                                                has_cu_seqlens=True), dtype=torch.uint8, device="cuda")
+    kda.forward_host(pin["q"], pin["k"], pin["v"], pin["g"], pin["beta"], pin["initial_state"], pin["cu_seqlens"],
+                     o=o_h, final_state=s_h, staging=staging)
+    torch.cuda.synchronize()
+    o_u, s_u = gpu_forward(x)
+    assert torch.equal(o_h, o_u.cpu()) and torch.equal(s_h, s_u.cpu())
+
+
+def test_windows_captured_in_a_cuda_graph():
+    import kda_gated_delta_prefill_b200 as kda
+    lengths = [2300, 5, 0, 1200]
+    cases = [gen.Case(f"wgraph{i}", B=1, T=sum(lengths), H=2, HV=4, lengths=lengths, state="n01", seed=681 + i)
+             for i in range(2)]
+    xs = [gen.make_inputs(c) for c in cases]
+    cu_h = xs[0]["cu_seqlens"]
+    assert _window_count(cases[0].T, 2, 4, cu_h) >= 2
+    xcs = [to_cuda(x) for x in xs]
+    N, T = cases[0].N, cases[0].T
+    buf = {k: v.clone() for k, v in xcs[0].items() if isinstance(v, torch.Tensor)}
+    ws = torch.empty(kda.workspace_size(1, T, 2, 4, 128, 128, N), dtype=torch.uint8, device="cuda")
+    o = torch.empty(1, T, 4, 128, dtype=torch.bfloat16, device="cuda")
+    s = torch.empty(N, 4, 128, 128, device="cuda")
+
+    def call():
+        kda.forward(buf["q"], buf["k"], buf["v"], buf["g"], buf["beta"], buf["initial_state"], buf["cu_seqlens"],
+                    o=o, final_state=s, workspace=ws, cu_seqlens_host=cu_h)
+
+    call()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    for xc in xcs:
+        for k, t in buf.items():
+            t.copy_(xc[k])
+        o.fill_(float("nan"))
+        s.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        o_ref, s_ref = kda.forward(xc["q"], xc["k"], xc["v"], xc["g"], xc["beta"], xc["initial_state"],
+                                   xc["cu_seqlens"])
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_ref) and torch.equal(s, s_ref)
+    del graph
+    assert kda.device_error(clear=True) == 0
+
+
 def test_parts_in_place_state_update():
     case = gen.Case("parts_inplace", B=1, T=3000, H=2, HV=2, state="n01", seed=321)
     x = gen.make_inputs(case)
