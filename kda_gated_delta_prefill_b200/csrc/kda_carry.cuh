@@ -69,6 +69,7 @@ struct CarryParams {
     // [K][V] (nearest even) at states + (global chunk * HV + h) * K * V (the item's index), for the backward.
     __nv_bfloat16 *states;
     int no_o;                      // unsegmented launches: skip o (the O products and stores)
+    int h_begin, h_count;          // plain batches, optional: only value heads [h_begin, h_begin + h_count)
 };
 
 // kDump: the backward's instantiation, which also stores every chunk's start state (p.states)
@@ -83,8 +84,9 @@ __global__ void __launch_bounds__(kCarryThreads, 1) kda_carry_kernel(const Carry
     // work, which reads nothing this kernel writes) may start once every CTA of this grid is resident.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    int h = blockIdx.x % p.HV;
-    int n = p.order ? p.order[blockIdx.x / p.HV] : blockIdx.x / p.HV;
+    const int nh = p.h_count ? p.h_count : p.HV;  // value heads this launch covers, from h_begin
+    int h = p.h_begin + static_cast<int>(blockIdx.x % nh);
+    int n = p.order ? p.order[blockIdx.x / nh] : blockIdx.x / nh;
     int64_t c_begin, tok0;
     int nck, len;
     // where the state starts and ends, and what the chunk loop produces

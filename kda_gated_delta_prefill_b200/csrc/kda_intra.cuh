@@ -75,6 +75,8 @@ struct IntraParams {
     // win_off[n] = the window's chunks in the sequences before n and win_off[N] = its total
     const int32_t *win_off;
     int win_begin;
+    // optional: only value heads [h_begin, h_begin + h_count) (h_count 0: all)
+    int h_begin, h_count;
 };
 
 // Off-diagonal block of X = (I+L)^-1, columns 16J+8nt .. +7:
@@ -162,11 +164,12 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
         }
         return true;
     };
-    const int h = blockIdx.x % p.HV;
+    const int nh = p.h_count ? p.h_count : p.HV;  // value heads this launch covers, from h_begin
+    const int h = p.h_begin + static_cast<int>(blockIdx.x % nh);
     int ci;
     int64_t row0;
     int nvalid;
-    if (!locate(blockIdx.x / p.HV, ci, row0, nvalid)) return;
+    if (!locate(blockIdx.x / nh, ci, row0, nvalid)) return;
     const int hq = h / (p.HV / p.H);
     uint8_t *out = p.items + (static_cast<int64_t>(ci) * p.HV + h) * ITEM_BYTES;  // item block (global)
 
@@ -195,8 +198,8 @@ __global__ void __launch_bounds__(256, kIntraCtasPerSm)
         const int pi = blockIdx.x + p.prefetch_stride;
         int pci, pvalid;
         int64_t prow;
-        if (p.prefetch_stride > 0 && pi < static_cast<int>(gridDim.x) && locate(pi / p.HV, pci, prow, pvalid)) {
-            const int ph = pi % p.HV, pz = static_cast<int>(prow), phq = ph / (p.HV / p.H);
+        if (p.prefetch_stride > 0 && pi < static_cast<int>(gridDim.x) && locate(pi / nh, pci, prow, pvalid)) {
+            const int ph = p.h_begin + pi % nh, pz = static_cast<int>(prow), phq = ph / (p.HV / p.H);
             tma_prefetch_3d(&tq, 0, phq, pz);
             tma_prefetch_3d(&tq, 64, phq, pz);
             tma_prefetch_3d(&tk, 0, phq, pz);

@@ -219,6 +219,21 @@ int pipeline_parts(int B, int T, int HV, bool varlen, int sms)
     return parts < 2 ? 1 : (parts < kMaxParts ? parts : kMaxParts);
 }
 
+// Plain batches with more (sequence, value head) units than SMs but fewer than twice as many carry in two waves,
+// and the second, partial wave runs alone.  Such a batch is instead split by value heads into two groups: the
+// last group is as many heads as make one full wave of carry CTAs (floor(SMs / B) heads), the first the rest.
+// The first group's carry then runs beside the last group's intra-chunk work, and the last group's carry is one
+// full wave at the end.  (More groups would not help: a carry costs more SM-time beside intra-chunk work than in
+// a full last wave.)  Returns the heads of the last group, or 0 for no split.
+int head_group_split(int B, int T, int HV, int sms)
+{
+    const int64_t units = static_cast<int64_t>(B) * HV;
+    const int chunks = (T + CH - 1) / CH;
+    if (units <= sms || units >= 2 * static_cast<int64_t>(sms) || chunks < kMinChunksPerPart) return 0;
+    const int last = sms / B;
+    return last > 0 && last < HV ? last : 0;
+}
+
 // Packed batches whose lengths the host knows: when the longest sequence is long and the units carried past its
 // first window fit beside the intra-chunk work, the batch is cut into windows of chunk index within each
 // sequence, the longest sequence's chunks split like a plain sequence into parts (the last a quarter of the
@@ -403,6 +418,8 @@ extern "C" int kda_prefill_kernel_launches(int B, int T, int H, int HV, int K, i
     if (device_info(info) != cudaSuccess) return 0;
     if (varlen) return 2 + (T > 0 ? 1 : 0) + 1;  // chunk offsets, order, intra (if any token), carry
     if (carry_segments(B, T, HV, false, info.sms) > 1) return 4;  // intra, segment maps, scan, segments with outputs
+    if (pipeline_parts(B, T, HV, false, info.sms) == 1 && head_group_split(B, T, HV, info.sms) > 0)
+        return 4;  // intra and carry of each head group
     return 2 * pipeline_parts(B, T, HV, false, info.sms);
 }
 
@@ -630,9 +647,39 @@ kda_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     const int parts = pipeline_parts(B, T, HV, varlen, info.sms);
     if (hio && parts == 1) return KDA_ERR_INVALID_ARG;  // the host-buffer forward copies part by part only here
     if (parts == 1) {
-        if (tokens > 0 && launch_intra(0, cp.chunks_per_seq, ws.max_chunks) != cudaSuccess) return KDA_ERR_CUDA;
         cp.chunk_begin = 0;
         cp.chunk_count = cp.chunks_per_seq;
+        const int last = varlen || tokens == 0 || hio ? 0 : head_group_split(B, T, HV, info.sms);
+        if (last > 0) {
+            // Two head groups on `stream`: the first group's carry is followed by the last group's intra-chunk
+            // kernel as a programmatic dependent launch (it starts once every carry CTA is resident and reads
+            // nothing the carry writes), then the last group's carry, an ordinary launch after both.
+            const int first = HV - last;
+            for (int grp = 0; grp < 2; ++grp) {
+                const int h0 = grp == 0 ? 0 : first, nh = grp == 0 ? first : last;
+                ip.h_begin = h0;
+                ip.h_count = nh;
+                ip.chunk_begin = 0;
+                ip.chunk_count = cp.chunks_per_seq;
+                cudaLaunchConfig_t cfg{};
+                cudaLaunchAttribute attr[1]{};
+                attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+                attr[0].val.programmaticStreamSerializationAllowed = 1;
+                cfg.gridDim = dim3(static_cast<unsigned>(static_cast<int64_t>(B) * cp.chunks_per_seq * nh));
+                cfg.blockDim = dim3(256);
+                cfg.dynamicSmemBytes = kda::IntraSmem::TOTAL;
+                cfg.stream = s;
+                cfg.attrs = attr;
+                cfg.numAttrs = grp > 0 ? 1 : 0;
+                if (cudaLaunchKernelEx(&cfg, kda::kda_intra_kernel, tq, tk, tv, tg, ip) != cudaSuccess)
+                    return KDA_ERR_CUDA;
+                cp.h_begin = h0;
+                cp.h_count = nh;
+                if (launch_carry(cp, B * nh, s) != cudaSuccess) return KDA_ERR_CUDA;
+            }
+            return KDA_OK;
+        }
+        if (tokens > 0 && launch_intra(0, cp.chunks_per_seq, ws.max_chunks) != cudaSuccess) return KDA_ERR_CUDA;
         return launch_carry(cp, d.N * HV, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     }
 

@@ -94,6 +94,28 @@ def test_wide_heads_sampled():
     compare(o[:, :, heads].contiguous(), s[:, heads].contiguous(), ref)
 
 
+def test_head_groups_match_per_head_calls_bit_for_bit():
+    # 2 x 96 units: between one and two waves of carry CTAs, so the forward splits the value heads into two
+    # groups (the first group's carry beside the second group's intra-chunk work).  Heads are independent, so
+    # the same batch run as two calls of 48 heads each (fewer units than SMs: another launch plan) must give
+    # the same bits.
+    import kda_gated_delta_prefill_b200 as kda
+    B, T, H = 2, 1024, 96
+    case = gen.Case("head_groups", B=B, T=T, H=H, HV=H, state="n01", seed=701)
+    assert kda.kernel_launches(B, T, H, H) == 4  # intra and carry of each group
+    x = to_cuda(gen.make_inputs(case))
+    o, s = kda.forward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["initial_state"])
+    for h0 in (0, 48):
+        hs = slice(h0, h0 + 48)
+        oh, sh = kda.forward(x["q"][:, :, hs].contiguous(), x["k"][:, :, hs].contiguous(),
+                             x["v"][:, :, hs].contiguous(), x["g"][:, :, hs].contiguous(),
+                             x["beta"][:, :, hs].contiguous(), x["initial_state"][:, hs].contiguous())
+        torch.cuda.synchronize()
+        assert torch.equal(o[:, :, hs], oh)
+        assert torch.equal(s[:, hs], sh)
+    assert kda.device_error(clear=True) == 0
+
+
 def test_long_prefill_sampled():
     # B=1, H=HV=64, T=65536 with state, generated on the device as the benchmark does.
     x = gen.make_inputs(gen.LONG_PREFILL, device="cuda")
@@ -597,8 +619,9 @@ def test_bf16_state_forward(B, T, H, HV, varlen):
 @pytest.mark.parametrize("B,T,H,HV,lengths", [(1, 2600, 4, 8, None),      # cut into parts (side stream)
                                               (1, 5120, 2, 2, None),      # segmented carry
                                               (1, 1300, 2, 4, [700, 0, 64, 536]),  # packed sequences
-                                              (2, 300, 2, 4, None)],      # plain, uncut
-                         ids=["parts", "segmented", "packed", "plain"])
+                                              (2, 300, 2, 4, None),       # plain, uncut
+                                              (2, 1024, 8, 96, None)],    # two head groups
+                         ids=["parts", "segmented", "packed", "plain", "head_groups"])
 def test_forward_captured_in_a_cuda_graph(B, T, H, HV, lengths):
     import kda_gated_delta_prefill_b200 as kda
     cases = [gen.Case(f"graph{i}", B=B, T=T, H=H, HV=HV, lengths=lengths, state="n01", seed=500 + 7 * i + T)
