@@ -52,6 +52,8 @@ struct BwdParams {
     const int32_t *cu, *chunk_off;          // packed sequences (cu [N+1], chunk_off [N+1]) or null
     unsigned *err;
     int T, H, HV, N, chunks_per_seq;
+    // H == HV: the chunk kernel applies the normalisation's Jacobian itself and writes dq, dk (no dqn, dkn)
+    int fuse_norm;
 };
 
 // (sequence, first token row, valid rows) of global chunk index `chunk`
@@ -978,21 +980,82 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 rG[j][q] = __fmaf_rn(-KB[i][d], ra[j][q], rG[j][q]);
             }
     }
-    // dqn, dkn out (valid rows)
+    // dqn, dkn out (valid rows), for kda_bwd_norm_kernel; or, with one value head per Q/K head, dq and dk here:
+    // dx = dy / n - x (x . dy) / n^3 (n: the row's denominator of the forward's normalisation), with x . dy
+    // summed by the four lanes that share a row in this warp and then across the two warps that hold its halves.
+    float xdy[2][2] = {};  // [row r0 / r1][q / k] partial x . dy of this thread's 16 columns
+    if (!p.fuse_norm) {
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-        const int i = hf ? r1 : r0;
-        if (i < nvalid) {
-            float *dq = p.dqn + ((row0 + i) * p.HV + h) * DK + 64 * nh + 2 * t4;
-            float *dk = p.dkn + ((row0 + i) * p.HV + h) * DK + 64 * nh + 2 * t4;
+        for (int hf = 0; hf < 2; ++hf) {
+            const int i = hf ? r1 : r0;
+            if (i < nvalid) {
+                float *dq = p.dqn + ((row0 + i) * p.HV + h) * DK + 64 * nh + 2 * t4;
+                float *dk = p.dkn + ((row0 + i) * p.HV + h) * DK + 64 * nh + 2 * t4;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                *reinterpret_cast<float2 *>(dq + 8 * j) = make_float2(rq[j][2 * hf], rq[j][2 * hf + 1]);
-                *reinterpret_cast<float2 *>(dk + 8 * j) = make_float2(rk[j][2 * hf], rk[j][2 * hf + 1]);
+                for (int j = 0; j < 8; ++j) {
+                    *reinterpret_cast<float2 *>(dq + 8 * j) = make_float2(rq[j][2 * hf], rq[j][2 * hf + 1]);
+                    *reinterpret_cast<float2 *>(dk + 8 * j) = make_float2(rk[j][2 * hf], rk[j][2 * hf + 1]);
+                }
+            }
+        }
+    } else {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int i = hf ? r1 : r0;
+            if (i < nvalid) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int64_t off = ((row0 + i) * p.H + hq) * DK + 64 * nh + 8 * j + 2 * t4;
+                    const uint32_t wq = *reinterpret_cast<const uint32_t *>(p.q + off);
+                    const uint32_t wk = *reinterpret_cast<const uint32_t *>(p.k + off);
+                    xdy[hf][0] = __fmaf_rn(bf16lo(wq), rq[j][2 * hf], xdy[hf][0]);
+                    xdy[hf][0] = __fmaf_rn(bf16hi(wq), rq[j][2 * hf + 1], xdy[hf][0]);
+                    xdy[hf][1] = __fmaf_rn(bf16lo(wk), rk[j][2 * hf], xdy[hf][1]);
+                    xdy[hf][1] = __fmaf_rn(bf16hi(wk), rk[j][2 * hf + 1], xdy[hf][1]);
+                }
+            }
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+                xdy[hf][w] = __fadd_rn(xdy[hf][w], __shfl_xor_sync(0xffffffffu, xdy[hf][w], 1));
+                xdy[hf][w] = __fadd_rn(xdy[hf][w], __shfl_xor_sync(0xffffffffu, xdy[hf][w], 2));
             }
         }
     }
     __syncthreads();  // KA/QA/KB/G reads done; dgl complete
+    if (p.fuse_norm) {
+        float *red = reinterpret_cast<float *>(sm + S::EM);  // [q|k][row][half]; exp(m_I) is no longer read
+        if (t4 == 0) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                for (int w = 0; w < 2; ++w) red[(w * CH + (hf ? r1 : r0)) * 2 + nh] = xdy[hf][w];
+        }
+        __syncthreads();
+        // row i's half of dx from dy = this thread's columns of dqn (or dkn), w = 0 (q) or 1 (k)
+        auto emit = [&](const float (&dy)[8][4], int hf, int w, const __nv_bfloat16 *x, __nv_bfloat16 *dx,
+                        float den) {
+            const int i = hf ? r1 : r0;
+            const float tot = __fadd_rn(red[(w * CH + i) * 2], red[(w * CH + i) * 2 + 1]);
+            const float inv = __frcp_rn(den);
+            const float c3 = __fmul_rn(tot, __fmul_rn(inv, __fmul_rn(inv, inv)));
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int64_t off = ((row0 + i) * p.H + hq) * DK + 64 * nh + 8 * j + 2 * t4;
+                const uint32_t wx = *reinterpret_cast<const uint32_t *>(x + off);
+                const float o0 = __fmaf_rn(-bf16lo(wx), c3, __fmul_rn(dy[j][2 * hf], inv));
+                const float o1 = __fmaf_rn(-bf16hi(wx), c3, __fmul_rn(dy[j][2 * hf + 1], inv));
+                *reinterpret_cast<uint32_t *>(dx + off) = pack_bf16(o0, o1);
+            }
+        };
+        if (r0 < nvalid) {
+            emit(rq, 0, 0, p.q, p.dq, denq[r0]);
+            emit(rk, 0, 1, p.k, p.dk, denk[r0]);
+        }
+        if (r1 < nvalid) {
+            emit(rq, 1, 0, p.q, p.dq, denq[r1]);
+            emit(rk, 1, 1, p.k, p.dk, denk[r1]);
+        }
+    }
     // dG rows into the KA region (unpadded [64][128]), then the reverse cumulative sum per key column
     float(*dG)[DK] = reinterpret_cast<float(*)[DK]>(sm + S::KA);
 #pragma unroll
@@ -1016,48 +1079,72 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
 
 // ---------------------------------------------------------------------------------------------------------
 // dq (dk) row of Q/K head hq = J(x)^T sum over the value heads of its group of dqn (dkn), with
-// J(x) the Jacobian of x / sqrt(sum x^2 + 1e-6): dx = dy / n - x (x . dy) / n^3.  One warp per (row, head, q|k).
+// J(x) the Jacobian of x / sqrt(sum x^2 + 1e-6): dx = dy / n - x (x . dy) / n^3.  A unit is one (row, head, q|k);
+// a warp takes kNormUnits consecutive units and issues all their loads before any arithmetic, so that several
+// rows' loads are in flight per warp (each unit alone is too little work to hide a DRAM round trip).
+constexpr int kNormUnits = 4;
 __global__ void __launch_bounds__(256) kda_bwd_norm_kernel(const BwdParams p, int64_t rows)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t w = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const int64_t w0 = (static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kNormUnits;
     const int64_t units = rows * p.H * 2;
-    if (w >= units) return;
-    const int which = static_cast<int>(w & 1);
-    const int64_t rh = w >> 1, row = rh / p.H;
-    const int hq = static_cast<int>(rh % p.H);
-    if (p.cu && row >= p.cu[p.N]) return;  // outside every sequence
-    const __nv_bfloat16 *x = (which ? p.k : p.q) + (row * p.H + hq) * DK + 4 * lane;
-    const float *dy = (which ? p.dkn : p.dqn) + (row * p.HV) * DK + 4 * lane;
+    if (w0 >= units) return;
     const int grp = p.HV / p.H;
-    const uint2 raw = *reinterpret_cast<const uint2 *>(x);
-    const float xv[4] = {bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y)};
-    float g[4] = {};
+    const int64_t end = p.cu ? p.cu[p.N] : rows;  // rows past it belong to no sequence
+    bool live[kNormUnits];
+    int64_t xoff[kNormUnits], yoff[kNormUnits];
+    uint2 raw[kNormUnits];
+#pragma unroll
+    for (int u = 0; u < kNormUnits; ++u) {
+        const int64_t w = w0 + u;
+        const int which = static_cast<int>(w & 1);
+        const int64_t rh = w >> 1, row = rh / p.H;
+        const int hq = static_cast<int>(rh % p.H);
+        live[u] = w < units && row < end;
+        xoff[u] = (row * p.H + hq) * DK + 4 * lane;  // into q or k, and into dq or dk
+        yoff[u] = (row * p.HV + hq * grp) * DK + 4 * lane;
+        raw[u] = make_uint2(0u, 0u);
+        if (live[u]) raw[u] = *reinterpret_cast<const uint2 *>((which ? p.k : p.q) + xoff[u]);
+    }
+    float g[kNormUnits][4] = {};
     for (int j = 0; j < grp; ++j) {
-        const float4 t = *reinterpret_cast<const float4 *>(dy + (hq * grp + j) * DK);
-        g[0] = __fadd_rn(g[0], t.x);
-        g[1] = __fadd_rn(g[1], t.y);
-        g[2] = __fadd_rn(g[2], t.z);
-        g[3] = __fadd_rn(g[3], t.w);
-    }
-    float ss = 0.f, xd = 0.f;
+        float4 t[kNormUnits];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        ss = __fmaf_rn(xv[e], xv[e], ss);
-        xd = __fmaf_rn(xv[e], g[e], xd);
+        for (int u = 0; u < kNormUnits; ++u) {
+            t[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (live[u]) t[u] = *reinterpret_cast<const float4 *>((((w0 + u) & 1) ? p.dkn : p.dqn) + yoff[u] + j * DK);
+        }
+#pragma unroll
+        for (int u = 0; u < kNormUnits; ++u) {
+            g[u][0] = __fadd_rn(g[u][0], t[u].x);
+            g[u][1] = __fadd_rn(g[u][1], t[u].y);
+            g[u][2] = __fadd_rn(g[u][2], t[u].z);
+            g[u][3] = __fadd_rn(g[u][3], t[u].w);
+        }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
-        xd = __fadd_rn(xd, __shfl_xor_sync(0xffffffffu, xd, off));
-    }
-    const float nrm = __fsqrt_rn(__fadd_rn(ss, 1e-6f));
-    const float inv = __frcp_rn(nrm), c3 = __fmul_rn(xd, __fmul_rn(inv, __fmul_rn(inv, inv)));
-    float out[4];
+    for (int u = 0; u < kNormUnits; ++u) {
+        const float xv[4] = {bf16lo(raw[u].x), bf16hi(raw[u].x), bf16lo(raw[u].y), bf16hi(raw[u].y)};
+        float ss = 0.f, xd = 0.f;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) out[e] = __fmaf_rn(-xv[e], c3, __fmul_rn(g[e], inv));
-    __nv_bfloat16 *dst = (which ? p.dk : p.dq) + (row * p.H + hq) * DK + 4 * lane;
-    *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16(out[0], out[1]), pack_bf16(out[2], out[3]));
+        for (int e = 0; e < 4; ++e) {
+            ss = __fmaf_rn(xv[e], xv[e], ss);
+            xd = __fmaf_rn(xv[e], g[u][e], xd);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
+            xd = __fadd_rn(xd, __shfl_xor_sync(0xffffffffu, xd, off));
+        }
+        const float nrm = __fsqrt_rn(__fadd_rn(ss, 1e-6f));
+        const float inv = __frcp_rn(nrm), c3 = __fmul_rn(xd, __fmul_rn(inv, __fmul_rn(inv, inv)));
+        float out[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) out[e] = __fmaf_rn(-xv[e], c3, __fmul_rn(g[u][e], inv));
+        if (live[u])
+            *reinterpret_cast<uint2 *>((((w0 + u) & 1) ? p.dk : p.dq) + xoff[u]) =
+                make_uint2(pack_bf16(out[0], out[1]), pack_bf16(out[2], out[3]));
+    }
 }
 
 }  // namespace kda

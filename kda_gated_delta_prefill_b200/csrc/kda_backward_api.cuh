@@ -70,8 +70,8 @@ extern "C" int kda_prefill_backward_kernel_launches(int B, int T, int H, int HV,
         parts = pipeline_parts(B, T, HV, false, info.sms);
     }
     // chunk offsets (packed), intra-chunk and carry with the start states per part, reverse carry, chunk
-    // gradients, norms
-    return (varlen ? 1 : 0) + (with_tokens + 1) * parts + 1 + 2 * with_tokens;
+    // gradients, and the Q/K normalisation's Jacobian (inside the chunk kernel when H == HV)
+    return (varlen ? 1 : 0) + (with_tokens + 1) * parts + 1 + with_tokens * (H == HV ? 1 : 2);
 }
 
 extern "C" kda_status_t kda_prefill_backward(const void *q, const void *k, const void *v, const float *g,
@@ -271,6 +271,7 @@ kda_status_t backward_impl(const void *q, const void *k, const void *v, const fl
     bp.dkn = reinterpret_cast<float *>(wsb + ws.dkn);
     bp.dq = static_cast<__nv_bfloat16 *>(dq);
     bp.dk = static_cast<__nv_bfloat16 *>(dk);
+    bp.fuse_norm = H == HV;
     bp.dv = static_cast<__nv_bfloat16 *>(dv);
     bp.dg = dg;
     bp.dbeta = dbeta;
@@ -296,7 +297,8 @@ kda_status_t backward_impl(const void *q, const void *k, const void *v, const fl
         return KDA_ERR_CUDA;
     kda::kda_bwd_chunk_kernel<<<static_cast<int>(ws.max_chunks * HV), kda::kBwThreads, kda::BwSmem::TOTAL, s>>>(bp);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
-    const int64_t warps = tokens * H * 2;
+    if (bp.fuse_norm) return KDA_OK;  // the chunk kernel wrote dq and dk
+    const int64_t warps = (tokens * H * 2 + kda::kNormUnits - 1) / kda::kNormUnits;
     kda::kda_bwd_norm_kernel<<<static_cast<int>((warps + 7) / 8), 256, 0, s>>>(bp, tokens);
     return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

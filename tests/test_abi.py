@@ -194,8 +194,11 @@ def test_backward_workspace_and_launch_counts(L):
     two = L.kda_prefill_backward_workspace_size(1, 128, 1, 1, 128, 128, 0)
     assert two - one >= 74240 + 2 * 65536
     assert L.kda_prefill_backward_workspace_size(1, 64, 1, 1, 64, 128, 0) == 0
-    assert L.kda_prefill_backward_kernel_launches(1, 64, 1, 1, 128, 128, 0) == 5
-    assert L.kda_prefill_backward_kernel_launches(1, 64, 1, 1, 128, 128, 3) == 6
+    # forward intra-chunk and carry, reverse carry, chunk gradients (+ chunk offsets when packed); with GQA
+    # (H < HV) also the kernel that sums each Q/K head's group through the normalisation's Jacobian
+    assert L.kda_prefill_backward_kernel_launches(1, 64, 1, 1, 128, 128, 0) == 4
+    assert L.kda_prefill_backward_kernel_launches(1, 64, 1, 1, 128, 128, 3) == 5
+    assert L.kda_prefill_backward_kernel_launches(1, 64, 1, 2, 128, 128, 0) == 5
 
 
 def test_saved_forward_and_backward_reject_small_or_overlapping_buffers(L):
