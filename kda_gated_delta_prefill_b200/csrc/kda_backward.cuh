@@ -312,8 +312,11 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
 }
 
 // ---------------------------------------------------------------------------------------------------------
-// Chunk gradients: one CTA of 256 threads per (chunk, value head); fp32 values, TF32 MMAs (fp32 accumulate).
-constexpr int kBwThreads = 256, kBwCols = 16;  // value columns per pass over the state
+// Chunk gradients: one CTA of 512 threads (16 warps) per (chunk, value head); fp32 values, TF32 MMAs (fp32
+// accumulate).  The MMA phases (the value-column passes and the pairwise terms) give each warp a row block and a
+// quarter of the columns; the phases written for 8 warps (gates, P/Aqk, the solve, dL) run on threads 0-255 while
+// the rest wait at the next barrier.  One CTA per SM: 16 warps hide more of the MMA chains' latency than 8.
+constexpr int kBwThreads = 512, kBwCols = 16;  // value columns per pass over the state
 constexpr int kRow = 132;                      // padded row stride (floats) of the [64][128] operand tiles
 constexpr int kRowC = 68;                      // padded row stride of the [64][64] tiles
 // element (r, c) of a [64][16] fp32 value-column tile: rows of 16 floats, the two 8-column halves swapped in
@@ -390,10 +393,10 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
 
     // ---- 1. gates: G = cumulative g, block references, beta ----
     // this warp's eight q and k rows, requested first so that their latency overlaps the gate work
-    uint2 rqv[CH / 8], rkv[CH / 8];
+    uint2 rqv[CH / 16], rkv[CH / 16];
 #pragma unroll
-    for (int m = 0; m < CH / 8; ++m) {
-        const int r = warp + 8 * m;
+    for (int m = 0; m < CH / 16; ++m) {
+        const int r = warp + 16 * m;
         rqv[m] = rkv[m] = make_uint2(0u, 0u);
         if (r < nvalid) {
             rqv[m] = *reinterpret_cast<const uint2 *>(p.q + ((row0 + r) * p.H + hq) * DK + 4 * lane);
@@ -401,10 +404,10 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         }
     }
     {
-        const int i = tid >> 2, c0 = 32 * (tid & 3);
+        const int i = tid >> 3, c0 = 16 * (tid & 7);
         const float *gr = p.g + ((row0 + i) * p.HV + h) * DK + c0;
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
+        for (int e = 0; e < 16; e += 4) {
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
             if (i < nvalid) x = *reinterpret_cast<const float4 *>(gr + e);
             *reinterpret_cast<float4 *>(&G[i][c0 + e]) = x;
@@ -437,8 +440,8 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     __syncthreads();
     // ---- normalised q/k rows and the gate-scaled operands ----
 #pragma unroll
-    for (int m = 0; m < CH / 8; ++m) {
-        const int r = warp + 8 * m;
+    for (int m = 0; m < CH / 16; ++m) {
+        const int r = warp + 16 * m;
         const uint2 rq = rqv[m], rk = rkv[m];
         // the forward's row denominators, kept to rebuild qn/kn bit for bit at the end
         const float dq = l2norm_den128_warp(rq), dk = l2norm_den128_warp(rk);
@@ -463,7 +466,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     __syncthreads();
 
     // ---- 2. P (j < i) and Aqk (j <= i); thread: rows 4rg..4rg+3 (block I), columns cg + 16 jb ----
-    {
+    if (tid < 256) {
         const int rg = tid >> 4, cg = tid & 15, I = rg >> 2;
         float pa[4][4] = {}, aa[4][4] = {};
         for (int d = 0; d < DK; d += 4) {
@@ -515,7 +518,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     //         column c, rows r4 + 4q; row m reaches the column's lanes by shuffle), then the blocks next to the
     //         diagonal T_{I,I-1} = -T_II L_{I,I-1} T_{I-1,I-1}, then the lower-left 32 x 32 block as
     //         -T_B (L_C T_A) with T_A, T_B the two 32 x 32 diagonal blocks ----
-    {
+    if (tid < 256) {
         const int I = tid >> 6, c = (tid >> 2) & 15, r4 = tid & 3;
         float x[4];
 #pragma unroll
@@ -536,7 +539,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     {
         // (the blocks above the diagonal of T are zero, so every sum below runs over a fixed range)
         float(*X)[16][16] = reinterpret_cast<float(*)[16][16]>(sm + S::WK);  // L_{I,I-1} T_{I-1,I-1}, I = 1..3
-        {
+        if (tid < 256) {
             const int i = (tid >> 4) & 15, j = tid & 15;  // this thread: element (i, j) of each of the three blocks
             float acc[3] = {};
 #pragma unroll
@@ -548,7 +551,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
             for (int b = 0; b < 3; ++b) X[b][i][j] = __fmul_rn(beta[16 * (b + 1) + i], acc[b]);
         }
         __syncthreads();
-        {
+        if (tid < 256) {
             const int i = (tid >> 4) & 15, j = tid & 15;
             float acc[3] = {};
 #pragma unroll
@@ -560,7 +563,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         }
         __syncthreads();
         float(*Y)[33] = reinterpret_cast<float(*)[33]>(sm + S::WK + 3 * 256 * 4);  // L_C T_A, [32][33]
-        {
+        if (tid < 256) {
             const int j = tid & 31, i0 = tid >> 5;  // this thread: rows i0 + 8 it, column j
             float acc[4] = {};
 #pragma unroll
@@ -573,7 +576,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
             for (int it = 0; it < 4; ++it) Y[i0 + 8 * it][j] = __fmul_rn(beta[32 + i0 + 8 * it], acc[it]);
         }
         __syncthreads();
-        {
+        if (tid < 256) {
             const int j = tid & 31, i0 = tid >> 5;
             float acc[4] = {};
 #pragma unroll
@@ -600,19 +603,23 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     const __nv_bfloat16 *Sg = p.states + item * DK * DV;
     const __nv_bfloat16 *dSg = p.dstates + item * DK * DV;
     const int rg = tid >> 4, cg = tid & 15;  // ownership of the 64 x 64 steps of phase 6
-    // MMA fragment ownership (g = lane / 4, t4 = lane % 4): warp (mt, nh) holds rows 16 mt + g and + 8, and key
-    // columns 64 nh + 8 j + 2 t4 (+1), j = 0..7 (dQg, dKb, dKg), or token columns 32 nh + 8 j + 2 t4 (+1),
-    // j = 0..3 (dAqk, dA)
+    // MMA fragment ownership (g = lane / 4, t4 = lane % 4): warp (mt, nh), nh = 0..3, holds rows 16 mt + g and + 8,
+    // and key columns 32 nh + 8 j + 2 t4 (+1), j = 0..3 (dQg, dKb, dKg), or token columns 16 nh + 8 j + 2 t4 (+1),
+    // j = 0..1 (dAqk, dA).  In steps (a)-(d) of a pass, warp (mt, role, ntw) = (warp % 4, warp / 4 % 2, warp / 8)
+    // computes rows 16 mt of the ntw-th 8-column tile of D and Vnew (role 0) or dVnew and dv (role 1).
     const int g = lane >> 2, t4 = lane & 3, mt = warp & 3, nh = warp >> 2;
+    const int role = (warp >> 2) & 1, ntw = warp >> 3;
     const int r0 = 16 * mt + g, r1 = r0 + 8;
     // bf16 values are exact in TF32 (8 of its 10 mantissa bits): the widened bits are the operand as they are
     auto bf = [](__nv_bfloat16 x) { return static_cast<uint32_t>(__bfloat16_as_ushort(x)) << 16; };
-    float aQ[8][4] = {}, aB[8][4] = {}, aG[8][4] = {}, aAq[4][4] = {}, aA[4][4] = {};
+    float aQ[4][4] = {}, aB[4][4] = {}, aG[4][4] = {}, aAq[2][4] = {}, aA[2][4] = {};
     // pass vb's columns into buffer b: S, dS' and dO rows are 32 bytes (two 16-byte copies each)
     auto fetch = [&](int vb, int b) {
         const int row = tid >> 1, half = 8 * (tid & 1);
-        cp_async16(smem_u32(&SVb(b)[row][bsw(row, half)]), Sg + row * DV + vb + half);
-        cp_async16(smem_u32(&DSVb(b)[row][bsw(row, half)]), dSg + row * DV + vb + half);
+        if (tid < 256) {
+            cp_async16(smem_u32(&SVb(b)[row][bsw(row, half)]), Sg + row * DV + vb + half);
+            cp_async16(smem_u32(&DSVb(b)[row][bsw(row, half)]), dSg + row * DV + vb + half);
+        }
         if (row < nvalid && tid < 2 * CH)
             cp_async16(smem_u32(&DOBb(b)[row][bsw(row, half)]), p.dout + ((row0 + row) * p.HV + h) * DV + vb + half);
         cp_async_commit();
@@ -646,94 +653,78 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 gl_acc = __fmaf_rn(x.y, y.y, __fmaf_rn(x.x, y.x, gl_acc));
             }
         }
-        if (warp < 4) {
-            // (a) D = v - Kb S for rows 16 mt .. (Kb = KA exp(m_I), block I = mt), two n8 tiles of columns
-            float c[2][4] = {};
+        const int cn = 8 * ntw + g;  // this warp's tile: B-fragment column of steps (a)-(d)
+        if (role == 0) {
+            // (a) D = v - Kb S for rows 16 mt .. (Kb = KA exp(m_I), block I = mt), columns 8 ntw ..
+            float c[4] = {};
             for (int ks = 0; ks < DK; ks += 8) {
                 const float e0 = EM[mt][ks + t4], e1 = EM[mt][ks + t4 + 4];
                 const uint32_t a[4] = {to_tf32(__fmul_rn(KA[r0][ks + t4], e0)), to_tf32(__fmul_rn(KA[r1][ks + t4], e0)),
                                        to_tf32(__fmul_rn(KA[r0][ks + t4 + 4], e1)),
                                        to_tf32(__fmul_rn(KA[r1][ks + t4 + 4], e1))};
                 const int k0 = ks + t4, k1 = ks + t4 + 4;
-                mma_tf32(c[0], a, bf(SVT[k0][bsw(k0, g)]), bf(SVT[k1][bsw(k1, g)]));
-                mma_tf32(c[1], a, bf(SVT[k0][bsw(k0, 8 + g)]), bf(SVT[k1][bsw(k1, 8 + g)]));
+                mma_tf32(c, a, bf(SVT[k0][bsw(k0, cn)]), bf(SVT[k1][bsw(k1, cn)]));
             }
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int i = hf ? r1 : r0, cc = 8 * nt + 2 * t4;
-                    float2 vv = make_float2(0.f, 0.f);
-                    if (i < nvalid)
-                        vv = __bfloat1622float2(
-                            *reinterpret_cast<const __nv_bfloat162 *>(p.v + ((row0 + i) * p.HV + h) * DV + vb + cc));
-                    *reinterpret_cast<float2 *>(&DDv[vsw(i, cc)]) =
-                        make_float2(__fsub_rn(vv.x, c[nt][2 * hf]), __fsub_rn(vv.y, c[nt][2 * hf + 1]));
-                }
+            for (int hf = 0; hf < 2; ++hf) {
+                const int i = hf ? r1 : r0, cc = 8 * ntw + 2 * t4;
+                float2 vv = make_float2(0.f, 0.f);
+                if (i < nvalid)
+                    vv = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162 *>(p.v + ((row0 + i) * p.HV + h) * DV + vb + cc));
+                *reinterpret_cast<float2 *>(&DDv[vsw(i, cc)]) =
+                    make_float2(__fsub_rn(vv.x, c[2 * hf]), __fsub_rn(vv.y, c[2 * hf + 1]));
+            }
         } else {
-            // (c) dVnew = Kg dS' + Aqk^T dO for rows 16 mt .. (Kg = KB exp(G_L - m_I))
-            float c[2][4] = {};
+            // (c) dVnew = Kg dS' + Aqk^T dO for rows 16 mt .. (Kg = KB exp(G_L - m_I)), columns 8 ntw ..
+            float c[4] = {};
             for (int ks = 0; ks < DK; ks += 8) {
                 const float e0 = EGLM[mt][ks + t4], e1 = EGLM[mt][ks + t4 + 4];
                 const uint32_t a[4] = {to_tf32(__fmul_rn(KB[r0][ks + t4], e0)), to_tf32(__fmul_rn(KB[r1][ks + t4], e0)),
                                        to_tf32(__fmul_rn(KB[r0][ks + t4 + 4], e1)),
                                        to_tf32(__fmul_rn(KB[r1][ks + t4 + 4], e1))};
                 const int k0 = ks + t4, k1 = ks + t4 + 4;
-                mma_tf32(c[0], a, bf(DST[k0][bsw(k0, g)]), bf(DST[k1][bsw(k1, g)]));
-                mma_tf32(c[1], a, bf(DST[k0][bsw(k0, 8 + g)]), bf(DST[k1][bsw(k1, 8 + g)]));
+                mma_tf32(c, a, bf(DST[k0][bsw(k0, cn)]), bf(DST[k1][bsw(k1, cn)]));
             }
             for (int js = 16 * mt; js < CH; js += 8) {  // Aqk^T[i][j] = Aqk[j][i], nonzero for j >= i
                 const uint32_t a[4] = {to_tf32(AQ[js + t4][r0]), to_tf32(AQ[js + t4][r1]), to_tf32(AQ[js + t4 + 4][r0]),
                                        to_tf32(AQ[js + t4 + 4][r1])};
                 const int k0 = js + t4, k1 = js + t4 + 4;
-                mma_tf32(c[0], a, bf(DOV[k0][bsw(k0, g)]), bf(DOV[k1][bsw(k1, g)]));
-                mma_tf32(c[1], a, bf(DOV[k0][bsw(k0, 8 + g)]), bf(DOV[k1][bsw(k1, 8 + g)]));
+                mma_tf32(c, a, bf(DOV[k0][bsw(k0, cn)]), bf(DOV[k1][bsw(k1, cn)]));
             }
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                *reinterpret_cast<float2 *>(&DVN[vsw(r0, 8 * nt + 2 * t4)]) = make_float2(c[nt][0], c[nt][1]);
-                *reinterpret_cast<float2 *>(&DVN[vsw(r1, 8 * nt + 2 * t4)]) = make_float2(c[nt][2], c[nt][3]);
-            }
+            *reinterpret_cast<float2 *>(&DVN[vsw(r0, 8 * ntw + 2 * t4)]) = make_float2(c[0], c[1]);
+            *reinterpret_cast<float2 *>(&DVN[vsw(r1, 8 * ntw + 2 * t4)]) = make_float2(c[2], c[3]);
         }
         __syncthreads();
-        if (warp < 4) {
+        if (role == 0) {
             // (b) Vnew = T diag(beta) D (T lower triangular: j < 16 (mt + 1))
-            float c[2][4] = {};
+            float c[4] = {};
             for (int js = 0; js < 16 * (mt + 1); js += 8) {
                 const float b0 = beta[js + t4], b1 = beta[js + t4 + 4];
                 const uint32_t a[4] = {to_tf32(__fmul_rn(TT[r0][js + t4], b0)), to_tf32(__fmul_rn(TT[r1][js + t4], b0)),
                                        to_tf32(__fmul_rn(TT[r0][js + t4 + 4], b1)),
                                        to_tf32(__fmul_rn(TT[r1][js + t4 + 4], b1))};
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-                    mma_tf32(c[nt], a, to_tf32(DDv[vsw(js + t4, 8 * nt + g)]), to_tf32(DDv[vsw(js + t4 + 4, 8 * nt + g)]));
+                mma_tf32(c, a, to_tf32(DDv[vsw(js + t4, cn)]), to_tf32(DDv[vsw(js + t4 + 4, cn)]));
             }
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                *reinterpret_cast<float2 *>(&VN[vsw(r0, 8 * nt + 2 * t4)]) = make_float2(c[nt][0], c[nt][1]);
-                *reinterpret_cast<float2 *>(&VN[vsw(r1, 8 * nt + 2 * t4)]) = make_float2(c[nt][2], c[nt][3]);
-            }
+            *reinterpret_cast<float2 *>(&VN[vsw(r0, 8 * ntw + 2 * t4)]) = make_float2(c[0], c[1]);
+            *reinterpret_cast<float2 *>(&VN[vsw(r1, 8 * ntw + 2 * t4)]) = make_float2(c[2], c[3]);
         } else {
             // (d) dv = diag(beta) T^T dVnew (j >= i)
-            float c[2][4] = {};
+            float c[4] = {};
             for (int js = 16 * mt; js < CH; js += 8) {
                 const uint32_t a[4] = {to_tf32(TT[js + t4][r0]), to_tf32(TT[js + t4][r1]), to_tf32(TT[js + t4 + 4][r0]),
                                        to_tf32(TT[js + t4 + 4][r1])};
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-                    mma_tf32(c[nt], a, to_tf32(DVN[vsw(js + t4, 8 * nt + g)]), to_tf32(DVN[vsw(js + t4 + 4, 8 * nt + g)]));
+                mma_tf32(c, a, to_tf32(DVN[vsw(js + t4, cn)]), to_tf32(DVN[vsw(js + t4 + 4, cn)]));
             }
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int i = hf ? r1 : r0, cc = 8 * nt + 2 * t4;
-                    const float x0 = __fmul_rn(beta[i], c[nt][2 * hf]), x1 = __fmul_rn(beta[i], c[nt][2 * hf + 1]);
-                    *reinterpret_cast<float2 *>(&DVv[vsw(i, cc)]) = make_float2(x0, x1);
-                    if (i < nvalid)
-                        *reinterpret_cast<__nv_bfloat162 *>(p.dv + ((row0 + i) * p.HV + h) * DV + vb + cc) =
-                            __floats2bfloat162_rn(x0, x1);
-                }
+            for (int hf = 0; hf < 2; ++hf) {
+                const int i = hf ? r1 : r0, cc = 8 * ntw + 2 * t4;
+                const float x0 = __fmul_rn(beta[i], c[2 * hf]), x1 = __fmul_rn(beta[i], c[2 * hf + 1]);
+                *reinterpret_cast<float2 *>(&DVv[vsw(i, cc)]) = make_float2(x0, x1);
+                if (i < nvalid)
+                    *reinterpret_cast<__nv_bfloat162 *>(p.dv + ((row0 + i) * p.HV + h) * DV + vb + cc) =
+                        __floats2bfloat162_rn(x0, x1);
+            }
         }
         __syncthreads();
         // (e) dQg += dO S^T, dKb -= dv S^T, dKg += Vnew dS'^T (K = these 16 columns, two k8 steps);
@@ -759,16 +750,16 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
             const uint32_t aN[4] = {to_tf32(n0.x), to_tf32(n1.x), to_tf32(n0.y), to_tf32(n1.y)};
             const uint32_t aD[4] = {to_tf32(e0.x), to_tf32(e1.x), to_tf32(e0.y), to_tf32(e1.y)};
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int d = 64 * nh + 8 * j + g;
+            for (int j = 0; j < 4; ++j) {
+                const int d = 32 * nh + 8 * j + g;
                 const uint32_t sp = pair(SVT, d, cp), qp = pair(DST, d, cp);
                 mma_tf32(aQ[j], aO, sp << 16, sp & kHi);
                 mma_tf32(aB[j], aV, sp << 16, sp & kHi);
                 mma_tf32(aG[j], aN, qp << 16, qp & kHi);
             }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int tk = 32 * nh + 8 * j + g;
+            for (int j = 0; j < 2; ++j) {
+                const int tk = 16 * nh + 8 * j + g;
                 const float2 vn = *reinterpret_cast<const float2 *>(&VN[vsw(tk, cp)]);
                 const float2 dd = *reinterpret_cast<const float2 *>(&DDv[vsw(tk, cp)]);
                 mma_tf32(aAq[j], aO, to_tf32(vn.x), to_tf32(vn.y));
@@ -783,10 +774,10 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     // ---- 6. dbeta, dL, M = diag(beta) dL, N = dAqk ----
     float(*DA)[kRowC] = reinterpret_cast<float(*)[kRowC]>(sm + S::DA);
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < 2; ++j)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int i = (q >> 1) ? r1 : r0, tk = 32 * nh + 8 * j + 2 * t4 + (q & 1);
+            const int i = (q >> 1) ? r1 : r0, tk = 16 * nh + 8 * j + 2 * t4 + (q & 1);
             DA[i][tk] = aA[j][q];
             AQ[i][tk] = tk <= i ? aAq[j][q] : 0.f;  // Aqk is no longer needed: N takes its place
         }
@@ -796,77 +787,86 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         for (int i = tid; i < CH; ++i) acc = __fmaf_rn(DA[i][tid], TT[i][tid], acc);
         dbeta[tid] = acc;
     }
-    // Y = T^T (dA diag(beta)): Y[a][e] = beta_e sum_{c >= a} T[c][a] dA[c][e]
+    // Y = T^T (dA diag(beta)): Y[a][e] = beta_e sum_{c >= a} T[c][a] dA[c][e]  (threads 0-255: rows 4rg.., columns cg + 16 jb)
+    const bool g64 = tid < 256;
     float y[4][4] = {};
-    for (int c = 4 * rg; c < CH; ++c) {
+    if (g64) {
+        for (int c = 4 * rg; c < CH; ++c) {
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-            const float t = TT[c][4 * rg + ii];
+            for (int ii = 0; ii < 4; ++ii) {
+                const float t = TT[c][4 * rg + ii];
 #pragma unroll
-            for (int jb = 0; jb < 4; ++jb) y[ii][jb] = __fmaf_rn(t, DA[c][cg + 16 * jb], y[ii][jb]);
+                for (int jb = 0; jb < 4; ++jb) y[ii][jb] = __fmaf_rn(t, DA[c][cg + 16 * jb], y[ii][jb]);
+            }
         }
     }
     __syncthreads();  // every read of dA is done
+    if (g64) {
 #pragma unroll
-    for (int ii = 0; ii < 4; ++ii)
+        for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-        for (int jb = 0; jb < 4; ++jb) DA[4 * rg + ii][cg + 16 * jb] = __fmul_rn(beta[cg + 16 * jb], y[ii][jb]);
+            for (int jb = 0; jb < 4; ++jb) DA[4 * rg + ii][cg + 16 * jb] = __fmul_rn(beta[cg + 16 * jb], y[ii][jb]);
+    }
     __syncthreads();
     // dL[a][b] = -sum_{e <= b} Y[a][e] T[b][e] (a > b); dbeta_a += sum_b dL_ab P_ab; M = diag(beta) dL
     {
-        float dl[4][4] = {};
-        for (int e = 0; e < CH; ++e) {
-            float ye[4];
+        float dl[4][4] = {}, rowp[4] = {};
+        if (g64) {
+            for (int e = 0; e < CH; ++e) {
+                float ye[4];
 #pragma unroll
-            for (int ii = 0; ii < 4; ++ii) ye[ii] = DA[4 * rg + ii][e];
+                for (int ii = 0; ii < 4; ++ii) ye[ii] = DA[4 * rg + ii][e];
 #pragma unroll
-            for (int jb = 0; jb < 4; ++jb) {
-                const float t = TT[cg + 16 * jb][e];  // zero for e > b
+                for (int jb = 0; jb < 4; ++jb) {
+                    const float t = TT[cg + 16 * jb][e];  // zero for e > b
 #pragma unroll
-                for (int ii = 0; ii < 4; ++ii) dl[ii][jb] = __fmaf_rn(-ye[ii], t, dl[ii][jb]);
+                    for (int ii = 0; ii < 4; ++ii) dl[ii][jb] = __fmaf_rn(-ye[ii], t, dl[ii][jb]);
+                }
             }
-        }
-        float rowp[4] = {};
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
+            for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-            for (int jb = 0; jb < 4; ++jb) {
-                const int a = 4 * rg + ii, b = cg + 16 * jb;
-                if (b < a) rowp[ii] = __fmaf_rn(dl[ii][jb], PP[a][b], rowp[ii]);
-                else dl[ii][jb] = 0.f;
+                for (int jb = 0; jb < 4; ++jb) {
+                    const int a = 4 * rg + ii, b = cg + 16 * jb;
+                    if (b < a) rowp[ii] = __fmaf_rn(dl[ii][jb], PP[a][b], rowp[ii]);
+                    else dl[ii][jb] = 0.f;
+                }
+            // the 16 threads of a row group are 16 consecutive lanes
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) {
+#pragma unroll
+                for (int off = 8; off > 0; off >>= 1)
+                    rowp[ii] = __fadd_rn(rowp[ii], __shfl_xor_sync(0xffffffffu, rowp[ii], off));
             }
-        // the 16 threads of a row group are 16 consecutive lanes
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-#pragma unroll
-            for (int off = 8; off > 0; off >>= 1) rowp[ii] = __fadd_rn(rowp[ii], __shfl_xor_sync(0xffffffffu, rowp[ii], off));
         }
         __syncthreads();  // every read of P and T is done (dbeta's column sums above included)
-        if (cg == 0) {
+        if (g64) {
+            if (cg == 0) {
 #pragma unroll
-            for (int ii = 0; ii < 4; ++ii) atomicAdd(&dbeta[4 * rg + ii], rowp[ii]);
+                for (int ii = 0; ii < 4; ++ii) atomicAdd(&dbeta[4 * rg + ii], rowp[ii]);
+            }
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                for (int jb = 0; jb < 4; ++jb) PP[4 * rg + ii][cg + 16 * jb] = __fmul_rn(beta[4 * rg + ii], dl[ii][jb]);
         }
-#pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-            for (int jb = 0; jb < 4; ++jb) PP[4 * rg + ii][cg + 16 * jb] = __fmul_rn(beta[4 * rg + ii], dl[ii][jb]);
     }
     __syncthreads();
     float(*MM)[kRowC] = PP;
     float(*NN)[kRowC] = AQ;
 
     // ---- 7. element terms and pairwise terms, in the fragment ownership of phase 5 ----
-    float rq[8][4], rk[8][4], rG[8][4];
+    float rq[4][4], rk[4][4], rG[4][4];
     {
         // qn/kn of the owned elements, rebuilt from the raw rows (the same normalisation, bit for bit)
-        float glp[8][2] = {};
+        float glp[4][2] = {};
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             const int i = hf ? r1 : r0;
             const float dq = denq[i], dk = denk[i], rqi = __frcp_rn(dq), rki = __frcp_rn(dk);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int d = 64 * nh + 8 * j + 2 * t4;
+            for (int j = 0; j < 4; ++j) {
+                const int d = 32 * nh + 8 * j + 2 * t4;
                 uint32_t wq = 0u, wk = 0u;
                 if (i < nvalid) {
                     wq = *reinterpret_cast<const uint32_t *>(p.q + ((row0 + i) * p.H + hq) * DK + d);
@@ -895,19 +895,19 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         // barrier) the four row blocks' partial sums, kept in the work region (free since phase 6)
         float(*glpart)[DK] = reinterpret_cast<float(*)[DK]>(sm + S::WK);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 float x = glp[j][e];
                 x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, 4));
                 x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, 8));
                 x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, 16));
-                if (g == 0) glpart[mt][64 * nh + 8 * j + 2 * t4 + e] = x;
+                if (g == 0) glpart[mt][32 * nh + 8 * j + 2 * t4 + e] = x;
             }
     }
     {
         // R1'_id = sum_{J <= I} sum_{j in J} M_ij KB_jd c_IJd and R3' the same with N (I = mt)
-        float ra[8][4] = {}, rb[8][4] = {};
+        float ra[4][4] = {}, rb[4][4] = {};
         for (int J = 0; J <= mt; ++J) {
             const float *cf = J < mt ? CF[cf_index(mt, J)] : nullptr;
             for (int ks = 16 * J; ks < 16 * J + 16; ks += 8) {
@@ -916,8 +916,8 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 const uint32_t an[4] = {to_tf32(NN[r0][ks + t4]), to_tf32(NN[r1][ks + t4]), to_tf32(NN[r0][ks + t4 + 4]),
                                         to_tf32(NN[r1][ks + t4 + 4])};
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int d = 64 * nh + 8 * j + g;
+                for (int j = 0; j < 4; ++j) {
+                    const int d = 32 * nh + 8 * j + g;
                     float b0 = KB[ks + t4][d], b1 = KB[ks + t4 + 4][d];
                     if (cf) {
                         b0 = __fmul_rn(b0, cf[d]);
@@ -931,10 +931,10 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         }
         // R1 = a R1', R3 = s a R3' (a = exp(G - m_I)): dkn += R1, dqn += R3, dG += kn R1 + qn R3
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const int i = (q >> 1) ? r1 : r0, d = 64 * nh + 8 * j + 2 * t4 + (q & 1);
+                const int i = (q >> 1) ? r1 : r0, d = 32 * nh + 8 * j + 2 * t4 + (q & 1);
                 const float a = bwd_exp(__fsub_rn(G[i][d], G[16 * mt + 7][d]));
                 rk[j][q] = __fmaf_rn(a, ra[j][q], rk[j][q]);
                 rq[j][q] = __fmaf_rn(__fmul_rn(s, a), rb[j][q], rq[j][q]);
@@ -944,7 +944,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     }
     {
         // R24'_jd = sum_{I' >= J} sum_{i in I'} (M_ij KA_id + s N_ij QA_id) c_I'Jd for rows j of block J = mt
-        float ra[8][4] = {};
+        float ra[4][4] = {};
         for (int I2 = mt; I2 < 4; ++I2) {
             const float *cf = I2 > mt ? CF[cf_index(I2, mt)] : nullptr;
             for (int ks = 16 * I2; ks < 16 * I2 + 16; ks += 8) {
@@ -953,8 +953,8 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 const uint32_t an[4] = {to_tf32(NN[ks + t4][r0]), to_tf32(NN[ks + t4][r1]), to_tf32(NN[ks + t4 + 4][r0]),
                                         to_tf32(NN[ks + t4 + 4][r1])};
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int d = 64 * nh + 8 * j + g;
+                for (int j = 0; j < 4; ++j) {
+                    const int d = 32 * nh + 8 * j + g;
                     float k0 = KA[ks + t4][d], k1 = KA[ks + t4 + 4][d];
                     float q0 = __fmul_rn(s, QA[ks + t4][d]), q1 = __fmul_rn(s, QA[ks + t4 + 4][d]);
                     if (cf) {
@@ -971,10 +971,10 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         }
         // R24 = b R24' (b = exp(m_J - G)): dkn += R24, dG -= kn R24 = KB R24'
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const int i = (q >> 1) ? r1 : r0, d = 64 * nh + 8 * j + 2 * t4 + (q & 1);
+                const int i = (q >> 1) ? r1 : r0, d = 32 * nh + 8 * j + 2 * t4 + (q & 1);
                 const float b = bwd_exp(__fsub_rn(G[16 * mt + 7][d], G[i][d]));
                 rk[j][q] = __fmaf_rn(b, ra[j][q], rk[j][q]);
                 rG[j][q] = __fmaf_rn(-KB[i][d], ra[j][q], rG[j][q]);
@@ -982,17 +982,17 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     }
     // dqn, dkn out (valid rows), for kda_bwd_norm_kernel; or, with one value head per Q/K head, dq and dk here:
     // dx = dy / n - x (x . dy) / n^3 (n: the row's denominator of the forward's normalisation), with x . dy
-    // summed by the four lanes that share a row in this warp and then across the two warps that hold its halves.
+    // summed by the four lanes that share a row in this warp and then across the four warps that hold its quarters.
     float xdy[2][2] = {};  // [row r0 / r1][q / k] partial x . dy of this thread's 16 columns
     if (!p.fuse_norm) {
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             const int i = hf ? r1 : r0;
             if (i < nvalid) {
-                float *dq = p.dqn + ((row0 + i) * p.HV + h) * DK + 64 * nh + 2 * t4;
-                float *dk = p.dkn + ((row0 + i) * p.HV + h) * DK + 64 * nh + 2 * t4;
+                float *dq = p.dqn + ((row0 + i) * p.HV + h) * DK + 32 * nh + 2 * t4;
+                float *dk = p.dkn + ((row0 + i) * p.HV + h) * DK + 32 * nh + 2 * t4;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < 4; ++j) {
                     *reinterpret_cast<float2 *>(dq + 8 * j) = make_float2(rq[j][2 * hf], rq[j][2 * hf + 1]);
                     *reinterpret_cast<float2 *>(dk + 8 * j) = make_float2(rk[j][2 * hf], rk[j][2 * hf + 1]);
                 }
@@ -1004,8 +1004,8 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
             const int i = hf ? r1 : r0;
             if (i < nvalid) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int64_t off = ((row0 + i) * p.H + hq) * DK + 64 * nh + 8 * j + 2 * t4;
+                for (int j = 0; j < 4; ++j) {
+                    const int64_t off = ((row0 + i) * p.H + hq) * DK + 32 * nh + 8 * j + 2 * t4;
                     const uint32_t wq = *reinterpret_cast<const uint32_t *>(p.q + off);
                     const uint32_t wk = *reinterpret_cast<const uint32_t *>(p.k + off);
                     xdy[hf][0] = __fmaf_rn(bf16lo(wq), rq[j][2 * hf], xdy[hf][0]);
@@ -1023,24 +1023,25 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     }
     __syncthreads();  // KA/QA/KB/G reads done; dgl complete
     if (p.fuse_norm) {
-        float *red = reinterpret_cast<float *>(sm + S::EM);  // [q|k][row][half]; exp(m_I) is no longer read
+        float *red = reinterpret_cast<float *>(sm + S::EM);  // [q|k][row][quarter]; exp(m_I) is no longer read
         if (t4 == 0) {
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-                for (int w = 0; w < 2; ++w) red[(w * CH + (hf ? r1 : r0)) * 2 + nh] = xdy[hf][w];
+                for (int w = 0; w < 2; ++w) red[(w * CH + (hf ? r1 : r0)) * 4 + nh] = xdy[hf][w];
         }
         __syncthreads();
         // row i's half of dx from dy = this thread's columns of dqn (or dkn), w = 0 (q) or 1 (k)
-        auto emit = [&](const float (&dy)[8][4], int hf, int w, const __nv_bfloat16 *x, __nv_bfloat16 *dx,
+        auto emit = [&](const float (&dy)[4][4], int hf, int w, const __nv_bfloat16 *x, __nv_bfloat16 *dx,
                         float den) {
             const int i = hf ? r1 : r0;
-            const float tot = __fadd_rn(red[(w * CH + i) * 2], red[(w * CH + i) * 2 + 1]);
+            const float *rr = red + (w * CH + i) * 4;
+            const float tot = __fadd_rn(__fadd_rn(rr[0], rr[1]), __fadd_rn(rr[2], rr[3]));
             const float inv = __frcp_rn(den);
             const float c3 = __fmul_rn(tot, __fmul_rn(inv, __fmul_rn(inv, inv)));
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int64_t off = ((row0 + i) * p.H + hq) * DK + 64 * nh + 8 * j + 2 * t4;
+            for (int j = 0; j < 4; ++j) {
+                const int64_t off = ((row0 + i) * p.H + hq) * DK + 32 * nh + 8 * j + 2 * t4;
                 const uint32_t wx = *reinterpret_cast<const uint32_t *>(x + off);
                 const float o0 = __fmaf_rn(-bf16lo(wx), c3, __fmul_rn(dy[j][2 * hf], inv));
                 const float o1 = __fmaf_rn(-bf16hi(wx), c3, __fmul_rn(dy[j][2 * hf + 1], inv));
@@ -1059,9 +1060,9 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     // dG rows into the KA region (unpadded [64][128]), then the reverse cumulative sum per key column
     float(*dG)[DK] = reinterpret_cast<float(*)[DK]>(sm + S::KA);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        *reinterpret_cast<float2 *>(&dG[r0][64 * nh + 8 * j + 2 * t4]) = make_float2(rG[j][0], rG[j][1]);
-        *reinterpret_cast<float2 *>(&dG[r1][64 * nh + 8 * j + 2 * t4]) = make_float2(rG[j][2], rG[j][3]);
+    for (int j = 0; j < 4; ++j) {
+        *reinterpret_cast<float2 *>(&dG[r0][32 * nh + 8 * j + 2 * t4]) = make_float2(rG[j][0], rG[j][1]);
+        *reinterpret_cast<float2 *>(&dG[r1][32 * nh + 8 * j + 2 * t4]) = make_float2(rG[j][2], rG[j][3]);
     }
     __syncthreads();
     if (tid < DK) {
