@@ -465,7 +465,9 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     }
     __syncthreads();
 
-    // ---- 2. P (j < i) and Aqk (j <= i); thread: rows 4rg..4rg+3 (block I), columns cg + 16 jb ----
+    // ---- 2. P (j < i) and Aqk (j <= i); thread: rows 4rg..4rg+3 (block I), columns cg + 16 jb (threads 0-255:
+    //         with more threads each would reread the same q/k rows for fewer column blocks, and the phase is
+    //         bound by those shared-memory reads) ----
     if (tid < 256) {
         const int rg = tid >> 4, cg = tid & 15, I = rg >> 2;
         float pa[4][4] = {}, aa[4][4] = {};
@@ -563,30 +565,30 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         }
         __syncthreads();
         float(*Y)[33] = reinterpret_cast<float(*)[33]>(sm + S::WK + 3 * 256 * 4);  // L_C T_A, [32][33]
-        if (tid < 256) {
-            const int j = tid & 31, i0 = tid >> 5;  // this thread: rows i0 + 8 it, column j
-            float acc[4] = {};
+        {
+            const int j = tid & 31, i0 = tid >> 5;  // this thread: rows i0 + 16 it, column j
+            float acc[2] = {};
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
                 const float tk = TT[k][j];
 #pragma unroll
-                for (int it = 0; it < 4; ++it) acc[it] = __fmaf_rn(PP[32 + i0 + 8 * it][k], tk, acc[it]);
+                for (int it = 0; it < 2; ++it) acc[it] = __fmaf_rn(PP[32 + i0 + 16 * it][k], tk, acc[it]);
             }
 #pragma unroll
-            for (int it = 0; it < 4; ++it) Y[i0 + 8 * it][j] = __fmul_rn(beta[32 + i0 + 8 * it], acc[it]);
+            for (int it = 0; it < 2; ++it) Y[i0 + 16 * it][j] = __fmul_rn(beta[32 + i0 + 16 * it], acc[it]);
         }
         __syncthreads();
-        if (tid < 256) {
+        {
             const int j = tid & 31, i0 = tid >> 5;
-            float acc[4] = {};
+            float acc[2] = {};
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
                 const float yk = Y[k][j];
 #pragma unroll
-                for (int it = 0; it < 4; ++it) acc[it] = __fmaf_rn(TT[32 + i0 + 8 * it][32 + k], yk, acc[it]);
+                for (int it = 0; it < 2; ++it) acc[it] = __fmaf_rn(TT[32 + i0 + 16 * it][32 + k], yk, acc[it]);
             }
 #pragma unroll
-            for (int it = 0; it < 4; ++it) TT[32 + i0 + 8 * it][j] = -acc[it];
+            for (int it = 0; it < 2; ++it) TT[32 + i0 + 16 * it][j] = -acc[it];
         }
         __syncthreads();
     }
@@ -602,7 +604,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     float *DVv = reinterpret_cast<float *>(sm + S::DV);
     const __nv_bfloat16 *Sg = p.states + item * DK * DV;
     const __nv_bfloat16 *dSg = p.dstates + item * DK * DV;
-    const int rg = tid >> 4, cg = tid & 15;  // ownership of the 64 x 64 steps of phase 6
+    const int cg = tid & 15;  // column of the 64 x 64 steps of phase 6 (with the row group and half below)
     // MMA fragment ownership (g = lane / 4, t4 = lane % 4): warp (mt, nh), nh = 0..3, holds rows 16 mt + g and + 8,
     // and key columns 32 nh + 8 j + 2 t4 (+1), j = 0..3 (dQg, dKb, dKg), or token columns 16 nh + 8 j + 2 t4 (+1),
     // j = 0..1 (dAqk, dA).  In steps (a)-(d) of a pass, warp (mt, role, ntw) = (warp % 4, warp / 4 % 2, warp / 8)
@@ -787,69 +789,68 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         for (int i = tid; i < CH; ++i) acc = __fmaf_rn(DA[i][tid], TT[i][tid], acc);
         dbeta[tid] = acc;
     }
-    // Y = T^T (dA diag(beta)): Y[a][e] = beta_e sum_{c >= a} T[c][a] dA[c][e]  (threads 0-255: rows 4rg.., columns cg + 16 jb)
-    const bool g64 = tid < 256;
-    float y[4][4] = {};
-    if (g64) {
-        for (int c = 4 * rg; c < CH; ++c) {
+    // Y = T^T (dA diag(beta)): Y[a][e] = beta_e sum_{c >= a} T[c][a] dA[c][e].  Thread: rows 4 rg6 .. 4 rg6 + 3
+    // and columns cg + 16 jb for the two column blocks jb = 2 jh, 2 jh + 1 of its half of the CTA.
+    const int rg6 = (tid >> 4) & 15, jh = tid >> 8;
+    float y[4][2] = {};
+    for (int c = 4 * rg6; c < CH; ++c) {
 #pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
-                const float t = TT[c][4 * rg + ii];
+        for (int ii = 0; ii < 4; ++ii) {
+            const float t = TT[c][4 * rg6 + ii];
 #pragma unroll
-                for (int jb = 0; jb < 4; ++jb) y[ii][jb] = __fmaf_rn(t, DA[c][cg + 16 * jb], y[ii][jb]);
-            }
+            for (int jj = 0; jj < 2; ++jj) y[ii][jj] = __fmaf_rn(t, DA[c][cg + 16 * (2 * jh + jj)], y[ii][jj]);
         }
     }
     __syncthreads();  // every read of dA is done
-    if (g64) {
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
+    for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-            for (int jb = 0; jb < 4; ++jb) DA[4 * rg + ii][cg + 16 * jb] = __fmul_rn(beta[cg + 16 * jb], y[ii][jb]);
-    }
+        for (int jj = 0; jj < 2; ++jj) {
+            const int col = cg + 16 * (2 * jh + jj);
+            DA[4 * rg6 + ii][col] = __fmul_rn(beta[col], y[ii][jj]);
+        }
     __syncthreads();
     // dL[a][b] = -sum_{e <= b} Y[a][e] T[b][e] (a > b); dbeta_a += sum_b dL_ab P_ab; M = diag(beta) dL
     {
-        float dl[4][4] = {}, rowp[4] = {};
-        if (g64) {
-            for (int e = 0; e < CH; ++e) {
-                float ye[4];
+        float *rowp2 = reinterpret_cast<float *>(sm + S::DA + CH * kRowC * 4);  // [2 halves][64 rows]
+        float dl[4][2] = {}, rowp[4] = {};
+        for (int e = 0; e < CH; ++e) {
+            float ye[4];
 #pragma unroll
-                for (int ii = 0; ii < 4; ++ii) ye[ii] = DA[4 * rg + ii][e];
+            for (int ii = 0; ii < 4; ++ii) ye[ii] = DA[4 * rg6 + ii][e];
 #pragma unroll
-                for (int jb = 0; jb < 4; ++jb) {
-                    const float t = TT[cg + 16 * jb][e];  // zero for e > b
+            for (int jj = 0; jj < 2; ++jj) {
+                const float t = TT[cg + 16 * (2 * jh + jj)][e];  // zero for e > b
 #pragma unroll
-                    for (int ii = 0; ii < 4; ++ii) dl[ii][jb] = __fmaf_rn(-ye[ii], t, dl[ii][jb]);
-                }
-            }
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-                for (int jb = 0; jb < 4; ++jb) {
-                    const int a = 4 * rg + ii, b = cg + 16 * jb;
-                    if (b < a) rowp[ii] = __fmaf_rn(dl[ii][jb], PP[a][b], rowp[ii]);
-                    else dl[ii][jb] = 0.f;
-                }
-            // the 16 threads of a row group are 16 consecutive lanes
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
-#pragma unroll
-                for (int off = 8; off > 0; off >>= 1)
-                    rowp[ii] = __fadd_rn(rowp[ii], __shfl_xor_sync(0xffffffffu, rowp[ii], off));
+                for (int ii = 0; ii < 4; ++ii) dl[ii][jj] = __fmaf_rn(-ye[ii], t, dl[ii][jj]);
             }
         }
-        __syncthreads();  // every read of P and T is done (dbeta's column sums above included)
-        if (g64) {
-            if (cg == 0) {
 #pragma unroll
-                for (int ii = 0; ii < 4; ++ii) atomicAdd(&dbeta[4 * rg + ii], rowp[ii]);
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int a = 4 * rg6 + ii, b = cg + 16 * (2 * jh + jj);
+                if (b < a) rowp[ii] = __fmaf_rn(dl[ii][jj], PP[a][b], rowp[ii]);
+                else dl[ii][jj] = 0.f;
             }
+        // the 16 threads of a row group are 16 consecutive lanes
 #pragma unroll
-            for (int ii = 0; ii < 4; ++ii)
+        for (int ii = 0; ii < 4; ++ii) {
 #pragma unroll
-                for (int jb = 0; jb < 4; ++jb) PP[4 * rg + ii][cg + 16 * jb] = __fmul_rn(beta[4 * rg + ii], dl[ii][jb]);
+            for (int off = 8; off > 0; off >>= 1)
+                rowp[ii] = __fadd_rn(rowp[ii], __shfl_xor_sync(0xffffffffu, rowp[ii], off));
         }
+        if (cg == 0) {
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) rowp2[jh * CH + 4 * rg6 + ii] = rowp[ii];
+        }
+        __syncthreads();  // every read of P and T is done (dbeta's column sums above included); halves stored
+        if (tid < CH) dbeta[tid] = __fadd_rn(dbeta[tid], __fadd_rn(rowp2[tid], rowp2[CH + tid]));
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj)
+                PP[4 * rg6 + ii][cg + 16 * (2 * jh + jj)] = __fmul_rn(beta[4 * rg6 + ii], dl[ii][jj]);
     }
     __syncthreads();
     float(*MM)[kRowC] = PP;
@@ -942,6 +943,23 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 rG[j][q] = __fmaf_rn(__fmul_rn(s, QA[i][d]), rb[j][q], rG[j][q]);
             }
     }
+    // the raw q/k pairs of the owned elements, for the normalisation's Jacobian at the end (requested here, so
+    // that their latency hides behind the MMAs below)
+    uint32_t xq[2][4] = {}, xk[2][4] = {};
+    if (p.fuse_norm) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int i = hf ? r1 : r0;
+            if (i < nvalid) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int64_t off = ((row0 + i) * p.H + hq) * DK + 32 * nh + 8 * j + 2 * t4;
+                    xq[hf][j] = *reinterpret_cast<const uint32_t *>(p.q + off);
+                    xk[hf][j] = *reinterpret_cast<const uint32_t *>(p.k + off);
+                }
+            }
+        }
+    }
     {
         // R24'_jd = sum_{I' >= J} sum_{i in I'} (M_ij KA_id + s N_ij QA_id) c_I'Jd for rows j of block J = mt
         float ra[4][4] = {};
@@ -1005,9 +1023,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
             if (i < nvalid) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const int64_t off = ((row0 + i) * p.H + hq) * DK + 32 * nh + 8 * j + 2 * t4;
-                    const uint32_t wq = *reinterpret_cast<const uint32_t *>(p.q + off);
-                    const uint32_t wk = *reinterpret_cast<const uint32_t *>(p.k + off);
+                    const uint32_t wq = xq[hf][j], wk = xk[hf][j];
                     xdy[hf][0] = __fmaf_rn(bf16lo(wq), rq[j][2 * hf], xdy[hf][0]);
                     xdy[hf][0] = __fmaf_rn(bf16hi(wq), rq[j][2 * hf + 1], xdy[hf][0]);
                     xdy[hf][1] = __fmaf_rn(bf16lo(wk), rk[j][2 * hf], xdy[hf][1]);
@@ -1032,7 +1048,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         }
         __syncthreads();
         // row i's half of dx from dy = this thread's columns of dqn (or dkn), w = 0 (q) or 1 (k)
-        auto emit = [&](const float (&dy)[4][4], int hf, int w, const __nv_bfloat16 *x, __nv_bfloat16 *dx,
+        auto emit = [&](const float (&dy)[4][4], int hf, int w, const uint32_t (&xw)[2][4], __nv_bfloat16 *dx,
                         float den) {
             const int i = hf ? r1 : r0;
             const float *rr = red + (w * CH + i) * 4;
@@ -1042,19 +1058,19 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int64_t off = ((row0 + i) * p.H + hq) * DK + 32 * nh + 8 * j + 2 * t4;
-                const uint32_t wx = *reinterpret_cast<const uint32_t *>(x + off);
+                const uint32_t wx = xw[hf][j];
                 const float o0 = __fmaf_rn(-bf16lo(wx), c3, __fmul_rn(dy[j][2 * hf], inv));
                 const float o1 = __fmaf_rn(-bf16hi(wx), c3, __fmul_rn(dy[j][2 * hf + 1], inv));
                 *reinterpret_cast<uint32_t *>(dx + off) = pack_bf16(o0, o1);
             }
         };
         if (r0 < nvalid) {
-            emit(rq, 0, 0, p.q, p.dq, denq[r0]);
-            emit(rk, 0, 1, p.k, p.dk, denk[r0]);
+            emit(rq, 0, 0, xq, p.dq, denq[r0]);
+            emit(rk, 0, 1, xk, p.dk, denk[r0]);
         }
         if (r1 < nvalid) {
-            emit(rq, 1, 0, p.q, p.dq, denq[r1]);
-            emit(rk, 1, 1, p.k, p.dk, denk[r1]);
+            emit(rq, 1, 0, xq, p.dq, denq[r1]);
+            emit(rk, 1, 1, xk, p.dk, denk[r1]);
         }
     }
     // dG rows into the KA region (unpadded [64][128]), then the reverse cumulative sum per key column
