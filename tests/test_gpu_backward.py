@@ -171,6 +171,27 @@ def test_saved_forward_then_backward(B, T, H, HV, cu, exact):
     _compare([t.float().cpu().numpy().astype(np.float64) for t in got_s[:5]] + [got_s[5].cpu().numpy()], ref)
 
 
+def test_saved_forward_with_head_groups():
+    """2 x 80 units (between one and two waves of carry CTAs): forward_save splits the value heads into two
+    groups, while the recomputing backward runs its forward in one launch of each kernel.  Heads are independent,
+    so the saved forward's outputs and the two backwards must agree bit for bit."""
+    import kda_gated_delta_prefill_b200 as kda
+    B, T, H, HV = 2, 1024, 80, 80
+    assert kda.kernel_launches(B, T, H, HV) == 4  # the two head groups
+    q, k, v, g, beta, s0, dout, dh, _ = _case(B, T, H, HV, seed=991)
+    c = lambda t: None if t is None else t.cuda()
+    xs = [c(t) for t in (q, k, v, g, beta)]
+    o1, sN1, saved = kda.forward_save(*xs, c(s0))
+    o2, sN2 = kda.forward(*xs, c(s0))
+    got_s = kda.backward(*xs, c(dout), c(s0), c(dh), want_dh0=True, saved=saved)
+    got_r = kda.backward(*xs, c(dout), c(s0), c(dh), want_dh0=True)
+    torch.cuda.synchronize()
+    assert kda.device_error(clear=True) == 0
+    assert torch.equal(o1, o2) and torch.equal(sN1, sN2)
+    for a, b in zip(got_s, got_r):
+        assert torch.equal(a, b)
+
+
 def _gen_run(x, gr, want_dh0):
     import kda_gated_delta_prefill_b200 as kda
     c = lambda t: None if t is None else t.cuda()
