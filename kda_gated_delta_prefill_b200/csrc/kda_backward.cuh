@@ -96,7 +96,8 @@ struct BcSmem {
     static constexpr int DSH = 2 * STAGE;                 // fp16 [128][72]  dS
     static constexpr int DOH = DSH + DK * kBcPad * 2;     // fp16 [64][72]   dO
     static constexpr int DVH = DOH + CH * kBcPad * 2;     // fp16 [64][72]   dVnew
-    static constexpr int BAR = DVH + CH * kBcPad * 2;     // mbarriers [2]
+    static constexpr int DSB = DVH + CH * kBcPad * 2;     // bf16 [128][72]  dS, as stored for the chunk kernel
+    static constexpr int BAR = DSB + DK * kBcPad * 2;     // mbarriers [2]
     static constexpr int FLAG = BAR + 16;
     static constexpr int TOTAL = FLAG + 16;
 };
@@ -165,13 +166,18 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
 #pragma unroll
         for (int q = 0; q < 4; ++q)
             acc[j][q] = p.dht ? p.dht[unit_off + key_of(q >> 1) * DV + vc0 + col_of(j, q & 1)] : 0.f;
+    // dS into shared memory: fp16 for the next chunk's MMAs, bf16 for the dstates row copy
+    __nv_bfloat16 *dSb = reinterpret_cast<__nv_bfloat16 *>(sm + S::DSB);
     auto store_dsh = [&]() {
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
+            for (int hf = 0; hf < 2; ++hf) {
                 *reinterpret_cast<__half2 *>(dSh + key_of(hf) * kBcPad + col_of(j, 0)) =
                     __floats2half2_rn(acc[j][2 * hf], acc[j][2 * hf + 1]);
+                *reinterpret_cast<__nv_bfloat162 *>(dSb + key_of(hf) * kBcPad + col_of(j, 0)) =
+                    __floats2bfloat162_rn(acc[j][2 * hf], acc[j][2 * hf + 1]);
+            }
     };
     store_dsh();
     __syncthreads();
@@ -199,16 +205,6 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
         const uint32_t blk = sb + st * S::STAGE;
         if (tid == 0 && c > 0) request(c - 1, st ^ 1);  // that stage was released by the previous iteration
         const uint4 next_dout = load_dout(c - 1);       // lands while this chunk computes
-        {
-            // dS is the gradient at chunk c's end state: store it
-            __nv_bfloat16 *dst = p.dstates + ((c_begin + c) * p.HV + h) * DK * DV + vc0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf)
-                    *reinterpret_cast<__nv_bfloat162 *>(dst + key_of(hf) * DV + col_of(j, 0)) =
-                        __floats2bfloat162_rn(acc[j][2 * hf], acc[j][2 * hf + 1]);
-        }
         if (tid == 0) {
             const bool landed = mbar_wait(sb + S::BAR + 8 * st, waited[st] & 1);
             if (landed) ++waited[st];
@@ -218,6 +214,17 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
         if (!flag[0]) {
             ok = false;
             break;
+        }
+        {
+            // dS is the gradient at chunk c's end state: store its bf16 copy (written to shared memory before the
+            // barrier above) as whole 128-byte rows, 16 bytes per thread
+            __nv_bfloat16 *dst = p.dstates + ((c_begin + c) * p.HV + h) * DK * DV + vc0;
+#pragma unroll
+            for (int i = 0; i < DK * kBcCols / 8 / kBcThreads; ++i) {
+                const int r = (tid >> 3) + i * (kBcThreads / 8), q = tid & 7;
+                *reinterpret_cast<uint4 *>(dst + r * DV + 8 * q) =
+                    *reinterpret_cast<const uint4 *>(dSb + r * kBcPad + 8 * q);
+            }
         }
         const uint32_t dsh = smem_u32(dSh), doh = smem_u32(dOh), dvh = smem_u32(dVh);
         {
