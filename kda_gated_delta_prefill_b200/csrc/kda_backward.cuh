@@ -32,9 +32,12 @@
 //   exp(G_i - G_j) = exp(G_i - m_I) * exp(m_I - m_J) * exp(m_J - G_j),
 // every factor at most exp(8 |g|max) away from 1 and the middle one <= 1.
 #pragma once
+#include <type_traits>
+
 #include "kda_common.cuh"
 #include "kda_norm.cuh"
 #include "ptx.cuh"
+#include "tc.cuh"
 
 namespace kda {
 
@@ -84,43 +87,59 @@ __device__ __forceinline__ void bwd_locate(const BwdParams &p, int chunk, int &n
 __device__ __forceinline__ float bwd_exp(float x) { return ex2(x * 1.4426950408889634f); }
 
 // ---------------------------------------------------------------------------------------------------------
-// Reverse carry: one CTA (16 warps) per (sequence, value head, half of the value columns), on fp16 tensor-core
-// MMAs (mma.sync m16n8k16, fp32 accumulate).  The fp32 gradient dS (128 keys x 64 columns) stays in the warps'
-// accumulator registers; an fp16 copy in shared memory feeds the next chunk's Kg dS.  Chunk c's block (the -W,
-// Qg, Kg, Aqk tiles in their SW128 layout, and exp(G_L)) arrives by bulk copy one chunk ahead.  Before chunk c
-// is folded in, dS is the gradient at chunk c's end state and is stored for the chunk kernel.
-constexpr int kBcThreads = 512, kBcCols = 64, kBcPad = 72;  // fp16 row stride (halves) of dS, dO, dVnew copies
-struct BcSmem {
-    static constexpr int PART = ITEM_U;                   // bytes [0, ITEM_U) of a block: -W, Qg, Kg, Aqk
-    static constexpr int STAGE = PART + 512;              // + exp(G_L)
-    static constexpr int DSH = 2 * STAGE;                 // fp16 [128][72]  dS
-    static constexpr int DOH = DSH + DK * kBcPad * 2;     // fp16 [64][72]   dO
-    static constexpr int DVH = DOH + CH * kBcPad * 2;     // fp16 [64][72]   dVnew
-    static constexpr int DSB = DVH + CH * kBcPad * 2;     // bf16 [128][72]  dS, as stored for the chunk kernel
-    static constexpr int BAR = DSB + DK * kBcPad * 2;     // mbarriers [2]
-    static constexpr int FLAG = BAR + 16;
-    static constexpr int TOTAL = FLAG + 16;
-};
-static_assert(ITEM_GL == ITEM_U + 16384, "block layout");
+// Reverse carry on the 5th-generation tensor cores: one CTA per (sequence, value head), walking the chunks
+// backwards.  Transposed, with the value dimension as the MMA's M = 128 and dS' the gradient at chunk c's end:
+//   dVnew^T = dS'^T Kg^T + dO^T Aqk                 (groups 1 and 2: M = 128 values, N = 64 tokens)
+//   dS^T    = dS'^T diag(exp(G_L)) + dO^T Qg + dVnew^T (-W)   (groups 3 and 4: N = 128 keys)
+// dS^T (fp32) stays in TMEM.  Its fp16 copy there is the A operand of group 1, and the fp16 dVnew^T of group 4.
+// dO^T is an MN-major A operand in shared memory: the epilogue stages each chunk's dO rows there in fp16 (the
+// blocks' tiles are fp16).  The blocks' -W, Qg, Kg and Aqk tiles are read in place from a three-stage bulk-copy
+// ring: Kg K-major (as Kg^T), Aqk, Qg and -W MN-major.
+// Warps 0-15 (epilogue) own TMEM lane v = 32 (warp % 4) + lane and a quarter of the key (and token) columns;
+// warp 16 streams the blocks; warp 17 allocates TMEM and issues the MMAs.  Every wait is bounded.
+__device__ __forceinline__ void bwd_mma_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate)
+{
+    asm volatile(
+        "{\n .reg .pred p, e;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+// kind::f16 instruction descriptor with either operand MN-major (bit 15: A, bit 16: B); fp16 operands
+__host__ __device__ constexpr uint32_t bwd_idesc(int M, int N, bool a_mn, bool b_mn)
+{
+    return (1u << 4) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
 
-// byte offset of the 16-byte group (row r, columns c..c+7) of a [64][128] SW128 tile pair / a [64][64] tile
-__device__ __forceinline__ uint32_t sw_off128(int r, int c)
-{
-    return static_cast<uint32_t>((c >> 6) * 8192 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4));
-}
-__device__ __forceinline__ uint32_t sw_off64(int r, int c)
-{
-    return static_cast<uint32_t>(r * 128 + (((c >> 3) ^ (r & 7)) << 4));
-}
+constexpr int kBcEpiWarps = 16;
+constexpr int kBcThreads = (kBcEpiWarps + 2) * 32;
+struct BcSmem {
+    static constexpr int PART = ITEM_U;                           // bytes [0, ITEM_U) of a block: -W, Qg, Kg, Aqk
+    static constexpr int GLO = PART;                              // exp(G_L) after them in the stage
+    static constexpr int STAGE = ((PART + 512 + 1023) / 1024) * 1024;
+    static constexpr int NST = 3;
+    static constexpr int DO = NST * STAGE;                        // fp16 dO [64 tok][128 v] x 2 (SW128, 64-v halves)
+    static constexpr int BAR = DO + 2 * CH * DV * 2;
+    // mbarriers: full[NST] empty[NST] barV barS sready vready dready oready[2]
+    static constexpr int TMEM_SLOT = BAR + (2 * NST + 7) * 8;
+    static constexpr int ABORT = TMEM_SLOT + 4;
+    static constexpr int TOTAL = ABORT + 4;
+};
+static_assert(BcSmem::TOTAL <= 232448, "reverse carry shared memory");
+static_assert(ITEM_GL == ITEM_U + 16384, "block layout");
+// TMEM columns: dS^T fp32 (128) | dVnew^T fp32 (64) | fp16 dS'^T (64) | fp16 dVnew^T (32)
+constexpr uint32_t BC_DS = 0, BC_DV = 128, BC_AS = 192, BC_AV = 256, BC_COLS = 512;
 
 __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdParams p)
 {
     using S = BcSmem;
+    constexpr int NST = S::NST;
+    static_assert(NST == 3, "the issuer body is instantiated for three stages");
     extern __shared__ __align__(1024) uint8_t sm[];
     const uint32_t sb = smem_u32(sm);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
-    const int unit = blockIdx.x >> 1, vc0 = (blockIdx.x & 1) * kBcCols;
-    const int n = unit / p.HV, h = unit % p.HV;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = blockIdx.x / p.HV, h = blockIdx.x % p.HV;
     int64_t c_begin, row0;
     int nck, len;
     if (p.cu) {
@@ -134,187 +153,255 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
         row0 = static_cast<int64_t>(n) * p.T;
         len = p.T;
     }
-    __half *dSh = reinterpret_cast<__half *>(sm + S::DSH);
-    __half *dOh = reinterpret_cast<__half *>(sm + S::DOH);
-    __half *dVh = reinterpret_cast<__half *>(sm + S::DVH);
-    volatile int *flag = reinterpret_cast<volatile int *>(sm + S::FLAG);
     const int64_t unit_off = (static_cast<int64_t>(n) * p.HV + h) * DK * DV;
 
-    // thread 0 bookkeeping: copies issued into / completions waited for, per stage
-    int issued[2] = {0, 0}, waited[2] = {0, 0};
-    auto request = [&](int c, int st) {  // thread 0: chunk c's block into stage st
-        ++issued[st];
-        const uint8_t *src = p.items + ((c_begin + c) * p.HV + h) * ITEM_BYTES;
-        const uint32_t bar = sb + S::BAR + 8 * st, dst = sb + st * S::STAGE;
-        mbar_expect_tx(bar, S::STAGE);
-        bulk_load(dst, src, S::PART, bar);
-        bulk_load(dst + S::PART, src + ITEM_GL, 512, bar);
-    };
+    const uint32_t full0 = sb + S::BAR, empty0 = full0 + 8 * NST, barV = full0 + 16 * NST, barS = barV + 8,
+                   sready = barV + 16, vready = barV + 24, dready = barV + 32, oready0 = barV + 40;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + S::ABORT);
     if (tid == 0) {
-        mbar_init(sb + S::BAR, 1);
-        mbar_init(sb + S::BAR + 8, 1);
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1 + kBcEpiWarps);
+        }
+        mbar_init(barV, 1);
+        mbar_init(barS, 1);
+        mbar_init(sready, kBcEpiWarps);
+        mbar_init(vready, kBcEpiWarps);
+        mbar_init(dready, kBcEpiWarps);
+        mbar_init(oready0, kBcEpiWarps);
+        mbar_init(oready0 + 8, kBcEpiWarps);
+        *abort_flag = 0;
         fence_mbar_init();
-        if (nck > 0) request(nck - 1, 0);
     }
-    // the warp's dS tile: keys 16 ms .. +15, value columns 32 nh .. +31 of this CTA's 64 (four n8 tiles)
-    const int ms = warp & 7, nh = warp >> 3;
-    float acc[4][4];
-    auto key_of = [&](int half) { return 16 * ms + g + 8 * half; };
-    auto col_of = [&](int j, int e) { return 32 * nh + 8 * j + 2 * t4 + e; };
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            acc[j][q] = p.dht ? p.dht[unit_off + key_of(q >> 1) * DV + vc0 + col_of(j, q & 1)] : 0.f;
-    // dS into shared memory: fp16 for the next chunk's MMAs, bf16 for the dstates row copy
-    __nv_bfloat16 *dSb = reinterpret_cast<__nv_bfloat16 *>(sm + S::DSB);
-    auto store_dsh = [&]() {
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                *reinterpret_cast<__half2 *>(dSh + key_of(hf) * kBcPad + col_of(j, 0)) =
-                    __floats2half2_rn(acc[j][2 * hf], acc[j][2 * hf + 1]);
-                *reinterpret_cast<__nv_bfloat162 *>(dSb + key_of(hf) * kBcPad + col_of(j, 0)) =
-                    __floats2bfloat162_rn(acc[j][2 * hf], acc[j][2 * hf + 1]);
-            }
-    };
-    store_dsh();
+    if (warp == kBcEpiWarps + 1) tc_alloc(sb + S::TMEM_SLOT, BC_COLS);
+    tc_fence_before();
     __syncthreads();
-
-    // this thread's share of a chunk's dO rows (row tid / 8, eight columns), loaded one chunk ahead
-    auto load_dout = [&](int c) {
-        const int i = tid >> 3, cc = 8 * (tid & 7);
-        uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-        if (c >= 0 && i < min(CH, len - c * CH))
-            raw = *reinterpret_cast<const uint4 *>(p.dout + ((row0 + static_cast<int64_t>(c) * CH + i) * p.HV + h) * DV +
-                                                   vc0 + cc);
-        return raw;
+    tc_fence_after();
+    // All 512 columns are allocated, so the allocation starts at lane 0, column 0.
+    const uint32_t tmem_alloc = *reinterpret_cast<volatile uint32_t *>(sm + S::TMEM_SLOT);
+    auto fail = [&](unsigned code) {
+        atomicOr(p.err, code);
+        *abort_flag = 1;
     };
-    auto put_dout = [&](uint4 raw) {  // as fp16 (zero past the sequence's end)
-        const int i = tid >> 3, cc = 8 * (tid & 7);
-        const uint4 w = make_uint4(pack_f16(bf16lo(raw.x), bf16hi(raw.x)), pack_f16(bf16lo(raw.y), bf16hi(raw.y)),
-                                   pack_f16(bf16lo(raw.z), bf16hi(raw.z)), pack_f16(bf16lo(raw.w), bf16hi(raw.w)));
-        *reinterpret_cast<uint4 *>(dOh + i * kBcPad + cc) = w;
-    };
-    if (nck > 0) put_dout(load_dout(nck - 1));  // visible after the first barrier below
+    if (tmem_alloc != 0) {
+        if (tid == 0) fail(ERR_TMEM_BASE);
+        nck = 0;
+    }
 
-    bool ok = true;
-    for (int it = 0; it < nck; ++it) {
-        const int c = nck - 1 - it, st = it & 1;
-        const uint32_t blk = sb + st * S::STAGE;
-        if (tid == 0 && c > 0) request(c - 1, st ^ 1);  // that stage was released by the previous iteration
-        const uint4 next_dout = load_dout(c - 1);       // lands while this chunk computes
-        if (tid == 0) {
-            const bool landed = mbar_wait(sb + S::BAR + 8 * st, waited[st] & 1);
-            if (landed) ++waited[st];
-            flag[0] = landed;
+    if (warp == kBcEpiWarps) {
+        // ---------------- producer: iteration it carries chunk nck - 1 - it ----------------
+        if (lane == 0) {
+            for (int it = 0; it < nck && !*abort_flag; ++it) {
+                const int s = it % NST;
+                if (it >= NST && !mbar_wait(empty0 + 8 * s, ((it / NST) - 1) & 1)) {
+                    fail(ERR_PIPE_EMPTY_WAIT);
+                    break;
+                }
+                const uint8_t *src = p.items + ((c_begin + nck - 1 - it) * p.HV + h) * ITEM_BYTES;
+                mbar_expect_tx(full0 + 8 * s, S::PART + 512);
+                bulk_load(sb + s * S::STAGE, src, S::PART, full0 + 8 * s);
+                bulk_load(sb + s * S::STAGE + S::GLO, src + ITEM_GL, 512, full0 + 8 * s);
+            }
         }
-        __syncthreads();
-        if (!flag[0]) {
-            ok = false;
-            break;
+    } else if (warp == kBcEpiWarps + 1) {
+        // ---------------- MMA issuer ----------------
+        const uint32_t iv_k = bwd_idesc(128, 64, false, false);   // A TMEM, B K-major (Kg^T)
+        const uint32_t iv_mm = bwd_idesc(128, 64, true, true);    // A dO^T MN-major, B Aqk MN-major
+        const uint32_t is_mm = bwd_idesc(128, 128, true, true);   // A dO^T MN-major, B Qg MN-major
+        const uint32_t is_tm = bwd_idesc(128, 128, false, true);  // A TMEM, B -W MN-major
+        const uint64_t dk0 = sw128_desc(sb, 16, 1024), kk0 = sw128_desc(sb, 8192, 1024);
+        const uint32_t dhi = static_cast<uint32_t>(dk0 >> 32), khi = static_cast<uint32_t>(kk0 >> 32);
+        auto kstep = [](int ks) { return static_cast<uint32_t>((ks >> 2) * 512 + (ks & 3) * 2); };
+        auto body = [&](int it, auto stage) -> bool {
+            constexpr int st = decltype(stage)::value;
+            constexpr uint32_t so = static_cast<uint32_t>(st * (S::STAGE >> 4));
+            uint32_t dlo = static_cast<uint32_t>(dk0), klo = static_cast<uint32_t>(kk0);
+            asm volatile("" : "+r"(dlo), "+r"(klo));
+            auto dd = [&](uint32_t off) { return (static_cast<uint64_t>(dhi) << 32) | (dlo + off); };
+            auto kd = [&](uint32_t off) { return (static_cast<uint64_t>(khi) << 32) | (klo + off); };
+            const int b = it & 1;
+            const uint32_t dob = static_cast<uint32_t>((S::DO + b * CH * DV * 2) >> 4);
+            bool w = mbar_wait(full0 + 8 * st, (it / NST) & 1) && mbar_wait_spin(oready0 + 8 * b, (it >> 1) & 1) &&
+                     mbar_wait_spin(sready, it & 1);
+            if (!__all_sync(0xffffffffu, w)) return false;
+            tc_fence_after();
+            // groups 1 and 2: dVnew^T = dS'^T Kg^T + dO^T Aqk
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                tc_mma_ts_warp(BC_DV, BC_AS + 8 * ks, dd(so + (ITEM_KG >> 4) + kstep(ks)), iv_k, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                bwd_mma_ss_warp(BC_DV, kd(dob + 128 * ks), kd(so + (ITEM_AQK >> 4) + 128 * ks), iv_mm, 1);
+            tc_commit_warp(barV);
+            // group 3: dS^T += dO^T Qg, onto dS'^T diag(exp(G_L)) (the epilogue's decay)
+            if (!__all_sync(0xffffffffu, mbar_wait_spin(dready, it & 1))) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                bwd_mma_ss_warp(BC_DS, kd(dob + 128 * ks), kd(so + (ITEM_QG >> 4) + 128 * ks), is_mm, 1);
+            // group 4: dS^T += dVnew^T (-W)
+            if (!__all_sync(0xffffffffu, mbar_wait_spin(vready, it & 1))) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc_mma_ts_warp(BC_DS, BC_AV + 8 * ks, kd(so + (ITEM_WN >> 4) + 128 * ks), is_tm, 1);
+            tc_commit_warp(barS);
+            tc_commit_warp(empty0 + 8 * st);
+            return true;
+        };
+        for (int it = 0; it < nck; ++it) {
+            if (__any_sync(0xffffffffu, *abort_flag)) break;
+            const int st = it % NST;
+            const bool ok = st == 0   ? body(it, std::integral_constant<int, 0>{})
+                            : st == 1 ? body(it, std::integral_constant<int, 1>{})
+                                      : body(it, std::integral_constant<int, 2>{});
+            if (!ok) {
+                if (lane == 0) fail(ERR_PIPE_FULL_WAIT);
+                break;
+            }
         }
+    } else {
+        // ---------------- epilogue: value column v, key quarter kq (keys 32kq..), token quarter (16kq..) ----------
+        const int qd = warp & 3, kq = warp >> 2;
+        const int v = 32 * qd + lane;
+        const uint32_t lb = static_cast<uint32_t>(32 * qd) << 16;
+        auto arrive = [&](uint32_t bar) {
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+        };
+        // fp16 copy of dS'^T[v][32kq ..] -> the A operand of the next group 1
+        auto pack_ds = [&](const uint32_t (&r)[32]) {
+            uint32_t w[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) w[j] = pack_f16(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+            tc_st16(lb + BC_AS + 16 * kq, w);
+        };
+        // dS' of chunk c (the gradient at its end state) -> dstates, bf16 [key][v]
+        auto store_dstates = [&](const uint32_t (&r)[32], int c) {
+            __nv_bfloat16 *dst = p.dstates + ((c_begin + c) * p.HV + h) * DK * DV + v;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) dst[(32 * kq + j) * DV] = __float2bfloat16_rn(__uint_as_float(r[j]));
+        };
+        // dO rows of chunk c, fp16, into buffer b: thread's two 16-byte pieces (row t, v-chunk vc), zero past the end
+        uint4 dov[2];
+        auto load_do = [&](int c) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int idx = tid + k * (kBcEpiWarps * 32), t = idx >> 4, vc = idx & 15;
+                dov[k] = make_uint4(0u, 0u, 0u, 0u);
+                if (c >= 0 && t < min(CH, len - c * CH))
+                    dov[k] = *reinterpret_cast<const uint4 *>(
+                        p.dout + ((row0 + static_cast<int64_t>(c) * CH + t) * p.HV + h) * DV + 8 * vc);
+            }
+        };
+        auto put_do = [&](int b) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int idx = tid + k * (kBcEpiWarps * 32), t = idx >> 4, vc = idx & 15;
+                const uint4 raw = dov[k];
+                const uint4 w = make_uint4(pack_f16(bf16lo(raw.x), bf16hi(raw.x)), pack_f16(bf16lo(raw.y), bf16hi(raw.y)),
+                                           pack_f16(bf16lo(raw.z), bf16hi(raw.z)), pack_f16(bf16lo(raw.w), bf16hi(raw.w)));
+                *reinterpret_cast<uint4 *>(sm + S::DO + b * CH * DV * 2 + (vc >> 3) * 8192 + t * 128 +
+                                           (((vc & 7) ^ (t & 7)) << 4)) = w;
+            }
+            fence_proxy_async();
+        };
+
+        bool alive = tmem_alloc == 0;
         {
-            // dS is the gradient at chunk c's end state: store its bf16 copy (written to shared memory before the
-            // barrier above) as whole 128-byte rows, 16 bytes per thread
-            __nv_bfloat16 *dst = p.dstates + ((c_begin + c) * p.HV + h) * DK * DV + vc0;
+            // dS' of the last chunk = dht (or zero)
+            uint32_t r[32];
 #pragma unroll
-            for (int i = 0; i < DK * kBcCols / 8 / kBcThreads; ++i) {
-                const int r = (tid >> 3) + i * (kBcThreads / 8), q = tid & 7;
-                *reinterpret_cast<uint4 *>(dst + r * DV + 8 * q) =
-                    *reinterpret_cast<const uint4 *>(dSb + r * kBcPad + 8 * q);
+            for (int j = 0; j < 32; ++j)
+                r[j] = __float_as_uint(p.dht ? p.dht[unit_off + (32 * kq + j) * DV + v] : 0.f);
+            if (alive && nck > 0) {
+                tc_st32(lb + BC_DS + 32 * kq, r);
+                pack_ds(r);
+                load_do(nck - 1);
+                put_do(0);
+                arrive(oready0);
+                arrive(sready);
+                store_dstates(r, nck - 1);
+                load_do(nck - 2);
+            } else if (alive && p.dh0) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) p.dh0[unit_off + (32 * kq + j) * DV + v] = __uint_as_float(r[j]);
             }
         }
-        const uint32_t dsh = smem_u32(dSh), doh = smem_u32(dOh), dvh = smem_u32(dVh);
-        {
-            // dVnew = Kg dS + Aqk^T dO; warp: tokens 16 mt .., columns 16 nq .. +15 (two n8 tiles)
-            const int mt = warp & 3, nq = warp >> 2;
-            float v[2][4] = {};
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                uint32_t a[4], b[4];
-                ldsm_x4(blk + ITEM_KG + sw_off128(16 * mt + (lane & 15), 16 * ks + (lane >> 4) * 8), a[0], a[1], a[2],
-                        a[3]);
-                ldsm_x4_t(dsh + 2 * ((16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8) * kBcPad + 16 * nq + (lane >> 4) * 8),
-                          b[0], b[1], b[2], b[3]);
-                mma_f16(v[0], a, b[0], b[1]);
-                mma_f16(v[1], a, b[2], b[3]);
+        for (int it = 0; it < nck && alive && !*abort_flag; ++it) {
+            const int c = nck - 1 - it, st = it % NST;
+            const float2 *gl = reinterpret_cast<const float2 *>(sm + st * S::STAGE + S::GLO) + 16 * kq;
+            if (!mbar_wait(full0 + 8 * st, (it / NST) & 1)) {
+                fail(ERR_PIPE_FULL_WAIT);
+                break;
             }
+            // 1. decay dS'^T by exp(G_L) of chunk c (group 1 reads only the fp16 copy)
+            {
+                uint32_t r[32];
+                tc_ld32(lb + BC_DS + 32 * kq, r);
+                tc_wait_ld();
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                uint32_t a[4], b[4];
-                ldsm_x4_t(blk + ITEM_AQK + sw_off64(16 * ks + (lane & 7) + ((lane >> 4) & 1) * 8,
-                                                   16 * mt + ((lane >> 3) & 1) * 8),
-                          a[0], a[1], a[2], a[3]);
-                ldsm_x4_t(doh + 2 * ((16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8) * kBcPad + 16 * nq + (lane >> 4) * 8),
-                          b[0], b[1], b[2], b[3]);
-                mma_f16(v[0], a, b[0], b[1]);
-                mma_f16(v[1], a, b[2], b[3]);
+                for (int j = 0; j < 16; ++j) {
+                    const float2 x = mul2(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])), gl[j]);
+                    r[2 * j] = __float_as_uint(x.x);
+                    r[2 * j + 1] = __float_as_uint(x.y);
+                }
+                tc_st32(lb + BC_DS + 32 * kq, r);
             }
+            arrive(dready);
+            // 2. dO of chunk c - 1 into the other buffer (its last reader, chunk c + 1's MMAs, completed before the
+            //    previous iteration's barS), then request chunk c - 2's rows
+            if (c > 0) {
+                put_do((it + 1) & 1);
+                arrive(oready0 + 8 * ((it + 1) & 1));
+                load_do(c - 2);
+            }
+            // 3. dVnew^T -> fp16 A operand of group 4
+            if (!mbar_wait_spin(barV, it & 1)) {
+                fail(ERR_PIPE_FULL_WAIT);
+                break;
+            }
+            tc_fence_after();
+            {
+                uint32_t pr[16], w[8];
+                tc_ld16(lb + BC_DV + 16 * kq, pr);
+                tc_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+                for (int j = 0; j < 8; ++j) w[j] = pack_f16(__uint_as_float(pr[2 * j]), __uint_as_float(pr[2 * j + 1]));
+                tc_st8(lb + BC_AV + 8 * kq, w);
+            }
+            arrive(vready);
+            // 4. dS^T is now dS' of chunk c - 1: its fp16 copy, then dstates (or dh0 after chunk 0)
+            if (!mbar_wait_spin(barS, it & 1)) {
+                fail(ERR_PIPE_FULL_WAIT);
+                break;
+            }
+            tc_fence_after();
+            {
+                uint32_t r[32];
+                tc_ld32(lb + BC_DS + 32 * kq, r);
+                tc_wait_ld();
+                if (c > 0) {
+                    pack_ds(r);
+                    arrive(sready);
+                    store_dstates(r, c - 1);
+                } else if (p.dh0) {
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf)
-                    *reinterpret_cast<__half2 *>(dVh + (16 * mt + g + 8 * hf) * kBcPad + 16 * nq + 8 * j + 2 * t4) =
-                        __floats2half2_rn(v[j][2 * hf], v[j][2 * hf + 1]);
+                    for (int j = 0; j < 32; ++j) p.dh0[unit_off + (32 * kq + j) * DV + v] = __uint_as_float(r[j]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty0 + 8 * st);  // exp(G_L) of this stage is consumed
         }
-        __syncthreads();
-        {
-            // dS <- exp(G_L) dS + Qg^T dO + (-W)^T dVnew
-            const float *egl = reinterpret_cast<const float *>(sm + st * S::STAGE + S::PART);
-            const float e0 = egl[key_of(0)], e1 = egl[key_of(1)];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                acc[j][0] *= e0;
-                acc[j][1] *= e0;
-                acc[j][2] *= e1;
-                acc[j][3] *= e1;
-            }
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const int tr = 16 * ks + (lane & 7) + ((lane >> 4) & 1) * 8, kc = 16 * ms + ((lane >> 3) & 1) * 8;
-                const int br = 16 * ks + (lane & 7) + ((lane >> 3) & 1) * 8;
-                uint32_t a[4], b[4], c2[4];
-                ldsm_x4_t(blk + ITEM_QG + sw_off128(tr, kc), a[0], a[1], a[2], a[3]);
-                ldsm_x4_t(doh + 2 * (br * kBcPad + 32 * nh + (lane >> 4) * 8), b[0], b[1], b[2], b[3]);
-                ldsm_x4_t(doh + 2 * (br * kBcPad + 32 * nh + 16 + (lane >> 4) * 8), c2[0], c2[1], c2[2], c2[3]);
-                mma_f16(acc[0], a, b[0], b[1]);
-                mma_f16(acc[1], a, b[2], b[3]);
-                mma_f16(acc[2], a, c2[0], c2[1]);
-                mma_f16(acc[3], a, c2[2], c2[3]);
-                ldsm_x4_t(blk + ITEM_WN + sw_off128(tr, kc), a[0], a[1], a[2], a[3]);
-                ldsm_x4_t(dvh + 2 * (br * kBcPad + 32 * nh + (lane >> 4) * 8), b[0], b[1], b[2], b[3]);
-                ldsm_x4_t(dvh + 2 * (br * kBcPad + 32 * nh + 16 + (lane >> 4) * 8), c2[0], c2[1], c2[2], c2[3]);
-                mma_f16(acc[0], a, b[0], b[1]);
-                mma_f16(acc[1], a, b[2], b[3]);
-                mma_f16(acc[2], a, c2[0], c2[1]);
-                mma_f16(acc[3], a, c2[2], c2[3]);
-            }
-        }
-        __syncthreads();  // every read of dS's fp16 copy, dO, dVnew and the stage is done
-        store_dsh();
-        put_dout(next_dout);
-        // (the next iteration's barrier orders these writes before their reads)
     }
-    if (!ok) {
-        if (tid == 0) {
-            atomicOr(p.err, ERR_TMA_WAIT);
-            // copies may still be in flight: wait for them (bounded) before leaving
-            for (int st = 0; st < 2; ++st)
-                for (int w = waited[st]; w < issued[st]; ++w)
-                    if (!mbar_wait(sb + S::BAR + 8 * st, w & 1)) break;
-        }
-        __syncthreads();
-        return;
-    }
-    if (p.dh0) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
-                *reinterpret_cast<float2 *>(p.dh0 + unit_off + key_of(hf) * DV + vc0 + col_of(j, 0)) =
-                    make_float2(acc[j][2 * hf], acc[j][2 * hf + 1]);
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kBcEpiWarps + 1) {
+        tc_fence_after();
+        tc_dealloc(tmem_alloc, BC_COLS);
     }
 }
 

@@ -286,7 +286,7 @@ kda_status_t backward_impl(const void *q, const void *k, const void *v, const fl
     if (cudaFuncSetAttribute(kda::kda_bwd_carry_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kda::BcSmem::TOTAL) != cudaSuccess)
         return KDA_ERR_CUDA;
-    kda::kda_bwd_carry_kernel<<<d.N * HV * (DV / kda::kBcCols), kda::kBcThreads, kda::BcSmem::TOTAL, s>>>(bp);
+    kda::kda_bwd_carry_kernel<<<d.N * HV, kda::kBcThreads, kda::BcSmem::TOTAL, s>>>(bp);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
     if (recompute && cudaStreamWaitEvent(s, lane->join, 0) != cudaSuccess) return KDA_ERR_CUDA;
     if (tokens == 0) return KDA_OK;
