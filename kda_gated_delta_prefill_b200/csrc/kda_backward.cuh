@@ -559,13 +559,14 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     }
     __syncthreads();
 
-    // ---- 2. P (j < i) and Aqk (j <= i); thread: rows 4rg..4rg+3 (block I), columns cg + 16 jb (threads 0-255:
-    //         with more threads each would reread the same q/k rows for fewer column blocks, and the phase is
-    //         bound by those shared-memory reads) ----
-    if (tid < 256) {
-        const int rg = tid >> 4, cg = tid & 15, I = rg >> 2;
+    // ---- 2. P (j < i) and Aqk (j <= i); thread: rows 4rg..4rg+3 (block I), columns cg + 16 jb, over the keys of its
+    //         half dh of the CTA (64 each).  The upper half leaves its partial sums in P and Aqk; the lower half
+    //         adds its own and writes the masked results.  (Splitting the column blocks instead would make every
+    //         thread reread the same q/k rows for fewer blocks, and the phase is bound by those shared-memory reads.) ----
+    {
+        const int rg = (tid >> 4) & 15, cg = tid & 15, I = rg >> 2, dh = tid >> 8;
         float pa[4][4] = {}, aa[4][4] = {};
-        for (int d = 0; d < DK; d += 4) {
+        for (int d = 64 * dh; d < 64 * dh + 64; d += 4) {
             float4 ka[4], qa[4];
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii) {
@@ -597,15 +598,33 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 }
             }
         }
+        if (dh == 1) {
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
+            for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
-            for (int jb = 0; jb < 4; ++jb) {
-                const int i = 4 * rg + ii, j = cg + 16 * jb;
-                PP[i][j] = j < i ? pa[ii][jb] : 0.f;
-                AQ[i][j] = j <= i ? __fmul_rn(s, aa[ii][jb]) : 0.f;
-                TT[i][j] = i == j ? 1.f : 0.f;
-            }
+                for (int jb = 0; jb < 4; ++jb)
+                    if (jb <= I) {
+                        PP[4 * rg + ii][cg + 16 * jb] = pa[ii][jb];
+                        AQ[4 * rg + ii][cg + 16 * jb] = aa[ii][jb];
+                    }
+        }
+        __syncthreads();
+        if (dh == 0) {
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                for (int jb = 0; jb < 4; ++jb) {
+                    const int i = 4 * rg + ii, j = cg + 16 * jb;
+                    float pv = 0.f, av = 0.f;
+                    if (jb <= I) {
+                        pv = __fadd_rn(pa[ii][jb], PP[i][j]);
+                        av = __fadd_rn(aa[ii][jb], AQ[i][j]);
+                    }
+                    PP[i][j] = j < i ? pv : 0.f;
+                    AQ[i][j] = j <= i ? __fmul_rn(s, av) : 0.f;
+                    TT[i][j] = i == j ? 1.f : 0.f;
+                }
+        }
     }
     __syncthreads();
 
