@@ -344,6 +344,20 @@ def test_windows_match_the_uncut_packed_run_bit_for_bit(mix):
     assert kda.device_error(clear=True) == 0
 
 
+def test_windows_with_many_sequences():
+    # 1500 sequences (more than one block of the window-offset scan) around one long one, in a shuffled order
+    rng = np.random.default_rng(7)
+    lengths = [int(x) for x in rng.integers(0, 12, size=1500)]
+    lengths[911] = 3000
+    case = gen.Case("win_many", B=1, T=sum(lengths), H=1, HV=2, lengths=lengths, state="n01", seed=691)
+    x = gen.make_inputs(case)
+    assert _window_count(case.T, 1, 2, x["cu_seqlens"]) >= 2
+    o_w, s_w = gpu_forward(x, cu_seqlens_host=x["cu_seqlens"])
+    o_u, s_u = gpu_forward(x)
+    assert torch.equal(o_w, o_u)
+    assert torch.equal(s_w, s_u)
+
+
 def test_windows_full_parity():
     lengths = [2049, 63, 0, 2111]
     case = gen.Case("win_oracle", B=1, T=sum(lengths), H=2, HV=2, lengths=lengths, state="n01", seed=641)
