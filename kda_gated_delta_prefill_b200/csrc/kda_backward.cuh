@@ -407,19 +407,49 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
 
 // ---------------------------------------------------------------------------------------------------------
 // Chunk gradients: one CTA of 512 threads (16 warps) per (chunk, value head); fp32 values, TF32 MMAs (fp32
-// accumulate).  The MMA phases (the value-column passes and the pairwise terms) give each warp a row block and a
-// quarter of the columns; the phases written for 8 warps (gates, P/Aqk, the solve, dL) run on threads 0-255 while
+// accumulate), except the passes' accumulations (step (e)), which run on tcgen05 with fp16 operand tiles and
+// fp32 accumulators in TMEM.  The MMA phases (the value-column passes and the pairwise terms) give each warp a
+// row block and a quarter of the columns; the gate scan and the solve's 16 x 16 steps run on threads 0-255 while
 // the rest wait at the next barrier.  One CTA per SM: 16 warps hide more of the MMA chains' latency than 8.
 constexpr int kBwThreads = 512, kBwCols = 16;  // value columns per pass over the state
 constexpr int kRow = 132;                      // padded row stride (floats) of the [64][128] operand tiles
 constexpr int kRowC = 68;                      // padded row stride of the [64][64] tiles
-// element (r, c) of a [64][16] fp32 value-column tile: rows of 16 floats, the two 8-column halves swapped in
-// rows with bit 1 set.  Scalar reads of 4 rows x 8 columns and 8-byte accesses of 4 rows x 4 column pairs
-// (a half warp) then fall into 32 distinct banks.
-__device__ __forceinline__ int vsw(int r, int c) { return r * kBwCols + (c ^ (((r >> 1) & 1) << 3)); }
-// column of element (r, c) in a [rows][16] bf16 pass buffer (S, dS', dO): the two 16-byte halves of a row swapped
-// in rows with bit 2 set, so that 4-byte reads of one column pair from 8 consecutive rows hit 8 distinct bank quads
-__device__ __forceinline__ int bsw(int r, int c) { return c ^ (((r >> 2) & 1) << 3); }
+// Byte offset of element (r, c) of a pass tile, fp16 [rows][16 value columns]: 8 x 8 core matrices of 128 bytes
+// (8 rows of 16 bytes), the two column halves of an 8-row group side by side.  This is the K-major operand layout
+// without swizzle, with the 16 columns as K: leading byte offset 128 (between the halves), stride byte offset 256
+// (between 8-row groups).  Reads of one column from 8 rows by 4 lanes each, and stores of 4-byte column pairs,
+// fall into distinct banks.
+__device__ __forceinline__ int tofs(int r, int c) { return (r >> 3) * 256 + (c >> 3) * 128 + (r & 7) * 16 + (c & 7) * 2; }
+__device__ __forceinline__ uint64_t bwd_tile_desc(uint32_t saddr)
+{
+    return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(128 >> 4) << 16) |
+           (static_cast<uint64_t>(256 >> 4) << 32) | (1ull << 46);
+}
+// 16 TMEM lanes (the address's lane onwards) x 8 (16) columns.  Thread (g, t) = (lane / 4, lane % 4) receives, for
+// each block j of 8 columns, rows g and g + 8 at columns 8 j + 2 t and 8 j + 2 t + 1: the accumulator fragment of
+// an m16n8 MMA, in the order (g, 2t), (g, 2t + 1), (g + 8, 2t), (g + 8, 2t + 1).
+__device__ __forceinline__ void bwd_ld_frag2(uint32_t taddr, float (&d)[2][4])
+{
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+    tc_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d[i >> 2][i & 3] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void bwd_ld_frag4(uint32_t taddr, float (&d)[4][4])
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    tc_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) d[i >> 2][i & 3] = __uint_as_float(r[i]);
+}
 struct BwSmem {
     static constexpr int KA = 0;                          // kn_id exp(G_id - m_Id)
     static constexpr int QA = KA + CH * kRow * 4;         // qn_id exp(G_id - m_Id)
@@ -437,15 +467,15 @@ struct BwSmem {
     static constexpr int DGL = EGL + 512;                 // [128] gradient at G_L
     static constexpr int DBETA = DGL + 512;               // [64]
     static constexpr int WK = DBETA + 256;                // work region
-    // V pass buffers (inside WK); S, dS' and dO columns are double-buffered (cp.async, one pass ahead)
-    static constexpr int SV = WK;                         // bf16 [2][128][16]  S[:, cols]
-    static constexpr int DSV = SV + 2 * DK * kBwCols * 2; // bf16 [2][128][16]  dS'[:, cols]
-    static constexpr int DOB = DSV + 2 * DK * kBwCols * 2;  // bf16 [2][64][16] dO
-    static constexpr int DD = DOB + 2 * CH * kBwCols * 2; // [64][16] (vsw) D = v - Kb S
-    static constexpr int VN = DD + CH * kBwCols * 4;      // [64][16] Vnew
-    static constexpr int DVN = VN + CH * kBwCols * 4;     // [64][16] dVnew
-    static constexpr int DV = DVN + CH * kBwCols * 4;     // [64][16] dv
-    static constexpr int WK_END = DV + CH * kBwCols * 4;
+    // pass tiles (inside WK), two buffers, each of fp16 tiles in the layout of tofs(): S[:, cols] and dS'[:, cols]
+    // (128 rows), dO, D = v - Kb S, Vnew, dVnew and -dv (64 rows)
+    static constexpr int P_S = 0, P_DS = 4096, P_O = 8192, P_D = 10240, P_N = 12288, P_DN = 14336, P_V = 16384;
+    static constexpr int PBUF = 18432;
+    static constexpr int WK_END = WK + 2 * PBUF;
+    // the TMEM base address and two mbarriers, in the padding columns 64..67 of row 0 of P and of T (no phase reads
+    // or writes a column of P or T past 63)
+    static constexpr int TMEM_SLOT = PP + CH * 4;
+    static constexpr int MBAR = TT + CH * 4;
     // phase-3 use of WK: the solve's products, 3 x [16][16] then [32][33]
     // phase-6 use of WK: dA, then Y = T^T dA diag(beta)
     static constexpr int DA = WK;                         // [64][kRowC]
@@ -467,6 +497,14 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     bwd_locate(p, chunk, n, row0, c_in_seq, nvalid);
     (void)n;
     (void)c_in_seq;
+    // TMEM (all 512 columns: the pass accumulators) and the two mbarriers of the pass MMAs
+    if (tid == 0) {
+        mbar_init(smem_u32(sm + S::MBAR), 1);
+        mbar_init(smem_u32(sm + S::MBAR) + 8, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) tc_alloc(smem_u32(sm + S::TMEM_SLOT), 512);
+    tc_fence_before();
     const float s = 0.08838834764831845f;  // K^-0.5
 
     float(*KA)[kRow] = reinterpret_cast<float(*)[kRow]>(sm + S::KA);
@@ -706,15 +744,21 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         __syncthreads();
     }
 
-    // ---- 4-5. passes over 16 value columns at a time, on TF32 tensor-core MMAs (m16n8k8, fp32 accumulate) ----
-    // S, dS' (bf16 [128][16]) and dO (bf16 [64][16]) of the current pass, the next pass's in the other buffer
-    auto SVb = [&](int b) { return reinterpret_cast<__nv_bfloat16(*)[kBwCols]>(sm + S::SV + b * DK * kBwCols * 2); };
-    auto DSVb = [&](int b) { return reinterpret_cast<__nv_bfloat16(*)[kBwCols]>(sm + S::DSV + b * DK * kBwCols * 2); };
-    auto DOBb = [&](int b) { return reinterpret_cast<__nv_bfloat16(*)[kBwCols]>(sm + S::DOB + b * CH * kBwCols * 2); };
-    float *DDv = reinterpret_cast<float *>(sm + S::DD);
-    float *VN = reinterpret_cast<float *>(sm + S::VN);
-    float *DVN = reinterpret_cast<float *>(sm + S::DVN);
-    float *DVv = reinterpret_cast<float *>(sm + S::DV);
+    // ---- 4-5. passes over 16 value columns at a time.  (a)-(d) on TF32 mma.sync (m16n8k8, fp32 accumulate); the
+    //      accumulations of (e) on tcgen05: five kind::f16 MMAs per pass (M = 64 tokens, K = the pass's 16
+    //      columns) add dQg, dKb, dKg (N = 128 keys) and dAqk, dA (N = 64 tokens) into TMEM.  An M = 64 accumulator
+    //      keeps rows 16 I .. 16 I + 15 in lanes 32 I .. 32 I + 15, the lane quarter of warps I, I + 4, ..., so
+    //      after the last pass each warp loads its phase-6/7 fragments from there.  S, dS' and dO of pass p + 1
+    //      are read into registers during pass p and stored as fp16 tiles into the other buffer once the MMAs of
+    //      pass p - 1, that buffer's last readers, have completed. ----
+    tc_fence_after();
+    const uint32_t tm = *reinterpret_cast<volatile uint32_t *>(sm + S::TMEM_SLOT);  // dQg 0, dKb 128, dKg 256,
+    if (tm != 0 && tid == 0) atomicOr(p.err, ERR_TMEM_BASE);                        // dAqk 384, dA 448
+    auto tile = [&](int b, int off) { return sm + S::WK + b * S::PBUF + off; };
+    // an fp16 tile element as a TF32 operand (fp16 values are exact in TF32)
+    auto hb = [&](int b, int off, int r, int c) {
+        return __float_as_uint(__half2float(*reinterpret_cast<const __half *>(tile(b, off) + tofs(r, c))));
+    };
     const __nv_bfloat16 *Sg = p.states + item * DK * DV;
     const __nv_bfloat16 *dSg = p.dstates + item * DK * DV;
     const int cg = tid & 15;  // column of the 64 x 64 steps of phase 6 (with the row group and half below)
@@ -725,47 +769,51 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     const int g = lane >> 2, t4 = lane & 3, mt = warp & 3, nh = warp >> 2;
     const int role = (warp >> 2) & 1, ntw = warp >> 3;
     const int r0 = 16 * mt + g, r1 = r0 + 8;
-    // bf16 values are exact in TF32 (8 of its 10 mantissa bits): the widened bits are the operand as they are
-    auto bf = [](__nv_bfloat16 x) { return static_cast<uint32_t>(__bfloat16_as_ushort(x)) << 16; };
-    float aQ[4][4] = {}, aB[4][4] = {}, aG[4][4] = {}, aAq[2][4] = {}, aA[2][4] = {};
-    // pass vb's columns into buffer b: S, dS' and dO rows are 32 bytes (two 16-byte copies each)
-    auto fetch = [&](int vb, int b) {
-        const int row = tid >> 1, half = 8 * (tid & 1);
-        if (tid < 256) {
-            cp_async16(smem_u32(&SVb(b)[row][bsw(row, half)]), Sg + row * DV + vb + half);
-            cp_async16(smem_u32(&DSVb(b)[row][bsw(row, half)]), dSg + row * DV + vb + half);
+    // staging: a thread takes one 16-byte row half (8 columns) of S (tid < 256) or dS' (tid >= 256) and, for
+    // tid < 128, one of dO; 8 consecutive threads take 8 rows of one half, so a quarter-warp's stores fill 128
+    // contiguous bytes
+    const int su = tid & 255, s_half = (su >> 3) & 1, s_row = (su & 7) | ((su >> 4) << 3);
+    const int o_half = (tid >> 3) & 1, o_row = (tid & 7) | ((tid >> 4) << 3);
+    uint4 rs, ro = make_uint4(0u, 0u, 0u, 0u);
+    auto load_pass = [&](int vb) {
+        rs = __ldg(reinterpret_cast<const uint4 *>((tid < 256 ? Sg : dSg) + s_row * DV + vb + 8 * s_half));
+        if (tid < 128) {
+            ro = make_uint4(0u, 0u, 0u, 0u);
+            if (o_row < nvalid)
+                ro = __ldg(reinterpret_cast<const uint4 *>(p.dout + ((row0 + o_row) * p.HV + h) * DV + vb + 8 * o_half));
         }
-        if (row < nvalid && tid < 2 * CH)
-            cp_async16(smem_u32(&DOBb(b)[row][bsw(row, half)]), p.dout + ((row0 + row) * p.HV + h) * DV + vb + half);
-        cp_async_commit();
     };
-    if (tid < CH && tid >= nvalid) {  // rows past the end stay zero in both buffers
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-            *reinterpret_cast<uint4 *>(&DOBb(b)[tid][0]) = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4 *>(&DOBb(b)[tid][8]) = make_uint4(0u, 0u, 0u, 0u);
-        }
-    }
-    fetch(0, 0);
+    auto to_f16x8 = [](uint4 x) {
+        return make_uint4(pack_f16(bf16lo(x.x), bf16hi(x.x)), pack_f16(bf16lo(x.y), bf16hi(x.y)),
+                          pack_f16(bf16lo(x.z), bf16hi(x.z)), pack_f16(bf16lo(x.w), bf16hi(x.w)));
+    };
+    auto store_pass = [&](int b) {
+        *reinterpret_cast<uint4 *>(tile(b, tid < 256 ? S::P_S : S::P_DS) + tofs(s_row, 8 * s_half)) = to_f16x8(rs);
+        if (tid < 128) *reinterpret_cast<uint4 *>(tile(b, S::P_O) + tofs(o_row, 8 * o_half)) = to_f16x8(ro);
+    };
+    const uint32_t mb0 = smem_u32(sm + S::MBAR);
+    auto wait_mma = [&](int pass) {  // the MMAs of `pass` (and of every pass before it) have completed
+        if (!mbar_wait(mb0 + 8 * (pass & 1), (pass >> 1) & 1)) atomicOr(p.err, ERR_PIPE_FULL_WAIT);
+    };
+    const uint32_t id128 = bwd_idesc(64, 128, false, false), id64 = bwd_idesc(64, 64, false, false);
+    load_pass(0);
+    store_pass(0);
     float gl_acc = 0.f;  // thread d < 128: sum over all columns of S[d][.] dS'[d][.]
-    for (int vb = 0; vb < DV; vb += kBwCols) {
-        const int buf = (vb / kBwCols) & 1;
-        if (vb + kBwCols < DV) {
-            fetch(vb + kBwCols, buf ^ 1);  // that buffer was released by the previous pass's last barrier
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        const __nv_bfloat16(*SVT)[kBwCols] = SVb(buf);
-        const __nv_bfloat16(*DST)[kBwCols] = DSVb(buf);
-        const __nv_bfloat16(*DOV)[kBwCols] = DOBb(buf);
-        if (tid < DK) {  // S and dS' rows share one column order, so physical positions pair up
+    for (int vb = 0, pass = 0; vb < DV; vb += kBwCols, ++pass) {
+        const int buf = pass & 1;
+        if (vb + kBwCols < DV) load_pass(vb + kBwCols);
+        __syncthreads();  // this pass's S, dS' and dO tiles are stored
+        if (tid < DK) {
 #pragma unroll
-            for (int c = 0; c < kBwCols; c += 2) {
-                const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&SVT[tid][c]));
-                const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&DST[tid][c]));
-                gl_acc = __fmaf_rn(x.y, y.y, __fmaf_rn(x.x, y.x, gl_acc));
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(tile(buf, S::P_S) + tofs(tid, 8 * hh));
+                const uint4 y = *reinterpret_cast<const uint4 *>(tile(buf, S::P_DS) + tofs(tid, 8 * hh));
+                const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 a = unpack_f16(xs[e]), b = unpack_f16(ys[e]);
+                    gl_acc = __fmaf_rn(a.y, b.y, __fmaf_rn(a.x, b.x, gl_acc));
+                }
             }
         }
         const int cn = 8 * ntw + g;  // this warp's tile: B-fragment column of steps (a)-(d)
@@ -777,8 +825,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 const uint32_t a[4] = {to_tf32(__fmul_rn(KA[r0][ks + t4], e0)), to_tf32(__fmul_rn(KA[r1][ks + t4], e0)),
                                        to_tf32(__fmul_rn(KA[r0][ks + t4 + 4], e1)),
                                        to_tf32(__fmul_rn(KA[r1][ks + t4 + 4], e1))};
-                const int k0 = ks + t4, k1 = ks + t4 + 4;
-                mma_tf32(c, a, bf(SVT[k0][bsw(k0, cn)]), bf(SVT[k1][bsw(k1, cn)]));
+                mma_tf32(c, a, hb(buf, S::P_S, ks + t4, cn), hb(buf, S::P_S, ks + t4 + 4, cn));
             }
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
@@ -787,8 +834,8 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 if (i < nvalid)
                     vv = __bfloat1622float2(
                         *reinterpret_cast<const __nv_bfloat162 *>(p.v + ((row0 + i) * p.HV + h) * DV + vb + cc));
-                *reinterpret_cast<float2 *>(&DDv[vsw(i, cc)]) =
-                    make_float2(__fsub_rn(vv.x, c[2 * hf]), __fsub_rn(vv.y, c[2 * hf + 1]));
+                *reinterpret_cast<uint32_t *>(tile(buf, S::P_D) + tofs(i, cc)) =
+                    pack_f16(__fsub_rn(vv.x, c[2 * hf]), __fsub_rn(vv.y, c[2 * hf + 1]));
             }
         } else {
             // (c) dVnew = Kg dS' + Aqk^T dO for rows 16 mt .. (Kg = KB exp(G_L - m_I)), columns 8 ntw ..
@@ -798,17 +845,15 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 const uint32_t a[4] = {to_tf32(__fmul_rn(KB[r0][ks + t4], e0)), to_tf32(__fmul_rn(KB[r1][ks + t4], e0)),
                                        to_tf32(__fmul_rn(KB[r0][ks + t4 + 4], e1)),
                                        to_tf32(__fmul_rn(KB[r1][ks + t4 + 4], e1))};
-                const int k0 = ks + t4, k1 = ks + t4 + 4;
-                mma_tf32(c, a, bf(DST[k0][bsw(k0, cn)]), bf(DST[k1][bsw(k1, cn)]));
+                mma_tf32(c, a, hb(buf, S::P_DS, ks + t4, cn), hb(buf, S::P_DS, ks + t4 + 4, cn));
             }
             for (int js = 16 * mt; js < CH; js += 8) {  // Aqk^T[i][j] = Aqk[j][i], nonzero for j >= i
                 const uint32_t a[4] = {to_tf32(AQ[js + t4][r0]), to_tf32(AQ[js + t4][r1]), to_tf32(AQ[js + t4 + 4][r0]),
                                        to_tf32(AQ[js + t4 + 4][r1])};
-                const int k0 = js + t4, k1 = js + t4 + 4;
-                mma_tf32(c, a, bf(DOV[k0][bsw(k0, cn)]), bf(DOV[k1][bsw(k1, cn)]));
+                mma_tf32(c, a, hb(buf, S::P_O, js + t4, cn), hb(buf, S::P_O, js + t4 + 4, cn));
             }
-            *reinterpret_cast<float2 *>(&DVN[vsw(r0, 8 * ntw + 2 * t4)]) = make_float2(c[0], c[1]);
-            *reinterpret_cast<float2 *>(&DVN[vsw(r1, 8 * ntw + 2 * t4)]) = make_float2(c[2], c[3]);
+            *reinterpret_cast<uint32_t *>(tile(buf, S::P_DN) + tofs(r0, 8 * ntw + 2 * t4)) = pack_f16(c[0], c[1]);
+            *reinterpret_cast<uint32_t *>(tile(buf, S::P_DN) + tofs(r1, 8 * ntw + 2 * t4)) = pack_f16(c[2], c[3]);
         }
         __syncthreads();
         if (role == 0) {
@@ -819,70 +864,56 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 const uint32_t a[4] = {to_tf32(__fmul_rn(TT[r0][js + t4], b0)), to_tf32(__fmul_rn(TT[r1][js + t4], b0)),
                                        to_tf32(__fmul_rn(TT[r0][js + t4 + 4], b1)),
                                        to_tf32(__fmul_rn(TT[r1][js + t4 + 4], b1))};
-                mma_tf32(c, a, to_tf32(DDv[vsw(js + t4, cn)]), to_tf32(DDv[vsw(js + t4 + 4, cn)]));
+                mma_tf32(c, a, hb(buf, S::P_D, js + t4, cn), hb(buf, S::P_D, js + t4 + 4, cn));
             }
-            *reinterpret_cast<float2 *>(&VN[vsw(r0, 8 * ntw + 2 * t4)]) = make_float2(c[0], c[1]);
-            *reinterpret_cast<float2 *>(&VN[vsw(r1, 8 * ntw + 2 * t4)]) = make_float2(c[2], c[3]);
+            *reinterpret_cast<uint32_t *>(tile(buf, S::P_N) + tofs(r0, 8 * ntw + 2 * t4)) = pack_f16(c[0], c[1]);
+            *reinterpret_cast<uint32_t *>(tile(buf, S::P_N) + tofs(r1, 8 * ntw + 2 * t4)) = pack_f16(c[2], c[3]);
         } else {
             // (d) dv = diag(beta) T^T dVnew (j >= i)
             float c[4] = {};
             for (int js = 16 * mt; js < CH; js += 8) {
                 const uint32_t a[4] = {to_tf32(TT[js + t4][r0]), to_tf32(TT[js + t4][r1]), to_tf32(TT[js + t4 + 4][r0]),
                                        to_tf32(TT[js + t4 + 4][r1])};
-                mma_tf32(c, a, to_tf32(DVN[vsw(js + t4, cn)]), to_tf32(DVN[vsw(js + t4 + 4, cn)]));
+                mma_tf32(c, a, hb(buf, S::P_DN, js + t4, cn), hb(buf, S::P_DN, js + t4 + 4, cn));
             }
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const int i = hf ? r1 : r0, cc = 8 * ntw + 2 * t4;
                 const float x0 = __fmul_rn(beta[i], c[2 * hf]), x1 = __fmul_rn(beta[i], c[2 * hf + 1]);
-                *reinterpret_cast<float2 *>(&DVv[vsw(i, cc)]) = make_float2(x0, x1);
+                *reinterpret_cast<uint32_t *>(tile(buf, S::P_V) + tofs(i, cc)) = pack_f16(-x0, -x1);
                 if (i < nvalid)
                     *reinterpret_cast<__nv_bfloat162 *>(p.dv + ((row0 + i) * p.HV + h) * DV + vb + cc) =
                         __floats2bfloat162_rn(x0, x1);
             }
         }
-        __syncthreads();
-        // (e) dQg += dO S^T, dKb -= dv S^T, dKg += Vnew dS'^T (K = these 16 columns, two k8 steps);
-        //     dAqk += dO Vnew^T, dA += dVnew D^T.  A k8 step's slots t4 and t4 + 4 carry this thread's column pair
-        //     cp, cp + 1 (any order of K is a valid order as long as A and B share it), so every operand pair
-        //     comes from one 4- or 8-byte shared-memory read.
-        auto pair = [](const __nv_bfloat16(*B)[kBwCols], int r, int c) {
-            return *reinterpret_cast<const uint32_t *>(&B[r][bsw(r, c)]);
-        };
-        constexpr uint32_t kHi = 0xffff0000u;
-#pragma unroll
-        for (int kc = 0; kc < kBwCols; kc += 8) {
-            const int cp = kc + 2 * t4;
-            const uint32_t o0 = pair(DOV, r0, cp), o1 = pair(DOV, r1, cp);
-            const uint32_t aO[4] = {o0 << 16, o1 << 16, o0 & kHi, o1 & kHi};
-            const float2 v0 = *reinterpret_cast<const float2 *>(&DVv[vsw(r0, cp)]);
-            const float2 v1 = *reinterpret_cast<const float2 *>(&DVv[vsw(r1, cp)]);
-            const float2 n0 = *reinterpret_cast<const float2 *>(&VN[vsw(r0, cp)]);
-            const float2 n1 = *reinterpret_cast<const float2 *>(&VN[vsw(r1, cp)]);
-            const float2 e0 = *reinterpret_cast<const float2 *>(&DVN[vsw(r0, cp)]);
-            const float2 e1 = *reinterpret_cast<const float2 *>(&DVN[vsw(r1, cp)]);
-            const uint32_t aV[4] = {to_tf32(-v0.x), to_tf32(-v1.x), to_tf32(-v0.y), to_tf32(-v1.y)};
-            const uint32_t aN[4] = {to_tf32(n0.x), to_tf32(n1.x), to_tf32(n0.y), to_tf32(n1.y)};
-            const uint32_t aD[4] = {to_tf32(e0.x), to_tf32(e1.x), to_tf32(e0.y), to_tf32(e1.y)};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int d = 32 * nh + 8 * j + g;
-                const uint32_t sp = pair(SVT, d, cp), qp = pair(DST, d, cp);
-                mma_tf32(aQ[j], aO, sp << 16, sp & kHi);
-                mma_tf32(aB[j], aV, sp << 16, sp & kHi);
-                mma_tf32(aG[j], aN, qp << 16, qp & kHi);
-            }
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int tk = 16 * nh + 8 * j + g;
-                const float2 vn = *reinterpret_cast<const float2 *>(&VN[vsw(tk, cp)]);
-                const float2 dd = *reinterpret_cast<const float2 *>(&DDv[vsw(tk, cp)]);
-                mma_tf32(aAq[j], aO, to_tf32(vn.x), to_tf32(vn.y));
-                mma_tf32(aA[j], aD, to_tf32(dd.x), to_tf32(dd.y));
-            }
+        fence_proxy_async();  // this thread's tile stores, visible to the tensor cores
+        __syncthreads();      // the pass's seven tiles are complete
+        if (warp == 0) {
+            // (e) dQg += dO S^T, dKb += (-dv) S^T, dKg += Vnew dS'^T, dAqk += dO Vnew^T, dA += dVnew D^T
+            tc_fence_after();
+            const uint32_t t0 = smem_u32(tile(buf, 0)), acc = vb > 0;
+            const uint64_t dS = bwd_tile_desc(t0 + S::P_S), dDS = bwd_tile_desc(t0 + S::P_DS),
+                           dO = bwd_tile_desc(t0 + S::P_O), dD = bwd_tile_desc(t0 + S::P_D),
+                           dN = bwd_tile_desc(t0 + S::P_N), dDN = bwd_tile_desc(t0 + S::P_DN),
+                           dV = bwd_tile_desc(t0 + S::P_V);
+            bwd_mma_ss_warp(tm + 0, dO, dS, id128, acc);
+            bwd_mma_ss_warp(tm + 128, dV, dS, id128, acc);
+            bwd_mma_ss_warp(tm + 256, dN, dDS, id128, acc);
+            bwd_mma_ss_warp(tm + 384, dO, dN, id64, acc);
+            bwd_mma_ss_warp(tm + 448, dDN, dD, id64, acc);
+            tc_commit_warp(mb0 + 8 * buf);
         }
-        __syncthreads();
+        if (vb + kBwCols < DV) {
+            if (pass > 0) wait_mma(pass - 1);  // the other buffer's last readers are done
+            store_pass(buf ^ 1);
+        }
     }
+    wait_mma(DV / kBwCols - 1);  // the last pass's MMAs, and with them every earlier one
+    tc_fence_after();
+    const uint32_t tl = tm + (static_cast<uint32_t>(32 * mt) << 16);  // this warp's lane quarter
+    float aAq[2][4], aA[2][4];
+    bwd_ld_frag2(tl + 384 + 16 * nh, aAq);
+    bwd_ld_frag2(tl + 448 + 16 * nh, aA);
 
     if (tid < DK) dgl[tid] = __fmaf_rn(egl[tid], gl_acc, dgl[tid]);  // the exp(G_L) S dS' term of dG_L
 
@@ -970,6 +1001,11 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     float(*NN)[kRowC] = AQ;
 
     // ---- 7. element terms and pairwise terms, in the fragment ownership of phase 5 ----
+    float aQ[4][4], aB[4][4], aG[4][4];
+    bwd_ld_frag4(tl + 0 + 32 * nh, aQ);
+    bwd_ld_frag4(tl + 128 + 32 * nh, aB);
+    bwd_ld_frag4(tl + 256 + 32 * nh, aG);
+    tc_fence_before();  // every TMEM read of this thread is done (TMEM is freed after the next barrier)
     float rq[4][4], rk[4][4], rG[4][4];
     {
         // qn/kn of the owned elements, rebuilt from the raw rows (the same normalisation, bit for bit)
@@ -1151,6 +1187,10 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         }
     }
     __syncthreads();  // KA/QA/KB/G reads done; dgl complete
+    if (warp == 0) {
+        tc_fence_after();
+        tc_dealloc(tm, 512);
+    }
     if (p.fuse_norm) {
         float *red = reinterpret_cast<float *>(sm + S::EM);  // [q|k][row][quarter]; exp(m_I) is no longer read
         if (t4 == 0) {
