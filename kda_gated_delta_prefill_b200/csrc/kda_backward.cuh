@@ -425,6 +425,10 @@ __device__ __forceinline__ uint64_t bwd_tile_desc(uint32_t saddr)
     return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(128 >> 4) << 16) |
            (static_cast<uint64_t>(256 >> 4) << 32) | (1ull << 46);
 }
+__device__ __forceinline__ void bwd_ldsm_x2_t(uint32_t addr, uint32_t &r0, uint32_t &r1)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
 // 16 TMEM lanes (the address's lane onwards) x 8 (16) columns.  Thread (g, t) = (lane / 4, lane % 4) receives, for
 // each block j of 8 columns, rows g and g + 8 at columns 8 j + 2 t and 8 j + 2 t + 1: the accumulator fragment of
 // an m16n8 MMA, in the order (g, 2t), (g, 2t + 1), (g + 8, 2t), (g + 8, 2t + 1).
@@ -755,10 +759,6 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     const uint32_t tm = *reinterpret_cast<volatile uint32_t *>(sm + S::TMEM_SLOT);  // dQg 0, dKb 128, dKg 256,
     if (tm != 0 && tid == 0) atomicOr(p.err, ERR_TMEM_BASE);                        // dAqk 384, dA 448
     auto tile = [&](int b, int off) { return sm + S::WK + b * S::PBUF + off; };
-    // an fp16 tile element as a TF32 operand (fp16 values are exact in TF32)
-    auto hb = [&](int b, int off, int r, int c) {
-        return __float_as_uint(__half2float(*reinterpret_cast<const __half *>(tile(b, off) + tofs(r, c))));
-    };
     const __nv_bfloat16 *Sg = p.states + item * DK * DV;
     const __nv_bfloat16 *dSg = p.dstates + item * DK * DV;
     const int cg = tid & 15;  // column of the 64 x 64 steps of phase 6 (with the row group and half below)
@@ -769,6 +769,22 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     const int g = lane >> 2, t4 = lane & 3, mt = warp & 3, nh = warp >> 2;
     const int role = (warp >> 2) & 1, ntw = warp >> 3;
     const int r0 = 16 * mt + g, r1 = r0 + 8;
+    // the A operand of step (a) (role 0: Kb = KA exp(m_I)) or (c) (role 1: Kg = KB exp(G_L - m_I)), rows 16 mt ..
+    // and all 128 keys, as fp16 m16n8k16 fragments (|Kb|, |Kg| <= |kn| <= 1): built once, used by every pass
+    uint32_t fa[8][4];
+    {
+        const float(*X)[kRow] = role ? KB : KA;
+        const float *e = role ? EGLM[mt] : EM[mt];
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int r = (q & 1) ? r1 : r0, k = 16 * kk + 2 * t4 + 8 * (q >> 1);
+                const float2 x = *reinterpret_cast<const float2 *>(&X[r][k]);
+                const float2 m = *reinterpret_cast<const float2 *>(&e[k]);
+                fa[kk][q] = pack_f16(__fmul_rn(x.x, m.x), __fmul_rn(x.y, m.y));
+            }
+    }
     // staging: a thread takes one 16-byte row half (8 columns) of S (tid < 256) or dS' (tid >= 256) and, for
     // tid < 128, one of dO; 8 consecutive threads take 8 rows of one half, so a quarter-warp's stores fill 128
     // contiguous bytes
@@ -816,16 +832,18 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 }
             }
         }
-        const int cn = 8 * ntw + g;  // this warp's tile: B-fragment column of steps (a)-(d)
+        // steps (a)-(d): fp16 m16n8k16 MMAs; B fragments from the tiles by ldmatrix.trans (8 rows of 16 bytes per
+        // matrix: thread (g, t4) receives rows 2 t4, 2 t4 + 1 of column g of this warp's 8 columns)
+        const uint32_t tb = smem_u32(tile(buf, 0)) + 128 * ntw;
         if (role == 0) {
-            // (a) D = v - Kb S for rows 16 mt .. (Kb = KA exp(m_I), block I = mt), columns 8 ntw ..
+            // (a) D = v - Kb S for rows 16 mt .., columns 8 ntw ..
             float c[4] = {};
-            for (int ks = 0; ks < DK; ks += 8) {
-                const float e0 = EM[mt][ks + t4], e1 = EM[mt][ks + t4 + 4];
-                const uint32_t a[4] = {to_tf32(__fmul_rn(KA[r0][ks + t4], e0)), to_tf32(__fmul_rn(KA[r1][ks + t4], e0)),
-                                       to_tf32(__fmul_rn(KA[r0][ks + t4 + 4], e1)),
-                                       to_tf32(__fmul_rn(KA[r1][ks + t4 + 4], e1))};
-                mma_tf32(c, a, hb(buf, S::P_S, ks + t4, cn), hb(buf, S::P_S, ks + t4 + 4, cn));
+#pragma unroll
+            for (int kk = 0; kk < 8; kk += 2) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(tb + S::P_S + tofs(16 * kk + lane, 0), b0, b1, b2, b3);
+                mma_f16(c, fa[kk], b0, b1);
+                mma_f16(c, fa[kk + 1], b2, b3);
             }
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
@@ -838,19 +856,24 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                     pack_f16(__fsub_rn(vv.x, c[2 * hf]), __fsub_rn(vv.y, c[2 * hf + 1]));
             }
         } else {
-            // (c) dVnew = Kg dS' + Aqk^T dO for rows 16 mt .. (Kg = KB exp(G_L - m_I)), columns 8 ntw ..
+            // (c) dVnew = Kg dS' + Aqk^T dO for rows 16 mt .., columns 8 ntw ..
             float c[4] = {};
-            for (int ks = 0; ks < DK; ks += 8) {
-                const float e0 = EGLM[mt][ks + t4], e1 = EGLM[mt][ks + t4 + 4];
-                const uint32_t a[4] = {to_tf32(__fmul_rn(KB[r0][ks + t4], e0)), to_tf32(__fmul_rn(KB[r1][ks + t4], e0)),
-                                       to_tf32(__fmul_rn(KB[r0][ks + t4 + 4], e1)),
-                                       to_tf32(__fmul_rn(KB[r1][ks + t4 + 4], e1))};
-                mma_tf32(c, a, hb(buf, S::P_DS, ks + t4, cn), hb(buf, S::P_DS, ks + t4 + 4, cn));
+#pragma unroll
+            for (int kk = 0; kk < 8; kk += 2) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(tb + S::P_DS + tofs(16 * kk + lane, 0), b0, b1, b2, b3);
+                mma_f16(c, fa[kk], b0, b1);
+                mma_f16(c, fa[kk + 1], b2, b3);
             }
-            for (int js = 16 * mt; js < CH; js += 8) {  // Aqk^T[i][j] = Aqk[j][i], nonzero for j >= i
-                const uint32_t a[4] = {to_tf32(AQ[js + t4][r0]), to_tf32(AQ[js + t4][r1]), to_tf32(AQ[js + t4 + 4][r0]),
-                                       to_tf32(AQ[js + t4 + 4][r1])};
-                mma_tf32(c, a, hb(buf, S::P_O, js + t4, cn), hb(buf, S::P_O, js + t4 + 4, cn));
+            for (int js = 16 * mt; js < CH; js += 16) {  // Aqk^T[i][j] = Aqk[j][i], nonzero for j >= i
+                uint32_t a[4], b0, b1;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int r = (q & 1) ? r1 : r0, k = js + 2 * t4 + 8 * (q >> 1);
+                    a[q] = pack_f16(AQ[k][r], AQ[k + 1][r]);
+                }
+                bwd_ldsm_x2_t(tb + S::P_O + tofs(js + (lane & 15), 0), b0, b1);
+                mma_f16(c, a, b0, b1);
             }
             *reinterpret_cast<uint32_t *>(tile(buf, S::P_DN) + tofs(r0, 8 * ntw + 2 * t4)) = pack_f16(c[0], c[1]);
             *reinterpret_cast<uint32_t *>(tile(buf, S::P_DN) + tofs(r1, 8 * ntw + 2 * t4)) = pack_f16(c[2], c[3]);
@@ -859,22 +882,32 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         if (role == 0) {
             // (b) Vnew = T diag(beta) D (T lower triangular: j < 16 (mt + 1))
             float c[4] = {};
-            for (int js = 0; js < 16 * (mt + 1); js += 8) {
-                const float b0 = beta[js + t4], b1 = beta[js + t4 + 4];
-                const uint32_t a[4] = {to_tf32(__fmul_rn(TT[r0][js + t4], b0)), to_tf32(__fmul_rn(TT[r1][js + t4], b0)),
-                                       to_tf32(__fmul_rn(TT[r0][js + t4 + 4], b1)),
-                                       to_tf32(__fmul_rn(TT[r1][js + t4 + 4], b1))};
-                mma_tf32(c, a, hb(buf, S::P_D, js + t4, cn), hb(buf, S::P_D, js + t4 + 4, cn));
+            for (int js = 0; js < 16 * (mt + 1); js += 16) {
+                uint32_t a[4], b0, b1;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int r = (q & 1) ? r1 : r0, k = js + 2 * t4 + 8 * (q >> 1);
+                    const float2 t = *reinterpret_cast<const float2 *>(&TT[r][k]);
+                    const float2 bb = *reinterpret_cast<const float2 *>(&beta[k]);
+                    a[q] = pack_f16(__fmul_rn(t.x, bb.x), __fmul_rn(t.y, bb.y));
+                }
+                bwd_ldsm_x2_t(tb + S::P_D + tofs(js + (lane & 15), 0), b0, b1);
+                mma_f16(c, a, b0, b1);
             }
             *reinterpret_cast<uint32_t *>(tile(buf, S::P_N) + tofs(r0, 8 * ntw + 2 * t4)) = pack_f16(c[0], c[1]);
             *reinterpret_cast<uint32_t *>(tile(buf, S::P_N) + tofs(r1, 8 * ntw + 2 * t4)) = pack_f16(c[2], c[3]);
         } else {
             // (d) dv = diag(beta) T^T dVnew (j >= i)
             float c[4] = {};
-            for (int js = 16 * mt; js < CH; js += 8) {
-                const uint32_t a[4] = {to_tf32(TT[js + t4][r0]), to_tf32(TT[js + t4][r1]), to_tf32(TT[js + t4 + 4][r0]),
-                                       to_tf32(TT[js + t4 + 4][r1])};
-                mma_tf32(c, a, hb(buf, S::P_DN, js + t4, cn), hb(buf, S::P_DN, js + t4 + 4, cn));
+            for (int js = 16 * mt; js < CH; js += 16) {
+                uint32_t a[4], b0, b1;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int r = (q & 1) ? r1 : r0, k = js + 2 * t4 + 8 * (q >> 1);
+                    a[q] = pack_f16(TT[k][r], TT[k + 1][r]);
+                }
+                bwd_ldsm_x2_t(tb + S::P_DN + tofs(js + (lane & 15), 0), b0, b1);
+                mma_f16(c, a, b0, b1);
             }
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
