@@ -23,8 +23,8 @@
 // cumulative sum is dg.  Three kernels:
 //   kda_bwd_carry_kernel  dS' of every chunk, walking each sequence backwards
 //                         (reads the forward's per-chunk blocks),
-//   kda_bwd_chunk_kernel  every chunk's gradients at once (fp32 arithmetic,
-//                         TF32 tensor-core MMAs for the products),
+//   kda_bwd_chunk_kernel  every chunk's gradients at once (fp32 arithmetic;
+//                         fp16 and TF32 tensor-core MMAs for the products),
 //   kda_bwd_norm_kernel   sums a Q/K head's group and applies the L2
 //                         normalisation's Jacobian.
 // Gate factors exp(G_i - G_j) are formed per 16-token block I with the
@@ -406,9 +406,9 @@ __global__ void __launch_bounds__(kBcThreads, 1) kda_bwd_carry_kernel(const BwdP
 }
 
 // ---------------------------------------------------------------------------------------------------------
-// Chunk gradients: one CTA of 512 threads (16 warps) per (chunk, value head); fp32 values, TF32 MMAs (fp32
-// accumulate), except the passes' accumulations (step (e)), which run on tcgen05 with fp16 operand tiles and
-// fp32 accumulators in TMEM.  The MMA phases (the value-column passes and the pairwise terms) give each warp a
+// Chunk gradients: one CTA of 512 threads (16 warps) per (chunk, value head); fp32 values.  The value-column
+// passes multiply fp16 operands (fp16 mma.sync for D, Vnew, dVnew and dv; tcgen05 with fp32 accumulators in TMEM
+// for their accumulations); the pairwise terms, whose gate factors reach exp(+-8 |g|max), use TF32 MMAs.  The MMA phases (the value-column passes and the pairwise terms) give each warp a
 // row block and a quarter of the columns; the gate scan and the solve's 16 x 16 steps run on threads 0-255 while
 // the rest wait at the next barrier.  One CTA per SM: 16 warps hide more of the MMA chains' latency than 8.
 constexpr int kBwThreads = 512, kBwCols = 16;  // value columns per pass over the state
@@ -748,7 +748,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         __syncthreads();
     }
 
-    // ---- 4-5. passes over 16 value columns at a time.  (a)-(d) on TF32 mma.sync (m16n8k8, fp32 accumulate); the
+    // ---- 4-5. passes over 16 value columns at a time.  (a)-(d) on fp16 mma.sync (m16n8k16, fp32 accumulate); the
     //      accumulations of (e) on tcgen05: five kind::f16 MMAs per pass (M = 64 tokens, K = the pass's 16
     //      columns) add dQg, dKb, dKg (N = 128 keys) and dAqk, dA (N = 64 tokens) into TMEM.  An M = 64 accumulator
     //      keeps rows 16 I .. 16 I + 15 in lanes 32 I .. 32 I + 15, the lane quarter of warps I, I + 4, ..., so
@@ -785,12 +785,42 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 fa[kk][q] = pack_f16(__fmul_rn(x.x, m.x), __fmul_rn(x.y, m.y));
             }
     }
+    // the other pass-invariant A operands, per 16-token K step s: role 0: T diag(beta) (step (b), tokens 16 s, s <= mt);
+    // role 1: Aqk^T (step (c), fb) and T^T (step (d), fc), tokens 16 (mt + s), s < 4 - mt
+    uint32_t fb[4][4], fc[4][4];
+#pragma unroll
+    for (int st = 0; st < 4; ++st)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = (q & 1) ? r1 : r0;
+            if (role == 0) {
+                const int k = 16 * st + 2 * t4 + 8 * (q >> 1);
+                const float2 t = *reinterpret_cast<const float2 *>(&TT[r][k]);
+                const float2 bb = *reinterpret_cast<const float2 *>(&beta[k]);
+                fb[st][q] = st <= mt ? pack_f16(__fmul_rn(t.x, bb.x), __fmul_rn(t.y, bb.y)) : 0u;
+                fc[st][q] = 0u;
+            } else {
+                const int k = min(16 * (mt + st), 48) + 2 * t4 + 8 * (q >> 1);
+                fb[st][q] = st < 4 - mt ? pack_f16(AQ[k][r], AQ[k + 1][r]) : 0u;
+                fc[st][q] = st < 4 - mt ? pack_f16(TT[k][r], TT[k + 1][r]) : 0u;
+            }
+        }
     // staging: a thread takes one 16-byte row half (8 columns) of S (tid < 256) or dS' (tid >= 256) and, for
     // tid < 128, one of dO; 8 consecutive threads take 8 rows of one half, so a quarter-warp's stores fill 128
     // contiguous bytes
     const int su = tid & 255, s_half = (su >> 3) & 1, s_row = (su & 7) | ((su >> 4) << 3);
     const int o_half = (tid >> 3) & 1, o_row = (tid & 7) | ((tid >> 4) << 3);
     uint4 rs, ro = make_uint4(0u, 0u, 0u, 0u);
+    uint32_t rv[2] = {0u, 0u}, rv_next[2] = {0u, 0u};  // v of rows r0, r1 (role 0), this pass and the next
+    auto load_v = [&](int vb, uint32_t (&x)[2]) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int i = hf ? r1 : r0;
+            x[hf] = 0u;
+            if (role == 0 && i < nvalid)
+                x[hf] = __ldg(reinterpret_cast<const unsigned int *>(p.v + ((row0 + i) * p.HV + h) * DV + vb + 8 * ntw + 2 * t4));
+        }
+    };
     auto load_pass = [&](int vb) {
         rs = __ldg(reinterpret_cast<const uint4 *>((tid < 256 ? Sg : dSg) + s_row * DV + vb + 8 * s_half));
         if (tid < 128) {
@@ -814,10 +844,14 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     const uint32_t id128 = bwd_idesc(64, 128, false, false), id64 = bwd_idesc(64, 64, false, false);
     load_pass(0);
     store_pass(0);
+    load_v(0, rv);
     float gl_acc = 0.f;  // thread d < 128: sum over all columns of S[d][.] dS'[d][.]
     for (int vb = 0, pass = 0; vb < DV; vb += kBwCols, ++pass) {
         const int buf = pass & 1;
-        if (vb + kBwCols < DV) load_pass(vb + kBwCols);
+        if (vb + kBwCols < DV) {
+            load_pass(vb + kBwCols);
+            load_v(vb + kBwCols, rv_next);
+        }
         __syncthreads();  // this pass's S, dS' and dO tiles are stored
         if (tid < DK) {
 #pragma unroll
@@ -848,10 +882,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const int i = hf ? r1 : r0, cc = 8 * ntw + 2 * t4;
-                float2 vv = make_float2(0.f, 0.f);
-                if (i < nvalid)
-                    vv = __bfloat1622float2(
-                        *reinterpret_cast<const __nv_bfloat162 *>(p.v + ((row0 + i) * p.HV + h) * DV + vb + cc));
+                const float2 vv = unpack_bf16(rv[hf]);
                 *reinterpret_cast<uint32_t *>(tile(buf, S::P_D) + tofs(i, cc)) =
                     pack_f16(__fsub_rn(vv.x, c[2 * hf]), __fsub_rn(vv.y, c[2 * hf + 1]));
             }
@@ -865,16 +896,13 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 mma_f16(c, fa[kk], b0, b1);
                 mma_f16(c, fa[kk + 1], b2, b3);
             }
-            for (int js = 16 * mt; js < CH; js += 16) {  // Aqk^T[i][j] = Aqk[j][i], nonzero for j >= i
-                uint32_t a[4], b0, b1;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int r = (q & 1) ? r1 : r0, k = js + 2 * t4 + 8 * (q >> 1);
-                    a[q] = pack_f16(AQ[k][r], AQ[k + 1][r]);
+            for (int st = 0; st < 4; ++st)  // Aqk^T[i][j] = Aqk[j][i], nonzero for j >= i
+                if (st < 4 - mt) {
+                    uint32_t b0, b1;
+                    bwd_ldsm_x2_t(tb + S::P_O + tofs(16 * (mt + st) + (lane & 15), 0), b0, b1);
+                    mma_f16(c, fb[st], b0, b1);
                 }
-                bwd_ldsm_x2_t(tb + S::P_O + tofs(js + (lane & 15), 0), b0, b1);
-                mma_f16(c, a, b0, b1);
-            }
             *reinterpret_cast<uint32_t *>(tile(buf, S::P_DN) + tofs(r0, 8 * ntw + 2 * t4)) = pack_f16(c[0], c[1]);
             *reinterpret_cast<uint32_t *>(tile(buf, S::P_DN) + tofs(r1, 8 * ntw + 2 * t4)) = pack_f16(c[2], c[3]);
         }
@@ -882,33 +910,25 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         if (role == 0) {
             // (b) Vnew = T diag(beta) D (T lower triangular: j < 16 (mt + 1))
             float c[4] = {};
-            for (int js = 0; js < 16 * (mt + 1); js += 16) {
-                uint32_t a[4], b0, b1;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int r = (q & 1) ? r1 : r0, k = js + 2 * t4 + 8 * (q >> 1);
-                    const float2 t = *reinterpret_cast<const float2 *>(&TT[r][k]);
-                    const float2 bb = *reinterpret_cast<const float2 *>(&beta[k]);
-                    a[q] = pack_f16(__fmul_rn(t.x, bb.x), __fmul_rn(t.y, bb.y));
+            for (int st = 0; st < 4; ++st)
+                if (st <= mt) {
+                    uint32_t b0, b1;
+                    bwd_ldsm_x2_t(tb + S::P_D + tofs(16 * st + (lane & 15), 0), b0, b1);
+                    mma_f16(c, fb[st], b0, b1);
                 }
-                bwd_ldsm_x2_t(tb + S::P_D + tofs(js + (lane & 15), 0), b0, b1);
-                mma_f16(c, a, b0, b1);
-            }
             *reinterpret_cast<uint32_t *>(tile(buf, S::P_N) + tofs(r0, 8 * ntw + 2 * t4)) = pack_f16(c[0], c[1]);
             *reinterpret_cast<uint32_t *>(tile(buf, S::P_N) + tofs(r1, 8 * ntw + 2 * t4)) = pack_f16(c[2], c[3]);
         } else {
             // (d) dv = diag(beta) T^T dVnew (j >= i)
             float c[4] = {};
-            for (int js = 16 * mt; js < CH; js += 16) {
-                uint32_t a[4], b0, b1;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int r = (q & 1) ? r1 : r0, k = js + 2 * t4 + 8 * (q >> 1);
-                    a[q] = pack_f16(TT[k][r], TT[k + 1][r]);
+            for (int st = 0; st < 4; ++st)
+                if (st < 4 - mt) {
+                    uint32_t b0, b1;
+                    bwd_ldsm_x2_t(tb + S::P_DN + tofs(16 * (mt + st) + (lane & 15), 0), b0, b1);
+                    mma_f16(c, fc[st], b0, b1);
                 }
-                bwd_ldsm_x2_t(tb + S::P_DN + tofs(js + (lane & 15), 0), b0, b1);
-                mma_f16(c, a, b0, b1);
-            }
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const int i = hf ? r1 : r0, cc = 8 * ntw + 2 * t4;
@@ -939,6 +959,8 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         if (vb + kBwCols < DV) {
             if (pass > 0) wait_mma(pass - 1);  // the other buffer's last readers are done
             store_pass(buf ^ 1);
+            rv[0] = rv_next[0];
+            rv[1] = rv_next[1];
         }
     }
     wait_mma(DV / kBwCols - 1);  // the last pass's MMAs, and with them every earlier one
