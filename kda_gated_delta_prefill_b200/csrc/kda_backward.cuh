@@ -601,72 +601,51 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     }
     __syncthreads();
 
-    // ---- 2. P (j < i) and Aqk (j <= i); thread: rows 4rg..4rg+3 (block I), columns cg + 16 jb, over the keys of its
-    //         half dh of the CTA (64 each).  The upper half leaves its partial sums in P and Aqk; the lower half
-    //         adds its own and writes the masked results.  (Splitting the column blocks instead would make every
-    //         thread reread the same q/k rows for fewer blocks, and the phase is bound by those shared-memory reads.) ----
+    // ---- 2. P (j < i) and Aqk (j <= i) on TF32 MMAs (m16n8k8, fp32 accumulate).  Task t < 20 is the 16 x 8 tile
+    //         n8 = t % 2 of block pair (I, J <= I), the pairs in the order (0,0), (1,0), (1,1), (2,0), ...; warp w
+    //         takes task w, warps 0-3 also task 16 + w (one of them on each SMSP).  B = KB_J exp(m_I - m_J) (J < I) ----
     {
-        const int rg = (tid >> 4) & 15, cg = tid & 15, I = rg >> 2, dh = tid >> 8;
-        float pa[4][4] = {}, aa[4][4] = {};
-        for (int d = 64 * dh; d < 64 * dh + 64; d += 4) {
-            float4 ka[4], qa[4];
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
-                ka[ii] = *reinterpret_cast<const float4 *>(&KA[4 * rg + ii][d]);
-                qa[ii] = *reinterpret_cast<const float4 *>(&QA[4 * rg + ii][d]);
-            }
-#pragma unroll
-            for (int jb = 0; jb < 4; ++jb) {
-                if (jb > I) break;
-                float4 kb = *reinterpret_cast<const float4 *>(&KB[cg + 16 * jb][d]);
-                if (jb < I) {
-                    const float4 cf = *reinterpret_cast<const float4 *>(&CF[cf_index(I, jb)][d]);
-                    kb = make_float4(__fmul_rn(kb.x, cf.x), __fmul_rn(kb.y, cf.y), __fmul_rn(kb.z, cf.z),
-                                     __fmul_rn(kb.w, cf.w));
-                }
-#pragma unroll
-                for (int ii = 0; ii < 4; ++ii) {
-                    float x = pa[ii][jb], y = aa[ii][jb];
-                    x = __fmaf_rn(ka[ii].x, kb.x, x);
-                    x = __fmaf_rn(ka[ii].y, kb.y, x);
-                    x = __fmaf_rn(ka[ii].z, kb.z, x);
-                    x = __fmaf_rn(ka[ii].w, kb.w, x);
-                    y = __fmaf_rn(qa[ii].x, kb.x, y);
-                    y = __fmaf_rn(qa[ii].y, kb.y, y);
-                    y = __fmaf_rn(qa[ii].z, kb.z, y);
-                    y = __fmaf_rn(qa[ii].w, kb.w, y);
-                    pa[ii][jb] = x;
-                    aa[ii][jb] = y;
-                }
+        for (int e = tid; e < CH * CH; e += kBwThreads) {  // T = I; P and Aqk above the diagonal blocks = 0
+            const int i = e >> 6, j = e & (CH - 1);
+            TT[i][j] = i == j ? 1.f : 0.f;
+            if ((j >> 4) > (i >> 4)) {
+                PP[i][j] = 0.f;
+                AQ[i][j] = 0.f;
             }
         }
-        if (dh == 1) {
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-                for (int jb = 0; jb < 4; ++jb)
-                    if (jb <= I) {
-                        PP[4 * rg + ii][cg + 16 * jb] = pa[ii][jb];
-                        AQ[4 * rg + ii][cg + 16 * jb] = aa[ii][jb];
-                    }
-        }
-        __syncthreads();
-        if (dh == 0) {
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-                for (int jb = 0; jb < 4; ++jb) {
-                    const int i = 4 * rg + ii, j = cg + 16 * jb;
-                    float pv = 0.f, av = 0.f;
-                    if (jb <= I) {
-                        pv = __fadd_rn(pa[ii][jb], PP[i][j]);
-                        av = __fadd_rn(aa[ii][jb], AQ[i][j]);
-                    }
-                    PP[i][j] = j < i ? pv : 0.f;
-                    AQ[i][j] = j <= i ? __fmul_rn(s, av) : 0.f;
-                    TT[i][j] = i == j ? 1.f : 0.f;
+        auto task = [&](int t) {
+            const int gq = lane >> 2, tq = lane & 3, n8 = t & 1;
+            int pr = t >> 1, I = 0;
+            while (pr > I) pr -= ++I;
+            const int J = pr;
+            const float *cf = J < I ? CF[cf_index(I, J)] : nullptr;
+            const int ra = 16 * I + gq, rb = 16 * J + 8 * n8 + gq;
+            float cp[4] = {}, cq[4] = {};
+#pragma unroll 4
+            for (int ks = 0; ks < DK; ks += 8) {
+                const int k0 = ks + tq, k1 = k0 + 4;
+                const uint32_t ap[4] = {to_tf32(KA[ra][k0]), to_tf32(KA[ra + 8][k0]), to_tf32(KA[ra][k1]),
+                                        to_tf32(KA[ra + 8][k1])};
+                const uint32_t aq[4] = {to_tf32(QA[ra][k0]), to_tf32(QA[ra + 8][k0]), to_tf32(QA[ra][k1]),
+                                        to_tf32(QA[ra + 8][k1])};
+                float b0 = KB[rb][k0], b1 = KB[rb][k1];
+                if (cf) {
+                    b0 = __fmul_rn(b0, cf[k0]);
+                    b1 = __fmul_rn(b1, cf[k1]);
                 }
-        }
+                const uint32_t u0 = to_tf32(b0), u1 = to_tf32(b1);
+                mma_tf32(cp, ap, u0, u1);
+                mma_tf32(cq, aq, u0, u1);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int i = ra + 8 * (q >> 1), j = 16 * J + 8 * n8 + 2 * tq + (q & 1);
+                PP[i][j] = j < i ? cp[q] : 0.f;
+                AQ[i][j] = j <= i ? __fmul_rn(s, cq[q]) : 0.f;
+            }
+        };
+        task(warp);
+        if (warp < 4) task(16 + warp);
     }
     __syncthreads();
 
