@@ -740,7 +740,6 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     auto tile = [&](int b, int off) { return sm + S::WK + b * S::PBUF + off; };
     const __nv_bfloat16 *Sg = p.states + item * DK * DV;
     const __nv_bfloat16 *dSg = p.dstates + item * DK * DV;
-    const int cg = tid & 15;  // column of the 64 x 64 steps of phase 6 (with the row group and half below)
     // MMA fragment ownership (g = lane / 4, t4 = lane % 4): warp (mt, nh), nh = 0..3, holds rows 16 mt + g and + 8,
     // and key columns 32 nh + 8 j + 2 t4 (+1), j = 0..3 (dQg, dKb, dKg), or token columns 16 nh + 8 j + 2 t4 (+1),
     // j = 0..1 (dAqk, dA).  In steps (a)-(d) of a pass, warp (mt, role, ntw) = (warp % 4, warp / 4 % 2, warp / 8)
@@ -967,68 +966,74 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
         for (int i = tid; i < CH; ++i) acc = __fmaf_rn(DA[i][tid], TT[i][tid], acc);
         dbeta[tid] = acc;
     }
-    // Y = T^T (dA diag(beta)): Y[a][e] = beta_e sum_{c >= a} T[c][a] dA[c][e].  Thread: rows 4 rg6 .. 4 rg6 + 3
-    // and columns cg + 16 jb for the two column blocks jb = 2 jh, 2 jh + 1 of its half of the CTA.
-    const int rg6 = (tid >> 4) & 15, jh = tid >> 8;
-    float y[4][2] = {};
-    for (int c = 4 * rg6; c < CH; ++c) {
+    // Y = T^T dA diag(beta), Y[a][e] = beta_e sum_{c >= a} T[c][a] dA[c][e], then dL = -Y T^T (a > b), both on TF32
+    // MMAs (m16n8k8): warp (mt, nh) holds rows 16 mt + g (+ 8) of the 8-column tiles nb = nh and nh + 4.
+    float y[2][4] = {};
+    for (int ks = 16 * mt; ks < CH; ks += 8) {  // T[c][a] = 0 for c < a
+        const uint32_t a[4] = {to_tf32(TT[ks + t4][r0]), to_tf32(TT[ks + t4][r1]), to_tf32(TT[ks + t4 + 4][r0]),
+                               to_tf32(TT[ks + t4 + 4][r1])};
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-            const float t = TT[c][4 * rg6 + ii];
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) y[ii][jj] = __fmaf_rn(t, DA[c][cg + 16 * (2 * jh + jj)], y[ii][jj]);
+        for (int jj = 0; jj < 2; ++jj) {
+            const int cn = 8 * (nh + 4 * jj) + g;
+            mma_tf32(y[jj], a, to_tf32(DA[ks + t4][cn]), to_tf32(DA[ks + t4 + 4][cn]));
         }
     }
     __syncthreads();  // every read of dA is done
 #pragma unroll
-    for (int ii = 0; ii < 4; ++ii)
+    for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-            const int col = cg + 16 * (2 * jh + jj);
-            DA[4 * rg6 + ii][col] = __fmul_rn(beta[col], y[ii][jj]);
+        for (int q = 0; q < 4; ++q) {
+            const int col = 8 * (nh + 4 * jj) + 2 * t4 + (q & 1);
+            DA[(q >> 1) ? r1 : r0][col] = __fmul_rn(beta[col], y[jj][q]);
         }
     __syncthreads();
     // dL[a][b] = -sum_{e <= b} Y[a][e] T[b][e] (a > b); dbeta_a += sum_b dL_ab P_ab; M = diag(beta) dL
     {
-        float *rowp2 = reinterpret_cast<float *>(sm + S::DA + CH * kRowC * 4);  // [2 halves][64 rows]
-        float dl[4][2] = {}, rowp[4] = {};
-        for (int e = 0; e < CH; ++e) {
-            float ye[4];
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii) ye[ii] = DA[4 * rg6 + ii][e];
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const float t = TT[cg + 16 * (2 * jh + jj)][e];  // zero for e > b
-#pragma unroll
-                for (int ii = 0; ii < 4; ++ii) dl[ii][jj] = __fmaf_rn(-ye[ii], t, dl[ii][jj]);
+        float *rowp4 = reinterpret_cast<float *>(sm + S::DA + CH * kRowC * 4);  // [4 column quarters][64 rows]
+        float dl[2][4] = {};
+        const int kend = 8 * (nh + 4) + 8;  // tile nh + 4 needs e < kend, tile nh e < 8 nh + 8
+        const bool live0 = 8 * nh < 16 * mt + 16, live1 = 8 * (nh + 4) < 16 * mt + 16;  // some a > b in the tile
+        if (live0 || live1) {
+            for (int ks = 0; ks < kend; ks += 8) {
+                const uint32_t a[4] = {to_tf32(DA[r0][ks + t4]), to_tf32(DA[r1][ks + t4]), to_tf32(DA[r0][ks + t4 + 4]),
+                                       to_tf32(DA[r1][ks + t4 + 4])};
+                if (live0 && ks < 8 * nh + 8)
+                    mma_tf32(dl[0], a, to_tf32(TT[8 * nh + g][ks + t4]), to_tf32(TT[8 * nh + g][ks + t4 + 4]));
+                if (live1)
+                    mma_tf32(dl[1], a, to_tf32(TT[8 * (nh + 4) + g][ks + t4]), to_tf32(TT[8 * (nh + 4) + g][ks + t4 + 4]));
             }
         }
+        float rowp[2] = {};
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
+        for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int a = 4 * rg6 + ii, b = cg + 16 * (2 * jh + jj);
-                if (b < a) rowp[ii] = __fmaf_rn(dl[ii][jj], PP[a][b], rowp[ii]);
-                else dl[ii][jj] = 0.f;
+            for (int q = 0; q < 4; ++q) {
+                const int a = (q >> 1) ? r1 : r0, b = 8 * (nh + 4 * jj) + 2 * t4 + (q & 1);
+                float v = -dl[jj][q];
+                if (b < a) rowp[q >> 1] = __fmaf_rn(v, PP[a][b], rowp[q >> 1]);
+                else v = 0.f;
+                dl[jj][q] = v;
             }
-        // the 16 threads of a row group are 16 consecutive lanes
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-#pragma unroll
-            for (int off = 8; off > 0; off >>= 1)
-                rowp[ii] = __fadd_rn(rowp[ii], __shfl_xor_sync(0xffffffffu, rowp[ii], off));
+        for (int hf = 0; hf < 2; ++hf) {  // the four lanes of a row, then (after the barrier) the four column quarters
+            rowp[hf] = __fadd_rn(rowp[hf], __shfl_xor_sync(0xffffffffu, rowp[hf], 1));
+            rowp[hf] = __fadd_rn(rowp[hf], __shfl_xor_sync(0xffffffffu, rowp[hf], 2));
         }
-        if (cg == 0) {
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii) rowp2[jh * CH + 4 * rg6 + ii] = rowp[ii];
+        if (t4 == 0) {
+            rowp4[nh * CH + r0] = rowp[0];
+            rowp4[nh * CH + r1] = rowp[1];
         }
-        __syncthreads();  // every read of P and T is done (dbeta's column sums above included); halves stored
-        if (tid < CH) dbeta[tid] = __fadd_rn(dbeta[tid], __fadd_rn(rowp2[tid], rowp2[CH + tid]));
+        __syncthreads();  // every read of P and T is done (dbeta's column sums above included); quarters stored
+        if (tid < CH)
+            dbeta[tid] = __fadd_rn(dbeta[tid], __fadd_rn(__fadd_rn(rowp4[tid], rowp4[CH + tid]),
+                                                         __fadd_rn(rowp4[2 * CH + tid], rowp4[3 * CH + tid])));
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
+        for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj)
-                PP[4 * rg6 + ii][cg + 16 * (2 * jh + jj)] = __fmul_rn(beta[4 * rg6 + ii], dl[ii][jj]);
+            for (int q = 0; q < 4; ++q) {
+                const int a = (q >> 1) ? r1 : r0, b = 8 * (nh + 4 * jj) + 2 * t4 + (q & 1);
+                PP[a][b] = __fmul_rn(beta[a], dl[jj][q]);
+            }
     }
     __syncthreads();
     float(*MM)[kRowC] = PP;
