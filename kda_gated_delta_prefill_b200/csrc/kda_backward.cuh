@@ -425,6 +425,10 @@ __device__ __forceinline__ uint64_t bwd_tile_desc(uint32_t saddr)
     return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(128 >> 4) << 16) |
            (static_cast<uint64_t>(256 >> 4) << 32) | (1ull << 46);
 }
+__device__ __forceinline__ void bwd_prefetch_l2(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void bwd_ldsm_x2_t(uint32_t addr, uint32_t &r0, uint32_t &r1)
 {
     asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(addr));
@@ -526,6 +530,16 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
     float *egl = reinterpret_cast<float *>(sm + S::EGL), *dgl = reinterpret_cast<float *>(sm + S::DGL);
     float *dbeta = reinterpret_cast<float *>(sm + S::DBETA);
     const int64_t item = static_cast<int64_t>(chunk) * p.HV + h;
+    // the passes' inputs (S, dS', and the rows of dO and v), pulled into L2 now: the passes read them 16 columns
+    // at a time, and each pass's registers would otherwise wait on HBM
+    if (tid == 0) {
+        bwd_prefetch_l2(p.states + item * DK * DV, DK * DV * 2);
+        bwd_prefetch_l2(p.dstates + item * DK * DV, DK * DV * 2);
+    }
+    if (tid < nvalid) {
+        bwd_prefetch_l2(p.dout + ((row0 + tid) * p.HV + h) * DV, DV * 2);
+        bwd_prefetch_l2(p.v + ((row0 + tid) * p.HV + h) * DV, DV * 2);
+    }
 
     // ---- 1. gates: G = cumulative g, block references, beta ----
     // this warp's eight q and k rows, requested first so that their latency overlaps the gate work
@@ -950,6 +964,21 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
 
     if (tid < DK) dgl[tid] = __fmaf_rn(egl[tid], gl_acc, dgl[tid]);  // the exp(G_L) S dS' term of dG_L
 
+    // the raw q/k pairs of the phase-7 elements (the element terms rebuild qn/kn from them; the normalisation's
+    // Jacobian reads them at the end), requested here so that their latency hides behind phase 6
+    uint32_t xq[2][4] = {}, xk[2][4] = {};
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        const int i = hf ? r1 : r0;
+        if (i < nvalid) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t off = ((row0 + i) * p.H + hq) * DK + 32 * nh + 8 * j + 2 * t4;
+                xq[hf][j] = *reinterpret_cast<const uint32_t *>(p.q + off);
+                xk[hf][j] = *reinterpret_cast<const uint32_t *>(p.k + off);
+            }
+        }
+    }
     // ---- 6. dbeta, dL, M = diag(beta) dL, N = dAqk ----
     float(*DA)[kRowC] = reinterpret_cast<float(*)[kRowC]>(sm + S::DA);
 #pragma unroll
@@ -1056,11 +1085,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int d = 32 * nh + 8 * j + 2 * t4;
-                uint32_t wq = 0u, wk = 0u;
-                if (i < nvalid) {
-                    wq = *reinterpret_cast<const uint32_t *>(p.q + ((row0 + i) * p.H + hq) * DK + d);
-                    wk = *reinterpret_cast<const uint32_t *>(p.k + ((row0 + i) * p.H + hq) * DK + d);
-                }
+                const uint32_t wq = xq[hf][j], wk = xk[hf][j];
                 const uint32_t pq = pack_bf16(div_rn_with_rcp(bf16lo(wq), dq, rqi), div_rn_with_rcp(bf16hi(wq), dq, rqi));
                 const uint32_t pk = pack_bf16(div_rn_with_rcp(bf16lo(wk), dk, rki), div_rn_with_rcp(bf16hi(wk), dk, rki));
                 const float qn[2] = {bf16lo(pq), bf16hi(pq)}, kn[2] = {bf16lo(pk), bf16hi(pk)};
@@ -1130,23 +1155,6 @@ __global__ void __launch_bounds__(kBwThreads, 1) kda_bwd_chunk_kernel(const BwdP
                 rG[j][q] = __fmaf_rn(KA[i][d], ra[j][q], rG[j][q]);
                 rG[j][q] = __fmaf_rn(__fmul_rn(s, QA[i][d]), rb[j][q], rG[j][q]);
             }
-    }
-    // the raw q/k pairs of the owned elements, for the normalisation's Jacobian at the end (requested here, so
-    // that their latency hides behind the MMAs below)
-    uint32_t xq[2][4] = {}, xk[2][4] = {};
-    if (p.fuse_norm) {
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const int i = hf ? r1 : r0;
-            if (i < nvalid) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int64_t off = ((row0 + i) * p.H + hq) * DK + 32 * nh + 8 * j + 2 * t4;
-                    xq[hf][j] = *reinterpret_cast<const uint32_t *>(p.q + off);
-                    xk[hf][j] = *reinterpret_cast<const uint32_t *>(p.k + off);
-                }
-            }
-        }
     }
     {
         // R24'_jd = sum_{I' >= J} sum_{i in I'} (M_ij KA_id + s N_ij QA_id) c_I'Jd for rows j of block J = mt
