@@ -297,9 +297,12 @@ kda_status_t kda_prefill_forward_state_bf16(const void *q, const void *k, const 
  * cuts it, each part's carry beside the next part's blocks); a reverse carry
  * walks each sequence backwards
  * for the gradient at every chunk's end state; a per-chunk kernel forms the
- * chunk's gradients; a last kernel sums each Q/K group and applies the
- * normalisation's Jacobian.  Accuracy assumes g <= 0 with every 8 consecutive
- * gates of a channel summing to >= -40 (per-token g >= -5 suffices).
+ * chunk's gradients (and, when H == HV, applies the normalisation's
+ * Jacobian); with H < HV a last kernel sums each Q/K group and applies it.
+ * Accuracy assumes g <= 0 with every 8 consecutive gates of a channel summing
+ * to >= -40 (per-token g >= -5 suffices), and, as for the forward's state,
+ * entries of the chunk states, of their gradients and of dout below 6e4: the
+ * reverse carry and the per-chunk passes multiply them as fp16 operands.
  */
 size_t kda_prefill_backward_workspace_size(int B, int T, int H, int HV, int K, int V, int num_seqs);
 /* Kernel launches of one kda_prefill_backward call (the recomputing form); 0 for invalid sizes, or when the
