@@ -490,6 +490,10 @@ struct BwSmem {
     static constexpr int TOTAL = (WK_END > DA + CH * kRowC * 4 ? WK_END : DA + CH * kRowC * 4);
 };
 static_assert(BwSmem::TOTAL <= 232448, "shared memory");
+static_assert((kRowC - CH) * 4 >= 16 && BwSmem::MBAR % 8 == 0 && BwSmem::TMEM_SLOT % 4 == 0,
+              "the TMEM address and the two mbarriers need 16 bytes of row padding, 8-byte aligned");
+static_assert(BwSmem::WK % 16 == 0 && BwSmem::PBUF % 16 == 0 && BwSmem::WK_END < (1 << 18),
+              "pass tiles: 16-byte aligned, inside the descriptors' 18-bit address range");
 
 __device__ __forceinline__ int cf_index(int I, int J) { return I * (I - 1) / 2 + J; }
 
